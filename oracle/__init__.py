@@ -1,0 +1,193 @@
+"""Float64 CPU oracle for two-stage block-sparse attention.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package; the product path (``block_sparse_attention_19_b200``) never does, and
+this package imports nothing from it.
+
+The arithmetic lives in ``bsa_oracle.c`` (plain C, float64, OpenMP over
+independent rows only); this module builds it with gcc and marshals numpy
+arrays through ctypes.  Each function follows the definition on the pages:
+
+* "2026 新一代卷积与 Transformer 网络架构" (qqiyuan.cn), section
+  "SparseFormer 注意力实现": mean-pool q/k over blocks, score blocks,
+  keep int(topk_ratio * nb) blocks with top-k, attend over the kept blocks
+  with scale 1/sqrt(D).
+* "从M2.7到M3：多模态模型稀疏注意力架构设计与实现全解析", §2.1 and §2.2:
+  Softmax(Mask(QK^T/sqrt(d_k)))V with a block mask from a coarse block score.
+
+Every function here is pinned by ``tests/test_oracle.py`` against closed forms,
+library routines (numpy matmul / lexsort, torch SDPA in float64), brute force
+and invariants; nothing in this package is "parity unpinned".
+
+Inputs may be float32, float64 or bfloat16; bfloat16 is passed as its raw
+16-bit patterns in a ``numpy.uint16`` array (tag ``"bf16"``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import time
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bsa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+F32, BF16, F64 = 0, 1, 2
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``bsa_oracle.c`` into ``liboracle.so`` (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall", "-o", tmp, _SRC, "-lm"],
+            check=True,
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i, d = ctypes.c_int, ctypes.c_double
+        lib.oracle_topk_count.argtypes = [i, d]
+        lib.oracle_topk_count.restype = i
+        lib.oracle_block_pool.argtypes = [P, i, i, i, i, i, i, P]
+        lib.oracle_block_scores.argtypes = [P, P, i, i, i, i, P, i, P]
+        lib.oracle_topk_row.argtypes = [P, i, i, P]
+        lib.oracle_topk.argtypes = [P, ctypes.c_long, i, i, P]
+        lib.oracle_sparse_attn.argtypes = [P, P, P, i, i, i, i, i, i, P, i, P, i, d, P]
+        lib.oracle_num_threads.restype = i
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _as_input(x: np.ndarray):
+    """Return (contiguous array, dtype code) for a q/k/v tensor."""
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float32:
+        return x, F32
+    if x.dtype == np.float64:
+        return x, F64
+    if x.dtype == np.uint16:
+        return x, BF16
+    raise TypeError(f"oracle inputs must be float32, float64 or bf16 bits (uint16), got {x.dtype}")
+
+
+def num_threads() -> int:
+    return _load().oracle_num_threads()
+
+
+def topk_count(nb: int, topk_ratio: float) -> int:
+    """k = int(topk_ratio * nb) exactly as Python evaluates it ([SF] step 2)."""
+    return _load().oracle_topk_count(int(nb), float(topk_ratio))
+
+
+def block_pool(x: np.ndarray, block_size: int) -> np.ndarray:
+    """[B,N,H,D] -> block means [B,H,nb,D] in float64 ([SF] step 1)."""
+    x, code = _as_input(x)
+    B, N, H, D = x.shape
+    if N % block_size:
+        raise ValueError("N must be a multiple of block_size")
+    nb = N // block_size
+    out = np.empty((B, H, nb, D), np.float64)
+    _load().oracle_block_pool(_ptr(x), code, B, N, H, D, block_size, _ptr(out))
+    return out
+
+
+def block_scores(qp: np.ndarray, kp: np.ndarray, rows: np.ndarray | None = None) -> np.ndarray:
+    """Block scores S[b,h,r,j] = qp[b,h,rows[b,h,r]] . kp[b,h,j] ([SF] step 1).
+
+    ``rows`` is an int array [B,H,nrows] of query-block ids (None = all)."""
+    qp = np.ascontiguousarray(qp, np.float64)
+    kp = np.ascontiguousarray(kp, np.float64)
+    B, H, nb, D = qp.shape
+    if rows is None:
+        nrows, rp = nb, None
+    else:
+        rows = np.ascontiguousarray(rows, np.int32)
+        nrows, rp = rows.shape[-1], _ptr(rows)
+    out = np.empty((B, H, nrows, nb), np.float64)
+    _load().oracle_block_scores(_ptr(qp), _ptr(kp), B, H, nb, D, rp, nrows, _ptr(out))
+    return out
+
+
+def topk(scores: np.ndarray, k: int) -> np.ndarray:
+    """Top-k block ids of every score row, ties to the lower id, ascending ([SF] step 2)."""
+    s = np.ascontiguousarray(scores, np.float64)
+    nb = s.shape[-1]
+    if not (1 <= k <= nb):
+        raise ValueError("need 1 <= k <= nb")
+    rows = int(np.prod(s.shape[:-1]))
+    out = np.empty(s.shape[:-1] + (k,), np.int32)
+    _load().oracle_topk(_ptr(s), rows, nb, k, _ptr(out))
+    return out
+
+
+def sparse_attn(q, k, v, idx, block_size: int, scale: float | None = None, rows=None) -> np.ndarray:
+    """Exact softmax attention over the selected key blocks ([SF] step 3, [MSA] §2.1).
+
+    ``idx`` is int [B,H,nrows,k] (the selected key blocks of each listed query
+    block); ``rows`` is int [B,H,nrows] (None = all nb query blocks in order).
+    Returns float64 [B,H,nrows,block_size,D]."""
+    q, code = _as_input(q)
+    k_, code_k = _as_input(k)
+    v, code_v = _as_input(v)
+    if not (code == code_k == code_v):
+        raise TypeError("q, k, v must share one dtype")
+    B, N, H, D = q.shape
+    nb = N // block_size
+    idx = np.ascontiguousarray(idx, np.int32)
+    kk = idx.shape[-1]
+    if rows is None:
+        nrows, rp = nb, None
+    else:
+        rows = np.ascontiguousarray(rows, np.int32)
+        nrows, rp = rows.shape[-1], _ptr(rows)
+    if idx.shape != (B, H, nrows, kk):
+        raise ValueError(f"idx shape {idx.shape} != {(B, H, nrows, kk)}")
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    out = np.empty((B, H, nrows, block_size, D), np.float64)
+    _load().oracle_sparse_attn(_ptr(q), _ptr(k_), _ptr(v), code, B, N, H, D, block_size,
+                               _ptr(idx), kk, rp, nrows, float(scale), _ptr(out))
+    return out
+
+
+def forward(q, k, v, block_size: int, topk_ratio: float, rows=None, scale=None) -> dict:
+    """The whole path of the [SF] listing on the oracle: pool, score, select, attend.
+
+    ``rows`` (int [B,H,nrows]) restricts the scored / attended query blocks to
+    a sample; pooling of k always covers every block since selection needs all
+    of them.  Returns a dict with qp, kp, scores, idx, o, k and timings."""
+    t0 = time.perf_counter()
+    qn, _ = _as_input(q)
+    B, N, H, D = qn.shape
+    nb = N // block_size
+    kk = topk_count(nb, topk_ratio)
+    qp = block_pool(q, block_size)
+    kp = block_pool(k, block_size)
+    S = block_scores(qp, kp, rows)
+    idx = topk(S, kk)
+    o = sparse_attn(q, k, v, idx, block_size, scale=scale, rows=rows)
+    return {"qp": qp, "kp": kp, "scores": S, "idx": idx, "o": o, "k": kk,
+            "seconds": time.perf_counter() - t0}
+
+
+def o_to_bnhd(o: np.ndarray) -> np.ndarray:
+    """Reorder an all-rows oracle output [B,H,nb,bs,D] to [B,N,H,D]."""
+    B, H, nb, bs, D = o.shape
+    return o.reshape(B, H, nb * bs, D).transpose(0, 2, 1, 3).copy()

@@ -1,0 +1,211 @@
+/*
+ * bsa_oracle.c -- float64 CPU oracle for two-stage block-sparse attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the reference definition that the
+ * CUDA library is checked against.  Only the tests, the smoke check and the
+ * CPU-baseline leg of the benchmark may load it; no product code path calls it.
+ * It shares no code, header or constant with the CUDA library.
+ *
+ * Sources (web pages; cited by title and section):
+ *   [SF]  "2026 新一代卷积与 Transformer 网络架构" (qqiyuan.cn), section
+ *         "SparseFormer 注意力实现": block_sparse_attention(q, k, v,
+ *         block_size=64, topk_ratio=0.3) with q/k/v of shape [B, N, H, D];
+ *         step 1 mean-pools q and k over blocks and forms block scores,
+ *         step 2 keeps int(topk_ratio * num_blocks) key blocks per query
+ *         block with torch.topk, step 3 runs attention over the kept blocks
+ *         with scale = 1/sqrt(D).
+ *   [MSA] "从M2.7到M3：多模态模型稀疏注意力架构设计与实现全解析"
+ *         (cloud.baidu.com), §2.1 (Attention = Softmax(Mask(QK^T/sqrt(d_k)))V)
+ *         and §2.2 (coarse block scoring, then full attention inside the
+ *         chosen blocks).
+ *
+ * Readings where the pages are silent or garbled (each one is listed in the
+ * design notes as well):
+ *   - The [SF] einsum 'bhid,bhjd->bhij' is applied to the pooled tensors
+ *     after moving the head axis next to the batch axis, so the scores are
+ *     per (b, h) and of size nb x nb, as the comment on step 1 states.
+ *   - The block score carries no 1/sqrt(D) factor (the [SF] code has none);
+ *     a positive factor would not change the ranking anyway.
+ *   - Pooled means are kept in float64 (no rounding to the input type).
+ *   - Ties in the top-k go to the lower key-block index; each selected list
+ *     is emitted in ascending block order.
+ *   - Attention is non-causal.
+ *
+ * Every function works in float64.  Inputs may be float32, bfloat16 (raw
+ * 16-bit patterns) or float64; each element is converted exactly to double.
+ * Parallelism (OpenMP) is only over independent output rows; the arithmetic
+ * inside a row follows the definition in plain order.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_F32 0
+#define ORACLE_BF16 1
+#define ORACLE_F64 2
+
+/* Exact conversion of one stored element to double. */
+static double elem(const void* base, int dtype, size_t i) {
+  if (dtype == ORACLE_F32) return (double)((const float*)base)[i];
+  if (dtype == ORACLE_F64) return ((const double*)base)[i];
+  /* bfloat16: the high 16 bits of an IEEE float32. */
+  uint32_t bits = ((uint32_t)((const uint16_t*)base)[i]) << 16;
+  float f;
+  memcpy(&f, &bits, sizeof f);
+  return (double)f;
+}
+
+/* Offset of element (b, n, h, d) of a contiguous [B, N, H, D] tensor. */
+static size_t at_bnhd(int N, int H, int D, int b, int n, int h, int d) {
+  return (((size_t)b * N + n) * H + h) * D + d;
+}
+
+/* [SF] step 2: k = int(topk_ratio * num_blocks), Python int() of a double. */
+int oracle_topk_count(int nb, double topk_ratio) {
+  double prod = topk_ratio * (double)nb;
+  if (!(prod >= 0.0)) return -1;
+  return (int)prod; /* truncation toward zero == Python int() for prod >= 0 */
+}
+
+/* [SF] step 1 (q.view(B, nb, bs, H, D).mean(2)):
+ * xp[b, h, i, d] = (1/bs) * sum_{t < bs} x[b, i*bs + t, h, d].
+ * Output layout [B, H, nb, D]. */
+void oracle_block_pool(const void* x, int dtype, int B, int N, int H, int D, int bs,
+                       double* xp) {
+  int nb = N / bs;
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int i = 0; i < nb; ++i)
+        for (int d = 0; d < D; ++d) {
+          double s = 0.0;
+          for (int t = 0; t < bs; ++t) s += elem(x, dtype, at_bnhd(N, H, D, b, i * bs + t, h, d));
+          xp[(((size_t)b * H + h) * nb + i) * D + d] = s / (double)bs;
+        }
+}
+
+/* [SF] step 1 (einsum of pooled q and pooled k, per (b, h)):
+ * S[b, h, r, j] = sum_d qp[b, h, rows[b,h,r], d] * kp[b, h, j, d]
+ * for the nrows query blocks listed per (b, h) in rows[B, H, nrows]
+ * (rows == NULL means all nb query blocks, nrows == nb). */
+void oracle_block_scores(const double* qp, const double* kp, int B, int H, int nb, int D,
+                         const int* rows, int nrows, double* S) {
+#pragma omp parallel for collapse(3) schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int r = 0; r < nrows; ++r) {
+        size_t bh = (size_t)b * H + h;
+        int i = rows ? rows[bh * nrows + r] : r;
+        const double* qi = qp + (bh * nb + i) * D;
+        for (int j = 0; j < nb; ++j) {
+          const double* kj = kp + (bh * nb + j) * D;
+          double s = 0.0;
+          for (int d = 0; d < D; ++d) s += qi[d] * kj[d];
+          S[(bh * nrows + r) * nb + j] = s;
+        }
+      }
+}
+
+/* Ordering for the top-k: larger score first, equal scores by lower index. */
+typedef struct {
+  double s;
+  int j;
+} scored_block;
+
+static int by_score_then_index(const void* a, const void* b) {
+  const scored_block* x = (const scored_block*)a;
+  const scored_block* y = (const scored_block*)b;
+  if (x->s > y->s) return -1;
+  if (x->s < y->s) return 1;
+  return (x->j > y->j) - (x->j < y->j);
+}
+
+static int ascending_int(const void* a, const void* b) {
+  int x = *(const int*)a, y = *(const int*)b;
+  return (x > y) - (x < y);
+}
+
+/* [SF] step 2 for one row: the k key blocks with the largest scores (ties to
+ * the lower block index), written to idx[0..k) in ascending block order. */
+void oracle_topk_row(const double* s_row, int nb, int k, int* idx) {
+  scored_block* order = (scored_block*)malloc((size_t)nb * sizeof(scored_block));
+  for (int j = 0; j < nb; ++j) {
+    order[j].s = s_row[j];
+    order[j].j = j;
+  }
+  qsort(order, (size_t)nb, sizeof(scored_block), by_score_then_index);
+  for (int t = 0; t < k; ++t) idx[t] = order[t].j;
+  qsort(idx, (size_t)k, sizeof(int), ascending_int);
+  free(order);
+}
+
+/* [SF] step 2 over many rows: S is [nrows_total, nb], idx is [nrows_total, k]. */
+void oracle_topk(const double* S, long nrows_total, int nb, int k, int* idx) {
+#pragma omp parallel for schedule(static)
+  for (long r = 0; r < nrows_total; ++r) oracle_topk_row(S + r * nb, nb, k, idx + r * k);
+}
+
+/* [SF] step 3 / [MSA] §2.1-§2.2: for every query row n of query block i,
+ *   l_t = scale * sum_d q[b,n,h,d] * k[b,t,h,d]   for t in the selected blocks,
+ *   o[n] = sum_t exp(l_t - max l) v[b,t,h,:] / sum_t exp(l_t - max l).
+ * The selected blocks of (b, h, rows[b,h,r]) are idx[b, h, r, 0..k).
+ * Output o is [B, H, nrows, bs, D] (float64). rows == NULL means all nb. */
+void oracle_sparse_attn(const void* q, const void* kmat, const void* v, int dtype, int B, int N,
+                        int H, int D, int bs, const int* idx, int k, const int* rows, int nrows,
+                        double scale, double* o) {
+  int nb = N / bs;
+  (void)nb;
+  long ntok = (long)k * bs;
+#pragma omp parallel
+  {
+    double* logit = (double*)malloc((size_t)ntok * sizeof(double));
+    double* qrow = (double*)malloc((size_t)D * sizeof(double));
+#pragma omp for collapse(4) schedule(dynamic, 4)
+    for (int b = 0; b < B; ++b)
+      for (int h = 0; h < H; ++h)
+        for (int r = 0; r < nrows; ++r)
+          for (int t_q = 0; t_q < bs; ++t_q) {
+            size_t bh = (size_t)b * H + h;
+            int i = rows ? rows[bh * nrows + r] : r;
+            const int* sel = idx + (bh * nrows + r) * k;
+            int n = i * bs + t_q;
+            for (int d = 0; d < D; ++d) qrow[d] = elem(q, dtype, at_bnhd(N, H, D, b, n, h, d));
+            /* logits over the tokens of the selected blocks */
+            double m = -INFINITY;
+            for (int s = 0; s < k; ++s)
+              for (int u = 0; u < bs; ++u) {
+                int t = sel[s] * bs + u;
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) dot += qrow[d] * elem(kmat, dtype, at_bnhd(N, H, D, b, t, h, d));
+                double l = scale * dot;
+                logit[(long)s * bs + u] = l;
+                if (l > m) m = l;
+              }
+            /* softmax weights and the weighted sum of v */
+            double* out = o + ((bh * nrows + r) * bs + t_q) * D;
+            for (int d = 0; d < D; ++d) out[d] = 0.0;
+            double z = 0.0;
+            for (int s = 0; s < k; ++s)
+              for (int u = 0; u < bs; ++u) {
+                int t = sel[s] * bs + u;
+                double w = exp(logit[(long)s * bs + u] - m);
+                z += w;
+                for (int d = 0; d < D; ++d) out[d] += w * elem(v, dtype, at_bnhd(N, H, D, b, t, h, d));
+              }
+            for (int d = 0; d < D; ++d) out[d] /= z;
+          }
+    free(logit);
+    free(qrow);
+  }
+}
+
+/* Number of OpenMP threads the oracle runs with (reported by the CPU baseline). */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  extern int omp_get_max_threads(void);
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

@@ -1,0 +1,309 @@
+"""Pins for the float64 oracle (CPU only).
+
+Every oracle function is checked against something other than itself: a
+hand-worked case with closed-form answers, library routines (numpy matmul,
+numpy lexsort, torch scaled_dot_product_attention in float64), brute force on
+tiny inputs and invariants of the definition.  The definition is the one on
+"2026 新一代卷积与 Transformer 网络架构" (qqiyuan.cn), section
+"SparseFormer 注意力实现", with the mask formula of
+"从M2.7到M3：多模态模型稀疏注意力架构设计与实现全解析" §2.1.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def _rand(shape, seed, offsets=True, bs=None):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal(shape)
+    if offsets and bs:
+        B, N, H, D = shape
+        off = rng.standard_normal((B, N // bs, 1, H, D))
+        x = (x.reshape(B, N // bs, bs, H, D) + off).reshape(shape)
+    return x
+
+
+def _closed(expr):
+    return eval(expr, {"exp": math.exp})
+
+
+# ---------------------------------------------------------------- hand-worked
+
+def test_hw1_hand_worked(oracle_mod):
+    g = json.load(open(os.path.join(HERE, "golden", "hw1.json")))
+    shp = (g["B"], g["N"], g["H"], g["D"])
+    q = np.array(g["q"], np.float64).reshape(shp)
+    k = np.array(g["k"], np.float64).reshape(shp)
+    v = np.array(g["v"], np.float64).reshape(shp)
+    bs = g["block_size"]
+    r = oracle_mod.forward(q, k, v, bs, g["topk_ratio"])
+    assert r["k"] == g["k_selected"]
+    np.testing.assert_array_equal(r["qp"][0, 0, :, 0], g["q_pooled"])
+    np.testing.assert_array_equal(r["kp"][0, 0, :, 0], g["k_pooled"])
+    np.testing.assert_array_equal(r["scores"][0, 0], g["scores"])
+    np.testing.assert_array_equal(r["idx"][0, 0], g["idx"])
+    o = oracle_mod.o_to_bnhd(r["o"]).reshape(-1)
+    want = [_closed(e) for e in g["o_closed_form"]]
+    np.testing.assert_allclose(o, want, rtol=1e-15, atol=0)
+    # ratio 1.0: row 0 attends to every token (dense)
+    rd = oracle_mod.forward(q, k, v, bs, 1.0)
+    np.testing.assert_allclose(oracle_mod.o_to_bnhd(rd["o"]).reshape(-1)[0],
+                               _closed(g["o_dense_row0_closed_form"]), rtol=1e-15)
+    # exact tie: both key blocks score the same, the lower id wins
+    kt = np.array(g["tie_variant"]["k"], np.float64).reshape(shp)
+    rt = oracle_mod.forward(q, kt, v, bs, g["topk_ratio"])
+    np.testing.assert_array_equal(rt["kp"][0, 0, :, 0], g["tie_variant"]["k_pooled"])
+    np.testing.assert_array_equal(rt["idx"][0, 0], g["tie_variant"]["idx"])
+
+
+# ---------------------------------------------------------------- k = int(ratio * nb)
+
+@pytest.mark.parametrize("nb,ratio,want", [
+    (8, 0.25, 2), (8, 1.0, 8), (128, 0.3, 38), (256, 0.2, 51), (1024, 0.15, 153),
+    (4096, 0.15, 614), (100, 0.29, 28), (3, 0.1, 0), (10, 0.7, 7),
+])
+def test_topk_count_matches_python_int(oracle_mod, nb, ratio, want):
+    assert int(ratio * nb) == want  # what the page's int(topk_ratio * num_blocks) gives
+    assert oracle_mod.topk_count(nb, ratio) == want
+
+
+# ---------------------------------------------------------------- pooling
+
+def test_pool_block_size_one_is_identity(oracle_mod):
+    x = _rand((2, 6, 3, 5), 1, offsets=False)
+    p = oracle_mod.block_pool(x, 1)
+    np.testing.assert_array_equal(p, x.transpose(0, 2, 1, 3))
+
+
+def test_pool_constant_block_gives_the_row(oracle_mod):
+    B, nb, bs, H, D = 2, 3, 4, 2, 8
+    rows = _rand((B, nb, 1, H, D), 2, offsets=False)
+    x = np.broadcast_to(rows, (B, nb, bs, H, D)).reshape(B, nb * bs, H, D)
+    p = oracle_mod.block_pool(x, bs)
+    np.testing.assert_allclose(p, rows[:, :, 0].transpose(0, 2, 1, 3), rtol=1e-15)
+
+
+def test_pool_matches_numpy_mean(oracle_mod):
+    B, N, H, D, bs = 2, 64, 3, 16, 8
+    x = _rand((B, N, H, D), 3, bs=bs)
+    p = oracle_mod.block_pool(x, bs)
+    ref = x.reshape(B, N // bs, bs, H, D).mean(axis=2).transpose(0, 2, 1, 3)
+    np.testing.assert_allclose(p, ref, rtol=1e-13, atol=1e-15)
+
+
+def test_bf16_and_f32_inputs_convert_exactly(oracle_mod):
+    B, N, H, D, bs = 1, 16, 2, 8, 4
+    xt = torch.from_numpy(_rand((B, N, H, D), 4, bs=bs))
+    for dt in (torch.bfloat16, torch.float32):
+        x = xt.to(dt)
+        arr = x.view(torch.int16).numpy().view(np.uint16) if dt == torch.bfloat16 else x.numpy()
+        p = oracle_mod.block_pool(arr, 1)
+        np.testing.assert_array_equal(p, x.to(torch.float64).numpy().transpose(0, 2, 1, 3))
+
+
+# ---------------------------------------------------------------- block scores
+
+def test_scores_match_numpy_matmul(oracle_mod):
+    rng = np.random.default_rng(5)
+    qp = rng.standard_normal((2, 3, 7, 16))
+    kp = rng.standard_normal((2, 3, 7, 16))
+    S = oracle_mod.block_scores(qp, kp)
+    np.testing.assert_allclose(S, np.matmul(qp, kp.transpose(0, 1, 3, 2)), rtol=1e-13, atol=1e-13)
+    # a sample of rows picks the same rows out of the full matrix
+    rows = np.array([[[6, 1], [0, 3], [2, 2]], [[5, 4], [1, 0], [3, 6]]], np.int32)
+    Sr = oracle_mod.block_scores(qp, kp, rows)
+    full = np.matmul(qp, kp.transpose(0, 1, 3, 2))
+    np.testing.assert_allclose(Sr, np.take_along_axis(full, rows[..., None].astype(np.int64), 2),
+                               rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- top-k selection
+
+def _brute_topk(S, k):
+    out = np.empty(S.shape[:-1] + (k,), np.int32)
+    flat = S.reshape(-1, S.shape[-1])
+    for r, row in enumerate(flat):
+        j = np.arange(row.size)
+        order = np.lexsort((j, -row))  # score descending, then index ascending
+        out.reshape(-1, k)[r] = np.sort(order[:k])
+    return out
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_topk_matches_lexsort_brute_force_with_ties(oracle_mod, seed):
+    rng = np.random.default_rng(seed)
+    nb = int(rng.integers(5, 40))
+    S = rng.integers(-3, 4, size=(3, 2, nb, nb)).astype(np.float64)  # many exact ties
+    for k in (1, nb // 3 + 1, nb - 1, nb):
+        np.testing.assert_array_equal(oracle_mod.topk(S, k), _brute_topk(S, k))
+
+
+def test_topk_invariants(oracle_mod):
+    rng = np.random.default_rng(7)
+    S = rng.standard_normal((2, 3, 50, 50))
+    idx = oracle_mod.topk(S, 13)
+    assert np.all(np.diff(idx, axis=-1) > 0)  # ascending, distinct
+    for r in range(idx.reshape(-1, 13).shape[0]):
+        row = S.reshape(-1, 50)[r]
+        sel = idx.reshape(-1, 13)[r]
+        mask = np.zeros(50, bool)
+        mask[sel] = True
+        assert row[mask].min() >= row[~mask].max()
+    np.testing.assert_array_equal(oracle_mod.topk(S, 50)[0, 0, 0], np.arange(50))
+
+
+def test_topk_ties_go_to_lower_index(oracle_mod):
+    S = np.array([[0.5, 2.0, 1.0, 2.0, 1.0, 1.0, -1.0]])
+    np.testing.assert_array_equal(oracle_mod.topk(S, 1), [[1]])
+    np.testing.assert_array_equal(oracle_mod.topk(S, 2), [[1, 3]])
+    np.testing.assert_array_equal(oracle_mod.topk(S, 3), [[1, 2, 3]])
+    np.testing.assert_array_equal(oracle_mod.topk(S, 4), [[1, 2, 3, 4]])
+
+
+# ---------------------------------------------------------------- attention
+
+def _masked_dense(q, k, v, idx, bs, scale):
+    """Softmax(Mask(Q K^T * scale)) V with Mask from the selected blocks
+    ([MSA] §2.1), written with numpy over [B,N,H,D] float64."""
+    B, N, H, D = q.shape
+    nb = N // bs
+    out = np.empty_like(q)
+    for b in range(B):
+        for h in range(H):
+            logits = (q[b, :, h] @ k[b, :, h].T) * scale
+            mask = np.zeros((N, N), bool)
+            for i in range(nb):
+                for j in idx[b, h, i]:
+                    mask[i * bs:(i + 1) * bs, j * bs:(j + 1) * bs] = True
+            logits = np.where(mask, logits, -np.inf)
+            w = np.exp(logits - logits.max(axis=1, keepdims=True))
+            out[b, :, h] = (w / w.sum(axis=1, keepdims=True)) @ v[b, :, h]
+    return out
+
+
+def test_ratio_one_equals_dense_sdpa(oracle_mod):
+    B, N, H, D, bs = 2, 64, 2, 16, 8
+    q, k, v = (_rand((B, N, H, D), s, bs=bs) for s in (10, 11, 12))
+    r = oracle_mod.forward(q, k, v, bs, 1.0)
+    o = oracle_mod.o_to_bnhd(r["o"])
+    t = lambda x: torch.from_numpy(x).permute(0, 2, 1, 3)  # [B,H,N,D]
+    ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v)).permute(0, 2, 1, 3)
+    np.testing.assert_allclose(o, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_any_index_list_equals_masked_dense(oracle_mod):
+    B, N, H, D, bs = 1, 48, 2, 8, 6
+    q, k, v = (_rand((B, N, H, D), s, bs=bs) for s in (20, 21, 22))
+    rng = np.random.default_rng(23)
+    nb, kk = N // bs, 3
+    idx = np.sort(np.stack([[[rng.choice(nb, kk, replace=False) for _ in range(nb)]
+                             for _ in range(H)] for _ in range(B)]), axis=-1).astype(np.int32)
+    for scale in (1.0 / math.sqrt(D), 0.37):
+        o = oracle_mod.o_to_bnhd(oracle_mod.sparse_attn(q, k, v, idx, bs, scale=scale))
+        np.testing.assert_allclose(o, _masked_dense(q, k, v, idx, bs, scale), rtol=1e-12, atol=1e-12)
+
+
+def test_block_size_one_full_k_is_token_attention(oracle_mod):
+    B, N, H, D = 1, 12, 1, 4
+    q, k, v = (_rand((B, N, H, D), s, offsets=False) for s in (30, 31, 32))
+    r = oracle_mod.forward(q, k, v, 1, 1.0)
+    logits = q[0, :, 0] @ k[0, :, 0].T / 2.0
+    w = np.exp(logits - logits.max(1, keepdims=True))
+    ref = (w / w.sum(1, keepdims=True)) @ v[0, :, 0]
+    np.testing.assert_allclose(oracle_mod.o_to_bnhd(r["o"])[0, :, 0], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_sampled_rows_match_full_run(oracle_mod):
+    B, N, H, D, bs = 1, 64, 2, 8, 8
+    q, k, v = (_rand((B, N, H, D), s, bs=bs) for s in (40, 41, 42))
+    full = oracle_mod.forward(q, k, v, bs, 0.5)
+    rows = np.array([[[1, 6], [0, 7]]], np.int32)
+    part = oracle_mod.forward(q, k, v, bs, 0.5, rows=rows)
+    for h in range(H):
+        for r, i in enumerate(rows[0, h]):
+            np.testing.assert_array_equal(part["idx"][0, h, r], full["idx"][0, h, i])
+            np.testing.assert_array_equal(part["o"][0, h, r], full["o"][0, h, i])
+
+
+# ---------------------------------------------------------------- invariants
+
+@pytest.fixture(scope="module")
+def small_case():
+    B, N, H, D, bs = 2, 64, 2, 8, 8
+    q, k, v = (_rand((B, N, H, D), s, bs=bs) for s in (50, 51, 52))
+    return q, k, v, bs, 0.375
+
+
+def test_shift_and_linearity_in_v(oracle_mod, small_case):
+    q, k, v, bs, ratio = small_case
+    o = oracle_mod.o_to_bnhd(oracle_mod.forward(q, k, v, bs, ratio)["o"])
+    c = np.linspace(-1, 1, v.shape[-1])
+    o_shift = oracle_mod.o_to_bnhd(oracle_mod.forward(q, k, v + c, bs, ratio)["o"])
+    np.testing.assert_allclose(o_shift, o + c, rtol=1e-12, atol=1e-12)
+    v2 = _rand(v.shape, 53, offsets=False)
+    o2 = oracle_mod.o_to_bnhd(oracle_mod.forward(q, k, v2, bs, ratio)["o"])
+    o_lin = oracle_mod.o_to_bnhd(oracle_mod.forward(q, k, 2.0 * v - 3.0 * v2, bs, ratio)["o"])
+    np.testing.assert_allclose(o_lin, 2.0 * o - 3.0 * o2, rtol=1e-11, atol=1e-11)
+
+
+def test_permutations_inside_blocks(oracle_mod, small_case):
+    q, k, v, bs, ratio = small_case
+    B, N, H, D = q.shape
+    base = oracle_mod.forward(q, k, v, bs, ratio)
+    o = oracle_mod.o_to_bnhd(base["o"])
+    perm = np.arange(N).reshape(-1, bs)[:, ::-1].reshape(-1)  # reverse rows inside every block
+    # permuting key rows (k and v together) inside blocks leaves o unchanged
+    rk = oracle_mod.forward(q, k[:, perm], v[:, perm], bs, ratio)
+    np.testing.assert_array_equal(rk["idx"], base["idx"])
+    np.testing.assert_allclose(oracle_mod.o_to_bnhd(rk["o"]), o, rtol=1e-12, atol=1e-12)
+    # permuting query rows inside blocks permutes the output rows the same way
+    rq = oracle_mod.forward(q[:, perm], k, v, bs, ratio)
+    np.testing.assert_allclose(oracle_mod.o_to_bnhd(rq["o"]), o[:, perm], rtol=1e-12, atol=1e-12)
+
+
+def test_batch_head_permutation_and_block_relabel(oracle_mod, small_case):
+    q, k, v, bs, ratio = small_case
+    B, N, H, D = q.shape
+    base = oracle_mod.forward(q, k, v, bs, ratio)
+    o = oracle_mod.o_to_bnhd(base["o"])
+    pb, ph = [1, 0], [1, 0]
+    r = oracle_mod.forward(q[pb][:, :, ph], k[pb][:, :, ph], v[pb][:, :, ph], bs, ratio)
+    np.testing.assert_allclose(oracle_mod.o_to_bnhd(r["o"]), o[pb][:, :, ph], rtol=1e-12, atol=1e-12)
+    # relabel key blocks: swap key blocks 1 and 5 (k and v together)
+    nb = N // bs
+    bperm = np.arange(nb)
+    bperm[[1, 5]] = bperm[[5, 1]]
+    tok = (bperm[:, None] * bs + np.arange(bs)).reshape(-1)
+    r2 = oracle_mod.forward(q, k[:, tok], v[:, tok], bs, ratio)
+    relabeled = np.sort(bperm[base["idx"]], axis=-1)
+    np.testing.assert_array_equal(r2["idx"], relabeled)
+    np.testing.assert_allclose(oracle_mod.o_to_bnhd(r2["o"]), o, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- the page's listing, restated
+
+def test_matches_restated_page_listing_in_torch(oracle_mod):
+    """The [SF] listing run in float64 torch on CPU, with the einsum applied to
+    head-major pooled tensors and the custom kernel replaced by dense attention
+    under the block mask; the random data has no exact score ties."""
+    B, N, H, D, bs, ratio = 2, 96, 3, 16, 8, 0.3
+    q, k, v = (torch.from_numpy(_rand((B, N, H, D), s, bs=bs)) for s in (60, 61, 62))
+    nb = N // bs
+    qb = q.view(B, nb, bs, H, D).mean(2).permute(0, 2, 1, 3)
+    kb = k.view(B, nb, bs, H, D).mean(2).permute(0, 2, 1, 3)
+    scores = torch.einsum("bhid,bhjd->bhij", qb, kb)
+    _, top = torch.topk(scores, k=int(ratio * nb), dim=-1)
+    mask = torch.zeros(B, H, nb, nb, dtype=torch.bool).scatter_(-1, top, True)
+    tok_mask = mask.repeat_interleave(bs, 2).repeat_interleave(bs, 3)
+    t = lambda x: x.permute(0, 2, 1, 3)
+    ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), attn_mask=tok_mask,
+                                                           scale=1.0 / math.sqrt(D))
+    r = oracle_mod.forward(q.numpy(), k.numpy(), v.numpy(), bs, ratio)
+    np.testing.assert_array_equal(r["idx"], np.sort(top.numpy(), -1))
+    np.testing.assert_allclose(oracle_mod.o_to_bnhd(r["o"]), t(ref).numpy(), rtol=1e-12, atol=1e-12)
