@@ -1,0 +1,350 @@
+#!/usr/bin/env python
+"""Throughput of the block-sparse attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c4] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch of synthetic inputs
+already resident in HBM: block pooling of q and k, block scores + top-k
+selection, and sparse attention, each through its C-ABI entry point (4 kernel
+launches), with CUDA events between the stages on the launching stream.
+value = query tokens processed by all ranks / (max over ranks of the device
+time of the K timed steps). With --gpus N > 1 (under torchrun) every rank runs
+its own copy of the workload on its own GPU (the (b, h) problems are
+independent, so there is no data-path collective): weak scaling.
+
+--impl reference times the float64 CPU oracle on the host cores instead (a
+bounded sample of query blocks per step; rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "block-sparse attn fwd tokens/s & effective TFLOP/s (% roofline), 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.path = None
+        try:
+            pr = torch.cuda.get_device_properties(device)
+            self.bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+        except Exception:
+            self.bus = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.bus:
+            cmd += ["-i", self.bus]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]), f[4], f[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[4]) if v.lower() == "active"})
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+
+
+# ---------------------------------------------------------------- oracle (CPU) timing
+
+def oracle_sample(q, k, v, cfg: W.Config, heads, blocks_per_head: int, seed: int):
+    """Runs the oracle's whole path for `blocks_per_head` random query blocks of
+    each head in `heads` (each head is an independent single-head problem) and
+    returns (query tokens, seconds, threads)."""
+    import oracle
+
+    oracle.build()
+    rng = np.random.default_rng(seed)
+    tokens, secs = 0, 0.0
+    for h in heads:
+        qa, ka, va = (np.ascontiguousarray(W.to_oracle_array(x[:, :, h:h + 1])) for x in (q, k, v))
+        rows = np.sort(rng.choice(cfg.nb, size=(1, 1, blocks_per_head), replace=False), axis=-1).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.forward(qa, ka, va, cfg.block_size, cfg.topk_ratio, rows=rows)
+        secs += time.perf_counter() - t0
+        tokens += blocks_per_head * cfg.block_size * cfg.B
+    return tokens, secs, oracle.num_threads()
+
+
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return
+    q, k, v = W.make_inputs(cfg, device="cpu")
+    heads = list(range(cfg.H))
+    for s in range(args.warmup):
+        oracle_sample(q, k, v, cfg, [heads[s % cfg.H]], 1, seed=100 + s)
+    tok, sec, thr = 0, 0.0, 1
+    for s in range(args.steps):
+        t, dt, thr = oracle_sample(q, k, v, cfg, [heads[s % cfg.H]], 1, seed=1000 + s)
+        tok += t
+        sec += dt
+    value = tok / sec
+    sample = (f"{args.steps} steps x 1 query block ({cfg.block_size * cfg.B} tokens) of one head each, "
+              f"whole oracle path per step incl. pooling that head's k")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": f"{cfg.name}: {cfg.describe()}", "seed": cfg.seed},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our path
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="c4", choices=sorted(W.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-blocks-per-head", type=int, default=8)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = W.CONFIGS[args.config]
+
+    if args.impl == "reference":
+        run_reference(args, cfg, rank, world)
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    import block_sparse_attention_19_b200 as bsa
+
+    B, N, H, D, bs, ratio = cfg.B, cfg.N, cfg.H, cfg.D, cfg.block_size, cfg.topk_ratio
+    kk = bsa.bsa_topk_count(N // bs, ratio)
+    q, k, v = W.make_inputs(cfg, device=dev)
+    ws = torch.empty(bsa.bsa_forward_workspace_bytes(B, N, H, D, bs, ratio), device=dev, dtype=torch.uint8)
+    qp, kp, idx = bsa.workspace_views(ws, B, N, H, D, bs, ratio)
+    o = torch.empty_like(q)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record()
+        bsa.bsa_block_pool(q, bs, out=qp)
+        bsa.bsa_block_pool(k, bs, out=kp)
+        if ev is not None:
+            ev[1].record()
+        bsa.bsa_block_scores_topk(qp, kp, kk, idx_out=idx)
+        if ev is not None:
+            ev[2].record()
+        bsa.bsa_sparse_attn_fwd(q, k, v, idx, bs, out=o)
+        if ev is not None:
+            ev[3].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if bsa.bsa_device_error() != 0:
+        raise RuntimeError("a kernel gave up on a bounded wait during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start.record()
+    for s in range(args.steps):
+        step(evs[s])
+    t_end.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    pool_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    sel_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    attn_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    if dist:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    err = bsa.bsa_device_error()
+    if err != 0:
+        raise RuntimeError(f"a kernel gave up on a bounded wait (code {err})")
+
+    # ---- fused entry point, same inputs (reported beside the stage-by-stage step)
+    fused_ms = None
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nf = max(3, args.steps // 4)
+    f0.record()
+    for _ in range(nf):
+        bsa.bsa_forward(q, k, v, bs, ratio, workspace=ws, out=o)
+    f1.record()
+    torch.cuda.synchronize()
+    fused_ms = f0.elapsed_time(f1) / nf
+
+    # ---- end to end: pinned host inputs -> device -> bsa_forward -> host output
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    for _ in range(2):
+        dq.copy_(hq, non_blocking=True); dk.copy_(hk, non_blocking=True); dv.copy_(hv, non_blocking=True)
+        bsa.bsa_forward(dq, dk, dv, bs, ratio, workspace=ws, out=o)
+        ho.copy_(o, non_blocking=True)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.e2e_steps):
+        dq.copy_(hq, non_blocking=True); dk.copy_(hk, non_blocking=True); dv.copy_(hv, non_blocking=True)
+        bsa.bsa_forward(dq, dk, dv, bs, ratio, workspace=ws, out=o)
+        ho.copy_(o, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(x.numel() * x.element_size() for x in (q, k, v))
+    d2h = o.numel() * o.element_size()
+    del hq, hk, hv, ho, dq, dk, dv
+
+    tokens_step = B * N
+    value = world * tokens_step * args.steps / (total_ms / 1e3)
+    e2e_value = world * tokens_step * args.e2e_steps / (e2e_ms / 1e3)
+    flops = 4.0 * B * H * N * kk * bs * D
+    esz = cfg.elem_bytes
+    tensor_bytes = B * N * H * D * esz
+    idx_bytes = B * H * (N // bs) * kk * 4
+    pooled_bytes = 2 * B * H * (N // bs) * D * 4
+    alg_bytes = 4 * tensor_bytes + idx_bytes  # q, k, v read + o written, and the index list
+    sel_bytes = 2 * tensor_bytes + idx_bytes  # selection stage: q, k read + index list written
+    peaks, peak_src = load_peaks()
+    step_ms = total_ms / args.steps
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: {cfg.describe()}", "seed": cfg.seed,
+                   "l2": f"inputs larger than L2 (q, k, v {tensor_bytes / 1e6:.0f} MB each)",
+                   "parallelism": f"replica per GPU x{world}"},
+        "tflops_effective": flops / (step_ms / 1e3) / 1e12,
+        "gpu_launches": 4 * args.steps,
+        "stages_ms": {"pool_qk": pool_ms, "scores_topk": sel_ms, "sparse_attn": attn_ms,
+                      "fused_bsa_forward": fused_ms},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": args.e2e_steps},
+        "clocks": clk,
+    }
+    if cfg.dtype == "bf16":
+        achieved = flops / (attn_ms / 1e3) / 1e12
+        roof_t = max(flops / (peaks["bf16_tflops"] * 1e12), alg_bytes / (peaks["hbm_gbs"] * 1e9))
+        line["roofline"] = {
+            "kernel": "sparse_attn_tc_kernel", "bound": "tensor", "achieved": achieved,
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+            "peak_source": f"{peak_src} bf16 burst", "traffic": None,
+            "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+            "frac_of_roofline_time": roof_t / (attn_ms / 1e3),
+            "flops_per_launch": flops, "algorithmic_bytes_per_launch": alg_bytes,
+        }
+    line["selection_stage"] = {
+        "bytes": sel_bytes, "ms": pool_ms + sel_ms,
+        "GB/s": sel_bytes / ((pool_ms + sel_ms) / 1e3) / 1e9,
+        "frac_of_hbm": sel_bytes / ((pool_ms + sel_ms) / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "pool_GB/s": (2 * tensor_bytes + pooled_bytes) / (pool_ms / 1e3) / 1e9,
+        "pool_frac_of_hbm": (2 * tensor_bytes + pooled_bytes) / (pool_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "peak": peaks["hbm_gbs"], "peak_source": f"{peak_src} HBM copy"}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        heads = list(range(cfg.H))
+        qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+        bpe = min(args.cpu_blocks_per_head, cfg.nb)
+        tok, sec, thr = oracle_sample(qc, kc, vc, cfg, heads, bpe, seed=cfg.seed + 2000)
+        line["cpu_baseline"] = {"value": tok / sec, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                                "sample": f"{bpe} random query blocks on each of {len(heads)} heads "
+                                          f"({tok} query tokens, {sec:.1f} s), whole oracle path per head "
+                                          f"incl. pooling all of that head's k"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+"""Python binding of libbsa: two-stage block-sparse attention on B200 (sm_100a).
+
+Argument marshalling only: every step runs in the CUDA kernels of
+``libbsa.so`` behind the C ABI of ``include/bsa.h``. PyTorch tensors serve as
+device buffers and torch's current stream is passed to each call. There is no
+fallback: if the library is missing or cannot load, importing this package
+raises.
+
+Functions carry the C names:
+
+* ``bsa_block_pool(x, block_size)``                -> pooled [B, H, nb, D] float32
+* ``bsa_block_scores_topk(q_pooled, k_pooled, topk, scores=False)`` -> idx (, scores)
+* ``bsa_sparse_attn_fwd(q, k, v, idx, block_size, scale=None)`` -> o
+* ``bsa_forward(q, k, v, block_size, topk_ratio, workspace=None)`` -> o
+* ``bsa_topk_count``, ``bsa_forward_workspace_bytes``, ``bsa_device_error``
+
+q, k, v, o are [B, N, H, D] (float32 or bfloat16), contiguous, on one CUDA
+device.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbsa.so")
+
+BSA_F32, BSA_BF16 = 0, 1
+_STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "BSA_ERR_MISALIGNED",
+           4: "BSA_ERR_WORKSPACE", 5: "BSA_ERR_CUDA", 6: "BSA_ERR_DEVICE"}
+
+#: every function include/bsa.h declares
+EXPORTED = ("bsa_topk_count", "bsa_forward_workspace_bytes", "bsa_block_pool",
+            "bsa_block_scores_topk", "bsa_sparse_attn_fwd", "bsa_forward", "bsa_status_string",
+            "bsa_last_error_detail", "bsa_device_error")
+
+
+class BsaError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        self.status = status
+        super().__init__(f"{_STATUS.get(status, status)}: {detail}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libbsa.so is not built ({LIB_PATH}); run "
+                          "`python -m block_sparse_attention_19_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, D, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
+    F = ctypes.c_float
+    sig = {
+        "bsa_topk_count": ([I, D], I),
+        "bsa_forward_workspace_bytes": ([I, I, I, I, I, D], Z),
+        "bsa_block_pool": ([P, P, I, I, I, I, I, I, P], I),
+        "bsa_block_scores_topk": ([P, P, P, P, I, I, I, I, I, P], I),
+        "bsa_sparse_attn_fwd": ([P, P, P, P, P, I, I, I, I, I, I, F, I, P], I),
+        "bsa_forward": ([P, P, P, P, I, I, I, I, I, D, I, P, Z, P], I),
+        "bsa_status_string": ([I], ctypes.c_char_p),
+        "bsa_last_error_detail": ([], ctypes.c_char_p),
+        "bsa_device_error": ([ctypes.POINTER(ctypes.c_int), P], I),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+lib = _load()
+
+
+def _check(status: int):
+    if status != 0:
+        raise BsaError(status, lib.bsa_last_error_detail().decode())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return BSA_F32
+    if t.dtype == torch.bfloat16:
+        return BSA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _p(t: torch.Tensor | None):
+    return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+
+
+def bsa_topk_count(nb: int, topk_ratio: float) -> int:
+    return lib.bsa_topk_count(int(nb), float(topk_ratio))
+
+
+def bsa_forward_workspace_bytes(B: int, N: int, H: int, D: int, block_size: int, topk_ratio: float) -> int:
+    return lib.bsa_forward_workspace_bytes(B, N, H, D, block_size, float(topk_ratio))
+
+
+def bsa_block_pool(x: torch.Tensor, block_size: int, out: torch.Tensor | None = None) -> torch.Tensor:
+    _dev(x, "x")
+    B, N, H, D = x.shape
+    if out is None:
+        out = torch.empty((B, H, N // block_size, D), device=x.device, dtype=torch.float32)
+    _check(lib.bsa_block_pool(_p(x), _p(out), B, N, H, D, block_size, _dtype_code(x), _stream(x)))
+    return out
+
+
+def bsa_block_scores_topk(q_pooled: torch.Tensor, k_pooled: torch.Tensor, topk: int,
+                          scores: bool = False, idx_out: torch.Tensor | None = None):
+    _dev(q_pooled, "q_pooled")
+    _dev(k_pooled, "k_pooled")
+    if q_pooled.dtype != torch.float32 or k_pooled.dtype != torch.float32:
+        raise TypeError("pooled tensors must be float32")
+    B, H, nb, D = q_pooled.shape
+    idx = idx_out if idx_out is not None else torch.empty((B, H, nb, topk), device=q_pooled.device, dtype=torch.int32)
+    S = torch.empty((B, H, nb, nb), device=q_pooled.device, dtype=torch.float32) if scores else None
+    _check(lib.bsa_block_scores_topk(_p(q_pooled), _p(k_pooled), _p(S), _p(idx), B, H, nb, D, topk,
+                                     _stream(q_pooled)))
+    return (idx, S) if scores else idx
+
+
+def bsa_sparse_attn_fwd(q, k, v, idx, block_size: int, scale: float | None = None,
+                        out: torch.Tensor | None = None) -> torch.Tensor:
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (idx, "idx")):
+        _dev(t, n)
+    if idx.dtype != torch.int32:
+        raise TypeError("idx must be int32")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    B, N, H, D = q.shape
+    topk = idx.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    o = out if out is not None else torch.empty_like(q)
+    _check(lib.bsa_sparse_attn_fwd(_p(q), _p(k), _p(v), _p(idx), _p(o), B, N, H, D, block_size, topk,
+                                   float(scale), _dtype_code(q), _stream(q)))
+    return o
+
+
+def bsa_forward(q, k, v, block_size: int, topk_ratio: float, workspace: torch.Tensor | None = None,
+                out: torch.Tensor | None = None) -> torch.Tensor:
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    B, N, H, D = q.shape
+    need = bsa_forward_workspace_bytes(B, N, H, D, block_size, topk_ratio)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
+    o = out if out is not None else torch.empty_like(q)
+    _check(lib.bsa_forward(_p(q), _p(k), _p(v), _p(o), B, N, H, D, block_size, float(topk_ratio),
+                           _dtype_code(q), _p(workspace), workspace.numel() * workspace.element_size(),
+                           _stream(q)))
+    return o
+
+
+def bsa_device_error(device=None) -> int:
+    """Synchronises the current stream and returns (and clears) the device error word."""
+    code = ctypes.c_int(0)
+    stream = torch.cuda.current_stream(device).cuda_stream
+    _check(lib.bsa_device_error(ctypes.byref(code), ctypes.c_void_p(stream)))
+    return code.value
+
+
+def workspace_views(ws: torch.Tensor, B: int, N: int, H: int, D: int, block_size: int, topk_ratio: float):
+    """The pooled q, pooled k and index-list sections of a bsa_forward workspace
+    (the layout of include/bsa.h: three 256-byte aligned sections)."""
+    nb = N // block_size
+    kk = bsa_topk_count(nb, topk_ratio)
+    pooled = ((B * H * nb * D * 4) + 255) // 256 * 256
+    base = ws.view(torch.uint8)
+    qp = base[:B * H * nb * D * 4].view(torch.float32).view(B, H, nb, D)
+    kp = base[pooled:pooled + B * H * nb * D * 4].view(torch.float32).view(B, H, nb, D)
+    idx = base[2 * pooled:2 * pooled + B * H * nb * kk * 4].view(torch.int32).view(B, H, nb, kk)
+    return qp, kp, idx

@@ -1,0 +1,390 @@
+// bsa_api.cu -- the C ABI declared in include/bsa.h: argument checks,
+// workspace layout, tensor-map encoding and kernel launches. The whole library
+// is this one translation unit (it includes the kernel headers), so the
+// device-side error word has a single definition.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "attn_simt.cuh"
+#include "attn_tc.cuh"
+#include "bsa.h"
+#include "bsa_ptx.cuh"
+#include "pool.cuh"
+#include "select.cuh"
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+bsa_status fail(bsa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+bsa_status ok() {
+  g_detail[0] = '\0';
+  return BSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bsa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(BSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------------ shapes
+
+bsa_status check_dims(int B, int N, int H, int D, int block_size) {
+  if (B < 1 || N < 1 || H < 1 || D < 1 || block_size < 1)
+    return fail(BSA_ERR_INVALID_ARG, "sizes must be positive (B=%d N=%d H=%d D=%d block_size=%d)",
+                B, N, H, D, block_size);
+  if (N % block_size != 0)
+    return fail(BSA_ERR_INVALID_ARG, "N=%d is not a multiple of block_size=%d", N, block_size);
+  if (D != 64 && D != 128) return fail(BSA_ERR_UNSUPPORTED, "D=%d (supported: 64, 128)", D);
+  if (block_size != 64 && block_size != 128 && block_size != 256)
+    return fail(BSA_ERR_UNSUPPORTED, "block_size=%d (supported: 64, 128, 256)", block_size);
+  if (static_cast<long long>(B) * H > (1ll << 24) || static_cast<long long>(N) > (1ll << 30))
+    return fail(BSA_ERR_UNSUPPORTED, "B*H or N too large for the launch grid");
+  return BSA_OK;
+}
+
+bsa_status check_dtype(bsa_dtype dt) {
+  if (dt != BSA_F32 && dt != BSA_BF16) return fail(BSA_ERR_UNSUPPORTED, "dtype %d", static_cast<int>(dt));
+  return BSA_OK;
+}
+
+// ------------------------------------------------------------------ device
+
+// The kernels are built for sm_100a only.
+bsa_status check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(BSA_ERR_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
+  static int cached_ok[64] = {0};  // 0 unknown, 1 ok, -1 unsupported
+  if (dev < 64 && cached_ok[dev] == 1) return BSA_OK;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) {
+    if (dev < 64) cached_ok[dev] = -1;
+    return fail(BSA_ERR_DEVICE, "device %d is sm_%d%d; libbsa is built for sm_100a", dev, major, minor);
+  }
+  if (dev < 64) cached_ok[dev] = 1;
+  return BSA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [B, N, H, D] bf16 tensor as a 4-D TMA map {D, H, N, B}; box = 64 columns x
+// 1 head x 64 rows x 1 batch, 128-byte swizzle (the UMMA K-/MN-major layout).
+bsa_status make_bnhd_map(CUtensorMap* map, const void* base, int B, int N, int H, int D) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
+                           static_cast<cuuint64_t>(N) * H * D * 2};
+  cuuint32_t box[4] = {64, 1, 64, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return BSA_OK;
+}
+
+// ------------------------------------------------------------------ launches
+
+bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int ntasks, int B,
+                       int N, int H, int D, int bs, bsa_dtype dt, cudaStream_t st) {
+  const int V = dt == BSA_F32 ? 4 : 8;
+  const int C = H * D / V;
+  const int cw = bsa::pool_column_group(C);
+  const long grid = static_cast<long>(ntasks) * B * (N / bs) * (C / cw);
+  if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "pool grid too large");
+  bsa::PoolTask t0{x0, p0}, t1{x1 ? x1 : x0, p1 ? p1 : p0};
+  if (dt == BSA_F32)
+    bsa::block_pool_kernel<float><<<static_cast<unsigned>(grid), bsa::kPoolThreads, 0, st>>>(t0, t1, B, N, H, D, bs, cw);
+  else
+    bsa::block_pool_kernel<__nv_bfloat16><<<static_cast<unsigned>(grid), bsa::kPoolThreads, 0, st>>>(t0, t1, B, N, H, D, bs, cw);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_pool_kernel launch");
+}
+
+template <int R>
+bsa_status launch_select_r(const float* qp, const float* kp, float* scores, int32_t* idx, int B,
+                           int H, int nb, int D, int k, cudaStream_t st) {
+  const size_t smem = (static_cast<size_t>(R) * D + static_cast<size_t>(R) * nb) * sizeof(float);
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(bsa::block_scores_topk_kernel<R>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (R * 128 + bsa::kSelSmemScoreBytes / 4) * 4);
+    if (e != cudaSuccess) return cuda_fail(e, "select smem attribute");
+    attr_set[dev] = true;
+  }
+  const long grid = static_cast<long>(B) * H * ((nb + R - 1) / R);
+  bsa::block_scores_topk_kernel<R><<<static_cast<unsigned>(grid), bsa::kSelThreads, smem, st>>>(
+      qp, kp, scores, idx, H, nb, D, k);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_scores_topk_kernel launch");
+}
+
+bsa_status launch_select(const float* qp, const float* kp, float* scores, int32_t* idx, int B,
+                         int H, int nb, int D, int k, cudaStream_t st) {
+  switch (bsa::select_rows_per_cta(nb)) {
+    case 32: return launch_select_r<32>(qp, kp, scores, idx, B, H, nb, D, k, st);
+    case 16: return launch_select_r<16>(qp, kp, scores, idx, B, H, nb, D, k, st);
+    case 8: return launch_select_r<8>(qp, kp, scores, idx, B, H, nb, D, k, st);
+    case 4: return launch_select_r<4>(qp, kp, scores, idx, B, H, nb, D, k, st);
+    case 2: return launch_select_r<2>(qp, kp, scores, idx, B, H, nb, D, k, st);
+    default: return launch_select_r<1>(qp, kp, scores, idx, B, H, nb, D, k, st);
+  }
+}
+
+template <int D>
+bsa_status launch_attn_simt(const float* q, const float* k, const float* v, const int32_t* idx,
+                            float* o, int B, int N, int H, int bs, int kk, float scale,
+                            cudaStream_t st) {
+  const size_t smem = sizeof(bsa::SimtSmem<D>);
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_simt_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_fail(e, "simt smem attribute");
+    attr_set[dev] = true;
+  }
+  const long grid = static_cast<long>(B) * H * (N / bs) * (bs / bsa::kSimtRows);
+  if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
+  bsa::sparse_attn_simt_kernel<D><<<static_cast<unsigned>(grid), bsa::kSimtThreads, smem, st>>>(
+      q, k, v, idx, o, N, H, bs, kk, scale);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_simt_kernel launch");
+}
+
+template <int D, int BM>
+bsa_status launch_attn_tc(const void* q, const void* k, const void* v, const int32_t* idx,
+                          void* o, int B, int N, int H, int bs, int kk, float scale,
+                          cudaStream_t st) {
+  using L = bsa::TcLayout<D, BM>;
+  CUtensorMap mq, mk, mv;
+  bsa_status s;
+  if ((s = make_bnhd_map(&mq, q, B, N, H, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mk, k, B, N, H, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mv, v, B, N, H, D)) != BSA_OK) return s;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_tc_kernel<D, BM>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
+    if (e != cudaSuccess) return cuda_fail(e, "tc smem attribute");
+    attr_set[dev] = true;
+  }
+  const int parts = bs > BM ? bs / BM : 1;
+  const long grid = static_cast<long>(B) * H * (N / bs) * parts;
+  if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
+  const float scale_log2 = scale * 1.4426950408889634f;
+  bsa::sparse_attn_tc_kernel<D, BM><<<static_cast<unsigned>(grid), bsa::kTcThreads, L::kSmemAlloc, st>>>(
+      mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, bs, kk, scale_log2);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc_kernel launch");
+}
+
+bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
+                       int B, int N, int H, int D, int bs, int kk, float scale, bsa_dtype dt,
+                       cudaStream_t st) {
+  if (dt == BSA_F32) {
+    const float *fq = static_cast<const float*>(q), *fk = static_cast<const float*>(k),
+                *fv = static_cast<const float*>(v);
+    float* fo = static_cast<float*>(o);
+    return D == 64 ? launch_attn_simt<64>(fq, fk, fv, idx, fo, B, N, H, bs, kk, scale, st)
+                   : launch_attn_simt<128>(fq, fk, fv, idx, fo, B, N, H, bs, kk, scale, st);
+  }
+  if (bs == 64)
+    return D == 64 ? launch_attn_tc<64, 64>(q, k, v, idx, o, B, N, H, bs, kk, scale, st)
+                   : launch_attn_tc<128, 64>(q, k, v, idx, o, B, N, H, bs, kk, scale, st);
+  return D == 64 ? launch_attn_tc<64, 128>(q, k, v, idx, o, B, N, H, bs, kk, scale, st)
+                 : launch_attn_tc<128, 128>(q, k, v, idx, o, B, N, H, bs, kk, scale, st);
+}
+
+struct Workspace {
+  float* qp;
+  float* kp;
+  int32_t* idx;
+  size_t bytes;
+};
+
+Workspace workspace_layout(void* base, int B, int N, int H, int D, int bs, int k) {
+  const size_t nb = static_cast<size_t>(N / bs);
+  const size_t pooled = align256(static_cast<size_t>(B) * H * nb * D * sizeof(float));
+  const size_t idxb = align256(static_cast<size_t>(B) * H * nb * k * sizeof(int32_t));
+  unsigned char* p = static_cast<unsigned char*>(base);
+  Workspace w;
+  w.qp = reinterpret_cast<float*>(p);
+  w.kp = reinterpret_cast<float*>(p + pooled);
+  w.idx = reinterpret_cast<int32_t*>(p + 2 * pooled);
+  w.bytes = 2 * pooled + idxb;
+  return w;
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+
+extern "C" {
+
+int bsa_topk_count(int nb, double topk_ratio) {
+  if (nb < 1 || !std::isfinite(topk_ratio) || topk_ratio < 0.0) return -1;
+  const double prod = topk_ratio * static_cast<double>(nb);
+  if (prod >= 2147483647.0) return -1;
+  return static_cast<int>(prod);  // truncation == Python int() for prod >= 0
+}
+
+size_t bsa_forward_workspace_bytes(int B, int N, int H, int D, int block_size, double topk_ratio) {
+  if (check_dims(B, N, H, D, block_size) != BSA_OK) return 0;
+  const int k = bsa_topk_count(N / block_size, topk_ratio);
+  if (k < 1 || k > N / block_size) return 0;
+  return workspace_layout(nullptr, B, N, H, D, block_size, k).bytes;
+}
+
+const char* bsa_status_string(bsa_status s) {
+  switch (s) {
+    case BSA_OK: return "ok";
+    case BSA_ERR_INVALID_ARG: return "invalid argument";
+    case BSA_ERR_UNSUPPORTED: return "unsupported size or type";
+    case BSA_ERR_MISALIGNED: return "device pointer not 16-byte aligned";
+    case BSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case BSA_ERR_CUDA: return "CUDA error";
+    case BSA_ERR_DEVICE: return "no usable sm_100 device";
+  }
+  return "unknown status";
+}
+
+const char* bsa_last_error_detail(void) { return g_detail; }
+
+bsa_status bsa_block_pool(const void* x, float* x_pooled, int B, int N, int H, int D,
+                          int block_size, bsa_dtype dt, void* stream) {
+  bsa_status s;
+  if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
+  if ((s = check_dtype(dt)) != BSA_OK) return s;
+  if (!x || !x_pooled) return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(x_pooled)) return fail(BSA_ERR_MISALIGNED, "x or x_pooled");
+  if ((s = check_device()) != BSA_OK) return s;
+  if ((s = launch_pool(x, x_pooled, nullptr, nullptr, 1, B, N, H, D, block_size, dt,
+                       static_cast<cudaStream_t>(stream))) != BSA_OK)
+    return s;
+  return ok();
+}
+
+bsa_status bsa_block_scores_topk(const float* q_pooled, const float* k_pooled, float* scores,
+                                 int32_t* idx, int B, int H, int nb, int D, int k, void* stream) {
+  bsa_status s;
+  if (B < 1 || H < 1 || nb < 1) return fail(BSA_ERR_INVALID_ARG, "sizes must be positive");
+  if (D != 64 && D != 128) return fail(BSA_ERR_UNSUPPORTED, "D=%d (supported: 64, 128)", D);
+  if (nb > 32768) return fail(BSA_ERR_UNSUPPORTED, "nb=%d > 32768", nb);
+  if (k < 1 || k > nb) return fail(BSA_ERR_INVALID_ARG, "k=%d outside [1, nb=%d]", k, nb);
+  if (!q_pooled || !k_pooled || !idx) return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q_pooled) || !aligned16(k_pooled) || !aligned16(idx) || (scores && !aligned16(scores)))
+    return fail(BSA_ERR_MISALIGNED, "q_pooled, k_pooled, idx or scores");
+  if ((s = check_device()) != BSA_OK) return s;
+  if ((s = launch_select(q_pooled, k_pooled, scores, idx, B, H, nb, D, k,
+                         static_cast<cudaStream_t>(stream))) != BSA_OK)
+    return s;
+  return ok();
+}
+
+bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx,
+                               void* o, int B, int N, int H, int D, int block_size, int kk,
+                               float scale, bsa_dtype dt, void* stream) {
+  bsa_status s;
+  if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
+  if ((s = check_dtype(dt)) != BSA_OK) return s;
+  const int nb = N / block_size;
+  if (kk < 1 || kk > nb) return fail(BSA_ERR_INVALID_ARG, "k=%d outside [1, nb=%d]", kk, nb);
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return fail(BSA_ERR_INVALID_ARG, "scale must be positive and finite");
+  if (!q || !k || !v || !idx || !o) return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(o))
+    return fail(BSA_ERR_MISALIGNED, "q, k, v, idx or o");
+  if (o == q || o == k || o == v) return fail(BSA_ERR_INVALID_ARG, "o aliases an input");
+  if ((s = check_device()) != BSA_OK) return s;
+  if ((s = launch_attn(q, k, v, idx, o, B, N, H, D, block_size, kk, scale, dt,
+                       static_cast<cudaStream_t>(stream))) != BSA_OK)
+    return s;
+  return ok();
+}
+
+bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int B, int N, int H,
+                       int D, int block_size, double topk_ratio, bsa_dtype dt, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  bsa_status s;
+  if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
+  if ((s = check_dtype(dt)) != BSA_OK) return s;
+  const int nb = N / block_size;
+  if (nb > 32768) return fail(BSA_ERR_UNSUPPORTED, "nb=%d > 32768", nb);
+  if (!std::isfinite(topk_ratio) || topk_ratio < 0.0 || topk_ratio > 1.0)
+    return fail(BSA_ERR_INVALID_ARG, "topk_ratio=%g outside [0, 1]", topk_ratio);
+  const int kk = bsa_topk_count(nb, topk_ratio);
+  if (kk < 1) return fail(BSA_ERR_INVALID_ARG, "k = int(%g * %d) = %d < 1", topk_ratio, nb, kk);
+  if (!q || !k || !v || !o) return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(BSA_ERR_MISALIGNED, "q, k, v or o");
+  if (o == q || o == k || o == v) return fail(BSA_ERR_INVALID_ARG, "o aliases an input");
+  const Workspace w = workspace_layout(workspace, B, N, H, D, block_size, kk);
+  if (!workspace || workspace_bytes < w.bytes)
+    return fail(BSA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", w.bytes, workspace ? workspace_bytes : 0);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(BSA_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  if ((s = check_device()) != BSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  if ((s = launch_pool(q, w.qp, k, w.kp, 2, B, N, H, D, block_size, dt, st)) != BSA_OK) return s;
+  if ((s = launch_select(w.qp, w.kp, nullptr, w.idx, B, H, nb, D, kk, st)) != BSA_OK) return s;
+  if ((s = launch_attn(q, k, v, w.idx, o, B, N, H, D, block_size, kk, scale, dt, st)) != BSA_OK) return s;
+  return ok();
+}
+
+bsa_status bsa_device_error(int* code_out, void* stream) {
+  if (!code_out) return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  bsa_status s;
+  if ((s = check_device()) != BSA_OK) return s;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int code = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&code, bsa::g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  e = cudaMemcpyToSymbol(bsa::g_device_error, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+  *code_out = code;
+  return ok();
+}
+
+}  // extern "C"

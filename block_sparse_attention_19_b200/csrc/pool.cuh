@@ -1,0 +1,130 @@
+// pool.cuh -- step 1a: block mean-pooling of q and k.
+//
+// Page "2026 新一代卷积与 Transformer 网络架构" (qqiyuan.cn), section
+// "SparseFormer 注意力实现", step 1: q.view(B, nb, bs, H, D).mean(2), and the
+// same for k. Output layout here is head-major [B, H, nb, D] float32 so that
+// each (b, h) score matrix reads contiguous rows.
+//
+// HBM-bound: every element of q and k is read exactly once with 16-byte
+// vector loads; the block's rows for all heads are contiguous in memory
+// (bs * H * D elements), so a work item is (tensor, b, block i, column group)
+// and its warps stream whole 512-byte row segments. Sums are float32.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace bsa {
+
+constexpr int kPoolThreads = 256;
+
+struct PoolTask {
+  const void* x;  // [B, N, H, D]
+  float* xp;      // [B, H, nb, D]
+};
+
+template <typename T>
+struct Vec16;  // 16 bytes of T, converted to floats
+template <>
+struct Vec16<float> {
+  static constexpr int kN = 4;
+  __device__ __forceinline__ static void add(float* acc, const uint4& u) {
+    acc[0] += __uint_as_float(u.x);
+    acc[1] += __uint_as_float(u.y);
+    acc[2] += __uint_as_float(u.z);
+    acc[3] += __uint_as_float(u.w);
+  }
+};
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int kN = 8;
+  __device__ __forceinline__ static void add(float* acc, const uint4& u) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      acc[2 * t] += __uint_as_float(w[t] << 16);
+      acc[2 * t + 1] += __uint_as_float(w[t] & 0xFFFF0000u);
+    }
+  }
+};
+
+// Columns (16-byte units) one work item covers: 64 when the row width allows,
+// else the largest divisor of the row width that fits the CTA.
+inline int pool_column_group(int C) {
+  if (C % 64 == 0) return 64;
+  int cw = C < kPoolThreads ? C : kPoolThreads;
+  while (C % cw) --cw;
+  return cw;
+}
+
+// grid.x = ntasks * B * nb * (C / cw). Each CTA reduces bs rows of one group of
+// cw 16-byte columns of one block; rows are split over kPoolThreads / cw
+// row groups.
+template <typename T>
+__global__ void __launch_bounds__(kPoolThreads)
+    block_pool_kernel(PoolTask t0, PoolTask t1, int B, int N, int H, int D, int bs, int cw) {
+  constexpr int V = Vec16<T>::kN;
+  const int nb = N / bs;
+  const int C = H * D / V;  // 16-byte columns per row
+  const int ngroups = C / cw;
+  const int G = kPoolThreads / cw;  // row groups (>= 1: cw <= 256 is checked by the host)
+
+  long item = blockIdx.x;
+  const int cg = static_cast<int>(item % ngroups);
+  item /= ngroups;
+  const int i = static_cast<int>(item % nb);
+  item /= nb;
+  const int b = static_cast<int>(item % B);
+  const int which = static_cast<int>(item / B);
+  const PoolTask task = which == 0 ? t0 : t1;
+
+  const int tid = threadIdx.x;
+  const int col = tid % cw;
+  const int rg = tid / cw;
+  const int c = cg * cw + col;  // 16-byte column within the row
+
+  float acc[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] = 0.f;
+
+  if (rg < G) {
+    const uint4* base = reinterpret_cast<const uint4*>(task.x) +
+                        (static_cast<size_t>(b) * N + static_cast<size_t>(i) * bs) * C + c;
+    int r = rg;
+    // 4 independent loads in flight per thread
+    for (; r + 3 * G < bs; r += 4 * G) {
+      uint4 u0 = __ldg(base + static_cast<size_t>(r) * C);
+      uint4 u1 = __ldg(base + static_cast<size_t>(r + G) * C);
+      uint4 u2 = __ldg(base + static_cast<size_t>(r + 2 * G) * C);
+      uint4 u3 = __ldg(base + static_cast<size_t>(r + 3 * G) * C);
+      Vec16<T>::add(acc, u0);
+      Vec16<T>::add(acc, u1);
+      Vec16<T>::add(acc, u2);
+      Vec16<T>::add(acc, u3);
+    }
+    for (; r < bs; r += G) Vec16<T>::add(acc, __ldg(base + static_cast<size_t>(r) * C));
+  }
+
+  // combine the row groups
+  __shared__ float part[kPoolThreads * 8];
+  if (rg < G) {
+#pragma unroll
+    for (int e = 0; e < V; ++e) part[(rg * cw + col) * V + e] = acc[e];
+  }
+  __syncthreads();
+  if (rg == 0) {
+    for (int g = 1; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < V; ++e) acc[e] += part[(g * cw + col) * V + e];
+    const float inv = 1.0f / static_cast<float>(bs);  // bs is a power of two: exact
+    const int h = (c * V) / D;
+    const int d0 = (c * V) % D;
+    float* out = task.xp + ((static_cast<size_t>(b) * H + h) * nb + i) * D + d0;
+#pragma unroll
+    for (int e = 0; e < V; e += 4)
+      *reinterpret_cast<float4*>(out + e) =
+          make_float4(acc[e] * inv, acc[e + 1] * inv, acc[e + 2] * inv, acc[e + 3] * inv);
+  }
+}
+
+}  // namespace bsa

@@ -1,0 +1,128 @@
+/*
+ * bsa.h -- C ABI of libbsa: two-stage block-sparse attention on NVIDIA B200
+ * (sm_100a).
+ *
+ * The method (page "2026 新一代卷积与 Transformer 网络架构", qqiyuan.cn,
+ * section "SparseFormer 注意力实现"; page "从M2.7到M3：多模态模型稀疏注意力架构
+ * 设计与实现全解析", cloud.baidu.com, §2.1-§2.2):
+ *   1. mean-pool q and k over blocks of block_size tokens and score every query
+ *      block against every key block: S[b,h,i,j] = qbar[b,h,i,:] . kbar[b,h,j,:];
+ *   2. keep, per (b, h, query block i), the k = floor(topk_ratio * nb) key
+ *      blocks with the largest scores (ties go to the lower block index);
+ *   3. for every query row n of block i, o[n] = softmax(scale * q[n] K_sel^T) V_sel
+ *      with K_sel / V_sel the k * block_size rows of the kept blocks and
+ *      scale = 1/sqrt(D) by default. Attention is non-causal.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are dense and row-major. q, k, v, o are [B, N, H, D] (the head
+ *     axis inside the token axis, as the page's listing takes them); pooled
+ *     tensors are [B, H, nb, D] float32; index lists are [B, H, nb, k] int32,
+ *     each row strictly ascending by key-block id.
+ *   - All pointers are DEVICE pointers unless stated otherwise. The caller owns
+ *     every buffer; the library allocates nothing on any call and keeps no
+ *     pointer after a call returns.
+ *   - Every device pointer must be 16-byte aligned (BSA_ERR_MISALIGNED).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream). Work is enqueued asynchronously; a call returns once its kernels
+ *     are launched. Faults inside a kernel surface at the caller's next
+ *     synchronisation; bsa_device_error() reports bounded-wait timeouts.
+ *   - Argument errors are detected on the host before anything is launched and
+ *     leave all buffers untouched. bsa_last_error_detail() then describes the
+ *     error (thread-local, valid until the next call on the same thread).
+ *   - Supported sizes: D in {64, 128}; block_size in {64, 128, 256};
+ *     N a multiple of block_size; 1 <= k <= nb; B, H >= 1. Offsets are
+ *     64-bit, so tensor sizes are bounded only by device memory.
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, N % block_size != 0, k out of range */
+  BSA_ERR_UNSUPPORTED = 2, /* D / block_size / dtype / size outside what the kernels implement */
+  BSA_ERR_MISALIGNED = 3,  /* a device pointer not 16-byte aligned */
+  BSA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than bsa_forward_workspace_bytes() */
+  BSA_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+  BSA_ERR_DEVICE = 6       /* no usable sm_100 device for this call */
+} bsa_status;
+
+typedef enum {
+  BSA_F32 = 0, /* float32 q/k/v/o; attention in float32 on CUDA cores */
+  BSA_BF16 = 1 /* bfloat16 q/k/v/o; attention on tcgen05 tensor cores, float32 accumulate */
+} bsa_dtype;
+
+/* Number of kept key blocks: floor(topk_ratio * nb) evaluated in IEEE double,
+ * which equals Python's int(topk_ratio * num_blocks) in the page's listing
+ * (step 2). Returns -1 if nb < 1 or topk_ratio is negative or not finite.
+ * Pure host function. */
+int bsa_topk_count(int nb, double topk_ratio);
+
+/* Bytes of device workspace bsa_forward() needs for these sizes (pooled q and
+ * k, and the index list, each section 256-byte aligned). Returns 0 when the
+ * arguments are invalid. Pure host function. */
+size_t bsa_forward_workspace_bytes(int B, int N, int H, int D, int block_size, double topk_ratio);
+
+/* Step 1a (page listing, step 1: x.view(B, nb, bs, H, D).mean(2)):
+ *   x_pooled[b, h, i, d] = (1/block_size) * sum_{t<block_size} x[b, i*block_size + t, h, d]
+ * x: [B, N, H, D] of dtype dt (read only). x_pooled: [B, H, nb, D] float32
+ * (written). Sums are accumulated in float32. */
+bsa_status bsa_block_pool(const void* x, float* x_pooled, int B, int N, int H, int D,
+                          int block_size, bsa_dtype dt, void* stream);
+
+/* Steps 1b + 2 (page listing: einsum of the pooled tensors per (b, h), then
+ * torch.topk over the key-block axis):
+ *   S[b, h, i, j] = sum_d q_pooled[b, h, i, d] * k_pooled[b, h, j, d]
+ *   idx[b, h, i, :] = the topk key blocks j with the largest S[b, h, i, j],
+ *                     ties to the lower j, written in ascending j.
+ * q_pooled, k_pooled: [B, H, nb, D] float32 (read). idx: [B, H, nb, topk] int32
+ * (written). scores: optional [B, H, nb, nb] float32 output of S (NULL = not
+ * written). Scores are float32 dot products; no 1/sqrt(D) factor (it would not
+ * change the ranking). */
+bsa_status bsa_block_scores_topk(const float* q_pooled, const float* k_pooled, float* scores,
+                                 int32_t* idx, int B, int H, int nb, int D, int topk, void* stream);
+
+/* Step 3 (page listing: sparse_attn_cuda(q, k, v, topk_indices, block_size,
+ * scale)): for every (b, h, query block i) and every row n of that block,
+ *   o[b, n, h, :] = sum_t softmax_t(scale * q[b,n,h,:] . k[b,t,h,:]) v[b,t,h,:]
+ * over the tokens t of the key blocks idx[b, h, i, 0..topk).
+ * q, k, v: [B, N, H, D] of dtype dt (read). idx: [B, H, nb, topk] int32 with
+ * entries in [0, nb) and each row strictly ascending (read; entries outside
+ * [0, nb) are clamped by the kernel). o: [B, N, H, D] of dtype dt (written);
+ * o must not alias q, k or v. scale: softmax scale (> 0, finite). */
+bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx,
+                               void* o, int B, int N, int H, int D, int block_size, int topk,
+                               float scale, bsa_dtype dt, void* stream);
+
+/* The whole path: bsa_block_pool on q and k, bsa_block_scores_topk (scores not
+ * kept), bsa_sparse_attn_fwd with scale = 1/sqrt(D); three kernel launches on
+ * `stream`, no host synchronisation. k = bsa_topk_count(N / block_size,
+ * topk_ratio) must be >= 1. workspace: device buffer of at least
+ * bsa_forward_workspace_bytes(...) bytes, 256-byte aligned, owned by the caller
+ * and not used concurrently by another call. */
+bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int B, int N, int H,
+                       int D, int block_size, double topk_ratio, bsa_dtype dt, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* Static description of a status code. */
+const char* bsa_status_string(bsa_status s);
+
+/* Detail of the last error returned on this thread ("" if none). */
+const char* bsa_last_error_detail(void);
+
+/* Reads and clears the device-side error word of the current device: 0 when no
+ * kernel gave up on a bounded wait since the last call, otherwise the code of
+ * the first wait that timed out. Synchronises `stream` first. */
+bsa_status bsa_device_error(int* code_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H */

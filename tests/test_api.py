@@ -1,0 +1,117 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+function include/bsa.h declares, and rejects bad arguments on the host before
+touching the device (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bsa():
+    from block_sparse_attention_19_b200 import build
+
+    build.build()
+    import block_sparse_attention_19_b200 as m
+
+    return m
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "bsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bsa_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(bsa):
+    declared = _declared_functions()
+    assert len(declared) >= 9
+    assert set(declared) == set(bsa.EXPORTED)
+    lib = ctypes.CDLL(bsa.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+@pytest.mark.parametrize("nb,ratio", [(8, 0.25), (8, 1.0), (128, 0.3), (256, 0.2), (1024, 0.15),
+                                      (4096, 0.15), (100, 0.29), (3, 0.1), (7, 0.999999)])
+def test_topk_count_is_python_int(bsa, nb, ratio):
+    assert bsa.bsa_topk_count(nb, ratio) == int(ratio * nb)
+
+
+def test_topk_count_rejects_bad_input(bsa):
+    assert bsa.bsa_topk_count(0, 0.5) == -1
+    assert bsa.bsa_topk_count(8, -0.1) == -1
+    assert bsa.bsa_topk_count(8, float("nan")) == -1
+    assert bsa.bsa_topk_count(8, float("inf")) == -1
+
+
+def test_workspace_bytes(bsa):
+    # c4: pooled q and k [1,16,1024,128] f32 = 8 MiB each, idx [1,16,1024,153] i32
+    got = bsa.bsa_forward_workspace_bytes(1, 131072, 16, 128, 128, 0.15)
+    idx = 16 * 1024 * 153 * 4
+    assert got == 2 * 8 * 2**20 + (idx + 255) // 256 * 256
+    assert bsa.bsa_forward_workspace_bytes(1, 100, 2, 64, 64, 0.5) == 0  # N % block_size
+    assert bsa.bsa_forward_workspace_bytes(1, 512, 2, 96, 64, 0.5) == 0  # D unsupported
+    assert bsa.bsa_forward_workspace_bytes(1, 512, 2, 64, 64, 0.1) == 0  # k = 0
+
+
+def test_status_strings(bsa):
+    for code in range(7):
+        s = bsa.lib.bsa_status_string(code).decode()
+        assert s and s != "unknown status"
+    assert bsa.lib.bsa_status_string(99).decode() == "unknown status"
+
+
+# Fake, never-dereferenced pointer values: every case below fails validation on
+# the host, before any CUDA call.
+A = 0x10000  # 16-byte aligned
+M = 0x10004  # misaligned
+
+
+def _fwd(bsa, q=A, k=A, v=A, o=A + 0x100, B=1, N=512, H=2, D=64, bs=64, ratio=0.25, dt=1, ws=A + 0x200,
+         wsb=1 << 30):
+    P = ctypes.c_void_p
+    return bsa.lib.bsa_forward(P(q), P(k), P(v), P(o), B, N, H, D, bs, ratio, dt, P(ws), wsb, P(0))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=0), 1), (dict(o=0), 1), (dict(N=500), 1), (dict(B=0), 1), (dict(ratio=0.1), 1),
+    (dict(ratio=1.5), 1), (dict(ratio=float("nan")), 1), (dict(D=96), 2), (dict(bs=32, N=512), 2),
+    (dict(dt=7), 2), (dict(q=M), 3), (dict(v=M), 3), (dict(ws=0), 4), (dict(wsb=16), 4),
+    (dict(ws=A + 0x210), 3), (dict(o=A), 1),
+])
+def test_forward_rejects_bad_arguments(bsa, kw, status):
+    assert _fwd(bsa, **kw) == status
+    assert bsa.lib.bsa_last_error_detail().decode() != ""
+
+
+def test_stage_entry_points_reject_bad_arguments(bsa):
+    P = ctypes.c_void_p
+    L = bsa.lib
+    assert L.bsa_block_pool(P(0), P(A), 1, 512, 2, 64, 64, 1, P(0)) == 1
+    assert L.bsa_block_pool(P(A), P(M), 1, 512, 2, 64, 64, 1, P(0)) == 3
+    assert L.bsa_block_pool(P(A), P(A), 1, 500, 2, 64, 64, 1, P(0)) == 1
+    assert L.bsa_block_scores_topk(P(A), P(A), P(0), P(A), 1, 2, 8, 64, 0, P(0)) == 1
+    assert L.bsa_block_scores_topk(P(A), P(A), P(0), P(A), 1, 2, 8, 64, 9, P(0)) == 1
+    assert L.bsa_block_scores_topk(P(A), P(A), P(M), P(A), 1, 2, 8, 64, 2, P(0)) == 3
+    assert L.bsa_block_scores_topk(P(A), P(A), P(0), P(A), 1, 2, 8, 32, 2, P(0)) == 2
+    assert L.bsa_sparse_attn_fwd(P(A), P(A), P(A), P(A), P(A + 0x100), 1, 512, 2, 64, 64, 9, 0.125, 1, P(0)) == 1
+    assert L.bsa_sparse_attn_fwd(P(A), P(A), P(A), P(A), P(A + 0x100), 1, 512, 2, 64, 64, 2, -1.0, 1, P(0)) == 1
+    assert L.bsa_sparse_attn_fwd(P(A), P(A), P(A), P(0), P(A + 0x100), 1, 512, 2, 64, 64, 2, 0.125, 1, P(0)) == 1
+    assert L.bsa_sparse_attn_fwd(P(A), P(A), P(A), P(A), P(M), 1, 512, 2, 64, 64, 2, 0.125, 1, P(0)) == 3
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    """Importing the package with the library absent raises instead of falling back."""
+    import subprocess
+    import sys
+
+    pkg = tmp_path / "block_sparse_attention_19_b200"
+    pkg.mkdir()
+    (pkg / "__init__.py").write_text(open(os.path.join(ROOT, "block_sparse_attention_19_b200", "__init__.py")).read())
+    r = subprocess.run([sys.executable, "-c", "import block_sparse_attention_19_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "libbsa.so is not built" in r.stderr
