@@ -163,6 +163,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-blocks-per-head", type=int, default=8)
+    ap.add_argument("--stages-only", action="store_true",
+                    help="time the stage-by-stage steps only (no fused, end-to-end or CPU legs); "
+                         "for profiler runs")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -243,6 +246,16 @@ def main():
     err = bsa.bsa_device_error()
     if err != 0:
         raise RuntimeError(f"a kernel gave up on a bounded wait (code {err})")
+
+    if args.stages_only:
+        if rank == 0:
+            print(json.dumps({"stages_only": True, "config": cfg.name, "steps": args.steps,
+                              "ms_per_step": total_ms / args.steps,
+                              "stages_ms": {"pool_qk": pool_ms, "scores_topk": sel_ms, "sparse_attn": attn_ms}}),
+                  flush=True)
+        if dist:
+            dist.destroy_process_group()
+        return
 
     # ---- fused entry point, same inputs (reported beside the stage-by-stage step)
     fused_ms = None

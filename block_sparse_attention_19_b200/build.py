@@ -1,6 +1,9 @@
 """Builds libbsa.so (the C-ABI library) in-tree for sm_100a with nvcc.
 
-    python -m block_sparse_attention_19_b200.build [--force] [--verbose]
+    python block_sparse_attention_19_b200/build.py [--force] [--verbose]
+
+(run it by path: importing the package loads libbsa.so, which may not exist
+yet)
 
 The library is one translation unit (csrc/bsa_api.cu includes the kernels)
 linked against the static CUDA runtime, so it only needs the driver at run

@@ -18,3 +18,15 @@ def oracle_mod():
 
     oracle.build()
     return oracle
+
+
+def build_library():
+    """Builds libbsa.so through the package's build.py loaded by path (importing
+    the package would load a possibly stale or missing library first)."""
+    import importlib.util
+
+    path = os.path.join(ROOT, "block_sparse_attention_19_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("bsa_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()

@@ -12,9 +12,9 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def bsa():
-    from block_sparse_attention_19_b200 import build
+    from conftest import build_library
 
-    build.build()
+    build_library()
     import block_sparse_attention_19_b200 as m
 
     return m
