@@ -35,7 +35,7 @@ _STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "
 #: every function include/bsa.h declares
 EXPORTED = ("bsa_topk_count", "bsa_forward_workspace_bytes", "bsa_block_pool",
             "bsa_block_scores_topk", "bsa_sparse_attn_fwd", "bsa_forward", "bsa_status_string",
-            "bsa_last_error_detail", "bsa_device_error")
+            "bsa_last_error_detail", "bsa_device_error", "bsa_forward_noalloc")
 
 
 class BsaError(RuntimeError):
@@ -61,6 +61,7 @@ def _load() -> ctypes.CDLL:
         "bsa_status_string": ([I], ctypes.c_char_p),
         "bsa_last_error_detail": ([], ctypes.c_char_p),
         "bsa_device_error": ([ctypes.POINTER(ctypes.c_int), P], I),
+        "bsa_forward_noalloc": ([P, P, P, P, I, I, I, I, I, D, I, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -164,6 +165,21 @@ def bsa_forward(q, k, v, block_size: int, topk_ratio: float, workspace: torch.Te
     _check(lib.bsa_forward(_p(q), _p(k), _p(v), _p(o), B, N, H, D, block_size, float(topk_ratio),
                            _dtype_code(q), _p(workspace), workspace.numel() * workspace.element_size(),
                            _stream(q)))
+    return o
+
+
+def bsa_forward_noalloc(q, k, v, block_size: int, topk_ratio: float, out: torch.Tensor | None = None) -> torch.Tensor:
+    """bsa_forward with its intermediates in the library's fixed device scratch
+    (for callers that cannot allocate device memory; see include/bsa.h for the
+    size limit and the sharing rules)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    B, N, H, D = q.shape
+    o = out if out is not None else torch.empty_like(q)
+    _check(lib.bsa_forward_noalloc(_p(q), _p(k), _p(v), _p(o), B, N, H, D, block_size, float(topk_ratio),
+                                   _dtype_code(q), _stream(q)))
     return o
 
 

@@ -388,3 +388,67 @@ bsa_status bsa_device_error(int* code_out, void* stream) {
 }
 
 }  // extern "C"
+
+// ==================================================================== forward without allocation
+//
+// bsa_forward needs a workspace (pooled q, pooled k, index list) that the
+// caller allocates. Some callers cannot allocate device memory at all: a
+// plugin running inside a host application that owns the whole device-memory
+// budget, or a latency-critical loop where a cudaMalloc (and the implicit
+// device synchronisation it may bring) is not allowed. bsa_forward_noalloc
+// serves them from a fixed scratch array that is part of the library image.
+//
+// The array below lives in device memory of every GPU that loads this
+// library, from module load until process exit. Host code must not use its
+// name as a device address (on the host it is only a stand-in symbol): the
+// device address is looked up once per device with cudaGetSymbolAddress.
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[BSA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device; the first call
+// on each device performs the lookup (with that device current).
+bsa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(BSA_ERR_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(BSA_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return BSA_OK;
+}
+
+}  // namespace
+
+extern "C" bsa_status bsa_forward_noalloc(const void* q, const void* k, const void* v, void* o,
+                                          int B, int N, int H, int D, int block_size,
+                                          double topk_ratio, bsa_dtype dt, void* stream) {
+  bsa_status s;
+  if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
+  if (!std::isfinite(topk_ratio) || topk_ratio < 0.0 || topk_ratio > 1.0)
+    return fail(BSA_ERR_INVALID_ARG, "topk_ratio=%g outside [0, 1]", topk_ratio);
+  const size_t need = bsa_forward_workspace_bytes(B, N, H, D, block_size, topk_ratio);
+  if (need == 0) return fail(BSA_ERR_INVALID_ARG, "k = int(topk_ratio * nb) < 1");
+  if (need > static_cast<size_t>(BSA_NOALLOC_SCRATCH_BYTES))
+    return fail(BSA_ERR_WORKSPACE,
+                "these sizes need %zu bytes of scratch; the built-in scratch holds %zu bytes "
+                "(use bsa_forward with a caller-provided workspace)",
+                need, static_cast<size_t>(BSA_NOALLOC_SCRATCH_BYTES));
+  if ((s = check_device()) != BSA_OK) return s;
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != BSA_OK) return s;
+  // Nothing in the scratch has to start at zero: every byte the three
+  // kernels read was written earlier in the same call.
+  return bsa_forward(q, k, v, o, B, N, H, D, block_size, topk_ratio, dt, scratch,
+                     static_cast<size_t>(BSA_NOALLOC_SCRATCH_BYTES), stream);
+}

@@ -110,6 +110,31 @@ bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int
                        int D, int block_size, double topk_ratio, bsa_dtype dt, void* workspace,
                        size_t workspace_bytes, void* stream);
 
+/* Size of the fixed device scratch that bsa_forward_noalloc uses: 64 MiB. */
+#define BSA_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* bsa_forward without a caller workspace, for callers that cannot allocate
+ * device memory (for example a plugin inside a host application that owns the
+ * whole device-memory budget, or a loop where cudaMalloc and its implicit
+ * synchronisation are not allowed). The pages have no counterpart of this
+ * entry point; it only changes where the intermediates live.
+ *
+ * Arguments and results are those of bsa_forward minus the workspace. The
+ * pooled q, pooled k and index list go to a fixed 256-byte aligned array of
+ * BSA_NOALLOC_SCRATCH_BYTES in the library's device image: every GPU that
+ * loads libbsa holds it until the process exits. Sizes whose workspace
+ * (bsa_forward_workspace_bytes) exceeds it return BSA_ERR_WORKSPACE before
+ * anything is launched. The call allocates nothing (no cudaMalloc/cudaFree).
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current), so make that first call
+ * before any stream capture. All calls on a device share the one array and
+ * it keeps the last call's contents (nothing in it needs to start at zero):
+ * calls that may overlap on the GPU (different streams, or concurrent host
+ * threads) race on it and must be serialised by the caller. */
+bsa_status bsa_forward_noalloc(const void* q, const void* k, const void* v, void* o, int B, int N,
+                               int H, int D, int block_size, double topk_ratio, bsa_dtype dt,
+                               void* stream);
+
 /* Static description of a status code. */
 const char* bsa_status_string(bsa_status s);
 
