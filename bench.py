@@ -328,7 +328,8 @@ def main():
         achieved = flops / (attn_ms / 1e3) / 1e12
         roof_t = max(flops / (peaks["bf16_tflops"] * 1e12), alg_bytes / (peaks["hbm_gbs"] * 1e9))
         line["roofline"] = {
-            "kernel": "sparse_attn_tc_kernel", "bound": "tensor", "achieved": achieved,
+            "kernel": "sparse_attn_tc2_kernel" if bs in (128, 256) else "sparse_attn_tc_kernel",
+            "bound": "tensor", "achieved": achieved,
             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
             "peak_source": f"{peak_src} bf16 burst", "traffic": None,
             "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),

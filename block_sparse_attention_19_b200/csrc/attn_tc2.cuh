@@ -1,0 +1,410 @@
+// attn_tc2.cuh -- step 3 for bfloat16 inputs with block_size 128 or 256: two
+// 128-row query tiles per CTA so that the tensor core works on one tile while
+// the softmax runs on the other.
+//
+// Page "2026 新一代卷积与 Transformer 网络架构" (qqiyuan.cn), section
+// "SparseFormer 注意力实现", step 3 (sparse_attn_cuda, scale 1/sqrt(D)); page
+// "从M2.7到M3：多模态模型稀疏注意力架构设计与实现全解析" §2.2 (full attention inside
+// the chosen blocks): o = softmax(scale * q K_sel^T) V_sel per query row.
+//
+// Work unit (one CTA): two "streams" A and B of 128 query rows each.
+//   * block_size 256: the two halves of one query block. They share the key
+//     list, so every gathered K/V tile feeds both streams (half the L2
+//     traffic per flop).
+//   * block_size 128: two consecutive query blocks of one (b, h), each with
+//     its own key list; K/V tiles of the two streams alternate in the rings.
+//     With an odd number of blocks the last CTA runs stream A only.
+// Roles:
+//   * warp 0 (one lane): TMA loads of both query tiles and the K ring; warp 2
+//     (one lane): the V ring. Rings are filled in the order the MMA consumes
+//     them.
+//   * warp 1, lane 0: tcgen05.mma issue in the order S_A(0), S_B(0), then per
+//     key tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1). The softmax warps
+//     release K ring entries (they see each S complete); the issuing thread
+//     commits only the S the softmax waits for and the V entry it just read. S_X lives in TMEM
+//     columns of stream X; P_X (bf16) is written over the first 64 of them and
+//     read from TMEM as the A operand of PV_X; O_X accumulates in TMEM.
+//     Because tcgen05.mma ops of one thread run in order, S_X(j+1) cannot
+//     overwrite P_X(j) before PV_X(j) has read it, and the completion of
+//     S_X(j+1) implies that PV_X(j) is done (so O_X is stable).
+//   * warps 4-7 (stream A) and 8-11 (stream B): one query row per thread.
+//     Per tile: pass 1 reads the row of S from TMEM for its max; the running
+//     max (log2 domain) moves only when the tile max exceeds it by more than
+//     8, in which case O_X is rescaled in TMEM; pass 2 re-reads S, computes
+//     P = exp2(S * scale * log2 e - m) (one pair in four on the FMA pipe) and
+//     stores it as packed bf16 over S, chunk by chunk behind the reads.
+//   * warp 3 idle.
+// Every wait is bounded; on a timeout the device error word and an abort flag
+// are set, roles leave their loops, copies and MMAs are drained, TMEM is freed.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+#include "bsa_ptx.cuh"
+
+namespace bsa {
+
+constexpr int kTc2Threads = 384;  // 12 warps
+constexpr int kTc2MaxStages = 12;
+
+template <int D>
+struct Tc2Layout {
+  static constexpr uint32_t kTileBytes = 128 * D * 2;  // a 128-row Q, K or V tile
+  static constexpr int kKStages = D == 128 ? 3 : 6;
+  static constexpr int kVStages = D == 128 ? 2 : 6;
+  static constexpr int kChunks = D / 64;
+  static constexpr uint32_t kQOff = 0;  // Q_A, Q_B
+  static constexpr uint32_t kKOff = 2 * kTileBytes;
+  static constexpr uint32_t kVOff = kKOff + kKStages * kTileBytes;
+  static constexpr uint32_t kBarOff = kVOff + kVStages * kTileBytes;
+  static constexpr uint32_t kBytes = kBarOff + 512;
+  static constexpr uint32_t kTmemCols = 512;  // S_A | S_B | O_A | O_B
+  __device__ static constexpr uint32_t col_s(int x) { return 128u * x; }
+  __device__ static constexpr uint32_t col_o(int x) { return 256u + 128u * x; }
+  static_assert(kBytes <= 232448, "shared memory budget");
+  static_assert(kKStages <= kTc2MaxStages && kVStages <= kTc2MaxStages, "stage count");
+};
+
+struct Tc2Barriers {
+  uint64_t q_full;
+  uint64_t k_full[kTc2MaxStages], k_empty[kTc2MaxStages];
+  uint64_t v_full[kTc2MaxStages], v_empty[kTc2MaxStages];
+  uint64_t s_full[2];   // phase j: S_X(j) computed
+  uint64_t p_full[2];   // phase j: P_X(j) stored (and O_X rescaled if needed)
+  uint64_t pv_last[2];  // phase 0: the last PV_X completed
+  uint64_t mma_drained;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Tc2Barriers) <= 512, "barrier area");
+
+// Token row where 64-row half `hf` of stream `x`'s key tile t starts.
+__device__ __forceinline__ int tc2_key_row(const int32_t* sel_a, const int32_t* sel_b, int x,
+                                           int t, int hf, int bs, int nb) {
+  if (bs == 128) {
+    const int32_t* sel = x == 0 ? sel_a : sel_b;
+    return clamp_block(__ldg(sel + t), nb) * 128 + hf * 64;
+  }
+  return clamp_block(__ldg(sel_a + t / 2), nb) * 256 + (t % 2) * 128 + hf * 64;  // bs == 256
+}
+
+// grid.x = B * H * ceil(nb / 2) for block_size 128, B * H * nb for 256.
+template <int D>
+__global__ void __launch_bounds__(kTc2Threads, 1)
+    sparse_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q,
+                           const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v,
+                           const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ o, int N,
+                           int H, int bs, int k, float scale_log2) {
+  using L = Tc2Layout<D>;
+  constexpr int KS = L::kKStages, VS = L::kVStages;
+  extern __shared__ __align__(1024) unsigned char tc2_raw[];
+  // swizzled tiles need 1024-byte alignment and the layout has no slack
+  if ((smem_u32(tc2_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) report_error(402);
+    return;
+  }
+  unsigned char* smem = tc2_raw;
+  Tc2Barriers& bar = *reinterpret_cast<Tc2Barriers*>(smem + L::kBarOff);
+  volatile int* abort_flag = &bar.abort;
+
+  const int nb = N / bs;
+  const bool shared_kv = bs == 256;
+  const int per_bh = shared_kv ? nb : (nb + 1) / 2;
+  long u = blockIdx.x;
+  const int unit = static_cast<int>(u % per_bh);
+  u /= per_bh;
+  const int h = static_cast<int>(u % H);
+  const int b = static_cast<int>(u / H);
+  // stream x covers query rows [row0[x], row0[x] + 128)
+  const int iA = shared_kv ? unit : 2 * unit;
+  const int nstreams = (!shared_kv && iA + 1 >= nb) ? 1 : 2;
+  const int row0[2] = {iA * bs, shared_kv ? iA * bs + 128 : (iA + 1) * bs};
+  const long bh = static_cast<long>(b) * H + h;
+  const int32_t* sel_a = idx + (bh * nb + iA) * k;
+  const int32_t* sel_b = shared_kv ? sel_a : idx + (bh * nb + (iA + 1 < nb ? iA + 1 : iA)) * k;
+  const int T = shared_kv ? 2 * k : k;  // key tiles per stream
+  // loads per ring: one per (stream, tile) when key lists differ, one per tile when shared
+  const int nloads = shared_kv ? T : T * nstreams;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  // ---------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    mbar_init(&bar.q_full, 1);
+    // a K entry is released by the softmax warp group(s) that saw its S
+    // complete; a V entry by an MMA commit right after its last P.V product
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(&bar.k_full[s], 1);
+      mbar_init(&bar.k_empty[s], shared_kv ? 2 : 1);
+    }
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(&bar.v_full[s], 1);
+      mbar_init(&bar.v_empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bar.s_full[x], 1);
+      mbar_init(&bar.p_full[x], 4);
+      mbar_init(&bar.pv_last[x], 1);
+    }
+    mbar_init(&bar.mma_drained, 1);
+    bar.abort = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(&bar.tmem_base, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+  const uint32_t sbase = smem_u32(smem);
+
+  if (warp == 0 || warp == 2) {
+    // ============================================================ TMA producers
+    // warp 0: query tiles and the K ring; warp 2: the V ring. Separate warps,
+    // so that one producer suspended in a wait never holds up the other.
+    if (lane == 0) {
+      const bool is_k = warp == 0;
+      const int S = is_k ? KS : VS;
+      const uint64_t keep = policy_evict_last();  // gathered K/V: reused across query blocks
+      const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+      uint64_t* full = is_k ? bar.k_full : bar.v_full;
+      uint64_t* empty = is_k ? bar.k_empty : bar.v_empty;
+      const uint32_t ring = is_k ? L::kKOff : L::kVOff;
+      int issued[kTc2MaxStages];
+      for (int s = 0; s < S; ++s) issued[s] = 0;
+      bool ok = true;
+      if (is_k) {
+        const uint64_t stream = policy_evict_first();  // query tiles: read once
+        mbar_arrive_expect_tx(&bar.q_full, nstreams * L::kTileBytes);
+        for (int x = 0; x < nstreams; ++x)
+          for (int hh = 0; hh < 2; ++hh)
+            for (int c = 0; c < L::kChunks; ++c)
+              tma_load_4d(smem + L::kQOff + x * L::kTileBytes + c * (128 * 128) + hh * 64 * 128,
+                          &tm_q, &bar.q_full, c * 64, h, row0[x] + hh * 64, b, stream);
+      }
+      for (int n = 0; n < nloads && ok; ++n) {
+        const int s = n % S, use = n / S;
+        const int x = shared_kv ? 0 : n % nstreams;
+        const int t = shared_kv ? n : n / nstreams;
+        int r[2];
+        for (int hf = 0; hf < 2; ++hf) r[hf] = tc2_key_row(sel_a, sel_b, x, t, hf, bs, nb);
+        if (n >= S) ok = mbar_wait(&empty[s], (use - 1) & 1, abort_flag, is_k ? 111 : 112);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&full[s], L::kTileBytes);
+        for (int hf = 0; hf < 2; ++hf)
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_4d(smem + ring + s * L::kTileBytes + c * (128 * 128) + hf * 64 * 128, map,
+                        &full[s], c * 64, h, r[hf], b, keep);
+        issued[s] = use + 1;
+      }
+      if (is_k) mbar_wait_teardown(&bar.q_full, 0);
+      for (int s = 0; s < S; ++s)
+        if (issued[s]) mbar_wait_teardown(&full[s], (issued[s] - 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    // One thread feeds the tensor core, and a tcgen05.mma issue returns only
+    // when the previous instruction starts, so any work between instructions
+    // is idle tensor time: the loop body is straight-line, waits take a
+    // one-instruction fast path, descriptors move by plain adds, and the only
+    // commit per group is the one the softmax needs (ring entries are released
+    // by the softmax warps, which see each S complete).
+    if (lane == 0) {
+      constexpr uint32_t kSBO = 1024;  // 8 rows x 128 bytes
+      const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);  // P from TMEM, V MN-major
+      const uint64_t dq0 = smem_desc_sw128(sbase + L::kQOff, 16, kSBO);
+      const uint64_t dk0 = smem_desc_sw128(sbase + L::kKOff, 16, kSBO);
+      const uint64_t dv0 = smem_desc_sw128(sbase + L::kVOff, 128 * 128, kSBO);
+      constexpr uint64_t kTileStep = L::kTileBytes >> 4;
+      // ring index of stream x's tile t (K and V rings are filled in the same order)
+      auto load_index = [&](int x, int t) { return shared_kv ? t : t * nstreams + x; };
+      bool ok = mbar_wait(&bar.q_full, 0, abort_flag, 211);
+      // S_X(0)
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        if (!ok || x >= nstreams) break;
+        const int n = load_index(x, 0);
+        ok = mbar_wait_fast(&bar.k_full[n % KS], (n / KS) & 1, abort_flag, 212);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dq = dq0 + x * kTileStep, dk = dk0 + (n % KS) * kTileStep;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+          mma_bf16_ss(tmem + L::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bar.s_full[x]);
+      }
+      for (int j = 0; j < T && ok; ++j) {
+        const bool more = j + 1 < T;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (x >= nstreams) break;
+          // PV_X(j) needs P_X(j) and V(x, j); S_X(j+1) needs K(x, j+1)
+          const int nv = load_index(x, j), nk = load_index(x, j + 1);
+          ok = mbar_wait_fast(&bar.p_full[x], j & 1, abort_flag, 213) &&
+               mbar_wait_fast(&bar.v_full[nv % VS], (nv / VS) & 1, abort_flag, 214) &&
+               (!more || mbar_wait_fast(&bar.k_full[nk % KS], (nk / KS) & 1, abort_flag, 215));
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dv = dv0 + (nv % VS) * kTileStep;
+          const uint32_t a_tmem = tmem + L::col_s(x);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tmem + L::col_o(x), a_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          // the V ring is shallow, so its entry is freed as soon as the product is done
+          if (!shared_kv || x == 1) mma_commit(&bar.v_empty[nv % VS]);
+          if (more) {
+            const uint64_t dq = dq0 + x * kTileStep, dk = dk0 + (nk % KS) * kTileStep;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+              mma_bf16_ss(tmem + L::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&bar.s_full[x]);
+          } else {
+            mma_commit(&bar.pv_last[x]);
+          }
+        }
+      }
+      mma_commit(&bar.mma_drained);
+      mbar_wait_teardown(&bar.mma_drained, 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && (warp - 4) / 4 < nstreams) {
+    // ============================================================ softmax / epilogue
+    const int x = (warp - 4) / 4;
+    const int quad = warp % 4;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t scol = lane_base + L::col_s(x);
+    const uint32_t ocol = lane_base + L::col_o(x);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_full[x], j & 1, abort_flag, 311));
+      if (!ok) break;
+      tc_fence_after();
+      if (quad == 0 && lane == 0) {
+        // S_X(j) is complete: the K tile it read can be refilled
+        const int nk = shared_kv ? j : j * nstreams + x;
+        mbar_arrive(&bar.k_empty[nk % KS]);
+      }
+      // pass 1: row max
+      float mx;
+      {
+        uint32_t r0[32], r1[32];
+        float m8[8];
+        tmem_ld32(scol, r0);
+        tmem_ld32(scol + 32, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m8[e] = fmaxf(__uint_as_float(r0[e]), __uint_as_float(r1[e]));
+#pragma unroll
+        for (int e = 8; e < 32; ++e)
+          m8[e % 8] = fmaxf(m8[e % 8], fmaxf(__uint_as_float(r0[e]), __uint_as_float(r1[e])));
+        tmem_ld32(scol + 64, r0);
+        tmem_ld32(scol + 96, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          m8[e % 8] = fmaxf(m8[e % 8], fmaxf(__uint_as_float(r0[e]), __uint_as_float(r1[e])));
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      }
+      const float mt = mx * scale_log2;
+      const float m_new = (j == 0 || mt > m_run + 8.0f) ? mt : m_run;
+      const bool rescale = j > 0 && m_new != m_run;
+      if (__any_sync(0xffffffffu, rescale)) {
+        // S_X(j) is complete, so PV_X(j-1) has finished accumulating into O_X
+        const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
+        l_run *= alpha;
+        uint32_t r[16];
+#pragma unroll 1
+        for (int c = 0; c < D / 16; ++c) {
+          tmem_ld16(ocol + c * 16, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st16(ocol + c * 16, r);
+        }
+      }
+      m_run = m_new;
+      // pass 2: P = exp2(S * scale_log2 - m), stored as packed bf16 over S
+      // (chunk c of 32 keys -> columns 16c .. 16c+15, never ahead of the reads)
+      float ps[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ps[e] = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32], pk[16];
+        tmem_ld32(scol + c * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float x0 = fmaf(__uint_as_float(r[e]), scale_log2, -m_new);
+          const float x1 = fmaf(__uint_as_float(r[e + 1]), scale_log2, -m_new);
+          float p0, p1;
+          if ((e / 2) % 4 == 3) {  // one pair in four on the FMA pipe
+            p0 = exp2_poly(x0);
+            p1 = exp2_poly(x1);
+          } else {
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
+          }
+          ps[(e / 2) % 8] += p0 + p1;
+          pk[e / 2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(scol + c * 16, pk);
+      }
+      tmem_wait_st();
+      l_run += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.p_full[x]);
+    }
+    // ---- epilogue: O_X / l -> bf16 -> global
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.pv_last[x], 0, abort_flag, 314));
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.0f / l_run;
+      const long n = row0[x] + row;
+      __nv_bfloat16* orow = o + ((static_cast<long>(b) * N + n) * H + h) * D;
+      uint32_t r[32];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        tmem_ld32(ocol + c * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(r[e + 4]) * inv, __uint_as_float(r[e + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(r[e + 6]) * inv, __uint_as_float(r[e + 7]) * inv);
+          *reinterpret_cast<uint4*>(orow + c * 32 + e) = w;
+        }
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace bsa

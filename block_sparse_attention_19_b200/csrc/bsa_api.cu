@@ -15,6 +15,7 @@
 
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
+#include "attn_tc2.cuh"
 #include "bsa.h"
 #include "bsa_ptx.cuh"
 #include "pool.cuh"
@@ -205,7 +206,7 @@ bsa_status launch_attn_tc(const void* q, const void* k, const void* v, const int
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_tc_kernel<D, BM>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return cuda_fail(e, "tc smem attribute");
     attr_set[dev] = true;
   }
@@ -213,10 +214,38 @@ bsa_status launch_attn_tc(const void* q, const void* k, const void* v, const int
   const long grid = static_cast<long>(B) * H * (N / bs) * parts;
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   const float scale_log2 = scale * 1.4426950408889634f;
-  bsa::sparse_attn_tc_kernel<D, BM><<<static_cast<unsigned>(grid), bsa::kTcThreads, L::kSmemAlloc, st>>>(
+  bsa::sparse_attn_tc_kernel<D, BM><<<static_cast<unsigned>(grid), bsa::kTcThreads, L::kBytes, st>>>(
       mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, bs, kk, scale_log2);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc_kernel launch");
+}
+
+template <int D>
+bsa_status launch_attn_tc2(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
+                           int B, int N, int H, int bs, int kk, float scale, cudaStream_t st) {
+  using L = bsa::Tc2Layout<D>;
+  CUtensorMap mq, mk, mv;
+  bsa_status s;
+  if ((s = make_bnhd_map(&mq, q, B, N, H, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mk, k, B, N, H, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mv, v, B, N, H, D)) != BSA_OK) return s;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_tc2_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "tc2 smem attribute");
+    attr_set[dev] = true;
+  }
+  const int nb = N / bs;
+  const long grid = static_cast<long>(B) * H * (bs == 256 ? nb : (nb + 1) / 2);
+  if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
+  const float scale_log2 = scale * 1.4426950408889634f;
+  bsa::sparse_attn_tc2_kernel<D><<<static_cast<unsigned>(grid), bsa::kTc2Threads, L::kBytes, st>>>(
+      mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, bs, kk, scale_log2);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc2_kernel launch");
 }
 
 bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
@@ -232,8 +261,8 @@ bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_
   if (bs == 64)
     return D == 64 ? launch_attn_tc<64, 64>(q, k, v, idx, o, B, N, H, bs, kk, scale, st)
                    : launch_attn_tc<128, 64>(q, k, v, idx, o, B, N, H, bs, kk, scale, st);
-  return D == 64 ? launch_attn_tc<64, 128>(q, k, v, idx, o, B, N, H, bs, kk, scale, st)
-                 : launch_attn_tc<128, 128>(q, k, v, idx, o, B, N, H, bs, kk, scale, st);
+  return D == 64 ? launch_attn_tc2<64>(q, k, v, idx, o, B, N, H, bs, kk, scale, st)
+                 : launch_attn_tc2<128>(q, k, v, idx, o, B, N, H, bs, kk, scale, st);
 }
 
 struct Workspace {
