@@ -28,11 +28,13 @@
 //     overwrite P_X(j) before PV_X(j) has read it, and the completion of
 //     S_X(j+1) implies that PV_X(j) is done (so O_X is stable).
 //   * warps 4-7 (stream A) and 8-11 (stream B): one query row per thread.
-//     Per tile: pass 1 reads the row of S from TMEM for its max; the running
-//     max (log2 domain) moves only when the tile max exceeds it by more than
-//     8, in which case O_X is rescaled in TMEM; pass 2 re-reads S, computes
-//     P = exp2(S * scale * log2 e - m) (one pair in four on the FMA pipe) and
-//     stores it as packed bf16 over S, chunk by chunk behind the reads.
+//     Per tile a thread loads its whole S row from TMEM into registers (the
+//     softmax warp groups take registers from warp group 0 with setmaxnreg),
+//     takes the row max; the running max (log2 domain) moves only when the
+//     tile max exceeds it by more than 8, in which case O_X is rescaled in
+//     TMEM; then P = exp2(S * scale * log2 e - m) with two-wide float32
+//     instructions (three key pairs in eight via a polynomial on the FMA
+//     pipe), stored as packed bf16 over the first 64 columns of S.
 //   * warp 3 idle.
 // Every wait is bounded; on a timeout the device error word and an abort flag
 // are set, roles leave their loops, copies and MMAs are drained, TMEM is freed.
@@ -47,6 +49,12 @@ namespace bsa {
 
 constexpr int kTc2Threads = 384;  // 12 warps
 constexpr int kTc2MaxStages = 12;
+// Register split: warp group 0 (producers, MMA issuer) gives registers to
+// the two softmax warp groups, which hold a whole 128-column S row. The sum
+// must fit in the launch allocation (kTc2Threads x the kernel's register
+// count), which the host verifies: kTc2LaunchRegs is what the split needs.
+constexpr uint32_t kTc2RegsLow = 80, kTc2RegsHigh = 208;
+constexpr uint32_t kTc2LaunchRegs = (128 * kTc2RegsLow + 256 * kTc2RegsHigh + kTc2Threads - 1) / kTc2Threads;
 
 template <int D>
 struct Tc2Layout {
@@ -164,8 +172,10 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
   const uint32_t sbase = smem_u32(smem);
-
+  // register split: each role adjusts its own allowance on entry (warp
+  // group 0: producers, MMA issuer and the idle warp 3 give registers away)
   if (warp == 0 || warp == 2) {
+    regs_decrease<kTc2RegsLow>();
     // ============================================================ TMA producers
     // warp 0: query tiles and the K ring; warp 2: the V ring. Separate warps,
     // so that one producer suspended in a wait never holds up the other.
@@ -210,6 +220,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
+    regs_decrease<kTc2RegsLow>();
     // ============================================================ MMA issuer
     // One thread feeds the tensor core, and a tcgen05.mma issue returns only
     // when the previous instruction starts, so any work between instructions
@@ -281,7 +292,10 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
       mbar_wait_teardown(&bar.mma_drained, 0);
     }
     __syncwarp();
-  } else if (warp >= 4 && (warp - 4) / 4 < nstreams) {
+  } else if (warp == 3) {
+    regs_decrease<kTc2RegsLow>();
+  } else if ((warp - 4) / 4 < nstreams) {
+    regs_increase<kTc2RegsHigh>();
     // ============================================================ softmax / epilogue
     const int x = (warp - 4) / 4;
     const int quad = warp % 4;
@@ -300,29 +314,21 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         const int nk = shared_kv ? j : j * nstreams + x;
         mbar_arrive(&bar.k_empty[nk % KS]);
       }
-      // pass 1: row max
-      float mx;
-      {
-        uint32_t r0[32], r1[32];
-        float m8[8];
-        tmem_ld32(scol, r0);
-        tmem_ld32(scol + 32, r1);
-        tmem_wait_ld();
+      // The whole S row in registers: four TMEM loads, one wait.
+      uint32_t sa[32], sb[32], sc[32], sd[32];
+      tmem_ld32(scol, sa);
+      tmem_ld32(scol + 32, sb);
+      tmem_ld32(scol + 64, sc);
+      tmem_ld32(scol + 96, sd);
+      tmem_wait_ld();
+#define BSA_S(i) __uint_as_float((i) < 32 ? sa[(i) & 31] : (i) < 64 ? sb[(i) & 31] : (i) < 96 ? sc[(i) & 31] : sd[(i) & 31])
+      float m4[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m8[e] = fmaxf(__uint_as_float(r0[e]), __uint_as_float(r1[e]));
+      for (int e = 0; e < 4; ++e) m4[e] = fmaxf(BSA_S(2 * e), BSA_S(2 * e + 1));
 #pragma unroll
-        for (int e = 8; e < 32; ++e)
-          m8[e % 8] = fmaxf(m8[e % 8], fmaxf(__uint_as_float(r0[e]), __uint_as_float(r1[e])));
-        tmem_ld32(scol + 64, r0);
-        tmem_ld32(scol + 96, r1);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          m8[e % 8] = fmaxf(m8[e % 8], fmaxf(__uint_as_float(r0[e]), __uint_as_float(r1[e])));
-        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      }
-      const float mt = mx * scale_log2;
+      for (int pr = 4; pr < 64; ++pr) m4[pr % 4] = fmax3(m4[pr % 4], BSA_S(2 * pr), BSA_S(2 * pr + 1));
+      const float mt = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]) * scale_log2;
+      // the running max moves only when the tile max exceeds it by more than 8
       const float m_new = (j == 0 || mt > m_run + 8.0f) ? mt : m_run;
       const bool rescale = j > 0 && m_new != m_run;
       if (__any_sync(0xffffffffu, rescale)) {
@@ -340,35 +346,42 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         }
       }
       m_run = m_new;
-      // pass 2: P = exp2(S * scale_log2 - m), stored as packed bf16 over S
-      // (chunk c of 32 keys -> columns 16c .. 16c+15, never ahead of the reads)
-      float ps[8];
+      // P = exp2(S * scale_log2 - m) for key pairs with two-wide float32
+      // instructions; three pairs in eight take the polynomial exp2 on the FMA
+      // pipe. P is stored as packed bf16 over the first 64 columns of S.
+      uint32_t pa[32], pb[32];
+      uint64_t ps[4] = {0, 0, 0, 0};
+      {
+        const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m_new, -m_new);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ps[e] = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32], pk[16];
-        tmem_ld32(scol + c * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float x0 = fmaf(__uint_as_float(r[e]), scale_log2, -m_new);
-          const float x1 = fmaf(__uint_as_float(r[e + 1]), scale_log2, -m_new);
-          float p0, p1;
-          if ((e / 2) % 4 == 3) {  // one pair in four on the FMA pipe
-            p0 = exp2_poly(x0);
-            p1 = exp2_poly(x1);
+        for (int pr = 0; pr < 64; ++pr) {
+          const uint64_t x2 = f2_fma(f2(BSA_S(2 * pr), BSA_S(2 * pr + 1)), sc2, nm2);
+          uint64_t p2;
+          if (pr % 8 == 1 || pr % 8 == 4 || pr % 8 == 6) {
+            p2 = exp2_poly2(x2);
           } else {
-            p0 = fast_exp2(x0);
-            p1 = fast_exp2(x1);
+            float x0, x1;
+            f2_split(x2, x0, x1);
+            p2 = f2(fast_exp2(x0), fast_exp2(x1));
           }
-          ps[(e / 2) % 8] += p0 + p1;
-          pk[e / 2] = pack_bf16x2(p0, p1);
+          ps[pr % 4] = f2_add(ps[pr % 4], p2);
+          float p0, p1;
+          f2_split(p2, p0, p1);
+          if (pr < 32)
+            pa[pr] = pack_bf16x2(p0, p1);
+          else
+            pb[pr - 32] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(scol + c * 16, pk);
       }
+#undef BSA_S
+      tmem_st32(scol, pa);
+      tmem_st32(scol + 32, pb);
       tmem_wait_st();
-      l_run += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      {
+        float a0, a1;
+        f2_split(f2_add(f2_add(ps[0], ps[1]), f2_add(ps[2], ps[3])), a0, a1);
+        l_run += a0 + a1;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.p_full[x]);

@@ -236,6 +236,15 @@ bsa_status launch_attn_tc2(const void* q, const void* k, const void* v, const in
     cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_tc2_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return cuda_fail(e, "tc2 smem attribute");
+    // The kernel moves registers between warp groups (setmaxnreg); an increase
+    // that the launch allocation cannot cover would wait forever, so refuse
+    // to launch unless the compiled register count covers the split.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, bsa::sparse_attn_tc2_kernel<D>);
+    if (e != cudaSuccess) return cuda_fail(e, "tc2 attributes");
+    if (fa.numRegs < static_cast<int>(bsa::kTc2LaunchRegs))
+      return fail(BSA_ERR_UNSUPPORTED, "attention kernel built with %d registers/thread, its register split needs %u",
+                  fa.numRegs, bsa::kTc2LaunchRegs);
     attr_set[dev] = true;
   }
   const int nb = N / bs;

@@ -296,6 +296,19 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
          | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Warp-group register reallocation (all warps of a warp group execute the
+// same one). An increase waits until the registers are available in the
+// CTA's pool, so the split must fit in the launch allocation; the host checks
+// that before launching.
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -320,6 +333,59 @@ __device__ __forceinline__ float exp2_poly(float x) {
   p = fmaf(p, f, 0.6931217908859253f);
   p = fmaf(p, f, 0.9999992847442627f);
   return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
+// ---- packed two-wide float32 arithmetic (sm_100): one instruction per pair
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// exp2_poly on a pair: the same range split and polynomial, two lanes per
+// instruction where the operation allows it.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  f2_split(x2, x0, x1);
+  x2 = f2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const float kRound = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t r2 = f2(kRound, kRound);
+  const uint64_t t2 = f2_add(x2, r2);
+  const uint64_t f = f2_sub(x2, f2_sub(t2, r2));
+  uint64_t p = f2(0.009570102207362652f, 0.009570102207362652f);
+  p = f2_fma(p, f, f2(0.05591785907745361f, 0.05591785907745361f));
+  p = f2_fma(p, f, f2(0.240247443318367f, 0.240247443318367f));
+  p = f2_fma(p, f, f2(0.6931217908859253f, 0.6931217908859253f));
+  p = f2_fma(p, f, f2(0.9999992847442627f, 0.9999992847442627f));
+  float t0, t1, p0, p1;
+  f2_split(t2, t0, t1);
+  f2_split(p, p0, p1);
+  const int n0 = __float_as_int(t0) - __float_as_int(kRound);
+  const int n1 = __float_as_int(t1) - __float_as_int(kRound);
+  return f2(__int_as_float(__float_as_int(p0) + (n0 << 23)), __int_as_float(__float_as_int(p1) + (n1 << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
