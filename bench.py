@@ -5,7 +5,7 @@
 
 One step = one pass of the whole hot path over one batch of synthetic inputs
 already resident in HBM: block pooling of q and k, block scores + top-k
-selection, and sparse attention, each through its C-ABI entry point (4 kernel
+selection, and sparse attention, each through its C-ABI entry point (5 kernel
 launches), with CUDA events between the stages on the launching stream.
 value = query tokens processed by all ranks / (max over ranks of the device
 time of the K timed steps). With --gpus N > 1 (under torchrun) every rank runs
@@ -197,7 +197,7 @@ def main():
     kk = bsa.bsa_topk_count(N // bs, ratio)
     q, k, v = W.make_inputs(cfg, device=dev)
     ws = torch.empty(bsa.bsa_forward_workspace_bytes(B, N, H, D, bs, ratio), device=dev, dtype=torch.uint8)
-    qp, kp, idx = bsa.workspace_views(ws, B, N, H, D, bs, ratio)
+    qp, kp, idx, S = bsa.workspace_views(ws, B, N, H, D, bs, ratio, with_scores=True)
     o = torch.empty_like(q)
 
     def step(ev=None):
@@ -207,7 +207,7 @@ def main():
         bsa.bsa_block_pool(k, bs, out=kp)
         if ev is not None:
             ev[1].record()
-        bsa.bsa_block_scores_topk(qp, kp, kk, idx_out=idx)
+        bsa.bsa_block_scores_topk(qp, kp, kk, idx_out=idx, scores_out=S)
         if ev is not None:
             ev[2].record()
         bsa.bsa_sparse_attn_fwd(q, k, v, idx, bs, out=o)
@@ -317,7 +317,7 @@ def main():
                    "l2": f"inputs larger than L2 (q, k, v {tensor_bytes / 1e6:.0f} MB each)",
                    "parallelism": f"replica per GPU x{world}"},
         "tflops_effective": flops / (step_ms / 1e3) / 1e12,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 5 * args.steps,
         "stages_ms": {"pool_qk": pool_ms, "scores_topk": sel_ms, "sparse_attn": attn_ms,
                       "fused_bsa_forward": fused_ms},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

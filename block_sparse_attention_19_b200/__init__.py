@@ -9,7 +9,7 @@ raises.
 Functions carry the C names:
 
 * ``bsa_block_pool(x, block_size)``                -> pooled [B, H, nb, D] float32
-* ``bsa_block_scores_topk(q_pooled, k_pooled, topk, scores=False)`` -> idx (, scores)
+* ``bsa_block_scores_topk(q_pooled, k_pooled, topk, scores=False)`` -> idx (, S)
 * ``bsa_sparse_attn_fwd(q, k, v, idx, block_size, scale=None)`` -> o
 * ``bsa_forward(q, k, v, block_size, topk_ratio, workspace=None)`` -> o
 * ``bsa_topk_count``, ``bsa_forward_workspace_bytes``, ``bsa_device_error``
@@ -120,14 +120,18 @@ def bsa_block_pool(x: torch.Tensor, block_size: int, out: torch.Tensor | None = 
 
 
 def bsa_block_scores_topk(q_pooled: torch.Tensor, k_pooled: torch.Tensor, topk: int,
-                          scores: bool = False, idx_out: torch.Tensor | None = None):
+                          scores: bool = False, idx_out: torch.Tensor | None = None,
+                          scores_out: torch.Tensor | None = None):
+    """Block scores S (written to ``scores_out``, allocated if absent) and the
+    top-k index list. Returns idx, or (idx, S) when ``scores`` is true."""
     _dev(q_pooled, "q_pooled")
     _dev(k_pooled, "k_pooled")
     if q_pooled.dtype != torch.float32 or k_pooled.dtype != torch.float32:
         raise TypeError("pooled tensors must be float32")
     B, H, nb, D = q_pooled.shape
     idx = idx_out if idx_out is not None else torch.empty((B, H, nb, topk), device=q_pooled.device, dtype=torch.int32)
-    S = torch.empty((B, H, nb, nb), device=q_pooled.device, dtype=torch.float32) if scores else None
+    S = scores_out if scores_out is not None else torch.empty((B, H, nb, nb), device=q_pooled.device,
+                                                              dtype=torch.float32)
     _check(lib.bsa_block_scores_topk(_p(q_pooled), _p(k_pooled), _p(S), _p(idx), B, H, nb, D, topk,
                                      _stream(q_pooled)))
     return (idx, S) if scores else idx
@@ -191,14 +195,22 @@ def bsa_device_error(device=None) -> int:
     return code.value
 
 
-def workspace_views(ws: torch.Tensor, B: int, N: int, H: int, D: int, block_size: int, topk_ratio: float):
-    """The pooled q, pooled k and index-list sections of a bsa_forward workspace
-    (the layout of include/bsa.h: three 256-byte aligned sections)."""
+def workspace_views(ws: torch.Tensor, B: int, N: int, H: int, D: int, block_size: int, topk_ratio: float,
+                    with_scores: bool = False):
+    """The pooled q, pooled k, index-list (and block-score) sections of a
+    bsa_forward workspace (the layout of include/bsa.h: 256-byte aligned
+    sections in that order)."""
     nb = N // block_size
     kk = bsa_topk_count(nb, topk_ratio)
-    pooled = ((B * H * nb * D * 4) + 255) // 256 * 256
+    a256 = lambda x: (x + 255) // 256 * 256
+    pooled = a256(B * H * nb * D * 4)
+    idxb = a256(B * H * nb * kk * 4)
     base = ws.view(torch.uint8)
     qp = base[:B * H * nb * D * 4].view(torch.float32).view(B, H, nb, D)
     kp = base[pooled:pooled + B * H * nb * D * 4].view(torch.float32).view(B, H, nb, D)
     idx = base[2 * pooled:2 * pooled + B * H * nb * kk * 4].view(torch.int32).view(B, H, nb, kk)
-    return qp, kp, idx
+    if not with_scores:
+        return qp, kp, idx
+    off = 2 * pooled + idxb
+    S = base[off:off + B * H * nb * nb * 4].view(torch.float32).view(B, H, nb, nb)
+    return qp, kp, idx, S

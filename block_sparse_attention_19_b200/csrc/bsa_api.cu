@@ -19,6 +19,7 @@
 #include "bsa.h"
 #include "bsa_ptx.cuh"
 #include "pool.cuh"
+#include "scores_tc.cuh"
 #include "select.cuh"
 
 namespace {
@@ -136,37 +137,54 @@ bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_pool_kernel launch");
 }
 
-template <int R>
-bsa_status launch_select_r(const float* qp, const float* kp, float* scores, int32_t* idx, int B,
-                           int H, int nb, int D, int k, cudaStream_t st) {
-  const size_t smem = (static_cast<size_t>(R) * D + static_cast<size_t>(R) * nb) * sizeof(float);
+// Block scores S = qbar kbar^T per (b, h) on the tensor cores (split TF32),
+// written to S [B, H, nb, nb]; then the top-k selection reads S back.
+bsa_status launch_scores(const float* qp, const float* kp, float* S, int B, int H, int nb, int D,
+                         cudaStream_t st) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(bsa::block_scores_topk_kernel<R>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (R * 128 + bsa::kSelSmemScoreBytes / 4) * 4);
-    if (e != cudaSuccess) return cuda_fail(e, "select smem attribute");
+    cudaError_t e = cudaFuncSetAttribute(bsa::block_scores_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bsa::kScSmem);
+    if (e != cudaSuccess) return cuda_fail(e, "scores smem attribute");
     attr_set[dev] = true;
   }
-  const long grid = static_cast<long>(B) * H * ((nb + R - 1) / R);
-  bsa::block_scores_topk_kernel<R><<<static_cast<unsigned>(grid), bsa::kSelThreads, smem, st>>>(
-      qp, kp, scores, idx, H, nb, D, k);
+  const long tiles = static_cast<long>(B) * H * ((nb + bsa::kScM - 1) / bsa::kScM) *
+                     ((nb + bsa::kScN - 1) / bsa::kScN);
+  if (tiles > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "score grid too large");
+  bsa::block_scores_tc_kernel<<<static_cast<unsigned>(tiles), bsa::kScThreads, bsa::kScSmem, st>>>(
+      qp, kp, S, nb, D);
   cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_scores_topk_kernel launch");
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_scores_tc_kernel launch");
 }
 
-bsa_status launch_select(const float* qp, const float* kp, float* scores, int32_t* idx, int B,
-                         int H, int nb, int D, int k, cudaStream_t st) {
-  switch (bsa::select_rows_per_cta(nb)) {
-    case 32: return launch_select_r<32>(qp, kp, scores, idx, B, H, nb, D, k, st);
-    case 16: return launch_select_r<16>(qp, kp, scores, idx, B, H, nb, D, k, st);
-    case 8: return launch_select_r<8>(qp, kp, scores, idx, B, H, nb, D, k, st);
-    case 4: return launch_select_r<4>(qp, kp, scores, idx, B, H, nb, D, k, st);
-    case 2: return launch_select_r<2>(qp, kp, scores, idx, B, H, nb, D, k, st);
-    default: return launch_select_r<1>(qp, kp, scores, idx, B, H, nb, D, k, st);
+bsa_status launch_topk(const float* S, int32_t* idx, int B, int H, int nb, int k, cudaStream_t st) {
+  const long rows = static_cast<long>(B) * H * nb;
+  const size_t stage_bytes = static_cast<size_t>(bsa::kSelWarps) * nb * sizeof(float);
+  const bool stage = nb > 1024 && stage_bytes <= 200 * 1024;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(bsa::block_topk_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e != cudaSuccess) return cuda_fail(e, "topk smem attribute");
+    attr_set[dev] = true;
   }
+  const long grid = (rows + bsa::kSelWarps - 1) / bsa::kSelWarps;
+  if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "top-k grid too large");
+  bsa::block_topk_kernel<<<static_cast<unsigned>(grid), bsa::kSelThreads, stage ? stage_bytes : 0, st>>>(
+      S, idx, rows, nb, k, stage ? 1 : 0);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_topk_kernel launch");
+}
+
+bsa_status launch_select(const float* qp, const float* kp, float* S, int32_t* idx, int B, int H,
+                         int nb, int D, int k, cudaStream_t st) {
+  bsa_status s;
+  if ((s = launch_scores(qp, kp, S, B, H, nb, D, st)) != BSA_OK) return s;
+  return launch_topk(S, idx, B, H, nb, k, st);
 }
 
 template <int D>
@@ -278,19 +296,23 @@ struct Workspace {
   float* qp;
   float* kp;
   int32_t* idx;
+  float* scores;
   size_t bytes;
 };
 
+// q_pooled | k_pooled | idx | scores, each section 256-byte aligned
 Workspace workspace_layout(void* base, int B, int N, int H, int D, int bs, int k) {
   const size_t nb = static_cast<size_t>(N / bs);
   const size_t pooled = align256(static_cast<size_t>(B) * H * nb * D * sizeof(float));
   const size_t idxb = align256(static_cast<size_t>(B) * H * nb * k * sizeof(int32_t));
+  const size_t scb = align256(static_cast<size_t>(B) * H * nb * nb * sizeof(float));
   unsigned char* p = static_cast<unsigned char*>(base);
   Workspace w;
   w.qp = reinterpret_cast<float*>(p);
   w.kp = reinterpret_cast<float*>(p + pooled);
   w.idx = reinterpret_cast<int32_t*>(p + 2 * pooled);
-  w.bytes = 2 * pooled + idxb;
+  w.scores = reinterpret_cast<float*>(p + 2 * pooled + idxb);
+  w.bytes = 2 * pooled + idxb + scb;
   return w;
 }
 
@@ -350,8 +372,8 @@ bsa_status bsa_block_scores_topk(const float* q_pooled, const float* k_pooled, f
   if (D != 64 && D != 128) return fail(BSA_ERR_UNSUPPORTED, "D=%d (supported: 64, 128)", D);
   if (nb > 32768) return fail(BSA_ERR_UNSUPPORTED, "nb=%d > 32768", nb);
   if (k < 1 || k > nb) return fail(BSA_ERR_INVALID_ARG, "k=%d outside [1, nb=%d]", k, nb);
-  if (!q_pooled || !k_pooled || !idx) return fail(BSA_ERR_INVALID_ARG, "null pointer");
-  if (!aligned16(q_pooled) || !aligned16(k_pooled) || !aligned16(idx) || (scores && !aligned16(scores)))
+  if (!q_pooled || !k_pooled || !idx || !scores) return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q_pooled) || !aligned16(k_pooled) || !aligned16(idx) || !aligned16(scores))
     return fail(BSA_ERR_MISALIGNED, "q_pooled, k_pooled, idx or scores");
   if ((s = check_device()) != BSA_OK) return s;
   if ((s = launch_select(q_pooled, k_pooled, scores, idx, B, H, nb, D, k,
@@ -405,7 +427,7 @@ bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   if ((s = launch_pool(q, w.qp, k, w.kp, 2, B, N, H, D, block_size, dt, st)) != BSA_OK) return s;
-  if ((s = launch_select(w.qp, w.kp, nullptr, w.idx, B, H, nb, D, kk, st)) != BSA_OK) return s;
+  if ((s = launch_select(w.qp, w.kp, w.scores, w.idx, B, H, nb, D, kk, st)) != BSA_OK) return s;
   if ((s = launch_attn(q, k, v, w.idx, o, B, N, H, D, block_size, kk, scale, dt, st)) != BSA_OK) return s;
   return ok();
 }

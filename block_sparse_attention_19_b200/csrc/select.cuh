@@ -1,19 +1,18 @@
-// select.cuh -- steps 1b + 2: block scores and top-k block selection.
+// select.cuh -- step 2: top-k block selection from the block scores.
 //
 // Page "2026 新一代卷积与 Transformer 网络架构" (qqiyuan.cn), section
-// "SparseFormer 注意力实现": block_scores = einsum of the pooled q and k per
-// (b, h) (an nb x nb matrix), then torch.topk(block_scores, k) over the key
-// blocks. Readings fixed here: float32 dot products with no 1/sqrt(D) factor;
-// ties go to the lower key-block index; each output row lists its k blocks in
-// ascending order (a canonical order, so results are exactly comparable).
+// "SparseFormer 注意力实现", step 2: torch.topk(block_scores, k) over the key
+// blocks. Readings fixed here: ties go to the lower key-block index; each
+// output row lists its k blocks in ascending order (a canonical order, so
+// results compare exactly).
 //
-// One CTA owns R consecutive query blocks of one (b, h). Phase A computes the
-// R score rows S[r, 0..nb) in float32 FFMA (each thread owns two key-block
-// columns at a time; pooled q rows are broadcast from shared memory, pooled k
-// rows stream from L2) and keeps them in shared memory. Phase B selects per
-// row with one warp: the k-th largest score is found exactly by a bitwise
-// binary search over order-preserving 32-bit keys, then one ordered pass
-// emits every key above it plus the lowest-index keys equal to it.
+// One warp per score row, scores as order-preserving 32-bit keys. For
+// nb <= 1024 the keys sit in registers and the k-th largest key is
+// bracketed by bisection (on the score value, then on the key) until at most
+// 64 keys remain in the bracket, which are sorted exactly (about 8 counting
+// passes on typical rows instead of 32); longer rows use a bitwise binary search over the keys
+// staged in shared memory. One ordered ballot pass then emits every key above
+// the k-th largest plus the lowest-index keys equal to it.
 #pragma once
 
 #include <stdint.h>
@@ -22,19 +21,11 @@ namespace bsa {
 
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kSelSmemScoreBytes = 128 * 1024;  // R * nb * 4 bytes at most
 
 // Order-preserving map float -> uint32 (larger float <=> larger key).
 __device__ __forceinline__ uint32_t float_key(float f) {
   uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Rows per CTA for a given nb (power of two, R * nb * 4 <= kSelSmemScoreBytes).
-inline int select_rows_per_cta(int nb) {
-  int r = 32;
-  while (r > 1 && static_cast<long>(r) * nb * 4 > kSelSmemScoreBytes) r >>= 1;
-  return r;
 }
 
 // Per-lane key capacity of the register path of phase B (nb <= 32 * KPL).
@@ -67,6 +58,143 @@ __device__ __forceinline__ void select_row_regs(const float* srow, int nb, int k
   const int need_eq = k - gt;  // >= 1 by the choice of T
 
   // ordered emission: ascending j, lanes cover 32 consecutive j per step
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int written = 0, eq_seen = 0;
+#pragma unroll
+  for (int t = 0; t < KPL; ++t) {
+    const int j = t * 32 + lane;
+    const bool eq = (j < nb) && key[t] == T;
+    const uint32_t eq_ballot = __ballot_sync(0xffffffffu, eq);
+    const int eq_rank = eq_seen + __popc(eq_ballot & lt_mask);
+    const bool sel = (j < nb) && (key[t] > T || (eq && eq_rank < need_eq));
+    const uint32_t sel_ballot = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[written + __popc(sel_ballot & lt_mask)] = j;
+    written += __popc(sel_ballot);
+    eq_seen += __popc(eq_ballot);
+  }
+}
+
+__device__ __forceinline__ float key_float(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
+}
+
+template <int KPL>
+__device__ __forceinline__ int warp_count_ge(const uint32_t (&key)[KPL], uint32_t t) {
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) c += key[i] >= t;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  return c;
+}
+
+// Bitonic sort of 64 keys held two per lane (element i = lane in a, lane + 32
+// in b) into descending order across the warp.
+__device__ __forceinline__ void warp_sort64_desc(uint32_t& a, uint32_t& b, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 64; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride == 32) {
+        // partners i and i + 32 sit in the same lane; size is 64: one descending block
+        const uint32_t hi = max(a, b), lo = min(a, b);
+        a = hi;
+        b = lo;
+      } else {
+#pragma unroll
+        for (int slot = 0; slot < 2; ++slot) {
+          uint32_t& x = slot == 0 ? a : b;
+          const int i = lane + 32 * slot;
+          const uint32_t y = __shfl_xor_sync(0xffffffffu, x, stride);
+          const bool lower = (i & stride) == 0;
+          const bool desc = (i & size) == 0;
+          x = (lower == desc) ? max(x, y) : min(x, y);
+        }
+      }
+    }
+  }
+}
+
+// Same result as select_row_regs with far fewer passes on typical rows: the
+// k-th largest key is bracketed by bisection (up to 12 steps on the score
+// value, then on the key, which needs at most 32 steps) until the bracket
+// [lo, hi) holds at most 64 keys, which are then sorted exactly; a
+// bracket that cannot be split holds equal keys only. `cand` is 64 words of
+// shared memory private to the warp.
+template <int KPL>
+__device__ __forceinline__ void select_row_bracket(const float* srow, int nb, int k, int32_t* out,
+                                                   int lane, uint32_t* cand) {
+  uint32_t key[KPL];
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+  for (int t = 0; t < KPL; ++t) {
+    const int j = t * 32 + lane;
+    key[t] = j < nb ? float_key(srow[j]) : 0u;  // padding 0 never reaches a bracket above 0
+    if (j < nb) {
+      kmin = min(kmin, key[t]);
+      kmax = max(kmax, key[t]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  // invariant: count(key >= lo) = clo >= k > chi = count(key >= hi); hi may be 2^32
+  uint32_t lo = kmin;
+  uint64_t hi = static_cast<uint64_t>(kmax) + 1;
+  int clo = nb, chi = 0;
+  if (kmin == 0u) clo = warp_count_ge(key, 0u) - (KPL * 32 - nb);  // real keys of value 0
+#pragma unroll 1
+  for (int it = 0; it < 64 && clo - chi > 64 && hi - lo > 1; ++it) {
+    const float flo = key_float(lo), fhi = key_float(static_cast<uint32_t>(hi - 1));
+    const float fm = 0.5f * flo + 0.5f * fhi;
+    uint32_t p = float_key(fm);
+    // value steps first (fast on smooth score distributions), then key
+    // midpoints, which end in at most 32 steps whatever the distribution
+    if (it >= 12 || !(isfinite(fm) && p > lo && static_cast<uint64_t>(p) < hi))
+      p = lo + static_cast<uint32_t>((hi - lo) >> 1);
+    const int c = warp_count_ge(key, p);
+    if (c >= k) {
+      lo = p;
+      clo = c;
+    } else {
+      hi = p;
+      chi = c;
+    }
+  }
+  uint32_t T;
+  if (hi - lo == 1) {
+    T = lo;  // the bracket holds copies of one key
+  } else if (clo - chi <= 64) {
+    // gather the bracket's keys and take the (k - chi)-th largest exactly
+    int base = 0;
+    const uint32_t lt_mask0 = (1u << lane) - 1u;
+#pragma unroll
+    for (int t = 0; t < KPL; ++t) {
+      const bool in = key[t] >= lo && static_cast<uint64_t>(key[t]) < hi && t * 32 + lane < nb;
+      const uint32_t bal = __ballot_sync(0xffffffffu, in);
+      if (in) cand[base + __popc(bal & lt_mask0)] = key[t];
+      base += __popc(bal);
+    }
+    __syncwarp();
+    uint32_t a = lane < base ? cand[lane] : 0u, b = lane + 32 < base ? cand[lane + 32] : 0u;
+    __syncwarp();
+    warp_sort64_desc(a, b, lane);
+    const int r = k - chi - 1;
+    const uint32_t va = __shfl_sync(0xffffffffu, a, r & 31), vb = __shfl_sync(0xffffffffu, b, r & 31);
+    T = r < 32 ? va : vb;
+  } else {
+    // not narrowed in time (pathological rows): exact bitwise search
+    T = 0;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t c = T | (1u << bit);
+      if (warp_count_ge(key, c) >= k) T = c;
+    }
+  }
+  const int gt = T == 0xFFFFFFFFu ? 0 : warp_count_ge(key, T + 1);
+  const int need_eq = k - gt;
   const uint32_t lt_mask = (1u << lane) - 1u;
   int written = 0, eq_seen = 0;
 #pragma unroll
@@ -117,91 +245,43 @@ __device__ __forceinline__ void select_row_smem(const float* srow, int nb, int k
   }
 }
 
-// grid.x = B * H * ceil(nb / R). Dynamic shared memory: R * D floats (pooled q
-// rows) + R * nb floats (score rows).
-template <int R>
-__global__ void __launch_bounds__(kSelThreads, 1)
-    block_scores_topk_kernel(const float* __restrict__ qp, const float* __restrict__ kp,
-                             float* __restrict__ scores_out, int32_t* __restrict__ idx, int H,
-                             int nb, int D, int k) {
-  extern __shared__ __align__(16) float sel_smem[];
-  float* qs = sel_smem;         // [R][D]
-  float* ss = sel_smem + R * D;  // [R][nb]
-
-  const int tiles = (nb + R - 1) / R;
-  const int tile = blockIdx.x % tiles;
-  const long bh = blockIdx.x / tiles;
-  const int i0 = tile * R;
-  const int rows = min(R, nb - i0);
-  const float* qbase = qp + (bh * nb + i0) * D;
-  const float* kbase = kp + bh * nb * D;
-  const int tid = threadIdx.x;
-
-  for (int e = tid; e < R * D; e += kSelThreads) qs[e] = (e < rows * D) ? qbase[e] : 0.f;
-  __syncthreads();
-
-  // ---- phase A: S[r][j] = sum_d qs[r][d] * kp[j][d], two columns per thread
-  for (int j0 = 2 * tid; j0 < nb; j0 += 2 * kSelThreads) {
-    const bool two = j0 + 1 < nb;
-    const float4* k0 = reinterpret_cast<const float4*>(kbase + static_cast<long>(j0) * D);
-    const float4* k1 = reinterpret_cast<const float4*>(kbase + static_cast<long>(two ? j0 + 1 : j0) * D);
-    float a0[R], a1[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) a0[r] = a1[r] = 0.f;
-#pragma unroll 2
-    for (int d4 = 0; d4 < D / 4; ++d4) {
-      const float4 x = __ldg(k0 + d4);
-      const float4 y = __ldg(k1 + d4);
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const float4 q = reinterpret_cast<const float4*>(qs + r * D)[d4];
-        a0[r] = fmaf(q.x, x.x, a0[r]);
-        a0[r] = fmaf(q.y, x.y, a0[r]);
-        a0[r] = fmaf(q.z, x.z, a0[r]);
-        a0[r] = fmaf(q.w, x.w, a0[r]);
-        a1[r] = fmaf(q.x, y.x, a1[r]);
-        a1[r] = fmaf(q.y, y.y, a1[r]);
-        a1[r] = fmaf(q.z, y.z, a1[r]);
-        a1[r] = fmaf(q.w, y.w, a1[r]);
-      }
+// grid.x = ceil(rows / kSelWarps); one warp per row of S ([rows, nb]).
+// Dynamic shared memory: kSelWarps * nb floats when nb > 1024 and stage_rows, else none.
+__global__ void __launch_bounds__(kSelThreads)
+    block_topk_kernel(const float* __restrict__ S, int32_t* __restrict__ idx, long rows, int nb,
+                      int k, int stage_rows) {
+  extern __shared__ __align__(16) float sel_rows[];
+  __shared__ uint32_t cand[kSelWarps][64];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const long r = static_cast<long>(blockIdx.x) * kSelWarps + warp;
+  if (r >= rows) return;
+  const float* srow = S + r * nb;
+  int32_t* out = idx + r * static_cast<long>(k);
+  if (nb <= 32)
+    select_row_bracket<1>(srow, nb, k, out, lane, cand[warp]);
+  else if (nb <= 64)
+    select_row_bracket<2>(srow, nb, k, out, lane, cand[warp]);
+  else if (nb <= 128)
+    select_row_bracket<4>(srow, nb, k, out, lane, cand[warp]);
+  else if (nb <= 256)
+    select_row_bracket<8>(srow, nb, k, out, lane, cand[warp]);
+  else if (nb <= 512)
+    select_row_bracket<16>(srow, nb, k, out, lane, cand[warp]);
+  else if (nb <= 1024)
+    select_row_bracket<32>(srow, nb, k, out, lane, cand[warp]);
+  else if (stage_rows) {
+    // the row is re-read once per key bit: stage it in shared memory
+    float* row = sel_rows + static_cast<long>(warp) * nb;
+    if ((nb & 3) == 0) {
+      for (int j = lane * 4; j < nb; j += 128)
+        *reinterpret_cast<float4*>(row + j) = __ldg(reinterpret_cast<const float4*>(srow + j));
+    } else {
+      for (int j = lane; j < nb; j += 32) row[j] = __ldg(srow + j);
     }
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      ss[r * nb + j0] = a0[r];
-      if (two) ss[r * nb + j0 + 1] = a1[r];
-    }
-    if (scores_out != nullptr) {
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        if (r < rows) {
-          float* srow = scores_out + (bh * nb + i0 + r) * static_cast<long>(nb);
-          srow[j0] = a0[r];
-          if (two) srow[j0 + 1] = a1[r];
-        }
-      }
-    }
-  }
-  __syncthreads();
-
-  // ---- phase B: one warp per row
-  const int warp = tid / 32, lane = tid % 32;
-  for (int r = warp; r < rows; r += kSelWarps) {
-    const float* srow = ss + r * nb;
-    int32_t* out = idx + (bh * nb + i0 + r) * static_cast<long>(k);
-    if (nb <= 32)
-      select_row_regs<1>(srow, nb, k, out, lane);
-    else if (nb <= 64)
-      select_row_regs<2>(srow, nb, k, out, lane);
-    else if (nb <= 128)
-      select_row_regs<4>(srow, nb, k, out, lane);
-    else if (nb <= 256)
-      select_row_regs<8>(srow, nb, k, out, lane);
-    else if (nb <= 512)
-      select_row_regs<16>(srow, nb, k, out, lane);
-    else if (nb <= 1024)
-      select_row_regs<32>(srow, nb, k, out, lane);
-    else
-      select_row_smem(srow, nb, k, out, lane);
+    __syncwarp();
+    select_row_smem(row, nb, k, out, lane);
+  } else {
+    select_row_smem(srow, nb, k, out, lane);  // rows too long to stage: read them from L2
   }
 }
 

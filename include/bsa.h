@@ -64,9 +64,10 @@ typedef enum {
  * Pure host function. */
 int bsa_topk_count(int nb, double topk_ratio);
 
-/* Bytes of device workspace bsa_forward() needs for these sizes (pooled q and
- * k, and the index list, each section 256-byte aligned). Returns 0 when the
- * arguments are invalid. Pure host function. */
+/* Bytes of device workspace bsa_forward() needs for these sizes: pooled q,
+ * pooled k, the index list and the [B, H, nb, nb] float32 block-score matrix,
+ * in that order, each section 256-byte aligned. Returns 0 when the arguments
+ * are invalid. Pure host function. */
 size_t bsa_forward_workspace_bytes(int B, int N, int H, int D, int block_size, double topk_ratio);
 
 /* Step 1a (page listing, step 1: x.view(B, nb, bs, H, D).mean(2)):
@@ -81,10 +82,12 @@ bsa_status bsa_block_pool(const void* x, float* x_pooled, int B, int N, int H, i
  *   S[b, h, i, j] = sum_d q_pooled[b, h, i, d] * k_pooled[b, h, j, d]
  *   idx[b, h, i, :] = the topk key blocks j with the largest S[b, h, i, j],
  *                     ties to the lower j, written in ascending j.
- * q_pooled, k_pooled: [B, H, nb, D] float32 (read). idx: [B, H, nb, topk] int32
- * (written). scores: optional [B, H, nb, nb] float32 output of S (NULL = not
- * written). Scores are float32 dot products; no 1/sqrt(D) factor (it would not
- * change the ranking). */
+ * q_pooled, k_pooled: [B, H, nb, D] float32 (read). scores: [B, H, nb, nb]
+ * float32 (written with S; the selection then reads it back). idx:
+ * [B, H, nb, topk] int32 (written). S is computed on the tensor cores with
+ * float32 accuracy (each operand split into two TF32 parts, three products
+ * accumulated in float32); there is no 1/sqrt(D) factor (it would not change
+ * the ranking). Two kernel launches. */
 bsa_status bsa_block_scores_topk(const float* q_pooled, const float* k_pooled, float* scores,
                                  int32_t* idx, int B, int H, int nb, int D, int topk, void* stream);
 
@@ -100,9 +103,9 @@ bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const void* v, cons
                                void* o, int B, int N, int H, int D, int block_size, int topk,
                                float scale, bsa_dtype dt, void* stream);
 
-/* The whole path: bsa_block_pool on q and k, bsa_block_scores_topk (scores not
- * kept), bsa_sparse_attn_fwd with scale = 1/sqrt(D); three kernel launches on
- * `stream`, no host synchronisation. k = bsa_topk_count(N / block_size,
+/* The whole path: bsa_block_pool on q and k, bsa_block_scores_topk (scores in
+ * the workspace), bsa_sparse_attn_fwd with scale = 1/sqrt(D); four kernel
+ * launches on `stream`, no host synchronisation. k = bsa_topk_count(N / block_size,
  * topk_ratio) must be >= 1. workspace: device buffer of at least
  * bsa_forward_workspace_bytes(...) bytes, 256-byte aligned, owned by the caller
  * and not used concurrently by another call. */

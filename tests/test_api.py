@@ -49,10 +49,11 @@ def test_topk_count_rejects_bad_input(bsa):
 
 
 def test_workspace_bytes(bsa):
-    # c4: pooled q and k [1,16,1024,128] f32 = 8 MiB each, idx [1,16,1024,153] i32
+    # c4: pooled q and k [1,16,1024,128] f32 = 8 MiB each, idx [1,16,1024,153] i32,
+    # block scores [1,16,1024,1024] f32 = 64 MiB
     got = bsa.bsa_forward_workspace_bytes(1, 131072, 16, 128, 128, 0.15)
     idx = 16 * 1024 * 153 * 4
-    assert got == 2 * 8 * 2**20 + (idx + 255) // 256 * 256
+    assert got == 2 * 8 * 2**20 + (idx + 255) // 256 * 256 + 64 * 2**20
     assert bsa.bsa_forward_workspace_bytes(1, 100, 2, 64, 64, 0.5) == 0  # N % block_size
     assert bsa.bsa_forward_workspace_bytes(1, 512, 2, 96, 64, 0.5) == 0  # D unsupported
     assert bsa.bsa_forward_workspace_bytes(1, 512, 2, 64, 64, 0.1) == 0  # k = 0
@@ -98,6 +99,7 @@ def test_stage_entry_points_reject_bad_arguments(bsa):
     assert L.bsa_block_scores_topk(P(A), P(A), P(0), P(A), 1, 2, 8, 64, 9, P(0)) == 1
     assert L.bsa_block_scores_topk(P(A), P(A), P(M), P(A), 1, 2, 8, 64, 2, P(0)) == 3
     assert L.bsa_block_scores_topk(P(A), P(A), P(0), P(A), 1, 2, 8, 32, 2, P(0)) == 2
+    assert L.bsa_block_scores_topk(P(A), P(A), P(0), P(A), 1, 2, 8, 64, 2, P(0)) == 1  # scores required
     assert L.bsa_sparse_attn_fwd(P(A), P(A), P(A), P(A), P(A + 0x100), 1, 512, 2, 64, 64, 9, 0.125, 1, P(0)) == 1
     assert L.bsa_sparse_attn_fwd(P(A), P(A), P(A), P(A), P(A + 0x100), 1, 512, 2, 64, 64, 2, -1.0, 1, P(0)) == 1
     assert L.bsa_sparse_attn_fwd(P(A), P(A), P(A), P(0), P(A + 0x100), 1, 512, 2, 64, 64, 2, 0.125, 1, P(0)) == 1

@@ -87,7 +87,7 @@ def test_noalloc_matches_bsa_forward_on_calls_in_a_row(bsa):
 
 
 def test_noalloc_refuses_sizes_beyond_its_scratch(bsa):
-    # million-token problem: pooled q and k plus the index list need about 114 MB
+    # million-token problem: pooled q and k, the index list and the block scores need about 650 MB
     need = bsa.bsa_forward_workspace_bytes(1, 1 << 20, 8, 128, 256, 0.15)
     assert need > SCRATCH_BYTES
     P = ctypes.c_void_p
