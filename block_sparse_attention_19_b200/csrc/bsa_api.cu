@@ -137,24 +137,59 @@ bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_pool_kernel launch");
 }
 
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
 // Block scores S = qbar kbar^T per (b, h) on the tensor cores (split TF32),
-// written to S [B, H, nb, nb]; then the top-k selection reads S back.
+// written to S [B, H, nb, nb] by TMA tensor stores when a row of S is a
+// multiple of 16 bytes; then the top-k selection reads S back.
 bsa_status launch_scores(const float* qp, const float* kp, float* S, int B, int H, int nb, int D,
                          cudaStream_t st) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(bsa::block_scores_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bsa::kScSmem);
-    if (e != cudaSuccess) return cuda_fail(e, "scores smem attribute");
+    for (auto fn : {bsa::block_scores_tc_kernel<128>, bsa::block_scores_tc_kernel<256>}) {
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bsa::kScSmem);
+      if (e != cudaSuccess) return cuda_fail(e, "scores smem attribute");
+    }
     attr_set[dev] = true;
   }
-  const long tiles = static_cast<long>(B) * H * ((nb + bsa::kScM - 1) / bsa::kScM) *
-                     ((nb + bsa::kScN - 1) / bsa::kScN);
-  if (tiles > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "score grid too large");
-  bsa::block_scores_tc_kernel<<<static_cast<unsigned>(tiles), bsa::kScThreads, bsa::kScSmem, st>>>(
-      qp, kp, S, nb, D);
+  const int ntile = nb <= 128 ? 128 : 256;
+  const long ntiles = static_cast<long>(B) * H * ((nb + bsa::kScM - 1) / bsa::kScM) *
+                      ((nb + ntile - 1) / ntile);
+  const int tma_store = (nb % 4 == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0) ? 1 : 0;
+  CUtensorMap tm_s;
+  std::memset(&tm_s, 0, sizeof(tm_s));
+  if (tma_store) {
+    auto encode = tensor_map_encoder();
+    if (!encode) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(nb),
+                          static_cast<cuuint64_t>(B) * H};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(nb) * 4,
+                             static_cast<cuuint64_t>(nb) * nb * 4};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = encode(&tm_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, S, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(BSA_ERR_CUDA, "score tensor map failed (%d)", static_cast<int>(r));
+  }
+  const long grid = ntiles < sm_count() ? ntiles : sm_count();
+  if (ntile == 128)
+    bsa::block_scores_tc_kernel<128><<<static_cast<unsigned>(grid), bsa::kScThreads, bsa::kScSmem, st>>>(
+        qp, kp, S, tm_s, nb, D, ntiles, tma_store);
+  else
+    bsa::block_scores_tc_kernel<256><<<static_cast<unsigned>(grid), bsa::kScThreads, bsa::kScSmem, st>>>(
+        qp, kp, S, tm_s, nb, D, ntiles, tma_store);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_scores_tc_kernel launch");
 }

@@ -22,70 +22,26 @@ namespace bsa {
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
 
-// Order-preserving map float -> uint32 (larger float <=> larger key).
+// Order-preserving map float -> uint32 (larger float <=> larger key). -0 is
+// mapped as +0: the two compare equal, so they must tie (and go to the lower
+// index) like any other equal scores.
 __device__ __forceinline__ uint32_t float_key(float f) {
   uint32_t u = __float_as_uint(f);
+  u = u == 0x80000000u ? 0u : u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Per-lane key capacity of the register path of phase B (nb <= 32 * KPL).
-template <int KPL>
-__device__ __forceinline__ void select_row_regs(const float* srow, int nb, int k, int32_t* out,
-                                                int lane) {
-  uint32_t key[KPL];
-#pragma unroll
-  for (int t = 0; t < KPL; ++t) {
-    const int j = t * 32 + lane;
-    key[t] = j < nb ? float_key(srow[j]) : 0u;  // padding key 0 is never counted (cand >= 1)
-  }
-  // T = largest key value with #{key >= T} >= k: the k-th largest key.
-  uint32_t T = 0;
-#pragma unroll 1
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = T | (1u << bit);
-    int cnt = 0;
-#pragma unroll
-    for (int t = 0; t < KPL; ++t) cnt += key[t] >= cand;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-    if (cnt >= k) T = cand;
-  }
-  int gt = 0;
-#pragma unroll
-  for (int t = 0; t < KPL; ++t) gt += key[t] > T;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) gt += __shfl_xor_sync(0xffffffffu, gt, o);
-  const int need_eq = k - gt;  // >= 1 by the choice of T
-
-  // ordered emission: ascending j, lanes cover 32 consecutive j per step
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  int written = 0, eq_seen = 0;
-#pragma unroll
-  for (int t = 0; t < KPL; ++t) {
-    const int j = t * 32 + lane;
-    const bool eq = (j < nb) && key[t] == T;
-    const uint32_t eq_ballot = __ballot_sync(0xffffffffu, eq);
-    const int eq_rank = eq_seen + __popc(eq_ballot & lt_mask);
-    const bool sel = (j < nb) && (key[t] > T || (eq && eq_rank < need_eq));
-    const uint32_t sel_ballot = __ballot_sync(0xffffffffu, sel);
-    if (sel) out[written + __popc(sel_ballot & lt_mask)] = j;
-    written += __popc(sel_ballot);
-    eq_seen += __popc(eq_ballot);
-  }
 }
 
 __device__ __forceinline__ float key_float(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
 }
 
+// Number of the warp's keys >= t (one redux.sync instead of a shuffle tree).
 template <int KPL>
 __device__ __forceinline__ int warp_count_ge(const uint32_t (&key)[KPL], uint32_t t) {
-  int c = 0;
+  unsigned c = 0;
 #pragma unroll
   for (int i = 0; i < KPL; ++i) c += key[i] >= t;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-  return c;
+  return static_cast<int>(__reduce_add_sync(0xffffffffu, c));
 }
 
 // Bitonic sort of 64 keys held two per lane (element i = lane in a, lane + 32
@@ -115,36 +71,56 @@ __device__ __forceinline__ void warp_sort64_desc(uint32_t& a, uint32_t& b, int l
   }
 }
 
-// Same result as select_row_regs with far fewer passes on typical rows: the
+// Key of a score for the register path: float_key with the -0 fix done by
+// an add, and clamped to >= 1 (this merges the two lowest NaN patterns only)
+// so that the padding key 0 never enters a bracket, a count or the output.
+__device__ __forceinline__ uint32_t score_key(float f) {
+  const uint32_t u = __float_as_uint(f + 0.0f);  // -0 + 0 = +0
+  const uint32_t flip = static_cast<uint32_t>(static_cast<int32_t>(u) >> 31) | 0x80000000u;
+  return max(u ^ flip, 1u);
+}
+
+// One warp selects the k largest of a row of nb <= 32 * KPL scores held as
+// keys in registers, lane-major: lane l holds keys j = l * KPL + t, so
+// ascending j is lane order and each lane loads a contiguous run (float4
+// loads when `vec`: the row starts 16-byte aligned and nb % 4 == 0). The
 // k-th largest key is bracketed by bisection (up to 12 steps on the score
 // value, then on the key, which needs at most 32 steps) until the bracket
-// [lo, hi) holds at most 64 keys, which are then sorted exactly; a
-// bracket that cannot be split holds equal keys only. `cand` is 64 words of
-// shared memory private to the warp.
+// [lo, hi) holds at most 64 keys, which are then sorted exactly; a bracket
+// that cannot be split holds equal keys only. `cand` is 64 words of shared
+// memory private to the warp.
 template <int KPL>
 __device__ __forceinline__ void select_row_bracket(const float* srow, int nb, int k, int32_t* out,
-                                                   int lane, uint32_t* cand) {
+                                                   int lane, uint32_t* cand, bool vec) {
   uint32_t key[KPL];
+  const int j0 = lane * KPL;
+  if (KPL % 4 == 0 && vec) {
+#pragma unroll
+    for (int v = 0; v < KPL / 4; ++v) {
+      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+      const bool in = j0 + 4 * v < nb;  // nb % 4 == 0: the whole float4 is in the row
+      if (in) f = __ldg(reinterpret_cast<const float4*>(srow + j0) + v);
+      key[4 * v] = in ? score_key(f.x) : 0u;
+      key[4 * v + 1] = in ? score_key(f.y) : 0u;
+      key[4 * v + 2] = in ? score_key(f.z) : 0u;
+      key[4 * v + 3] = in ? score_key(f.w) : 0u;
+    }
+  } else {
+#pragma unroll
+    for (int t = 0; t < KPL; ++t) key[t] = j0 + t < nb ? score_key(__ldg(srow + j0 + t)) : 0u;
+  }
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll
   for (int t = 0; t < KPL; ++t) {
-    const int j = t * 32 + lane;
-    key[t] = j < nb ? float_key(srow[j]) : 0u;  // padding 0 never reaches a bracket above 0
-    if (j < nb) {
-      kmin = min(kmin, key[t]);
-      kmax = max(kmax, key[t]);
-    }
+    kmin = min(kmin, key[t] == 0u ? 0xFFFFFFFFu : key[t]);  // padding is not a key
+    kmax = max(kmax, key[t]);
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
   // invariant: count(key >= lo) = clo >= k > chi = count(key >= hi); hi may be 2^32
   uint32_t lo = kmin;
   uint64_t hi = static_cast<uint64_t>(kmax) + 1;
   int clo = nb, chi = 0;
-  if (kmin == 0u) clo = warp_count_ge(key, 0u) - (KPL * 32 - nb);  // real keys of value 0
 #pragma unroll 1
   for (int it = 0; it < 64 && clo - chi > 64 && hi - lo > 1; ++it) {
     const float flo = key_float(lo), fhi = key_float(static_cast<uint32_t>(hi - 1));
@@ -163,27 +139,40 @@ __device__ __forceinline__ void select_row_bracket(const float* srow, int nb, in
       chi = c;
     }
   }
+  // T = the k-th largest key, gt = #keys > T, eq = #keys == T
   uint32_t T;
+  int gt, eq;
   if (hi - lo == 1) {
     T = lo;  // the bracket holds copies of one key
+    gt = chi;
+    eq = clo - chi;
   } else if (clo - chi <= 64) {
-    // gather the bracket's keys and take the (k - chi)-th largest exactly
-    int base = 0;
-    const uint32_t lt_mask0 = (1u << lane) - 1u;
+    // gather the bracket's keys (in any order) and sort them
+    const uint32_t top = static_cast<uint32_t>(hi - 1);
+    unsigned mine = 0;
 #pragma unroll
-    for (int t = 0; t < KPL; ++t) {
-      const bool in = key[t] >= lo && static_cast<uint64_t>(key[t]) < hi && t * 32 + lane < nb;
-      const uint32_t bal = __ballot_sync(0xffffffffu, in);
-      if (in) cand[base + __popc(bal & lt_mask0)] = key[t];
-      base += __popc(bal);
+    for (int t = 0; t < KPL; ++t) mine += key[t] >= lo && key[t] <= top;
+    unsigned incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
+    const int total = static_cast<int>(__shfl_sync(0xffffffffu, incl, 31));
+    int off = static_cast<int>(incl - mine);
+#pragma unroll
+    for (int t = 0; t < KPL; ++t)
+      if (key[t] >= lo && key[t] <= top && off < 64) cand[off++] = key[t];
     __syncwarp();
-    uint32_t a = lane < base ? cand[lane] : 0u, b = lane + 32 < base ? cand[lane + 32] : 0u;
+    uint32_t a = lane < total ? cand[lane] : 0u, b = lane + 32 < total ? cand[lane + 32] : 0u;
     __syncwarp();
     warp_sort64_desc(a, b, lane);
-    const int r = k - chi - 1;
+    const int r = k - chi - 1;  // 0 <= r < clo - chi <= 64
     const uint32_t va = __shfl_sync(0xffffffffu, a, r & 31), vb = __shfl_sync(0xffffffffu, b, r & 31);
     T = r < 32 ? va : vb;
+    // every key == T lies in the bracket; keys above it are the chi keys >= hi
+    gt = chi + __popc(__ballot_sync(0xffffffffu, a > T)) + __popc(__ballot_sync(0xffffffffu, b > T));
+    eq = __popc(__ballot_sync(0xffffffffu, a == T)) + __popc(__ballot_sync(0xffffffffu, b == T));
   } else {
     // not narrowed in time (pathological rows): exact bitwise search
     T = 0;
@@ -192,22 +181,47 @@ __device__ __forceinline__ void select_row_bracket(const float* srow, int nb, in
       const uint32_t c = T | (1u << bit);
       if (warp_count_ge(key, c) >= k) T = c;
     }
+    gt = T == 0xFFFFFFFFu ? 0 : warp_count_ge(key, T + 1);
+    eq = warp_count_ge(key, T) - gt;
   }
-  const int gt = T == 0xFFFFFFFFu ? 0 : warp_count_ge(key, T + 1);
-  const int need_eq = k - gt;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  int written = 0, eq_seen = 0;
+  const int need_eq = k - gt;  // >= 1 by the choice of T
+  // this lane's picks as a bit mask over t (padding keys are 0 < T)
+  uint32_t sel = 0;
+  if (eq == need_eq) {
+    // no tie straddles the cut: the selection is every key >= T
 #pragma unroll
-  for (int t = 0; t < KPL; ++t) {
-    const int j = t * 32 + lane;
-    const bool eq = (j < nb) && key[t] == T;
-    const uint32_t eq_ballot = __ballot_sync(0xffffffffu, eq);
-    const int eq_rank = eq_seen + __popc(eq_ballot & lt_mask);
-    const bool sel = (j < nb) && (key[t] > T || (eq && eq_rank < need_eq));
-    const uint32_t sel_ballot = __ballot_sync(0xffffffffu, sel);
-    if (sel) out[written + __popc(sel_ballot & lt_mask)] = j;
-    written += __popc(sel_ballot);
-    eq_seen += __popc(eq_ballot);
+    for (int t = 0; t < KPL; ++t) sel |= (key[t] >= T ? 1u : 0u) << t;
+  } else {
+    // keys equal to T are taken in ascending j (lane order, then t) until k
+    uint32_t eqm = 0;
+#pragma unroll
+    for (int t = 0; t < KPL; ++t) {
+      sel |= (key[t] > T ? 1u : 0u) << t;
+      eqm |= (key[t] == T ? 1u : 0u) << t;
+    }
+    const int neq = __popc(eqm);
+    int incl = neq;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int take = need_eq - (incl - neq);  // equal keys this lane still takes
+    for (; take > 0 && eqm; --take) {
+      sel |= eqm & (0u - eqm);  // lowest remaining equal key
+      eqm &= eqm - 1u;
+    }
+  }
+  const int nsel = __popc(sel);
+  int incl = nsel;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  for (int pos = incl - nsel; sel && pos < k; ++pos) {
+    out[pos] = j0 + __ffs(sel) - 1;
+    sel &= sel - 1u;
   }
 }
 
@@ -239,7 +253,8 @@ __device__ __forceinline__ void select_row_smem(const float* srow, int nb, int k
     const int eq_rank = eq_seen + __popc(eq_ballot & lt_mask);
     const bool sel = (j < nb) && (key > T || (eq && eq_rank < need_eq));
     const uint32_t sel_ballot = __ballot_sync(0xffffffffu, sel);
-    if (sel) out[written + __popc(sel_ballot & lt_mask)] = j;
+    const int pos = written + __popc(sel_ballot & lt_mask);
+    if (sel && pos < k) out[pos] = j;
     written += __popc(sel_ballot);
     eq_seen += __popc(eq_ballot);
   }
@@ -247,7 +262,7 @@ __device__ __forceinline__ void select_row_smem(const float* srow, int nb, int k
 
 // grid.x = ceil(rows / kSelWarps); one warp per row of S ([rows, nb]).
 // Dynamic shared memory: kSelWarps * nb floats when nb > 1024 and stage_rows, else none.
-__global__ void __launch_bounds__(kSelThreads)
+__global__ void __launch_bounds__(kSelThreads, 4)
     block_topk_kernel(const float* __restrict__ S, int32_t* __restrict__ idx, long rows, int nb,
                       int k, int stage_rows) {
   extern __shared__ __align__(16) float sel_rows[];
@@ -257,18 +272,19 @@ __global__ void __launch_bounds__(kSelThreads)
   if (r >= rows) return;
   const float* srow = S + r * nb;
   int32_t* out = idx + r * static_cast<long>(k);
+  const bool vec = (nb & 3) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0;
   if (nb <= 32)
-    select_row_bracket<1>(srow, nb, k, out, lane, cand[warp]);
+    select_row_bracket<1>(srow, nb, k, out, lane, cand[warp], vec);
   else if (nb <= 64)
-    select_row_bracket<2>(srow, nb, k, out, lane, cand[warp]);
+    select_row_bracket<2>(srow, nb, k, out, lane, cand[warp], vec);
   else if (nb <= 128)
-    select_row_bracket<4>(srow, nb, k, out, lane, cand[warp]);
+    select_row_bracket<4>(srow, nb, k, out, lane, cand[warp], vec);
   else if (nb <= 256)
-    select_row_bracket<8>(srow, nb, k, out, lane, cand[warp]);
+    select_row_bracket<8>(srow, nb, k, out, lane, cand[warp], vec);
   else if (nb <= 512)
-    select_row_bracket<16>(srow, nb, k, out, lane, cand[warp]);
+    select_row_bracket<16>(srow, nb, k, out, lane, cand[warp], vec);
   else if (nb <= 1024)
-    select_row_bracket<32>(srow, nb, k, out, lane, cand[warp]);
+    select_row_bracket<32>(srow, nb, k, out, lane, cand[warp], vec);
   else if (stage_rows) {
     // the row is re-read once per key bit: stage it in shared memory
     float* row = sel_rows + static_cast<long>(warp) * nb;

@@ -210,6 +210,27 @@ def test_scores_topk_stage(bsa, oracle_mod, nb, D):
         accept_index_rows(idx.cpu().numpy(), S_ref, kk, idx_ref)
 
 
+@pytest.mark.parametrize("nb", [40, 100, 1024, 1501])
+def test_integer_scores_with_many_ties(bsa, oracle_mod, nb):
+    """Small-integer pooled inputs make every score an exact integer (or a
+    zero of either sign), so ties straddle the k-th score in most rows: the
+    index lists must equal the oracle's bit-exactly, lower ids winning, and
+    -0 must tie with +0."""
+    B, H, D = 1, 2, 64
+    rng = np.random.default_rng(77 + nb)
+    qp = rng.integers(-1, 2, (B, H, nb, D)).astype(np.float32)
+    kp = rng.integers(-2, 3, (B, H, nb, D)).astype(np.float32)
+    kp[:, :, ::7] = -0.0  # rows of negative zeros: their scores are zeros of either sign
+    kp[:, :, 3::7] = 0.0
+    S_ref = oracle_mod.block_scores(qp.astype(np.float64), kp.astype(np.float64))
+    for kk in sorted({1, max(1, nb // 7), nb // 2, nb}):
+        idx, S = bsa.bsa_block_scores_topk(torch.from_numpy(qp).cuda(), torch.from_numpy(kp).cuda(), kk,
+                                           scores=True)
+        torch.cuda.synchronize()
+        assert np.array_equal(S.cpu().numpy().astype(np.float64), S_ref)  # exact: integers below 2^24
+        assert np.array_equal(idx.cpu().numpy(), oracle_mod.topk(S_ref, kk)), f"k={kk}"
+
+
 def test_exact_score_ties_pick_lower_block(bsa, oracle_mod):
     """Duplicated key blocks give exactly equal pooled keys, hence exact score
     ties on both sides: the lower block id must win, bit-exactly."""
