@@ -347,8 +347,10 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
       }
       m_run = m_new;
       // P = exp2(S * scale_log2 - m) for key pairs with two-wide float32
-      // instructions; three pairs in eight take the polynomial exp2 on the FMA
-      // pipe. P is stored as packed bf16 over the first 64 columns of S.
+      // instructions; one pair in four takes the polynomial exp2 on the FMA
+      // pipe (the split measured fastest: the softmax is bound by issue slots
+      // more than by MUFU). P is stored as packed bf16 over the first 64
+      // columns of S.
       uint32_t pa[32], pb[32];
       uint64_t ps[4] = {0, 0, 0, 0};
       {
@@ -357,7 +359,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         for (int pr = 0; pr < 64; ++pr) {
           const uint64_t x2 = f2_fma(f2(BSA_S(2 * pr), BSA_S(2 * pr + 1)), sc2, nm2);
           uint64_t p2;
-          if (pr % 8 == 1 || pr % 8 == 4 || pr % 8 == 6) {
+          if (pr % 4 == 1) {
             p2 = exp2_poly2(x2);
           } else {
             float x0, x1;
