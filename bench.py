@@ -36,6 +36,11 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 METRIC = "block-sparse attn fwd tokens/s & effective TFLOP/s (% roofline), 1 B200"
+
+# DRAM read + write bytes per launch of the attention kernel, from the ncu
+# capture recorded in profiles/sparse_attn_tc2_traffic.md (the kernel as it
+# stands); workloads not captured report null.
+NCU_TRAFFIC = {"c3": 807.93e6 + 249.50e6, "c4": 4.98e9 + 585.72e6}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -331,7 +336,7 @@ def main():
             "kernel": "sparse_attn_tc2_kernel" if bs in (128, 256) else "sparse_attn_tc_kernel",
             "bound": "tensor", "achieved": achieved,
             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-            "peak_source": f"{peak_src} bf16 burst", "traffic": None,
+            "peak_source": f"{peak_src} bf16 burst", "traffic": NCU_TRAFFIC.get(cfg.name),
             "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
             "frac_of_roofline_time": roof_t / (attn_ms / 1e3),
             "flops_per_launch": flops, "algorithmic_bytes_per_launch": alg_bytes,
