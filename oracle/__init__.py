@@ -66,6 +66,8 @@ def _load():
         lib.oracle_topk_row.argtypes = [P, i, i, P]
         lib.oracle_topk.argtypes = [P, ctypes.c_long, i, i, P]
         lib.oracle_sparse_attn.argtypes = [P, P, P, i, i, i, i, i, i, P, i, P, i, d, P]
+        lib.oracle_topk_ex.argtypes = [P, ctypes.c_long, i, i, P, i, P]
+        lib.oracle_sparse_attn_ex.argtypes = [P, P, P, i, i, i, i, i, i, P, i, P, i, d, i, P]
         lib.oracle_num_threads.restype = i
         _lib = lib
     return _lib
@@ -125,24 +127,41 @@ def block_scores(qp: np.ndarray, kp: np.ndarray, rows: np.ndarray | None = None)
     return out
 
 
-def topk(scores: np.ndarray, k: int) -> np.ndarray:
-    """Top-k block ids of every score row, ties to the lower id, ascending ([SF] step 2)."""
+CAUSAL, FORCE_DIAG = 1, 2
+
+
+def topk(scores: np.ndarray, k: int, causal: bool = False, force_diag: bool = False,
+         qblocks: np.ndarray | None = None) -> np.ndarray:
+    """Top-k block ids of every score row, ties to the lower id, ascending ([SF] step 2).
+
+    With ``causal`` the row of query block i ranks only blocks j <= i and keeps
+    min(k, i+1) of them (with ``force_diag`` block i always, plus the best
+    j < i), padding the row with -1.  ``qblocks`` gives the query block of each
+    row (shape of ``scores`` without its last axis); None means the rows are all
+    nb query blocks in order."""
     s = np.ascontiguousarray(scores, np.float64)
     nb = s.shape[-1]
     if not (1 <= k <= nb):
         raise ValueError("need 1 <= k <= nb")
     rows = int(np.prod(s.shape[:-1]))
     out = np.empty(s.shape[:-1] + (k,), np.int32)
-    _load().oracle_topk(_ptr(s), rows, nb, k, _ptr(out))
+    if not causal:
+        _load().oracle_topk(_ptr(s), rows, nb, k, _ptr(out))
+        return out
+    flags = CAUSAL | (FORCE_DIAG if force_diag else 0)
+    qb = None if qblocks is None else np.ascontiguousarray(np.broadcast_to(qblocks, s.shape[:-1]), np.int32)
+    _load().oracle_topk_ex(_ptr(s), rows, nb, k, None if qb is None else _ptr(qb), flags, _ptr(out))
     return out
 
 
-def sparse_attn(q, k, v, idx, block_size: int, scale: float | None = None, rows=None) -> np.ndarray:
+def sparse_attn(q, k, v, idx, block_size: int, scale: float | None = None, rows=None,
+                causal: bool = False) -> np.ndarray:
     """Exact softmax attention over the selected key blocks ([SF] step 3, [MSA] §2.1).
 
     ``idx`` is int [B,H,nrows,k] (the selected key blocks of each listed query
-    block); ``rows`` is int [B,H,nrows] (None = all nb query blocks in order).
-    Returns float64 [B,H,nrows,block_size,D]."""
+    block; entries below 0 select nothing); ``rows`` is int [B,H,nrows] (None =
+    all nb query blocks in order).  With ``causal`` query token n ignores key
+    tokens t > n.  Returns float64 [B,H,nrows,block_size,D]."""
     q, code = _as_input(q)
     k_, code_k = _as_input(k)
     v, code_v = _as_input(v)
@@ -162,12 +181,18 @@ def sparse_attn(q, k, v, idx, block_size: int, scale: float | None = None, rows=
     if scale is None:
         scale = 1.0 / np.sqrt(D)
     out = np.empty((B, H, nrows, block_size, D), np.float64)
-    _load().oracle_sparse_attn(_ptr(q), _ptr(k_), _ptr(v), code, B, N, H, D, block_size,
-                               _ptr(idx), kk, rp, nrows, float(scale), _ptr(out))
+    if causal or (idx < 0).any():
+        _load().oracle_sparse_attn_ex(_ptr(q), _ptr(k_), _ptr(v), code, B, N, H, D, block_size,
+                                      _ptr(idx), kk, rp, nrows, float(scale), CAUSAL if causal else 0,
+                                      _ptr(out))
+    else:
+        _load().oracle_sparse_attn(_ptr(q), _ptr(k_), _ptr(v), code, B, N, H, D, block_size,
+                                   _ptr(idx), kk, rp, nrows, float(scale), _ptr(out))
     return out
 
 
-def forward(q, k, v, block_size: int, topk_ratio: float, rows=None, scale=None) -> dict:
+def forward(q, k, v, block_size: int, topk_ratio: float, rows=None, scale=None,
+            causal: bool = False, force_diag: bool = False) -> dict:
     """The whole path of the [SF] listing on the oracle: pool, score, select, attend.
 
     ``rows`` (int [B,H,nrows]) restricts the scored / attended query blocks to
@@ -181,8 +206,8 @@ def forward(q, k, v, block_size: int, topk_ratio: float, rows=None, scale=None) 
     qp = block_pool(q, block_size)
     kp = block_pool(k, block_size)
     S = block_scores(qp, kp, rows)
-    idx = topk(S, kk)
-    o = sparse_attn(q, k, v, idx, block_size, scale=scale, rows=rows)
+    idx = topk(S, kk, causal=causal, force_diag=force_diag, qblocks=rows)
+    o = sparse_attn(q, k, v, idx, block_size, scale=scale, rows=rows, causal=causal)
     return {"qp": qp, "kp": kp, "scores": S, "idx": idx, "o": o, "k": kk,
             "seconds": time.perf_counter() - t0}
 

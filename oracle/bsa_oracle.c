@@ -209,3 +209,107 @@ int oracle_num_threads(void) {
   return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------
+ * Causal variant (readings, listed in the design notes as well):
+ *   - query block i may select only key blocks j <= i, so it keeps
+ *     n_i = min(k, i + 1) blocks;
+ *   - with force_diag, block i itself is always kept and the other n_i - 1
+ *     are the highest-scoring blocks j < i;
+ *   - a selected list holds its n_i ids in ascending order, followed by
+ *     k - n_i entries of -1;
+ *   - inside the selected blocks, query token n sees key token t only if
+ *     t <= n ([MSA] §2.1: Softmax(Mask(QK^T/sqrt(d_k)))V, with the causal
+ *     mask), so only the diagonal block is masked token by token.
+ * ------------------------------------------------------------------------ */
+#define ORACLE_CAUSAL 1
+#define ORACLE_FORCE_DIAG 2
+
+/* Causal top-k for query block i of one row of scores. */
+void oracle_topk_row_causal(const double* s_row, int nb, int i, int k, int force_diag, int* idx) {
+  int n = k < i + 1 ? k : i + 1;
+  int ncand = force_diag ? i : i + 1; /* candidates ranked by score */
+  int nrank = force_diag ? n - 1 : n; /* how many of them are kept */
+  scored_block* order = (scored_block*)malloc((size_t)(ncand > 0 ? ncand : 1) * sizeof(scored_block));
+  for (int j = 0; j < ncand; ++j) {
+    order[j].s = s_row[j];
+    order[j].j = j;
+  }
+  qsort(order, (size_t)ncand, sizeof(scored_block), by_score_then_index);
+  for (int t = 0; t < nrank; ++t) idx[t] = order[t].j;
+  if (force_diag) idx[nrank] = i;
+  qsort(idx, (size_t)n, sizeof(int), ascending_int);
+  for (int t = n; t < k; ++t) idx[t] = -1;
+  free(order);
+  (void)nb;
+}
+
+/* Top-k over many rows with flags (bit 0: causal, bit 1: force the diagonal
+ * block). qblock[r] is the query block of row r (NULL: r % nb). */
+void oracle_topk_ex(const double* S, long nrows_total, int nb, int k, const int* qblock, int flags,
+                    int* idx) {
+#pragma omp parallel for schedule(static)
+  for (long r = 0; r < nrows_total; ++r) {
+    if (flags & ORACLE_CAUSAL) {
+      int i = qblock ? qblock[r] : (int)(r % nb);
+      oracle_topk_row_causal(S + r * nb, nb, i, k, (flags & ORACLE_FORCE_DIAG) != 0, idx + r * k);
+    } else {
+      oracle_topk_row(S + r * nb, nb, k, idx + r * k);
+    }
+  }
+}
+
+/* oracle_sparse_attn with flags: entries of idx below 0 select nothing, and
+ * with ORACLE_CAUSAL key token t is left out of the softmax of query token n
+ * when t > n. */
+void oracle_sparse_attn_ex(const void* q, const void* kmat, const void* v, int dtype, int B, int N,
+                           int H, int D, int bs, const int* idx, int k, const int* rows, int nrows,
+                           double scale, int flags, double* o) {
+  long ntok = (long)k * bs;
+#pragma omp parallel
+  {
+    double* logit = (double*)malloc((size_t)ntok * sizeof(double));
+    double* qrow = (double*)malloc((size_t)D * sizeof(double));
+#pragma omp for collapse(4) schedule(dynamic, 4)
+    for (int b = 0; b < B; ++b)
+      for (int h = 0; h < H; ++h)
+        for (int r = 0; r < nrows; ++r)
+          for (int t_q = 0; t_q < bs; ++t_q) {
+            size_t bh = (size_t)b * H + h;
+            int i = rows ? rows[bh * nrows + r] : r;
+            const int* sel = idx + (bh * nrows + r) * k;
+            int n = i * bs + t_q;
+            for (int d = 0; d < D; ++d) qrow[d] = elem(q, dtype, at_bnhd(N, H, D, b, n, h, d));
+            double m = -INFINITY;
+            for (int s = 0; s < k; ++s)
+              for (int u = 0; u < bs; ++u) {
+                double l = -INFINITY; /* masked or unselected */
+                if (sel[s] >= 0) {
+                  int t = sel[s] * bs + u;
+                  if (!(flags & ORACLE_CAUSAL) || t <= n) {
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += qrow[d] * elem(kmat, dtype, at_bnhd(N, H, D, b, t, h, d));
+                    l = scale * dot;
+                  }
+                }
+                logit[(long)s * bs + u] = l;
+                if (l > m) m = l;
+              }
+            double* out = o + ((bh * nrows + r) * bs + t_q) * D;
+            for (int d = 0; d < D; ++d) out[d] = 0.0;
+            double z = 0.0;
+            for (int s = 0; s < k; ++s)
+              for (int u = 0; u < bs; ++u) {
+                double l = logit[(long)s * bs + u];
+                if (l == -INFINITY) continue;
+                int t = sel[s] * bs + u;
+                double w = exp(l - m);
+                z += w;
+                for (int d = 0; d < D; ++d) out[d] += w * elem(v, dtype, at_bnhd(N, H, D, b, t, h, d));
+              }
+            for (int d = 0; d < D; ++d) out[d] /= z;
+          }
+    free(logit);
+    free(qrow);
+  }
+}

@@ -307,3 +307,118 @@ def test_matches_restated_page_listing_in_torch(oracle_mod):
     r = oracle_mod.forward(q.numpy(), k.numpy(), v.numpy(), bs, ratio)
     np.testing.assert_array_equal(r["idx"], np.sort(top.numpy(), -1))
     np.testing.assert_allclose(oracle_mod.o_to_bnhd(r["o"]), t(ref).numpy(), rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- causal variant
+# Readings: query block i ranks only key blocks j <= i and keeps min(k, i+1)
+# of them (with the diagonal forced in when asked), rows padded with -1; query
+# token n never sees key token t > n ([MSA] §2.1, Mask(QK^T) with the causal mask).
+
+def _lexsort_topk_causal(S, k, force_diag):
+    out = np.full(S.shape[:-1] + (k,), -1, np.int32)
+    for pos in np.ndindex(S.shape[:-1]):
+        i = pos[-1]
+        n = min(k, i + 1)
+        cand = np.arange(i if force_diag else i + 1)
+        order = cand[np.lexsort((cand, -S[pos][cand]))]
+        keep = list(order[: (n - 1 if force_diag else n)]) + ([i] if force_diag else [])
+        out[pos][:n] = np.sort(keep)
+    return out
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+@pytest.mark.parametrize("force_diag", [False, True])
+def test_causal_topk_matches_lexsort_brute_force(oracle_mod, seed, force_diag):
+    rng = np.random.default_rng(100 + seed)
+    S = rng.integers(-3, 4, (2, 3, 9, 9)).astype(np.float64)  # many exact ties
+    for k in (1, 3, 9):
+        got = oracle_mod.topk(S, k, causal=True, force_diag=force_diag)
+        np.testing.assert_array_equal(got, _lexsort_topk_causal(S, k, force_diag))
+
+
+def test_causal_topk_invariants(oracle_mod):
+    rng = np.random.default_rng(7)
+    S = rng.standard_normal((1, 2, 16, 16))
+    k = 5
+    for fd in (False, True):
+        idx = oracle_mod.topk(S, k, causal=True, force_diag=fd)
+        for h in range(2):
+            for i in range(16):
+                row, n = idx[0, h, i], min(k, i + 1)
+                valid = row[:n]
+                assert (row[n:] == -1).all() and (valid >= 0).all() and (valid <= i).all()
+                assert (np.diff(valid) > 0).all()
+                if fd:
+                    assert i in valid
+                ranked = [j for j in valid if not (fd and j == i)]
+                dropped = [j for j in range(i if fd else i + 1) if j not in valid]
+                if ranked and dropped:
+                    assert S[0, h, i, ranked].min() >= S[0, h, i, dropped].max()
+    # rows named explicitly give the same lists as the all-rows run
+    rows = np.array([[[3, 11, 15], [0, 7, 8]]])
+    sub = np.take_along_axis(S, rows[..., None], 2)
+    got = oracle_mod.topk(sub, k, causal=True, qblocks=rows)
+    np.testing.assert_array_equal(got, np.take_along_axis(oracle_mod.topk(S, k, causal=True), rows[..., None], 2))
+
+
+def test_causal_ratio_one_equals_causal_sdpa(oracle_mod):
+    """k = nb keeps every block j <= i, so the method is dense causal attention
+    (block_size 1 makes it token-level causal attention)."""
+    B, N, H, D = 2, 64, 2, 16
+    t = lambda x: torch.from_numpy(x).permute(0, 2, 1, 3)  # [B,H,N,D]
+    for bs in (1, 4, 8):
+        q, k, v = (_rand((B, N, H, D), s, bs=bs) for s in (70, 71, 72))
+        ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), is_causal=True)
+        for fd in (False, True):
+            r = oracle_mod.forward(q, k, v, bs, 1.0, causal=True, force_diag=fd)
+            np.testing.assert_allclose(oracle_mod.o_to_bnhd(r["o"]), ref.permute(0, 2, 1, 3).numpy(),
+                                       rtol=1e-12, atol=1e-12)
+
+
+def test_causal_index_list_equals_masked_dense(oracle_mod):
+    """Any causal index list (with -1 padding) equals dense attention under the
+    block mask and the token causal mask, built here in torch."""
+    B, N, H, D, bs, kk = 1, 48, 2, 8, 6, 3
+    nb = N // bs
+    q, k, v = (_rand((B, N, H, D), s, bs=bs) for s in (80, 81, 82))
+    rng = np.random.default_rng(83)
+    idx = np.full((B, H, nb, kk), -1, np.int32)
+    for h in range(H):
+        for i in range(nb):
+            n = min(kk, i + 1)
+            idx[0, h, i, :n] = np.sort(rng.choice(i + 1, n, replace=False))
+    o = oracle_mod.o_to_bnhd(oracle_mod.sparse_attn(q, k, v, idx, bs, causal=True))
+    blk = np.zeros((B, H, nb, nb), bool)
+    for h in range(H):
+        for i in range(nb):
+            blk[0, h, i, idx[0, h, i][idx[0, h, i] >= 0]] = True
+    mask = torch.from_numpy(blk).repeat_interleave(bs, 2).repeat_interleave(bs, 3)
+    mask &= torch.ones(N, N, dtype=torch.bool).tril()
+    t = lambda x: torch.from_numpy(x).permute(0, 2, 1, 3)
+    ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), attn_mask=mask)
+    np.testing.assert_allclose(o, ref.permute(0, 2, 1, 3).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_causal_future_tokens_change_nothing_before_them(oracle_mod):
+    """Changing q, k, v in blocks >= c leaves selection and output of every
+    query block < c bit-identical (pooling, scoring, selection and attention
+    all look only backwards)."""
+    B, N, H, D, bs, ratio, c = 1, 64, 2, 8, 4, 0.3, 9
+    q, k, v = (_rand((B, N, H, D), s, bs=bs) for s in (90, 91, 92))
+    q2, k2, v2 = (x.copy() for x in (q, k, v))
+    rng = np.random.default_rng(93)
+    for x in (q2, k2, v2):
+        x[:, c * bs:] += rng.standard_normal(x[:, c * bs:].shape) * 3
+    for fd in (False, True):
+        r1 = oracle_mod.forward(q, k, v, bs, ratio, causal=True, force_diag=fd)
+        r2 = oracle_mod.forward(q2, k2, v2, bs, ratio, causal=True, force_diag=fd)
+        np.testing.assert_array_equal(r1["idx"][:, :, :c], r2["idx"][:, :, :c])
+        np.testing.assert_array_equal(r1["o"][:, :, :c], r2["o"][:, :, :c])
+        assert not np.array_equal(r1["o"][:, :, c:], r2["o"][:, :, c:])
+
+
+def test_minus_one_entries_select_nothing(oracle_mod, small_case):
+    q, k, v, bs, ratio = small_case
+    r = oracle_mod.forward(q, k, v, bs, ratio)
+    pad = np.concatenate([r["idx"], np.full(r["idx"].shape[:-1] + (2,), -1, np.int32)], -1)
+    np.testing.assert_array_equal(oracle_mod.sparse_attn(q, k, v, pad, bs), r["o"])
