@@ -35,7 +35,11 @@ _STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "
 #: every function include/bsa.h declares
 EXPORTED = ("bsa_topk_count", "bsa_forward_workspace_bytes", "bsa_block_pool",
             "bsa_block_scores_topk", "bsa_sparse_attn_fwd", "bsa_forward", "bsa_status_string",
-            "bsa_last_error_detail", "bsa_device_error", "bsa_forward_noalloc")
+            "bsa_last_error_detail", "bsa_device_error", "bsa_forward_noalloc",
+            "bsa_block_scores_topk_ex", "bsa_sparse_attn_fwd_ex", "bsa_forward_ex")
+
+#: variant flags of the *_ex entry points (include/bsa.h)
+BSA_FLAG_CAUSAL, BSA_FLAG_FORCE_DIAG = 1, 2
 
 
 class BsaError(RuntimeError):
@@ -50,7 +54,7 @@ def _load() -> ctypes.CDLL:
                           "`python -m block_sparse_attention_19_b200.build`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, D, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
-    F = ctypes.c_float
+    F, U = ctypes.c_float, ctypes.c_uint
     sig = {
         "bsa_topk_count": ([I, D], I),
         "bsa_forward_workspace_bytes": ([I, I, I, I, I, D], Z),
@@ -62,6 +66,9 @@ def _load() -> ctypes.CDLL:
         "bsa_last_error_detail": ([], ctypes.c_char_p),
         "bsa_device_error": ([ctypes.POINTER(ctypes.c_int), P], I),
         "bsa_forward_noalloc": ([P, P, P, P, I, I, I, I, I, D, I, P], I),
+        "bsa_block_scores_topk_ex": ([P, P, P, P, I, I, I, I, I, U, P], I),
+        "bsa_sparse_attn_fwd_ex": ([P, P, P, P, P, I, I, I, I, I, I, F, I, U, P], I),
+        "bsa_forward_ex": ([P, P, P, P, I, I, I, I, I, D, I, U, P, Z, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -121,9 +128,10 @@ def bsa_block_pool(x: torch.Tensor, block_size: int, out: torch.Tensor | None = 
 
 def bsa_block_scores_topk(q_pooled: torch.Tensor, k_pooled: torch.Tensor, topk: int,
                           scores: bool = False, idx_out: torch.Tensor | None = None,
-                          scores_out: torch.Tensor | None = None):
+                          scores_out: torch.Tensor | None = None, flags: int = 0):
     """Block scores S (written to ``scores_out``, allocated if absent) and the
-    top-k index list. Returns idx, or (idx, S) when ``scores`` is true."""
+    top-k index list. Returns idx, or (idx, S) when ``scores`` is true.
+    ``flags``: BSA_FLAG_CAUSAL / BSA_FLAG_FORCE_DIAG (bsa_block_scores_topk_ex)."""
     _dev(q_pooled, "q_pooled")
     _dev(k_pooled, "k_pooled")
     if q_pooled.dtype != torch.float32 or k_pooled.dtype != torch.float32:
@@ -132,13 +140,17 @@ def bsa_block_scores_topk(q_pooled: torch.Tensor, k_pooled: torch.Tensor, topk: 
     idx = idx_out if idx_out is not None else torch.empty((B, H, nb, topk), device=q_pooled.device, dtype=torch.int32)
     S = scores_out if scores_out is not None else torch.empty((B, H, nb, nb), device=q_pooled.device,
                                                               dtype=torch.float32)
-    _check(lib.bsa_block_scores_topk(_p(q_pooled), _p(k_pooled), _p(S), _p(idx), B, H, nb, D, topk,
-                                     _stream(q_pooled)))
+    if flags:
+        _check(lib.bsa_block_scores_topk_ex(_p(q_pooled), _p(k_pooled), _p(S), _p(idx), B, H, nb, D, topk,
+                                            flags, _stream(q_pooled)))
+    else:
+        _check(lib.bsa_block_scores_topk(_p(q_pooled), _p(k_pooled), _p(S), _p(idx), B, H, nb, D, topk,
+                                         _stream(q_pooled)))
     return (idx, S) if scores else idx
 
 
 def bsa_sparse_attn_fwd(q, k, v, idx, block_size: int, scale: float | None = None,
-                        out: torch.Tensor | None = None) -> torch.Tensor:
+                        out: torch.Tensor | None = None, flags: int = 0) -> torch.Tensor:
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (idx, "idx")):
         _dev(t, n)
     if idx.dtype != torch.int32:
@@ -150,13 +162,17 @@ def bsa_sparse_attn_fwd(q, k, v, idx, block_size: int, scale: float | None = Non
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     o = out if out is not None else torch.empty_like(q)
-    _check(lib.bsa_sparse_attn_fwd(_p(q), _p(k), _p(v), _p(idx), _p(o), B, N, H, D, block_size, topk,
-                                   float(scale), _dtype_code(q), _stream(q)))
+    if flags:
+        _check(lib.bsa_sparse_attn_fwd_ex(_p(q), _p(k), _p(v), _p(idx), _p(o), B, N, H, D, block_size, topk,
+                                          float(scale), _dtype_code(q), flags, _stream(q)))
+    else:
+        _check(lib.bsa_sparse_attn_fwd(_p(q), _p(k), _p(v), _p(idx), _p(o), B, N, H, D, block_size, topk,
+                                       float(scale), _dtype_code(q), _stream(q)))
     return o
 
 
 def bsa_forward(q, k, v, block_size: int, topk_ratio: float, workspace: torch.Tensor | None = None,
-                out: torch.Tensor | None = None) -> torch.Tensor:
+                out: torch.Tensor | None = None, flags: int = 0) -> torch.Tensor:
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _dev(t, n)
     if not (q.dtype == k.dtype == v.dtype):
@@ -166,9 +182,13 @@ def bsa_forward(q, k, v, block_size: int, topk_ratio: float, workspace: torch.Te
     if workspace is None:
         workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
     o = out if out is not None else torch.empty_like(q)
-    _check(lib.bsa_forward(_p(q), _p(k), _p(v), _p(o), B, N, H, D, block_size, float(topk_ratio),
-                           _dtype_code(q), _p(workspace), workspace.numel() * workspace.element_size(),
-                           _stream(q)))
+    nbytes = workspace.numel() * workspace.element_size()
+    if flags:
+        _check(lib.bsa_forward_ex(_p(q), _p(k), _p(v), _p(o), B, N, H, D, block_size, float(topk_ratio),
+                                  _dtype_code(q), flags, _p(workspace), nbytes, _stream(q)))
+    else:
+        _check(lib.bsa_forward(_p(q), _p(k), _p(v), _p(o), B, N, H, D, block_size, float(topk_ratio),
+                               _dtype_code(q), _p(workspace), nbytes, _stream(q)))
     return o
 
 

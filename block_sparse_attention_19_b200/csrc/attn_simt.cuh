@@ -12,9 +12,13 @@
 // shared memory in tiles of 64 keys and keeps a flash-style running max, sum
 // and output per row (each warp owns 4 rows; lane l owns output columns
 // l, l+32, ...). Logits for a tile are computed one key per lane.
+// An index row ends at its first -1 entry; with kFlagCausal key token t is
+// left out for query token n when t > n.
 #pragma once
 
 #include <stdint.h>
+
+#include "bsa_ptx.cuh"
 
 namespace bsa {
 
@@ -35,7 +39,8 @@ template <int D>
 __global__ void __launch_bounds__(kSimtThreads)
     sparse_attn_simt_kernel(const float* __restrict__ q, const float* __restrict__ kmat,
                             const float* __restrict__ v, const int32_t* __restrict__ idx,
-                            float* __restrict__ o, int N, int H, int bs, int k, float scale) {
+                            float* __restrict__ o, int N, int H, int bs, int k, float scale,
+                            unsigned flags) {
   extern __shared__ __align__(16) unsigned char simt_raw[];
   SimtSmem<D>& sm = *reinterpret_cast<SimtSmem<D>*>(simt_raw);
   constexpr int DL = D / 32;  // output columns per lane
@@ -73,9 +78,14 @@ __global__ void __launch_bounds__(kSimtThreads)
 
   const int32_t* sel = idx + ((b * H + h) * static_cast<long>(nb) + i) * k;
   const int tiles_per_block = bs / kSimtKeys;
+  const bool causal = (flags & kFlagCausal) != 0;
   for (int s = 0; s < k; ++s) {
     int blk = sel[s];
-    blk = blk < 0 ? 0 : (blk >= nb ? nb - 1 : blk);
+    if (blk < 0) {
+      if (s > 0) break;  // the row's valid entries end here (a row of only -1 reads block 0)
+      blk = 0;
+    }
+    blk = blk >= nb ? nb - 1 : blk;
     for (int tt = 0; tt < tiles_per_block; ++tt) {
       const int t0 = blk * bs + tt * kSimtKeys;
       __syncthreads();  // previous tile fully consumed
@@ -98,12 +108,19 @@ __global__ void __launch_bounds__(kSimtThreads)
         }
         s0 *= scale;
         s1 *= scale;
+        if (causal) {
+          if (t0 + lane > n0 + r) s0 = -INFINITY;
+          if (t0 + lane + 32 > n0 + r) s1 = -INFINITY;
+        }
         float mx = fmaxf(s0, s1);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
         const float m_new = fmaxf(m[rr], mx);
-        const float alpha = expf(m[rr] - m_new);  // 0 on the first tile (m = -inf)
-        const float p0 = expf(s0 - m_new), p1 = expf(s1 - m_new);
+        // reference point of the exponentials: finite even while every key so
+        // far is masked (then alpha and p are 0, as are l and acc)
+        const float m_ref = m_new == -INFINITY ? 0.f : m_new;
+        const float alpha = expf(m[rr] - m_ref);  // 0 on the first tile (m = -inf)
+        const float p0 = expf(s0 - m_ref), p1 = expf(s1 - m_ref);
         float ps = p0 + p1;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);

@@ -77,6 +77,7 @@ struct TcBarriers {
   uint64_t mma_drained;
   uint32_t tmem_base;
   int abort;
+  int kvalid;  // valid entries of the index row (at least 1)
 };
 static_assert(sizeof(TcBarriers) <= 512, "barrier area");
 
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
                           const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ o, int N,
-                          int H, int bs, int k, float scale_log2) {
+                          int H, int bs, int k, float scale_log2, unsigned flags) {
   using L = TcLayout<D, BM>;
   constexpr int KS = L::kStages;
   extern __shared__ __align__(1024) unsigned char tc_raw[];
@@ -153,7 +154,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int h = static_cast<int>(u % H);
   const int b = static_cast<int>(u / H);
   const int32_t* sel = idx + ((static_cast<long>(b) * H + h) * nb + i) * k;
-  const int T = bs == 64 ? (k + 1) / 2 : (bs == 128 ? k : 2 * k);  // key tiles
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -173,6 +173,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int q = 0; q < 4; ++q) mbar_init(&bar.pair[q], 64);
     mbar_init(&bar.mma_drained, 1);
     bar.abort = 0;
+    // a row lists its blocks, then pads with -1; a row of only -1 reads block 0
+    bar.kvalid = max(index_row_valid(sel, k), 1);
     fence_mbarrier_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -187,6 +189,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
   const uint32_t sbase = smem_u32(smem);
+  const int kv = bar.kvalid;
+  const int T = bs == 64 ? (kv + 1) / 2 : (bs == 128 ? kv : 2 * kv);  // key tiles
 
   if (warp == 0) {
     // ============================================================ TMA producers
@@ -212,7 +216,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       for (int t = 0; t < T && ok; ++t) {
         const int s = t % KS, use = t / KS;
-        const int halves = tile_keys(t, bs, k) / 64;
+        const int halves = tile_keys(t, bs, kv) / 64;
         int row0[2];
         for (int hf = 0; hf < halves; ++hf) row0[hf] = half_row0(sel, t, hf, bs, nb);
         if (t >= KS) ok = mbar_wait(&empty[s], (use - 1) & 1, abort_flag, is_k ? 101 : 102);
@@ -241,7 +245,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int t = 0; t <= T && ok; ++t) {
         if (t < T) {  // ---- S_t = Q K_t^T
           const int s = t % KS, use = t / KS;
-          const int nk = tile_keys(t, bs, k);
+          const int nk = tile_keys(t, bs, kv);
           ok = mbar_wait(&bar.k_full[s], use & 1, abort_flag, 202);
           if (!ok) break;
           tc_fence_after();
@@ -261,7 +265,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (t >= 1) {  // ---- O += P_j V_j, j = t - 1
           const int j = t - 1;
           const int s = j % KS, use = j / KS;
-          const int nk = tile_keys(j, bs, k);
+          const int nk = tile_keys(j, bs, kv);
           ok = mbar_wait(&bar.p_full, j & 1, abort_flag, 204);
           if (ok) ok = mbar_wait(&bar.v_full[s], use & 1, abort_flag, 205);
           if (!ok) break;
@@ -300,7 +304,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
-      const bool has = half == 0 || tile_keys(j, bs, k) == 128;  // this half holds keys
+      const bool has = half == 0 || tile_keys(j, bs, kv) == 128;  // this half holds keys
       ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_full[j % 2], (j / 2) & 1, abort_flag, 301));
       if (!ok) break;
       tc_fence_after();
@@ -311,6 +315,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_ld32(scol, sv[0]);
         tmem_ld32(scol + 32, sv[1]);
         tmem_wait_ld();
+        if (flags & kFlagCausal) {
+          // key c of this half is token kbase + c; keys after the thread's
+          // query token (c > lim) are left out (only the diagonal block)
+          const int kbase = half_row0(sel, j, half, bs, nb);
+          const int lim = i * bs + part * BM + row - kbase;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (e > lim) sv[0][e] = __float_as_uint(-INFINITY);
+            if (e + 32 > lim) sv[1][e] = __float_as_uint(-INFINITY);
+          }
+        }
         float m8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) m8[e] = fmaxf(__uint_as_float(sv[0][e]), __uint_as_float(sv[1][e]));

@@ -84,6 +84,7 @@ struct Tc2Barriers {
   uint64_t mma_drained;
   uint32_t tmem_base;
   int abort;
+  int tiles[2];  // key tiles of stream A and B (valid index entries, x2 for block_size 256)
 };
 static_assert(sizeof(Tc2Barriers) <= 512, "barrier area");
 
@@ -97,8 +98,17 @@ __device__ __forceinline__ int tc2_key_row(const int32_t* sel_a, const int32_t* 
   return clamp_block(__ldg(sel_a + t / 2), nb) * 256 + (t % 2) * 128 + hf * 64;  // bs == 256
 }
 
+// Causal mask on 32 scores of a row: column c0 + e becomes -inf when it is
+// above lim.
+__device__ __forceinline__ void tc2_mask_after(uint32_t (&r)[32], int c0, int lim) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e)
+    if (c0 + e > lim) r[e] = __float_as_uint(-INFINITY);
+}
+
 // grid.x = B * H * ceil(nb / 2) for block_size 128, B * H * nb for 256.
-template <int D>
+// kCausal: key tokens after the query token are masked (kFlagCausal).
+template <int D, bool kCausal>
 __global__ void __launch_bounds__(kTc2Threads, 1)
     sparse_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
@@ -132,9 +142,6 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
   const long bh = static_cast<long>(b) * H + h;
   const int32_t* sel_a = idx + (bh * nb + iA) * k;
   const int32_t* sel_b = shared_kv ? sel_a : idx + (bh * nb + (iA + 1 < nb ? iA + 1 : iA)) * k;
-  const int T = shared_kv ? 2 * k : k;  // key tiles per stream
-  // loads per ring: one per (stream, tile) when key lists differ, one per tile when shared
-  const int nloads = shared_kv ? T : T * nstreams;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -158,6 +165,12 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     }
     mbar_init(&bar.mma_drained, 1);
     bar.abort = 0;
+    // key tiles per stream: the valid entries of its index row (at least one,
+    // so that a row of only -1 still reads block 0 instead of nothing)
+    const int ta = max(index_row_valid(sel_a, k), 1);
+    const int tb = nstreams == 2 && !shared_kv ? max(index_row_valid(sel_b, k), 1) : 0;
+    bar.tiles[0] = shared_kv ? 2 * ta : ta;
+    bar.tiles[1] = shared_kv ? 2 * ta : tb;
     fence_mbarrier_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -172,6 +185,15 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
   const uint32_t sbase = smem_u32(smem);
+  const int TA = bar.tiles[0], TB = bar.tiles[1];
+  // Ring order of the K and V loads: one per (stream, tile), alternating A, B
+  // while both streams have tiles, then the longer stream alone; one per tile
+  // when the streams share their key tiles.
+  const int Tmin = min(TA, TB);
+  const int nloads = shared_kv ? TA : TA + TB;
+  auto load_index = [&](int x, int t) {
+    return shared_kv ? t : (t < Tmin ? 2 * t + x : 2 * Tmin + (t - Tmin));
+  };
   // register split: each role adjusts its own allowance on entry (warp
   // group 0: producers, MMA issuer and the idle warp 3 give registers away)
   if (warp == 0 || warp == 2) {
@@ -201,8 +223,9 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
       }
       for (int n = 0; n < nloads && ok; ++n) {
         const int s = n % S, use = n / S;
-        const int x = shared_kv ? 0 : n % nstreams;
-        const int t = shared_kv ? n : n / nstreams;
+        // inverse of load_index
+        const int x = shared_kv ? 0 : (n < 2 * Tmin ? (n & 1) : (TA > TB ? 0 : 1));
+        const int t = shared_kv ? n : (n < 2 * Tmin ? (n >> 1) : Tmin + (n - 2 * Tmin));
         int r[2];
         for (int hf = 0; hf < 2; ++hf) r[hf] = tc2_key_row(sel_a, sel_b, x, t, hf, bs, nb);
         if (n >= S) ok = mbar_wait(&empty[s], (use - 1) & 1, abort_flag, is_k ? 111 : 112);
@@ -237,13 +260,17 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
       const uint64_t dv0 = smem_desc_sw128(sbase + L::kVOff, 128 * 128, kSBO);
       constexpr uint64_t kTileStep = L::kTileBytes >> 4;
       // ring index of stream x's tile t (K and V rings are filled in the same order)
-      auto load_index = [&](int x, int t) { return shared_kv ? t : t * nstreams + x; };
       bool ok = mbar_wait(&bar.q_full, 0, abort_flag, 211);
+      // The rings are consumed in load order: kn and vn are the next K and
+      // V loads (a load serves both streams, stream B last, when they share
+      // their key tiles).
+      int kn = 0, vn = 0;
       // S_X(0)
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
         if (!ok || x >= nstreams) break;
-        const int n = load_index(x, 0);
+        const int n = kn;
+        if (!shared_kv || x == 1) ++kn;
         ok = mbar_wait_fast(&bar.k_full[n % KS], (n / KS) & 1, abort_flag, 212);
         if (!ok) break;
         tc_fence_after();
@@ -255,13 +282,18 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         }
         mma_commit(&bar.s_full[x]);
       }
-      for (int j = 0; j < T && ok; ++j) {
-        const bool more = j + 1 < T;
+      const int Tmax = max(TA, TB);
+      for (int j = 0; j < Tmax && ok; ++j) {
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-          if (x >= nstreams) break;
+          const int Tx = x == 0 ? TA : TB;
+          if (j >= Tx) continue;  // this stream is done (or absent)
+          const bool more = j + 1 < Tx;
           // PV_X(j) needs P_X(j) and V(x, j); S_X(j+1) needs K(x, j+1)
-          const int nv = load_index(x, j), nk = load_index(x, j + 1);
+          const int nv = vn, nk = kn;
+          const bool last_user = !shared_kv || x == 1;
+          vn += last_user;
+          if (more) kn += last_user;
           ok = mbar_wait_fast(&bar.p_full[x], j & 1, abort_flag, 213) &&
                mbar_wait_fast(&bar.v_full[nv % VS], (nv / VS) & 1, abort_flag, 214) &&
                (!more || mbar_wait_fast(&bar.k_full[nk % KS], (nk / KS) & 1, abort_flag, 215));
@@ -274,7 +306,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
             mma_bf16_ts(tmem + L::col_o(x), a_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv,
                         (j > 0 || kk > 0) ? 1u : 0u);
           // the V ring is shallow, so its entry is freed as soon as the product is done
-          if (!shared_kv || x == 1) mma_commit(&bar.v_empty[nv % VS]);
+          if (last_user) mma_commit(&bar.v_empty[nv % VS]);
           if (more) {
             const uint64_t dq = dq0 + x * kTileStep, dk = dk0 + (nk % KS) * kTileStep;
 #pragma unroll
@@ -305,15 +337,20 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     const uint32_t ocol = lane_base + L::col_o(x);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < T; ++j) {
+    const int Tx = x == 0 ? TA : TB;
+    for (int j = 0; j < Tx; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_full[x], j & 1, abort_flag, 311));
       if (!ok) break;
       tc_fence_after();
       if (quad == 0 && lane == 0) {
         // S_X(j) is complete: the K tile it read can be refilled
-        const int nk = shared_kv ? j : j * nstreams + x;
-        mbar_arrive(&bar.k_empty[nk % KS]);
+        mbar_arrive(&bar.k_empty[load_index(x, j) % KS]);
       }
+      // first key token of this tile; with the causal flag a tile that
+      // reaches past the tile's first query token masks key c for row r when
+      // kbase + c > qbase + r (only the diagonal block does)
+      const int kbase = kCausal ? tc2_key_row(sel_a, sel_b, x, j, 0, bs, nb) : 0;
+      const bool mask_tile = kCausal && kbase + 127 > row0[x];
       // The whole S row in registers: four TMEM loads, one wait.
       uint32_t sa[32], sb[32], sc[32], sd[32];
       tmem_ld32(scol, sa);
@@ -321,6 +358,14 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
       tmem_ld32(scol + 64, sc);
       tmem_ld32(scol + 96, sd);
       tmem_wait_ld();
+      if (mask_tile) {
+        // keys c > lim of this tile lie after the thread's query token
+        const int lim = row0[x] + row - kbase;
+        tc2_mask_after(sa, 0, lim);
+        tc2_mask_after(sb, 32, lim);
+        tc2_mask_after(sc, 64, lim);
+        tc2_mask_after(sd, 96, lim);
+      }
 #define BSA_S(i) __uint_as_float((i) < 32 ? sa[(i) & 31] : (i) < 64 ? sb[(i) & 31] : (i) < 96 ? sc[(i) & 31] : sd[(i) & 31])
       float m4[4];
 #pragma unroll

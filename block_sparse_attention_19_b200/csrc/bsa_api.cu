@@ -63,6 +63,17 @@ bsa_status check_dims(int B, int N, int H, int D, int block_size) {
   return BSA_OK;
 }
 
+static_assert(BSA_FLAG_CAUSAL == bsa::kFlagCausal && BSA_FLAG_FORCE_DIAG == bsa::kFlagForceDiag,
+              "flag values of the header and the kernels");
+
+bsa_status check_flags(unsigned flags) {
+  if (flags & ~(BSA_FLAG_CAUSAL | BSA_FLAG_FORCE_DIAG))
+    return fail(BSA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  if ((flags & BSA_FLAG_FORCE_DIAG) && !(flags & BSA_FLAG_CAUSAL))
+    return fail(BSA_ERR_INVALID_ARG, "BSA_FLAG_FORCE_DIAG needs BSA_FLAG_CAUSAL");
+  return BSA_OK;
+}
+
 bsa_status check_dtype(bsa_dtype dt) {
   if (dt != BSA_F32 && dt != BSA_BF16) return fail(BSA_ERR_UNSUPPORTED, "dtype %d", static_cast<int>(dt));
   return BSA_OK;
@@ -194,7 +205,8 @@ bsa_status launch_scores(const float* qp, const float* kp, float* S, int B, int 
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_scores_tc_kernel launch");
 }
 
-bsa_status launch_topk(const float* S, int32_t* idx, int B, int H, int nb, int k, cudaStream_t st) {
+bsa_status launch_topk(const float* S, int32_t* idx, int B, int H, int nb, int k, unsigned flags,
+                       cudaStream_t st) {
   const long rows = static_cast<long>(B) * H * nb;
   const size_t stage_bytes = static_cast<size_t>(bsa::kSelWarps) * nb * sizeof(float);
   const bool stage = nb > 1024 && stage_bytes <= 200 * 1024;
@@ -210,22 +222,22 @@ bsa_status launch_topk(const float* S, int32_t* idx, int B, int H, int nb, int k
   const long grid = (rows + bsa::kSelWarps - 1) / bsa::kSelWarps;
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "top-k grid too large");
   bsa::block_topk_kernel<<<static_cast<unsigned>(grid), bsa::kSelThreads, stage ? stage_bytes : 0, st>>>(
-      S, idx, rows, nb, k, stage ? 1 : 0);
+      S, idx, rows, nb, k, stage ? 1 : 0, flags);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_topk_kernel launch");
 }
 
 bsa_status launch_select(const float* qp, const float* kp, float* S, int32_t* idx, int B, int H,
-                         int nb, int D, int k, cudaStream_t st) {
+                         int nb, int D, int k, unsigned flags, cudaStream_t st) {
   bsa_status s;
   if ((s = launch_scores(qp, kp, S, B, H, nb, D, st)) != BSA_OK) return s;
-  return launch_topk(S, idx, B, H, nb, k, st);
+  return launch_topk(S, idx, B, H, nb, k, flags, st);
 }
 
 template <int D>
 bsa_status launch_attn_simt(const float* q, const float* k, const float* v, const int32_t* idx,
                             float* o, int B, int N, int H, int bs, int kk, float scale,
-                            cudaStream_t st) {
+                            unsigned flags, cudaStream_t st) {
   const size_t smem = sizeof(bsa::SimtSmem<D>);
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -239,7 +251,7 @@ bsa_status launch_attn_simt(const float* q, const float* k, const float* v, cons
   const long grid = static_cast<long>(B) * H * (N / bs) * (bs / bsa::kSimtRows);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   bsa::sparse_attn_simt_kernel<D><<<static_cast<unsigned>(grid), bsa::kSimtThreads, smem, st>>>(
-      q, k, v, idx, o, N, H, bs, kk, scale);
+      q, k, v, idx, o, N, H, bs, kk, scale, flags);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_simt_kernel launch");
 }
@@ -247,7 +259,7 @@ bsa_status launch_attn_simt(const float* q, const float* k, const float* v, cons
 template <int D, int BM>
 bsa_status launch_attn_tc(const void* q, const void* k, const void* v, const int32_t* idx,
                           void* o, int B, int N, int H, int bs, int kk, float scale,
-                          cudaStream_t st) {
+                          unsigned flags, cudaStream_t st) {
   using L = bsa::TcLayout<D, BM>;
   CUtensorMap mq, mk, mv;
   bsa_status s;
@@ -268,14 +280,14 @@ bsa_status launch_attn_tc(const void* q, const void* k, const void* v, const int
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   const float scale_log2 = scale * 1.4426950408889634f;
   bsa::sparse_attn_tc_kernel<D, BM><<<static_cast<unsigned>(grid), bsa::kTcThreads, L::kBytes, st>>>(
-      mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, bs, kk, scale_log2);
+      mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, bs, kk, scale_log2, flags);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc_kernel launch");
 }
 
-template <int D>
-bsa_status launch_attn_tc2(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
-                           int B, int N, int H, int bs, int kk, float scale, cudaStream_t st) {
+template <int D, bool kCausal>
+bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
+                              int B, int N, int H, int bs, int kk, float scale, cudaStream_t st) {
   using L = bsa::Tc2Layout<D>;
   CUtensorMap mq, mk, mv;
   bsa_status s;
@@ -286,14 +298,14 @@ bsa_status launch_attn_tc2(const void* q, const void* k, const void* v, const in
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_tc2_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_tc2_kernel<D, kCausal>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return cuda_fail(e, "tc2 smem attribute");
     // The kernel moves registers between warp groups (setmaxnreg); an increase
     // that the launch allocation cannot cover would wait forever, so refuse
     // to launch unless the compiled register count covers the split.
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, bsa::sparse_attn_tc2_kernel<D>);
+    e = cudaFuncGetAttributes(&fa, bsa::sparse_attn_tc2_kernel<D, kCausal>);
     if (e != cudaSuccess) return cuda_fail(e, "tc2 attributes");
     if (fa.numRegs < static_cast<int>(bsa::kTc2LaunchRegs))
       return fail(BSA_ERR_UNSUPPORTED, "attention kernel built with %d registers/thread, its register split needs %u",
@@ -304,27 +316,35 @@ bsa_status launch_attn_tc2(const void* q, const void* k, const void* v, const in
   const long grid = static_cast<long>(B) * H * (bs == 256 ? nb : (nb + 1) / 2);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   const float scale_log2 = scale * 1.4426950408889634f;
-  bsa::sparse_attn_tc2_kernel<D><<<static_cast<unsigned>(grid), bsa::kTc2Threads, L::kBytes, st>>>(
+  bsa::sparse_attn_tc2_kernel<D, kCausal><<<static_cast<unsigned>(grid), bsa::kTc2Threads, L::kBytes, st>>>(
       mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, bs, kk, scale_log2);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc2_kernel launch");
 }
 
+template <int D>
+bsa_status launch_attn_tc2(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
+                           int B, int N, int H, int bs, int kk, float scale, unsigned flags,
+                           cudaStream_t st) {
+  return (flags & BSA_FLAG_CAUSAL) ? launch_attn_tc2_as<D, true>(q, k, v, idx, o, B, N, H, bs, kk, scale, st)
+                                   : launch_attn_tc2_as<D, false>(q, k, v, idx, o, B, N, H, bs, kk, scale, st);
+}
+
 bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                        int B, int N, int H, int D, int bs, int kk, float scale, bsa_dtype dt,
-                       cudaStream_t st) {
+                       unsigned flags, cudaStream_t st) {
   if (dt == BSA_F32) {
     const float *fq = static_cast<const float*>(q), *fk = static_cast<const float*>(k),
                 *fv = static_cast<const float*>(v);
     float* fo = static_cast<float*>(o);
-    return D == 64 ? launch_attn_simt<64>(fq, fk, fv, idx, fo, B, N, H, bs, kk, scale, st)
-                   : launch_attn_simt<128>(fq, fk, fv, idx, fo, B, N, H, bs, kk, scale, st);
+    return D == 64 ? launch_attn_simt<64>(fq, fk, fv, idx, fo, B, N, H, bs, kk, scale, flags, st)
+                   : launch_attn_simt<128>(fq, fk, fv, idx, fo, B, N, H, bs, kk, scale, flags, st);
   }
   if (bs == 64)
-    return D == 64 ? launch_attn_tc<64, 64>(q, k, v, idx, o, B, N, H, bs, kk, scale, st)
-                   : launch_attn_tc<128, 64>(q, k, v, idx, o, B, N, H, bs, kk, scale, st);
-  return D == 64 ? launch_attn_tc2<64>(q, k, v, idx, o, B, N, H, bs, kk, scale, st)
-                 : launch_attn_tc2<128>(q, k, v, idx, o, B, N, H, bs, kk, scale, st);
+    return D == 64 ? launch_attn_tc<64, 64>(q, k, v, idx, o, B, N, H, bs, kk, scale, flags, st)
+                   : launch_attn_tc<128, 64>(q, k, v, idx, o, B, N, H, bs, kk, scale, flags, st);
+  return D == 64 ? launch_attn_tc2<64>(q, k, v, idx, o, B, N, H, bs, kk, scale, flags, st)
+                 : launch_attn_tc2<128>(q, k, v, idx, o, B, N, H, bs, kk, scale, flags, st);
 }
 
 struct Workspace {
@@ -400,9 +420,11 @@ bsa_status bsa_block_pool(const void* x, float* x_pooled, int B, int N, int H, i
   return ok();
 }
 
-bsa_status bsa_block_scores_topk(const float* q_pooled, const float* k_pooled, float* scores,
-                                 int32_t* idx, int B, int H, int nb, int D, int k, void* stream) {
+bsa_status bsa_block_scores_topk_ex(const float* q_pooled, const float* k_pooled, float* scores,
+                                    int32_t* idx, int B, int H, int nb, int D, int k, unsigned flags,
+                                    void* stream) {
   bsa_status s;
+  if ((s = check_flags(flags)) != BSA_OK) return s;
   if (B < 1 || H < 1 || nb < 1) return fail(BSA_ERR_INVALID_ARG, "sizes must be positive");
   if (D != 64 && D != 128) return fail(BSA_ERR_UNSUPPORTED, "D=%d (supported: 64, 128)", D);
   if (nb > 32768) return fail(BSA_ERR_UNSUPPORTED, "nb=%d > 32768", nb);
@@ -411,16 +433,22 @@ bsa_status bsa_block_scores_topk(const float* q_pooled, const float* k_pooled, f
   if (!aligned16(q_pooled) || !aligned16(k_pooled) || !aligned16(idx) || !aligned16(scores))
     return fail(BSA_ERR_MISALIGNED, "q_pooled, k_pooled, idx or scores");
   if ((s = check_device()) != BSA_OK) return s;
-  if ((s = launch_select(q_pooled, k_pooled, scores, idx, B, H, nb, D, k,
+  if ((s = launch_select(q_pooled, k_pooled, scores, idx, B, H, nb, D, k, flags,
                          static_cast<cudaStream_t>(stream))) != BSA_OK)
     return s;
   return ok();
 }
 
-bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx,
-                               void* o, int B, int N, int H, int D, int block_size, int kk,
-                               float scale, bsa_dtype dt, void* stream) {
+bsa_status bsa_block_scores_topk(const float* q_pooled, const float* k_pooled, float* scores,
+                                 int32_t* idx, int B, int H, int nb, int D, int k, void* stream) {
+  return bsa_block_scores_topk_ex(q_pooled, k_pooled, scores, idx, B, H, nb, D, k, 0u, stream);
+}
+
+bsa_status bsa_sparse_attn_fwd_ex(const void* q, const void* k, const void* v, const int32_t* idx,
+                                  void* o, int B, int N, int H, int D, int block_size, int kk,
+                                  float scale, bsa_dtype dt, unsigned flags, void* stream) {
   bsa_status s;
+  if ((s = check_flags(flags)) != BSA_OK) return s;
   if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
   if ((s = check_dtype(dt)) != BSA_OK) return s;
   const int nb = N / block_size;
@@ -431,16 +459,23 @@ bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const void* v, cons
     return fail(BSA_ERR_MISALIGNED, "q, k, v, idx or o");
   if (o == q || o == k || o == v) return fail(BSA_ERR_INVALID_ARG, "o aliases an input");
   if ((s = check_device()) != BSA_OK) return s;
-  if ((s = launch_attn(q, k, v, idx, o, B, N, H, D, block_size, kk, scale, dt,
+  if ((s = launch_attn(q, k, v, idx, o, B, N, H, D, block_size, kk, scale, dt, flags,
                        static_cast<cudaStream_t>(stream))) != BSA_OK)
     return s;
   return ok();
 }
 
-bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int B, int N, int H,
-                       int D, int block_size, double topk_ratio, bsa_dtype dt, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx,
+                               void* o, int B, int N, int H, int D, int block_size, int kk,
+                               float scale, bsa_dtype dt, void* stream) {
+  return bsa_sparse_attn_fwd_ex(q, k, v, idx, o, B, N, H, D, block_size, kk, scale, dt, 0u, stream);
+}
+
+bsa_status bsa_forward_ex(const void* q, const void* k, const void* v, void* o, int B, int N,
+                          int H, int D, int block_size, double topk_ratio, bsa_dtype dt,
+                          unsigned flags, void* workspace, size_t workspace_bytes, void* stream) {
   bsa_status s;
+  if ((s = check_flags(flags)) != BSA_OK) return s;
   if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
   if ((s = check_dtype(dt)) != BSA_OK) return s;
   const int nb = N / block_size;
@@ -462,9 +497,17 @@ bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   if ((s = launch_pool(q, w.qp, k, w.kp, 2, B, N, H, D, block_size, dt, st)) != BSA_OK) return s;
-  if ((s = launch_select(w.qp, w.kp, w.scores, w.idx, B, H, nb, D, kk, st)) != BSA_OK) return s;
-  if ((s = launch_attn(q, k, v, w.idx, o, B, N, H, D, block_size, kk, scale, dt, st)) != BSA_OK) return s;
+  if ((s = launch_select(w.qp, w.kp, w.scores, w.idx, B, H, nb, D, kk, flags, st)) != BSA_OK) return s;
+  if ((s = launch_attn(q, k, v, w.idx, o, B, N, H, D, block_size, kk, scale, dt, flags, st)) != BSA_OK)
+    return s;
   return ok();
+}
+
+bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int B, int N, int H,
+                       int D, int block_size, double topk_ratio, bsa_dtype dt, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return bsa_forward_ex(q, k, v, o, B, N, H, D, block_size, topk_ratio, dt, 0u, workspace,
+                        workspace_bytes, stream);
 }
 
 bsa_status bsa_device_error(int* code_out, void* stream) {

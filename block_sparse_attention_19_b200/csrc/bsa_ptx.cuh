@@ -18,6 +18,27 @@ __device__ __forceinline__ void report_error(int code) { atomicCAS(&g_device_err
 
 // A bounded wait gives up after this many polls; each poll may suspend the
 // thread for up to kSuspendNs, so a stuck wait ends within about a second.
+// Variant flags passed down from the entry points (same values as the
+// BSA_FLAG_* macros of the public header).
+constexpr unsigned kFlagCausal = 1u, kFlagForceDiag = 2u;
+
+// Number of leading entries >= 0 of an index row of k entries (a row lists
+// its blocks in ascending order, then pads with -1): binary search.
+__device__ __forceinline__ int index_row_valid(const int32_t* sel, int k) {
+  // a full row (the common case) costs one load; the search's loads are
+  // dependent, each a full memory latency, and the CTA waits for them
+  if (k < 1 || __ldg(sel + k - 1) >= 0) return k;
+  int lo = 0, hi = k - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi) / 2;
+    if (__ldg(sel + mid) >= 0)
+      lo = mid + 1;
+    else
+      hi = mid;
+  }
+  return lo;
+}
+
 constexpr uint32_t kMaxPolls = 1u << 20;
 constexpr uint32_t kSuspendNs = 1000;
 

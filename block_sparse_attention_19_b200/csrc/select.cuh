@@ -17,6 +17,8 @@
 
 #include <stdint.h>
 
+#include "bsa_ptx.cuh"
+
 namespace bsa {
 
 constexpr int kSelThreads = 256;
@@ -90,24 +92,24 @@ __device__ __forceinline__ uint32_t score_key(float f) {
 // that cannot be split holds equal keys only. `cand` is 64 words of shared
 // memory private to the warp.
 template <int KPL>
-__device__ __forceinline__ void select_row_bracket(const float* srow, int nb, int k, int32_t* out,
-                                                   int lane, uint32_t* cand, bool vec) {
+__device__ __forceinline__ void select_row_bracket(const float* srow, int nb, int nvalid, int k,
+                                                   int32_t* out, int lane, uint32_t* cand, bool vec) {
   uint32_t key[KPL];
   const int j0 = lane * KPL;
   if (KPL % 4 == 0 && vec) {
 #pragma unroll
     for (int v = 0; v < KPL / 4; ++v) {
       float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-      const bool in = j0 + 4 * v < nb;  // nb % 4 == 0: the whole float4 is in the row
-      if (in) f = __ldg(reinterpret_cast<const float4*>(srow + j0) + v);
-      key[4 * v] = in ? score_key(f.x) : 0u;
-      key[4 * v + 1] = in ? score_key(f.y) : 0u;
-      key[4 * v + 2] = in ? score_key(f.z) : 0u;
-      key[4 * v + 3] = in ? score_key(f.w) : 0u;
+      const int j = j0 + 4 * v;
+      if (j < nb) f = __ldg(reinterpret_cast<const float4*>(srow + j0) + v);  // nb % 4 == 0
+      key[4 * v] = j < nvalid ? score_key(f.x) : 0u;
+      key[4 * v + 1] = j + 1 < nvalid ? score_key(f.y) : 0u;
+      key[4 * v + 2] = j + 2 < nvalid ? score_key(f.z) : 0u;
+      key[4 * v + 3] = j + 3 < nvalid ? score_key(f.w) : 0u;
     }
   } else {
 #pragma unroll
-    for (int t = 0; t < KPL; ++t) key[t] = j0 + t < nb ? score_key(__ldg(srow + j0 + t)) : 0u;
+    for (int t = 0; t < KPL; ++t) key[t] = j0 + t < nvalid ? score_key(__ldg(srow + j0 + t)) : 0u;
   }
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll
@@ -120,7 +122,7 @@ __device__ __forceinline__ void select_row_bracket(const float* srow, int nb, in
   // invariant: count(key >= lo) = clo >= k > chi = count(key >= hi); hi may be 2^32
   uint32_t lo = kmin;
   uint64_t hi = static_cast<uint64_t>(kmax) + 1;
-  int clo = nb, chi = 0;
+  int clo = nvalid, chi = 0;
 #pragma unroll 1
   for (int it = 0; it < 64 && clo - chi > 64 && hi - lo > 1; ++it) {
     const float flo = key_float(lo), fhi = key_float(static_cast<uint32_t>(hi - 1));
@@ -262,9 +264,12 @@ __device__ __forceinline__ void select_row_smem(const float* srow, int nb, int k
 
 // grid.x = ceil(rows / kSelWarps); one warp per row of S ([rows, nb]).
 // Dynamic shared memory: kSelWarps * nb floats when nb > 1024 and stage_rows, else none.
+// flags: with kFlagCausal, row r is query block i = r % nb: only key blocks
+// j <= i are ranked and min(k, i + 1) are kept (with kFlagForceDiag block i
+// always, plus the best j < i), then the row is padded with -1.
 __global__ void __launch_bounds__(kSelThreads, 4)
     block_topk_kernel(const float* __restrict__ S, int32_t* __restrict__ idx, long rows, int nb,
-                      int k, int stage_rows) {
+                      int k, int stage_rows, unsigned flags) {
   extern __shared__ __align__(16) float sel_rows[];
   __shared__ uint32_t cand[kSelWarps][64];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -273,18 +278,30 @@ __global__ void __launch_bounds__(kSelThreads, 4)
   const float* srow = S + r * nb;
   int32_t* out = idx + r * static_cast<long>(k);
   const bool vec = (nb & 3) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0;
+  // candidates are the key blocks [0, ncand); ksel of them are ranked in
+  int ncand = nb, ksel = k;
+  if (flags & kFlagCausal) {
+    const int i = static_cast<int>(r % nb);
+    const bool force = (flags & kFlagForceDiag) != 0;
+    const int n = min(k, i + 1);
+    ncand = force ? i : i + 1;
+    ksel = force ? n - 1 : n;
+    if (force && lane == 0) out[ksel] = i;  // above every ranked id: the list stays ascending
+    for (int t = n + lane; t < k; t += 32) out[t] = -1;
+    if (ksel == 0) return;
+  }
   if (nb <= 32)
-    select_row_bracket<1>(srow, nb, k, out, lane, cand[warp], vec);
+    select_row_bracket<1>(srow, nb, ncand, ksel, out, lane, cand[warp], vec);
   else if (nb <= 64)
-    select_row_bracket<2>(srow, nb, k, out, lane, cand[warp], vec);
+    select_row_bracket<2>(srow, nb, ncand, ksel, out, lane, cand[warp], vec);
   else if (nb <= 128)
-    select_row_bracket<4>(srow, nb, k, out, lane, cand[warp], vec);
+    select_row_bracket<4>(srow, nb, ncand, ksel, out, lane, cand[warp], vec);
   else if (nb <= 256)
-    select_row_bracket<8>(srow, nb, k, out, lane, cand[warp], vec);
+    select_row_bracket<8>(srow, nb, ncand, ksel, out, lane, cand[warp], vec);
   else if (nb <= 512)
-    select_row_bracket<16>(srow, nb, k, out, lane, cand[warp], vec);
+    select_row_bracket<16>(srow, nb, ncand, ksel, out, lane, cand[warp], vec);
   else if (nb <= 1024)
-    select_row_bracket<32>(srow, nb, k, out, lane, cand[warp], vec);
+    select_row_bracket<32>(srow, nb, ncand, ksel, out, lane, cand[warp], vec);
   else if (stage_rows) {
     // the row is re-read once per key bit: stage it in shared memory
     float* row = sel_rows + static_cast<long>(warp) * nb;
@@ -295,9 +312,9 @@ __global__ void __launch_bounds__(kSelThreads, 4)
       for (int j = lane; j < nb; j += 32) row[j] = __ldg(srow + j);
     }
     __syncwarp();
-    select_row_smem(row, nb, k, out, lane);
+    select_row_smem(row, ncand, ksel, out, lane);
   } else {
-    select_row_smem(srow, nb, k, out, lane);  // rows too long to stage: read them from L2
+    select_row_smem(srow, ncand, ksel, out, lane);  // rows too long to stage: read them from L2
   }
 }
 

@@ -96,8 +96,9 @@ bsa_status bsa_block_scores_topk(const float* q_pooled, const float* k_pooled, f
  *   o[b, n, h, :] = sum_t softmax_t(scale * q[b,n,h,:] . k[b,t,h,:]) v[b,t,h,:]
  * over the tokens t of the key blocks idx[b, h, i, 0..topk).
  * q, k, v: [B, N, H, D] of dtype dt (read). idx: [B, H, nb, topk] int32 with
- * entries in [0, nb) and each row strictly ascending (read; entries outside
- * [0, nb) are clamped by the kernel). o: [B, N, H, D] of dtype dt (written);
+ * entries in [0, nb) and each row strictly ascending (read; a negative entry
+ * ends its row, as in bsa_sparse_attn_fwd_ex, and entries >= nb are clamped
+ * by the kernel). o: [B, N, H, D] of dtype dt (written);
  * o must not alias q, k or v. scale: softmax scale (> 0, finite). */
 bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx,
                                void* o, int B, int N, int H, int D, int block_size, int topk,
@@ -112,6 +113,45 @@ bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const void* v, cons
 bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int B, int N, int H,
                        int D, int block_size, double topk_ratio, bsa_dtype dt, void* workspace,
                        size_t workspace_bytes, void* stream);
+
+/* ---- Variants (flags of the _ex entry points) -------------------------
+ * The base entry points above are the _ex ones with flags = 0.
+ *
+ * BSA_FLAG_CAUSAL: the causal variant. Page "从M2.7到M3：多模态模型稀疏注意力
+ *   架构设计与实现全解析" §2.1 writes the attention as
+ *   Softmax(Mask(QK^T/sqrt(d_k)))V; with a causal mask the readings are:
+ *   - selection: query block i ranks only key blocks j <= i and keeps
+ *     n_i = min(topk, i + 1) of them; its index row lists them ascending and
+ *     pads the remaining topk - n_i entries with -1;
+ *   - attention: query token n never sees key token t > n (so, of the kept
+ *     blocks, only the diagonal block i is masked token by token).
+ * BSA_FLAG_FORCE_DIAG (with BSA_FLAG_CAUSAL): block i is always kept and the
+ *   other n_i - 1 are the highest-scoring blocks j < i.
+ * Other bits are reserved and rejected (BSA_ERR_INVALID_ARG). */
+#define BSA_FLAG_CAUSAL 1u
+#define BSA_FLAG_FORCE_DIAG 2u
+
+/* bsa_block_scores_topk with variant flags (see above). With
+ * BSA_FLAG_CAUSAL, scores is still written in full (all nb x nb entries). */
+bsa_status bsa_block_scores_topk_ex(const float* q_pooled, const float* k_pooled, float* scores,
+                                    int32_t* idx, int B, int H, int nb, int D, int topk,
+                                    unsigned flags, void* stream);
+
+/* bsa_sparse_attn_fwd with variant flags. idx rows may end in -1 entries
+ * (rows as bsa_block_scores_topk_ex writes them): a row's valid entries are
+ * its leading entries >= 0, which must be strictly ascending, and a row needs
+ * at least one (a row of only -1 reads block 0). With BSA_FLAG_CAUSAL, key
+ * token t is left out of the softmax of query token n when t > n; the caller
+ * is responsible for keeping blocks j <= i (the kernel masks tokens, it does
+ * not check the list). */
+bsa_status bsa_sparse_attn_fwd_ex(const void* q, const void* k, const void* v, const int32_t* idx,
+                                  void* o, int B, int N, int H, int D, int block_size, int topk,
+                                  float scale, bsa_dtype dt, unsigned flags, void* stream);
+
+/* bsa_forward with variant flags; same workspace. */
+bsa_status bsa_forward_ex(const void* q, const void* k, const void* v, void* o, int B, int N,
+                          int H, int D, int block_size, double topk_ratio, bsa_dtype dt,
+                          unsigned flags, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Size of the fixed device scratch that bsa_forward_noalloc uses: 64 MiB. */
 #define BSA_NOALLOC_SCRATCH_BYTES (64u << 20)

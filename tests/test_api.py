@@ -117,3 +117,20 @@ def test_binding_fails_loudly_without_library(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import block_sparse_attention_19_b200"], cwd=tmp_path,
                        capture_output=True, text=True)
     assert r.returncode != 0 and "libbsa.so is not built" in r.stderr
+
+
+def test_ex_entry_points_reject_bad_flags(bsa):
+    """Flag validation happens on the host before any device work."""
+    bsa_lib = bsa.lib
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    # unknown bit
+    st = bsa_lib.bsa_forward_ex(fake, fake, fake, P(0x20000), 1, 1024, 2, 64, 64, 0.25, 1, 4, fake,
+                                1 << 30, P(0))
+    assert st == 1 and b"flag" in bsa_lib.bsa_last_error_detail()
+    # forcing the diagonal block only makes sense with the causal flag
+    st = bsa_lib.bsa_sparse_attn_fwd_ex(fake, fake, fake, fake, P(0x20000), 1, 1024, 2, 64, 64, 4,
+                                        0.125, 1, 2, P(0))
+    assert st == 1 and b"CAUSAL" in bsa_lib.bsa_last_error_detail()
+    st = bsa_lib.bsa_block_scores_topk_ex(fake, fake, fake, fake, 1, 2, 16, 64, 4, 8, P(0))
+    assert st == 1
