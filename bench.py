@@ -112,7 +112,8 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- oracle (CPU) timing
 
-def oracle_sample(q, k, v, cfg: W.Config, heads, blocks_per_head: int, seed: int):
+def oracle_sample(q, k, v, cfg: W.Config, heads, blocks_per_head: int, seed: int, causal=False,
+                  force_diag=False):
     """Runs the oracle's whole path for `blocks_per_head` random query blocks of
     each head in `heads` (each head is an independent single-head problem) and
     returns (query tokens, seconds, threads)."""
@@ -125,7 +126,8 @@ def oracle_sample(q, k, v, cfg: W.Config, heads, blocks_per_head: int, seed: int
         qa, ka, va = (np.ascontiguousarray(W.to_oracle_array(x[:, :, h:h + 1])) for x in (q, k, v))
         rows = np.sort(rng.choice(cfg.nb, size=(1, 1, blocks_per_head), replace=False), axis=-1).astype(np.int32)
         t0 = time.perf_counter()
-        oracle.forward(qa, ka, va, cfg.block_size, cfg.topk_ratio, rows=rows)
+        oracle.forward(qa, ka, va, cfg.block_size, cfg.topk_ratio, rows=rows, causal=causal,
+                       force_diag=force_diag)
         secs += time.perf_counter() - t0
         tokens += blocks_per_head * cfg.block_size * cfg.B
     return tokens, secs, oracle.num_threads()
@@ -168,12 +170,18 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-blocks-per-head", type=int, default=8)
+    ap.add_argument("--causal", action="store_true",
+                    help="the causal variant (BSA_FLAG_CAUSAL): block-causal selection, token-causal attention")
+    ap.add_argument("--force-diag", action="store_true",
+                    help="with --causal: always keep the diagonal block (BSA_FLAG_FORCE_DIAG)")
     ap.add_argument("--stages-only", action="store_true",
                     help="time the stage-by-stage steps only (no fused, end-to-end or CPU legs); "
                          "for profiler runs")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.force_diag and not args.causal:
+        ap.error("--force-diag needs --causal")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -198,6 +206,9 @@ def main():
 
     import block_sparse_attention_19_b200 as bsa
 
+    flags = (bsa.BSA_FLAG_CAUSAL if args.causal else 0) | (bsa.BSA_FLAG_FORCE_DIAG if args.force_diag else 0)
+    variant = (" causal" + (" force_diag" if args.force_diag else "")) if args.causal else ""
+
     B, N, H, D, bs, ratio = cfg.B, cfg.N, cfg.H, cfg.D, cfg.block_size, cfg.topk_ratio
     kk = bsa.bsa_topk_count(N // bs, ratio)
     q, k, v = W.make_inputs(cfg, device=dev)
@@ -212,10 +223,10 @@ def main():
         bsa.bsa_block_pool(k, bs, out=kp)
         if ev is not None:
             ev[1].record()
-        bsa.bsa_block_scores_topk(qp, kp, kk, idx_out=idx, scores_out=S)
+        bsa.bsa_block_scores_topk(qp, kp, kk, idx_out=idx, scores_out=S, flags=flags)
         if ev is not None:
             ev[2].record()
-        bsa.bsa_sparse_attn_fwd(q, k, v, idx, bs, out=o)
+        bsa.bsa_sparse_attn_fwd(q, k, v, idx, bs, out=o, flags=flags)
         if ev is not None:
             ev[3].record()
 
@@ -268,7 +279,7 @@ def main():
     nf = max(3, args.steps // 4)
     f0.record()
     for _ in range(nf):
-        bsa.bsa_forward(q, k, v, bs, ratio, workspace=ws, out=o)
+        bsa.bsa_forward(q, k, v, bs, ratio, workspace=ws, out=o, flags=flags)
     f1.record()
     torch.cuda.synchronize()
     fused_ms = f0.elapsed_time(f1) / nf
@@ -279,7 +290,7 @@ def main():
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     for _ in range(2):
         dq.copy_(hq, non_blocking=True); dk.copy_(hk, non_blocking=True); dv.copy_(hv, non_blocking=True)
-        bsa.bsa_forward(dq, dk, dv, bs, ratio, workspace=ws, out=o)
+        bsa.bsa_forward(dq, dk, dv, bs, ratio, workspace=ws, out=o, flags=flags)
         ho.copy_(o, non_blocking=True)
     torch.cuda.synchronize()
     if dist:
@@ -288,7 +299,7 @@ def main():
     e0.record()
     for _ in range(args.e2e_steps):
         dq.copy_(hq, non_blocking=True); dk.copy_(hk, non_blocking=True); dv.copy_(hv, non_blocking=True)
-        bsa.bsa_forward(dq, dk, dv, bs, ratio, workspace=ws, out=o)
+        bsa.bsa_forward(dq, dk, dv, bs, ratio, workspace=ws, out=o, flags=flags)
         ho.copy_(o, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
@@ -305,6 +316,13 @@ def main():
     value = world * tokens_step * args.steps / (total_ms / 1e3)
     e2e_value = world * tokens_step * args.e2e_steps / (e2e_ms / 1e3)
     flops = 4.0 * B * H * N * kk * bs * D
+    if args.causal:
+        # visible (query, key) token pairs of the lists the step produced:
+        # bs^2 per kept block below the diagonal, bs(bs+1)/2 for the diagonal
+        il = idx.cpu().numpy().astype(np.int64)
+        qi = np.arange(N // bs)[None, None, :, None]
+        pairs = np.where(il < 0, 0, np.where(il < qi, bs * bs, bs * (bs + 1) // 2)).sum()
+        flops = 4.0 * D * float(pairs)
     esz = cfg.elem_bytes
     tensor_bytes = B * N * H * D * esz
     idx_bytes = B * H * (N // bs) * kk * 4
@@ -318,7 +336,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-        "config": {"workload": f"{cfg.name}: {cfg.describe()}", "seed": cfg.seed,
+        "config": {"workload": f"{cfg.name}{variant}: {cfg.describe()}", "seed": cfg.seed,
                    "l2": f"inputs larger than L2 (q, k, v {tensor_bytes / 1e6:.0f} MB each)",
                    "parallelism": f"replica per GPU x{world}"},
         "tflops_effective": flops / (step_ms / 1e3) / 1e12,
@@ -336,7 +354,7 @@ def main():
             "kernel": "sparse_attn_tc2_kernel" if bs in (128, 256) else "sparse_attn_tc_kernel",
             "bound": "tensor", "achieved": achieved,
             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-            "peak_source": f"{peak_src} bf16 burst", "traffic": NCU_TRAFFIC.get(cfg.name),
+            "peak_source": f"{peak_src} bf16 burst", "traffic": None if args.causal else NCU_TRAFFIC.get(cfg.name),
             "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
             "frac_of_roofline_time": roof_t / (attn_ms / 1e3),
             "flops_per_launch": flops, "algorithmic_bytes_per_launch": alg_bytes,
@@ -353,7 +371,8 @@ def main():
         heads = list(range(cfg.H))
         qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
         bpe = min(args.cpu_blocks_per_head, cfg.nb)
-        tok, sec, thr = oracle_sample(qc, kc, vc, cfg, heads, bpe, seed=cfg.seed + 2000)
+        tok, sec, thr = oracle_sample(qc, kc, vc, cfg, heads, bpe, seed=cfg.seed + 2000,
+                                      causal=args.causal, force_diag=args.force_diag)
         line["cpu_baseline"] = {"value": tok / sec, "unit": "tokens/s", "cores": thr, "kind": "oracle",
                                 "sample": f"{bpe} random query blocks on each of {len(heads)} heads "
                                           f"({tok} query tokens, {sec:.1f} s), whole oracle path per head "
