@@ -68,6 +68,7 @@ def _load():
         lib.oracle_sparse_attn.argtypes = [P, P, P, i, i, i, i, i, i, P, i, P, i, d, P]
         lib.oracle_topk_ex.argtypes = [P, ctypes.c_long, i, i, P, i, P]
         lib.oracle_sparse_attn_ex.argtypes = [P, P, P, i, i, i, i, i, i, P, i, P, i, d, i, P]
+        lib.oracle_sparse_attn_gqa.argtypes = [P, P, P, i, i, i, i, i, i, i, P, i, P, i, d, i, P]
         lib.oracle_num_threads.restype = i
         _lib = lib
     return _lib
@@ -210,6 +211,79 @@ def forward(q, k, v, block_size: int, topk_ratio: float, rows=None, scale=None,
     o = sparse_attn(q, k, v, idx, block_size, scale=scale, rows=rows, causal=causal)
     return {"qp": qp, "kp": kp, "scores": S, "idx": idx, "o": o, "k": kk,
             "seconds": time.perf_counter() - t0}
+
+
+# ---------------------------------------------------------------- grouped-query variant
+# Readings ("从M2.7到M3" §3.1: the attention block is GQA-based): q has H heads,
+# k and v have Hkv = H / G; query head h reads key/value head h // G; each
+# key/value head has one selection, scored with the group's pooled query (the
+# mean over its G heads of their block means).
+
+def group_pool(qp: np.ndarray, Hkv: int) -> np.ndarray:
+    """Pooled queries [B,H,nb,D] -> the group means [B,Hkv,nb,D] (heads h with h // G == g)."""
+    B, H, nb, D = qp.shape
+    if H % Hkv:
+        raise ValueError("H must be a multiple of Hkv")
+    return np.asarray(qp, np.float64).reshape(B, Hkv, H // Hkv, nb, D).mean(axis=2)
+
+
+def sparse_attn_gqa(q, k, v, idx, block_size: int, scale: float | None = None, rows=None,
+                    causal: bool = False) -> np.ndarray:
+    """sparse_attn with Hkv key/value heads: q [B,N,H,D], k and v [B,N,Hkv,D];
+    ``idx`` [B,H,nrows,k] and ``rows`` [B,H,nrows] are per query head.
+    Returns float64 [B,H,nrows,block_size,D]."""
+    q, code = _as_input(q)
+    k_, code_k = _as_input(k)
+    v, code_v = _as_input(v)
+    if not (code == code_k == code_v):
+        raise TypeError("q, k, v must share one dtype")
+    B, N, H, D = q.shape
+    Hkv = k_.shape[2]
+    if H % Hkv or k_.shape != (B, N, Hkv, D) or v.shape != k_.shape:
+        raise ValueError("need k, v of shape [B,N,Hkv,D] with H a multiple of Hkv")
+    nb = N // block_size
+    idx = np.ascontiguousarray(idx, np.int32)
+    kk = idx.shape[-1]
+    if rows is None:
+        nrows, rp = nb, None
+    else:
+        rows = np.ascontiguousarray(rows, np.int32)
+        nrows, rp = rows.shape[-1], _ptr(rows)
+    if idx.shape != (B, H, nrows, kk):
+        raise ValueError(f"idx shape {idx.shape} != {(B, H, nrows, kk)}")
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    out = np.empty((B, H, nrows, block_size, D), np.float64)
+    _load().oracle_sparse_attn_gqa(_ptr(q), _ptr(k_), _ptr(v), code, B, N, H, Hkv, D, block_size,
+                                   _ptr(idx), kk, rp, nrows, float(scale), CAUSAL if causal else 0,
+                                   _ptr(out))
+    return out
+
+
+def forward_gqa(q, k, v, block_size: int, topk_ratio: float, rows=None, scale=None,
+                causal: bool = False, force_diag: bool = False) -> dict:
+    """The whole path with grouped queries. ``rows`` (int [B,Hkv,nrows]) picks
+    query blocks per key/value head; every query head of the group is attended
+    for those blocks. Returns qp (per head), qg (group means), kp, scores and
+    idx (per key/value head), idx_q / rows_q (expanded to query heads) and o
+    [B,H,nrows,bs,D]."""
+    qn, _ = _as_input(q)
+    kn, _ = _as_input(k)
+    B, N, H, D = qn.shape
+    Hkv = kn.shape[2]
+    G = H // Hkv
+    nb = N // block_size
+    kk = topk_count(nb, topk_ratio)
+    qp = block_pool(q, block_size)
+    qg = group_pool(qp, Hkv)
+    kp = block_pool(k, block_size)
+    S = block_scores(qg, kp, rows)
+    idx = topk(S, kk, causal=causal, force_diag=force_diag, qblocks=rows)
+    idx_q = np.repeat(idx, G, axis=1)
+    rows_q = None if rows is None else np.repeat(np.asarray(rows, np.int32), G, axis=1)
+    o = sparse_attn_gqa(q, k, v, idx_q, block_size, scale=scale, rows=rows_q, causal=causal)
+    return {"qp": qp, "qg": qg, "kp": kp, "scores": S, "idx": idx, "idx_q": idx_q, "rows_q": rows_q,
+            "o": o, "k": kk}
 
 
 def o_to_bnhd(o: np.ndarray) -> np.ndarray:

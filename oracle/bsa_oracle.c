@@ -313,3 +313,68 @@ void oracle_sparse_attn_ex(const void* q, const void* kmat, const void* v, int d
     free(qrow);
   }
 }
+
+/* ------------------------------------------------------------------------
+ * Grouped-query variant ([MSA] §3.1: the attention block is GQA-based).
+ * Readings (listed in the design notes as well): q has H heads and k, v have
+ * Hkv heads, H = G * Hkv; query head h reads key/value head h / G. One block
+ * selection serves each key/value head: it is scored with the group's pooled
+ * query (the mean over the group's G heads of their block means), which by
+ * linearity is the mean of the G heads' block scores.
+ * ------------------------------------------------------------------------ */
+
+/* oracle_sparse_attn_ex with Hkv key/value heads: q and o have H heads, k and
+ * v have Hkv; idx and rows are per query head ([B, H, nrows, k], [B, H, nrows]). */
+void oracle_sparse_attn_gqa(const void* q, const void* kmat, const void* v, int dtype, int B, int N,
+                            int H, int Hkv, int D, int bs, const int* idx, int k, const int* rows,
+                            int nrows, double scale, int flags, double* o) {
+  long ntok = (long)k * bs;
+  int G = H / Hkv;
+#pragma omp parallel
+  {
+    double* logit = (double*)malloc((size_t)ntok * sizeof(double));
+    double* qrow = (double*)malloc((size_t)D * sizeof(double));
+#pragma omp for collapse(4) schedule(dynamic, 4)
+    for (int b = 0; b < B; ++b)
+      for (int h = 0; h < H; ++h)
+        for (int r = 0; r < nrows; ++r)
+          for (int t_q = 0; t_q < bs; ++t_q) {
+            size_t bh = (size_t)b * H + h;
+            int g = h / G;
+            int i = rows ? rows[bh * nrows + r] : r;
+            const int* sel = idx + (bh * nrows + r) * k;
+            int n = i * bs + t_q;
+            for (int d = 0; d < D; ++d) qrow[d] = elem(q, dtype, at_bnhd(N, H, D, b, n, h, d));
+            double m = -INFINITY;
+            for (int s = 0; s < k; ++s)
+              for (int u = 0; u < bs; ++u) {
+                double l = -INFINITY; /* masked or unselected */
+                if (sel[s] >= 0) {
+                  int t = sel[s] * bs + u;
+                  if (!(flags & ORACLE_CAUSAL) || t <= n) {
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += qrow[d] * elem(kmat, dtype, at_bnhd(N, Hkv, D, b, t, g, d));
+                    l = scale * dot;
+                  }
+                }
+                logit[(long)s * bs + u] = l;
+                if (l > m) m = l;
+              }
+            double* out = o + ((bh * nrows + r) * bs + t_q) * D;
+            for (int d = 0; d < D; ++d) out[d] = 0.0;
+            double z = 0.0;
+            for (int s = 0; s < k; ++s)
+              for (int u = 0; u < bs; ++u) {
+                double l = logit[(long)s * bs + u];
+                if (l == -INFINITY) continue;
+                int t = sel[s] * bs + u;
+                double w = exp(l - m);
+                z += w;
+                for (int d = 0; d < D; ++d) out[d] += w * elem(v, dtype, at_bnhd(N, Hkv, D, b, t, g, d));
+              }
+            for (int d = 0; d < D; ++d) out[d] /= z;
+          }
+    free(logit);
+    free(qrow);
+  }
+}

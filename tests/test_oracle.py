@@ -422,3 +422,75 @@ def test_minus_one_entries_select_nothing(oracle_mod, small_case):
     r = oracle_mod.forward(q, k, v, bs, ratio)
     pad = np.concatenate([r["idx"], np.full(r["idx"].shape[:-1] + (2,), -1, np.int32)], -1)
     np.testing.assert_array_equal(oracle_mod.sparse_attn(q, k, v, pad, bs), r["o"])
+
+
+# ---------------------------------------------------------------- grouped-query variant
+# Readings: q has H heads, k and v Hkv = H / G; query head h reads key/value
+# head h // G; one selection per key/value head, scored with the group's pooled
+# query (mean of its heads' block means).
+
+def _repeat_kv(x, G):
+    return np.repeat(x, G, axis=2)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_ratio_one_equals_sdpa_with_repeated_kv(oracle_mod, causal):
+    B, N, H, Hkv, D, bs = 2, 64, 6, 2, 16, 8
+    q = _rand((B, N, H, D), 110, bs=bs)
+    k, v = (_rand((B, N, Hkv, D), s, bs=bs) for s in (111, 112))
+    r = oracle_mod.forward_gqa(q, k, v, bs, 1.0, causal=causal)
+    t = lambda x: torch.from_numpy(x).permute(0, 2, 1, 3)
+    ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(_repeat_kv(k, H // Hkv)),
+                                                           t(_repeat_kv(v, H // Hkv)), is_causal=causal)
+    np.testing.assert_allclose(oracle_mod.o_to_bnhd(r["o"]), ref.permute(0, 2, 1, 3).numpy(),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_gqa_group_score_is_mean_of_head_scores(oracle_mod):
+    """By linearity the group score q̄_g . k̄_j equals the mean over the group's
+    heads of q̄_h . k̄_j, computed here with numpy per head."""
+    B, N, H, Hkv, D, bs = 1, 96, 8, 2, 16, 8
+    q = _rand((B, N, H, D), 120, bs=bs)
+    k, v = (_rand((B, N, Hkv, D), s, bs=bs) for s in (121, 122))
+    r = oracle_mod.forward_gqa(q, k, v, bs, 0.25)
+    qp = q.reshape(B, N // bs, bs, H, D).mean(2).transpose(0, 2, 1, 3)  # [B,H,nb,D]
+    kp = k.reshape(B, N // bs, bs, Hkv, D).mean(2).transpose(0, 2, 1, 3)
+    G = H // Hkv
+    per_head = np.stack([qp[:, h] @ kp[:, h // G].transpose(0, 2, 1) for h in range(H)], 1)
+    want = per_head.reshape(B, Hkv, G, N // bs, N // bs).mean(2)
+    np.testing.assert_allclose(r["scores"], want, rtol=1e-12, atol=1e-12)
+
+
+def test_gqa_attention_equals_per_head_attention_on_repeated_kv(oracle_mod):
+    B, N, H, Hkv, D, bs, kk = 1, 48, 4, 2, 8, 6, 3
+    nb = N // bs
+    q = _rand((B, N, H, D), 130, bs=bs)
+    k, v = (_rand((B, N, Hkv, D), s, bs=bs) for s in (131, 132))
+    rng = np.random.default_rng(133)
+    idx = np.sort(np.stack([[[rng.choice(nb, kk, replace=False) for _ in range(nb)]
+                             for _ in range(H)]]), axis=-1).astype(np.int32)
+    for causal in (False, True):
+        got = oracle_mod.sparse_attn_gqa(q, k, v, idx, bs, causal=causal)
+        want = oracle_mod.sparse_attn(q, _repeat_kv(k, H // Hkv), _repeat_kv(v, H // Hkv), idx, bs,
+                                      causal=causal)
+        np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-13)
+
+
+def test_gqa_head_permutation_within_a_group(oracle_mod):
+    B, N, H, Hkv, D, bs = 1, 64, 6, 2, 8, 8
+    q = _rand((B, N, H, D), 140, bs=bs)
+    k, v = (_rand((B, N, Hkv, D), s, bs=bs) for s in (141, 142))
+    r = oracle_mod.forward_gqa(q, k, v, bs, 0.375)
+    perm = np.array([2, 0, 1, 4, 5, 3])  # within groups {0,1,2} and {3,4,5}
+    r2 = oracle_mod.forward_gqa(q[:, :, perm], k, v, bs, 0.375)
+    np.testing.assert_array_equal(r2["idx"], r["idx"])
+    np.testing.assert_allclose(r2["o"], r["o"][:, perm], rtol=1e-12, atol=1e-12)
+
+
+def test_gqa_with_one_head_per_group_is_the_plain_path(oracle_mod, small_case):
+    q, k, v, bs, ratio = small_case
+    for causal in (False, True):
+        a = oracle_mod.forward(q, k, v, bs, ratio, causal=causal)
+        b = oracle_mod.forward_gqa(q, k, v, bs, ratio, causal=causal)
+        np.testing.assert_array_equal(a["idx"], b["idx"])
+        np.testing.assert_allclose(a["o"], b["o"], rtol=1e-13, atol=1e-13)
