@@ -18,6 +18,7 @@ bounded sample of query blocks per step; rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -115,21 +116,28 @@ class ClockSampler:
 def oracle_sample(q, k, v, cfg: W.Config, heads, blocks_per_head: int, seed: int, causal=False,
                   force_diag=False):
     """Runs the oracle's whole path for `blocks_per_head` random query blocks of
-    each head in `heads` (each head is an independent single-head problem) and
-    returns (query tokens, seconds, threads)."""
+    each key/value head in `heads` (each an independent problem: one head, or
+    with grouped queries one key/value head and its G query heads) and returns
+    (query tokens, seconds, threads)."""
     import oracle
 
     oracle.build()
     rng = np.random.default_rng(seed)
+    G = cfg.H // cfg.Hkv
     tokens, secs = 0, 0.0
-    for h in heads:
-        qa, ka, va = (np.ascontiguousarray(W.to_oracle_array(x[:, :, h:h + 1])) for x in (q, k, v))
+    for g in heads:
+        qa = np.ascontiguousarray(W.to_oracle_array(q[:, :, g * G:(g + 1) * G]))
+        ka, va = (np.ascontiguousarray(W.to_oracle_array(x[:, :, g:g + 1])) for x in (k, v))
         rows = np.sort(rng.choice(cfg.nb, size=(1, 1, blocks_per_head), replace=False), axis=-1).astype(np.int32)
         t0 = time.perf_counter()
-        oracle.forward(qa, ka, va, cfg.block_size, cfg.topk_ratio, rows=rows, causal=causal,
-                       force_diag=force_diag)
+        if G == 1:
+            oracle.forward(qa, ka, va, cfg.block_size, cfg.topk_ratio, rows=rows, causal=causal,
+                           force_diag=force_diag)
+        else:
+            oracle.forward_gqa(qa, ka, va, cfg.block_size, cfg.topk_ratio, rows=rows, causal=causal,
+                               force_diag=force_diag)
         secs += time.perf_counter() - t0
-        tokens += blocks_per_head * cfg.block_size * cfg.B
+        tokens += blocks_per_head * cfg.block_size * cfg.B * G
     return tokens, secs, oracle.num_threads()
 
 
@@ -137,22 +145,25 @@ def run_reference(args, cfg, rank, world):
     if rank != 0:
         return
     q, k, v = W.make_inputs(cfg, device="cpu")
-    heads = list(range(cfg.H))
+    heads = list(range(cfg.Hkv))
+    causal = dict(causal=args.causal, force_diag=args.force_diag)
     for s in range(args.warmup):
-        oracle_sample(q, k, v, cfg, [heads[s % cfg.H]], 1, seed=100 + s)
+        oracle_sample(q, k, v, cfg, [heads[s % cfg.Hkv]], 1, seed=100 + s, **causal)
     tok, sec, thr = 0, 0.0, 1
     for s in range(args.steps):
-        t, dt, thr = oracle_sample(q, k, v, cfg, [heads[s % cfg.H]], 1, seed=1000 + s)
+        t, dt, thr = oracle_sample(q, k, v, cfg, [heads[s % cfg.Hkv]], 1, seed=1000 + s, **causal)
         tok += t
         sec += dt
     value = tok / sec
-    sample = (f"{args.steps} steps x 1 query block ({cfg.block_size * cfg.B} tokens) of one head each, "
-              f"whole oracle path per step incl. pooling that head's k")
+    sample = (f"{args.steps} steps x 1 query block ({cfg.block_size * cfg.B * (cfg.H // cfg.Hkv)} tokens) "
+              f"of one key/value head each, whole oracle path per step incl. pooling that head's k")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": f"{cfg.name}: {cfg.describe()}", "seed": cfg.seed},
+            "config": {"workload": f"{cfg.name}{' causal' if args.causal else ''}"
+                                   f"{' force_diag' if args.force_diag else ''}: {cfg.describe()}",
+                       "seed": cfg.seed},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -174,6 +185,8 @@ def main():
                     help="the causal variant (BSA_FLAG_CAUSAL): block-causal selection, token-causal attention")
     ap.add_argument("--force-diag", action="store_true",
                     help="with --causal: always keep the diagonal block (BSA_FLAG_FORCE_DIAG)")
+    ap.add_argument("--kv-heads", type=int, default=None,
+                    help="grouped queries: the config with this many key/value heads (H a multiple of it)")
     ap.add_argument("--stages-only", action="store_true",
                     help="time the stage-by-stage steps only (no fused, end-to-end or CPU legs); "
                          "for profiler runs")
@@ -187,6 +200,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     cfg = W.CONFIGS[args.config]
+    if args.kv_heads is not None:
+        if args.kv_heads < 1 or cfg.H % args.kv_heads:
+            ap.error(f"--kv-heads must divide H={cfg.H}")
+        cfg = dataclasses.replace(cfg, H_kv=args.kv_heads)
 
     if args.impl == "reference":
         run_reference(args, cfg, rank, world)
@@ -212,8 +229,10 @@ def main():
     B, N, H, D, bs, ratio = cfg.B, cfg.N, cfg.H, cfg.D, cfg.block_size, cfg.topk_ratio
     kk = bsa.bsa_topk_count(N // bs, ratio)
     q, k, v = W.make_inputs(cfg, device=dev)
-    ws = torch.empty(bsa.bsa_forward_workspace_bytes(B, N, H, D, bs, ratio), device=dev, dtype=torch.uint8)
-    qp, kp, idx, S = bsa.workspace_views(ws, B, N, H, D, bs, ratio, with_scores=True)
+    Hk = cfg.Hkv
+    ws = torch.empty(bsa.bsa_forward_workspace_bytes(B, N, H, D, bs, ratio, H_kv=Hk), device=dev,
+                     dtype=torch.uint8)
+    qp, kp, idx, S = bsa.workspace_views(ws, B, N, H, D, bs, ratio, with_scores=True, H_kv=Hk)
     o = torch.empty_like(q)
 
     def step(ev=None):
@@ -322,13 +341,14 @@ def main():
         il = idx.cpu().numpy().astype(np.int64)
         qi = np.arange(N // bs)[None, None, :, None]
         pairs = np.where(il < 0, 0, np.where(il < qi, bs * bs, bs * (bs + 1) // 2)).sum()
-        flops = 4.0 * D * float(pairs)
+        flops = 4.0 * D * float(pairs) * (H // Hk)  # each key/value head's lists serve G query heads
     esz = cfg.elem_bytes
-    tensor_bytes = B * N * H * D * esz
-    idx_bytes = B * H * (N // bs) * kk * 4
-    pooled_bytes = 2 * B * H * (N // bs) * D * 4
-    alg_bytes = 4 * tensor_bytes + idx_bytes  # q, k, v read + o written, and the index list
-    sel_bytes = 2 * tensor_bytes + idx_bytes  # selection stage: q, k read + index list written
+    tensor_bytes = B * N * H * D * esz  # q (and o)
+    kv_bytes = B * N * Hk * D * esz     # k (and v): fewer heads with grouped queries
+    idx_bytes = B * Hk * (N // bs) * kk * 4
+    pooled_bytes = B * (H + Hk) * (N // bs) * D * 4
+    alg_bytes = 2 * tensor_bytes + 2 * kv_bytes + idx_bytes  # q, k, v read + o written, and the index list
+    sel_bytes = tensor_bytes + kv_bytes + idx_bytes  # selection stage: q, k read + index list written
     peaks, peak_src = load_peaks()
     step_ms = total_ms / args.steps
 
@@ -354,7 +374,7 @@ def main():
             "kernel": "sparse_attn_tc2_kernel" if bs in (128, 256) else "sparse_attn_tc_kernel",
             "bound": "tensor", "achieved": achieved,
             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-            "peak_source": f"{peak_src} bf16 burst", "traffic": None if args.causal else NCU_TRAFFIC.get(cfg.name),
+            "peak_source": f"{peak_src} bf16 burst", "traffic": None if (args.causal or Hk != H) else NCU_TRAFFIC.get(cfg.name),
             "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
             "frac_of_roofline_time": roof_t / (attn_ms / 1e3),
             "flops_per_launch": flops, "algorithmic_bytes_per_launch": alg_bytes,
@@ -363,18 +383,18 @@ def main():
         "bytes": sel_bytes, "ms": pool_ms + sel_ms,
         "GB/s": sel_bytes / ((pool_ms + sel_ms) / 1e3) / 1e9,
         "frac_of_hbm": sel_bytes / ((pool_ms + sel_ms) / 1e3) / 1e9 / peaks["hbm_gbs"],
-        "pool_GB/s": (2 * tensor_bytes + pooled_bytes) / (pool_ms / 1e3) / 1e9,
-        "pool_frac_of_hbm": (2 * tensor_bytes + pooled_bytes) / (pool_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "pool_GB/s": (tensor_bytes + kv_bytes + pooled_bytes) / (pool_ms / 1e3) / 1e9,
+        "pool_frac_of_hbm": (tensor_bytes + kv_bytes + pooled_bytes) / (pool_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
         "peak": peaks["hbm_gbs"], "peak_source": f"{peak_src} HBM copy"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        heads = list(range(cfg.H))
+        heads = list(range(cfg.Hkv))
         qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
         bpe = min(args.cpu_blocks_per_head, cfg.nb)
         tok, sec, thr = oracle_sample(qc, kc, vc, cfg, heads, bpe, seed=cfg.seed + 2000,
                                       causal=args.causal, force_diag=args.force_diag)
         line["cpu_baseline"] = {"value": tok / sec, "unit": "tokens/s", "cores": thr, "kind": "oracle",
-                                "sample": f"{bpe} random query blocks on each of {len(heads)} heads "
+                                "sample": f"{bpe} random query blocks on each of {len(heads)} key/value heads "
                                           f"({tok} query tokens, {sec:.1f} s), whole oracle path per head "
                                           f"incl. pooling all of that head's k"}
     if rank == 0:

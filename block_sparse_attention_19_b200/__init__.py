@@ -36,7 +36,9 @@ _STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "
 EXPORTED = ("bsa_topk_count", "bsa_forward_workspace_bytes", "bsa_block_pool",
             "bsa_block_scores_topk", "bsa_sparse_attn_fwd", "bsa_forward", "bsa_status_string",
             "bsa_last_error_detail", "bsa_device_error", "bsa_forward_noalloc",
-            "bsa_block_scores_topk_ex", "bsa_sparse_attn_fwd_ex", "bsa_forward_ex")
+            "bsa_block_scores_topk_ex", "bsa_sparse_attn_fwd_ex", "bsa_forward_ex",
+            "bsa_forward_gqa_workspace_bytes", "bsa_block_scores_topk_gqa", "bsa_sparse_attn_fwd_gqa",
+            "bsa_forward_gqa")
 
 #: variant flags of the *_ex entry points (include/bsa.h)
 BSA_FLAG_CAUSAL, BSA_FLAG_FORCE_DIAG = 1, 2
@@ -69,6 +71,10 @@ def _load() -> ctypes.CDLL:
         "bsa_block_scores_topk_ex": ([P, P, P, P, I, I, I, I, I, U, P], I),
         "bsa_sparse_attn_fwd_ex": ([P, P, P, P, P, I, I, I, I, I, I, F, I, U, P], I),
         "bsa_forward_ex": ([P, P, P, P, I, I, I, I, I, D, I, U, P, Z, P], I),
+        "bsa_forward_gqa_workspace_bytes": ([I, I, I, I, I, I, D], Z),
+        "bsa_block_scores_topk_gqa": ([P, P, P, P, I, I, I, I, I, I, U, P], I),
+        "bsa_sparse_attn_fwd_gqa": ([P, P, P, P, P, I, I, I, I, I, I, I, F, I, U, P], I),
+        "bsa_forward_gqa": ([P, P, P, P, I, I, I, I, I, I, D, I, U, P, Z, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -113,8 +119,11 @@ def bsa_topk_count(nb: int, topk_ratio: float) -> int:
     return lib.bsa_topk_count(int(nb), float(topk_ratio))
 
 
-def bsa_forward_workspace_bytes(B: int, N: int, H: int, D: int, block_size: int, topk_ratio: float) -> int:
-    return lib.bsa_forward_workspace_bytes(B, N, H, D, block_size, float(topk_ratio))
+def bsa_forward_workspace_bytes(B: int, N: int, H: int, D: int, block_size: int, topk_ratio: float,
+                                H_kv: int | None = None) -> int:
+    if H_kv is None or H_kv == H:
+        return lib.bsa_forward_workspace_bytes(B, N, H, D, block_size, float(topk_ratio))
+    return lib.bsa_forward_gqa_workspace_bytes(B, N, H, H_kv, D, block_size, float(topk_ratio))
 
 
 def bsa_block_pool(x: torch.Tensor, block_size: int, out: torch.Tensor | None = None) -> torch.Tensor:
@@ -137,10 +146,14 @@ def bsa_block_scores_topk(q_pooled: torch.Tensor, k_pooled: torch.Tensor, topk: 
     if q_pooled.dtype != torch.float32 or k_pooled.dtype != torch.float32:
         raise TypeError("pooled tensors must be float32")
     B, H, nb, D = q_pooled.shape
-    idx = idx_out if idx_out is not None else torch.empty((B, H, nb, topk), device=q_pooled.device, dtype=torch.int32)
-    S = scores_out if scores_out is not None else torch.empty((B, H, nb, nb), device=q_pooled.device,
+    Hk = k_pooled.shape[1]  # key/value heads: fewer than H for grouped queries
+    idx = idx_out if idx_out is not None else torch.empty((B, Hk, nb, topk), device=q_pooled.device, dtype=torch.int32)
+    S = scores_out if scores_out is not None else torch.empty((B, Hk, nb, nb), device=q_pooled.device,
                                                               dtype=torch.float32)
-    if flags:
+    if Hk != H:
+        _check(lib.bsa_block_scores_topk_gqa(_p(q_pooled), _p(k_pooled), _p(S), _p(idx), B, H, Hk, nb, D,
+                                             topk, flags, _stream(q_pooled)))
+    elif flags:
         _check(lib.bsa_block_scores_topk_ex(_p(q_pooled), _p(k_pooled), _p(S), _p(idx), B, H, nb, D, topk,
                                             flags, _stream(q_pooled)))
     else:
@@ -158,11 +171,15 @@ def bsa_sparse_attn_fwd(q, k, v, idx, block_size: int, scale: float | None = Non
     if not (q.dtype == k.dtype == v.dtype):
         raise TypeError("q, k, v must share one dtype")
     B, N, H, D = q.shape
+    Hk = k.shape[2]  # key/value heads: fewer than H for grouped queries
     topk = idx.shape[-1]
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     o = out if out is not None else torch.empty_like(q)
-    if flags:
+    if Hk != H:
+        _check(lib.bsa_sparse_attn_fwd_gqa(_p(q), _p(k), _p(v), _p(idx), _p(o), B, N, H, Hk, D, block_size,
+                                           topk, float(scale), _dtype_code(q), flags, _stream(q)))
+    elif flags:
         _check(lib.bsa_sparse_attn_fwd_ex(_p(q), _p(k), _p(v), _p(idx), _p(o), B, N, H, D, block_size, topk,
                                           float(scale), _dtype_code(q), flags, _stream(q)))
     else:
@@ -178,12 +195,16 @@ def bsa_forward(q, k, v, block_size: int, topk_ratio: float, workspace: torch.Te
     if not (q.dtype == k.dtype == v.dtype):
         raise TypeError("q, k, v must share one dtype")
     B, N, H, D = q.shape
-    need = bsa_forward_workspace_bytes(B, N, H, D, block_size, topk_ratio)
+    Hk = k.shape[2]  # key/value heads: fewer than H for grouped queries
+    need = bsa_forward_workspace_bytes(B, N, H, D, block_size, topk_ratio, H_kv=Hk)
     if workspace is None:
         workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
     o = out if out is not None else torch.empty_like(q)
     nbytes = workspace.numel() * workspace.element_size()
-    if flags:
+    if Hk != H:
+        _check(lib.bsa_forward_gqa(_p(q), _p(k), _p(v), _p(o), B, N, H, Hk, D, block_size, float(topk_ratio),
+                                   _dtype_code(q), flags, _p(workspace), nbytes, _stream(q)))
+    elif flags:
         _check(lib.bsa_forward_ex(_p(q), _p(k), _p(v), _p(o), B, N, H, D, block_size, float(topk_ratio),
                                   _dtype_code(q), flags, _p(workspace), nbytes, _stream(q)))
     else:
@@ -216,21 +237,22 @@ def bsa_device_error(device=None) -> int:
 
 
 def workspace_views(ws: torch.Tensor, B: int, N: int, H: int, D: int, block_size: int, topk_ratio: float,
-                    with_scores: bool = False):
-    """The pooled q, pooled k, index-list (and block-score) sections of a
-    bsa_forward workspace (the layout of include/bsa.h: 256-byte aligned
-    sections in that order)."""
+                    with_scores: bool = False, H_kv: int | None = None):
+    """The pooled q [B,H,nb,D], pooled k [B,H_kv,nb,D], index-list [B,H_kv,nb,k]
+    (and block-score [B,H_kv,nb,nb]) sections of a bsa_forward(_gqa)
+    workspace (the layout of include/bsa.h: 256-byte aligned sections in that
+    order)."""
+    Hk = H if H_kv is None else H_kv
     nb = N // block_size
     kk = bsa_topk_count(nb, topk_ratio)
     a256 = lambda x: (x + 255) // 256 * 256
-    pooled = a256(B * H * nb * D * 4)
-    idxb = a256(B * H * nb * kk * 4)
+    qpb, kpb, idxb = a256(B * H * nb * D * 4), a256(B * Hk * nb * D * 4), a256(B * Hk * nb * kk * 4)
     base = ws.view(torch.uint8)
     qp = base[:B * H * nb * D * 4].view(torch.float32).view(B, H, nb, D)
-    kp = base[pooled:pooled + B * H * nb * D * 4].view(torch.float32).view(B, H, nb, D)
-    idx = base[2 * pooled:2 * pooled + B * H * nb * kk * 4].view(torch.int32).view(B, H, nb, kk)
+    kp = base[qpb:qpb + B * Hk * nb * D * 4].view(torch.float32).view(B, Hk, nb, D)
+    idx = base[qpb + kpb:qpb + kpb + B * Hk * nb * kk * 4].view(torch.int32).view(B, Hk, nb, kk)
     if not with_scores:
         return qp, kp, idx
-    off = 2 * pooled + idxb
-    S = base[off:off + B * H * nb * nb * 4].view(torch.float32).view(B, H, nb, nb)
+    off = qpb + kpb + idxb
+    S = base[off:off + B * Hk * nb * nb * 4].view(torch.float32).view(B, Hk, nb, nb)
     return qp, kp, idx, S

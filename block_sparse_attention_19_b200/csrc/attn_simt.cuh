@@ -39,7 +39,7 @@ template <int D>
 __global__ void __launch_bounds__(kSimtThreads)
     sparse_attn_simt_kernel(const float* __restrict__ q, const float* __restrict__ kmat,
                             const float* __restrict__ v, const int32_t* __restrict__ idx,
-                            float* __restrict__ o, int N, int H, int bs, int k, float scale,
+                            float* __restrict__ o, int N, int H, int Hkv, int bs, int k, float scale,
                             unsigned flags) {
   extern __shared__ __align__(16) unsigned char simt_raw[];
   SimtSmem<D>& sm = *reinterpret_cast<SimtSmem<D>*>(simt_raw);
@@ -56,10 +56,12 @@ __global__ void __launch_bounds__(kSimtThreads)
   const long b = u / H;
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const long row_stride = static_cast<long>(H) * D;
+  const long row_stride = static_cast<long>(H) * D;  // q and o rows
+  const long kv_stride = static_cast<long>(Hkv) * D;  // k and v rows
+  const int g = h / (H / Hkv);                        // key/value head of query head h
   const float* qb = q + (b * N) * row_stride + static_cast<long>(h) * D;
-  const float* kb = kmat + (b * N) * row_stride + static_cast<long>(h) * D;
-  const float* vb = v + (b * N) * row_stride + static_cast<long>(h) * D;
+  const float* kb = kmat + (b * N) * kv_stride + static_cast<long>(g) * D;
+  const float* vb = v + (b * N) * kv_stride + static_cast<long>(g) * D;
   const int n0 = i * bs + chunk * kSimtRows;
 
   for (int e = tid; e < kSimtRows * D; e += kSimtThreads) {
@@ -76,7 +78,7 @@ __global__ void __launch_bounds__(kSimtThreads)
     for (int c = 0; c < DL; ++c) acc[rr][c] = 0.f;
   }
 
-  const int32_t* sel = idx + ((b * H + h) * static_cast<long>(nb) + i) * k;
+  const int32_t* sel = idx + ((b * Hkv + g) * static_cast<long>(nb) + i) * k;
   const int tiles_per_block = bs / kSimtKeys;
   const bool causal = (flags & kFlagCausal) != 0;
   for (int s = 0; s < k; ++s) {
@@ -91,8 +93,8 @@ __global__ void __launch_bounds__(kSimtThreads)
       __syncthreads();  // previous tile fully consumed
       for (int e = tid; e < kSimtKeys * D; e += kSimtThreads) {
         const int r = e / D, d = e % D;
-        sm.k[r][d] = kb[static_cast<long>(t0 + r) * row_stride + d];
-        sm.v[r][d] = vb[static_cast<long>(t0 + r) * row_stride + d];
+        sm.k[r][d] = kb[static_cast<long>(t0 + r) * kv_stride + d];
+        sm.v[r][d] = vb[static_cast<long>(t0 + r) * kv_stride + d];
       }
       __syncthreads();
 #pragma unroll

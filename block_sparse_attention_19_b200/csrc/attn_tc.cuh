@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
                           const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ o, int N,
-                          int H, int bs, int k, float scale_log2, unsigned flags) {
+                          int H, int Hkv, int bs, int k, float scale_log2, unsigned flags) {
   using L = TcLayout<D, BM>;
   constexpr int KS = L::kStages;
   extern __shared__ __align__(1024) unsigned char tc_raw[];
@@ -153,7 +153,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   u /= nb;
   const int h = static_cast<int>(u % H);
   const int b = static_cast<int>(u / H);
-  const int32_t* sel = idx + ((static_cast<long>(b) * H + h) * nb + i) * k;
+  const int g = h / (H / Hkv);  // key/value head (and selection) of query head h
+  const int32_t* sel = idx + ((static_cast<long>(b) * Hkv + g) * nb + i) * k;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int hf = 0; hf < halves; ++hf)
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(smem + ring + s * L::kKVBytes + c * (kKeyTile * 128) + hf * 64 * 128, map,
-                        &full[s], c * 64, h, row0[hf], b, keep);
+                        &full[s], c * 64, g, row0[hf], b, keep);
         issued[s] = use + 1;
       }
       // drain: every copy this thread issued has landed before teardown

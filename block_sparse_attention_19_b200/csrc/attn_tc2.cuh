@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
                            const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v,
                            const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ o, int N,
-                           int H, int bs, int k, float scale_log2) {
+                           int H, int Hkv, int bs, int k, float scale_log2) {
   using L = Tc2Layout<D>;
   constexpr int KS = L::kKStages, VS = L::kVStages;
   extern __shared__ __align__(1024) unsigned char tc2_raw[];
@@ -128,20 +128,40 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
   volatile int* abort_flag = &bar.abort;
 
   const int nb = N / bs;
-  const bool shared_kv = bs == 256;
-  const int per_bh = shared_kv ? nb : (nb + 1) / 2;
+  // What the two query tiles (streams) of a CTA are:
+  //  - block_size 256: the two 128-row halves of one query block of one head;
+  //  - block_size 128, an even number G of query heads per key/value head:
+  //    one query block of two heads of the same group;
+  //  - otherwise: two consecutive query blocks of one head.
+  // In the first two the streams read the same key tiles (one selection),
+  // so each K and V tile is loaded once for both.
+  const int G = H / Hkv;
+  const bool head_pairs = bs == 128 && (G % 2) == 0;
+  const bool shared_kv = bs == 256 || head_pairs;
   long u = blockIdx.x;
-  const int unit = static_cast<int>(u % per_bh);
-  u /= per_bh;
-  const int h = static_cast<int>(u % H);
-  const int b = static_cast<int>(u / H);
-  // stream x covers query rows [row0[x], row0[x] + 128)
-  const int iA = shared_kv ? unit : 2 * unit;
+  int iA, b, qh[2];
+  if (head_pairs) {
+    iA = static_cast<int>(u % nb);
+    u /= nb;
+    const int hp = static_cast<int>(u % (H / 2));
+    b = static_cast<int>(u / (H / 2));
+    qh[0] = 2 * hp;
+    qh[1] = 2 * hp + 1;
+  } else {
+    const int per_bh = bs == 256 ? nb : (nb + 1) / 2;
+    const int unit = static_cast<int>(u % per_bh);
+    u /= per_bh;
+    qh[0] = qh[1] = static_cast<int>(u % H);
+    b = static_cast<int>(u / H);
+    iA = bs == 256 ? unit : 2 * unit;
+  }
+  const int g = qh[0] / G;  // the key/value head (and selection) of both streams
   const int nstreams = (!shared_kv && iA + 1 >= nb) ? 1 : 2;
-  const int row0[2] = {iA * bs, shared_kv ? iA * bs + 128 : (iA + 1) * bs};
-  const long bh = static_cast<long>(b) * H + h;
-  const int32_t* sel_a = idx + (bh * nb + iA) * k;
-  const int32_t* sel_b = shared_kv ? sel_a : idx + (bh * nb + (iA + 1 < nb ? iA + 1 : iA)) * k;
+  // stream x covers query rows [row0[x], row0[x] + 128) of query head qh[x]
+  const int row0[2] = {iA * bs, bs == 256 ? iA * bs + 128 : (head_pairs ? iA * bs : (iA + 1) * bs)};
+  const long bg = static_cast<long>(b) * Hkv + g;
+  const int32_t* sel_a = idx + (bg * nb + iA) * k;
+  const int32_t* sel_b = shared_kv ? sel_a : idx + (bg * nb + (iA + 1 < nb ? iA + 1 : iA)) * k;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -169,8 +189,9 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     // so that a row of only -1 still reads block 0 instead of nothing)
     const int ta = max(index_row_valid(sel_a, k), 1);
     const int tb = nstreams == 2 && !shared_kv ? max(index_row_valid(sel_b, k), 1) : 0;
-    bar.tiles[0] = shared_kv ? 2 * ta : ta;
-    bar.tiles[1] = shared_kv ? 2 * ta : tb;
+    const int tpb = bs == 256 ? 2 : 1;  // key tiles per block
+    bar.tiles[0] = tpb * ta;
+    bar.tiles[1] = shared_kv ? tpb * ta : tb;
     fence_mbarrier_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -219,7 +240,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
           for (int hh = 0; hh < 2; ++hh)
             for (int c = 0; c < L::kChunks; ++c)
               tma_load_4d(smem + L::kQOff + x * L::kTileBytes + c * (128 * 128) + hh * 64 * 128,
-                          &tm_q, &bar.q_full, c * 64, h, row0[x] + hh * 64, b, stream);
+                          &tm_q, &bar.q_full, c * 64, qh[x], row0[x] + hh * 64, b, stream);
       }
       for (int n = 0; n < nloads && ok; ++n) {
         const int s = n % S, use = n / S;
@@ -234,7 +255,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         for (int hf = 0; hf < 2; ++hf)
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(smem + ring + s * L::kTileBytes + c * (128 * 128) + hf * 64 * 128, map,
-                        &full[s], c * 64, h, r[hf], b, keep);
+                        &full[s], c * 64, g, r[hf], b, keep);
         issued[s] = use + 1;
       }
       if (is_k) mbar_wait_teardown(&bar.q_full, 0);
@@ -439,7 +460,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
       tc_fence_after();
       const float inv = 1.0f / l_run;
       const long n = row0[x] + row;
-      __nv_bfloat16* orow = o + ((static_cast<long>(b) * N + n) * H + h) * D;
+      __nv_bfloat16* orow = o + ((static_cast<long>(b) * N + n) * H + qh[x]) * D;
       uint32_t r[32];
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {

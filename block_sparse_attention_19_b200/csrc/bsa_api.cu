@@ -74,6 +74,12 @@ bsa_status check_flags(unsigned flags) {
   return BSA_OK;
 }
 
+bsa_status check_heads(int H, int Hkv) {
+  if (Hkv < 1 || H % Hkv != 0)
+    return fail(BSA_ERR_INVALID_ARG, "H=%d must be a positive multiple of H_kv=%d", H, Hkv);
+  return BSA_OK;
+}
+
 bsa_status check_dtype(bsa_dtype dt) {
   if (dt != BSA_F32 && dt != BSA_BF16) return fail(BSA_ERR_UNSUPPORTED, "dtype %d", static_cast<int>(dt));
   return BSA_OK;
@@ -162,20 +168,23 @@ int sm_count() {
 // Block scores S = qbar kbar^T per (b, h) on the tensor cores (split TF32),
 // written to S [B, H, nb, nb] by TMA tensor stores when a row of S is a
 // multiple of 16 bytes; then the top-k selection reads S back.
-bsa_status launch_scores(const float* qp, const float* kp, float* S, int B, int H, int nb, int D,
-                         cudaStream_t st) {
+// H query heads, Hkv key/value heads (score matrices); H > Hkv averages each
+// group's pooled queries.
+bsa_status launch_scores(const float* qp, const float* kp, float* S, int B, int H, int Hkv, int nb,
+                         int D, cudaStream_t st) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    for (auto fn : {bsa::block_scores_tc_kernel<128>, bsa::block_scores_tc_kernel<256>}) {
+    for (auto fn : {bsa::block_scores_tc_kernel<128, false>, bsa::block_scores_tc_kernel<256, false>,
+                    bsa::block_scores_tc_kernel<128, true>, bsa::block_scores_tc_kernel<256, true>}) {
       cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bsa::kScSmem);
       if (e != cudaSuccess) return cuda_fail(e, "scores smem attribute");
     }
     attr_set[dev] = true;
   }
   const int ntile = nb <= 128 ? 128 : 256;
-  const long ntiles = static_cast<long>(B) * H * ((nb + bsa::kScM - 1) / bsa::kScM) *
+  const long ntiles = static_cast<long>(B) * Hkv * ((nb + bsa::kScM - 1) / bsa::kScM) *
                       ((nb + ntile - 1) / ntile);
   const int tma_store = (nb % 4 == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0) ? 1 : 0;
   CUtensorMap tm_s;
@@ -184,7 +193,7 @@ bsa_status launch_scores(const float* qp, const float* kp, float* S, int B, int 
     auto encode = tensor_map_encoder();
     if (!encode) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(nb),
-                          static_cast<cuuint64_t>(B) * H};
+                          static_cast<cuuint64_t>(B) * Hkv};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(nb) * 4,
                              static_cast<cuuint64_t>(nb) * nb * 4};
     cuuint32_t box[3] = {32, 32, 1};
@@ -195,12 +204,20 @@ bsa_status launch_scores(const float* qp, const float* kp, float* S, int B, int 
     if (r != CUDA_SUCCESS) return fail(BSA_ERR_CUDA, "score tensor map failed (%d)", static_cast<int>(r));
   }
   const long grid = ntiles < sm_count() ? ntiles : sm_count();
-  if (ntile == 128)
-    bsa::block_scores_tc_kernel<128><<<static_cast<unsigned>(grid), bsa::kScThreads, bsa::kScSmem, st>>>(
-        qp, kp, S, tm_s, nb, D, ntiles, tma_store);
+  const unsigned gr = static_cast<unsigned>(grid);
+  const bool grouped = H != Hkv;
+  if (ntile == 128 && !grouped)
+    bsa::block_scores_tc_kernel<128, false><<<gr, bsa::kScThreads, bsa::kScSmem, st>>>(
+        qp, kp, S, tm_s, nb, D, ntiles, tma_store, H, Hkv);
+  else if (ntile == 128)
+    bsa::block_scores_tc_kernel<128, true><<<gr, bsa::kScThreads, bsa::kScSmem, st>>>(
+        qp, kp, S, tm_s, nb, D, ntiles, tma_store, H, Hkv);
+  else if (!grouped)
+    bsa::block_scores_tc_kernel<256, false><<<gr, bsa::kScThreads, bsa::kScSmem, st>>>(
+        qp, kp, S, tm_s, nb, D, ntiles, tma_store, H, Hkv);
   else
-    bsa::block_scores_tc_kernel<256><<<static_cast<unsigned>(grid), bsa::kScThreads, bsa::kScSmem, st>>>(
-        qp, kp, S, tm_s, nb, D, ntiles, tma_store);
+    bsa::block_scores_tc_kernel<256, true><<<gr, bsa::kScThreads, bsa::kScSmem, st>>>(
+        qp, kp, S, tm_s, nb, D, ntiles, tma_store, H, Hkv);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_scores_tc_kernel launch");
 }
@@ -228,15 +245,15 @@ bsa_status launch_topk(const float* S, int32_t* idx, int B, int H, int nb, int k
 }
 
 bsa_status launch_select(const float* qp, const float* kp, float* S, int32_t* idx, int B, int H,
-                         int nb, int D, int k, unsigned flags, cudaStream_t st) {
+                         int Hkv, int nb, int D, int k, unsigned flags, cudaStream_t st) {
   bsa_status s;
-  if ((s = launch_scores(qp, kp, S, B, H, nb, D, st)) != BSA_OK) return s;
-  return launch_topk(S, idx, B, H, nb, k, flags, st);
+  if ((s = launch_scores(qp, kp, S, B, H, Hkv, nb, D, st)) != BSA_OK) return s;
+  return launch_topk(S, idx, B, Hkv, nb, k, flags, st);
 }
 
 template <int D>
 bsa_status launch_attn_simt(const float* q, const float* k, const float* v, const int32_t* idx,
-                            float* o, int B, int N, int H, int bs, int kk, float scale,
+                            float* o, int B, int N, int H, int Hkv, int bs, int kk, float scale,
                             unsigned flags, cudaStream_t st) {
   const size_t smem = sizeof(bsa::SimtSmem<D>);
   static bool attr_set[64] = {false};
@@ -251,21 +268,21 @@ bsa_status launch_attn_simt(const float* q, const float* k, const float* v, cons
   const long grid = static_cast<long>(B) * H * (N / bs) * (bs / bsa::kSimtRows);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   bsa::sparse_attn_simt_kernel<D><<<static_cast<unsigned>(grid), bsa::kSimtThreads, smem, st>>>(
-      q, k, v, idx, o, N, H, bs, kk, scale, flags);
+      q, k, v, idx, o, N, H, Hkv, bs, kk, scale, flags);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_simt_kernel launch");
 }
 
 template <int D, int BM>
 bsa_status launch_attn_tc(const void* q, const void* k, const void* v, const int32_t* idx,
-                          void* o, int B, int N, int H, int bs, int kk, float scale,
+                          void* o, int B, int N, int H, int Hkv, int bs, int kk, float scale,
                           unsigned flags, cudaStream_t st) {
   using L = bsa::TcLayout<D, BM>;
   CUtensorMap mq, mk, mv;
   bsa_status s;
   if ((s = make_bnhd_map(&mq, q, B, N, H, D)) != BSA_OK) return s;
-  if ((s = make_bnhd_map(&mk, k, B, N, H, D)) != BSA_OK) return s;
-  if ((s = make_bnhd_map(&mv, v, B, N, H, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mk, k, B, N, Hkv, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mv, v, B, N, Hkv, D)) != BSA_OK) return s;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -280,20 +297,21 @@ bsa_status launch_attn_tc(const void* q, const void* k, const void* v, const int
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   const float scale_log2 = scale * 1.4426950408889634f;
   bsa::sparse_attn_tc_kernel<D, BM><<<static_cast<unsigned>(grid), bsa::kTcThreads, L::kBytes, st>>>(
-      mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, bs, kk, scale_log2, flags);
+      mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, Hkv, bs, kk, scale_log2, flags);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc_kernel launch");
 }
 
 template <int D, bool kCausal>
 bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
-                              int B, int N, int H, int bs, int kk, float scale, cudaStream_t st) {
+                              int B, int N, int H, int Hkv, int bs, int kk, float scale,
+                              cudaStream_t st) {
   using L = bsa::Tc2Layout<D>;
   CUtensorMap mq, mk, mv;
   bsa_status s;
   if ((s = make_bnhd_map(&mq, q, B, N, H, D)) != BSA_OK) return s;
-  if ((s = make_bnhd_map(&mk, k, B, N, H, D)) != BSA_OK) return s;
-  if ((s = make_bnhd_map(&mv, v, B, N, H, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mk, k, B, N, Hkv, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mv, v, B, N, Hkv, D)) != BSA_OK) return s;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -313,38 +331,43 @@ bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const
     attr_set[dev] = true;
   }
   const int nb = N / bs;
-  const long grid = static_cast<long>(B) * H * (bs == 256 ? nb : (nb + 1) / 2);
+  // the kernel's CTA layouts: halves of a 256-block; two query heads of a
+  // group on one block (an even group size); two blocks of one head
+  const bool head_pairs = bs == 128 && ((H / Hkv) % 2) == 0;
+  const long grid = head_pairs ? static_cast<long>(B) * (H / 2) * nb
+                               : static_cast<long>(B) * H * (bs == 256 ? nb : (nb + 1) / 2);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   const float scale_log2 = scale * 1.4426950408889634f;
   bsa::sparse_attn_tc2_kernel<D, kCausal><<<static_cast<unsigned>(grid), bsa::kTc2Threads, L::kBytes, st>>>(
-      mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, bs, kk, scale_log2);
+      mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, Hkv, bs, kk, scale_log2);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc2_kernel launch");
 }
 
 template <int D>
 bsa_status launch_attn_tc2(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
-                           int B, int N, int H, int bs, int kk, float scale, unsigned flags,
+                           int B, int N, int H, int Hkv, int bs, int kk, float scale, unsigned flags,
                            cudaStream_t st) {
-  return (flags & BSA_FLAG_CAUSAL) ? launch_attn_tc2_as<D, true>(q, k, v, idx, o, B, N, H, bs, kk, scale, st)
-                                   : launch_attn_tc2_as<D, false>(q, k, v, idx, o, B, N, H, bs, kk, scale, st);
+  return (flags & BSA_FLAG_CAUSAL)
+             ? launch_attn_tc2_as<D, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, st)
+             : launch_attn_tc2_as<D, false>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, st);
 }
 
 bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
-                       int B, int N, int H, int D, int bs, int kk, float scale, bsa_dtype dt,
+                       int B, int N, int H, int Hkv, int D, int bs, int kk, float scale, bsa_dtype dt,
                        unsigned flags, cudaStream_t st) {
   if (dt == BSA_F32) {
     const float *fq = static_cast<const float*>(q), *fk = static_cast<const float*>(k),
                 *fv = static_cast<const float*>(v);
     float* fo = static_cast<float*>(o);
-    return D == 64 ? launch_attn_simt<64>(fq, fk, fv, idx, fo, B, N, H, bs, kk, scale, flags, st)
-                   : launch_attn_simt<128>(fq, fk, fv, idx, fo, B, N, H, bs, kk, scale, flags, st);
+    return D == 64 ? launch_attn_simt<64>(fq, fk, fv, idx, fo, B, N, H, Hkv, bs, kk, scale, flags, st)
+                   : launch_attn_simt<128>(fq, fk, fv, idx, fo, B, N, H, Hkv, bs, kk, scale, flags, st);
   }
   if (bs == 64)
-    return D == 64 ? launch_attn_tc<64, 64>(q, k, v, idx, o, B, N, H, bs, kk, scale, flags, st)
-                   : launch_attn_tc<128, 64>(q, k, v, idx, o, B, N, H, bs, kk, scale, flags, st);
-  return D == 64 ? launch_attn_tc2<64>(q, k, v, idx, o, B, N, H, bs, kk, scale, flags, st)
-                 : launch_attn_tc2<128>(q, k, v, idx, o, B, N, H, bs, kk, scale, flags, st);
+    return D == 64 ? launch_attn_tc<64, 64>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, st)
+                   : launch_attn_tc<128, 64>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, st);
+  return D == 64 ? launch_attn_tc2<64>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, st)
+                 : launch_attn_tc2<128>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, st);
 }
 
 struct Workspace {
@@ -355,19 +378,21 @@ struct Workspace {
   size_t bytes;
 };
 
-// q_pooled | k_pooled | idx | scores, each section 256-byte aligned
-Workspace workspace_layout(void* base, int B, int N, int H, int D, int bs, int k) {
+// q_pooled [B,H,nb,D] | k_pooled [B,Hkv,nb,D] | idx [B,Hkv,nb,k] | scores
+// [B,Hkv,nb,nb], each section 256-byte aligned
+Workspace workspace_layout(void* base, int B, int N, int H, int Hkv, int D, int bs, int k) {
   const size_t nb = static_cast<size_t>(N / bs);
-  const size_t pooled = align256(static_cast<size_t>(B) * H * nb * D * sizeof(float));
-  const size_t idxb = align256(static_cast<size_t>(B) * H * nb * k * sizeof(int32_t));
-  const size_t scb = align256(static_cast<size_t>(B) * H * nb * nb * sizeof(float));
+  const size_t qpb = align256(static_cast<size_t>(B) * H * nb * D * sizeof(float));
+  const size_t kpb = align256(static_cast<size_t>(B) * Hkv * nb * D * sizeof(float));
+  const size_t idxb = align256(static_cast<size_t>(B) * Hkv * nb * k * sizeof(int32_t));
+  const size_t scb = align256(static_cast<size_t>(B) * Hkv * nb * nb * sizeof(float));
   unsigned char* p = static_cast<unsigned char*>(base);
   Workspace w;
   w.qp = reinterpret_cast<float*>(p);
-  w.kp = reinterpret_cast<float*>(p + pooled);
-  w.idx = reinterpret_cast<int32_t*>(p + 2 * pooled);
-  w.scores = reinterpret_cast<float*>(p + 2 * pooled + idxb);
-  w.bytes = 2 * pooled + idxb + scb;
+  w.kp = reinterpret_cast<float*>(p + qpb);
+  w.idx = reinterpret_cast<int32_t*>(p + qpb + kpb);
+  w.scores = reinterpret_cast<float*>(p + qpb + kpb + idxb);
+  w.bytes = qpb + kpb + idxb + scb;
   return w;
 }
 
@@ -384,11 +409,16 @@ int bsa_topk_count(int nb, double topk_ratio) {
   return static_cast<int>(prod);  // truncation == Python int() for prod >= 0
 }
 
-size_t bsa_forward_workspace_bytes(int B, int N, int H, int D, int block_size, double topk_ratio) {
-  if (check_dims(B, N, H, D, block_size) != BSA_OK) return 0;
+size_t bsa_forward_gqa_workspace_bytes(int B, int N, int H, int Hkv, int D, int block_size,
+                                       double topk_ratio) {
+  if (check_dims(B, N, H, D, block_size) != BSA_OK || check_heads(H, Hkv) != BSA_OK) return 0;
   const int k = bsa_topk_count(N / block_size, topk_ratio);
   if (k < 1 || k > N / block_size) return 0;
-  return workspace_layout(nullptr, B, N, H, D, block_size, k).bytes;
+  return workspace_layout(nullptr, B, N, H, Hkv, D, block_size, k).bytes;
+}
+
+size_t bsa_forward_workspace_bytes(int B, int N, int H, int D, int block_size, double topk_ratio) {
+  return bsa_forward_gqa_workspace_bytes(B, N, H, H, D, block_size, topk_ratio);
 }
 
 const char* bsa_status_string(bsa_status s) {
@@ -420,12 +450,13 @@ bsa_status bsa_block_pool(const void* x, float* x_pooled, int B, int N, int H, i
   return ok();
 }
 
-bsa_status bsa_block_scores_topk_ex(const float* q_pooled, const float* k_pooled, float* scores,
-                                    int32_t* idx, int B, int H, int nb, int D, int k, unsigned flags,
-                                    void* stream) {
+bsa_status bsa_block_scores_topk_gqa(const float* q_pooled, const float* k_pooled, float* scores,
+                                     int32_t* idx, int B, int H, int Hkv, int nb, int D, int k,
+                                     unsigned flags, void* stream) {
   bsa_status s;
   if ((s = check_flags(flags)) != BSA_OK) return s;
   if (B < 1 || H < 1 || nb < 1) return fail(BSA_ERR_INVALID_ARG, "sizes must be positive");
+  if ((s = check_heads(H, Hkv)) != BSA_OK) return s;
   if (D != 64 && D != 128) return fail(BSA_ERR_UNSUPPORTED, "D=%d (supported: 64, 128)", D);
   if (nb > 32768) return fail(BSA_ERR_UNSUPPORTED, "nb=%d > 32768", nb);
   if (k < 1 || k > nb) return fail(BSA_ERR_INVALID_ARG, "k=%d outside [1, nb=%d]", k, nb);
@@ -433,10 +464,16 @@ bsa_status bsa_block_scores_topk_ex(const float* q_pooled, const float* k_pooled
   if (!aligned16(q_pooled) || !aligned16(k_pooled) || !aligned16(idx) || !aligned16(scores))
     return fail(BSA_ERR_MISALIGNED, "q_pooled, k_pooled, idx or scores");
   if ((s = check_device()) != BSA_OK) return s;
-  if ((s = launch_select(q_pooled, k_pooled, scores, idx, B, H, nb, D, k, flags,
+  if ((s = launch_select(q_pooled, k_pooled, scores, idx, B, H, Hkv, nb, D, k, flags,
                          static_cast<cudaStream_t>(stream))) != BSA_OK)
     return s;
   return ok();
+}
+
+bsa_status bsa_block_scores_topk_ex(const float* q_pooled, const float* k_pooled, float* scores,
+                                    int32_t* idx, int B, int H, int nb, int D, int k, unsigned flags,
+                                    void* stream) {
+  return bsa_block_scores_topk_gqa(q_pooled, k_pooled, scores, idx, B, H, H, nb, D, k, flags, stream);
 }
 
 bsa_status bsa_block_scores_topk(const float* q_pooled, const float* k_pooled, float* scores,
@@ -444,12 +481,13 @@ bsa_status bsa_block_scores_topk(const float* q_pooled, const float* k_pooled, f
   return bsa_block_scores_topk_ex(q_pooled, k_pooled, scores, idx, B, H, nb, D, k, 0u, stream);
 }
 
-bsa_status bsa_sparse_attn_fwd_ex(const void* q, const void* k, const void* v, const int32_t* idx,
-                                  void* o, int B, int N, int H, int D, int block_size, int kk,
-                                  float scale, bsa_dtype dt, unsigned flags, void* stream) {
+bsa_status bsa_sparse_attn_fwd_gqa(const void* q, const void* k, const void* v, const int32_t* idx,
+                                   void* o, int B, int N, int H, int Hkv, int D, int block_size, int kk,
+                                   float scale, bsa_dtype dt, unsigned flags, void* stream) {
   bsa_status s;
   if ((s = check_flags(flags)) != BSA_OK) return s;
   if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
+  if ((s = check_heads(H, Hkv)) != BSA_OK) return s;
   if ((s = check_dtype(dt)) != BSA_OK) return s;
   const int nb = N / block_size;
   if (kk < 1 || kk > nb) return fail(BSA_ERR_INVALID_ARG, "k=%d outside [1, nb=%d]", kk, nb);
@@ -459,10 +497,16 @@ bsa_status bsa_sparse_attn_fwd_ex(const void* q, const void* k, const void* v, c
     return fail(BSA_ERR_MISALIGNED, "q, k, v, idx or o");
   if (o == q || o == k || o == v) return fail(BSA_ERR_INVALID_ARG, "o aliases an input");
   if ((s = check_device()) != BSA_OK) return s;
-  if ((s = launch_attn(q, k, v, idx, o, B, N, H, D, block_size, kk, scale, dt, flags,
+  if ((s = launch_attn(q, k, v, idx, o, B, N, H, Hkv, D, block_size, kk, scale, dt, flags,
                        static_cast<cudaStream_t>(stream))) != BSA_OK)
     return s;
   return ok();
+}
+
+bsa_status bsa_sparse_attn_fwd_ex(const void* q, const void* k, const void* v, const int32_t* idx,
+                                  void* o, int B, int N, int H, int D, int block_size, int kk,
+                                  float scale, bsa_dtype dt, unsigned flags, void* stream) {
+  return bsa_sparse_attn_fwd_gqa(q, k, v, idx, o, B, N, H, H, D, block_size, kk, scale, dt, flags, stream);
 }
 
 bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx,
@@ -471,12 +515,13 @@ bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const void* v, cons
   return bsa_sparse_attn_fwd_ex(q, k, v, idx, o, B, N, H, D, block_size, kk, scale, dt, 0u, stream);
 }
 
-bsa_status bsa_forward_ex(const void* q, const void* k, const void* v, void* o, int B, int N,
-                          int H, int D, int block_size, double topk_ratio, bsa_dtype dt,
-                          unsigned flags, void* workspace, size_t workspace_bytes, void* stream) {
+bsa_status bsa_forward_gqa(const void* q, const void* k, const void* v, void* o, int B, int N,
+                           int H, int Hkv, int D, int block_size, double topk_ratio, bsa_dtype dt,
+                           unsigned flags, void* workspace, size_t workspace_bytes, void* stream) {
   bsa_status s;
   if ((s = check_flags(flags)) != BSA_OK) return s;
   if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
+  if ((s = check_heads(H, Hkv)) != BSA_OK) return s;
   if ((s = check_dtype(dt)) != BSA_OK) return s;
   const int nb = N / block_size;
   if (nb > 32768) return fail(BSA_ERR_UNSUPPORTED, "nb=%d > 32768", nb);
@@ -488,7 +533,7 @@ bsa_status bsa_forward_ex(const void* q, const void* k, const void* v, void* o, 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return fail(BSA_ERR_MISALIGNED, "q, k, v or o");
   if (o == q || o == k || o == v) return fail(BSA_ERR_INVALID_ARG, "o aliases an input");
-  const Workspace w = workspace_layout(workspace, B, N, H, D, block_size, kk);
+  const Workspace w = workspace_layout(workspace, B, N, H, Hkv, D, block_size, kk);
   if (!workspace || workspace_bytes < w.bytes)
     return fail(BSA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", w.bytes, workspace ? workspace_bytes : 0);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -496,11 +541,23 @@ bsa_status bsa_forward_ex(const void* q, const void* k, const void* v, void* o, 
   if ((s = check_device()) != BSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
-  if ((s = launch_pool(q, w.qp, k, w.kp, 2, B, N, H, D, block_size, dt, st)) != BSA_OK) return s;
-  if ((s = launch_select(w.qp, w.kp, w.scores, w.idx, B, H, nb, D, kk, flags, st)) != BSA_OK) return s;
-  if ((s = launch_attn(q, k, v, w.idx, o, B, N, H, D, block_size, kk, scale, dt, flags, st)) != BSA_OK)
+  if (H == Hkv) {
+    if ((s = launch_pool(q, w.qp, k, w.kp, 2, B, N, H, D, block_size, dt, st)) != BSA_OK) return s;
+  } else {
+    if ((s = launch_pool(q, w.qp, nullptr, nullptr, 1, B, N, H, D, block_size, dt, st)) != BSA_OK) return s;
+    if ((s = launch_pool(k, w.kp, nullptr, nullptr, 1, B, N, Hkv, D, block_size, dt, st)) != BSA_OK) return s;
+  }
+  if ((s = launch_select(w.qp, w.kp, w.scores, w.idx, B, H, Hkv, nb, D, kk, flags, st)) != BSA_OK) return s;
+  if ((s = launch_attn(q, k, v, w.idx, o, B, N, H, Hkv, D, block_size, kk, scale, dt, flags, st)) != BSA_OK)
     return s;
   return ok();
+}
+
+bsa_status bsa_forward_ex(const void* q, const void* k, const void* v, void* o, int B, int N,
+                          int H, int D, int block_size, double topk_ratio, bsa_dtype dt,
+                          unsigned flags, void* workspace, size_t workspace_bytes, void* stream) {
+  return bsa_forward_gqa(q, k, v, o, B, N, H, H, D, block_size, topk_ratio, dt, flags, workspace,
+                         workspace_bytes, stream);
 }
 
 bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int B, int N, int H,

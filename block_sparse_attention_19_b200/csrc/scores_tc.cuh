@@ -106,11 +106,14 @@ __device__ __forceinline__ ScTile sc_tile(long t, int nb, int ntile) {
 
 // grid.x = min(tiles, SMs); S = qbar kbar^T as [B*H, nb, nb] float32.
 // tm_s describes S as {nb, nb, B*H} with 32 x 32 boxes (used when tma_store).
-template <int NT>
+// kGroup: grouped queries (H = G * Hkv query heads): the A operand of score
+// matrix (b, g) is the mean of the pooled rows of query heads g*G .. g*G+G-1
+// (summed in float32, then scaled by 1/G).
+template <int NT, bool kGroup>
 __global__ void __launch_bounds__(kScThreads, 1)
     block_scores_tc_kernel(const float* __restrict__ qp, const float* __restrict__ kp,
                            float* __restrict__ S, const __grid_constant__ CUtensorMap tm_s, int nb,
-                           int D, long ntiles, int tma_store) {
+                           int D, long ntiles, int tma_store, int H, int Hkv) {
   constexpr int ntile = NT;
   extern __shared__ unsigned char sc_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -157,8 +160,12 @@ __global__ void __launch_bounds__(kScThreads, 1)
     for (long tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++i) {
       const ScTile tl = sc_tile(tile, nb, ntile);
       // this thread's rows: i0 + rsub + 16 u of qbar, j0 + rsub + 16 u of kbar
+      // tl.bh = b * Hkv + g: the query rows of (b, g) start at head g * G of batch b
+      const int G = kGroup ? H / Hkv : 1;
+      const long qhead = kGroup ? (tl.bh / Hkv) * H + (tl.bh % Hkv) * G : tl.bh;
       const float4* pa = reinterpret_cast<const float4*>(
-                             qp + (tl.bh * nb + tl.i0 + rsub) * static_cast<long>(D)) + q4;
+                             qp + (qhead * nb + tl.i0 + rsub) * static_cast<long>(D)) + q4;
+      const long hstep = static_cast<long>(nb) * D / 4;  // float4 per query head
       const float4* pb = reinterpret_cast<const float4*>(
                              kp + (tl.bh * nb + tl.j0 + rsub) * static_cast<long>(D)) + q4;
       const int ra = nb - tl.i0 - rsub, rb = nb - tl.j0 - rsub;  // rows left below this thread's first
@@ -174,6 +181,20 @@ __global__ void __launch_bounds__(kScThreads, 1)
           v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
           if (16 * uu < (is_a ? ra : rb))
             v[u] = __ldg((is_a ? pa : pb) + uu * step + c * (kScChunk / 4));
+          if (kGroup && is_a && 16 * uu < ra) {
+            for (int gg = 1; gg < G; ++gg) {
+              const float4 w = __ldg(pa + gg * hstep + uu * step + c * (kScChunk / 4));
+              v[u].x += w.x;
+              v[u].y += w.y;
+              v[u].z += w.z;
+              v[u].w += w.w;
+            }
+            const float inv = 1.0f / static_cast<float>(G);
+            v[u].x *= inv;
+            v[u].y *= inv;
+            v[u].z *= inv;
+            v[u].w *= inv;
+          }
         }
         const long use = gi >> 1;
         if (use > 0) ok = mbar_wait(&freed[grp], static_cast<uint32_t>((use - 1) & 1), abort_flag, 601);

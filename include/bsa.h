@@ -153,6 +153,48 @@ bsa_status bsa_forward_ex(const void* q, const void* k, const void* v, void* o, 
                           int H, int D, int block_size, double topk_ratio, bsa_dtype dt,
                           unsigned flags, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Grouped-query attention ------------------------------------------
+ * Page "从M2.7到M3：多模态模型稀疏注意力架构设计与实现全解析" §3.1: the MSA attention
+ * block is GQA-based. Readings: q (and o) have H heads, k and v have H_kv
+ * heads, H = G * H_kv; query head h reads key/value head h / G. Each
+ * key/value head has one block selection per query block, scored with the
+ * group's pooled query: the mean over its G query heads of their block means
+ * (equal, by linearity, to the mean of the G heads' block scores); every
+ * query head of the group then attends over that selection. H_kv = H is the
+ * plain method (the _ex entry points are these with H_kv = H). Flags as for
+ * the _ex entry points. Error codes as for the plain entry points, plus
+ * BSA_ERR_INVALID_ARG when H is not a positive multiple of H_kv. */
+
+/* Workspace bytes of bsa_forward_gqa: pooled q [B, H, nb, D], pooled k
+ * [B, H_kv, nb, D], the index list [B, H_kv, nb, topk] and the block scores
+ * [B, H_kv, nb, nb] (float32). 0 if the arguments are invalid. */
+size_t bsa_forward_gqa_workspace_bytes(int B, int N, int H, int H_kv, int D, int block_size,
+                                       double topk_ratio);
+
+/* q_pooled: [B, H, nb, D] float32 (the per-head block means, as
+ * bsa_block_pool writes them). k_pooled: [B, H_kv, nb, D]. scores:
+ * [B, H_kv, nb, nb] float32 (written: S[b, g] = qbar_g kbar_g^T with qbar_g
+ * the group mean, summed in float32 and scaled by 1/G). idx:
+ * [B, H_kv, nb, topk] int32 (written). */
+bsa_status bsa_block_scores_topk_gqa(const float* q_pooled, const float* k_pooled, float* scores,
+                                     int32_t* idx, int B, int H, int H_kv, int nb, int D, int topk,
+                                     unsigned flags, void* stream);
+
+/* q, o: [B, N, H, D]; k, v: [B, N, H_kv, D]; idx: [B, H_kv, nb, topk] (the
+ * selection of each key/value head, rows as bsa_sparse_attn_fwd_ex reads
+ * them). With an even G and block_size 128, two query heads of a group are
+ * computed together and share every gathered key/value tile. */
+bsa_status bsa_sparse_attn_fwd_gqa(const void* q, const void* k, const void* v, const int32_t* idx,
+                                   void* o, int B, int N, int H, int H_kv, int D, int block_size,
+                                   int topk, float scale, bsa_dtype dt, unsigned flags, void* stream);
+
+/* The whole path with grouped queries: pooling of q (H heads) and k (H_kv),
+ * scores and selection per key/value head, attention per query head; four
+ * or five kernel launches on `stream`. */
+bsa_status bsa_forward_gqa(const void* q, const void* k, const void* v, void* o, int B, int N,
+                           int H, int H_kv, int D, int block_size, double topk_ratio, bsa_dtype dt,
+                           unsigned flags, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Size of the fixed device scratch that bsa_forward_noalloc uses: 64 MiB. */
 #define BSA_NOALLOC_SCRATCH_BYTES (64u << 20)
 

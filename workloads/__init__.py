@@ -34,6 +34,11 @@ class Config:
     seed: int
     sample_blocks: int | None  # query blocks per (b, h) the oracle checks; None = all
     note: str = ""
+    H_kv: int | None = None  # key/value heads for grouped queries (None: H)
+
+    @property
+    def Hkv(self) -> int:
+        return self.H if self.H_kv is None else self.H_kv
 
     @property
     def nb(self) -> int:
@@ -55,7 +60,8 @@ class Config:
         return dataclasses.replace(self, topk_ratio=ratio, name=f"{self.name}@{ratio}")
 
     def describe(self) -> str:
-        return (f"B={self.B} N={self.N} H={self.H} D={self.D} block_size={self.block_size} "
+        kv = "" if self.Hkv == self.H else f" H_kv={self.Hkv}"
+        return (f"B={self.B} N={self.N} H={self.H}{kv} D={self.D} block_size={self.block_size} "
                 f"(nb={self.nb}) topk_ratio={self.topk_ratio} (k={self.k}) {self.dtype}")
 
 
@@ -77,16 +83,19 @@ def make_inputs(cfg: Config, device="cpu", seed: int | None = None):
     """Draw (q, k, v) for ``cfg`` on ``device`` following the module recipe."""
     g = torch.Generator(device=device)
     g.manual_seed(cfg.seed if seed is None else seed)
+    # k and v have cfg.Hkv heads (= H unless grouped queries); the draw order
+    # is the same either way
     shape = (cfg.B, cfg.N, cfg.H, cfg.D)
-    oshape = (cfg.B, cfg.nb, 1, cfg.H, cfg.D)
+    kshape = (cfg.B, cfg.N, cfg.Hkv, cfg.D)
     q = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
-    k = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
-    v = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
-    q_off = torch.randn(oshape, generator=g, device=device, dtype=torch.float32) * cfg.offset_sigma
-    k_off = torch.randn(oshape, generator=g, device=device, dtype=torch.float32) * cfg.offset_sigma
-    bshape = (cfg.B, cfg.nb, cfg.block_size, cfg.H, cfg.D)
-    q.view(bshape).add_(q_off)
-    k.view(bshape).add_(k_off)
+    k = torch.randn(kshape, generator=g, device=device, dtype=torch.float32)
+    v = torch.randn(kshape, generator=g, device=device, dtype=torch.float32)
+    q_off = torch.randn((cfg.B, cfg.nb, 1, cfg.H, cfg.D), generator=g, device=device,
+                        dtype=torch.float32) * cfg.offset_sigma
+    k_off = torch.randn((cfg.B, cfg.nb, 1, cfg.Hkv, cfg.D), generator=g, device=device,
+                        dtype=torch.float32) * cfg.offset_sigma
+    q.view(cfg.B, cfg.nb, cfg.block_size, cfg.H, cfg.D).add_(q_off)
+    k.view(cfg.B, cfg.nb, cfg.block_size, cfg.Hkv, cfg.D).add_(k_off)
     dt = cfg.torch_dtype
     return q.to(dt), k.to(dt), v.to(dt)
 
