@@ -20,8 +20,9 @@ Every function here is pinned by ``tests/test_oracle.py`` against closed forms,
 library routines (numpy matmul / lexsort, torch SDPA in float64), brute force
 and invariants; nothing in this package is "parity unpinned".
 
-Inputs may be float32, float64 or bfloat16; bfloat16 is passed as its raw
-16-bit patterns in a ``numpy.uint16`` array (tag ``"bf16"``).
+Inputs may be float32, float64, bfloat16 or FP8 E4M3; bfloat16 is passed as
+its raw 16-bit patterns in a ``numpy.uint16`` array and E4M3 as raw bytes in a
+``numpy.uint8`` array.
 """
 from __future__ import annotations
 
@@ -36,7 +37,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "bsa_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-F32, BF16, F64 = 0, 1, 2
+F32, BF16, F64, E4M3 = 0, 1, 2, 3
 _lib = None
 
 
@@ -69,6 +70,8 @@ def _load():
         lib.oracle_topk_ex.argtypes = [P, ctypes.c_long, i, i, P, i, P]
         lib.oracle_sparse_attn_ex.argtypes = [P, P, P, i, i, i, i, i, i, P, i, P, i, d, i, P]
         lib.oracle_sparse_attn_gqa.argtypes = [P, P, P, i, i, i, i, i, i, i, P, i, P, i, d, i, P]
+        lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_double.restype = d
         lib.oracle_num_threads.restype = i
         _lib = lib
     return _lib
@@ -87,7 +90,16 @@ def _as_input(x: np.ndarray):
         return x, F64
     if x.dtype == np.uint16:
         return x, BF16
-    raise TypeError(f"oracle inputs must be float32, float64 or bf16 bits (uint16), got {x.dtype}")
+    if x.dtype == np.uint8:
+        return x, E4M3
+    raise TypeError("oracle inputs must be float32, float64, bf16 bits (uint16) or e4m3 bytes (uint8), "
+                    f"got {x.dtype}")
+
+
+def e4m3_to_double(code: int) -> float:
+    """Value of an FP8 E4M3 byte (sign, 4-bit exponent with bias 7, 3-bit
+    mantissa, subnormals at exponent 0, NaN at S.1111.111; no infinities)."""
+    return _load().oracle_e4m3_to_double(int(code))
 
 
 def num_threads() -> int:

@@ -32,7 +32,8 @@
  *   - Attention is non-causal.
  *
  * Every function works in float64.  Inputs may be float32, bfloat16 (raw
- * 16-bit patterns) or float64; each element is converted exactly to double.
+ * 16-bit patterns), FP8 E4M3 (raw bytes) or float64; each element is
+ * converted exactly to double.
  * Parallelism (OpenMP) is only over independent output rows; the arithmetic
  * inside a row follows the definition in plain order.
  */
@@ -44,11 +45,27 @@
 #define ORACLE_F32 0
 #define ORACLE_BF16 1
 #define ORACLE_F64 2
+#define ORACLE_E4M3 3
+
+/* FP8 E4M3 (the "fn" variant: no infinities): 1 sign bit, 4 exponent bits with
+ * bias 7, 3 mantissa bits; exponent 0 holds subnormals (m / 8 * 2^-6); the
+ * pattern with every exponent and mantissa bit set is NaN. */
+double oracle_e4m3_to_double(uint8_t x) {
+  int sign = x >> 7, e = (x >> 3) & 15, m = x & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    v = ldexp((double)m / 8.0, -6);
+  else
+    v = ldexp(1.0 + (double)m / 8.0, e - 7);
+  return sign ? -v : v;
+}
 
 /* Exact conversion of one stored element to double. */
 static double elem(const void* base, int dtype, size_t i) {
   if (dtype == ORACLE_F32) return (double)((const float*)base)[i];
   if (dtype == ORACLE_F64) return ((const double*)base)[i];
+  if (dtype == ORACLE_E4M3) return oracle_e4m3_to_double(((const uint8_t*)base)[i]);
   /* bfloat16: the high 16 bits of an IEEE float32. */
   uint32_t bits = ((uint32_t)((const uint16_t*)base)[i]) << 16;
   float f;

@@ -494,3 +494,28 @@ def test_gqa_with_one_head_per_group_is_the_plain_path(oracle_mod, small_case):
         b = oracle_mod.forward_gqa(q, k, v, bs, ratio, causal=causal)
         np.testing.assert_array_equal(a["idx"], b["idx"])
         np.testing.assert_allclose(a["o"], b["o"], rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- FP8 E4M3 inputs
+
+def test_e4m3_decoding_matches_torch_for_every_code(oracle_mod):
+    codes = torch.arange(256, dtype=torch.uint8)
+    want = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle_mod.e4m3_to_double(c) for c in range(256)])
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan) and nan.sum() == 2  # S.1111.111
+    np.testing.assert_array_equal(got[~nan], want[~nan])
+
+
+def test_e4m3_inputs_are_their_exact_values(oracle_mod):
+    """The whole path on e4m3 bytes equals the path on the same values given
+    as float64 (the conversion is exact, nothing else changes)."""
+    B, N, H, D, bs = 1, 64, 2, 16, 8
+    x = [torch.from_numpy(_rand((B, N, H, D), s, bs=bs)).to(torch.float8_e4m3fn) for s in (150, 151, 152)]
+    raw = [t.view(torch.uint8).numpy() for t in x]
+    f64 = [t.to(torch.float64).numpy() for t in x]
+    for causal in (False, True):
+        a = oracle_mod.forward(*raw, bs, 0.375, causal=causal)
+        b = oracle_mod.forward(*f64, bs, 0.375, causal=causal)
+        np.testing.assert_array_equal(a["idx"], b["idx"])
+        np.testing.assert_array_equal(a["o"], b["o"])
