@@ -185,6 +185,8 @@ def main():
                     help="the causal variant (BSA_FLAG_CAUSAL): block-causal selection, token-causal attention")
     ap.add_argument("--force-diag", action="store_true",
                     help="with --causal: always keep the diagonal block (BSA_FLAG_FORCE_DIAG)")
+    ap.add_argument("--dtype", choices=["bf16", "e4m3"], default=None,
+                    help="override the config's input type (e4m3: FP8 inputs, bf16 output)")
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="grouped queries: the config with this many key/value heads (H a multiple of it)")
     ap.add_argument("--stages-only", action="store_true",
@@ -200,6 +202,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     cfg = W.CONFIGS[args.config]
+    if args.dtype is not None:
+        cfg = dataclasses.replace(cfg, dtype=args.dtype)
     if args.kv_heads is not None:
         if args.kv_heads < 1 or cfg.H % args.kv_heads:
             ap.error(f"--kv-heads must divide H={cfg.H}")
@@ -233,7 +237,7 @@ def main():
     ws = torch.empty(bsa.bsa_forward_workspace_bytes(B, N, H, D, bs, ratio, H_kv=Hk), device=dev,
                      dtype=torch.uint8)
     qp, kp, idx, S = bsa.workspace_views(ws, B, N, H, D, bs, ratio, with_scores=True, H_kv=Hk)
-    o = torch.empty_like(q)
+    o = torch.empty(q.shape, device=dev, dtype=torch.bfloat16 if cfg.dtype == "e4m3" else q.dtype)
 
     def step(ev=None):
         if ev is not None:
@@ -347,7 +351,8 @@ def main():
     kv_bytes = B * N * Hk * D * esz     # k (and v): fewer heads with grouped queries
     idx_bytes = B * Hk * (N // bs) * kk * 4
     pooled_bytes = B * (H + Hk) * (N // bs) * D * 4
-    alg_bytes = 2 * tensor_bytes + 2 * kv_bytes + idx_bytes  # q, k, v read + o written, and the index list
+    o_bytes = B * N * H * D * (2 if cfg.dtype == "e4m3" else esz)  # e4m3 inputs give a bf16 output
+    alg_bytes = tensor_bytes + o_bytes + 2 * kv_bytes + idx_bytes  # q, k, v read + o written, and the index list
     sel_bytes = tensor_bytes + kv_bytes + idx_bytes  # selection stage: q, k read + index list written
     peaks, peak_src = load_peaks()
     step_ms = total_ms / args.steps
@@ -367,15 +372,21 @@ def main():
                 "steps": args.e2e_steps},
         "clocks": clk,
     }
-    if cfg.dtype == "bf16":
+    if cfg.dtype in ("bf16", "e4m3"):
+        # the tensor-core peak for the path's own type: FP8 takes the measured
+        # bf16 peak times the nominal dense FP8 / bf16 ratio (4.5 / 2.25)
+        mult = 2.0 if cfg.dtype == "e4m3" else 1.0
+        peak, peak_sus = peaks["bf16_tflops"] * mult, peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * mult
         achieved = flops / (attn_ms / 1e3) / 1e12
-        roof_t = max(flops / (peaks["bf16_tflops"] * 1e12), alg_bytes / (peaks["hbm_gbs"] * 1e9))
+        roof_t = max(flops / (peak * 1e12), alg_bytes / (peaks["hbm_gbs"] * 1e9))
+        plain = not args.causal and Hk == H and cfg.dtype == "bf16"
         line["roofline"] = {
             "kernel": "sparse_attn_tc2_kernel" if bs in (128, 256) else "sparse_attn_tc_kernel",
             "bound": "tensor", "achieved": achieved,
-            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-            "peak_source": f"{peak_src} bf16 burst", "traffic": None if (args.causal or Hk != H) else NCU_TRAFFIC.get(cfg.name),
-            "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+            "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_source": f"{peak_src} bf16 burst" + (" x 2 (nominal e4m3 / bf16 dense ratio)" if mult > 1 else ""),
+            "traffic": NCU_TRAFFIC.get(cfg.name) if plain else None,
+            "frac_of_sustained": achieved / peak_sus,
             "frac_of_roofline_time": roof_t / (attn_ms / 1e3),
             "flops_per_launch": flops, "algorithmic_bytes_per_launch": alg_bytes,
         }

@@ -28,7 +28,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libbsa.so")
 
-BSA_F32, BSA_BF16 = 0, 1
+BSA_F32, BSA_BF16, BSA_E4M3 = 0, 1, 2
 _STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "BSA_ERR_MISALIGNED",
            4: "BSA_ERR_WORKSPACE", 5: "BSA_ERR_CUDA", 6: "BSA_ERR_DEVICE"}
 
@@ -96,7 +96,15 @@ def _dtype_code(t: torch.Tensor) -> int:
         return BSA_F32
     if t.dtype == torch.bfloat16:
         return BSA_BF16
-    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+    if t.dtype == torch.float8_e4m3fn:
+        return BSA_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype} (float32, bfloat16 or float8_e4m3fn)")
+
+
+def _out_like(q: torch.Tensor) -> torch.Tensor:
+    """The output tensor for inputs like q: same dtype, bfloat16 for e4m3 inputs."""
+    return torch.empty(q.shape, device=q.device,
+                       dtype=torch.bfloat16 if q.dtype == torch.float8_e4m3fn else q.dtype)
 
 
 def _stream(t: torch.Tensor):
@@ -175,7 +183,7 @@ def bsa_sparse_attn_fwd(q, k, v, idx, block_size: int, scale: float | None = Non
     topk = idx.shape[-1]
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    o = out if out is not None else torch.empty_like(q)
+    o = out if out is not None else _out_like(q)
     if Hk != H:
         _check(lib.bsa_sparse_attn_fwd_gqa(_p(q), _p(k), _p(v), _p(idx), _p(o), B, N, H, Hk, D, block_size,
                                            topk, float(scale), _dtype_code(q), flags, _stream(q)))
@@ -199,7 +207,7 @@ def bsa_forward(q, k, v, block_size: int, topk_ratio: float, workspace: torch.Te
     need = bsa_forward_workspace_bytes(B, N, H, D, block_size, topk_ratio, H_kv=Hk)
     if workspace is None:
         workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
-    o = out if out is not None else torch.empty_like(q)
+    o = out if out is not None else _out_like(q)
     nbytes = workspace.numel() * workspace.element_size()
     if Hk != H:
         _check(lib.bsa_forward_gqa(_p(q), _p(k), _p(v), _p(o), B, N, H, Hk, D, block_size, float(topk_ratio),
@@ -222,7 +230,7 @@ def bsa_forward_noalloc(q, k, v, block_size: int, topk_ratio: float, out: torch.
     if not (q.dtype == k.dtype == v.dtype):
         raise TypeError("q, k, v must share one dtype")
     B, N, H, D = q.shape
-    o = out if out is not None else torch.empty_like(q)
+    o = out if out is not None else _out_like(q)
     _check(lib.bsa_forward_noalloc(_p(q), _p(k), _p(v), _p(o), B, N, H, D, block_size, float(topk_ratio),
                                    _dtype_code(q), _stream(q)))
     return o

@@ -56,12 +56,15 @@ constexpr int kTc2MaxStages = 12;
 constexpr uint32_t kTc2RegsLow = 80, kTc2RegsHigh = 208;
 constexpr uint32_t kTc2LaunchRegs = (128 * kTc2RegsLow + 256 * kTc2RegsHigh + kTc2Threads - 1) / kTc2Threads;
 
-template <int D>
+// F8: FP8 E4M3 inputs (one byte per element) instead of bfloat16.
+template <int D, bool F8 = false>
 struct Tc2Layout {
-  static constexpr uint32_t kTileBytes = 128 * D * 2;  // a 128-row Q, K or V tile
-  static constexpr int kKStages = D == 128 ? 3 : 6;
-  static constexpr int kVStages = D == 128 ? 2 : 6;
-  static constexpr int kChunks = D / 64;
+  static constexpr int kElem = F8 ? 1 : 2;                  // bytes per element
+  static constexpr uint32_t kTileBytes = 128 * D * kElem;  // a 128-row Q, K or V tile
+  static constexpr int kKStages = F8 ? 6 : (D == 128 ? 3 : 6);
+  static constexpr int kVStages = F8 ? 6 : (D == 128 ? 2 : 6);
+  static constexpr int kChunks = D * kElem / 128;          // 128-byte column chunks of a row
+  static constexpr int kChunkElems = 128 / kElem;          // elements per chunk (TMA box width)
   static constexpr uint32_t kQOff = 0;  // Q_A, Q_B
   static constexpr uint32_t kKOff = 2 * kTileBytes;
   static constexpr uint32_t kVOff = kKOff + kKStages * kTileBytes;
@@ -108,14 +111,18 @@ __device__ __forceinline__ void tc2_mask_after(uint32_t (&r)[32], int c0, int li
 
 // grid.x = B * H * ceil(nb / 2) for block_size 128, B * H * nb for 256.
 // kCausal: key tokens after the query token are masked (kFlagCausal).
-template <int D, bool kCausal>
+template <int D, bool kCausal, bool kF8 = false>
 __global__ void __launch_bounds__(kTc2Threads, 1)
     sparse_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v,
                            const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ o, int N,
                            int H, int Hkv, int bs, int k, float scale_log2) {
-  using L = Tc2Layout<D>;
+  using L = Tc2Layout<D, kF8>;
+  // MMA steps: K = 32 bytes of the row per instruction (16 bf16 or 32 e4m3)
+  constexpr int kStepsS = D * L::kElem / 32;
+  constexpr int kKeysPerStep = 32 / L::kElem;
+  constexpr int kStepsPV = 128 / kKeysPerStep;
   constexpr int KS = L::kKStages, VS = L::kVStages;
   extern __shared__ __align__(1024) unsigned char tc2_raw[];
   // swizzled tiles need 1024-byte alignment and the layout has no slack
@@ -240,7 +247,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
           for (int hh = 0; hh < 2; ++hh)
             for (int c = 0; c < L::kChunks; ++c)
               tma_load_4d(smem + L::kQOff + x * L::kTileBytes + c * (128 * 128) + hh * 64 * 128,
-                          &tm_q, &bar.q_full, c * 64, qh[x], row0[x] + hh * 64, b, stream);
+                          &tm_q, &bar.q_full, c * L::kChunkElems, qh[x], row0[x] + hh * 64, b, stream);
       }
       for (int n = 0; n < nloads && ok; ++n) {
         const int s = n % S, use = n / S;
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         for (int hf = 0; hf < 2; ++hf)
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(smem + ring + s * L::kTileBytes + c * (128 * 128) + hf * 64 * 128, map,
-                        &full[s], c * 64, g, r[hf], b, keep);
+                        &full[s], c * L::kChunkElems, g, r[hf], b, keep);
         issued[s] = use + 1;
       }
       if (is_k) mbar_wait_teardown(&bar.q_full, 0);
@@ -274,8 +281,9 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     // by the softmax warps, which see each S complete).
     if (lane == 0) {
       constexpr uint32_t kSBO = 1024;  // 8 rows x 128 bytes
-      const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);  // P from TMEM, V MN-major
+      const uint32_t idesc_s = kF8 ? idesc_e4m3_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 128, 0, 0);
+      // P from TMEM, V MN-major
+      const uint32_t idesc_pv = kF8 ? idesc_e4m3_f32(128, D, 0, 1) : idesc_bf16_f32(128, D, 0, 1);
       const uint64_t dq0 = smem_desc_sw128(sbase + L::kQOff, 16, kSBO);
       const uint64_t dk0 = smem_desc_sw128(sbase + L::kKOff, 16, kSBO);
       const uint64_t dv0 = smem_desc_sw128(sbase + L::kVOff, 128 * 128, kSBO);
@@ -297,9 +305,12 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         tc_fence_after();
         const uint64_t dq = dq0 + x * kTileStep, dk = dk0 + (n % KS) * kTileStep;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < kStepsS; ++kk) {
           const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
-          mma_bf16_ss(tmem + L::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
+          if (kF8)
+            mma_f8_ss(tmem + L::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
+          else
+            mma_bf16_ss(tmem + L::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bar.s_full[x]);
       }
@@ -323,17 +334,25 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
           const uint64_t dv = dv0 + (nv % VS) * kTileStep;
           const uint32_t a_tmem = tmem + L::col_s(x);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts(tmem + L::col_o(x), a_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv,
-                        (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kStepsPV; ++kk) {
+            // kKeysPerStep keys: 8 TMEM columns of P, kKeysPerStep 128-byte rows of V
+            const uint64_t bv = dv + ((kk * kKeysPerStep * 128) >> 4);
+            if (kF8)
+              mma_f8_ts(tmem + L::col_o(x), a_tmem + kk * 8, bv, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+            else
+              mma_bf16_ts(tmem + L::col_o(x), a_tmem + kk * 8, bv, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          }
           // the V ring is shallow, so its entry is freed as soon as the product is done
           if (last_user) mma_commit(&bar.v_empty[nv % VS]);
           if (more) {
             const uint64_t dq = dq0 + x * kTileStep, dk = dk0 + (nk % KS) * kTileStep;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
+            for (int kk = 0; kk < kStepsS; ++kk) {
               const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
-              mma_bf16_ss(tmem + L::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
+              if (kF8)
+                mma_f8_ss(tmem + L::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
+              else
+                mma_bf16_ss(tmem + L::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
             }
             mma_commit(&bar.s_full[x]);
           } else {
@@ -415,9 +434,9 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
       // P = exp2(S * scale_log2 - m) for key pairs with two-wide float32
       // instructions; one pair in four takes the polynomial exp2 on the FMA
       // pipe (the split measured fastest: the softmax is bound by issue slots
-      // more than by MUFU). P is stored as packed bf16 over the first 64
-      // columns of S.
-      uint32_t pa[32], pb[32];
+      // more than by MUFU). P is stored over the first columns of S: packed
+      // bf16, two per column (64 columns), or e4m3, four per column (32).
+      uint32_t pa[32], pb[kF8 ? 1 : 32];
       uint64_t ps[4] = {0, 0, 0, 0};
       {
         const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m_new, -m_new);
@@ -435,15 +454,23 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
           ps[pr % 4] = f2_add(ps[pr % 4], p2);
           float p0, p1;
           f2_split(p2, p0, p1);
-          if (pr < 32)
+          if (kF8) {
+            // four e4m3 per 32-bit column, the lowest byte the lowest key
+            const uint32_t h16 = pack_e4m3x2(p0, p1);
+            if (pr % 2 == 0)
+              pa[pr / 2] = h16;
+            else
+              pa[pr / 2] |= h16 << 16;
+          } else if (pr < 32) {
             pa[pr] = pack_bf16x2(p0, p1);
-          else
+          } else {
             pb[pr - 32] = pack_bf16x2(p0, p1);
+          }
         }
       }
 #undef BSA_S
       tmem_st32(scol, pa);
-      tmem_st32(scol + 32, pb);
+      if constexpr (!kF8) tmem_st32(scol + 32, pb);
       tmem_wait_st();
       {
         float a0, a1;

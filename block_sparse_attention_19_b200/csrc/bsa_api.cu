@@ -81,7 +81,8 @@ bsa_status check_heads(int H, int Hkv) {
 }
 
 bsa_status check_dtype(bsa_dtype dt) {
-  if (dt != BSA_F32 && dt != BSA_BF16) return fail(BSA_ERR_UNSUPPORTED, "dtype %d", static_cast<int>(dt));
+  if (dt != BSA_F32 && dt != BSA_BF16 && dt != BSA_E4M3)
+    return fail(BSA_ERR_UNSUPPORTED, "dtype %d", static_cast<int>(dt));
   return BSA_OK;
 }
 
@@ -118,20 +119,24 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [B, N, H, D] bf16 tensor as a 4-D TMA map {D, H, N, B}; box = 64 columns x
-// 1 head x 64 rows x 1 batch, 128-byte swizzle (the UMMA K-/MN-major layout).
-bsa_status make_bnhd_map(CUtensorMap* map, const void* base, int B, int N, int H, int D) {
+// [B, N, H, D] bf16 (or e4m3 with e4m3 = true) tensor as a 4-D TMA map
+// {D, H, N, B}; box = 128 bytes of a row (64 bf16 or 128 e4m3 columns) x 1
+// head x 64 rows x 1 batch, 128-byte swizzle (the UMMA K-/MN-major layout).
+bsa_status make_bnhd_map(CUtensorMap* map, const void* base, int B, int N, int H, int D,
+                         bool e4m3 = false) {
   auto encode = tensor_map_encoder();
   if (!encode) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t es = e4m3 ? 1 : 2;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
-                           static_cast<cuuint64_t>(N) * H * D * 2};
-  cuuint32_t box[4] = {64, 1, 64, 1};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * es, static_cast<cuuint64_t>(H) * D * es,
+                           static_cast<cuuint64_t>(N) * H * D * es};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / es), 1, 64, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
-                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = encode(map, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return BSA_OK;
 }
@@ -140,7 +145,7 @@ bsa_status make_bnhd_map(CUtensorMap* map, const void* base, int B, int N, int H
 
 bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int ntasks, int B,
                        int N, int H, int D, int bs, bsa_dtype dt, cudaStream_t st) {
-  const int V = dt == BSA_F32 ? 4 : 8;
+  const int V = dt == BSA_F32 ? 4 : (dt == BSA_E4M3 ? 16 : 8);  // elements per 16 bytes
   const int C = H * D / V;
   const int cw = bsa::pool_column_group(C);
   const long grid = static_cast<long>(ntasks) * B * (N / bs) * (C / cw);
@@ -148,6 +153,8 @@ bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int
   bsa::PoolTask t0{x0, p0}, t1{x1 ? x1 : x0, p1 ? p1 : p0};
   if (dt == BSA_F32)
     bsa::block_pool_kernel<float><<<static_cast<unsigned>(grid), bsa::kPoolThreads, 0, st>>>(t0, t1, B, N, H, D, bs, cw);
+  else if (dt == BSA_E4M3)
+    bsa::block_pool_kernel<__nv_fp8_e4m3><<<static_cast<unsigned>(grid), bsa::kPoolThreads, 0, st>>>(t0, t1, B, N, H, D, bs, cw);
   else
     bsa::block_pool_kernel<__nv_bfloat16><<<static_cast<unsigned>(grid), bsa::kPoolThreads, 0, st>>>(t0, t1, B, N, H, D, bs, cw);
   cudaError_t e = cudaGetLastError();
@@ -302,28 +309,28 @@ bsa_status launch_attn_tc(const void* q, const void* k, const void* v, const int
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc_kernel launch");
 }
 
-template <int D, bool kCausal>
+template <int D, bool kCausal, bool kF8>
 bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                               int B, int N, int H, int Hkv, int bs, int kk, float scale,
                               cudaStream_t st) {
-  using L = bsa::Tc2Layout<D>;
+  using L = bsa::Tc2Layout<D, kF8>;
   CUtensorMap mq, mk, mv;
   bsa_status s;
-  if ((s = make_bnhd_map(&mq, q, B, N, H, D)) != BSA_OK) return s;
-  if ((s = make_bnhd_map(&mk, k, B, N, Hkv, D)) != BSA_OK) return s;
-  if ((s = make_bnhd_map(&mv, v, B, N, Hkv, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mq, q, B, N, H, D, kF8)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mk, k, B, N, Hkv, D, kF8)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mv, v, B, N, Hkv, D, kF8)) != BSA_OK) return s;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_tc2_kernel<D, kCausal>,
+    cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_tc2_kernel<D, kCausal, kF8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return cuda_fail(e, "tc2 smem attribute");
     // The kernel moves registers between warp groups (setmaxnreg); an increase
     // that the launch allocation cannot cover would wait forever, so refuse
     // to launch unless the compiled register count covers the split.
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, bsa::sparse_attn_tc2_kernel<D, kCausal>);
+    e = cudaFuncGetAttributes(&fa, bsa::sparse_attn_tc2_kernel<D, kCausal, kF8>);
     if (e != cudaSuccess) return cuda_fail(e, "tc2 attributes");
     if (fa.numRegs < static_cast<int>(bsa::kTc2LaunchRegs))
       return fail(BSA_ERR_UNSUPPORTED, "attention kernel built with %d registers/thread, its register split needs %u",
@@ -338,19 +345,19 @@ bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const
                                : static_cast<long>(B) * H * (bs == 256 ? nb : (nb + 1) / 2);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   const float scale_log2 = scale * 1.4426950408889634f;
-  bsa::sparse_attn_tc2_kernel<D, kCausal><<<static_cast<unsigned>(grid), bsa::kTc2Threads, L::kBytes, st>>>(
+  bsa::sparse_attn_tc2_kernel<D, kCausal, kF8><<<static_cast<unsigned>(grid), bsa::kTc2Threads, L::kBytes, st>>>(
       mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, Hkv, bs, kk, scale_log2);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc2_kernel launch");
 }
 
-template <int D>
+template <int D, bool kF8 = false>
 bsa_status launch_attn_tc2(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                            int B, int N, int H, int Hkv, int bs, int kk, float scale, unsigned flags,
                            cudaStream_t st) {
   return (flags & BSA_FLAG_CAUSAL)
-             ? launch_attn_tc2_as<D, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, st)
-             : launch_attn_tc2_as<D, false>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, st);
+             ? launch_attn_tc2_as<D, true, kF8>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, st)
+             : launch_attn_tc2_as<D, false, kF8>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, st);
 }
 
 bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
@@ -362,6 +369,11 @@ bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_
     float* fo = static_cast<float*>(o);
     return D == 64 ? launch_attn_simt<64>(fq, fk, fv, idx, fo, B, N, H, Hkv, bs, kk, scale, flags, st)
                    : launch_attn_simt<128>(fq, fk, fv, idx, fo, B, N, H, Hkv, bs, kk, scale, flags, st);
+  }
+  if (dt == BSA_E4M3) {
+    if (D != 128 || bs == 64)
+      return fail(BSA_ERR_UNSUPPORTED, "e4m3 inputs need D = 128 and block_size 128 or 256");
+    return launch_attn_tc2<128, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, st);
   }
   if (bs == 64)
     return D == 64 ? launch_attn_tc<64, 64>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, st)

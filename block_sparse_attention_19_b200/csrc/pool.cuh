@@ -12,6 +12,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 namespace bsa {
@@ -44,6 +45,24 @@ struct Vec16<__nv_bfloat16> {
     for (int t = 0; t < 4; ++t) {
       acc[2 * t] += __uint_as_float(w[t] << 16);
       acc[2 * t + 1] += __uint_as_float(w[t] & 0xFFFF0000u);
+    }
+  }
+};
+
+template <>
+struct Vec16<__nv_fp8_e4m3> {
+  static constexpr int kN = 16;
+  __device__ __forceinline__ static void add(float* acc, const uint4& u) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      __nv_fp8x4_e4m3 x;
+      x.__x = w[t];
+      const float4 f = static_cast<float4>(x);  // exact: byte 0 -> .x
+      acc[4 * t] += f.x;
+      acc[4 * t + 1] += f.y;
+      acc[4 * t + 2] += f.z;
+      acc[4 * t + 3] += f.w;
     }
   }
 };
@@ -106,7 +125,7 @@ __global__ void __launch_bounds__(kPoolThreads)
   }
 
   // combine the row groups
-  __shared__ float part[kPoolThreads * 8];
+  __shared__ float part[kPoolThreads * V];
   if (rg < G) {
 #pragma unroll
     for (int e = 0; e < V; ++e) part[(rg * cw + col) * V + e] = acc[e];

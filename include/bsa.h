@@ -55,7 +55,17 @@ typedef enum {
 
 typedef enum {
   BSA_F32 = 0, /* float32 q/k/v/o; attention in float32 on CUDA cores */
-  BSA_BF16 = 1 /* bfloat16 q/k/v/o; attention on tcgen05 tensor cores, float32 accumulate */
+  BSA_BF16 = 1, /* bfloat16 q/k/v/o; attention on tcgen05 tensor cores, float32 accumulate */
+  /* FP8 E4M3 q/k/v with bfloat16 o (page "2026 新一代卷积与 Transformer 网络架构",
+   * section "基准测试": SparseFormer run in FP8; its closing advice: use FP8
+   * tensor cores). The stored e4m3 values are the inputs (a caller with
+   * scaled FP8 folds the q and k scales into `scale` and multiplies o by the
+   * v scale). Both products run as tcgen05 kind::f8f6f4 with float32
+   * accumulation; the softmax weights P are rounded to e4m3 (round to
+   * nearest, saturating) for the P.V product, the row sums use float32 P.
+   * Supported for D = 128 and block_size 128 or 256 (else
+   * BSA_ERR_UNSUPPORTED). */
+  BSA_E4M3 = 2
 } bsa_dtype;
 
 /* Number of kept key blocks: floor(topk_ratio * nb) evaluated in IEEE double,

@@ -1,0 +1,97 @@
+"""GPU parity of the FP8 (E4M3) inputs against the float64 oracle.
+
+Reading (page "2026 新一代卷积与 Transformer 网络架构", section "基准测试": SparseFormer
+run in FP8; closing advice: use FP8 tensor cores): q, k, v are e4m3 values
+and the method computed on them is unchanged; the oracle runs on their exact
+values. The GPU path computes both products as tcgen05 kind::f8f6f4 with
+float32 accumulation and rounds the softmax weights P to e4m3 for the P.V
+product (row sums from float32 P); the output is bfloat16.
+
+Tolerance, from that arithmetic: rounding P to e4m3 changes each weight by
+at most 2^-4 of itself in e4m3's normal range (P >= 2^-6 of the row's running
+max) and by at most the weight itself below it, so per output element
+|d| <= 2^-4 (sum_t p_t |v_t|) / l + (sum over the small weights) / l + the
+bfloat16 rounding of o. The first term is computed here exactly with the
+oracle run on |v| (same weights); the small-weight term and the rounding are
+covered by an absolute 2^-8 * max|v| and a relative 2^-8 |o|. Over a whole
+output the weights' rounding errors (uniform, at most 2^-4 of each weight)
+have an rms of 2^-4 / sqrt(3) = 0.036 of the weights, and o's error is a
+weighted combination of them: relative L2 <= 0.036. Index lists follow the
+near-tie rule (pooling reads the exact e4m3 values).
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from test_causal import accept_causal_rows
+from test_parity import _host, accept_index_rows, gpu_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bsa():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    import block_sparse_attention_19_b200 as m
+
+    return m
+
+
+def check_fp8_output(o_gpu, o_ref, o_abs, vmax):
+    d = np.abs(o_gpu - o_ref)
+    bound = 2.0 ** -4 * o_abs + 2.0 ** -8 * vmax + 2.0 ** -8 * np.abs(o_ref)
+    rel = np.linalg.norm(o_gpu - o_ref) / np.linalg.norm(o_ref)
+    print(f"fp8: max|d| {d.max():.3g}, max|d|/bound {(d / bound).max():.3g}, rel L2 {rel:.3g}")
+    assert np.all(d <= bound), f"max|d|/bound = {(d / bound).max()}"
+    assert rel <= 2.0 ** -4 / np.sqrt(3.0), f"rel L2 = {rel}"
+
+
+CASES = [  # (B, N, H, H_kv, block_size, ratio, causal)
+    (1, 2048, 2, 2, 128, 0.25, False),
+    (1, 2048, 4, 2, 128, 0.3, False),   # grouped queries, heads paired in a CTA
+    (1, 1920, 2, 2, 128, 0.4, True),    # causal, odd nb
+    (1, 4096, 2, 2, 256, 0.3, False),   # block_size 256
+    (1, 1024, 2, 2, 128, 1.0, False),   # k = nb
+]
+
+
+@pytest.mark.parametrize("ci", range(len(CASES)))
+def test_fp8_full_path(bsa, oracle_mod, ci):
+    B, N, H, Hkv, bs, ratio, causal = CASES[ci]
+    cfg = W.Config(f"fp8{ci}", B, N, H, 128, bs, ratio, "e4m3", 1.0, 950 + ci, None, H_kv=Hkv)
+    q, k, v = W.make_inputs(cfg, device="cuda")
+    assert q.dtype == torch.float8_e4m3fn
+    flags = bsa.BSA_FLAG_CAUSAL if causal else 0
+    ws = torch.empty(bsa.bsa_forward_workspace_bytes(B, N, H, 128, bs, ratio, H_kv=Hkv), device="cuda",
+                     dtype=torch.uint8)
+    o = bsa.bsa_forward(q, k, v, bs, ratio, workspace=ws, flags=flags)
+    torch.cuda.synchronize()
+    assert bsa.bsa_device_error() == 0 and o.dtype == torch.bfloat16
+    _, _, idx_g = bsa.workspace_views(ws, B, N, H, 128, bs, ratio, H_kv=Hkv)
+    qa, ka, va = _host(q), _host(k), _host(v)
+    ref = oracle_mod.forward_gqa(qa, ka, va, bs, ratio, causal=causal)
+    g = idx_g.cpu().numpy()
+    if causal:
+        accept_causal_rows(g, ref["scores"], cfg.k, ref["idx"], False)
+    else:
+        accept_index_rows(g, ref["scores"], cfg.k, ref["idx"])
+    gq = np.repeat(g, H // Hkv, axis=1)
+    o_ref = oracle_mod.sparse_attn_gqa(qa, ka, va, gq, bs, causal=causal)
+    # sum_t p_t |v_t| / l: the oracle on the same (exact) q, k with |v| as values
+    q64, k64 = (x.to(torch.float64).cpu().numpy() for x in (q, k))
+    vabs = np.abs(v.to(torch.float64).cpu().numpy())
+    o_abs = oracle_mod.sparse_attn_gqa(q64, k64, vabs, gq, bs, causal=causal)
+    rows = np.broadcast_to(np.arange(cfg.nb, dtype=np.int32), (B, H, cfg.nb)).copy()
+    check_fp8_output(gpu_rows(o, rows, bs), o_ref, o_abs, vabs.max())
+
+
+def test_fp8_refused_where_unsupported(bsa):
+    """FP8 inputs need D = 128 and block_size 128 or 256."""
+    q = torch.zeros(1, 512, 2, 64, device="cuda", dtype=torch.float8_e4m3fn)
+    with pytest.raises(bsa.BsaError, match="UNSUPPORTED"):
+        bsa.bsa_forward(q, q, q, 128, 0.5)
+    q = torch.zeros(1, 512, 2, 128, device="cuda", dtype=torch.float8_e4m3fn)
+    with pytest.raises(bsa.BsaError, match="UNSUPPORTED"):
+        bsa.bsa_forward(q, q, q, 64, 0.5)

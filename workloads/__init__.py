@@ -29,7 +29,7 @@ class Config:
     D: int
     block_size: int
     topk_ratio: float
-    dtype: str  # "f32" or "bf16"
+    dtype: str  # "f32", "bf16" or "e4m3"
     offset_sigma: float
     seed: int
     sample_blocks: int | None  # query blocks per (b, h) the oracle checks; None = all
@@ -50,11 +50,11 @@ class Config:
 
     @property
     def torch_dtype(self):
-        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+        return {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn}[self.dtype]
 
     @property
     def elem_bytes(self) -> int:
-        return 4 if self.dtype == "f32" else 2
+        return {"f32": 4, "bf16": 2, "e4m3": 1}[self.dtype]
 
     def with_ratio(self, ratio: float) -> "Config":
         return dataclasses.replace(self, topk_ratio=ratio, name=f"{self.name}@{ratio}")
@@ -106,6 +106,8 @@ def to_oracle_array(x: torch.Tensor):
     x = x.detach().cpu().contiguous()
     if x.dtype == torch.bfloat16:
         return x.view(torch.int16).numpy().view("uint16")
+    if x.dtype == torch.float8_e4m3fn:
+        return x.view(torch.uint8).numpy()
     if x.dtype in (torch.float32, torch.float64):
         return x.numpy()
     raise TypeError(f"unsupported dtype {x.dtype}")
