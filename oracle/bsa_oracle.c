@@ -395,3 +395,91 @@ void oracle_sparse_attn_gqa(const void* q, const void* kmat, const void* v, int 
     free(qrow);
   }
 }
+
+/* ------------------------------------------------------------------------
+ * Backward pass. The selection is a set of indices (top-k carries no
+ * gradient), so the gradients are those of the attention with the index
+ * lists held fixed. For each query token n with the kept key tokens T(n) (and
+ * the causal mask when flagged):
+ *   p_t = softmax_t(scale q_n . k_t),  o_n = sum_t p_t v_t,
+ *   D_n = dO_n . o_n,  dP_t = dO_n . v_t,  dS_t = p_t (dP_t - D_n),
+ *   dq_n = scale sum_t dS_t k_t,  dk_t += scale dS_t q_n,  dv_t += p_t dO_n.
+ * dq, dk, dv are [B, N, H, D] float64; do_ is read like q (same dtype).
+ * Parallel over (b, h) only, so every sum has a fixed order.
+ * ------------------------------------------------------------------------ */
+void oracle_sparse_attn_bwd(const void* q, const void* kmat, const void* v, const void* do_, int dtype,
+                            int B, int N, int H, int D, int bs, const int* idx, int k, double scale,
+                            int flags, double* dq, double* dk, double* dv) {
+  int nb = N / bs;
+  long ntok = (long)k * bs;
+  size_t total = (size_t)B * N * H * D;
+  for (size_t e = 0; e < total; ++e) dq[e] = dk[e] = dv[e] = 0.0;
+#pragma omp parallel
+  {
+    double* p = (double*)malloc((size_t)ntok * sizeof(double));
+    int* tok = (int*)malloc((size_t)ntok * sizeof(int));
+    double* qrow = (double*)malloc((size_t)D * sizeof(double));
+    double* dorow = (double*)malloc((size_t)D * sizeof(double));
+    double* orow = (double*)malloc((size_t)D * sizeof(double));
+#pragma omp for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b)
+      for (int h = 0; h < H; ++h) {
+        size_t bh = (size_t)b * H + h;
+        for (int i = 0; i < nb; ++i) {
+          const int* sel = idx + (bh * nb + i) * k;
+          for (int t_q = 0; t_q < bs; ++t_q) {
+            int n = i * bs + t_q;
+            for (int d = 0; d < D; ++d) {
+              qrow[d] = elem(q, dtype, at_bnhd(N, H, D, b, n, h, d));
+              dorow[d] = elem(do_, dtype, at_bnhd(N, H, D, b, n, h, d));
+            }
+            /* the softmax weights over the kept, unmasked key tokens */
+            long cnt = 0;
+            double m = -INFINITY;
+            for (int s = 0; s < k; ++s) {
+              if (sel[s] < 0) continue;
+              for (int u = 0; u < bs; ++u) {
+                int t = sel[s] * bs + u;
+                if ((flags & ORACLE_CAUSAL) && t > n) continue;
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) dot += qrow[d] * elem(kmat, dtype, at_bnhd(N, H, D, b, t, h, d));
+                p[cnt] = scale * dot;
+                tok[cnt] = t;
+                if (p[cnt] > m) m = p[cnt];
+                ++cnt;
+              }
+            }
+            double z = 0.0;
+            for (long c = 0; c < cnt; ++c) {
+              p[c] = exp(p[c] - m);
+              z += p[c];
+            }
+            for (long c = 0; c < cnt; ++c) p[c] /= z;
+            /* o_n and D_n = dO_n . o_n */
+            for (int d = 0; d < D; ++d) orow[d] = 0.0;
+            for (long c = 0; c < cnt; ++c)
+              for (int d = 0; d < D; ++d) orow[d] += p[c] * elem(v, dtype, at_bnhd(N, H, D, b, tok[c], h, d));
+            double Dn = 0.0;
+            for (int d = 0; d < D; ++d) Dn += dorow[d] * orow[d];
+            /* dS_t, then the three gradients */
+            for (long c = 0; c < cnt; ++c) {
+              int t = tok[c];
+              double dP = 0.0;
+              for (int d = 0; d < D; ++d) dP += dorow[d] * elem(v, dtype, at_bnhd(N, H, D, b, t, h, d));
+              double dS = p[c] * (dP - Dn);
+              for (int d = 0; d < D; ++d) {
+                dq[at_bnhd(N, H, D, b, n, h, d)] += scale * dS * elem(kmat, dtype, at_bnhd(N, H, D, b, t, h, d));
+                dk[at_bnhd(N, H, D, b, t, h, d)] += scale * dS * qrow[d];
+                dv[at_bnhd(N, H, D, b, t, h, d)] += p[c] * dorow[d];
+              }
+            }
+          }
+        }
+      }
+    free(p);
+    free(tok);
+    free(qrow);
+    free(dorow);
+    free(orow);
+  }
+}

@@ -519,3 +519,62 @@ def test_e4m3_inputs_are_their_exact_values(oracle_mod):
         b = oracle_mod.forward(*f64, bs, 0.375, causal=causal)
         np.testing.assert_array_equal(a["idx"], b["idx"])
         np.testing.assert_array_equal(a["o"], b["o"])
+
+
+# ---------------------------------------------------------------- backward pass
+# Reading: the top-k indices carry no gradient, so the backward is the
+# gradient of the attention over the kept blocks with the lists held fixed.
+
+def _dense_mask(idx, bs, N, causal):
+    B, H, nb, _ = idx.shape
+    blk = np.zeros((B, H, nb, nb), bool)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nb):
+                row = idx[b, h, i]
+                blk[b, h, i, row[row >= 0]] = True
+    m = torch.from_numpy(blk).repeat_interleave(bs, 2).repeat_interleave(bs, 3)
+    if causal:
+        m &= torch.ones(N, N, dtype=torch.bool).tril()
+    return m
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_matches_torch_autograd_of_masked_dense_attention(oracle_mod, causal):
+    """float64 torch autograd of SDPA under the block (and causal) mask."""
+    B, N, H, D, bs = 2, 48, 2, 8, 6
+    q, k, v, do = (_rand((B, N, H, D), s, bs=bs) for s in (160, 161, 162, 163))
+    r = oracle_mod.forward(q, k, v, bs, 0.4, causal=causal)
+    dq, dk, dv = oracle_mod.sparse_attn_bwd(q, k, v, do, r["idx"], bs, causal=causal)
+    t = lambda x: torch.from_numpy(x).permute(0, 2, 1, 3).clone().requires_grad_(True)
+    tq, tk, tv = t(q), t(k), t(v)
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv,
+                                                           attn_mask=_dense_mask(r["idx"], bs, N, causal))
+    out.backward(torch.from_numpy(do).permute(0, 2, 1, 3))
+    for got, ref in ((dq, tq), (dk, tk), (dv, tv)):
+        np.testing.assert_allclose(got, ref.grad.permute(0, 2, 1, 3).numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_backward_matches_finite_differences(oracle_mod):
+    """Central differences of sum(o * dO) on a tiny case, for a few entries of
+    q, k and v (the selection is held fixed)."""
+    B, N, H, D, bs = 1, 16, 1, 4, 4
+    q, k, v, do = (_rand((B, N, H, D), s, bs=bs) for s in (170, 171, 172, 173))
+    idx = oracle_mod.forward(q, k, v, bs, 0.5)["idx"]
+    dq, dk, dv = oracle_mod.sparse_attn_bwd(q, k, v, do, idx, bs)
+
+    def loss(qq, kk, vv):
+        o = oracle_mod.o_to_bnhd(oracle_mod.sparse_attn(qq, kk, vv, idx, bs))
+        return float((o * do).sum())
+
+    eps = 1e-6
+    rng = np.random.default_rng(174)
+    for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(4):
+            pos = tuple(int(rng.integers(0, s)) for s in arr.shape)
+            plus, minus = arr.copy(), arr.copy()
+            plus[pos] += eps
+            minus[pos] -= eps
+            args = lambda x: [x if n == name else a for n, a in (("q", q), ("k", k), ("v", v))]
+            fd = (loss(*args(plus)) - loss(*args(minus))) / (2 * eps)
+            assert abs(fd - grad[pos]) <= 1e-7 * max(1.0, abs(fd)), (name, pos, fd, grad[pos])
