@@ -111,13 +111,14 @@ __device__ __forceinline__ void tc2_mask_after(uint32_t (&r)[32], int c0, int li
 
 // grid.x = B * H * ceil(nb / 2) for block_size 128, B * H * nb for 256.
 // kCausal: key tokens after the query token are masked (kFlagCausal).
+// lse (optional, [B, H, N] float32): ln sum_t exp(scale q_n . k_t) per row.
 template <int D, bool kCausal, bool kF8 = false>
 __global__ void __launch_bounds__(kTc2Threads, 1)
     sparse_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v,
                            const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ o, int N,
-                           int H, int Hkv, int bs, int k, float scale_log2) {
+                           int H, int Hkv, int bs, int k, float scale_log2, float* __restrict__ lse) {
   using L = Tc2Layout<D, kF8>;
   // MMA steps: K = 32 bytes of the row per instruction (16 bf16 or 32 e4m3)
   constexpr int kStepsS = D * L::kElem / 32;
@@ -487,6 +488,8 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
       tc_fence_after();
       const float inv = 1.0f / l_run;
       const long n = row0[x] + row;
+      // natural log of the row's softmax denominator (m_run is in log2 units)
+      if (lse) lse[(static_cast<long>(b) * H + qh[x]) * N + n] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
       __nv_bfloat16* orow = o + ((static_cast<long>(b) * N + n) * H + qh[x]) * D;
       uint32_t r[32];
 #pragma unroll

@@ -16,6 +16,7 @@
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "attn_tc2.cuh"
+#include "bwd.cuh"
 #include "bsa.h"
 #include "bsa_ptx.cuh"
 #include "pool.cuh"
@@ -312,7 +313,7 @@ bsa_status launch_attn_tc(const void* q, const void* k, const void* v, const int
 template <int D, bool kCausal, bool kF8>
 bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                               int B, int N, int H, int Hkv, int bs, int kk, float scale,
-                              cudaStream_t st) {
+                              float* lse, cudaStream_t st) {
   using L = bsa::Tc2Layout<D, kF8>;
   CUtensorMap mq, mk, mv;
   bsa_status s;
@@ -346,7 +347,7 @@ bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   const float scale_log2 = scale * 1.4426950408889634f;
   bsa::sparse_attn_tc2_kernel<D, kCausal, kF8><<<static_cast<unsigned>(grid), bsa::kTc2Threads, L::kBytes, st>>>(
-      mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, Hkv, bs, kk, scale_log2);
+      mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, Hkv, bs, kk, scale_log2, lse);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc2_kernel launch");
 }
@@ -354,15 +355,15 @@ bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const
 template <int D, bool kF8 = false>
 bsa_status launch_attn_tc2(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                            int B, int N, int H, int Hkv, int bs, int kk, float scale, unsigned flags,
-                           cudaStream_t st) {
+                           float* lse, cudaStream_t st) {
   return (flags & BSA_FLAG_CAUSAL)
-             ? launch_attn_tc2_as<D, true, kF8>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, st)
-             : launch_attn_tc2_as<D, false, kF8>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, st);
+             ? launch_attn_tc2_as<D, true, kF8>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, st)
+             : launch_attn_tc2_as<D, false, kF8>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, st);
 }
 
 bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                        int B, int N, int H, int Hkv, int D, int bs, int kk, float scale, bsa_dtype dt,
-                       unsigned flags, cudaStream_t st) {
+                       unsigned flags, cudaStream_t st, float* lse = nullptr) {
   if (dt == BSA_F32) {
     const float *fq = static_cast<const float*>(q), *fk = static_cast<const float*>(k),
                 *fv = static_cast<const float*>(v);
@@ -373,13 +374,90 @@ bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_
   if (dt == BSA_E4M3) {
     if (D != 128 || bs == 64)
       return fail(BSA_ERR_UNSUPPORTED, "e4m3 inputs need D = 128 and block_size 128 or 256");
-    return launch_attn_tc2<128, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, st);
+    return launch_attn_tc2<128, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st);
   }
   if (bs == 64)
     return D == 64 ? launch_attn_tc<64, 64>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, st)
                    : launch_attn_tc<128, 64>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, st);
-  return D == 64 ? launch_attn_tc2<64>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, st)
-                 : launch_attn_tc2<128>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, st);
+  return D == 64 ? launch_attn_tc2<64>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st)
+                 : launch_attn_tc2<128>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st);
+}
+
+// Backward: transpose of the selection (bit matrix), D_n, dQ, dK/dV.
+struct BwdWorkspace {
+  uint32_t* mask;  // [B, H, nb, ceil(nb / 32)]
+  float* dsum;     // [B, H, N]
+  size_t bytes;
+};
+
+BwdWorkspace bwd_workspace_layout(void* base, int B, int N, int H, int bs) {
+  const size_t nb = static_cast<size_t>(N / bs), words = (nb + 31) / 32;
+  const size_t mb = align256(static_cast<size_t>(B) * H * nb * words * sizeof(uint32_t));
+  const size_t db = align256(static_cast<size_t>(B) * H * N * sizeof(float));
+  unsigned char* p = static_cast<unsigned char*>(base);
+  BwdWorkspace w;
+  w.mask = reinterpret_cast<uint32_t*>(p);
+  w.dsum = reinterpret_cast<float*>(p + mb);
+  w.bytes = mb + db;
+  return w;
+}
+
+template <int D, bool kCausal>
+bsa_status launch_bwd_as(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const int32_t* idx, const float* lse, const BwdWorkspace& w, void* dq, void* dk,
+                         void* dv, int B, int N, int H, int bs, int kk, float scale, cudaStream_t st) {
+  using L = bsa::BwdLayout<D>;
+  CUtensorMap mq, mk, mv, mdo;
+  bsa_status s;
+  if ((s = make_bnhd_map(&mq, q, B, N, H, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mk, k, B, N, H, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mv, v, B, N, H, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mdo, dO, B, N, H, D)) != BSA_OK) return s;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(bsa::bwd_dq_kernel<D, kCausal>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bsa::bwd_dkdv_kernel<D, kCausal>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               L::kBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "backward smem attribute");
+    attr_set[dev] = true;
+  }
+  const int nb = N / bs, words = (nb + 31) / 32;
+  // 1. the transpose of the selection, as bits
+  cudaError_t e = cudaMemsetAsync(w.mask, 0, static_cast<size_t>(B) * H * nb * words * sizeof(uint32_t), st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward mask clear");
+  const long entries = static_cast<long>(B) * H * nb * kk;
+  bsa::bwd_mask_kernel<<<static_cast<unsigned>((entries + 255) / 256), 256, 0, st>>>(idx, w.mask, entries, nb,
+                                                                                     kk, words);
+  // 2. D_n = dO_n . o_n
+  const long rows = static_cast<long>(B) * N * H;
+  bsa::bwd_rowdot_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), w.dsum, rows, N, H, D);
+  // 3. dQ per query tile, 4. dK and dV per key tile
+  const long tiles = static_cast<long>(B) * H * nb * (bs / 128);
+  if (tiles > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "backward grid too large");
+  const float scale_log2 = scale * 1.4426950408889634f;
+  bsa::bwd_dq_kernel<D, kCausal><<<static_cast<unsigned>(tiles), bsa::kBwdThreads, L::kBytes, st>>>(
+      mq, mk, mv, mdo, idx, lse, w.dsum, static_cast<__nv_bfloat16*>(dq), N, H, bs, kk, scale, scale_log2);
+  bsa::bwd_dkdv_kernel<D, kCausal><<<static_cast<unsigned>(tiles), bsa::kBwdThreads, L::kBytes, st>>>(
+      mq, mk, mv, mdo, w.mask, lse, w.dsum, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), N,
+      H, bs, scale, scale_log2);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "backward launches");
+}
+
+bsa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                      const int32_t* idx, const float* lse, const BwdWorkspace& w, void* dq, void* dk, void* dv,
+                      int B, int N, int H, int D, int bs, int kk, float scale, unsigned flags, cudaStream_t st) {
+  const bool causal = (flags & BSA_FLAG_CAUSAL) != 0;
+  if (D == 64)
+    return causal ? launch_bwd_as<64, true>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, bs, kk, scale, st)
+                  : launch_bwd_as<64, false>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, bs, kk, scale, st);
+  return causal ? launch_bwd_as<128, true>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, bs, kk, scale, st)
+                : launch_bwd_as<128, false>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, bs, kk, scale, st);
 }
 
 struct Workspace {
@@ -577,6 +655,72 @@ bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int
                        size_t workspace_bytes, void* stream) {
   return bsa_forward_ex(q, k, v, o, B, N, H, D, block_size, topk_ratio, dt, 0u, workspace,
                         workspace_bytes, stream);
+}
+
+// ---- training: the forward with the row log-sum-exp, and the backward
+
+// The shapes the training entry points cover: bf16, D in {64, 128},
+// block_size 128 or 256, one key/value head per query head.
+bsa_status check_train(int B, int N, int H, int D, int block_size, int kk, bsa_dtype dt, unsigned flags) {
+  bsa_status s;
+  if ((s = check_flags(flags)) != BSA_OK) return s;
+  if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
+  if (dt != BSA_BF16) return fail(BSA_ERR_UNSUPPORTED, "training entry points take bf16");
+  if (block_size == 64) return fail(BSA_ERR_UNSUPPORTED, "training entry points need block_size 128 or 256");
+  const int nb = N / block_size;
+  if (kk < 1 || kk > nb) return fail(BSA_ERR_INVALID_ARG, "k=%d outside [1, nb=%d]", kk, nb);
+  return BSA_OK;
+}
+
+bsa_status bsa_sparse_attn_fwd_train(const void* q, const void* k, const void* v, const int32_t* idx,
+                                     void* o, float* lse, int B, int N, int H, int D, int block_size,
+                                     int kk, float scale, bsa_dtype dt, unsigned flags, void* stream) {
+  bsa_status s;
+  if ((s = check_train(B, N, H, D, block_size, kk, dt, flags)) != BSA_OK) return s;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return fail(BSA_ERR_INVALID_ARG, "scale must be positive and finite");
+  if (!q || !k || !v || !idx || !o || !lse) return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(o) || !aligned16(lse))
+    return fail(BSA_ERR_MISALIGNED, "q, k, v, idx, o or lse");
+  if (o == q || o == k || o == v) return fail(BSA_ERR_INVALID_ARG, "o aliases an input");
+  if ((s = check_device()) != BSA_OK) return s;
+  if ((s = launch_attn(q, k, v, idx, o, B, N, H, H, D, block_size, kk, scale, dt, flags,
+                       static_cast<cudaStream_t>(stream), lse)) != BSA_OK)
+    return s;
+  return ok();
+}
+
+size_t bsa_sparse_attn_bwd_workspace_bytes(int B, int N, int H, int D, int block_size) {
+  if (check_dims(B, N, H, D, block_size) != BSA_OK) return 0;
+  return bwd_workspace_layout(nullptr, B, N, H, block_size).bytes;
+}
+
+bsa_status bsa_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                               const int32_t* idx, const float* lse, void* dq, void* dk, void* dv, int B,
+                               int N, int H, int D, int block_size, int kk, float scale, bsa_dtype dt,
+                               unsigned flags, void* workspace, size_t workspace_bytes, void* stream) {
+  bsa_status s;
+  if ((s = check_train(B, N, H, D, block_size, kk, dt, flags)) != BSA_OK) return s;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return fail(BSA_ERR_INVALID_ARG, "scale must be positive and finite");
+  if (!q || !k || !v || !o || !dO || !idx || !lse || !dq || !dk || !dv)
+    return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  const void* ptrs[] = {q, k, v, o, dO, idx, lse, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(BSA_ERR_MISALIGNED, "a tensor is not 16-byte aligned");
+  const void* outs[] = {dq, dk, dv};
+  const void* ins[] = {q, k, v, o, dO};
+  for (const void* a : outs)
+    for (const void* b : ins)
+      if (a == b) return fail(BSA_ERR_INVALID_ARG, "a gradient aliases an input");
+  const BwdWorkspace w = bwd_workspace_layout(workspace, B, N, H, block_size);
+  if (!workspace || workspace_bytes < w.bytes)
+    return fail(BSA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", w.bytes, workspace ? workspace_bytes : 0);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(BSA_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  if ((s = check_device()) != BSA_OK) return s;
+  if ((s = launch_bwd(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, D, block_size, kk, scale, flags,
+                      static_cast<cudaStream_t>(stream))) != BSA_OK)
+    return s;
+  return ok();
 }
 
 bsa_status bsa_device_error(int* code_out, void* stream) {

@@ -1,0 +1,577 @@
+// bwd.cuh -- backward pass of the attention over the kept blocks.
+//
+// Page "2026 新一代卷积与 Transformer 网络架构" (qqiyuan.cn), section
+// "SparseFormer 注意力实现": step 2 keeps key blocks with torch.topk, whose
+// indices carry no gradient, so the gradients are those of step 3 (the
+// attention over the kept blocks, "从M2.7到M3" §2.1 Softmax(Mask(QK^T/sqrt(d_k)))V)
+// with the index lists held fixed. Per query token n and kept key token t:
+//   p = exp(scale q.k - lse_n), D_n = dO_n . o_n, dP = dO_n . v_t,
+//   dS = p (dP - D_n), dq_n = scale sum_t dS k_t,
+//   dk_t = scale sum_n dS q_n, dv_t = sum_n p dO_n.
+// The forward leaves lse (ln of each row's softmax denominator).
+//
+// Kernels:
+//  * bwd_mask_kernel: the transpose of the selection as a bit matrix
+//    [B, H, nb, ceil(nb / 32)] (bit i of row j: query block i kept key
+//    block j); deterministic (atomicOr of bits).
+//  * bwd_rowdot_kernel: D_n = dO_n . o_n in float32.
+//  * bwd_dq_kernel: one CTA per 128-row query tile walks its kept key tiles:
+//    S = Q K^T and dP = dO V^T (tcgen05, TMEM), then dS (bf16, over S in
+//    TMEM) and dQ += dS K; dQ accumulates in TMEM.
+//  * bwd_dkdv_kernel: one CTA per 128-key tile walks the query tiles that
+//    kept its block (the bit row): S^T = K Q^T and dP^T = V dO^T, then P^T
+//    and dS^T (bf16 over S^T and dP^T) and dV += P^T dO, dK += dS^T Q; all
+//    four products and both accumulators live in TMEM (512 columns).
+// Each CTA has a TMA producer warp, an MMA warp (one issuing thread) and four
+// compute warps (one row per thread); every wait is bounded.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "bsa_ptx.cuh"
+
+namespace bsa {
+
+constexpr int kBwdThreads = 192;  // producer warp, MMA warp, 4 compute warps
+
+// ---------------------------------------------------------------- transpose
+// grid.x = ceil(B * H * nb * k / 256)
+__global__ void bwd_mask_kernel(const int32_t* __restrict__ idx, uint32_t* __restrict__ mask,
+                                long entries, int nb, int k, int words) {
+  const long e = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= entries) return;
+  const int j = __ldg(idx + e);
+  if (j < 0 || j >= nb) return;
+  const long row = e / k;                   // (b, h, i)
+  const int i = static_cast<int>(row % nb);
+  const long bh = row / nb;
+  atomicOr(mask + (bh * nb + j) * words + i / 32, 1u << (i % 32));
+}
+
+// ---------------------------------------------------------------- D_n
+// One warp per row: D_n = sum_d dO[n, d] * o[n, d] (bf16 inputs, float32 sum),
+// written to dsum [B, H, N]. grid.x = ceil(B * N * H / 8), 256 threads.
+__global__ void bwd_rowdot_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+                                  float* __restrict__ dsum, long rows, int N, int H, int D) {
+  const long r = static_cast<long>(blockIdx.x) * 8 + threadIdx.x / 32;  // (b, n, h) row of [B, N, H, D]
+  const int lane = threadIdx.x % 32;
+  if (r >= rows) return;
+  float acc = 0.f;
+  for (int d = lane * 2; d < D; d += 64) {
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(o + r * D + d);
+    const __nv_bfloat162 g = *reinterpret_cast<const __nv_bfloat162*>(dO + r * D + d);
+    acc = fmaf(__low2float(a), __low2float(g), acc);
+    acc = fmaf(__high2float(a), __high2float(g), acc);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) {
+    const int h = static_cast<int>(r % H);
+    const long bn = r / H;
+    const int n = static_cast<int>(bn % N);
+    const long b = bn / N;
+    dsum[(b * H + h) * N + n] = acc;
+  }
+}
+
+// ---------------------------------------------------------------- shared pieces
+template <int D>
+struct BwdLayout {
+  static constexpr uint32_t kTile = 128 * D * 2;  // a 128-row bf16 tile
+  static constexpr int kChunks = D / 64;          // 128-byte column chunks
+  static constexpr uint32_t kOffA = 0;            // dq: Q, dO     dkdv: K, V
+  static constexpr uint32_t kOffRing = 2 * kTile; // dq: K, V x 2  dkdv: Q, dO x 2
+  static constexpr uint32_t kBarOff = kOffRing + 4 * kTile;
+  static constexpr uint32_t kBytes = kBarOff + 256;
+  static_assert(kBytes <= 232448, "shared memory budget");
+};
+
+struct BwdBarriers {
+  uint64_t a_full;        // the two resident tiles
+  uint64_t full[2];       // ring stage holds its two tiles
+  uint64_t empty[2];      // ring stage read by the products
+  uint64_t prod_full;     // phase t: the two score-like products of tile t done
+  uint64_t soft_full;     // phase t: the compute warps stored tile t's bf16 operands
+  uint64_t done;          // the last accumulating products done
+  uint64_t drained;
+  uint32_t tmem_base;
+  int abort;
+  int tiles;  // key tiles (dq) or query tiles (dkdv) this CTA walks
+};
+static_assert(sizeof(BwdBarriers) <= 256, "barrier area");
+
+// First token row of 64-row half hf of tile t of a row of kept blocks:
+// block sel[t / tpb], 128-row part t % tpb.
+__device__ __forceinline__ int bwd_tile_row(const int32_t* sel, int t, int hf, int bs, int nb) {
+  const int tpb = bs / 128;
+  int blk = __ldg(sel + t / tpb);
+  blk = blk < 0 ? 0 : (blk >= nb ? nb - 1 : blk);
+  return blk * bs + (t % tpb) * 128 + hf * 64;
+}
+
+// Loads one 128-row tile (two 64-row boxes per 128-byte chunk) at token row
+// `row` of head h, batch b into `dst`, completing on `bar`.
+template <int D>
+__device__ __forceinline__ void bwd_load_tile(unsigned char* dst, const CUtensorMap* map, uint64_t* bar,
+                                              int h, int row, int b, uint64_t policy) {
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+    for (int c = 0; c < BwdLayout<D>::kChunks; ++c)
+      tma_load_4d(dst + c * (128 * 128) + hf * 64 * 128, map, bar, c * 64, h, row + hf * 64, b, policy);
+}
+
+// 32 bf16 pairs of a row chunk to 16 packed words.
+__device__ __forceinline__ void bwd_pack16(const float (&v)[32], uint32_t (&w)[16]) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+}
+
+// ---------------------------------------------------------------- dQ
+// grid.x = B * H * nb * (bs / 128): one CTA per 128-row query tile, which
+// walks the key tiles of its query block's kept blocks.
+// TMEM: S [0, 128), dP [128, 256), dQ [256, 256 + D).
+template <int D, bool kCausal>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const int32_t* __restrict__ idx, const float* __restrict__ lse,
+                  const float* __restrict__ dsum, __nv_bfloat16* __restrict__ dq, int N, int H, int bs,
+                  int k, float scale, float scale_log2) {
+  using L = BwdLayout<D>;
+  extern __shared__ __align__(1024) unsigned char bwd_raw[];
+  if ((smem_u32(bwd_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) report_error(701);
+    return;
+  }
+  unsigned char* smem = bwd_raw;
+  BwdBarriers& bar = *reinterpret_cast<BwdBarriers*>(smem + L::kBarOff);
+  volatile int* abort_flag = &bar.abort;
+  constexpr uint32_t kColS = 0, kColP = 128, kColQ = 256;
+
+  const int nb = N / bs, tpb = bs / 128;
+  long u = blockIdx.x;
+  const int part = static_cast<int>(u % tpb);
+  u /= tpb;
+  const int i = static_cast<int>(u % nb);
+  u /= nb;
+  const int h = static_cast<int>(u % H);
+  const int b = static_cast<int>(u / H);
+  const long bh = static_cast<long>(b) * H + h;
+  const int qrow0 = i * bs + part * 128;
+  const int32_t* sel = idx + (bh * nb + i) * k;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar.a_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar.full[s], 1);
+      mbar_init(&bar.empty[s], 1);
+    }
+    mbar_init(&bar.prod_full, 1);
+    mbar_init(&bar.soft_full, 4);
+    mbar_init(&bar.done, 1);
+    mbar_init(&bar.drained, 1);
+    bar.abort = 0;
+    bar.tiles = max(index_row_valid(sel, k), 1) * tpb;  // a row of only -1 reads block 0
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bar.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+  const int T = bar.tiles;
+  const uint32_t sbase = smem_u32(smem);
+
+  if (warp == 0) {
+    // ============================================================ TMA producer
+    if (lane == 0) {
+      const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
+      mbar_arrive_expect_tx(&bar.a_full, 2 * L::kTile);
+      bwd_load_tile<D>(smem + L::kOffA, &tm_q, &bar.a_full, h, qrow0, b, stream);
+      bwd_load_tile<D>(smem + L::kOffA + L::kTile, &tm_do, &bar.a_full, h, qrow0, b, stream);
+      int issued[2] = {0, 0};
+      bool ok = true;
+      for (int t = 0; t < T && ok; ++t) {
+        const int s = t & 1, use = t >> 1;
+        const int row = bwd_tile_row(sel, t, 0, bs, nb);
+        if (t >= 2) ok = mbar_wait(&bar.empty[s], (use - 1) & 1, abort_flag, 711);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bar.full[s], 2 * L::kTile);
+        unsigned char* st = smem + L::kOffRing + s * 2 * L::kTile;  // K, then V
+        bwd_load_tile<D>(st, &tm_k, &bar.full[s], h, row, b, keep);
+        bwd_load_tile<D>(st + L::kTile, &tm_v, &bar.full[s], h, row, b, keep);
+        issued[s] = use + 1;
+      }
+      mbar_wait_teardown(&bar.a_full, 0);
+      for (int s = 0; s < 2; ++s)
+        if (issued[s]) mbar_wait_teardown(&bar.full[s], (issued[s] - 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t id_q = idesc_bf16_f32(128, D, 0, 1);  // dS from TMEM, K used MN-major
+      const uint64_t dqd = smem_desc_sw128(sbase + L::kOffA, 16, 1024);
+      const uint64_t ddo = smem_desc_sw128(sbase + L::kOffA + L::kTile, 16, 1024);
+      const uint64_t dring = smem_desc_sw128(sbase + L::kOffRing, 16, 1024);           // K-major
+      const uint64_t dring_mn = smem_desc_sw128(sbase + L::kOffRing, 128 * 128, 1024);  // MN-major
+      constexpr uint64_t kStep = L::kTile >> 4;
+      bool ok = mbar_wait(&bar.a_full, 0, abort_flag, 721);
+      for (int t = 0; t <= T && ok; ++t) {
+        if (t > 0) {
+          // dQ += dS(t-1) K(t-1); dS is bf16 over the first 64 columns of S
+          ok = mbar_wait(&bar.soft_full, (t - 1) & 1, abort_flag, 722);
+          if (!ok) break;
+          tc_fence_after();
+          const int s = (t - 1) & 1;
+          const uint64_t dk = dring_mn + (2 * s) * kStep;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tmem + kColQ, tmem + kColS + kk * 8, dk + ((kk * 16 * 128) >> 4), id_q,
+                        (t > 1 || kk > 0) ? 1u : 0u);
+          mma_commit(&bar.empty[s]);
+        }
+        if (t < T) {
+          // S(t) = Q K(t)^T and dP(t) = dO V(t)^T (issued after dQ(t-1), which
+          // reads the dS these overwrite: the tensor pipe runs them in order)
+          const int s = t & 1;
+          ok = mbar_wait(&bar.full[s], (t >> 1) & 1, abort_flag, 723);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dk = dring + (2 * s) * kStep, dv = dring + (2 * s + 1) * kStep;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+            mma_bf16_ss(tmem + kColS, dqd + off, dk + off, id_s, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+            mma_bf16_ss(tmem + kColP, ddo + off, dv + off, id_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bar.prod_full);
+        }
+      }
+      if (ok) mma_commit(&bar.done);
+      mma_commit(&bar.drained);
+      mbar_wait_teardown(&bar.drained, 0);
+    }
+    __syncwarp();
+  } else {
+    // ============================================================ dS, then the dQ epilogue
+    const int quad = warp % 4;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const long n = qrow0 + row;
+    const float lse2 = __ldg(lse + bh * N + n) * 1.4426950408889634f;  // log2 units
+    const float dn = __ldg(dsum + bh * N + n);
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar.prod_full, t & 1, abort_flag, 731));
+      if (!ok) break;
+      tc_fence_after();
+      // keys c of this tile with kbase + c > n are masked (causal)
+      const int lim = kCausal ? static_cast<int>(n - bwd_tile_row(sel, t, 0, bs, nb)) : (1 << 30);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], pv[32];
+        tmem_ld32(lane_base + kColS + c * 32, sv);
+        tmem_ld32(lane_base + kColP + c * 32, pv);
+        tmem_wait_ld();
+        float ds[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float p = (c * 32 + e > lim) ? 0.f : fast_exp2(fmaf(__uint_as_float(sv[e]), scale_log2, -lse2));
+          ds[e] = p * (__uint_as_float(pv[e]) - dn);
+        }
+        uint32_t w[16];
+        bwd_pack16(ds, w);
+        tmem_st16(lane_base + kColS + c * 16, w);  // over S columns already read
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.soft_full);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.done, 0, abort_flag, 732));
+    if (ok) {
+      tc_fence_after();
+      __nv_bfloat16* out = dq + ((static_cast<long>(b) * N + n) * H + h) * D;
+      uint32_t r[32];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        tmem_ld32(lane_base + kColQ + c * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          uint4 w4;
+          w4.x = pack_bf16x2(__uint_as_float(r[e]) * scale, __uint_as_float(r[e + 1]) * scale);
+          w4.y = pack_bf16x2(__uint_as_float(r[e + 2]) * scale, __uint_as_float(r[e + 3]) * scale);
+          w4.z = pack_bf16x2(__uint_as_float(r[e + 4]) * scale, __uint_as_float(r[e + 5]) * scale);
+          w4.w = pack_bf16x2(__uint_as_float(r[e + 6]) * scale, __uint_as_float(r[e + 7]) * scale);
+          *reinterpret_cast<uint4*>(out + c * 32 + e) = w4;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- dK, dV
+// Query block of the u-th query tile of a bit row (tpb tiles per block):
+// walks the set bits in ascending order. `w` and `cur` carry the position.
+__device__ __forceinline__ int bwd_next_block(const uint32_t* row, int words, int& w, uint32_t& cur) {
+  while (cur == 0 && w + 1 < words) cur = __ldg(row + ++w);
+  const int i = w * 32 + __ffs(cur) - 1;
+  cur &= cur - 1;
+  return i;
+}
+
+// grid.x = B * H * nb * (bs / 128): one CTA per 128-key tile, which walks the
+// query tiles of the query blocks that kept its block (bit row of `mask`).
+// TMEM: S^T [0, 128), dP^T [128, 256), dV [256, 256 + D), dK [256 + D, 256 + 2D).
+template <int D, bool kCausal>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const uint32_t* __restrict__ mask, const float* __restrict__ lse,
+                    const float* __restrict__ dsum, __nv_bfloat16* __restrict__ dk,
+                    __nv_bfloat16* __restrict__ dv, int N, int H, int bs, float scale, float scale_log2) {
+  using L = BwdLayout<D>;
+  static_assert(256 + 2 * D <= 512, "TMEM columns");
+  extern __shared__ __align__(1024) unsigned char bwd_raw[];
+  if ((smem_u32(bwd_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) report_error(702);
+    return;
+  }
+  unsigned char* smem = bwd_raw;
+  BwdBarriers& bar = *reinterpret_cast<BwdBarriers*>(smem + L::kBarOff);
+  volatile int* abort_flag = &bar.abort;
+  constexpr uint32_t kColS = 0, kColP = 128, kColV = 256, kColK = 256 + D;
+
+  const int nb = N / bs, tpb = bs / 128, words = (nb + 31) / 32;
+  long u = blockIdx.x;
+  const int part = static_cast<int>(u % tpb);
+  u /= tpb;
+  const int j = static_cast<int>(u % nb);
+  u /= nb;
+  const int h = static_cast<int>(u % H);
+  const int b = static_cast<int>(u / H);
+  const long bh = static_cast<long>(b) * H + h;
+  const int krow0 = j * bs + part * 128;  // first key token of this tile
+  const uint32_t* mrow = mask + (bh * nb + j) * words;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar.a_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar.full[s], 1);
+      mbar_init(&bar.empty[s], 1);
+    }
+    mbar_init(&bar.prod_full, 1);
+    mbar_init(&bar.soft_full, 4);
+    mbar_init(&bar.done, 1);
+    mbar_init(&bar.drained, 1);
+    bar.abort = 0;
+    int blocks = 0;
+    for (int w = 0; w < words; ++w) blocks += __popc(__ldg(mrow + w));
+    bar.tiles = blocks * tpb;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bar.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+  const int U = bar.tiles;
+  const uint32_t sbase = smem_u32(smem);
+
+  if (warp == 0) {
+    // ============================================================ TMA producer
+    if (lane == 0 && U > 0) {
+      const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
+      mbar_arrive_expect_tx(&bar.a_full, 2 * L::kTile);
+      bwd_load_tile<D>(smem + L::kOffA, &tm_k, &bar.a_full, h, krow0, b, stream);
+      bwd_load_tile<D>(smem + L::kOffA + L::kTile, &tm_v, &bar.a_full, h, krow0, b, stream);
+      int issued[2] = {0, 0};
+      bool ok = true;
+      int w = 0, qb = 0;
+      uint32_t cur = __ldg(mrow);
+      for (int t = 0; t < U && ok; ++t) {
+        if (t % tpb == 0) qb = bwd_next_block(mrow, words, w, cur);
+        const int s = t & 1, use = t >> 1;
+        const int row = qb * bs + (t % tpb) * 128;
+        if (t >= 2) ok = mbar_wait(&bar.empty[s], (use - 1) & 1, abort_flag, 741);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bar.full[s], 2 * L::kTile);
+        unsigned char* st = smem + L::kOffRing + s * 2 * L::kTile;  // Q, then dO
+        bwd_load_tile<D>(st, &tm_q, &bar.full[s], h, row, b, keep);
+        bwd_load_tile<D>(st + L::kTile, &tm_do, &bar.full[s], h, row, b, keep);
+        issued[s] = use + 1;
+      }
+      mbar_wait_teardown(&bar.a_full, 0);
+      for (int s = 0; s < 2; ++s)
+        if (issued[s]) mbar_wait_teardown(&bar.full[s], (issued[s] - 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (lane == 0 && U > 0) {
+      const uint32_t id_s = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t id_a = idesc_bf16_f32(128, D, 0, 1);  // P^T / dS^T from TMEM, dO / Q MN-major
+      const uint64_t dkd = smem_desc_sw128(sbase + L::kOffA, 16, 1024);
+      const uint64_t dvd = smem_desc_sw128(sbase + L::kOffA + L::kTile, 16, 1024);
+      const uint64_t dring = smem_desc_sw128(sbase + L::kOffRing, 16, 1024);           // K-major
+      const uint64_t dring_mn = smem_desc_sw128(sbase + L::kOffRing, 128 * 128, 1024);  // MN-major
+      constexpr uint64_t kStep = L::kTile >> 4;
+      bool ok = mbar_wait(&bar.a_full, 0, abort_flag, 751);
+      for (int t = 0; t <= U && ok; ++t) {
+        if (t > 0) {
+          // dV += P^T(t-1) dO(t-1), dK += dS^T(t-1) Q(t-1)
+          ok = mbar_wait(&bar.soft_full, (t - 1) & 1, abort_flag, 752);
+          if (!ok) break;
+          tc_fence_after();
+          const int s = (t - 1) & 1;
+          const uint64_t dq_mn = dring_mn + (2 * s) * kStep, ddo_mn = dring_mn + (2 * s + 1) * kStep;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tmem + kColV, tmem + kColS + kk * 8, ddo_mn + ((kk * 16 * 128) >> 4), id_a,
+                        (t > 1 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tmem + kColK, tmem + kColP + kk * 8, dq_mn + ((kk * 16 * 128) >> 4), id_a,
+                        (t > 1 || kk > 0) ? 1u : 0u);
+          mma_commit(&bar.empty[s]);
+        }
+        if (t < U) {
+          // S^T(t) = K Q(t)^T and dP^T(t) = V dO(t)^T (after the products above,
+          // which read the P^T / dS^T these overwrite; the pipe runs in order)
+          const int s = t & 1;
+          ok = mbar_wait(&bar.full[s], (t >> 1) & 1, abort_flag, 753);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dqk = dring + (2 * s) * kStep, ddok = dring + (2 * s + 1) * kStep;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+            mma_bf16_ss(tmem + kColS, dkd + off, dqk + off, id_s, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+            mma_bf16_ss(tmem + kColP, dvd + off, ddok + off, id_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bar.prod_full);
+        }
+      }
+      if (ok) mma_commit(&bar.done);
+      mma_commit(&bar.drained);
+      mbar_wait_teardown(&bar.drained, 0);
+    }
+    __syncwarp();
+  } else {
+    // ============================================================ P^T, dS^T, then the epilogue
+    const int quad = warp % 4;
+    const int kr = quad * 32 + lane;  // key row of the tile
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const long key = krow0 + kr;
+    bool ok = true;
+    int w = 0, qb = 0;
+    uint32_t cur = __ldg(mrow);
+    for (int t = 0; t < U; ++t) {
+      if (t % tpb == 0) qb = bwd_next_block(mrow, words, w, cur);
+      const int qrow0 = qb * bs + (t % tpb) * 128;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar.prod_full, t & 1, abort_flag, 761));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        // this chunk's 32 query columns: ln-sum (as log2) and D of each, one per lane
+        const long qn = qrow0 + c * 32 + lane;
+        const float lse_l = __ldg(lse + bh * N + qn) * 1.4426950408889634f;
+        const float dn_l = __ldg(dsum + bh * N + qn);
+        uint32_t sv[32], pv[32];
+        tmem_ld32(lane_base + kColS + c * 32, sv);
+        tmem_ld32(lane_base + kColP + c * 32, pv);
+        tmem_wait_ld();
+        float pt[32], dst[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float lse2 = __shfl_sync(0xffffffffu, lse_l, e);
+          const float dn = __shfl_sync(0xffffffffu, dn_l, e);
+          const bool masked = kCausal && key > qrow0 + c * 32 + e;
+          const float p = masked ? 0.f : fast_exp2(fmaf(__uint_as_float(sv[e]), scale_log2, -lse2));
+          pt[e] = p;
+          dst[e] = p * (__uint_as_float(pv[e]) - dn);
+        }
+        uint32_t wp[16], wd[16];
+        bwd_pack16(pt, wp);
+        bwd_pack16(dst, wd);
+        tmem_st16(lane_base + kColS + c * 16, wp);  // over S^T columns already read
+        tmem_st16(lane_base + kColP + c * 16, wd);  // over dP^T columns already read
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.soft_full);
+    }
+    if (ok && U > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar.done, 0, abort_flag, 762));
+    if (ok) {
+      tc_fence_after();
+      __nv_bfloat16* ov = dv + ((static_cast<long>(b) * N + key) * H + h) * D;
+      __nv_bfloat16* ok_ = dk + ((static_cast<long>(b) * N + key) * H + h) * D;
+      uint32_t r[32];
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which == 0 ? kColV : kColK;
+        const float f = which == 0 ? 1.0f : scale;
+        __nv_bfloat16* out = which == 0 ? ov : ok_;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          if (U > 0) {
+            tmem_ld32(lane_base + col + c * 32, r);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0u;  // no query block kept this key block
+          }
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w4;
+            w4.x = pack_bf16x2(__uint_as_float(r[e]) * f, __uint_as_float(r[e + 1]) * f);
+            w4.y = pack_bf16x2(__uint_as_float(r[e + 2]) * f, __uint_as_float(r[e + 3]) * f);
+            w4.z = pack_bf16x2(__uint_as_float(r[e + 4]) * f, __uint_as_float(r[e + 5]) * f);
+            w4.w = pack_bf16x2(__uint_as_float(r[e + 6]) * f, __uint_as_float(r[e + 7]) * f);
+            *reinterpret_cast<uint4*>(out + c * 32 + e) = w4;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace bsa

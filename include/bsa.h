@@ -205,6 +205,40 @@ bsa_status bsa_forward_gqa(const void* q, const void* k, const void* v, void* o,
                            int H, int H_kv, int D, int block_size, double topk_ratio, bsa_dtype dt,
                            unsigned flags, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Training: forward with the row log-sum-exp, and the backward -------
+ * The page listing's step 2 keeps blocks with torch.topk, whose indices
+ * carry no gradient, so the backward is the gradient of step 3 (the
+ * attention over the kept blocks) with the index lists held fixed. Per query
+ * token n and kept key token t (p = softmax weight, o = output):
+ *   D_n = dO_n . o_n,  dS = p (dO_n . v_t - D_n),
+ *   dq_n = scale sum_t dS k_t,  dk_t = scale sum_n dS q_n,  dv_t = sum_n p dO_n.
+ * Covered shapes: dt = BSA_BF16, D = 64 or 128, block_size 128 or 256, one
+ * key/value head per query head (others: BSA_ERR_UNSUPPORTED). Flags: as for
+ * the _ex entry points (BSA_FLAG_CAUSAL masks as in the forward). */
+
+/* bsa_sparse_attn_fwd_ex that also writes lse [B, H, N] float32 (written):
+ * ln sum_t exp(scale q_n . k_t) over the row's kept (unmasked) key tokens. */
+bsa_status bsa_sparse_attn_fwd_train(const void* q, const void* k, const void* v, const int32_t* idx,
+                                     void* o, float* lse, int B, int N, int H, int D, int block_size,
+                                     int topk, float scale, bsa_dtype dt, unsigned flags, void* stream);
+
+/* Workspace bytes of bsa_sparse_attn_bwd: the transpose of the selection as
+ * a bit matrix [B, H, nb, ceil(nb / 32)] and D [B, H, N] float32. */
+size_t bsa_sparse_attn_bwd_workspace_bytes(int B, int N, int H, int D, int block_size);
+
+/* Gradients dq, dk, dv ([B, N, H, D] bf16, written) of the attention of
+ * bsa_sparse_attn_fwd_train, given q, k, v, its output o and lse, the output
+ * gradient dO ([B, N, H, D] bf16) and the same idx, scale and flags. Four
+ * kernel launches (and one memset) on `stream`: the transpose of idx, D, dQ
+ * (one CTA per 128-row query tile over its kept key tiles) and dK/dV (one
+ * CTA per 128-key tile over the query tiles that kept its block; a key block
+ * no query block kept gets zero gradients). The gradients must not alias the
+ * inputs. Deterministic: every sum has a fixed order. */
+bsa_status bsa_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                               const int32_t* idx, const float* lse, void* dq, void* dk, void* dv, int B,
+                               int N, int H, int D, int block_size, int topk, float scale, bsa_dtype dt,
+                               unsigned flags, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Size of the fixed device scratch that bsa_forward_noalloc uses: 64 MiB. */
 #define BSA_NOALLOC_SCRATCH_BYTES (64u << 20)
 
