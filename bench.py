@@ -169,6 +169,137 @@ def run_reference(args, cfg, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- training step
+
+def run_backward(args, cfg, dev, rank, world, dist, bsa, flags, variant):
+    """Times the training step: bsa_sparse_attn_fwd_train (the forward with
+    lse) then bsa_sparse_attn_bwd, on the selection of the workload."""
+    B, N, H, D, bs, ratio = cfg.B, cfg.N, cfg.H, cfg.D, cfg.block_size, cfg.topk_ratio
+    kk = cfg.k
+    q, k, v = W.make_inputs(cfg, device=dev)
+    g = torch.Generator(device=dev).manual_seed(cfg.seed + 77)
+    do = torch.randn(q.shape, generator=g, device=dev, dtype=torch.float32).to(q.dtype)
+    ws = torch.empty(bsa.bsa_forward_workspace_bytes(B, N, H, D, bs, ratio), device=dev, dtype=torch.uint8)
+    bsa.bsa_forward(q, k, v, bs, ratio, workspace=ws, flags=flags)  # the selection the step trains through
+    idx = bsa.workspace_views(ws, B, N, H, D, bs, ratio)[2].clone()
+    bws = torch.empty(bsa.lib.bsa_sparse_attn_bwd_workspace_bytes(B, N, H, D, bs), device=dev, dtype=torch.uint8)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record()
+        bsa.bsa_sparse_attn_fwd_train(q, k, v, idx, bs, flags=flags, out=o, lse=lse)
+        if ev is not None:
+            ev[1].record()
+        grads = bsa.bsa_sparse_attn_bwd(q, k, v, o, do, idx, lse, bs, flags=flags, workspace=bws)
+        if ev is not None:
+            ev[2].record()
+        return grads
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record()
+    for s_ in range(args.steps):
+        step(evs[s_])
+    t1.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    if dist:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if bsa.bsa_device_error() != 0:
+        raise RuntimeError("a kernel gave up on a bounded wait")
+
+    # end to end through the public API: host inputs in, gradients out
+    hq, hk, hv, hdo = (x.cpu().pin_memory() for x in (q, k, v, do))
+    hg = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(3)]
+    dq_, dk_, dv_, ddo = (torch.empty_like(q) for _ in range(4))
+
+    def e2e_step():
+        for d_, h_ in ((dq_, hq), (dk_, hk), (dv_, hv), (ddo, hdo)):
+            d_.copy_(h_, non_blocking=True)
+        oo, ll = bsa.bsa_sparse_attn_fwd_train(dq_, dk_, dv_, idx, bs, flags=flags)
+        grads = bsa.bsa_sparse_attn_bwd(dq_, dk_, dv_, oo, ddo, idx, ll, bs, flags=flags, workspace=bws)
+        for h_, g_ in zip(hg, grads):
+            h_.copy_(g_, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    flops_f = 4.0 * B * H * N * kk * bs * D
+    if args.causal:
+        il = idx.cpu().numpy().astype(np.int64)
+        qi = np.arange(N // bs)[None, None, :, None]
+        pairs = np.where(il < 0, 0, np.where(il < qi, bs * bs, bs * (bs + 1) // 2)).sum()
+        flops_f = 4.0 * D * float(pairs)
+    flops_b = 2.5 * flops_f  # five products of the forward's size (dS, dP recomputation not counted)
+    peaks, peak_src = load_peaks()
+    achieved = flops_b / (bwd_ms / 1e3) / 1e12
+    nbytes = q.numel() * q.element_size()
+    line = {
+        "metric": METRIC, "value": world * B * N * args.steps / (total_ms / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+        "config": {"workload": f"{cfg.name}{variant} training step (forward with lse + backward): {cfg.describe()}",
+                   "seed": cfg.seed, "l2": f"inputs larger than L2 (q, k, v, dO {nbytes / 1e6:.0f} MB each)",
+                   "parallelism": f"replica per GPU x{world}"},
+        "gpu_launches": 5 * args.steps,
+        "stages_ms": {"fwd_train": fwd_ms, "bwd": bwd_ms},
+        "e2e": {"value": world * B * N * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": 4 * nbytes, "d2h_bytes_per_step": 3 * nbytes, "steps": args.e2e_steps},
+        "clocks": clk,
+        "roofline": {"kernel": "bwd_dq_kernel + bwd_dkdv_kernel", "bound": "tensor", "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "peak_source": f"{peak_src} bf16 burst", "traffic": None,
+                     "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                     "flops_per_launch": flops_b,
+                     "forward_achieved": flops_f / (fwd_ms / 1e3) / 1e12},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        oracle.build()
+        rng = np.random.default_rng(cfg.seed + 3000)
+        il = idx.cpu().numpy()
+        tok, sec = 0, 0.0
+        for h in range(min(cfg.H, 2)):
+            qa, ka, va, da = (np.ascontiguousarray(W.to_oracle_array(x[:, :, h:h + 1])) for x in (q, k, v, do))
+            rows = np.sort(rng.choice(cfg.nb, size=(B, 1, 2), replace=False), axis=-1).astype(np.int32)
+            t_ = time.perf_counter()
+            oracle.sparse_attn_bwd(qa, ka, va, da, np.ascontiguousarray(il[:, h:h + 1]), bs, causal=args.causal,
+                                   rows=rows)
+            sec += time.perf_counter() - t_
+            tok += 2 * bs * B
+        line["cpu_baseline"] = {"value": tok / sec, "unit": "tokens/s", "cores": oracle.num_threads(),
+                                "kind": "oracle",
+                                "sample": f"backward of 2 random query blocks on each of {min(cfg.H, 2)} heads "
+                                          f"({tok} query tokens, {sec:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------- our path
 
 def main():
@@ -189,6 +320,8 @@ def main():
                     help="override the config's input type (e4m3: FP8 inputs, bf16 output)")
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="grouped queries: the config with this many key/value heads (H a multiple of it)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the training step (forward with lse + backward) instead of the forward")
     ap.add_argument("--stages-only", action="store_true",
                     help="time the stage-by-stage steps only (no fused, end-to-end or CPU legs); "
                          "for profiler runs")
@@ -229,6 +362,11 @@ def main():
 
     flags = (bsa.BSA_FLAG_CAUSAL if args.causal else 0) | (bsa.BSA_FLAG_FORCE_DIAG if args.force_diag else 0)
     variant = (" causal" + (" force_diag" if args.force_diag else "")) if args.causal else ""
+    if args.backward:
+        run_backward(args, cfg, dev, rank, world, dist, bsa, flags, variant)
+        if dist:
+            dist.destroy_process_group()
+        return
 
     B, N, H, D, bs, ratio = cfg.B, cfg.N, cfg.H, cfg.D, cfg.block_size, cfg.topk_ratio
     kk = bsa.bsa_topk_count(N // bs, ratio)

@@ -70,7 +70,7 @@ def _load():
         lib.oracle_topk_ex.argtypes = [P, ctypes.c_long, i, i, P, i, P]
         lib.oracle_sparse_attn_ex.argtypes = [P, P, P, i, i, i, i, i, i, P, i, P, i, d, i, P]
         lib.oracle_sparse_attn_gqa.argtypes = [P, P, P, i, i, i, i, i, i, i, P, i, P, i, d, i, P]
-        lib.oracle_sparse_attn_bwd.argtypes = [P, P, P, P, i, i, i, i, i, i, P, i, d, i, P, P, P]
+        lib.oracle_sparse_attn_bwd.argtypes = [P, P, P, P, i, i, i, i, i, i, P, i, P, i, d, i, P, P, P]
         lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
         lib.oracle_e4m3_to_double.restype = d
         lib.oracle_num_threads.restype = i
@@ -227,13 +227,14 @@ def forward(q, k, v, block_size: int, topk_ratio: float, rows=None, scale=None,
 
 
 def sparse_attn_bwd(q, k, v, do, idx, block_size: int, scale: float | None = None,
-                    causal: bool = False):
+                    causal: bool = False, rows=None):
     """Gradients (dq, dk, dv) of the attention over the kept blocks with the
     index lists held fixed (the top-k indices carry no gradient): for each query
     token, dS_t = p_t (dO . v_t - dO . o), dq = scale sum_t dS_t k_t,
     dk_t += scale dS_t q, dv_t += p_t dO. ``idx`` [B,H,nb,k] for all query blocks
-    (entries below 0 select nothing); ``do`` has q's dtype. Returns float64
-    [B,N,H,D] arrays."""
+    (entries below 0 select nothing); ``do`` has q's dtype. ``rows`` (int
+    [B,H,nrows]) sums only those query blocks' contributions (a timing
+    sample). Returns float64 [B,N,H,D] arrays."""
     q, code = _as_input(q)
     k_, code_k = _as_input(k)
     v, code_v = _as_input(v)
@@ -249,8 +250,13 @@ def sparse_attn_bwd(q, k, v, do, idx, block_size: int, scale: float | None = Non
     if scale is None:
         scale = 1.0 / np.sqrt(D)
     dq, dk, dv = (np.empty((B, N, H, D), np.float64) for _ in range(3))
+    if rows is None:
+        nrows, rp = nb, None
+    else:
+        rows = np.ascontiguousarray(rows, np.int32)
+        nrows, rp = rows.shape[-1], _ptr(rows)
     _load().oracle_sparse_attn_bwd(_ptr(q), _ptr(k_), _ptr(v), _ptr(do), code, B, N, H, D, block_size,
-                                   _ptr(idx), kk, float(scale), CAUSAL if causal else 0,
+                                   _ptr(idx), kk, rp, nrows, float(scale), CAUSAL if causal else 0,
                                    _ptr(dq), _ptr(dk), _ptr(dv))
     return dq, dk, dv
 

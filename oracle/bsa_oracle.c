@@ -405,11 +405,13 @@ void oracle_sparse_attn_gqa(const void* q, const void* kmat, const void* v, int 
  *   D_n = dO_n . o_n,  dP_t = dO_n . v_t,  dS_t = p_t (dP_t - D_n),
  *   dq_n = scale sum_t dS_t k_t,  dk_t += scale dS_t q_n,  dv_t += p_t dO_n.
  * dq, dk, dv are [B, N, H, D] float64; do_ is read like q (same dtype).
+ * rows [B, H, nrows] (NULL: every query block) restricts the query blocks
+ * whose contributions are summed (a sample, for timing).
  * Parallel over (b, h) only, so every sum has a fixed order.
  * ------------------------------------------------------------------------ */
 void oracle_sparse_attn_bwd(const void* q, const void* kmat, const void* v, const void* do_, int dtype,
-                            int B, int N, int H, int D, int bs, const int* idx, int k, double scale,
-                            int flags, double* dq, double* dk, double* dv) {
+                            int B, int N, int H, int D, int bs, const int* idx, int k, const int* rows,
+                            int nrows, double scale, int flags, double* dq, double* dk, double* dv) {
   int nb = N / bs;
   long ntok = (long)k * bs;
   size_t total = (size_t)B * N * H * D;
@@ -425,7 +427,8 @@ void oracle_sparse_attn_bwd(const void* q, const void* kmat, const void* v, cons
     for (int b = 0; b < B; ++b)
       for (int h = 0; h < H; ++h) {
         size_t bh = (size_t)b * H + h;
-        for (int i = 0; i < nb; ++i) {
+        for (int r = 0; r < (rows ? nrows : nb); ++r) {
+          int i = rows ? rows[bh * nrows + r] : r;
           const int* sel = idx + (bh * nb + i) * k;
           for (int t_q = 0; t_q < bs; ++t_q) {
             int n = i * bs + t_q;
