@@ -55,6 +55,21 @@ def load_peaks():
 
 # ---------------------------------------------------------------- clocks
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest value of x over all ranks (the job's time is its slowest
+    rank's); x itself without a process group."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank_step: int, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank_step * steps / (max_ms / 1e3)
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples while the timed region runs."""
 
@@ -218,10 +233,7 @@ def run_backward(args, cfg, dev, rank, world, dist, bsa, flags, variant):
     total_ms = t0.elapsed_time(t1)
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
     if bsa.bsa_device_error() != 0:
         raise RuntimeError("a kernel gave up on a bounded wait")
 
@@ -246,7 +258,7 @@ def run_backward(args, cfg, dev, rank, world, dist, bsa, flags, variant):
         e2e_step()
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
 
     flops_f = 4.0 * B * H * N * kk * bs * D
     if args.causal:
@@ -259,7 +271,7 @@ def run_backward(args, cfg, dev, rank, world, dist, bsa, flags, variant):
     achieved = flops_b / (bwd_ms / 1e3) / 1e12
     nbytes = q.numel() * q.element_size()
     line = {
-        "metric": METRIC, "value": world * B * N * args.steps / (total_ms / 1e3), "unit": "tokens/s",
+        "metric": METRIC, "value": job_tokens_per_s(B * N, world, args.steps, total_ms), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
         "config": {"workload": f"{cfg.name}{variant} training step (forward with lse + backward): {cfg.describe()}",
@@ -267,7 +279,7 @@ def run_backward(args, cfg, dev, rank, world, dist, bsa, flags, variant):
                    "parallelism": f"replica per GPU x{world}"},
         "gpu_launches": 5 * args.steps,
         "stages_ms": {"fwd_train": fwd_ms, "bwd": bwd_ms},
-        "e2e": {"value": world * B * N * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(B * N, world, args.e2e_steps, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": 4 * nbytes, "d2h_bytes_per_step": 3 * nbytes, "steps": args.e2e_steps},
         "clocks": clk,
         "roofline": {"kernel": "bwd_dq_kernel + bwd_dkdv_kernel", "bound": "tensor", "achieved": achieved,
@@ -416,10 +428,7 @@ def main():
     pool_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     sel_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     attn_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
     err = bsa.bsa_device_error()
     if err != 0:
         raise RuntimeError(f"a kernel gave up on a bounded wait (code {err})")
@@ -465,17 +474,14 @@ def main():
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     h2d = sum(x.numel() * x.element_size() for x in (q, k, v))
     d2h = o.numel() * o.element_size()
     del hq, hk, hv, ho, dq, dk, dv
 
     tokens_step = B * N
-    value = world * tokens_step * args.steps / (total_ms / 1e3)
-    e2e_value = world * tokens_step * args.e2e_steps / (e2e_ms / 1e3)
+    value = job_tokens_per_s(tokens_step, world, args.steps, total_ms)
+    e2e_value = job_tokens_per_s(tokens_step, world, args.e2e_steps, e2e_ms)
     flops = 4.0 * B * H * N * kk * bs * D
     if args.causal:
         # visible (query, key) token pairs of the lists the step produced:
