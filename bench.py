@@ -525,7 +525,7 @@ def main():
         roof_t = max(flops / (peak * 1e12), alg_bytes / (peaks["hbm_gbs"] * 1e9))
         plain = not args.causal and Hk == H and cfg.dtype == "bf16"
         line["roofline"] = {
-            "kernel": "sparse_attn_tc2_kernel" if bs in (128, 256) else "sparse_attn_tc_kernel",
+            "kernel": "sparse_attn_tc2_kernel",
             "bound": "tensor", "achieved": achieved,
             "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "peak_source": f"{peak_src} bf16 burst" + (" x 2 (nominal e4m3 / bf16 dense ratio)" if mult > 1 else ""),
@@ -534,6 +534,11 @@ def main():
             "frac_of_roofline_time": roof_t / (attn_ms / 1e3),
             "flops_per_launch": flops, "algorithmic_bytes_per_launch": alg_bytes,
         }
+        if bs == 64:
+            # two query blocks share one 128 x 128 score tile, of which the
+            # block-diagonal half is used: the tensor core runs twice the
+            # algorithmic FLOPs, so frac cannot exceed 0.5
+            line["roofline"]["tensor_flops_per_launch"] = 2 * flops
     line["selection_stage"] = {
         "bytes": sel_bytes, "ms": pool_ms + sel_ms,
         "GB/s": sel_bytes / ((pool_ms + sel_ms) / 1e3) / 1e9,

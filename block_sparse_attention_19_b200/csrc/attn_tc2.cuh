@@ -88,6 +88,7 @@ struct Tc2Barriers {
   uint32_t tmem_base;
   int abort;
   int tiles[2];  // key tiles of stream A and B (valid index entries, x2 for block_size 256)
+  int valid[4];  // block_size 64: valid index entries of the four query blocks
 };
 static_assert(sizeof(Tc2Barriers) <= 512, "barrier area");
 
@@ -109,10 +110,80 @@ __device__ __forceinline__ void tc2_mask_after(uint32_t (&r)[32], int c0, int li
     if (c0 + e > lim) r[e] = __float_as_uint(-INFINITY);
 }
 
+// The max of 64 scores.
+__device__ __forceinline__ float tc2_max64(const uint32_t (&s0)[32], const uint32_t (&s1)[32]) {
+  float m4[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) m4[e] = fmaxf(__uint_as_float(s0[2 * e]), __uint_as_float(s0[2 * e + 1]));
+#pragma unroll
+  for (int pr = 4; pr < 32; ++pr) {
+    const float a = __uint_as_float(pr < 16 ? s0[(2 * pr) & 31] : s1[(2 * pr) & 31]);
+    const float c = __uint_as_float(pr < 16 ? s0[(2 * pr + 1) & 31] : s1[(2 * pr + 1) & 31]);
+    m4[pr % 4] = fmax3(m4[pr % 4], a, c);
+  }
+  return fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
+}
+
+// O_X *= alpha for the thread's row (alpha is 1 on rows whose max stayed).
+template <int D>
+__device__ __forceinline__ void tc2_rescale_o(uint32_t ocol, float alpha) {
+  uint32_t r[16];
+#pragma unroll 1
+  for (int c = 0; c < D / 16; ++c) {
+    tmem_ld16(ocol + c * 16, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+    tmem_st16(ocol + c * 16, r);
+  }
+}
+
+// P = exp2(S * scale_log2 - m) for 32 scores of a row, packed as the P.V
+// product reads it from TMEM: bf16 two per column (16 columns) or e4m3 four
+// per column (8), the lowest key in the lowest bits; one key pair in four via
+// the polynomial exp2. ps: four partial sums of the float32 P, accumulated.
+template <bool kF8>
+__device__ __forceinline__ void tc2_make_p32(const uint32_t (&sv)[32], float m, float scale_log2,
+                                             uint32_t (&pk)[kF8 ? 8 : 16], uint64_t (&ps)[4]) {
+  const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m, -m);
+#pragma unroll
+  for (int pr = 0; pr < 16; ++pr) {
+    const uint64_t x2 = f2_fma(f2(__uint_as_float(sv[2 * pr]), __uint_as_float(sv[2 * pr + 1])), sc2, nm2);
+    uint64_t p2;
+    if (pr % 4 == 1) {
+      p2 = exp2_poly2(x2);
+    } else {
+      float x0, x1;
+      f2_split(x2, x0, x1);
+      p2 = f2(fast_exp2(x0), fast_exp2(x1));
+    }
+    ps[pr % 4] = f2_add(ps[pr % 4], p2);
+    float p0, p1;
+    f2_split(p2, p0, p1);
+    if constexpr (kF8) {
+      const uint32_t h16 = pack_e4m3x2(p0, p1);
+      if (pr % 2 == 0)
+        pk[pr / 2] = h16;
+      else
+        pk[pr / 2] |= h16 << 16;
+    } else {
+      pk[pr] = pack_bf16x2(p0, p1);
+    }
+  }
+}
+
 // grid.x = B * H * ceil(nb / 2) for block_size 128, B * H * nb for 256.
+// kStack (block_size 64): grid.x = B * H * ceil(nb / 4); stream x stacks
+// query blocks 4u + 2x (rows 0-63) and 4u + 2x + 1 (rows 64-127), and its
+// key tile t stacks the t-th kept block of each (keys 0-63, 64-127). The
+// 128 x 128 score tile is then block diagonal: rows 0-63 keep keys 0-63,
+// rows 64-127 keys 64-127; the other quadrants are computed and discarded,
+// and P is zero there, so one M = 128 product serves both blocks (the same
+// tensor time as two M = 64 products, with every TMEM lane and softmax
+// thread in use).
 // kCausal: key tokens after the query token are masked (kFlagCausal).
 // lse (optional, [B, H, N] float32): ln sum_t exp(scale q_n . k_t) per row.
-template <int D, bool kCausal, bool kF8 = false>
+template <int D, bool kCausal, bool kF8 = false, bool kStack = false>
 __global__ void __launch_bounds__(kTc2Threads, 1)
     sparse_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
@@ -144,11 +215,17 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
   // In the first two the streams read the same key tiles (one selection),
   // so each K and V tile is loaded once for both.
   const int G = H / Hkv;
-  const bool head_pairs = bs == 128 && (G % 2) == 0;
-  const bool shared_kv = bs == 256 || head_pairs;
+  const bool head_pairs = !kStack && bs == 128 && (G % 2) == 0;
+  const bool shared_kv = !kStack && (bs == 256 || head_pairs);
   long u = blockIdx.x;
   int iA, b, qh[2];
-  if (head_pairs) {
+  if (kStack) {
+    const int per_bh = (nb + 3) / 4;
+    iA = 4 * static_cast<int>(u % per_bh);
+    u /= per_bh;
+    qh[0] = qh[1] = static_cast<int>(u % H);
+    b = static_cast<int>(u / H);
+  } else if (head_pairs) {
     iA = static_cast<int>(u % nb);
     u /= nb;
     const int hp = static_cast<int>(u % (H / 2));
@@ -164,12 +241,21 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     iA = bs == 256 ? unit : 2 * unit;
   }
   const int g = qh[0] / G;  // the key/value head (and selection) of both streams
-  const int nstreams = (!shared_kv && iA + 1 >= nb) ? 1 : 2;
+  const int nstreams = kStack ? (iA + 2 < nb ? 2 : 1) : ((!shared_kv && iA + 1 >= nb) ? 1 : 2);
   // stream x covers query rows [row0[x], row0[x] + 128) of query head qh[x]
-  const int row0[2] = {iA * bs, bs == 256 ? iA * bs + 128 : (head_pairs ? iA * bs : (iA + 1) * bs)};
+  const int row0[2] = {iA * bs, kStack ? (iA + 2) * 64
+                                       : (bs == 256 ? iA * bs + 128 : (head_pairs ? iA * bs : (iA + 1) * bs))};
   const long bg = static_cast<long>(b) * Hkv + g;
   const int32_t* sel_a = idx + (bg * nb + iA) * k;
   const int32_t* sel_b = shared_kv ? sel_a : idx + (bg * nb + (iA + 1 < nb ? iA + 1 : iA)) * k;
+  // kStack: index rows of query blocks iA + q (an absent second block of a
+  // stream takes its first block's row, whose rows are then not written)
+  const int32_t* sel4[4];
+  if (kStack)
+    for (int q = 0; q < 4; ++q) {
+      const int blk = iA + q < nb ? iA + q : min(iA + (q & 2), nb - 1);
+      sel4[q] = idx + (bg * nb + blk) * k;
+    }
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -195,11 +281,18 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     bar.abort = 0;
     // key tiles per stream: the valid entries of its index row (at least one,
     // so that a row of only -1 still reads block 0 instead of nothing)
-    const int ta = max(index_row_valid(sel_a, k), 1);
-    const int tb = nstreams == 2 && !shared_kv ? max(index_row_valid(sel_b, k), 1) : 0;
-    const int tpb = bs == 256 ? 2 : 1;  // key tiles per block
-    bar.tiles[0] = tpb * ta;
-    bar.tiles[1] = shared_kv ? tpb * ta : tb;
+    if (kStack) {
+      // a stream walks as many tiles as the longer of its two rows
+      for (int q = 0; q < 4; ++q) bar.valid[q] = q / 2 < nstreams ? max(index_row_valid(sel4[q], k), 1) : 0;
+      bar.tiles[0] = max(bar.valid[0], bar.valid[1]);
+      bar.tiles[1] = max(bar.valid[2], bar.valid[3]);
+    } else {
+      const int ta = max(index_row_valid(sel_a, k), 1);
+      const int tb = nstreams == 2 && !shared_kv ? max(index_row_valid(sel_b, k), 1) : 0;
+      const int tpb = bs == 256 ? 2 : 1;  // key tiles per block
+      bar.tiles[0] = tpb * ta;
+      bar.tiles[1] = shared_kv ? tpb * ta : tb;
+    }
     fence_mbarrier_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -256,7 +349,9 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         const int x = shared_kv ? 0 : (n < 2 * Tmin ? (n & 1) : (TA > TB ? 0 : 1));
         const int t = shared_kv ? n : (n < 2 * Tmin ? (n >> 1) : Tmin + (n - 2 * Tmin));
         int r[2];
-        for (int hf = 0; hf < 2; ++hf) r[hf] = tc2_key_row(sel_a, sel_b, x, t, hf, bs, nb);
+        for (int hf = 0; hf < 2; ++hf)
+          r[hf] = kStack ? clamp_block(__ldg(sel4[2 * x + hf] + t), nb) * 64  // -1 entries load block 0, unused
+                         : tc2_key_row(sel_a, sel_b, x, t, hf, bs, nb);
         if (n >= S) ok = mbar_wait(&empty[s], (use - 1) & 1, abort_flag, is_k ? 111 : 112);
         if (!ok) break;
         mbar_arrive_expect_tx(&full[s], L::kTileBytes);
@@ -379,6 +474,9 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     const int Tx = x == 0 ? TA : TB;
+    // kStack: valid tiles of the thread's query block; rows of an absent block are not written
+    const int vt = kStack ? bar.valid[2 * x + quad / 2] : Tx;
+    const bool live = !kStack || iA + 2 * x + quad / 2 < nb;
     for (int j = 0; j < Tx; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_full[x], j & 1, abort_flag, 311));
       if (!ok) break;
@@ -387,96 +485,152 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         // S_X(j) is complete: the K tile it read can be refilled
         mbar_arrive(&bar.k_empty[load_index(x, j) % KS]);
       }
-      // first key token of this tile; with the causal flag a tile that
-      // reaches past the tile's first query token masks key c for row r when
-      // kbase + c > qbase + r (only the diagonal block does)
-      const int kbase = kCausal ? tc2_key_row(sel_a, sel_b, x, j, 0, bs, nb) : 0;
-      const bool mask_tile = kCausal && kbase + 127 > row0[x];
-      // The whole S row in registers: four TMEM loads, one wait.
-      uint32_t sa[32], sb[32], sc[32], sd[32];
-      tmem_ld32(scol, sa);
-      tmem_ld32(scol + 32, sb);
-      tmem_ld32(scol + 64, sc);
-      tmem_ld32(scol + 96, sd);
-      tmem_wait_ld();
-      if (mask_tile) {
-        // keys c > lim of this tile lie after the thread's query token
-        const int lim = row0[x] + row - kbase;
-        tc2_mask_after(sa, 0, lim);
-        tc2_mask_after(sb, 32, lim);
-        tc2_mask_after(sc, 64, lim);
-        tc2_mask_after(sd, 96, lim);
-      }
-#define BSA_S(i) __uint_as_float((i) < 32 ? sa[(i) & 31] : (i) < 64 ? sb[(i) & 31] : (i) < 96 ? sc[(i) & 31] : sd[(i) & 31])
-      float m4[4];
+      if constexpr (kStack) {
+        // rows 64 hf.. of the stream belong to query block iA + 2x + hf, whose
+        // keys are columns 64 hf.. of the tile
+        const int hf = quad / 2;
+        if (j >= vt) {
+          // this block's list has ended: its P is zero on the whole tile
+          uint32_t z[32];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) m4[e] = fmaxf(BSA_S(2 * e), BSA_S(2 * e + 1));
-#pragma unroll
-      for (int pr = 4; pr < 64; ++pr) m4[pr % 4] = fmax3(m4[pr % 4], BSA_S(2 * pr), BSA_S(2 * pr + 1));
-      const float mt = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]) * scale_log2;
-      // the running max moves only when the tile max exceeds it by more than 8
-      const float m_new = (j == 0 || mt > m_run + 8.0f) ? mt : m_run;
-      const bool rescale = j > 0 && m_new != m_run;
-      if (__any_sync(0xffffffffu, rescale)) {
-        // S_X(j) is complete, so PV_X(j-1) has finished accumulating into O_X
-        const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
-        l_run *= alpha;
-        uint32_t r[16];
-#pragma unroll 1
-        for (int c = 0; c < D / 16; ++c) {
-          tmem_ld16(ocol + c * 16, r);
+          for (int e = 0; e < 32; ++e) z[e] = 0;
+          tmem_st32(scol, z);
+          if constexpr (!kF8) tmem_st32(scol + 32, z);
+        } else {
+          uint32_t s0[32], s1[32];
+          tmem_ld32(scol + 64 * hf, s0);
+          tmem_ld32(scol + 64 * hf + 32, s1);
           tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st16(ocol + c * 16, r);
-        }
-      }
-      m_run = m_new;
-      // P = exp2(S * scale_log2 - m) for key pairs with two-wide float32
-      // instructions; one pair in four takes the polynomial exp2 on the FMA
-      // pipe (the split measured fastest: the softmax is bound by issue slots
-      // more than by MUFU). P is stored over the first columns of S: packed
-      // bf16, two per column (64 columns), or e4m3, four per column (32).
-      uint32_t pa[32], pb[kF8 ? 1 : 32];
-      uint64_t ps[4] = {0, 0, 0, 0};
-      {
-        const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m_new, -m_new);
-#pragma unroll
-        for (int pr = 0; pr < 64; ++pr) {
-          const uint64_t x2 = f2_fma(f2(BSA_S(2 * pr), BSA_S(2 * pr + 1)), sc2, nm2);
-          uint64_t p2;
-          if (pr % 4 == 1) {
-            p2 = exp2_poly2(x2);
-          } else {
-            float x0, x1;
-            f2_split(x2, x0, x1);
-            p2 = f2(fast_exp2(x0), fast_exp2(x1));
+          if (kCausal) {
+            // keys c > lim of the block follow the thread's query token
+            const int lim = row0[x] + row - clamp_block(__ldg(sel4[2 * x + hf] + j), nb) * 64;
+            if (lim < 63) {
+              tc2_mask_after(s0, 0, lim);
+              tc2_mask_after(s1, 32, lim);
+            }
           }
-          ps[pr % 4] = f2_add(ps[pr % 4], p2);
-          float p0, p1;
-          f2_split(p2, p0, p1);
-          if (kF8) {
-            // four e4m3 per 32-bit column, the lowest byte the lowest key
-            const uint32_t h16 = pack_e4m3x2(p0, p1);
-            if (pr % 2 == 0)
-              pa[pr / 2] = h16;
-            else
-              pa[pr / 2] |= h16 << 16;
-          } else if (pr < 32) {
-            pa[pr] = pack_bf16x2(p0, p1);
+          const float mt = tc2_max64(s0, s1) * scale_log2;
+          const float m_new = (j == 0 || mt > m_run + 8.0f) ? mt : m_run;
+          const bool rescale = j > 0 && m_new != m_run;
+          if (__any_sync(0xffffffffu, rescale)) {
+            const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
+            l_run *= alpha;
+            tc2_rescale_o<D>(ocol, alpha);
+          }
+          m_run = m_new;
+          uint64_t ps[4] = {0, 0, 0, 0};
+          uint32_t pk0[kF8 ? 8 : 16], pk1[kF8 ? 8 : 16], z[kF8 ? 16 : 32];
+          tc2_make_p32<kF8>(s0, m_new, scale_log2, pk0, ps);
+          tc2_make_p32<kF8>(s1, m_new, scale_log2, pk1, ps);
+#pragma unroll
+          for (int e = 0; e < (kF8 ? 16 : 32); ++e) z[e] = 0;
+          // P of the block's keys; zeros where the tile holds the other block's
+          if constexpr (kF8) {
+            tmem_st8(scol + 16 * hf, pk0);
+            tmem_st8(scol + 16 * hf + 8, pk1);
+            tmem_st16(scol + 16 * (1 - hf), z);
           } else {
-            pb[pr - 32] = pack_bf16x2(p0, p1);
+            tmem_st16(scol + 32 * hf, pk0);
+            tmem_st16(scol + 32 * hf + 16, pk1);
+            tmem_st32(scol + 32 * (1 - hf), z);
+          }
+          float a0, a1;
+          f2_split(f2_add(f2_add(ps[0], ps[1]), f2_add(ps[2], ps[3])), a0, a1);
+          l_run += a0 + a1;
+        }
+        tmem_wait_st();
+      } else {
+        // first key token of this tile; with the causal flag a tile that
+        // reaches past the tile's first query token masks key c for row r when
+        // kbase + c > qbase + r (only the diagonal block does)
+        const int kbase = kCausal ? tc2_key_row(sel_a, sel_b, x, j, 0, bs, nb) : 0;
+        const bool mask_tile = kCausal && kbase + 127 > row0[x];
+        // The whole S row in registers: four TMEM loads, one wait.
+        uint32_t sa[32], sb[32], sc[32], sd[32];
+        tmem_ld32(scol, sa);
+        tmem_ld32(scol + 32, sb);
+        tmem_ld32(scol + 64, sc);
+        tmem_ld32(scol + 96, sd);
+        tmem_wait_ld();
+        if (mask_tile) {
+          // keys c > lim of this tile lie after the thread's query token
+          const int lim = row0[x] + row - kbase;
+          tc2_mask_after(sa, 0, lim);
+          tc2_mask_after(sb, 32, lim);
+          tc2_mask_after(sc, 64, lim);
+          tc2_mask_after(sd, 96, lim);
+        }
+#define BSA_S(i) __uint_as_float((i) < 32 ? sa[(i) & 31] : (i) < 64 ? sb[(i) & 31] : (i) < 96 ? sc[(i) & 31] : sd[(i) & 31])
+        float m4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) m4[e] = fmaxf(BSA_S(2 * e), BSA_S(2 * e + 1));
+#pragma unroll
+        for (int pr = 4; pr < 64; ++pr) m4[pr % 4] = fmax3(m4[pr % 4], BSA_S(2 * pr), BSA_S(2 * pr + 1));
+        const float mt = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]) * scale_log2;
+        // the running max moves only when the tile max exceeds it by more than 8
+        const float m_new = (j == 0 || mt > m_run + 8.0f) ? mt : m_run;
+        const bool rescale = j > 0 && m_new != m_run;
+        if (__any_sync(0xffffffffu, rescale)) {
+          // S_X(j) is complete, so PV_X(j-1) has finished accumulating into O_X
+          const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
+          l_run *= alpha;
+          uint32_t r[16];
+#pragma unroll 1
+          for (int c = 0; c < D / 16; ++c) {
+            tmem_ld16(ocol + c * 16, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st16(ocol + c * 16, r);
           }
         }
-      }
+        m_run = m_new;
+        // P = exp2(S * scale_log2 - m) for key pairs with two-wide float32
+        // instructions; one pair in four takes the polynomial exp2 on the FMA
+        // pipe (the split measured fastest: the softmax is bound by issue slots
+        // more than by MUFU). P is stored over the first columns of S: packed
+        // bf16, two per column (64 columns), or e4m3, four per column (32).
+        uint32_t pa[32], pb[kF8 ? 1 : 32];
+        uint64_t ps[4] = {0, 0, 0, 0};
+        {
+          const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m_new, -m_new);
+#pragma unroll
+          for (int pr = 0; pr < 64; ++pr) {
+            const uint64_t x2 = f2_fma(f2(BSA_S(2 * pr), BSA_S(2 * pr + 1)), sc2, nm2);
+            uint64_t p2;
+            if (pr % 4 == 1) {
+              p2 = exp2_poly2(x2);
+            } else {
+              float x0, x1;
+              f2_split(x2, x0, x1);
+              p2 = f2(fast_exp2(x0), fast_exp2(x1));
+            }
+            ps[pr % 4] = f2_add(ps[pr % 4], p2);
+            float p0, p1;
+            f2_split(p2, p0, p1);
+            if (kF8) {
+              // four e4m3 per 32-bit column, the lowest byte the lowest key
+              const uint32_t h16 = pack_e4m3x2(p0, p1);
+              if (pr % 2 == 0)
+                pa[pr / 2] = h16;
+              else
+                pa[pr / 2] |= h16 << 16;
+            } else if (pr < 32) {
+              pa[pr] = pack_bf16x2(p0, p1);
+            } else {
+              pb[pr - 32] = pack_bf16x2(p0, p1);
+            }
+          }
+        }
 #undef BSA_S
-      tmem_st32(scol, pa);
-      if constexpr (!kF8) tmem_st32(scol + 32, pb);
-      tmem_wait_st();
-      {
-        float a0, a1;
-        f2_split(f2_add(f2_add(ps[0], ps[1]), f2_add(ps[2], ps[3])), a0, a1);
-        l_run += a0 + a1;
+        tmem_st32(scol, pa);
+        if constexpr (!kF8) tmem_st32(scol + 32, pb);
+        tmem_wait_st();
+        {
+          float a0, a1;
+          f2_split(f2_add(f2_add(ps[0], ps[1]), f2_add(ps[2], ps[3])), a0, a1);
+          l_run += a0 + a1;
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -484,7 +638,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     }
     // ---- epilogue: O_X / l -> bf16 -> global
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.pv_last[x], 0, abort_flag, 314));
-    if (ok) {
+    if (ok && live) {
       tc_fence_after();
       const float inv = 1.0f / l_run;
       const long n = row0[x] + row;

@@ -14,7 +14,6 @@
 #include <mutex>
 
 #include "attn_simt.cuh"
-#include "attn_tc.cuh"
 #include "attn_tc2.cuh"
 #include "bwd.cuh"
 #include "bsa.h"
@@ -281,36 +280,7 @@ bsa_status launch_attn_simt(const float* q, const float* k, const float* v, cons
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_simt_kernel launch");
 }
 
-template <int D, int BM>
-bsa_status launch_attn_tc(const void* q, const void* k, const void* v, const int32_t* idx,
-                          void* o, int B, int N, int H, int Hkv, int bs, int kk, float scale,
-                          unsigned flags, cudaStream_t st) {
-  using L = bsa::TcLayout<D, BM>;
-  CUtensorMap mq, mk, mv;
-  bsa_status s;
-  if ((s = make_bnhd_map(&mq, q, B, N, H, D)) != BSA_OK) return s;
-  if ((s = make_bnhd_map(&mk, k, B, N, Hkv, D)) != BSA_OK) return s;
-  if ((s = make_bnhd_map(&mv, v, B, N, Hkv, D)) != BSA_OK) return s;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_tc_kernel<D, BM>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
-    if (e != cudaSuccess) return cuda_fail(e, "tc smem attribute");
-    attr_set[dev] = true;
-  }
-  const int parts = bs > BM ? bs / BM : 1;
-  const long grid = static_cast<long>(B) * H * (N / bs) * parts;
-  if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
-  const float scale_log2 = scale * 1.4426950408889634f;
-  bsa::sparse_attn_tc_kernel<D, BM><<<static_cast<unsigned>(grid), bsa::kTcThreads, L::kBytes, st>>>(
-      mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, Hkv, bs, kk, scale_log2, flags);
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc_kernel launch");
-}
-
-template <int D, bool kCausal, bool kF8>
+template <int D, bool kCausal, bool kF8, bool kStack>
 bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                               int B, int N, int H, int Hkv, int bs, int kk, float scale,
                               float* lse, cudaStream_t st) {
@@ -324,14 +294,14 @@ bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_tc2_kernel<D, kCausal, kF8>,
+    cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_tc2_kernel<D, kCausal, kF8, kStack>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return cuda_fail(e, "tc2 smem attribute");
     // The kernel moves registers between warp groups (setmaxnreg); an increase
     // that the launch allocation cannot cover would wait forever, so refuse
     // to launch unless the compiled register count covers the split.
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, bsa::sparse_attn_tc2_kernel<D, kCausal, kF8>);
+    e = cudaFuncGetAttributes(&fa, bsa::sparse_attn_tc2_kernel<D, kCausal, kF8, kStack>);
     if (e != cudaSuccess) return cuda_fail(e, "tc2 attributes");
     if (fa.numRegs < static_cast<int>(bsa::kTc2LaunchRegs))
       return fail(BSA_ERR_UNSUPPORTED, "attention kernel built with %d registers/thread, its register split needs %u",
@@ -341,24 +311,26 @@ bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const
   const int nb = N / bs;
   // the kernel's CTA layouts: halves of a 256-block; two query heads of a
   // group on one block (an even group size); two blocks of one head
+  // block_size 64: two streams of two stacked query blocks each
   const bool head_pairs = bs == 128 && ((H / Hkv) % 2) == 0;
-  const long grid = head_pairs ? static_cast<long>(B) * (H / 2) * nb
-                               : static_cast<long>(B) * H * (bs == 256 ? nb : (nb + 1) / 2);
+  const long grid = kStack       ? static_cast<long>(B) * H * ((nb + 3) / 4)
+                    : head_pairs ? static_cast<long>(B) * (H / 2) * nb
+                                 : static_cast<long>(B) * H * (bs == 256 ? nb : (nb + 1) / 2);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   const float scale_log2 = scale * 1.4426950408889634f;
-  bsa::sparse_attn_tc2_kernel<D, kCausal, kF8><<<static_cast<unsigned>(grid), bsa::kTc2Threads, L::kBytes, st>>>(
+  bsa::sparse_attn_tc2_kernel<D, kCausal, kF8, kStack><<<static_cast<unsigned>(grid), bsa::kTc2Threads, L::kBytes, st>>>(
       mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, Hkv, bs, kk, scale_log2, lse);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc2_kernel launch");
 }
 
-template <int D, bool kF8 = false>
+template <int D, bool kF8 = false, bool kStack = false>
 bsa_status launch_attn_tc2(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                            int B, int N, int H, int Hkv, int bs, int kk, float scale, unsigned flags,
                            float* lse, cudaStream_t st) {
   return (flags & BSA_FLAG_CAUSAL)
-             ? launch_attn_tc2_as<D, true, kF8>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, st)
-             : launch_attn_tc2_as<D, false, kF8>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, st);
+             ? launch_attn_tc2_as<D, true, kF8, kStack>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, st)
+             : launch_attn_tc2_as<D, false, kF8, kStack>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, st);
 }
 
 bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
@@ -372,13 +344,13 @@ bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_
                    : launch_attn_simt<128>(fq, fk, fv, idx, fo, B, N, H, Hkv, bs, kk, scale, flags, st);
   }
   if (dt == BSA_E4M3) {
-    if (D != 128 || bs == 64)
-      return fail(BSA_ERR_UNSUPPORTED, "e4m3 inputs need D = 128 and block_size 128 or 256");
-    return launch_attn_tc2<128, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st);
+    if (D != 128) return fail(BSA_ERR_UNSUPPORTED, "e4m3 inputs need D = 128");
+    return bs == 64 ? launch_attn_tc2<128, true, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st)
+                    : launch_attn_tc2<128, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st);
   }
   if (bs == 64)
-    return D == 64 ? launch_attn_tc<64, 64>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, st)
-                   : launch_attn_tc<128, 64>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, st);
+    return D == 64 ? launch_attn_tc2<64, false, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st)
+                   : launch_attn_tc2<128, false, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st);
   return D == 64 ? launch_attn_tc2<64>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st)
                  : launch_attn_tc2<128>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st);
 }

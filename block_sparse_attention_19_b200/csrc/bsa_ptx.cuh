@@ -22,6 +22,12 @@ __device__ __forceinline__ void report_error(int code) { atomicCAS(&g_device_err
 // BSA_FLAG_* macros of the public header).
 constexpr unsigned kFlagCausal = 1u, kFlagForceDiag = 2u;
 
+// An index entry as a block number in [0, nb): -1 padding (causal rows)
+// reads block 0, whose contribution the caller masks.
+__device__ __forceinline__ int clamp_block(int blk, int nb) {
+  return blk < 0 ? 0 : (blk >= nb ? nb - 1 : blk);
+}
+
 // Number of leading entries >= 0 of an index row of k entries (a row lists
 // its blocks in ascending order, then pads with -1): binary search.
 __device__ __forceinline__ int index_row_valid(const int32_t* sel, int k) {
@@ -302,6 +308,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
       "r"(r[15])
+      : "memory");
+}
+
+// 32 lanes x 32 bits, 8 consecutive columns.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
       : "memory");
 }
 

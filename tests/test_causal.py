@@ -73,6 +73,7 @@ CASES = [  # (B, N, H, D, block_size, ratio, dtype)
     (1, 1920, 2, 128, 128, 0.4, "bf16"),    # odd nb: a CTA with one query tile
     (1, 4096, 2, 128, 256, 0.3, "bf16"),    # block_size 256: halves of the diagonal
     (2, 2048, 2, 64, 64, 0.3, "bf16"),      # block_size 64, odd k
+    (1, 448, 2, 128, 64, 0.5, "bf16"),      # block_size 64, nb 7: stacked blocks with unequal counts
     (1, 1024, 2, 128, 128, 1.0, "bf16"),    # k = nb: dense causal attention
     (1, 1024, 2, 64, 64, 0.5, "f32"),       # float32 path
     (1, 512, 2, 128, 64, 0.25, "f32"),

@@ -54,6 +54,8 @@ CASES = [  # (B, N, H, H_kv, block_size, ratio, causal)
     (1, 1920, 2, 2, 128, 0.4, True),    # causal, odd nb
     (1, 4096, 2, 2, 256, 0.3, False),   # block_size 256
     (1, 1024, 2, 2, 128, 1.0, False),   # k = nb
+    (1, 2048, 2, 2, 64, 0.25, False),   # block_size 64: two query blocks stacked per tile
+    (1, 1344, 4, 2, 64, 0.3, True),     # block_size 64, causal, nb 21 (a CTA with one block)
 ]
 
 
@@ -88,10 +90,9 @@ def test_fp8_full_path(bsa, oracle_mod, ci):
 
 
 def test_fp8_refused_where_unsupported(bsa):
-    """FP8 inputs need D = 128 and block_size 128 or 256."""
+    """FP8 inputs need D = 128."""
     q = torch.zeros(1, 512, 2, 64, device="cuda", dtype=torch.float8_e4m3fn)
     with pytest.raises(bsa.BsaError, match="UNSUPPORTED"):
         bsa.bsa_forward(q, q, q, 128, 0.5)
-    q = torch.zeros(1, 512, 2, 128, device="cuda", dtype=torch.float8_e4m3fn)
     with pytest.raises(bsa.BsaError, match="UNSUPPORTED"):
         bsa.bsa_forward(q, q, q, 64, 0.5)

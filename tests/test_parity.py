@@ -154,6 +154,12 @@ SMALL = [  # (B, N, H, D, bs, ratio, dtype) spanning several key tiles and a rag
     (1, 512, 2, 128, 128, 1.0, "bf16"),   # k = nb (dense)
     (1, 1024, 1, 128, 128, 0.125, "bf16"),  # k = 1
     (1, 256, 2, 64, 256, 1.0, "bf16"),    # nb = 1
+    # block_size 64 stacks query blocks 4u..4u+3 in one CTA: counts that leave
+    # blocks absent
+    (1, 64, 2, 64, 64, 1.0, "bf16"),      # nb = 1
+    (1, 192, 2, 64, 64, 0.67, "bf16"),    # nb = 3: second stream with one block
+    (2, 320, 2, 128, 64, 0.4, "bf16"),    # nb = 5: a CTA with one block
+    (1, 384, 3, 64, 64, 0.5, "bf16"),     # nb = 6: a CTA with one stream
     (2, 512, 3, 64, 64, 0.5, "f32"),
     (1, 1024, 2, 128, 128, 0.5, "f32"),
     (1, 1024, 2, 64, 256, 0.5, "f32"),
