@@ -124,6 +124,22 @@ def block_pool(x: np.ndarray, block_size: int) -> np.ndarray:
     return out
 
 
+def _rows(rows, B: int, H: int, nb: int):
+    """(nrows, pointer, array) for a query-block list: ``rows`` broadcast to
+    [B, H, nrows] (so [1, 1, nrows] picks the same blocks in every batch
+    entry and head), or (nb, None, None) for all blocks. The C routines read
+    B * H * nrows entries, so anything else is refused here."""
+    if rows is None:
+        return nb, None, None
+    r = np.asarray(rows)
+    if r.ndim != 3:
+        raise ValueError(f"rows must be [B, H, nrows], got shape {r.shape}")
+    r = np.ascontiguousarray(np.broadcast_to(r, (B, H, r.shape[-1])), np.int32)
+    if r.size and (r.min() < 0 or r.max() >= nb):
+        raise ValueError(f"rows must lie in [0, {nb})")
+    return r.shape[-1], _ptr(r), r
+
+
 def block_scores(qp: np.ndarray, kp: np.ndarray, rows: np.ndarray | None = None) -> np.ndarray:
     """Block scores S[b,h,r,j] = qp[b,h,rows[b,h,r]] . kp[b,h,j] ([SF] step 1).
 
@@ -131,11 +147,7 @@ def block_scores(qp: np.ndarray, kp: np.ndarray, rows: np.ndarray | None = None)
     qp = np.ascontiguousarray(qp, np.float64)
     kp = np.ascontiguousarray(kp, np.float64)
     B, H, nb, D = qp.shape
-    if rows is None:
-        nrows, rp = nb, None
-    else:
-        rows = np.ascontiguousarray(rows, np.int32)
-        nrows, rp = rows.shape[-1], _ptr(rows)
+    nrows, rp, rows = _rows(rows, B, H, nb)
     out = np.empty((B, H, nrows, nb), np.float64)
     _load().oracle_block_scores(_ptr(qp), _ptr(kp), B, H, nb, D, rp, nrows, _ptr(out))
     return out
@@ -185,11 +197,7 @@ def sparse_attn(q, k, v, idx, block_size: int, scale: float | None = None, rows=
     nb = N // block_size
     idx = np.ascontiguousarray(idx, np.int32)
     kk = idx.shape[-1]
-    if rows is None:
-        nrows, rp = nb, None
-    else:
-        rows = np.ascontiguousarray(rows, np.int32)
-        nrows, rp = rows.shape[-1], _ptr(rows)
+    nrows, rp, rows = _rows(rows, B, H, nb)
     if idx.shape != (B, H, nrows, kk):
         raise ValueError(f"idx shape {idx.shape} != {(B, H, nrows, kk)}")
     if scale is None:
@@ -250,11 +258,7 @@ def sparse_attn_bwd(q, k, v, do, idx, block_size: int, scale: float | None = Non
     if scale is None:
         scale = 1.0 / np.sqrt(D)
     dq, dk, dv = (np.empty((B, N, H, D), np.float64) for _ in range(3))
-    if rows is None:
-        nrows, rp = nb, None
-    else:
-        rows = np.ascontiguousarray(rows, np.int32)
-        nrows, rp = rows.shape[-1], _ptr(rows)
+    nrows, rp, rows = _rows(rows, B, H, nb)
     _load().oracle_sparse_attn_bwd(_ptr(q), _ptr(k_), _ptr(v), _ptr(do), code, B, N, H, D, block_size,
                                    _ptr(idx), kk, rp, nrows, float(scale), CAUSAL if causal else 0,
                                    _ptr(dq), _ptr(dk), _ptr(dv))
@@ -292,11 +296,7 @@ def sparse_attn_gqa(q, k, v, idx, block_size: int, scale: float | None = None, r
     nb = N // block_size
     idx = np.ascontiguousarray(idx, np.int32)
     kk = idx.shape[-1]
-    if rows is None:
-        nrows, rp = nb, None
-    else:
-        rows = np.ascontiguousarray(rows, np.int32)
-        nrows, rp = rows.shape[-1], _ptr(rows)
+    nrows, rp, rows = _rows(rows, B, H, nb)
     if idx.shape != (B, H, nrows, kk):
         raise ValueError(f"idx shape {idx.shape} != {(B, H, nrows, kk)}")
     if scale is None:
@@ -322,6 +322,8 @@ def forward_gqa(q, k, v, block_size: int, topk_ratio: float, rows=None, scale=No
     G = H // Hkv
     nb = N // block_size
     kk = topk_count(nb, topk_ratio)
+    if rows is not None:
+        _, _, rows = _rows(rows, B, Hkv, nb)
     qp = block_pool(q, block_size)
     qg = group_pool(qp, Hkv)
     kp = block_pool(k, block_size)

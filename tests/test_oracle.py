@@ -578,3 +578,37 @@ def test_backward_matches_finite_differences(oracle_mod):
             args = lambda x: [x if n == name else a for n, a in (("q", q), ("k", k), ("v", v))]
             fd = (loss(*args(plus)) - loss(*args(minus))) / (2 * eps)
             assert abs(fd - grad[pos]) <= 1e-7 * max(1.0, abs(fd)), (name, pos, fd, grad[pos])
+
+
+def test_row_lists_broadcast_over_batch_and_heads_and_are_checked(oracle_mod):
+    """A [1, 1, nrows] list of query blocks means the same blocks in every
+    (b, h); lists that do not broadcast, or name blocks outside [0, nb), are
+    refused before the C routines read them."""
+    import workloads as W
+
+    oracle = oracle_mod
+    cfg = W.Config("rows", 2, 512, 3, 64, 64, 0.5, "f32", 1.0, 77, None)
+    q, k, v = (W.to_oracle_array(x) for x in W.make_inputs(cfg, device="cpu"))
+    full = oracle.forward(q, k, v, 64, 0.5)
+    rows = np.array([[[1, 6]]], np.int32)
+    part = oracle.forward(q, k, v, 64, 0.5, rows=rows)
+    np.testing.assert_array_equal(part["idx"], full["idx"][:, :, [1, 6]])
+    np.testing.assert_allclose(part["o"], full["o"][:, :, [1, 6]], rtol=0, atol=0)
+    with pytest.raises(ValueError):
+        oracle.forward(q, k, v, 64, 0.5, rows=np.zeros((3, 3, 2), np.int32))  # B = 2
+    with pytest.raises(ValueError):
+        oracle.forward(q, k, v, 64, 0.5, rows=np.array([[[8]]], np.int32))  # nb = 8
+    with pytest.raises(ValueError):
+        oracle.sparse_attn(q, k, v, full["idx"][:, :, :2], 64, rows=np.array([0, 1], np.int32))
+
+
+def test_bench_cpu_sample_with_several_batch_entries():
+    """The benchmark's oracle sample on a B = 2 workload (one head, sampled
+    query blocks): it runs and counts the tokens of every batch entry."""
+    import bench
+    import workloads as W
+
+    cfg = W.Config("bench_rows", 2, 1024, 2, 64, 64, 0.25, "bf16", 1.0, 78, None)
+    q, k, v = W.make_inputs(cfg, device="cpu")
+    tok, sec, thr = bench.oracle_sample(q, k, v, cfg, [1], 3, seed=5)
+    assert tok == 3 * 64 * 2 and sec > 0 and thr >= 1
