@@ -39,7 +39,7 @@ EXPORTED = ("bsa_topk_count", "bsa_forward_workspace_bytes", "bsa_block_pool",
             "bsa_block_scores_topk_ex", "bsa_sparse_attn_fwd_ex", "bsa_forward_ex",
             "bsa_forward_gqa_workspace_bytes", "bsa_block_scores_topk_gqa", "bsa_sparse_attn_fwd_gqa",
             "bsa_forward_gqa", "bsa_sparse_attn_fwd_train", "bsa_sparse_attn_bwd_workspace_bytes",
-            "bsa_sparse_attn_bwd")
+            "bsa_sparse_attn_bwd", "bsa_forward_host_workspace_bytes", "bsa_forward_host")
 
 #: variant flags of the *_ex entry points (include/bsa.h)
 BSA_FLAG_CAUSAL, BSA_FLAG_FORCE_DIAG = 1, 2
@@ -79,6 +79,8 @@ def _load() -> ctypes.CDLL:
         "bsa_sparse_attn_fwd_train": ([P, P, P, P, P, P, I, I, I, I, I, I, F, I, U, P], I),
         "bsa_sparse_attn_bwd_workspace_bytes": ([I, I, I, I, I], Z),
         "bsa_sparse_attn_bwd": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, U, P, Z, P], I),
+        "bsa_forward_host_workspace_bytes": ([I, I, I, I, I, I, D, I], Z),
+        "bsa_forward_host": ([P, P, P, P, I, I, I, I, I, I, D, I, U, P, Z, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -223,6 +225,49 @@ def bsa_forward(q, k, v, block_size: int, topk_ratio: float, workspace: torch.Te
         _check(lib.bsa_forward(_p(q), _p(k), _p(v), _p(o), B, N, H, D, block_size, float(topk_ratio),
                                _dtype_code(q), _p(workspace), nbytes, _stream(q)))
     return o
+
+
+def bsa_forward_host_workspace_bytes(B: int, N: int, H: int, D: int, block_size: int, topk_ratio: float,
+                                     dtype: torch.dtype, H_kv: int | None = None) -> int:
+    """Device workspace bytes of bsa_forward_host (its two chunk slots)."""
+    code = _dtype_code(torch.empty(0, dtype=dtype))
+    return int(lib.bsa_forward_host_workspace_bytes(B, N, H, H if H_kv is None else H_kv, D, block_size,
+                                                    float(topk_ratio), code))
+
+
+def bsa_forward_host(q, k, v, block_size: int, topk_ratio: float, out: torch.Tensor | None = None,
+                     flags: int = 0, workspace: torch.Tensor | None = None, device=None,
+                     synchronize: bool = True) -> torch.Tensor:
+    """The whole forward from host tensors: q [B, N, H, D], k and v [B, N, H_kv, D]
+    on the CPU (pinned memory lets the copies overlap the compute), o returned
+    (or written to `out`) on the CPU. The library copies head-group chunks to
+    `device` (default: the current CUDA device) on its own streams, computes
+    them on the current stream there and copies the results back. With
+    synchronize=False the call returns once the work is enqueued; the output
+    is complete when the current stream of `device` is."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous CPU tensor")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    B, N, H, D = q.shape
+    Hk = k.shape[2]
+    need = bsa_forward_host_workspace_bytes(B, N, H, D, block_size, topk_ratio, q.dtype, H_kv=Hk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), device=dev, dtype=torch.uint8)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16 if q.dtype == torch.float8_e4m3fn else q.dtype,
+                          pin_memory=True)
+    elif out.is_cuda or not out.is_contiguous():
+        raise ValueError("out must be a contiguous CPU tensor")
+    with torch.cuda.device(dev):
+        st = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+        _check(lib.bsa_forward_host(_p(q), _p(k), _p(v), _p(out), B, N, H, Hk, D, block_size, float(topk_ratio),
+                                    _dtype_code(q), flags, _p(workspace), workspace.numel(), st))
+        if synchronize:
+            torch.cuda.current_stream(dev).synchronize()
+    return out
 
 
 def bsa_sparse_attn_fwd_train(q, k, v, idx, block_size: int, scale: float | None = None, flags: int = 0,

@@ -775,3 +775,156 @@ extern "C" bsa_status bsa_forward_noalloc(const void* q, const void* k, const vo
   return bsa_forward(q, k, v, o, B, N, H, D, block_size, topk_ratio, dt, scratch,
                      static_cast<size_t>(BSA_NOALLOC_SCRATCH_BYTES), stream);
 }
+
+// ---- the whole path from host buffers, copies overlapped with the compute
+
+namespace {
+
+size_t elem_bytes(bsa_dtype dt) { return dt == BSA_F32 ? 4 : (dt == BSA_BF16 ? 2 : 1); }
+size_t out_elem_bytes(bsa_dtype dt) { return dt == BSA_F32 ? 4 : 2; }  // e4m3 inputs give bf16 o
+
+// The job is cut into chunks of (one batch entry, gc consecutive key/value
+// heads with their G query heads each): independent problems, each held on
+// the device as compact [1, N, heads, D] tensors. Two chunk slots let the
+// copies of one chunk run while the other computes.
+constexpr size_t kHostChunkBytes = size_t(64) << 20;  // aim: at least this much input+output per chunk
+
+struct HostPlan {
+  int gc = 0, chunks = 0, slots = 0;
+  size_t q = 0, kv = 0, o = 0, ws = 0, slot = 0, bytes = 0;
+};
+
+HostPlan host_plan(int B, int N, int H, int Hkv, int D, int bs, double ratio, bsa_dtype dt) {
+  HostPlan p;
+  const int G = H / Hkv;
+  const size_t es = elem_bytes(dt), oes = out_elem_bytes(dt);
+  const size_t per_g = static_cast<size_t>(N) * D * (G * es + 2 * es + G * oes);
+  p.gc = Hkv;
+  for (int gc = 1; gc <= Hkv; ++gc)
+    if (Hkv % gc == 0 && static_cast<size_t>(gc) * per_g >= kHostChunkBytes) {
+      p.gc = gc;
+      break;
+    }
+  p.chunks = B * (Hkv / p.gc);
+  p.slots = p.chunks > 1 ? 2 : 1;
+  p.q = align256(static_cast<size_t>(N) * G * p.gc * D * es);
+  p.kv = align256(static_cast<size_t>(N) * p.gc * D * es);
+  p.o = align256(static_cast<size_t>(N) * G * p.gc * D * oes);
+  p.ws = align256(bsa_forward_gqa_workspace_bytes(1, N, G * p.gc, p.gc, D, bs, ratio));
+  p.slot = p.q + 2 * p.kv + p.o + p.ws;
+  p.bytes = p.ws == 0 ? 0 : p.slots * p.slot;
+  return p;
+}
+
+// Per device: the copy-in and copy-out streams and the events that order the
+// chunk slots (guarded by g_host_mu while a call enqueues its work).
+struct HostStreams {
+  bool ready = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, end = nullptr, in[2] = {}, comp[2] = {}, out[2] = {};
+};
+HostStreams g_host[64];
+std::mutex g_host_mu;
+
+bsa_status host_streams(int dev, HostStreams** out) {
+  HostStreams& h = g_host[dev];
+  if (!h.ready) {
+    cudaError_t e = cudaStreamCreateWithFlags(&h.h2d, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h.d2h, cudaStreamNonBlocking);
+    cudaEvent_t* evs[] = {&h.start, &h.end, &h.in[0], &h.in[1], &h.comp[0], &h.comp[1], &h.out[0], &h.out[1]};
+    for (cudaEvent_t* ev : evs)
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "host-path streams and events");
+    h.ready = true;
+  }
+  *out = &h;
+  return BSA_OK;
+}
+
+// The N token rows of a head group as one 2-D copy: `width` bytes per token,
+// rows `spitch` bytes apart in the source and `dpitch` in the destination.
+cudaError_t copy_heads(void* dst, size_t dpitch, const void* src, size_t spitch, size_t width, int N,
+                       cudaMemcpyKind kind, cudaStream_t st) {
+  return cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, static_cast<size_t>(N), kind, st);
+}
+
+}  // namespace
+
+extern "C" size_t bsa_forward_host_workspace_bytes(int B, int N, int H, int H_kv, int D, int block_size,
+                                                   double topk_ratio, bsa_dtype dt) {
+  if (check_dtype(dt) != BSA_OK) return 0;
+  if (check_dims(B, N, H, D, block_size) != BSA_OK || check_heads(H, H_kv) != BSA_OK) return 0;
+  return host_plan(B, N, H, H_kv, D, block_size, topk_ratio, dt).bytes;
+}
+
+extern "C" bsa_status bsa_forward_host(const void* q, const void* k, const void* v, void* o, int B, int N,
+                                       int H, int H_kv, int D, int block_size, double topk_ratio, bsa_dtype dt,
+                                       unsigned flags, void* workspace, size_t workspace_bytes, void* stream) {
+  bsa_status s;
+  if ((s = check_flags(flags)) != BSA_OK) return s;
+  if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
+  if ((s = check_heads(H, H_kv)) != BSA_OK) return s;
+  if ((s = check_dtype(dt)) != BSA_OK) return s;
+  if (!q || !k || !v || !o) return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  const HostPlan p = host_plan(B, N, H, H_kv, D, block_size, topk_ratio, dt);
+  if (p.bytes == 0) return fail(BSA_ERR_INVALID_ARG, "k = int(topk_ratio * nb) < 1 or topk_ratio outside [0, 1]");
+  if (!workspace || workspace_bytes < p.bytes)
+    return fail(BSA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", p.bytes, workspace ? workspace_bytes : 0);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(BSA_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  if ((s = check_device()) != BSA_OK) return s;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(BSA_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  HostStreams* hs = nullptr;
+  if ((s = host_streams(dev, &hs)) != BSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int G = H / H_kv, groups = H_kv / p.gc;
+  const size_t es = elem_bytes(dt), oes = out_elem_bytes(dt);
+  // host rows: one token of all heads; chunk rows: one token of the chunk's heads
+  const size_t q_row = static_cast<size_t>(H) * D * es, kv_row = static_cast<size_t>(H_kv) * D * es;
+  const size_t o_row = static_cast<size_t>(H) * D * oes;
+  const size_t cq_row = static_cast<size_t>(G) * p.gc * D * es, ckv_row = static_cast<size_t>(p.gc) * D * es;
+  const size_t co_row = static_cast<size_t>(G) * p.gc * D * oes;
+  // the internal streams start after the work already on `stream`
+  if ((e = cudaEventRecord(hs->start, st)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = cudaStreamWaitEvent(hs->h2d, hs->start, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
+  if ((e = cudaStreamWaitEvent(hs->d2h, hs->start, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
+  for (int c = 0; c < p.chunks; ++c) {
+    const int sl = c % p.slots, b = c / groups, g0 = (c % groups) * p.gc;
+    unsigned char* base = static_cast<unsigned char*>(workspace) + sl * p.slot;
+    unsigned char *dq = base, *dk = base + p.q, *dv = dk + p.kv, *dout = dv + p.kv, *dws = dout + p.o;
+    const size_t tok = static_cast<size_t>(b) * N;  // first token row of batch entry b
+    const unsigned char* hq = static_cast<const unsigned char*>(q) + tok * q_row + static_cast<size_t>(g0) * G * D * es;
+    const unsigned char* hk = static_cast<const unsigned char*>(k) + tok * kv_row + static_cast<size_t>(g0) * D * es;
+    const unsigned char* hv = static_cast<const unsigned char*>(v) + tok * kv_row + static_cast<size_t>(g0) * D * es;
+    unsigned char* ho = static_cast<unsigned char*>(o) + tok * o_row + static_cast<size_t>(g0) * G * D * oes;
+    // copy in once the slot's previous chunk has been computed
+    if (c >= p.slots && (e = cudaStreamWaitEvent(hs->h2d, hs->comp[sl], 0)) != cudaSuccess)
+      return cuda_fail(e, "stream wait");
+    if ((e = copy_heads(dq, cq_row, hq, q_row, cq_row, N, cudaMemcpyHostToDevice, hs->h2d)) != cudaSuccess ||
+        (e = copy_heads(dk, ckv_row, hk, kv_row, ckv_row, N, cudaMemcpyHostToDevice, hs->h2d)) != cudaSuccess ||
+        (e = copy_heads(dv, ckv_row, hv, kv_row, ckv_row, N, cudaMemcpyHostToDevice, hs->h2d)) != cudaSuccess)
+      return cuda_fail(e, "host to device copy");
+    if ((e = cudaEventRecord(hs->in[sl], hs->h2d)) != cudaSuccess) return cuda_fail(e, "event record");
+    // compute once the inputs are in and the slot's previous output is out
+    if ((e = cudaStreamWaitEvent(st, hs->in[sl], 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
+    if (c >= p.slots && (e = cudaStreamWaitEvent(st, hs->out[sl], 0)) != cudaSuccess)
+      return cuda_fail(e, "stream wait");
+    if ((s = bsa_forward_gqa(dq, dk, dv, dout, 1, N, G * p.gc, p.gc, D, block_size, topk_ratio, dt, flags, dws,
+                             p.ws, st)) != BSA_OK)
+      return s;
+    if ((e = cudaEventRecord(hs->comp[sl], st)) != cudaSuccess) return cuda_fail(e, "event record");
+    // copy out
+    if ((e = cudaStreamWaitEvent(hs->d2h, hs->comp[sl], 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
+    if ((e = copy_heads(ho, o_row, dout, co_row, co_row, N, cudaMemcpyDeviceToHost, hs->d2h)) != cudaSuccess)
+      return cuda_fail(e, "device to host copy");
+    if ((e = cudaEventRecord(hs->out[sl], hs->d2h)) != cudaSuccess) return cuda_fail(e, "event record");
+  }
+  // `stream` continues after the last output copy
+  if ((e = cudaEventRecord(hs->end, hs->d2h)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = cudaStreamWaitEvent(st, hs->end, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
+  return ok();
+}

@@ -204,6 +204,31 @@ bsa_status bsa_forward_gqa(const void* q, const void* k, const void* v, void* o,
                            int H, int H_kv, int D, int block_size, double topk_ratio, bsa_dtype dt,
                            unsigned flags, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- The whole path from host memory ----------------------------------
+ * bsa_forward_gqa on HOST buffers: q [B, N, H, D], k and v [B, N, H_kv, D]
+ * and o [B, N, H, D] live in host memory (page-locked memory lets the copies
+ * run asynchronously). The (batch entry, key/value head) problems are
+ * independent, so the job is cut into chunks of one batch entry and a group
+ * of consecutive key/value heads (with their query heads), sized to at least
+ * 64 MB of inputs and output where the head count allows. Each chunk is
+ * copied into a compact device slot on an internal copy-in stream, computed
+ * on `stream` exactly as bsa_forward_gqa computes it (the same kernels, so
+ * the same results bit for bit), and copied out on an internal copy-out
+ * stream; two slots let the copies of one chunk overlap the compute of the
+ * other. Work already on `stream` is finished before the first copy, and
+ * `stream` resumes after the last output copy: synchronize `stream` before
+ * reading o. The host buffers must stay valid until then.
+ * workspace: device memory of bsa_forward_host_workspace_bytes() bytes,
+ * 256-byte aligned (the chunk slots: q, k, v, o copies and a forward
+ * workspace each). Calls on one device are serialized while they enqueue
+ * (the internal streams are per device). Errors as for bsa_forward_gqa. */
+size_t bsa_forward_host_workspace_bytes(int B, int N, int H, int H_kv, int D, int block_size,
+                                        double topk_ratio, bsa_dtype dt);
+
+bsa_status bsa_forward_host(const void* q, const void* k, const void* v, void* o, int B, int N, int H,
+                            int H_kv, int D, int block_size, double topk_ratio, bsa_dtype dt, unsigned flags,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- Training: forward with the row log-sum-exp, and the backward -------
  * The page listing's step 2 keeps blocks with torch.topk, whose indices
  * carry no gradient, so the backward is the gradient of step 3 (the

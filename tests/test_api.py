@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -134,3 +135,40 @@ def test_ex_entry_points_reject_bad_flags(bsa):
     assert st == 1 and b"CAUSAL" in bsa_lib.bsa_last_error_detail()
     st = bsa_lib.bsa_block_scores_topk_ex(fake, fake, fake, fake, 1, 2, 16, 64, 4, 8, P(0))
     assert st == 1
+
+
+def _host_plan_bytes(B, N, H, Hkv, D, bs, ratio, es, oes, gqa_ws):
+    """bsa_forward_host's workspace, restated from its documented chunking:
+    chunks of one batch entry and the fewest consecutive key/value heads
+    whose inputs and output reach 64 MB (else all of them); two slots of
+    q, k, v, o copies and a forward workspace, each 256-byte aligned, when
+    there is more than one chunk."""
+    a = lambda x: (x + 255) // 256 * 256
+    G = H // Hkv
+    per_g = N * D * (G * es + 2 * es + G * oes)
+    gc = next((g for g in range(1, Hkv + 1) if Hkv % g == 0 and g * per_g >= 64 << 20), Hkv)
+    chunks = B * (Hkv // gc)
+    slot = a(N * G * gc * D * es) + 2 * a(N * gc * D * es) + a(N * G * gc * D * oes) + a(gqa_ws(1, N, G * gc, gc))
+    return (2 if chunks > 1 else 1) * slot
+
+
+@pytest.mark.parametrize("B,N,H,Hkv,D,bs,ratio,dt", [
+    (1, 131072, 16, 16, 128, 128, 0.15, torch.bfloat16),   # one head per chunk, 16 chunks
+    (32, 8192, 16, 16, 64, 64, 0.3, torch.bfloat16),        # one batch entry per chunk
+    (1, 1024, 4, 2, 64, 64, 0.5, torch.float32),            # a single chunk: one slot
+    (2, 65536, 8, 2, 128, 128, 0.2, torch.float8_e4m3fn),   # e4m3 in, bf16 out
+])
+def test_host_workspace_bytes(bsa, B, N, H, Hkv, D, bs, ratio, dt):
+    es = {torch.float32: 4, torch.bfloat16: 2, torch.float8_e4m3fn: 1}[dt]
+    oes = 4 if dt == torch.float32 else 2
+    gqa_ws = lambda b, n, h, hk: bsa.lib.bsa_forward_gqa_workspace_bytes(b, n, h, hk, D, bs, float(ratio))
+    want = _host_plan_bytes(B, N, H, Hkv, D, bs, ratio, es, oes, gqa_ws)
+    assert bsa.bsa_forward_host_workspace_bytes(B, N, H, D, bs, ratio, dt, H_kv=Hkv) == want
+
+
+def test_host_workspace_bytes_rejects_bad_sizes(bsa):
+    f = bsa.lib.bsa_forward_host_workspace_bytes
+    assert f(1, 1000, 2, 2, 64, 64, 0.5, 1) == 0   # N not a multiple of block_size
+    assert f(1, 1024, 3, 2, 64, 64, 0.5, 1) == 0   # H not a multiple of H_kv
+    assert f(1, 1024, 2, 2, 64, 64, 0.01, 1) == 0  # k = 0
+    assert f(1, 1024, 2, 2, 64, 64, 0.5, 7) == 0   # no such dtype
