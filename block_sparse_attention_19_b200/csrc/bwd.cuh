@@ -81,20 +81,28 @@ template <int D>
 struct BwdLayout {
   static constexpr uint32_t kTile = 128 * D * 2;  // a 128-row bf16 tile
   static constexpr int kChunks = D / 64;          // 128-byte column chunks
-  static constexpr uint32_t kOffA = 0;            // dq: Q, dO     dkdv: K, V
-  static constexpr uint32_t kOffRing = 2 * kTile; // dq: K, V x 2  dkdv: Q, dO x 2
-  static constexpr uint32_t kBarOff = kOffRing + 4 * kTile;
+  static constexpr int kXStages = 3, kYStages = 2;
+  static constexpr uint32_t kOffA = 0;                           // dq: Q, dO     dkdv: K, V
+  static constexpr uint32_t kOffX = 2 * kTile;                   // dq: K ring    dkdv: Q ring
+  static constexpr uint32_t kOffY = kOffX + kXStages * kTile;    // dq: V ring    dkdv: dO ring
+  static constexpr uint32_t kBarOff = kOffY + kYStages * kTile;
   static constexpr uint32_t kBytes = kBarOff + 256;
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
+// Ring X holds the operand each tile reads twice, first by the score-like
+// product issued a tile ahead and last by the accumulating product (dq: K;
+// dkdv: Q), so it is three deep; ring Y (dq: V; dkdv: dO) is two deep.
 struct BwdBarriers {
-  uint64_t a_full;        // the two resident tiles
-  uint64_t full[2];       // ring stage holds its two tiles
-  uint64_t empty[2];      // ring stage read by the products
-  uint64_t prod_full;     // phase t: the two score-like products of tile t done
-  uint64_t soft_full;     // phase t: the compute warps stored tile t's bf16 operands
-  uint64_t done;          // the last accumulating products done
+  uint64_t a_full;          // the two resident tiles
+  uint64_t x_full[3], x_empty[3];
+  uint64_t y_full[2], y_empty[2];
+  uint64_t prod_full;       // phase t: both score-like products of tile t done
+  uint64_t s_loaded;        // phase t: the compute warps hold tile t's S (dkdv: S^T)
+  uint64_t p_loaded;        // dq, phase t: the compute warps hold tile t's dP
+  uint64_t soft_full;       // phase t: tile t's bf16 operands stored
+  uint64_t acc_free;        // dq, phase t: dQ += dS(t) K(t) done, the dS columns are free
+  uint64_t done;            // the last accumulating products done
   uint64_t drained;
   uint32_t tmem_base;
   int abort;
@@ -132,7 +140,11 @@ __device__ __forceinline__ void bwd_pack16(const float (&v)[32], uint32_t (&w)[1
 // ---------------------------------------------------------------- dQ
 // grid.x = B * H * nb * (bs / 128): one CTA per 128-row query tile, which
 // walks the key tiles of its query block's kept blocks.
-// TMEM: S [0, 128), dP [128, 256), dQ [256, 256 + D).
+// TMEM: S [0, 128), dP [128, 256), dQ [256, 256 + D), dS (bf16) [384, 448).
+// dS has columns of its own, so the products of tile t+1 need only wait
+// until the compute warps have read tile t's S and dP into registers: dP(t+1)
+// runs while tile t's dS is being computed, S(t+1) right after its last S
+// load, and dQ += dS(t) K(t) after them.
 template <int D, bool kCausal>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -149,7 +161,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   unsigned char* smem = bwd_raw;
   BwdBarriers& bar = *reinterpret_cast<BwdBarriers*>(smem + L::kBarOff);
   volatile int* abort_flag = &bar.abort;
-  constexpr uint32_t kColS = 0, kColP = 128, kColQ = 256;
+  constexpr uint32_t kColS = 0, kColP = 128, kColQ = 256, kColDS = 384;
+  constexpr int XS = L::kXStages, YS = L::kYStages;
 
   const int nb = N / bs, tpb = bs / 128;
   long u = blockIdx.x;
@@ -166,12 +179,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bar.a_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar.full[s], 1);
-      mbar_init(&bar.empty[s], 1);
+    for (int s = 0; s < XS; ++s) {
+      mbar_init(&bar.x_full[s], 1);
+      mbar_init(&bar.x_empty[s], 1);
+    }
+    for (int s = 0; s < YS; ++s) {
+      mbar_init(&bar.y_full[s], 1);
+      mbar_init(&bar.y_empty[s], 1);
     }
     mbar_init(&bar.prod_full, 1);
+    mbar_init(&bar.s_loaded, 4);
+    mbar_init(&bar.p_loaded, 4);
     mbar_init(&bar.soft_full, 4);
+    mbar_init(&bar.acc_free, 1);
     mbar_init(&bar.done, 1);
     mbar_init(&bar.drained, 1);
     bar.abort = 0;
@@ -190,28 +210,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sbase = smem_u32(smem);
 
   if (warp == 0) {
-    // ============================================================ TMA producer
-    if (lane == 0) {
-      const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
-      mbar_arrive_expect_tx(&bar.a_full, 2 * L::kTile);
-      bwd_load_tile<D>(smem + L::kOffA, &tm_q, &bar.a_full, h, qrow0, b, stream);
-      bwd_load_tile<D>(smem + L::kOffA + L::kTile, &tm_do, &bar.a_full, h, qrow0, b, stream);
-      int issued[2] = {0, 0};
+    // ============================================================ TMA producers
+    // lane 0: Q and dO, then the K ring; lane 1: the V ring
+    if (lane < 2) {
+      const bool is_x = lane == 0;
+      const int S = is_x ? XS : YS;
+      uint64_t* full = is_x ? bar.x_full : bar.y_full;
+      uint64_t* empty = is_x ? bar.x_empty : bar.y_empty;
+      const uint32_t ring = is_x ? L::kOffX : L::kOffY;
+      const CUtensorMap* map = is_x ? &tm_k : &tm_v;
+      const uint64_t keep = policy_evict_last();
+      if (is_x) {
+        const uint64_t stream = policy_evict_first();
+        mbar_arrive_expect_tx(&bar.a_full, 2 * L::kTile);
+        bwd_load_tile<D>(smem + L::kOffA, &tm_q, &bar.a_full, h, qrow0, b, stream);
+        bwd_load_tile<D>(smem + L::kOffA + L::kTile, &tm_do, &bar.a_full, h, qrow0, b, stream);
+      }
+      int issued[XS] = {};
       bool ok = true;
       for (int t = 0; t < T && ok; ++t) {
-        const int s = t & 1, use = t >> 1;
+        const int s = t % S, use = t / S;
         const int row = bwd_tile_row(sel, t, 0, bs, nb);
-        if (t >= 2) ok = mbar_wait(&bar.empty[s], (use - 1) & 1, abort_flag, 711);
+        if (t >= S) ok = mbar_wait(&empty[s], (use - 1) & 1, abort_flag, is_x ? 711 : 712);
         if (!ok) break;
-        mbar_arrive_expect_tx(&bar.full[s], 2 * L::kTile);
-        unsigned char* st = smem + L::kOffRing + s * 2 * L::kTile;  // K, then V
-        bwd_load_tile<D>(st, &tm_k, &bar.full[s], h, row, b, keep);
-        bwd_load_tile<D>(st + L::kTile, &tm_v, &bar.full[s], h, row, b, keep);
+        mbar_arrive_expect_tx(&full[s], L::kTile);
+        bwd_load_tile<D>(smem + ring + s * L::kTile, map, &full[s], h, row, b, keep);
         issued[s] = use + 1;
       }
-      mbar_wait_teardown(&bar.a_full, 0);
-      for (int s = 0; s < 2; ++s)
-        if (issued[s]) mbar_wait_teardown(&bar.full[s], (issued[s] - 1) & 1);
+      if (is_x) mbar_wait_teardown(&bar.a_full, 0);
+      for (int s = 0; s < S; ++s)
+        if (issued[s]) mbar_wait_teardown(&full[s], (issued[s] - 1) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -221,44 +249,59 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t id_q = idesc_bf16_f32(128, D, 0, 1);  // dS from TMEM, K used MN-major
       const uint64_t dqd = smem_desc_sw128(sbase + L::kOffA, 16, 1024);
       const uint64_t ddo = smem_desc_sw128(sbase + L::kOffA + L::kTile, 16, 1024);
-      const uint64_t dring = smem_desc_sw128(sbase + L::kOffRing, 16, 1024);           // K-major
-      const uint64_t dring_mn = smem_desc_sw128(sbase + L::kOffRing, 128 * 128, 1024);  // MN-major
+      const uint64_t dx = smem_desc_sw128(sbase + L::kOffX, 16, 1024);              // K, K-major
+      const uint64_t dx_mn = smem_desc_sw128(sbase + L::kOffX, 128 * 128, 1024);    // K, MN-major
+      const uint64_t dy = smem_desc_sw128(sbase + L::kOffY, 16, 1024);              // V, K-major
       constexpr uint64_t kStep = L::kTile >> 4;
       bool ok = mbar_wait(&bar.a_full, 0, abort_flag, 721);
-      for (int t = 0; t <= T && ok; ++t) {
-        if (t > 0) {
-          // dQ += dS(t-1) K(t-1); dS is bf16 over the first 64 columns of S
-          ok = mbar_wait(&bar.soft_full, (t - 1) & 1, abort_flag, 722);
-          if (!ok) break;
-          tc_fence_after();
-          const int s = (t - 1) & 1;
-          const uint64_t dk = dring_mn + (2 * s) * kStep;
+      // dP(t) = dO V(t)^T; frees its V ring entry when done
+      auto issue_dp = [&](int t) {
+        ok = ok && mbar_wait(&bar.y_full[t % YS], (t / YS) & 1, abort_flag, 723);
+        if (!ok) return;
+        tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts(tmem + kColQ, tmem + kColS + kk * 8, dk + ((kk * 16 * 128) >> 4), id_q,
-                        (t > 1 || kk > 0) ? 1u : 0u);
-          mma_commit(&bar.empty[s]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+          mma_bf16_ss(tmem + kColP, ddo + off, dy + (t % YS) * kStep + off, id_s, kk > 0 ? 1u : 0u);
         }
-        if (t < T) {
-          // S(t) = Q K(t)^T and dP(t) = dO V(t)^T (issued after dQ(t-1), which
-          // reads the dS these overwrite: the tensor pipe runs them in order)
-          const int s = t & 1;
-          ok = mbar_wait(&bar.full[s], (t >> 1) & 1, abort_flag, 723);
+        mma_commit(&bar.y_empty[t % YS]);
+      };
+      // S(t) = Q K(t)^T
+      auto issue_s = [&](int t) {
+        ok = ok && mbar_wait(&bar.x_full[t % XS], (t / XS) & 1, abort_flag, 724);
+        if (!ok) return;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+          mma_bf16_ss(tmem + kColS, dqd + off, dx + (t % XS) * kStep + off, id_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      if (T > 0) {
+        issue_dp(0);
+        issue_s(0);
+        if (ok) mma_commit(&bar.prod_full);
+      }
+      for (int t = 0; t < T && ok; ++t) {
+        if (t + 1 < T) {
+          // tile t+1's products overwrite S and dP once the compute warps hold them
+          ok = mbar_wait(&bar.p_loaded, t & 1, abort_flag, 725);
+          issue_dp(t + 1);
+          ok = ok && mbar_wait(&bar.s_loaded, t & 1, abort_flag, 726);
+          issue_s(t + 1);
           if (!ok) break;
-          tc_fence_after();
-          const uint64_t dk = dring + (2 * s) * kStep, dv = dring + (2 * s + 1) * kStep;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
-            mma_bf16_ss(tmem + kColS, dqd + off, dk + off, id_s, kk > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
-            mma_bf16_ss(tmem + kColP, ddo + off, dv + off, id_s, kk > 0 ? 1u : 0u);
-          }
           mma_commit(&bar.prod_full);
         }
+        // dQ += dS(t) K(t)
+        ok = mbar_wait(&bar.soft_full, t & 1, abort_flag, 722);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + kColQ, tmem + kColDS + kk * 8, dx_mn + (t % XS) * kStep + ((kk * 16 * 128) >> 4), id_q,
+                      (t > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bar.x_empty[t % XS]);
+        mma_commit(&bar.acc_free);
       }
       if (ok) mma_commit(&bar.done);
       mma_commit(&bar.drained);
@@ -280,22 +323,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       // keys c of this tile with kbase + c > n are masked (causal)
       const int lim = kCausal ? static_cast<int>(n - bwd_tile_row(sel, t, 0, bs, nb)) : (1 << 30);
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sv[32], pv[32];
+      // the whole dP row, then the tensor core may overwrite it
+      uint32_t p0[32], p1[32], p2[32], p3[32];
+      tmem_ld32(lane_base + kColP, p0);
+      tmem_ld32(lane_base + kColP + 32, p1);
+      tmem_ld32(lane_base + kColP + 64, p2);
+      tmem_ld32(lane_base + kColP + 96, p3);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.p_loaded);
+      // S in 32-column pieces; dS packed to bf16 as it is made
+      uint32_t w0[16], w1[16], w2[16], w3[16];
+      auto piece = [&](int c, const uint32_t (&pv)[32], uint32_t (&w)[16]) {
+        uint32_t sv[32];
         tmem_ld32(lane_base + kColS + c * 32, sv);
-        tmem_ld32(lane_base + kColP + c * 32, pv);
         tmem_wait_ld();
+        if (c == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar.s_loaded);
+        }
         float ds[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const float p = (c * 32 + e > lim) ? 0.f : fast_exp2(fmaf(__uint_as_float(sv[e]), scale_log2, -lse2));
           ds[e] = p * (__uint_as_float(pv[e]) - dn);
         }
-        uint32_t w[16];
         bwd_pack16(ds, w);
-        tmem_st16(lane_base + kColS + c * 16, w);  // over S columns already read
+      };
+      piece(0, p0, w0);
+      piece(1, p1, w1);
+      piece(2, p2, w2);
+      piece(3, p3, w3);
+      // the dS columns are free once dQ(t-1) has read them
+      if (t > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar.acc_free, (t - 1) & 1, abort_flag, 733));
+        if (!ok) break;
+        tc_fence_after();
       }
+      tmem_st16(lane_base + kColDS, w0);
+      tmem_st16(lane_base + kColDS + 16, w1);
+      tmem_st16(lane_base + kColDS + 32, w2);
+      tmem_st16(lane_base + kColDS + 48, w3);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -344,6 +414,10 @@ __device__ __forceinline__ int bwd_next_block(const uint32_t* row, int words, in
 // grid.x = B * H * nb * (bs / 128): one CTA per 128-key tile, which walks the
 // query tiles of the query blocks that kept its block (bit row of `mask`).
 // TMEM: S^T [0, 128), dP^T [128, 256), dV [256, 256 + D), dK [256 + D, 256 + 2D).
+// The compute warps read the whole S^T row first, so S^T(t+1) is computed
+// while tile t's P^T and dS^T are made; those go over dP^T, 32-query piece
+// c at columns 128 + 32c: P^T in its first 16 columns, dS^T in the last 16
+// (each piece is read before it is overwritten).
 template <int D, bool kCausal>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -362,6 +436,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   BwdBarriers& bar = *reinterpret_cast<BwdBarriers*>(smem + L::kBarOff);
   volatile int* abort_flag = &bar.abort;
   constexpr uint32_t kColS = 0, kColP = 128, kColV = 256, kColK = 256 + D;
+  constexpr int XS = L::kXStages, YS = L::kYStages;
 
   const int nb = N / bs, tpb = bs / 128, words = (nb + 31) / 32;
   long u = blockIdx.x;
@@ -378,11 +453,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bar.a_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar.full[s], 1);
-      mbar_init(&bar.empty[s], 1);
+    for (int s = 0; s < XS; ++s) {
+      mbar_init(&bar.x_full[s], 1);
+      mbar_init(&bar.x_empty[s], 1);
+    }
+    for (int s = 0; s < YS; ++s) {
+      mbar_init(&bar.y_full[s], 1);
+      mbar_init(&bar.y_empty[s], 1);
     }
     mbar_init(&bar.prod_full, 1);
+    mbar_init(&bar.s_loaded, 4);
     mbar_init(&bar.soft_full, 4);
     mbar_init(&bar.done, 1);
     mbar_init(&bar.drained, 1);
@@ -404,31 +484,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sbase = smem_u32(smem);
 
   if (warp == 0) {
-    // ============================================================ TMA producer
-    if (lane == 0 && U > 0) {
-      const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
-      mbar_arrive_expect_tx(&bar.a_full, 2 * L::kTile);
-      bwd_load_tile<D>(smem + L::kOffA, &tm_k, &bar.a_full, h, krow0, b, stream);
-      bwd_load_tile<D>(smem + L::kOffA + L::kTile, &tm_v, &bar.a_full, h, krow0, b, stream);
-      int issued[2] = {0, 0};
+    // ============================================================ TMA producers
+    // lane 0: K and V, then the Q ring; lane 1: the dO ring
+    if (lane < 2 && U > 0) {
+      const bool is_x = lane == 0;
+      const int S = is_x ? XS : YS;
+      uint64_t* full = is_x ? bar.x_full : bar.y_full;
+      uint64_t* empty = is_x ? bar.x_empty : bar.y_empty;
+      const uint32_t ring = is_x ? L::kOffX : L::kOffY;
+      const CUtensorMap* map = is_x ? &tm_q : &tm_do;
+      const uint64_t keep = policy_evict_last();
+      if (is_x) {
+        const uint64_t stream = policy_evict_first();
+        mbar_arrive_expect_tx(&bar.a_full, 2 * L::kTile);
+        bwd_load_tile<D>(smem + L::kOffA, &tm_k, &bar.a_full, h, krow0, b, stream);
+        bwd_load_tile<D>(smem + L::kOffA + L::kTile, &tm_v, &bar.a_full, h, krow0, b, stream);
+      }
+      int issued[XS] = {};
       bool ok = true;
       int w = 0, qb = 0;
       uint32_t cur = __ldg(mrow);
       for (int t = 0; t < U && ok; ++t) {
         if (t % tpb == 0) qb = bwd_next_block(mrow, words, w, cur);
-        const int s = t & 1, use = t >> 1;
+        const int s = t % S, use = t / S;
         const int row = qb * bs + (t % tpb) * 128;
-        if (t >= 2) ok = mbar_wait(&bar.empty[s], (use - 1) & 1, abort_flag, 741);
+        if (t >= S) ok = mbar_wait(&empty[s], (use - 1) & 1, abort_flag, is_x ? 741 : 742);
         if (!ok) break;
-        mbar_arrive_expect_tx(&bar.full[s], 2 * L::kTile);
-        unsigned char* st = smem + L::kOffRing + s * 2 * L::kTile;  // Q, then dO
-        bwd_load_tile<D>(st, &tm_q, &bar.full[s], h, row, b, keep);
-        bwd_load_tile<D>(st + L::kTile, &tm_do, &bar.full[s], h, row, b, keep);
+        mbar_arrive_expect_tx(&full[s], L::kTile);
+        bwd_load_tile<D>(smem + ring + s * L::kTile, map, &full[s], h, row, b, keep);
         issued[s] = use + 1;
       }
-      mbar_wait_teardown(&bar.a_full, 0);
-      for (int s = 0; s < 2; ++s)
-        if (issued[s]) mbar_wait_teardown(&bar.full[s], (issued[s] - 1) & 1);
+      if (is_x) mbar_wait_teardown(&bar.a_full, 0);
+      for (int s = 0; s < S; ++s)
+        if (issued[s]) mbar_wait_teardown(&full[s], (issued[s] - 1) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -438,46 +526,64 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t id_a = idesc_bf16_f32(128, D, 0, 1);  // P^T / dS^T from TMEM, dO / Q MN-major
       const uint64_t dkd = smem_desc_sw128(sbase + L::kOffA, 16, 1024);
       const uint64_t dvd = smem_desc_sw128(sbase + L::kOffA + L::kTile, 16, 1024);
-      const uint64_t dring = smem_desc_sw128(sbase + L::kOffRing, 16, 1024);           // K-major
-      const uint64_t dring_mn = smem_desc_sw128(sbase + L::kOffRing, 128 * 128, 1024);  // MN-major
+      const uint64_t dx = smem_desc_sw128(sbase + L::kOffX, 16, 1024);              // Q, K-major
+      const uint64_t dx_mn = smem_desc_sw128(sbase + L::kOffX, 128 * 128, 1024);    // Q, MN-major
+      const uint64_t dy = smem_desc_sw128(sbase + L::kOffY, 16, 1024);              // dO, K-major
+      const uint64_t dy_mn = smem_desc_sw128(sbase + L::kOffY, 128 * 128, 1024);    // dO, MN-major
       constexpr uint64_t kStep = L::kTile >> 4;
       bool ok = mbar_wait(&bar.a_full, 0, abort_flag, 751);
-      for (int t = 0; t <= U && ok; ++t) {
-        if (t > 0) {
-          // dV += P^T(t-1) dO(t-1), dK += dS^T(t-1) Q(t-1)
-          ok = mbar_wait(&bar.soft_full, (t - 1) & 1, abort_flag, 752);
-          if (!ok) break;
-          tc_fence_after();
-          const int s = (t - 1) & 1;
-          const uint64_t dq_mn = dring_mn + (2 * s) * kStep, ddo_mn = dring_mn + (2 * s + 1) * kStep;
+      // S^T(t) = K Q(t)^T
+      auto issue_s = [&](int t) {
+        ok = ok && mbar_wait(&bar.x_full[t % XS], (t / XS) & 1, abort_flag, 753);
+        if (!ok) return;
+        tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts(tmem + kColV, tmem + kColS + kk * 8, ddo_mn + ((kk * 16 * 128) >> 4), id_a,
-                        (t > 1 || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts(tmem + kColK, tmem + kColP + kk * 8, dq_mn + ((kk * 16 * 128) >> 4), id_a,
-                        (t > 1 || kk > 0) ? 1u : 0u);
-          mma_commit(&bar.empty[s]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+          mma_bf16_ss(tmem + kColS, dkd + off, dx + (t % XS) * kStep + off, id_s, kk > 0 ? 1u : 0u);
         }
-        if (t < U) {
-          // S^T(t) = K Q(t)^T and dP^T(t) = V dO(t)^T (after the products above,
-          // which read the P^T / dS^T these overwrite; the pipe runs in order)
-          const int s = t & 1;
-          ok = mbar_wait(&bar.full[s], (t >> 1) & 1, abort_flag, 753);
+      };
+      // dP^T(t) = V dO(t)^T
+      auto issue_dp = [&](int t) {
+        ok = ok && mbar_wait(&bar.y_full[t % YS], (t / YS) & 1, abort_flag, 754);
+        if (!ok) return;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+          mma_bf16_ss(tmem + kColP, dvd + off, dy + (t % YS) * kStep + off, id_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      issue_s(0);
+      issue_dp(0);
+      if (ok) mma_commit(&bar.prod_full);
+      for (int t = 0; t < U && ok; ++t) {
+        // S^T(t+1) once the compute warps hold S^T(t)
+        if (t + 1 < U) {
+          ok = mbar_wait(&bar.s_loaded, t & 1, abort_flag, 755);
+          issue_s(t + 1);
           if (!ok) break;
-          tc_fence_after();
-          const uint64_t dqk = dring + (2 * s) * kStep, ddok = dring + (2 * s + 1) * kStep;
+        }
+        // dV += P^T(t) dO(t), dK += dS^T(t) Q(t); the 16 queries of
+        // instruction kk sit in piece kk / 2, at its column 8 (kk % 2)
+        ok = mbar_wait(&bar.soft_full, t & 1, abort_flag, 752);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dq_mn = dx_mn + (t % XS) * kStep, ddo_mn = dy_mn + (t % YS) * kStep;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
-            mma_bf16_ss(tmem + kColS, dkd + off, dqk + off, id_s, kk > 0 ? 1u : 0u);
-          }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + kColV, tmem + kColP + 32 * (kk / 2) + 8 * (kk % 2), ddo_mn + ((kk * 16 * 128) >> 4),
+                      id_a, (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
-            mma_bf16_ss(tmem + kColP, dvd + off, ddok + off, id_s, kk > 0 ? 1u : 0u);
-          }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + kColK, tmem + kColP + 32 * (kk / 2) + 8 * (kk % 2) + 16,
+                      dq_mn + ((kk * 16 * 128) >> 4), id_a, (t > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bar.x_empty[t % XS]);
+        mma_commit(&bar.y_empty[t % YS]);
+        // dP^T(t+1) overwrites the columns the products above read (in order)
+        if (t + 1 < U) {
+          issue_dp(t + 1);
+          if (!ok) break;
           mma_commit(&bar.prod_full);
         }
       }
@@ -501,14 +607,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&bar.prod_full, t & 1, abort_flag, 761));
       if (!ok) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        // this chunk's 32 query columns: ln-sum (as log2) and D of each, one per lane
+      // the whole S^T row, then the tensor core may overwrite it
+      uint32_t s0[32], s1[32], s2[32], s3[32];
+      tmem_ld32(lane_base + kColS, s0);
+      tmem_ld32(lane_base + kColS + 32, s1);
+      tmem_ld32(lane_base + kColS + 64, s2);
+      tmem_ld32(lane_base + kColS + 96, s3);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.s_loaded);
+      auto piece = [&](int c, const uint32_t (&sv)[32]) {
+        // this piece's 32 query columns: ln-sum (as log2) and D of each, one per lane
         const long qn = qrow0 + c * 32 + lane;
         const float lse_l = __ldg(lse + bh * N + qn) * 1.4426950408889634f;
         const float dn_l = __ldg(dsum + bh * N + qn);
-        uint32_t sv[32], pv[32];
-        tmem_ld32(lane_base + kColS + c * 32, sv);
+        uint32_t pv[32];
         tmem_ld32(lane_base + kColP + c * 32, pv);
         tmem_wait_ld();
         float pt[32], dst[32];
@@ -524,9 +638,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t wp[16], wd[16];
         bwd_pack16(pt, wp);
         bwd_pack16(dst, wd);
-        tmem_st16(lane_base + kColS + c * 16, wp);  // over S^T columns already read
-        tmem_st16(lane_base + kColP + c * 16, wd);  // over dP^T columns already read
-      }
+        tmem_st16(lane_base + kColP + c * 32, wp);       // over dP^T columns this piece has read
+        tmem_st16(lane_base + kColP + c * 32 + 16, wd);
+      };
+      piece(0, s0);
+      piece(1, s1);
+      piece(2, s2);
+      piece(3, s3);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
