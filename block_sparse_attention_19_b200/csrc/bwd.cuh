@@ -86,7 +86,8 @@ struct BwdLayout {
   static constexpr uint32_t kOffX = 2 * kTile;                   // dq: K ring    dkdv: Q ring
   static constexpr uint32_t kOffY = kOffX + kXStages * kTile;    // dq: V ring    dkdv: dO ring
   static constexpr uint32_t kBarOff = kOffY + kYStages * kTile;
-  static constexpr uint32_t kBytes = kBarOff + 256;
+  static constexpr uint32_t kStatOff = kBarOff + 256;  // dkdv: float [2 tiles][lse2, D][128 queries]
+  static constexpr uint32_t kBytes = kStatOff + 2 * 2 * 128 * 4;
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
@@ -101,6 +102,8 @@ struct BwdBarriers {
   uint64_t s_loaded;        // phase t: the compute warps hold tile t's S (dkdv: S^T)
   uint64_t p_loaded;        // dq, phase t: the compute warps hold tile t's dP
   uint64_t soft_full;       // phase t: tile t's bf16 operands stored
+  uint64_t half_full;       // dkdv, phase t: the operands of tile t's first 64 queries stored
+  uint64_t stats_ready[2];  // dkdv, tile t's query statistics in shared memory (slot t % 2)
   uint64_t acc_free;        // dq, phase t: dQ += dS(t) K(t) done, the dS columns are free
   uint64_t done;            // the last accumulating products done
   uint64_t drained;
@@ -464,6 +467,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&bar.prod_full, 1);
     mbar_init(&bar.s_loaded, 4);
     mbar_init(&bar.soft_full, 4);
+    mbar_init(&bar.half_full, 4);
+    for (int s = 0; s < 2; ++s) mbar_init(&bar.stats_ready[s], 4);
     mbar_init(&bar.done, 1);
     mbar_init(&bar.drained, 1);
     bar.abort = 0;
@@ -564,20 +569,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           issue_s(t + 1);
           if (!ok) break;
         }
-        // dV += P^T(t) dO(t), dK += dS^T(t) Q(t); the 16 queries of
+        // dV += P^T(t) dO(t), dK += dS^T(t) Q(t), queries 0-63 as soon as
+        // their operands are stored, then 64-127; the 16 queries of
         // instruction kk sit in piece kk / 2, at its column 8 (kk % 2)
-        ok = mbar_wait(&bar.soft_full, t & 1, abort_flag, 752);
-        if (!ok) break;
-        tc_fence_after();
         const uint64_t dq_mn = dx_mn + (t % XS) * kStep, ddo_mn = dy_mn + (t % YS) * kStep;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + kColV, tmem + kColP + 32 * (kk / 2) + 8 * (kk % 2), ddo_mn + ((kk * 16 * 128) >> 4),
-                      id_a, (t > 0 || kk > 0) ? 1u : 0u);
+        for (int hq = 0; hq < 2; ++hq) {
+          ok = mbar_wait(hq == 0 ? &bar.half_full : &bar.soft_full, t & 1, abort_flag, hq == 0 ? 756 : 752);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + kColK, tmem + kColP + 32 * (kk / 2) + 8 * (kk % 2) + 16,
-                      dq_mn + ((kk * 16 * 128) >> 4), id_a, (t > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 4 * hq; kk < 4 * hq + 4; ++kk)
+            mma_bf16_ts(tmem + kColV, tmem + kColP + 32 * (kk / 2) + 8 * (kk % 2), ddo_mn + ((kk * 16 * 128) >> 4),
+                        id_a, (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 4 * hq; kk < 4 * hq + 4; ++kk)
+            mma_bf16_ts(tmem + kColK, tmem + kColP + 32 * (kk / 2) + 8 * (kk % 2) + 16,
+                        dq_mn + ((kk * 16 * 128) >> 4), id_a, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (!ok) break;
         mma_commit(&bar.x_empty[t % XS]);
         mma_commit(&bar.y_empty[t % YS]);
         // dP^T(t+1) overwrites the columns the products above read (in order)
@@ -601,9 +611,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     int w = 0, qb = 0;
     uint32_t cur = __ldg(mrow);
+    float* stats = reinterpret_cast<float*>(smem + L::kStatOff);
     for (int t = 0; t < U; ++t) {
       if (t % tpb == 0) qb = bwd_next_block(mrow, words, w, cur);
       const int qrow0 = qb * bs + (t % tpb) * 128;
+      // the tile's per-query ln-sum (as log2) and D, one query per thread,
+      // into slot t % 2. The slot's previous tile, t - 2, is done: this warp
+      // has seen tile t - 1's products complete, which the MMA thread issues
+      // only after every compute warp has stored tile t - 2's operands.
+      float* st_lse = stats + (t & 1) * 256;
+      float* st_dn = st_lse + 128;
+      st_lse[kr] = __ldg(lse + bh * N + qrow0 + kr) * 1.4426950408889634f;
+      st_dn[kr] = __ldg(dsum + bh * N + qrow0 + kr);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.stats_ready[t & 1]);
       ok = __all_sync(0xffffffffu, mbar_wait(&bar.prod_full, t & 1, abort_flag, 761));
       if (!ok) break;
       tc_fence_after();
@@ -617,19 +638,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.s_loaded);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar.stats_ready[t & 1], (t >> 1) & 1, abort_flag, 763));
+      if (!ok) break;
       auto piece = [&](int c, const uint32_t (&sv)[32]) {
-        // this piece's 32 query columns: ln-sum (as log2) and D of each, one per lane
-        const long qn = qrow0 + c * 32 + lane;
-        const float lse_l = __ldg(lse + bh * N + qn) * 1.4426950408889634f;
-        const float dn_l = __ldg(dsum + bh * N + qn);
         uint32_t pv[32];
         tmem_ld32(lane_base + kColP + c * 32, pv);
         tmem_wait_ld();
+        // this piece's 32 query columns (the same for every lane: broadcast reads)
+        float lq[32], dq_[32];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 a = *reinterpret_cast<const float4*>(st_lse + c * 32 + e);
+          const float4 d = *reinterpret_cast<const float4*>(st_dn + c * 32 + e);
+          lq[e] = a.x, lq[e + 1] = a.y, lq[e + 2] = a.z, lq[e + 3] = a.w;
+          dq_[e] = d.x, dq_[e + 1] = d.y, dq_[e + 2] = d.z, dq_[e + 3] = d.w;
+        }
         float pt[32], dst[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float lse2 = __shfl_sync(0xffffffffu, lse_l, e);
-          const float dn = __shfl_sync(0xffffffffu, dn_l, e);
+          const float lse2 = lq[e];
+          const float dn = dq_[e];
           const bool masked = kCausal && key > qrow0 + c * 32 + e;
           const float p = masked ? 0.f : fast_exp2(fmaf(__uint_as_float(sv[e]), scale_log2, -lse2));
           pt[e] = p;
@@ -643,6 +671,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       };
       piece(0, s0);
       piece(1, s1);
+      // queries 0-63 are ready for the accumulating products
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.half_full);
       piece(2, s2);
       piece(3, s3);
       tmem_wait_st();
