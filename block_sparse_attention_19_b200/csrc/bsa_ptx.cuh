@@ -392,25 +392,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x on the FMA/ALU pipes, for x <= 8: round-to-nearest split x = n + f with
-// f in [-1/2, 1/2] (adding and subtracting 1.5 * 2^23), a degree-4 polynomial
-// for 2^f fitted here by Remez exchange on the relative error (max 2.7e-6),
-// and n added to the exponent field. Inputs below -125 are clamped (2^-125 is
-// negligible next to the row sum, which is at least 1).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.0f);
-  const float kRound = 12582912.0f;  // 1.5 * 2^23
-  const float t = x + kRound;
-  const int n = __float_as_int(t) - __float_as_int(kRound);
-  const float f = x - (t - kRound);
-  float p = 0.009570102207362652f;
-  p = fmaf(p, f, 0.05591785907745361f);
-  p = fmaf(p, f, 0.240247443318367f);
-  p = fmaf(p, f, 0.6931217908859253f);
-  p = fmaf(p, f, 0.9999992847442627f);
-  return __int_as_float(__float_as_int(p) + (n << 23));
-}
-
 // ---- packed two-wide float32 arithmetic (sm_100): one instruction per pair
 __device__ __forceinline__ uint64_t f2(float lo, float hi) {
   uint64_t r;
@@ -441,8 +422,16 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// exp2_poly on a pair: the same range split and polynomial, two lanes per
-// instruction where the operation allows it.
+// 2^x for a pair of floats on the FMA/ALU pipes, for x <= 8: round-to-nearest
+// split x = n + f with f in [-1/2, 1/2] (adding and subtracting 1.5 * 2^23),
+// a degree-3 polynomial for 2^f fitted here by Remez exchange on the relative
+// error (max 7.5e-5 in float32, far below the 2^-9 of the bf16 P it feeds),
+// and n added to the exponent field. The low 9 bits of the rounding constant
+// are zero, so bits(x + 1.5 * 2^23) << 23 equals n << 23 and one integer
+// multiply-add adds it. Inputs below -125 are clamped (2^-125 is negligible
+// next to the row sum, which is at least 1).
+constexpr float kExp2C0 = 0.9999280571937561f, kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f, kExp2C3 = 0.0551716685295105f;
 __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
   float x0, x1;
   f2_split(x2, x0, x1);
@@ -451,17 +440,15 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
   const uint64_t r2 = f2(kRound, kRound);
   const uint64_t t2 = f2_add(x2, r2);
   const uint64_t f = f2_sub(x2, f2_sub(t2, r2));
-  uint64_t p = f2(0.009570102207362652f, 0.009570102207362652f);
-  p = f2_fma(p, f, f2(0.05591785907745361f, 0.05591785907745361f));
-  p = f2_fma(p, f, f2(0.240247443318367f, 0.240247443318367f));
-  p = f2_fma(p, f, f2(0.6931217908859253f, 0.6931217908859253f));
-  p = f2_fma(p, f, f2(0.9999992847442627f, 0.9999992847442627f));
+  uint64_t p = f2(kExp2C3, kExp2C3);
+  p = f2_fma(p, f, f2(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2(kExp2C0, kExp2C0));
   float t0, t1, p0, p1;
   f2_split(t2, t0, t1);
   f2_split(p, p0, p1);
-  const int n0 = __float_as_int(t0) - __float_as_int(kRound);
-  const int n1 = __float_as_int(t1) - __float_as_int(kRound);
-  return f2(__int_as_float(__float_as_int(p0) + (n0 << 23)), __int_as_float(__float_as_int(p1) + (n1 << 23)));
+  return f2(__int_as_float(__float_as_int(t0) * 8388608 + __float_as_int(p0)),
+            __int_as_float(__float_as_int(t1) * 8388608 + __float_as_int(p1)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

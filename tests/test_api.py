@@ -172,3 +172,29 @@ def test_host_workspace_bytes_rejects_bad_sizes(bsa):
     assert f(1, 1024, 3, 2, 64, 64, 0.5, 1) == 0   # H not a multiple of H_kv
     assert f(1, 1024, 2, 2, 64, 64, 0.01, 1) == 0  # k = 0
     assert f(1, 1024, 2, 2, 64, 64, 0.5, 7) == 0   # no such dtype
+
+
+def test_polynomial_exp2_of_the_softmax():
+    """The kernels' polynomial 2^x (one key pair in four of the softmax), as
+    the header defines it, evaluated step by step in float32: the range
+    split, the degree-3 polynomial and the exponent added through
+    bits(x + 1.5 * 2^23) << 23. Its relative error stays below 1e-4 on the
+    range the softmax uses (far below the bf16 rounding of P, 2^-9), and the
+    clamp gives 2^-125-sized values below it."""
+    import numpy as np
+
+    src = open(os.path.join(ROOT, "block_sparse_attention_19_b200", "csrc", "bsa_ptx.cuh")).read()
+    c = {k: np.float32(v) for k, v in re.findall(r"(kExp2C\d) = ([0-9.e+-]+)f", src)}
+    assert len(c) == 4
+    x = np.concatenate([np.linspace(-30, 8, 2_000_001), [-124.9, -125.0, -200.0, -1e30]]).astype(np.float32)
+    xc = np.maximum(x, np.float32(-125.0))
+    rnd = np.float32(12582912.0)
+    t = (xc + rnd).astype(np.float32)
+    f = (xc - (t - rnd)).astype(np.float32)
+    p = c["kExp2C3"]
+    for k in ("kExp2C2", "kExp2C1", "kExp2C0"):
+        p = (p * f + c[k]).astype(np.float32)
+    bits = (t.view(np.int32).astype(np.int64) * 8388608 + p.view(np.int32).astype(np.int64)) & 0xFFFFFFFF
+    y = bits.astype(np.uint32).view(np.float32).astype(np.float64)
+    ref = np.exp2(np.maximum(x.astype(np.float64), -125.0))
+    assert np.all(np.abs(y / ref - 1) < 1e-4), np.abs(y / ref - 1).max()

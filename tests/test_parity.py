@@ -85,6 +85,7 @@ def check_output(o_gpu: np.ndarray, o_ref: np.ndarray, dtype: str):
         assert d.max() <= 1e-4, f"max|d| = {d.max()}"
     else:
         rel = np.linalg.norm(o_gpu - o_ref) / np.linalg.norm(o_ref)
+        print(f"{dtype}: max|d| {d.max():.3g}, rel L2 {rel:.3g}")
         assert d.max() <= 2e-2, f"max|d| = {d.max()}"
         assert rel <= 5e-3, f"rel L2 = {rel}"
 
