@@ -194,10 +194,12 @@ def run_backward(args, cfg, dev, rank, world, dist, bsa, flags, variant):
     q, k, v = W.make_inputs(cfg, device=dev)
     g = torch.Generator(device=dev).manual_seed(cfg.seed + 77)
     do = torch.randn(q.shape, generator=g, device=dev, dtype=torch.float32).to(q.dtype)
-    ws = torch.empty(bsa.bsa_forward_workspace_bytes(B, N, H, D, bs, ratio), device=dev, dtype=torch.uint8)
+    Hk = cfg.Hkv  # key/value heads (fewer than H with grouped queries)
+    ws = torch.empty(bsa.bsa_forward_workspace_bytes(B, N, H, D, bs, ratio, H_kv=Hk), device=dev, dtype=torch.uint8)
     bsa.bsa_forward(q, k, v, bs, ratio, workspace=ws, flags=flags)  # the selection the step trains through
-    idx = bsa.workspace_views(ws, B, N, H, D, bs, ratio)[2].clone()
-    bws = torch.empty(bsa.lib.bsa_sparse_attn_bwd_workspace_bytes(B, N, H, D, bs), device=dev, dtype=torch.uint8)
+    idx = bsa.workspace_views(ws, B, N, H, D, bs, ratio, H_kv=Hk)[2].clone()
+    bws = torch.empty(bsa.lib.bsa_sparse_attn_bwd_gqa_workspace_bytes(B, N, H, Hk, D, bs), device=dev,
+                      dtype=torch.uint8)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
 
@@ -239,8 +241,8 @@ def run_backward(args, cfg, dev, rank, world, dist, bsa, flags, variant):
 
     # end to end through the public API: host inputs in, gradients out
     hq, hk, hv, hdo = (x.cpu().pin_memory() for x in (q, k, v, do))
-    hg = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(3)]
-    dq_, dk_, dv_, ddo = (torch.empty_like(q) for _ in range(4))
+    hg = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (q, k, v)]  # dq, dk, dv
+    dq_, dk_, dv_, ddo = (torch.empty_like(x) for x in (q, k, v, do))  # device copies of q, k, v, dO
 
     def e2e_step():
         for d_, h_ in ((dq_, hq), (dk_, hk), (dv_, hv), (ddo, hdo)):
@@ -265,11 +267,12 @@ def run_backward(args, cfg, dev, rank, world, dist, bsa, flags, variant):
         il = idx.cpu().numpy().astype(np.int64)
         qi = np.arange(N // bs)[None, None, :, None]
         pairs = np.where(il < 0, 0, np.where(il < qi, bs * bs, bs * (bs + 1) // 2)).sum()
-        flops_f = 4.0 * D * float(pairs)
+        flops_f = 4.0 * D * float(pairs) * (H // Hk)  # each key/value head's lists serve G query heads
     flops_b = 2.5 * flops_f  # five products of the forward's size (dS, dP recomputation not counted)
     peaks, peak_src = load_peaks()
     achieved = flops_b / (bwd_ms / 1e3) / 1e12
     nbytes = q.numel() * q.element_size()
+    kvbytes = k.numel() * k.element_size()
     line = {
         "metric": METRIC, "value": job_tokens_per_s(B * N, world, args.steps, total_ms), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
@@ -280,7 +283,8 @@ def run_backward(args, cfg, dev, rank, world, dist, bsa, flags, variant):
         "gpu_launches": 5 * args.steps,
         "stages_ms": {"fwd_train": fwd_ms, "bwd": bwd_ms},
         "e2e": {"value": job_tokens_per_s(B * N, world, args.e2e_steps, e2e_ms), "unit": "tokens/s",
-                "h2d_bytes_per_step": 4 * nbytes, "d2h_bytes_per_step": 3 * nbytes, "steps": args.e2e_steps},
+                "h2d_bytes_per_step": 2 * nbytes + 2 * kvbytes, "d2h_bytes_per_step": nbytes + 2 * kvbytes,
+                "steps": args.e2e_steps},
         "clocks": clk,
         "roofline": {"kernel": "bwd_dq_kernel + bwd_dkdv_kernel", "bound": "tensor", "achieved": achieved,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
@@ -297,10 +301,12 @@ def run_backward(args, cfg, dev, rank, world, dist, bsa, flags, variant):
         il = idx.cpu().numpy()
         tok, sec = 0, 0.0
         for h in range(min(cfg.H, 2)):
-            qa, ka, va, da = (np.ascontiguousarray(W.to_oracle_array(x[:, :, h:h + 1])) for x in (q, k, v, do))
+            gk = h // (H // Hk)  # the query head's key/value head
+            qa, da = (np.ascontiguousarray(W.to_oracle_array(x[:, :, h:h + 1])) for x in (q, do))
+            ka, va = (np.ascontiguousarray(W.to_oracle_array(x[:, :, gk:gk + 1])) for x in (k, v))
             rows = np.sort(rng.choice(cfg.nb, size=(B, 1, 2), replace=False), axis=-1).astype(np.int32)
             t_ = time.perf_counter()
-            oracle.sparse_attn_bwd(qa, ka, va, da, np.ascontiguousarray(il[:, h:h + 1]), bs, causal=args.causal,
+            oracle.sparse_attn_bwd(qa, ka, va, da, np.ascontiguousarray(il[:, gk:gk + 1]), bs, causal=args.causal,
                                    rows=rows)
             sec += time.perf_counter() - t_
             tok += 2 * bs * B

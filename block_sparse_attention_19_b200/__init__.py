@@ -39,7 +39,8 @@ EXPORTED = ("bsa_topk_count", "bsa_forward_workspace_bytes", "bsa_block_pool",
             "bsa_block_scores_topk_ex", "bsa_sparse_attn_fwd_ex", "bsa_forward_ex",
             "bsa_forward_gqa_workspace_bytes", "bsa_block_scores_topk_gqa", "bsa_sparse_attn_fwd_gqa",
             "bsa_forward_gqa", "bsa_sparse_attn_fwd_train", "bsa_sparse_attn_bwd_workspace_bytes",
-            "bsa_sparse_attn_bwd", "bsa_forward_host_workspace_bytes", "bsa_forward_host")
+            "bsa_sparse_attn_bwd", "bsa_forward_host_workspace_bytes", "bsa_forward_host",
+            "bsa_sparse_attn_fwd_train_gqa", "bsa_sparse_attn_bwd_gqa_workspace_bytes", "bsa_sparse_attn_bwd_gqa")
 
 #: variant flags of the *_ex entry points (include/bsa.h)
 BSA_FLAG_CAUSAL, BSA_FLAG_FORCE_DIAG = 1, 2
@@ -80,6 +81,9 @@ def _load() -> ctypes.CDLL:
         "bsa_sparse_attn_bwd_workspace_bytes": ([I, I, I, I, I], Z),
         "bsa_sparse_attn_bwd": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, U, P, Z, P], I),
         "bsa_forward_host_workspace_bytes": ([I, I, I, I, I, I, D, I], Z),
+        "bsa_sparse_attn_fwd_train_gqa": ([P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, U, P], I),
+        "bsa_sparse_attn_bwd_gqa_workspace_bytes": ([I, I, I, I, I, I], Z),
+        "bsa_sparse_attn_bwd_gqa": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, U, P, Z, P], I),
         "bsa_forward_host": ([P, P, P, P, I, I, I, I, I, I, D, I, U, P, Z, P], I),
     }
     for name, (args, res) in sig.items():
@@ -273,37 +277,43 @@ def bsa_forward_host(q, k, v, block_size: int, topk_ratio: float, out: torch.Ten
 def bsa_sparse_attn_fwd_train(q, k, v, idx, block_size: int, scale: float | None = None, flags: int = 0,
                               out: torch.Tensor | None = None, lse: torch.Tensor | None = None):
     """The attention forward that also returns lse [B,H,N] (ln of each row's
-    softmax denominator), for bsa_sparse_attn_bwd. Returns (o, lse)."""
+    softmax denominator), for bsa_sparse_attn_bwd. Returns (o, lse). k and v
+    may have fewer heads than q (grouped queries; idx per key/value head)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (idx, "idx")):
         _dev(t, n)
     B, N, H, D = q.shape
+    Hk = k.shape[2]
     topk = idx.shape[-1]
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     o = out if out is not None else _out_like(q)
     lse = lse if lse is not None else torch.empty((B, H, N), device=q.device, dtype=torch.float32)
-    _check(lib.bsa_sparse_attn_fwd_train(_p(q), _p(k), _p(v), _p(idx), _p(o), _p(lse), B, N, H, D, block_size,
-                                         topk, float(scale), _dtype_code(q), flags, _stream(q)))
+    _check(lib.bsa_sparse_attn_fwd_train_gqa(_p(q), _p(k), _p(v), _p(idx), _p(o), _p(lse), B, N, H, Hk, D,
+                                             block_size, topk, float(scale), _dtype_code(q), flags, _stream(q)))
     return o, lse
 
 
 def bsa_sparse_attn_bwd(q, k, v, o, do, idx, lse, block_size: int, scale: float | None = None, flags: int = 0,
                         workspace: torch.Tensor | None = None):
     """Gradients (dq, dk, dv) of the attention over the kept blocks with the
-    index lists held fixed; o and lse from bsa_sparse_attn_fwd_train."""
+    index lists held fixed; o and lse from bsa_sparse_attn_fwd_train. With
+    grouped queries (k, v with fewer heads than q) dk and dv are per
+    key/value head, summed over the group's query heads."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do"), (idx, "idx"), (lse, "lse")):
         _dev(t, n)
     B, N, H, D = q.shape
+    Hk = k.shape[2]
     topk = idx.shape[-1]
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    need = lib.bsa_sparse_attn_bwd_workspace_bytes(B, N, H, D, block_size)
+    need = lib.bsa_sparse_attn_bwd_gqa_workspace_bytes(B, N, H, Hk, D, block_size)
     if workspace is None:
         workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    _check(lib.bsa_sparse_attn_bwd(_p(q), _p(k), _p(v), _p(o), _p(do), _p(idx), _p(lse), _p(dq), _p(dk), _p(dv),
-                                   B, N, H, D, block_size, topk, float(scale), _dtype_code(q), flags,
-                                   _p(workspace), workspace.numel() * workspace.element_size(), _stream(q)))
+    _check(lib.bsa_sparse_attn_bwd_gqa(_p(q), _p(k), _p(v), _p(o), _p(do), _p(idx), _p(lse), _p(dq), _p(dk),
+                                       _p(dv), B, N, H, Hk, D, block_size, topk, float(scale), _dtype_code(q),
+                                       flags, _p(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream(q)))
     return dq, dk, dv
 
 

@@ -357,14 +357,14 @@ bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_
 
 // Backward: transpose of the selection (bit matrix), D_n, dQ, dK/dV.
 struct BwdWorkspace {
-  uint32_t* mask;  // [B, H, nb, ceil(nb / 32)]
+  uint32_t* mask;  // [B, Hkv, nb, ceil(nb / 32)]
   float* dsum;     // [B, H, N]
   size_t bytes;
 };
 
-BwdWorkspace bwd_workspace_layout(void* base, int B, int N, int H, int bs) {
+BwdWorkspace bwd_workspace_layout(void* base, int B, int N, int H, int Hkv, int bs) {
   const size_t nb = static_cast<size_t>(N / bs), words = (nb + 31) / 32;
-  const size_t mb = align256(static_cast<size_t>(B) * H * nb * words * sizeof(uint32_t));
+  const size_t mb = align256(static_cast<size_t>(B) * Hkv * nb * words * sizeof(uint32_t));
   const size_t db = align256(static_cast<size_t>(B) * H * N * sizeof(float));
   unsigned char* p = static_cast<unsigned char*>(base);
   BwdWorkspace w;
@@ -377,13 +377,13 @@ BwdWorkspace bwd_workspace_layout(void* base, int B, int N, int H, int bs) {
 template <int D, bool kCausal>
 bsa_status launch_bwd_as(const void* q, const void* k, const void* v, const void* o, const void* dO,
                          const int32_t* idx, const float* lse, const BwdWorkspace& w, void* dq, void* dk,
-                         void* dv, int B, int N, int H, int bs, int kk, float scale, cudaStream_t st) {
+                         void* dv, int B, int N, int H, int Hkv, int bs, int kk, float scale, cudaStream_t st) {
   using L = bsa::BwdLayout<D>;
   CUtensorMap mq, mk, mv, mdo;
   bsa_status s;
   if ((s = make_bnhd_map(&mq, q, B, N, H, D)) != BSA_OK) return s;
-  if ((s = make_bnhd_map(&mk, k, B, N, H, D)) != BSA_OK) return s;
-  if ((s = make_bnhd_map(&mv, v, B, N, H, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mk, k, B, N, Hkv, D)) != BSA_OK) return s;
+  if ((s = make_bnhd_map(&mv, v, B, N, Hkv, D)) != BSA_OK) return s;
   if ((s = make_bnhd_map(&mdo, dO, B, N, H, D)) != BSA_OK) return s;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -399,37 +399,39 @@ bsa_status launch_bwd_as(const void* q, const void* k, const void* v, const void
   }
   const int nb = N / bs, words = (nb + 31) / 32;
   // 1. the transpose of the selection, as bits
-  cudaError_t e = cudaMemsetAsync(w.mask, 0, static_cast<size_t>(B) * H * nb * words * sizeof(uint32_t), st);
+  cudaError_t e = cudaMemsetAsync(w.mask, 0, static_cast<size_t>(B) * Hkv * nb * words * sizeof(uint32_t), st);
   if (e != cudaSuccess) return cuda_fail(e, "backward mask clear");
-  const long entries = static_cast<long>(B) * H * nb * kk;
+  const long entries = static_cast<long>(B) * Hkv * nb * kk;
   bsa::bwd_mask_kernel<<<static_cast<unsigned>((entries + 255) / 256), 256, 0, st>>>(idx, w.mask, entries, nb,
                                                                                      kk, words);
   // 2. D_n = dO_n . o_n
   const long rows = static_cast<long>(B) * N * H;
   bsa::bwd_rowdot_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), w.dsum, rows, N, H, D);
-  // 3. dQ per query tile, 4. dK and dV per key tile
-  const long tiles = static_cast<long>(B) * H * nb * (bs / 128);
-  if (tiles > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "backward grid too large");
+  // 3. dQ per query tile, 4. dK and dV per key tile of each key/value head
+  const long qtiles = static_cast<long>(B) * H * nb * (bs / 128);
+  const long ktiles = static_cast<long>(B) * Hkv * nb * (bs / 128);
+  if (qtiles > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "backward grid too large");
   const float scale_log2 = scale * 1.4426950408889634f;
-  bsa::bwd_dq_kernel<D, kCausal><<<static_cast<unsigned>(tiles), bsa::kBwdThreads, L::kBytes, st>>>(
-      mq, mk, mv, mdo, idx, lse, w.dsum, static_cast<__nv_bfloat16*>(dq), N, H, bs, kk, scale, scale_log2);
-  bsa::bwd_dkdv_kernel<D, kCausal><<<static_cast<unsigned>(tiles), bsa::kBwdThreads, L::kBytes, st>>>(
+  bsa::bwd_dq_kernel<D, kCausal><<<static_cast<unsigned>(qtiles), bsa::kBwdThreads, L::kBytes, st>>>(
+      mq, mk, mv, mdo, idx, lse, w.dsum, static_cast<__nv_bfloat16*>(dq), N, H, Hkv, bs, kk, scale, scale_log2);
+  bsa::bwd_dkdv_kernel<D, kCausal><<<static_cast<unsigned>(ktiles), bsa::kBwdThreads, L::kBytes, st>>>(
       mq, mk, mv, mdo, w.mask, lse, w.dsum, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), N,
-      H, bs, scale, scale_log2);
+      H, Hkv, bs, scale, scale_log2);
   e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "backward launches");
 }
 
 bsa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                       const int32_t* idx, const float* lse, const BwdWorkspace& w, void* dq, void* dk, void* dv,
-                      int B, int N, int H, int D, int bs, int kk, float scale, unsigned flags, cudaStream_t st) {
+                      int B, int N, int H, int Hkv, int D, int bs, int kk, float scale, unsigned flags,
+                      cudaStream_t st) {
   const bool causal = (flags & BSA_FLAG_CAUSAL) != 0;
   if (D == 64)
-    return causal ? launch_bwd_as<64, true>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, bs, kk, scale, st)
-                  : launch_bwd_as<64, false>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, bs, kk, scale, st);
-  return causal ? launch_bwd_as<128, true>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, bs, kk, scale, st)
-                : launch_bwd_as<128, false>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, bs, kk, scale, st);
+    return causal ? launch_bwd_as<64, true>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, Hkv, bs, kk, scale, st)
+                  : launch_bwd_as<64, false>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, Hkv, bs, kk, scale, st);
+  return causal ? launch_bwd_as<128, true>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, Hkv, bs, kk, scale, st)
+                : launch_bwd_as<128, false>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, Hkv, bs, kk, scale, st);
 }
 
 struct Workspace {
@@ -632,11 +634,12 @@ bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int
 // ---- training: the forward with the row log-sum-exp, and the backward
 
 // The shapes the training entry points cover: bf16, D in {64, 128},
-// block_size 128 or 256, one key/value head per query head.
-bsa_status check_train(int B, int N, int H, int D, int block_size, int kk, bsa_dtype dt, unsigned flags) {
+// block_size 128 or 256, H a multiple of H_kv.
+bsa_status check_train(int B, int N, int H, int Hkv, int D, int block_size, int kk, bsa_dtype dt, unsigned flags) {
   bsa_status s;
   if ((s = check_flags(flags)) != BSA_OK) return s;
   if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
+  if ((s = check_heads(H, Hkv)) != BSA_OK) return s;
   if (dt != BSA_BF16) return fail(BSA_ERR_UNSUPPORTED, "training entry points take bf16");
   if (block_size == 64) return fail(BSA_ERR_UNSUPPORTED, "training entry points need block_size 128 or 256");
   const int nb = N / block_size;
@@ -644,34 +647,47 @@ bsa_status check_train(int B, int N, int H, int D, int block_size, int kk, bsa_d
   return BSA_OK;
 }
 
-bsa_status bsa_sparse_attn_fwd_train(const void* q, const void* k, const void* v, const int32_t* idx,
-                                     void* o, float* lse, int B, int N, int H, int D, int block_size,
-                                     int kk, float scale, bsa_dtype dt, unsigned flags, void* stream) {
+bsa_status bsa_sparse_attn_fwd_train_gqa(const void* q, const void* k, const void* v, const int32_t* idx,
+                                         void* o, float* lse, int B, int N, int H, int H_kv, int D,
+                                         int block_size, int kk, float scale, bsa_dtype dt, unsigned flags,
+                                         void* stream) {
   bsa_status s;
-  if ((s = check_train(B, N, H, D, block_size, kk, dt, flags)) != BSA_OK) return s;
+  if ((s = check_train(B, N, H, H_kv, D, block_size, kk, dt, flags)) != BSA_OK) return s;
   if (!(scale > 0.0f) || !std::isfinite(scale)) return fail(BSA_ERR_INVALID_ARG, "scale must be positive and finite");
   if (!q || !k || !v || !idx || !o || !lse) return fail(BSA_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(o) || !aligned16(lse))
     return fail(BSA_ERR_MISALIGNED, "q, k, v, idx, o or lse");
   if (o == q || o == k || o == v) return fail(BSA_ERR_INVALID_ARG, "o aliases an input");
   if ((s = check_device()) != BSA_OK) return s;
-  if ((s = launch_attn(q, k, v, idx, o, B, N, H, H, D, block_size, kk, scale, dt, flags,
+  if ((s = launch_attn(q, k, v, idx, o, B, N, H, H_kv, D, block_size, kk, scale, dt, flags,
                        static_cast<cudaStream_t>(stream), lse)) != BSA_OK)
     return s;
   return ok();
 }
 
-size_t bsa_sparse_attn_bwd_workspace_bytes(int B, int N, int H, int D, int block_size) {
-  if (check_dims(B, N, H, D, block_size) != BSA_OK) return 0;
-  return bwd_workspace_layout(nullptr, B, N, H, block_size).bytes;
+bsa_status bsa_sparse_attn_fwd_train(const void* q, const void* k, const void* v, const int32_t* idx,
+                                     void* o, float* lse, int B, int N, int H, int D, int block_size,
+                                     int kk, float scale, bsa_dtype dt, unsigned flags, void* stream) {
+  return bsa_sparse_attn_fwd_train_gqa(q, k, v, idx, o, lse, B, N, H, H, D, block_size, kk, scale, dt, flags,
+                                       stream);
 }
 
-bsa_status bsa_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
-                               const int32_t* idx, const float* lse, void* dq, void* dk, void* dv, int B,
-                               int N, int H, int D, int block_size, int kk, float scale, bsa_dtype dt,
-                               unsigned flags, void* workspace, size_t workspace_bytes, void* stream) {
+size_t bsa_sparse_attn_bwd_gqa_workspace_bytes(int B, int N, int H, int H_kv, int D, int block_size) {
+  if (check_dims(B, N, H, D, block_size) != BSA_OK || check_heads(H, H_kv) != BSA_OK) return 0;
+  return bwd_workspace_layout(nullptr, B, N, H, H_kv, block_size).bytes;
+}
+
+size_t bsa_sparse_attn_bwd_workspace_bytes(int B, int N, int H, int D, int block_size) {
+  return bsa_sparse_attn_bwd_gqa_workspace_bytes(B, N, H, H, D, block_size);
+}
+
+bsa_status bsa_sparse_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                   const int32_t* idx, const float* lse, void* dq, void* dk, void* dv, int B,
+                                   int N, int H, int H_kv, int D, int block_size, int kk, float scale,
+                                   bsa_dtype dt, unsigned flags, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
   bsa_status s;
-  if ((s = check_train(B, N, H, D, block_size, kk, dt, flags)) != BSA_OK) return s;
+  if ((s = check_train(B, N, H, H_kv, D, block_size, kk, dt, flags)) != BSA_OK) return s;
   if (!(scale > 0.0f) || !std::isfinite(scale)) return fail(BSA_ERR_INVALID_ARG, "scale must be positive and finite");
   if (!q || !k || !v || !o || !dO || !idx || !lse || !dq || !dk || !dv)
     return fail(BSA_ERR_INVALID_ARG, "null pointer");
@@ -683,16 +699,24 @@ bsa_status bsa_sparse_attn_bwd(const void* q, const void* k, const void* v, cons
   for (const void* a : outs)
     for (const void* b : ins)
       if (a == b) return fail(BSA_ERR_INVALID_ARG, "a gradient aliases an input");
-  const BwdWorkspace w = bwd_workspace_layout(workspace, B, N, H, block_size);
+  const BwdWorkspace w = bwd_workspace_layout(workspace, B, N, H, H_kv, block_size);
   if (!workspace || workspace_bytes < w.bytes)
     return fail(BSA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", w.bytes, workspace ? workspace_bytes : 0);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(BSA_ERR_MISALIGNED, "workspace must be 256-byte aligned");
   if ((s = check_device()) != BSA_OK) return s;
-  if ((s = launch_bwd(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, D, block_size, kk, scale, flags,
+  if ((s = launch_bwd(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, H_kv, D, block_size, kk, scale, flags,
                       static_cast<cudaStream_t>(stream))) != BSA_OK)
     return s;
   return ok();
+}
+
+bsa_status bsa_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                               const int32_t* idx, const float* lse, void* dq, void* dk, void* dv, int B,
+                               int N, int H, int D, int block_size, int kk, float scale, bsa_dtype dt,
+                               unsigned flags, void* workspace, size_t workspace_bytes, void* stream) {
+  return bsa_sparse_attn_bwd_gqa(q, k, v, o, dO, idx, lse, dq, dk, dv, B, N, H, H, D, block_size, kk, scale, dt,
+                                 flags, workspace, workspace_bytes, stream);
 }
 
 bsa_status bsa_device_error(int* code_out, void* stream) {

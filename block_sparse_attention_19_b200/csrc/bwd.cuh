@@ -109,7 +109,8 @@ struct BwdBarriers {
   uint64_t drained;
   uint32_t tmem_base;
   int abort;
-  int tiles;  // key tiles (dq) or query tiles (dkdv) this CTA walks
+  int tiles;   // key tiles (dq) or query tiles (dkdv) this CTA walks
+  int blocks;  // dkdv: query blocks that kept this key block (per query head of the group)
 };
 static_assert(sizeof(BwdBarriers) <= 256, "barrier area");
 
@@ -153,8 +154,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const int32_t* __restrict__ idx, const float* __restrict__ lse,
-                  const float* __restrict__ dsum, __nv_bfloat16* __restrict__ dq, int N, int H, int bs,
-                  int k, float scale, float scale_log2) {
+                  const float* __restrict__ dsum, __nv_bfloat16* __restrict__ dq, int N, int H, int Hkv,
+                  int bs, int k, float scale, float scale_log2) {
   using L = BwdLayout<D>;
   extern __shared__ __align__(1024) unsigned char bwd_raw[];
   if ((smem_u32(bwd_raw) & 1023u) != 0) {
@@ -176,8 +177,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int h = static_cast<int>(u % H);
   const int b = static_cast<int>(u / H);
   const long bh = static_cast<long>(b) * H + h;
+  const int g = h / (H / Hkv);  // the key/value head (and selection) of query head h
   const int qrow0 = i * bs + part * 128;
-  const int32_t* sel = idx + (bh * nb + i) * k;
+  const int32_t* sel = idx + ((static_cast<long>(b) * Hkv + g) * nb + i) * k;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
@@ -237,7 +239,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (t >= S) ok = mbar_wait(&empty[s], (use - 1) & 1, abort_flag, is_x ? 711 : 712);
         if (!ok) break;
         mbar_arrive_expect_tx(&full[s], L::kTile);
-        bwd_load_tile<D>(smem + ring + s * L::kTile, map, &full[s], h, row, b, keep);
+        bwd_load_tile<D>(smem + ring + s * L::kTile, map, &full[s], g, row, b, keep);
         issued[s] = use + 1;
       }
       if (is_x) mbar_wait_teardown(&bar.a_full, 0);
@@ -414,8 +416,10 @@ __device__ __forceinline__ int bwd_next_block(const uint32_t* row, int words, in
   return i;
 }
 
-// grid.x = B * H * nb * (bs / 128): one CTA per 128-key tile, which walks the
-// query tiles of the query blocks that kept its block (bit row of `mask`).
+// grid.x = B * Hkv * nb * (bs / 128): one CTA per 128-key tile of key/value
+// head g, which walks, for each of the G = H / Hkv query heads of its group in
+// turn, the query tiles of the query blocks that kept its block (bit row of
+// `mask`, one per key/value head: the group shares its selection).
 // TMEM: S^T [0, 128), dP^T [128, 256), dV [256, 256 + D), dK [256 + D, 256 + 2D).
 // The compute warps read the whole S^T row first, so S^T(t+1) is computed
 // while tile t's P^T and dS^T are made; those go over dP^T, 32-query piece
@@ -427,7 +431,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const uint32_t* __restrict__ mask, const float* __restrict__ lse,
                     const float* __restrict__ dsum, __nv_bfloat16* __restrict__ dk,
-                    __nv_bfloat16* __restrict__ dv, int N, int H, int bs, float scale, float scale_log2) {
+                    __nv_bfloat16* __restrict__ dv, int N, int H, int Hkv, int bs, float scale,
+                    float scale_log2) {
   using L = BwdLayout<D>;
   static_assert(256 + 2 * D <= 512, "TMEM columns");
   extern __shared__ __align__(1024) unsigned char bwd_raw[];
@@ -447,11 +452,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   u /= tpb;
   const int j = static_cast<int>(u % nb);
   u /= nb;
-  const int h = static_cast<int>(u % H);
-  const int b = static_cast<int>(u / H);
-  const long bh = static_cast<long>(b) * H + h;
+  const int g = static_cast<int>(u % Hkv);
+  const int b = static_cast<int>(u / Hkv);
+  const int G = H / Hkv;
   const int krow0 = j * bs + part * 128;  // first key token of this tile
-  const uint32_t* mrow = mask + (bh * nb + j) * words;
+  const uint32_t* mrow = mask + ((static_cast<long>(b) * Hkv + g) * nb + j) * words;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
@@ -474,7 +479,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bar.abort = 0;
     int blocks = 0;
     for (int w = 0; w < words; ++w) blocks += __popc(__ldg(mrow + w));
-    bar.tiles = blocks * tpb;
+    bar.blocks = blocks;
+    bar.tiles = G * blocks * tpb;
     fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -485,8 +491,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
-  const int U = bar.tiles;
+  const int U = bar.tiles, UB = bar.blocks * tpb;  // tiles in all, tiles per query head
   const uint32_t sbase = smem_u32(smem);
+  // Tile t is query tile t % UB of query head g * G + t / UB; the bit row is
+  // walked again for each query head.
+  auto walk = [&](int t, int& w, uint32_t& cur, int& qb, int& hq) {
+    const int tt = t % UB;
+    if (tt == 0) {
+      w = 0;
+      cur = __ldg(mrow);
+      hq = g * G + t / UB;
+    }
+    if (tt % tpb == 0) qb = bwd_next_block(mrow, words, w, cur);
+    return qb * bs + (tt % tpb) * 128;  // first query token of the tile
+  };
 
   if (warp == 0) {
     // ============================================================ TMA producers
@@ -502,21 +520,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (is_x) {
         const uint64_t stream = policy_evict_first();
         mbar_arrive_expect_tx(&bar.a_full, 2 * L::kTile);
-        bwd_load_tile<D>(smem + L::kOffA, &tm_k, &bar.a_full, h, krow0, b, stream);
-        bwd_load_tile<D>(smem + L::kOffA + L::kTile, &tm_v, &bar.a_full, h, krow0, b, stream);
+        bwd_load_tile<D>(smem + L::kOffA, &tm_k, &bar.a_full, g, krow0, b, stream);
+        bwd_load_tile<D>(smem + L::kOffA + L::kTile, &tm_v, &bar.a_full, g, krow0, b, stream);
       }
       int issued[XS] = {};
       bool ok = true;
-      int w = 0, qb = 0;
-      uint32_t cur = __ldg(mrow);
+      int w = 0, qb = 0, hq = 0;
+      uint32_t cur = 0;
       for (int t = 0; t < U && ok; ++t) {
-        if (t % tpb == 0) qb = bwd_next_block(mrow, words, w, cur);
         const int s = t % S, use = t / S;
-        const int row = qb * bs + (t % tpb) * 128;
+        const int row = walk(t, w, cur, qb, hq);
         if (t >= S) ok = mbar_wait(&empty[s], (use - 1) & 1, abort_flag, is_x ? 741 : 742);
         if (!ok) break;
         mbar_arrive_expect_tx(&full[s], L::kTile);
-        bwd_load_tile<D>(smem + ring + s * L::kTile, map, &full[s], h, row, b, keep);
+        bwd_load_tile<D>(smem + ring + s * L::kTile, map, &full[s], hq, row, b, keep);
         issued[s] = use + 1;
       }
       if (is_x) mbar_wait_teardown(&bar.a_full, 0);
@@ -609,12 +626,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const long key = krow0 + kr;
     bool ok = true;
-    int w = 0, qb = 0;
-    uint32_t cur = __ldg(mrow);
+    int w = 0, qb = 0, hq = 0;
+    uint32_t cur = 0;
     float* stats = reinterpret_cast<float*>(smem + L::kStatOff);
     for (int t = 0; t < U; ++t) {
-      if (t % tpb == 0) qb = bwd_next_block(mrow, words, w, cur);
-      const int qrow0 = qb * bs + (t % tpb) * 128;
+      const int qrow0 = walk(t, w, cur, qb, hq);
+      const long bh = static_cast<long>(b) * H + hq;
       // the tile's per-query ln-sum (as log2) and D, one query per thread,
       // into slot t % 2. The slot's previous tile, t - 2, is done: this warp
       // has seen tile t - 1's products complete, which the MMA thread issues
@@ -686,8 +703,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok && U > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar.done, 0, abort_flag, 762));
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* ov = dv + ((static_cast<long>(b) * N + key) * H + h) * D;
-      __nv_bfloat16* ok_ = dk + ((static_cast<long>(b) * N + key) * H + h) * D;
+      __nv_bfloat16* ov = dv + ((static_cast<long>(b) * N + key) * Hkv + g) * D;
+      __nv_bfloat16* ok_ = dk + ((static_cast<long>(b) * N + key) * Hkv + g) * D;
       uint32_t r[32];
 #pragma unroll 1
       for (int which = 0; which < 2; ++which) {

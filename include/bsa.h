@@ -236,9 +236,12 @@ bsa_status bsa_forward_host(const void* q, const void* k, const void* v, void* o
  * token n and kept key token t (p = softmax weight, o = output):
  *   D_n = dO_n . o_n,  dS = p (dO_n . v_t - D_n),
  *   dq_n = scale sum_t dS k_t,  dk_t = scale sum_n dS q_n,  dv_t = sum_n p dO_n.
- * Covered shapes: dt = BSA_BF16, D = 64 or 128, block_size 128 or 256, one
- * key/value head per query head (others: BSA_ERR_UNSUPPORTED). Flags: as for
- * the _ex entry points (BSA_FLAG_CAUSAL masks as in the forward). */
+ * Covered shapes: dt = BSA_BF16, D = 64 or 128, block_size 128 or 256 (others:
+ * BSA_ERR_UNSUPPORTED); H a multiple of H_kv in the _gqa forms, where query
+ * head h reads key/value head h / (H / H_kv) and that head's selection (idx
+ * [B, H_kv, nb, topk], as bsa_sparse_attn_fwd_gqa reads it), and dk, dv sum
+ * over the group's query heads. Flags: as for the _ex entry points
+ * (BSA_FLAG_CAUSAL masks as in the forward). */
 
 /* bsa_sparse_attn_fwd_ex that also writes lse [B, H, N] float32 (written):
  * ln sum_t exp(scale q_n . k_t) over the row's kept (unmasked) key tokens. */
@@ -246,9 +249,20 @@ bsa_status bsa_sparse_attn_fwd_train(const void* q, const void* k, const void* v
                                      void* o, float* lse, int B, int N, int H, int D, int block_size,
                                      int topk, float scale, bsa_dtype dt, unsigned flags, void* stream);
 
+/* The same with grouped queries: q, o, lse per query head ([B, N, H, D],
+ * [B, H, N]); k, v [B, N, H_kv, D]; idx [B, H_kv, nb, topk]. */
+bsa_status bsa_sparse_attn_fwd_train_gqa(const void* q, const void* k, const void* v, const int32_t* idx,
+                                         void* o, float* lse, int B, int N, int H, int H_kv, int D,
+                                         int block_size, int topk, float scale, bsa_dtype dt, unsigned flags,
+                                         void* stream);
+
 /* Workspace bytes of bsa_sparse_attn_bwd: the transpose of the selection as
  * a bit matrix [B, H, nb, ceil(nb / 32)] and D [B, H, N] float32. */
 size_t bsa_sparse_attn_bwd_workspace_bytes(int B, int N, int H, int D, int block_size);
+
+/* Workspace bytes of bsa_sparse_attn_bwd_gqa: the bit matrix per key/value
+ * head [B, H_kv, nb, ceil(nb / 32)] and D [B, H, N] float32. */
+size_t bsa_sparse_attn_bwd_gqa_workspace_bytes(int B, int N, int H, int H_kv, int D, int block_size);
 
 /* Gradients dq, dk, dv ([B, N, H, D] bf16, written) of the attention of
  * bsa_sparse_attn_fwd_train, given q, k, v, its output o and lse, the output
@@ -262,6 +276,16 @@ bsa_status bsa_sparse_attn_bwd(const void* q, const void* k, const void* v, cons
                                const int32_t* idx, const float* lse, void* dq, void* dk, void* dv, int B,
                                int N, int H, int D, int block_size, int topk, float scale, bsa_dtype dt,
                                unsigned flags, void* workspace, size_t workspace_bytes, void* stream);
+
+/* The same with grouped queries: dq [B, N, H, D]; dk, dv [B, N, H_kv, D],
+ * each the sum over the G = H / H_kv query heads of its group (one CTA per
+ * 128-key tile of a key/value head walks the kept query tiles of all G heads
+ * in turn, so the sum keeps a fixed order). */
+bsa_status bsa_sparse_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                   const int32_t* idx, const float* lse, void* dq, void* dk, void* dv, int B,
+                                   int N, int H, int H_kv, int D, int block_size, int topk, float scale,
+                                   bsa_dtype dt, unsigned flags, void* workspace, size_t workspace_bytes,
+                                   void* stream);
 
 /* Size of the fixed device scratch that bsa_forward_noalloc uses: 64 MiB. */
 #define BSA_NOALLOC_SCRATCH_BYTES (64u << 20)

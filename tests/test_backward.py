@@ -104,3 +104,46 @@ def test_backward_refuses_uncovered_shapes(bsa):
     idx = torch.zeros(1, 2, 8, 2, device="cuda", dtype=torch.int32)
     with pytest.raises(bsa.BsaError, match="UNSUPPORTED"):
         bsa.bsa_sparse_attn_fwd_train(q, q, q, idx, 64)  # block_size 64
+
+
+GQA_CASES = [  # (B, N, H, H_kv, D, block_size, ratio, causal)
+    (1, 2048, 4, 2, 128, 128, 0.25, False),
+    (1, 2048, 6, 2, 64, 128, 0.3, True),     # G = 3
+    (2, 1024, 4, 1, 128, 256, 0.5, False),   # all query heads in one group, block_size 256
+]
+
+
+@pytest.mark.parametrize("ci", range(len(GQA_CASES)))
+def test_backward_gqa_matches_oracle(bsa, oracle_mod, ci):
+    """Grouped queries: dq per query head, dk and dv per key/value head. The
+    reference is the oracle's per-head backward with k and v repeated to the
+    query heads and each query head given its group's index lists; the
+    gradient of a shared k (or v) is the sum of those per-head gradients over
+    its group, which is exact."""
+    B, N, H, Hkv, D, bs, ratio, causal = GQA_CASES[ci]
+    cfg = W.Config(f"bwdg{ci}", B, N, H, D, bs, ratio, "bf16", 1.0, 1500 + ci, None, H_kv=Hkv)
+    q, k, v = W.make_inputs(cfg, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(1600 + ci)
+    do = torch.randn(q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    flags = bsa.BSA_FLAG_CAUSAL if causal else 0
+    ws = torch.empty(bsa.bsa_forward_workspace_bytes(B, N, H, D, bs, ratio, H_kv=Hkv), device="cuda",
+                     dtype=torch.uint8)
+    bsa.bsa_forward(q, k, v, bs, ratio, workspace=ws, flags=flags)
+    idx = bsa.workspace_views(ws, B, N, H, D, bs, ratio, H_kv=Hkv)[2].clone()  # [B, H_kv, nb, k]
+    o, lse = bsa.bsa_sparse_attn_fwd_train(q, k, v, idx, bs, flags=flags)
+    dq, dk, dv = bsa.bsa_sparse_attn_bwd(q, k, v, o, do, idx, lse, bs, flags=flags)
+    torch.cuda.synchronize()
+    assert bsa.bsa_device_error() == 0
+    assert dk.shape == k.shape and dv.shape == v.shape
+    G = H // Hkv
+    qa, ka, va, doa = (_host(x) for x in (q, k, v, do))
+    idx_q = np.repeat(idx.cpu().numpy(), G, axis=1)
+    rows = np.broadcast_to(np.arange(cfg.nb, dtype=np.int32), (B, H, cfg.nb)).copy()
+    check_output(gpu_rows(o, rows, bs), oracle_mod.sparse_attn_gqa(qa, ka, va, idx_q, bs, causal=causal), "bf16")
+    ke, ve = np.repeat(ka, G, axis=2), np.repeat(va, G, axis=2)
+    rq, rk, rv = oracle_mod.sparse_attn_bwd(qa, ke, ve, doa, idx_q, bs, causal=causal)
+    rk = rk.reshape(B, N, Hkv, G, D).sum(axis=3)
+    rv = rv.reshape(B, N, Hkv, G, D).sum(axis=3)
+    check_grad(dq, rq, "dq")
+    check_grad(dk, rk, "dk")
+    check_grad(dv, rv, "dv")
