@@ -41,7 +41,7 @@ METRIC = "block-sparse attn fwd tokens/s & effective TFLOP/s (% roofline), 1 B20
 # DRAM read + write bytes per launch of the attention kernel, from the ncu
 # capture recorded in profiles/sparse_attn_tc2_traffic.md (the kernel as it
 # stands); workloads not captured report null.
-NCU_TRAFFIC = {"c3": 807.93e6 + 249.50e6, "c4": 4.98e9 + 585.72e6}
+NCU_TRAFFIC = {"c3": 810.46e6 + 249.09e6, "c4": 4.93e9 + 588.97e6}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
