@@ -1,6 +1,6 @@
-// attn_tc2.cuh -- step 3 for bfloat16 inputs with block_size 128 or 256: two
-// 128-row query tiles per CTA so that the tensor core works on one tile while
-// the softmax runs on the other.
+// attn_tc2.cuh -- step 3 for bfloat16 or e4m3 inputs on the tensor cores:
+// two 128-row query tiles per CTA so that the tensor core works on one tile
+// while the softmax runs on the other.
 //
 // Page "2026 新一代卷积与 Transformer 网络架构" (qqiyuan.cn), section
 // "SparseFormer 注意力实现", step 3 (sparse_attn_cuda, scale 1/sqrt(D)); page
@@ -9,11 +9,14 @@
 //
 // Work unit (one CTA): two "streams" A and B of 128 query rows each.
 //   * block_size 256: the two halves of one query block. They share the key
-//     list, so every gathered K/V tile feeds both streams (half the L2
-//     traffic per flop).
-//   * block_size 128: two consecutive query blocks of one (b, h), each with
-//     its own key list; K/V tiles of the two streams alternate in the rings.
-//     With an odd number of blocks the last CTA runs stream A only.
+//     list, so every gathered K/V tile feeds both streams.
+//   * block_size 128 with an even number of query heads per key/value head:
+//     one query block of two heads of a group, which share the key list.
+//   * block_size 128 otherwise: two consecutive query blocks of one head,
+//     each with its own key list; K/V tiles of the two streams alternate in
+//     the rings. With an odd number of blocks the last CTA runs stream A only.
+//   * block_size 64 (kStack): each stream stacks two consecutive query blocks
+//     (see the kernel's comment).
 // Roles:
 //   * warp 0 (one lane): TMA loads of both query tiles and the K ring; warp 2
 //     (one lane): the V ring. Rings are filled in the order the MMA consumes
@@ -21,20 +24,21 @@
 //   * warp 1, lane 0: tcgen05.mma issue in the order S_A(0), S_B(0), then per
 //     key tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1). The softmax warps
 //     release K ring entries (they see each S complete); the issuing thread
-//     commits only the S the softmax waits for and the V entry it just read. S_X lives in TMEM
-//     columns of stream X; P_X (bf16) is written over the first 64 of them and
-//     read from TMEM as the A operand of PV_X; O_X accumulates in TMEM.
-//     Because tcgen05.mma ops of one thread run in order, S_X(j+1) cannot
-//     overwrite P_X(j) before PV_X(j) has read it, and the completion of
-//     S_X(j+1) implies that PV_X(j) is done (so O_X is stable).
+//     commits only the S the softmax waits for and the V entry it just read.
+//     S_X lives in TMEM columns of stream X; P_X (bf16, or e4m3) is written
+//     over the first 64 (32) of them and read from TMEM as the A operand of
+//     PV_X; O_X accumulates in TMEM. Because tcgen05.mma ops of one thread run
+//     in order, S_X(j+1) cannot overwrite P_X(j) before PV_X(j) has read it,
+//     and the completion of S_X(j+1) implies that PV_X(j) is done (so O_X is
+//     stable).
 //   * warps 4-7 (stream A) and 8-11 (stream B): one query row per thread.
 //     Per tile a thread loads its whole S row from TMEM into registers (the
 //     softmax warp groups take registers from warp group 0 with setmaxnreg),
 //     takes the row max; the running max (log2 domain) moves only when the
 //     tile max exceeds it by more than 8, in which case O_X is rescaled in
 //     TMEM; then P = exp2(S * scale * log2 e - m) with two-wide float32
-//     instructions (three key pairs in eight via a polynomial on the FMA
-//     pipe), stored as packed bf16 over the first 64 columns of S.
+//     instructions (one key pair in four via a polynomial on the FMA pipe),
+//     stored packed over the first columns of S.
 //   * warp 3 idle.
 // Every wait is bounded; on a timeout the device error word and an abort flag
 // are set, roles leave their loops, copies and MMAs are drained, TMEM is freed.
