@@ -41,6 +41,8 @@ __global__ void __launch_bounds__(kSimtThreads)
                             const float* __restrict__ v, const int32_t* __restrict__ idx,
                             float* __restrict__ o, int N, int H, int Hkv, int bs, int k, float scale,
                             unsigned flags) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ __align__(16) unsigned char simt_raw[];
   SimtSmem<D>& sm = *reinterpret_cast<SimtSmem<D>*>(simt_raw);
   constexpr int DL = D / 32;  // output columns per lane

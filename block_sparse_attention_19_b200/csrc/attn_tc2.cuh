@@ -200,6 +200,8 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
   constexpr int kKeysPerStep = 32 / L::kElem;
   constexpr int kStepsPV = 128 / kKeysPerStep;
   constexpr int KS = L::kKStages, VS = L::kVStages;
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ __align__(1024) unsigned char tc2_raw[];
   // swizzled tiles need 1024-byte alignment and the layout has no slack
   if ((smem_u32(tc2_raw) & 1023u) != 0) {

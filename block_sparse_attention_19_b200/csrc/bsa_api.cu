@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "attn_simt.cuh"
 #include "attn_tc2.cuh"
@@ -143,6 +144,25 @@ bsa_status make_bnhd_map(CUtensorMap* map, const void* base, int B, int N, int H
 
 // ------------------------------------------------------------------ launches
 
+// Launches `kernel` with programmatic stream serialization: it may be
+// scheduled while the previous kernel of the stream finishes (the forward
+// path's kernels wait for their predecessor on entry, pdl_wait).
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int ntasks, int B,
                        int N, int H, int D, int bs, bsa_dtype dt, cudaStream_t st) {
   const int V = dt == BSA_F32 ? 4 : (dt == BSA_E4M3 ? 16 : 8);  // elements per 16 bytes
@@ -151,13 +171,15 @@ bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int
   const long grid = static_cast<long>(ntasks) * B * (N / bs) * (C / cw);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "pool grid too large");
   bsa::PoolTask t0{x0, p0}, t1{x1 ? x1 : x0, p1 ? p1 : p0};
+  const unsigned g = static_cast<unsigned>(grid);
+  cudaError_t e;
   if (dt == BSA_F32)
-    bsa::block_pool_kernel<float><<<static_cast<unsigned>(grid), bsa::kPoolThreads, 0, st>>>(t0, t1, B, N, H, D, bs, cw);
+    e = launch_pdl(bsa::block_pool_kernel<float>, g, bsa::kPoolThreads, 0, st, t0, t1, B, N, H, D, bs, cw);
   else if (dt == BSA_E4M3)
-    bsa::block_pool_kernel<__nv_fp8_e4m3><<<static_cast<unsigned>(grid), bsa::kPoolThreads, 0, st>>>(t0, t1, B, N, H, D, bs, cw);
+    e = launch_pdl(bsa::block_pool_kernel<__nv_fp8_e4m3>, g, bsa::kPoolThreads, 0, st, t0, t1, B, N, H, D, bs, cw);
   else
-    bsa::block_pool_kernel<__nv_bfloat16><<<static_cast<unsigned>(grid), bsa::kPoolThreads, 0, st>>>(t0, t1, B, N, H, D, bs, cw);
-  cudaError_t e = cudaGetLastError();
+    e = launch_pdl(bsa::block_pool_kernel<__nv_bfloat16>, g, bsa::kPoolThreads, 0, st, t0, t1, B, N, H, D, bs, cw);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_pool_kernel launch");
 }
 
@@ -213,19 +235,11 @@ bsa_status launch_scores(const float* qp, const float* kp, float* S, int B, int 
   const long grid = ntiles < sm_count() ? ntiles : sm_count();
   const unsigned gr = static_cast<unsigned>(grid);
   const bool grouped = H != Hkv;
-  if (ntile == 128 && !grouped)
-    bsa::block_scores_tc_kernel<128, false><<<gr, bsa::kScThreads, bsa::kScSmem, st>>>(
-        qp, kp, S, tm_s, nb, D, ntiles, tma_store, H, Hkv);
-  else if (ntile == 128)
-    bsa::block_scores_tc_kernel<128, true><<<gr, bsa::kScThreads, bsa::kScSmem, st>>>(
-        qp, kp, S, tm_s, nb, D, ntiles, tma_store, H, Hkv);
-  else if (!grouped)
-    bsa::block_scores_tc_kernel<256, false><<<gr, bsa::kScThreads, bsa::kScSmem, st>>>(
-        qp, kp, S, tm_s, nb, D, ntiles, tma_store, H, Hkv);
-  else
-    bsa::block_scores_tc_kernel<256, true><<<gr, bsa::kScThreads, bsa::kScSmem, st>>>(
-        qp, kp, S, tm_s, nb, D, ntiles, tma_store, H, Hkv);
-  cudaError_t e = cudaGetLastError();
+  auto kern = ntile == 128 ? (grouped ? bsa::block_scores_tc_kernel<128, true> : bsa::block_scores_tc_kernel<128, false>)
+                            : (grouped ? bsa::block_scores_tc_kernel<256, true> : bsa::block_scores_tc_kernel<256, false>);
+  cudaError_t e = launch_pdl(kern, gr, bsa::kScThreads, bsa::kScSmem, st, qp, kp, S, tm_s, nb, D, ntiles, tma_store,
+                             H, Hkv);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_scores_tc_kernel launch");
 }
 
@@ -245,9 +259,9 @@ bsa_status launch_topk(const float* S, int32_t* idx, int B, int H, int nb, int k
   }
   const long grid = (rows + bsa::kSelWarps - 1) / bsa::kSelWarps;
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "top-k grid too large");
-  bsa::block_topk_kernel<<<static_cast<unsigned>(grid), bsa::kSelThreads, stage ? stage_bytes : 0, st>>>(
-      S, idx, rows, nb, k, stage ? 1 : 0, flags);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(bsa::block_topk_kernel, static_cast<unsigned>(grid), bsa::kSelThreads,
+                             stage ? stage_bytes : 0, st, S, idx, rows, nb, k, stage ? 1 : 0, flags);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_topk_kernel launch");
 }
 
@@ -274,9 +288,9 @@ bsa_status launch_attn_simt(const float* q, const float* k, const float* v, cons
   }
   const long grid = static_cast<long>(B) * H * (N / bs) * (bs / bsa::kSimtRows);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
-  bsa::sparse_attn_simt_kernel<D><<<static_cast<unsigned>(grid), bsa::kSimtThreads, smem, st>>>(
-      q, k, v, idx, o, N, H, Hkv, bs, kk, scale, flags);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(bsa::sparse_attn_simt_kernel<D>, static_cast<unsigned>(grid), bsa::kSimtThreads, smem,
+                             st, q, k, v, idx, o, N, H, Hkv, bs, kk, scale, flags);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_simt_kernel launch");
 }
 
@@ -318,9 +332,10 @@ bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const
                                  : static_cast<long>(B) * H * (bs == 256 ? nb : (nb + 1) / 2);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   const float scale_log2 = scale * 1.4426950408889634f;
-  bsa::sparse_attn_tc2_kernel<D, kCausal, kF8, kStack><<<static_cast<unsigned>(grid), bsa::kTc2Threads, L::kBytes, st>>>(
-      mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H, Hkv, bs, kk, scale_log2, lse);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(bsa::sparse_attn_tc2_kernel<D, kCausal, kF8, kStack>, static_cast<unsigned>(grid),
+                             bsa::kTc2Threads, L::kBytes, st, mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H,
+                             Hkv, bs, kk, scale_log2, lse);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc2_kernel launch");
 }
 

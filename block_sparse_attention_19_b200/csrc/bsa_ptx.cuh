@@ -386,6 +386,18 @@ __device__ __forceinline__ void regs_increase() {
 }
 
 // ---------------------------------------------------------------- misc
+// Programmatic dependent launch. pdl_launch_dependents lets the next kernel
+// of the stream (when it is launched with programmatic stream serialization)
+// be scheduled once every CTA of this grid has executed it; pdl_wait blocks
+// until the grids this one depends on have completed and their memory writes
+// are visible. Without that launch attribute both are no-ops. Every kernel of
+// the forward path calls both on entry, before it touches global memory:
+// only launch latency and scheduling overlap, never data.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -82,6 +82,8 @@ inline int pool_column_group(int C) {
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
     block_pool_kernel(PoolTask t0, PoolTask t1, int B, int N, int H, int D, int bs, int cw) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr int V = Vec16<T>::kN;
   const int nb = N / bs;
   const int C = H * D / V;  // 16-byte columns per row

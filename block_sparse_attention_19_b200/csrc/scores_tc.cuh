@@ -114,6 +114,8 @@ __global__ void __launch_bounds__(kScThreads, 1)
     block_scores_tc_kernel(const float* __restrict__ qp, const float* __restrict__ kp,
                            float* __restrict__ S, const __grid_constant__ CUtensorMap tm_s, int nb,
                            int D, long ntiles, int tma_store, int H, int Hkv) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr int ntile = NT;
   extern __shared__ unsigned char sc_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(

@@ -270,6 +270,8 @@ __device__ __forceinline__ void select_row_smem(const float* srow, int nb, int k
 __global__ void __launch_bounds__(kSelThreads, 4)
     block_topk_kernel(const float* __restrict__ S, int32_t* __restrict__ idx, long rows, int nb,
                       int k, int stage_rows, unsigned flags) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ __align__(16) float sel_rows[];
   __shared__ uint32_t cand[kSelWarps][64];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
