@@ -172,13 +172,14 @@ bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "pool grid too large");
   bsa::PoolTask t0{x0, p0}, t1{x1 ? x1 : x0, p1 ? p1 : p0};
   const unsigned g = static_cast<unsigned>(grid);
+  const unsigned threads = static_cast<unsigned>(bsa::kPoolRowGroups * cw);
   cudaError_t e;
   if (dt == BSA_F32)
-    e = launch_pdl(bsa::block_pool_kernel<float>, g, bsa::kPoolThreads, 0, st, t0, t1, B, N, H, D, bs, cw);
+    e = launch_pdl(bsa::block_pool_kernel<float>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw);
   else if (dt == BSA_E4M3)
-    e = launch_pdl(bsa::block_pool_kernel<__nv_fp8_e4m3>, g, bsa::kPoolThreads, 0, st, t0, t1, B, N, H, D, bs, cw);
+    e = launch_pdl(bsa::block_pool_kernel<__nv_fp8_e4m3>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw);
   else
-    e = launch_pdl(bsa::block_pool_kernel<__nv_bfloat16>, g, bsa::kPoolThreads, 0, st, t0, t1, B, N, H, D, bs, cw);
+    e = launch_pdl(bsa::block_pool_kernel<__nv_bfloat16>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_pool_kernel launch");
 }
@@ -212,7 +213,10 @@ bsa_status launch_scores(const float* qp, const float* kp, float* S, int B, int 
     }
     attr_set[dev] = true;
   }
-  const int ntile = nb <= 128 ? 128 : 256;
+  // 128-wide score tiles up to nb = 256 (256-wide ones would leave most SMs
+  // idle there), 256-wide beyond; the choice depends on nb alone, so that a
+  // subset of the heads is scored exactly like the whole tensor
+  const int ntile = nb <= 256 ? 128 : 256;
   const long ntiles = static_cast<long>(B) * Hkv * ((nb + bsa::kScM - 1) / bsa::kScM) *
                       ((nb + ntile - 1) / ntile);
   const int tma_store = (nb % 4 == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0) ? 1 : 0;

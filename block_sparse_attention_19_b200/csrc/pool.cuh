@@ -18,6 +18,11 @@
 namespace bsa {
 
 constexpr int kPoolThreads = 256;
+// Rows of a block are split over this many row groups whatever the row width
+// (the host launches kPoolRowGroups * cw threads), so every block mean is
+// summed in the same order for any number of heads: the host-buffer path
+// pools one head group at a time and must match the whole tensor.
+constexpr int kPoolRowGroups = 4;
 
 struct PoolTask {
   const void* x;  // [B, N, H, D]
@@ -67,18 +72,18 @@ struct Vec16<__nv_fp8_e4m3> {
   }
 };
 
-// Columns (16-byte units) one work item covers: 64 when the row width allows,
-// else the largest divisor of the row width that fits the CTA.
+// Columns (16-byte units) one work item covers: the largest divisor of the
+// row width up to kPoolThreads / kPoolRowGroups = 64.
 inline int pool_column_group(int C) {
-  if (C % 64 == 0) return 64;
-  int cw = C < kPoolThreads ? C : kPoolThreads;
+  int cw = C < kPoolThreads / kPoolRowGroups ? C : kPoolThreads / kPoolRowGroups;
   while (C % cw) --cw;
   return cw;
 }
 
-// grid.x = ntasks * B * nb * (C / cw). Each CTA reduces bs rows of one group of
-// cw 16-byte columns of one block; rows are split over kPoolThreads / cw
-// row groups.
+// grid.x = ntasks * B * nb * (C / cw), blockDim.x = kPoolRowGroups * cw. Each
+// CTA reduces bs rows of one group of cw 16-byte columns of one block; row r
+// goes to row group r % kPoolRowGroups, and the groups' partial sums are
+// added in group order.
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
     block_pool_kernel(PoolTask t0, PoolTask t1, int B, int N, int H, int D, int bs, int cw) {
@@ -88,7 +93,7 @@ __global__ void __launch_bounds__(kPoolThreads)
   const int nb = N / bs;
   const int C = H * D / V;  // 16-byte columns per row
   const int ngroups = C / cw;
-  const int G = kPoolThreads / cw;  // row groups (>= 1: cw <= 256 is checked by the host)
+  const int G = blockDim.x / cw;  // kPoolRowGroups (read at run time: the compiled loop is faster)
 
   long item = blockIdx.x;
   const int cg = static_cast<int>(item % ngroups);

@@ -32,6 +32,7 @@ CASES = [  # (B, N, H, H_kv, D, block_size, ratio, dtype, causal, pinned)
     (2, 32768, 8, 2, 128, 128, 0.2, "bf16", True, True),     # grouped queries, causal, 2 kv heads per chunk
     (3, 512, 2, 2, 64, 64, 0.5, "f32", False, False),        # float32, pageable host memory
     (2, 2048, 4, 2, 128, 64, 0.25, "e4m3", False, True),     # e4m3 inputs, bf16 output
+    (1, 65536, 2, 2, 64, 64, 0.05, "f32", False, True),      # float32, one head per chunk (sums that round)
 ]
 
 
@@ -66,3 +67,17 @@ def test_host_path_rejects_device_tensors_and_small_workspace(bsa):
     ws = torch.empty(256, device="cuda", dtype=torch.uint8)
     with pytest.raises(bsa.BsaError, match="WORKSPACE"):
         bsa.bsa_forward_host(q, q, q, 64, 0.5, workspace=ws)
+
+
+@pytest.mark.parametrize("dtype,D", [(torch.float32, 128), (torch.bfloat16, 64), (torch.float8_e4m3fn, 128)])
+def test_pooling_does_not_depend_on_the_head_count(bsa, dtype, D):
+    """Each block mean is summed in one fixed order whatever the number of
+    heads in the tensor (the host-buffer path pools one head group at a time
+    and must reproduce the whole-tensor result bit for bit). float32 data has
+    sums that round, so a different order would show."""
+    g = torch.Generator(device="cuda").manual_seed(1700)
+    x = (torch.randn(2, 4096, 8, D, generator=g, device="cuda") * 3 + 1).to(dtype)
+    full = bsa.bsa_block_pool(x, 256)
+    for h in (0, 3, 7):
+        one = bsa.bsa_block_pool(x[:, :, h:h + 1].contiguous(), 256)
+        assert torch.equal(one[:, 0], full[:, h]), h
