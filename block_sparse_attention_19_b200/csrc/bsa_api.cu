@@ -250,23 +250,29 @@ bsa_status launch_scores(const float* qp, const float* kp, float* S, int B, int 
 bsa_status launch_topk(const float* S, int32_t* idx, int B, int H, int nb, int k, unsigned flags,
                        cudaStream_t st) {
   const long rows = static_cast<long>(B) * H * nb;
-  const size_t stage_bytes = static_cast<size_t>(bsa::kSelWarps) * nb * sizeof(float);
-  const bool stage = nb > 1024 && stage_bytes <= 200 * 1024;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(bsa::block_topk_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    if (e != cudaSuccess) return cuda_fail(e, "topk smem attribute");
-    attr_set[dev] = true;
-  }
   const long grid = (rows + bsa::kSelWarps - 1) / bsa::kSelWarps;
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "top-k grid too large");
-  cudaError_t e = launch_pdl(bsa::block_topk_kernel, static_cast<unsigned>(grid), bsa::kSelThreads,
-                             stage ? stage_bytes : 0, st, S, idx, rows, nb, k, stage ? 1 : 0, flags);
+  cudaError_t e;
+  if (nb <= 1024) {
+    e = launch_pdl(bsa::block_topk_kernel, static_cast<unsigned>(grid), bsa::kSelThreads, 0, st, S, idx, rows, nb,
+                   k, flags);
+  } else {
+    // long rows: each warp stages its row's keys in shared memory when they fit
+    const size_t stage_bytes = static_cast<size_t>(bsa::kSelWarps) * bsa::staged_row_keys(nb) * sizeof(uint32_t);
+    const bool stage = stage_bytes <= 200 * 1024;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+      e = cudaFuncSetAttribute(bsa::block_topk_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+      if (e != cudaSuccess) return cuda_fail(e, "top-k smem attribute");
+      attr_set[dev] = true;
+    }
+    e = launch_pdl(bsa::block_topk_wide_kernel, static_cast<unsigned>(grid), bsa::kSelThreads,
+                   stage ? stage_bytes : 0, st, S, idx, rows, nb, k, stage ? 1 : 0, flags);
+  }
   if (e == cudaSuccess) e = cudaGetLastError();
-  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_topk_kernel launch");
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "top-k kernel launch");
 }
 
 bsa_status launch_select(const float* qp, const float* kp, float* S, int32_t* idx, int B, int H,

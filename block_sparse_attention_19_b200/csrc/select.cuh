@@ -6,13 +6,15 @@
 // output row lists its k blocks in ascending order (a canonical order, so
 // results compare exactly).
 //
-// One warp per score row, scores as order-preserving 32-bit keys. For
-// nb <= 1024 the keys sit in registers and the k-th largest key is
-// bracketed by bisection (on the score value, then on the key) until at most
-// 64 keys remain in the bracket, which are sorted exactly (about 8 counting
-// passes on typical rows instead of 32); longer rows use a bitwise binary search over the keys
-// staged in shared memory. One ordered ballot pass then emits every key above
-// the k-th largest plus the lowest-index keys equal to it.
+// One warp per score row, scores as order-preserving 32-bit keys. The k-th
+// largest key is bracketed by bisection (on the score value, then on the
+// key) until at most 64 keys remain in the bracket, which are sorted exactly
+// (about 8 counting passes on typical rows instead of 32). For nb <= 1024
+// the keys sit in registers (block_topk_kernel); longer rows are converted
+// once into shared memory and counted from there (block_topk_wide_kernel;
+// rows too long to stage fall back to a bitwise search read from L2). One
+// ordered ballot pass then emits every key above the k-th largest plus the
+// lowest-index keys equal to it.
 #pragma once
 
 #include <stdint.h>
@@ -262,26 +264,124 @@ __device__ __forceinline__ void select_row_smem(const float* srow, int nb, int k
   }
 }
 
-// grid.x = ceil(rows / kSelWarps); one warp per row of S ([rows, nb]).
-// Dynamic shared memory: kSelWarps * nb floats when nb > 1024 and stage_rows, else none.
-// flags: with kFlagCausal, row r is query block i = r % nb: only key blocks
-// j <= i are ranked and min(k, i + 1) are kept (with kFlagForceDiag block i
-// always, plus the best j < i), then the row is padded with -1.
-__global__ void __launch_bounds__(kSelThreads, 4)
-    block_topk_kernel(const float* __restrict__ S, int32_t* __restrict__ idx, long rows, int nb,
-                      int k, int stage_rows, unsigned flags) {
-  pdl_launch_dependents();
-  pdl_wait();
-  extern __shared__ __align__(16) float sel_rows[];
-  __shared__ uint32_t cand[kSelWarps][64];
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const long r = static_cast<long>(blockIdx.x) * kSelWarps + warp;
-  if (r >= rows) return;
-  const float* srow = S + r * nb;
-  int32_t* out = idx + r * static_cast<long>(k);
-  const bool vec = (nb & 3) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0;
-  // candidates are the key blocks [0, ncand); ksel of them are ranked in
-  int ncand = nb, ksel = k;
+// Row length a warp stages in shared memory for nb > 1024: whole 128-key
+// chunks (the tail is padding key 0).
+__host__ __device__ constexpr int staged_row_keys(int nb) { return (nb + 127) & ~127; }
+
+// The selection of select_row_bracket for a row too long for registers:
+// keys (score_key, padding 0) staged once in shared memory, nbp of them
+// (a multiple of 128). Counting passes read four keys per lane per
+// 16-byte load; the bracket is narrowed on the score value, then on the key,
+// to at most 64 keys, which are gathered and sorted; the emission is one
+// ordered ballot pass. `cand` is 64 words of shared memory private to the warp.
+__device__ __forceinline__ void select_row_staged(const uint32_t* keys, int nbp, int nvalid, int k,
+                                                  int32_t* out, int lane, uint32_t* cand) {
+  const uint4* kv = reinterpret_cast<const uint4*>(keys);
+  const int nv4 = nbp / 4;
+  auto count_ge = [&](uint32_t t) {
+    unsigned c = 0;
+    for (int q = lane; q < nv4; q += 32) {
+      const uint4 u = kv[q];
+      c += (u.x >= t) + (u.y >= t) + (u.z >= t) + (u.w >= t);
+    }
+    return static_cast<int>(__reduce_add_sync(0xffffffffu, c));
+  };
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int q = lane; q < nv4; q += 32) {
+    const uint4 u = kv[q];
+    const uint32_t e[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      kmin = min(kmin, e[t] == 0u ? 0xFFFFFFFFu : e[t]);  // padding is not a key
+      kmax = max(kmax, e[t]);
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  // invariant: count(key >= lo) = clo >= k > chi = count(key >= hi); hi may be 2^32
+  uint32_t lo = kmin;
+  uint64_t hi = static_cast<uint64_t>(kmax) + 1;
+  int clo = nvalid, chi = 0;
+#pragma unroll 1
+  for (int it = 0; it < 64 && clo - chi > 64 && hi - lo > 1; ++it) {
+    const float flo = key_float(lo), fhi = key_float(static_cast<uint32_t>(hi - 1));
+    const float fm = 0.5f * flo + 0.5f * fhi;
+    uint32_t p = float_key(fm);
+    if (it >= 12 || !(isfinite(fm) && p > lo && static_cast<uint64_t>(p) < hi))
+      p = lo + static_cast<uint32_t>((hi - lo) >> 1);
+    const int c = count_ge(p);
+    if (c >= k) {
+      lo = p;
+      clo = c;
+    } else {
+      hi = p;
+      chi = c;
+    }
+  }
+  uint32_t T;
+  int gt;
+  if (hi - lo == 1) {
+    T = lo;
+    gt = chi;
+  } else if (clo - chi <= 64) {
+    // gather the bracket's keys and sort them
+    const uint32_t top = static_cast<uint32_t>(hi - 1);
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int base = 0;
+    for (int j0 = 0; j0 < nbp; j0 += 32) {
+      const uint32_t key = keys[j0 + lane];
+      const bool in = key >= lo && key <= top;
+      const uint32_t b = __ballot_sync(0xffffffffu, in);
+      const int pos = base + __popc(b & lt_mask);
+      if (in && pos < 64) cand[pos] = key;
+      base += __popc(b);
+    }
+    __syncwarp();
+    const int total = base;
+    uint32_t a = lane < total ? cand[lane] : 0u, b = lane + 32 < total ? cand[lane + 32] : 0u;
+    __syncwarp();
+    warp_sort64_desc(a, b, lane);
+    const int r = k - chi - 1;  // 0 <= r < clo - chi <= 64
+    const uint32_t va = __shfl_sync(0xffffffffu, a, r & 31), vb = __shfl_sync(0xffffffffu, b, r & 31);
+    T = r < 32 ? va : vb;
+    gt = chi + __popc(__ballot_sync(0xffffffffu, a > T)) + __popc(__ballot_sync(0xffffffffu, b > T));
+  } else {
+    // not narrowed in time (pathological rows): exact bitwise search
+    T = 0;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t c = T | (1u << bit);
+      if (count_ge(c) >= k) T = c;
+    }
+    gt = T == 0xFFFFFFFFu ? 0 : count_ge(T + 1);
+  }
+  // keys above T, then the lowest-index keys equal to T, in ascending index
+  const int need_eq = k - gt;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int written = 0, eq_seen = 0;
+  for (int j0 = 0; j0 < nbp && written < k; j0 += 32) {
+    const uint32_t key = keys[j0 + lane];
+    const bool eq = key == T;
+    const uint32_t eq_ballot = __ballot_sync(0xffffffffu, eq);
+    const int eq_rank = eq_seen + __popc(eq_ballot & lt_mask);
+    const bool sel = key > T || (eq && eq_rank < need_eq);
+    const uint32_t sel_ballot = __ballot_sync(0xffffffffu, sel);
+    const int pos = written + __popc(sel_ballot & lt_mask);
+    if (sel && pos < k) out[pos] = j0 + lane;
+    written += __popc(sel_ballot);
+    eq_seen += __popc(eq_ballot);
+  }
+}
+
+// Row setup shared by the two top-k kernels: the output row, and with the
+// causal flag the candidates [0, ncand) and the count ksel ranked among them
+// (row r is query block i = r % nb: only key blocks j <= i are ranked and
+// min(k, i + 1) are kept; with kFlagForceDiag block i always, plus the best
+// j < i; the row is padded with -1). Returns false when nothing is ranked.
+__device__ __forceinline__ bool topk_row_setup(long r, int nb, int k, unsigned flags, int32_t* out, int lane,
+                                               int& ncand, int& ksel) {
+  ncand = nb;
+  ksel = k;
   if (flags & kFlagCausal) {
     const int i = static_cast<int>(r % nb);
     const bool force = (flags & kFlagForceDiag) != 0;
@@ -290,8 +390,27 @@ __global__ void __launch_bounds__(kSelThreads, 4)
     ksel = force ? n - 1 : n;
     if (force && lane == 0) out[ksel] = i;  // above every ranked id: the list stays ascending
     for (int t = n + lane; t < k; t += 32) out[t] = -1;
-    if (ksel == 0) return;
+    if (ksel == 0) return false;
   }
+  return true;
+}
+
+// grid.x = ceil(rows / kSelWarps); one warp per row of S ([rows, nb]), nb <= 1024:
+// keys in registers.
+__global__ void __launch_bounds__(kSelThreads, 4)
+    block_topk_kernel(const float* __restrict__ S, int32_t* __restrict__ idx, long rows, int nb,
+                      int k, unsigned flags) {
+  pdl_launch_dependents();
+  pdl_wait();
+  __shared__ uint32_t cand[kSelWarps][64];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const long r = static_cast<long>(blockIdx.x) * kSelWarps + warp;
+  if (r >= rows) return;
+  const float* srow = S + r * nb;
+  int32_t* out = idx + r * static_cast<long>(k);
+  const bool vec = (nb & 3) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0;
+  int ncand, ksel;
+  if (!topk_row_setup(r, nb, k, flags, out, lane, ncand, ksel)) return;
   if (nb <= 32)
     select_row_bracket<1>(srow, nb, ncand, ksel, out, lane, cand[warp], vec);
   else if (nb <= 64)
@@ -302,19 +421,50 @@ __global__ void __launch_bounds__(kSelThreads, 4)
     select_row_bracket<8>(srow, nb, ncand, ksel, out, lane, cand[warp], vec);
   else if (nb <= 512)
     select_row_bracket<16>(srow, nb, ncand, ksel, out, lane, cand[warp], vec);
-  else if (nb <= 1024)
+  else
     select_row_bracket<32>(srow, nb, ncand, ksel, out, lane, cand[warp], vec);
-  else if (stage_rows) {
-    // the row is re-read once per key bit: stage it in shared memory
-    float* row = sel_rows + static_cast<long>(warp) * nb;
-    if ((nb & 3) == 0) {
-      for (int j = lane * 4; j < nb; j += 128)
-        *reinterpret_cast<float4*>(row + j) = __ldg(reinterpret_cast<const float4*>(srow + j));
+}
+
+// The same for nb > 1024. Dynamic shared memory: kSelWarps *
+// staged_row_keys(nb) keys when stage_rows (the keys of each warp's row,
+// converted once), else none (rows too long to stage are searched bit by bit
+// from L2).
+__global__ void __launch_bounds__(kSelThreads, 1)
+    block_topk_wide_kernel(const float* __restrict__ S, int32_t* __restrict__ idx, long rows, int nb,
+                           int k, int stage_rows, unsigned flags) {
+  pdl_launch_dependents();
+  pdl_wait();
+  extern __shared__ __align__(16) uint32_t sel_keys[];
+  __shared__ uint32_t cand[kSelWarps][64];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const long r = static_cast<long>(blockIdx.x) * kSelWarps + warp;
+  if (r >= rows) return;
+  const float* srow = S + r * nb;
+  int32_t* out = idx + r * static_cast<long>(k);
+  const bool vec = (nb & 3) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0;
+  int ncand, ksel;
+  if (!topk_row_setup(r, nb, k, flags, out, lane, ncand, ksel)) return;
+  if (stage_rows) {
+    const int nbp = staged_row_keys(nb);
+    uint32_t* keys = sel_keys + static_cast<long>(warp) * nbp;
+    if (vec) {
+      // 16-byte loads (nb % 4 == 0), several in flight per lane
+#pragma unroll 4
+      for (int j = 4 * lane; j < nbp; j += 128) {
+        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j < nb) f = __ldg(reinterpret_cast<const float4*>(srow + j));
+        uint4 u;
+        u.x = j < ncand ? score_key(f.x) : 0u;
+        u.y = j + 1 < ncand ? score_key(f.y) : 0u;
+        u.z = j + 2 < ncand ? score_key(f.z) : 0u;
+        u.w = j + 3 < ncand ? score_key(f.w) : 0u;
+        *reinterpret_cast<uint4*>(keys + j) = u;
+      }
     } else {
-      for (int j = lane; j < nb; j += 32) row[j] = __ldg(srow + j);
+      for (int j = lane; j < nbp; j += 32) keys[j] = j < ncand ? score_key(__ldg(srow + j)) : 0u;
     }
     __syncwarp();
-    select_row_smem(row, ncand, ksel, out, lane);
+    select_row_staged(keys, nbp, ncand, ksel, out, lane, cand[warp]);
   } else {
     select_row_smem(srow, ncand, ksel, out, lane);  // rows too long to stage: read them from L2
   }
