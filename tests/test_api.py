@@ -198,3 +198,47 @@ def test_polynomial_exp2_of_the_softmax():
     y = bits.astype(np.uint32).view(np.float32).astype(np.float64)
     ref = np.exp2(np.maximum(x.astype(np.float64), -125.0))
     assert np.all(np.abs(y / ref - 1) < 1e-4), np.abs(y / ref - 1).max()
+
+
+def _host_fwd(bsa, q=A, k=A, v=A, o=A + 0x100, B=1, N=512, H=2, Hkv=2, D=64, bs=64, ratio=0.25, dt=1, flags=0,
+              ws=A + 0x200, wsb=1 << 30):
+    P = ctypes.c_void_p
+    return bsa.lib.bsa_forward_host(P(q), P(k), P(v), P(o), B, N, H, Hkv, D, bs, ratio, dt, flags, P(ws), wsb,
+                                    P(0))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=0), 1), (dict(o=0), 1), (dict(N=500), 1), (dict(Hkv=3), 1), (dict(ratio=0.01), 1),
+    (dict(flags=4), 1), (dict(flags=2), 1), (dict(D=96), 2), (dict(dt=7), 2), (dict(ws=0), 4),
+    (dict(wsb=16), 4), (dict(ws=A + 0x210), 3),
+])
+def test_host_entry_point_rejects_bad_arguments(bsa, kw, status):
+    """bsa_forward_host validates on the host before touching a device (the
+    host pointers are not dereferenced here)."""
+    assert _host_fwd(bsa, **kw) == status
+
+
+def _bwd_gqa(bsa, H=4, Hkv=2, D=64, bs=128, kk=2, dt=1, flags=0, scale=0.125, ws=A + 0x400, wsb=1 << 30, dq=A + 0x100):
+    P = ctypes.c_void_p
+    return bsa.lib.bsa_sparse_attn_bwd_gqa(P(A), P(A), P(A), P(A), P(A), P(A), P(A), P(dq), P(A + 0x200),
+                                           P(A + 0x300), 1, 1024, H, Hkv, D, bs, kk, scale, dt, flags, P(ws), wsb,
+                                           P(0))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hkv=3), 1), (dict(bs=64), 2), (dict(dt=0), 2), (dict(kk=0), 1), (dict(kk=9), 1),
+    (dict(scale=0.0), 1), (dict(flags=2), 1), (dict(dq=A), 1), (dict(ws=0), 4), (dict(wsb=8), 4),
+])
+def test_grouped_backward_rejects_bad_arguments(bsa, kw, status):
+    assert _bwd_gqa(bsa, **kw) == status
+
+
+def test_grouped_training_workspace_is_per_key_value_head(bsa):
+    """The backward's bit matrix is per key/value head, D per query head."""
+    f = bsa.lib.bsa_sparse_attn_bwd_gqa_workspace_bytes
+    a = lambda x: (x + 255) // 256 * 256
+    B, N, H, Hkv, bs = 2, 8192, 8, 2, 128
+    nb = N // bs
+    assert f(B, N, H, Hkv, 128, bs) == a(B * Hkv * nb * ((nb + 31) // 32) * 4) + a(B * H * N * 4)
+    assert bsa.lib.bsa_sparse_attn_bwd_workspace_bytes(B, N, H, 128, bs) == f(B, N, H, H, 128, bs)
+    assert f(B, N, H, 3, 128, bs) == 0
