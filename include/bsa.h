@@ -221,7 +221,11 @@ bsa_status bsa_forward_gqa(const void* q, const void* k, const void* v, void* o,
  * workspace: device memory of bsa_forward_host_workspace_bytes() bytes,
  * 256-byte aligned (the chunk slots: q, k, v, o copies and a forward
  * workspace each). Calls on one device are serialized while they enqueue
- * (the internal streams are per device). Errors as for bsa_forward_gqa. */
+ * (the internal streams are per device). Errors as for bsa_forward_gqa;
+ * argument errors return before anything is enqueued, but a CUDA error
+ * returned after the first chunk may leave earlier copies and kernels
+ * running on the internal streams, so synchronize the device before reusing
+ * the buffers after such an error. */
 size_t bsa_forward_host_workspace_bytes(int B, int N, int H, int H_kv, int D, int block_size,
                                         double topk_ratio, bsa_dtype dt);
 
