@@ -10,12 +10,22 @@ Functions carry the C names:
 
 * ``bsa_block_pool(x, block_size)``                -> pooled [B, H, nb, D] float32
 * ``bsa_block_scores_topk(q_pooled, k_pooled, topk, scores=False)`` -> idx (, S)
-* ``bsa_sparse_attn_fwd(q, k, v, idx, block_size, scale=None)`` -> o
-* ``bsa_forward(q, k, v, block_size, topk_ratio, workspace=None)`` -> o
-* ``bsa_topk_count``, ``bsa_forward_workspace_bytes``, ``bsa_device_error``
+* ``bsa_sparse_attn_fwd(q, k, v, idx, block_size, scale=None, flags=0)`` -> o
+* ``bsa_forward(q, k, v, block_size, topk_ratio, workspace=None, flags=0)`` -> o
+* ``bsa_forward_host(q, k, v, block_size, topk_ratio)`` -> o, from and to
+  CPU tensors (chunked copies overlapped with the compute)
+* ``bsa_forward_noalloc(q, k, v, block_size, topk_ratio)`` -> o, with no
+  device allocation (a fixed scratch in the library)
+* ``bsa_sparse_attn_fwd_train(q, k, v, idx, block_size)`` -> (o, lse) and
+  ``bsa_sparse_attn_bwd(q, k, v, o, do, idx, lse, block_size)`` -> (dq, dk, dv)
+* ``bsa_topk_count``, ``bsa_forward_workspace_bytes``,
+  ``bsa_forward_host_workspace_bytes``, ``workspace_views``, ``bsa_device_error``
 
-q, k, v, o are [B, N, H, D] (float32 or bfloat16), contiguous, on one CUDA
-device.
+q, o are [B, N, H, D]; k, v are [B, N, H_kv, D] with H a multiple of H_kv
+(grouped queries; H_kv = H otherwise), contiguous, on one CUDA device
+(except for bsa_forward_host). Inputs are float32, bfloat16 or
+float8_e4m3fn (e4m3 gives a bfloat16 o). ``flags`` takes BSA_FLAG_CAUSAL and
+BSA_FLAG_FORCE_DIAG.
 """
 from __future__ import annotations
 
