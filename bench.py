@@ -70,6 +70,21 @@ def job_tokens_per_s(tokens_per_rank_step: int, world: int, steps: int, max_ms: 
     return world * tokens_per_rank_step * steps / (max_ms / 1e3)
 
 
+def attn_flops(B: int, H: int, Hk: int, N: int, D: int, bs: int, kk: int, idx=None, causal: bool = False) -> float:
+    """FLOPs of the attention over the kept blocks: 4 D per visible (query
+    token, key token) pair (two products). Without the causal mask every
+    query token sees k * bs keys: 4 B H N k bs D. With it, counted on the
+    index lists `idx` ([B, H_kv, nb, k], -1 padded) the step produced: bs^2
+    pairs per kept block below the query block, bs (bs + 1) / 2 for the
+    diagonal block; each key/value head's lists serve H / H_kv query heads."""
+    if not causal:
+        return 4.0 * B * H * N * kk * bs * D
+    il = np.asarray(idx, dtype=np.int64)
+    qi = np.arange(N // bs)[None, None, :, None]
+    pairs = np.where(il < 0, 0, np.where(il < qi, bs * bs, bs * (bs + 1) // 2)).sum()
+    return 4.0 * D * float(pairs) * (H // Hk)
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples while the timed region runs."""
 
@@ -262,12 +277,7 @@ def run_backward(args, cfg, dev, rank, world, dist, bsa, flags, variant):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
 
-    flops_f = 4.0 * B * H * N * kk * bs * D
-    if args.causal:
-        il = idx.cpu().numpy().astype(np.int64)
-        qi = np.arange(N // bs)[None, None, :, None]
-        pairs = np.where(il < 0, 0, np.where(il < qi, bs * bs, bs * (bs + 1) // 2)).sum()
-        flops_f = 4.0 * D * float(pairs) * (H // Hk)  # each key/value head's lists serve G query heads
+    flops_f = attn_flops(B, H, Hk, N, D, bs, kk, idx.cpu().numpy() if args.causal else None, args.causal)
     flops_b = 2.5 * flops_f  # five products of the forward's size (dS, dP recomputation not counted)
     peaks, peak_src = load_peaks()
     achieved = flops_b / (bwd_ms / 1e3) / 1e12
@@ -489,14 +499,7 @@ def main():
     tokens_step = B * N
     value = job_tokens_per_s(tokens_step, world, args.steps, total_ms)
     e2e_value = job_tokens_per_s(tokens_step, world, args.e2e_steps, e2e_ms)
-    flops = 4.0 * B * H * N * kk * bs * D
-    if args.causal:
-        # visible (query, key) token pairs of the lists the step produced:
-        # bs^2 per kept block below the diagonal, bs(bs+1)/2 for the diagonal
-        il = idx.cpu().numpy().astype(np.int64)
-        qi = np.arange(N // bs)[None, None, :, None]
-        pairs = np.where(il < 0, 0, np.where(il < qi, bs * bs, bs * (bs + 1) // 2)).sum()
-        flops = 4.0 * D * float(pairs) * (H // Hk)  # each key/value head's lists serve G query heads
+    flops = attn_flops(B, H, Hk, N, D, bs, kk, idx.cpu().numpy() if args.causal else None, args.causal)
     esz = cfg.elem_bytes
     tensor_bytes = B * N * H * D * esz  # q (and o)
     kv_bytes = B * N * Hk * D * esz     # k (and v): fewer heads with grouped queries

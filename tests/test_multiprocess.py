@@ -72,3 +72,36 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero():
     assert len(lines) == 1, r.stdout[-2000:]
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["value"] > 0 and line["n_gpus"] == 2
+
+
+def test_attention_flop_count_matches_a_brute_force_count():
+    """bench.attn_flops against 4 D times the visible (query token, key
+    token) pairs counted one by one, causal and not, with grouped queries and
+    -1 padded lists."""
+    import numpy as np
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    rng = np.random.default_rng(3)
+    B, H, Hk, nb, bs, D, kk = 2, 4, 2, 6, 8, 16, 3
+    N = nb * bs
+    idx = np.full((B, Hk, nb, kk), -1, np.int64)
+    for b in range(B):
+        for g in range(Hk):
+            for i in range(nb):
+                n = min(kk, i + 1)
+                idx[b, g, i, :n] = np.sort(rng.choice(i + 1, n, replace=False))
+    brute = 0
+    for b in range(B):
+        for g in range(Hk):
+            for i in range(nb):
+                for j in idx[b, g, i]:
+                    if j < 0:
+                        continue
+                    for r in range(bs):
+                        for c in range(bs):
+                            brute += (j * bs + c) <= (i * bs + r)
+    assert bench.attn_flops(B, H, Hk, N, D, bs, kk, idx, causal=True) == 4.0 * D * brute * (H // Hk)
+    full = B * H * N * kk * bs  # every query token sees k * bs keys
+    assert bench.attn_flops(B, H, Hk, N, D, bs, kk) == 4.0 * D * full
