@@ -139,6 +139,36 @@ def _dev(t: torch.Tensor, name: str) -> torch.Tensor:
     return t
 
 
+def _shape(t: torch.Tensor, want, name: str):
+    if tuple(t.shape) != tuple(want):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(want)}")
+
+
+def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
+    """q [B, N, H, D]; k and v [B, N, H_kv, D] with H a multiple of H_kv. The
+    library takes plain pointers, so a mismatch would read past a buffer: it
+    is refused here, before anything reaches the device."""
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, N, heads, D]")
+    B, N, H, D = q.shape
+    Hk = k.shape[2]
+    if k.shape[0] != B or k.shape[1] != N or k.shape[3] != D or Hk < 1 or H % Hk:
+        raise ValueError(f"k has shape {tuple(k.shape)}; q {tuple(q.shape)} needs [B, N, H_kv, D] with H % H_kv == 0")
+    _shape(v, k.shape, "v")
+
+
+def _check_idx(idx: torch.Tensor, B: int, Hk: int, N: int, block_size: int):
+    if idx.dim() != 4 or block_size < 1 or tuple(idx.shape[:3]) != (B, Hk, N // block_size):
+        raise ValueError(f"idx has shape {tuple(idx.shape)}, expected [{B}, {Hk}, {N // max(block_size, 1)}, topk]")
+
+
+def _check_out(out: torch.Tensor, q: torch.Tensor, name: str = "out"):
+    _shape(out, q.shape, name)
+    want = torch.bfloat16 if q.dtype == torch.float8_e4m3fn else q.dtype
+    if out.dtype != want:
+        raise TypeError(f"{name} must be {want}")
+
+
 def _p(t: torch.Tensor | None):
     return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
 
@@ -155,8 +185,12 @@ def bsa_forward_workspace_bytes(B: int, N: int, H: int, D: int, block_size: int,
 
 
 def bsa_block_pool(x: torch.Tensor, block_size: int, out: torch.Tensor | None = None) -> torch.Tensor:
-    _dev(x, "x")
+    if x.dim() != 4:
+        raise ValueError("x must be [B, N, H, D]")
     B, N, H, D = x.shape
+    if out is not None:
+        _shape(out, (B, H, N // max(block_size, 1), D), "out")
+    _dev(x, "x")
     if out is None:
         out = torch.empty((B, H, N // block_size, D), device=x.device, dtype=torch.float32)
     _check(lib.bsa_block_pool(_p(x), _p(out), B, N, H, D, block_size, _dtype_code(x), _stream(x)))
@@ -169,12 +203,20 @@ def bsa_block_scores_topk(q_pooled: torch.Tensor, k_pooled: torch.Tensor, topk: 
     """Block scores S (written to ``scores_out``, allocated if absent) and the
     top-k index list. Returns idx, or (idx, S) when ``scores`` is true.
     ``flags``: BSA_FLAG_CAUSAL / BSA_FLAG_FORCE_DIAG (bsa_block_scores_topk_ex)."""
+    if q_pooled.dim() != 4 or k_pooled.dim() != 4:
+        raise ValueError("pooled tensors must be [B, heads, nb, D]")
+    B, H, nb, D = q_pooled.shape
+    Hk = k_pooled.shape[1]  # key/value heads: fewer than H for grouped queries
+    if (k_pooled.shape[0], k_pooled.shape[2], k_pooled.shape[3]) != (B, nb, D) or Hk < 1 or H % Hk:
+        raise ValueError(f"k_pooled has shape {tuple(k_pooled.shape)}; q_pooled {tuple(q_pooled.shape)}")
+    if idx_out is not None:
+        _shape(idx_out, (B, Hk, nb, topk), "idx_out")
+    if scores_out is not None:
+        _shape(scores_out, (B, Hk, nb, nb), "scores_out")
     _dev(q_pooled, "q_pooled")
     _dev(k_pooled, "k_pooled")
     if q_pooled.dtype != torch.float32 or k_pooled.dtype != torch.float32:
         raise TypeError("pooled tensors must be float32")
-    B, H, nb, D = q_pooled.shape
-    Hk = k_pooled.shape[1]  # key/value heads: fewer than H for grouped queries
     idx = idx_out if idx_out is not None else torch.empty((B, Hk, nb, topk), device=q_pooled.device, dtype=torch.int32)
     S = scores_out if scores_out is not None else torch.empty((B, Hk, nb, nb), device=q_pooled.device,
                                                               dtype=torch.float32)
@@ -192,6 +234,10 @@ def bsa_block_scores_topk(q_pooled: torch.Tensor, k_pooled: torch.Tensor, topk: 
 
 def bsa_sparse_attn_fwd(q, k, v, idx, block_size: int, scale: float | None = None,
                         out: torch.Tensor | None = None, flags: int = 0) -> torch.Tensor:
+    _check_qkv(q, k, v)
+    _check_idx(idx, q.shape[0], k.shape[2], q.shape[1], block_size)
+    if out is not None:
+        _check_out(out, q)
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (idx, "idx")):
         _dev(t, n)
     if idx.dtype != torch.int32:
@@ -218,6 +264,9 @@ def bsa_sparse_attn_fwd(q, k, v, idx, block_size: int, scale: float | None = Non
 
 def bsa_forward(q, k, v, block_size: int, topk_ratio: float, workspace: torch.Tensor | None = None,
                 out: torch.Tensor | None = None, flags: int = 0) -> torch.Tensor:
+    _check_qkv(q, k, v)
+    if out is not None:
+        _check_out(out, q)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _dev(t, n)
     if not (q.dtype == k.dtype == v.dtype):
@@ -259,6 +308,9 @@ def bsa_forward_host(q, k, v, block_size: int, topk_ratio: float, out: torch.Ten
     them on the current stream there and copies the results back. With
     synchronize=False the call returns once the work is enqueued; the output
     is complete when the current stream of `device` is."""
+    _check_qkv(q, k, v)
+    if out is not None:
+        _check_out(out, q)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         if t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{n} must be a contiguous CPU tensor")
@@ -289,6 +341,12 @@ def bsa_sparse_attn_fwd_train(q, k, v, idx, block_size: int, scale: float | None
     """The attention forward that also returns lse [B,H,N] (ln of each row's
     softmax denominator), for bsa_sparse_attn_bwd. Returns (o, lse). k and v
     may have fewer heads than q (grouped queries; idx per key/value head)."""
+    _check_qkv(q, k, v)
+    _check_idx(idx, q.shape[0], k.shape[2], q.shape[1], block_size)
+    if out is not None:
+        _check_out(out, q)
+    if lse is not None:
+        _shape(lse, (q.shape[0], q.shape[2], q.shape[1]), "lse")
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (idx, "idx")):
         _dev(t, n)
     B, N, H, D = q.shape
@@ -309,6 +367,11 @@ def bsa_sparse_attn_bwd(q, k, v, o, do, idx, lse, block_size: int, scale: float 
     index lists held fixed; o and lse from bsa_sparse_attn_fwd_train. With
     grouped queries (k, v with fewer heads than q) dk and dv are per
     key/value head, summed over the group's query heads."""
+    _check_qkv(q, k, v)
+    _check_idx(idx, q.shape[0], k.shape[2], q.shape[1], block_size)
+    _check_out(o, q, "o")
+    _shape(do, q.shape, "do")
+    _shape(lse, (q.shape[0], q.shape[2], q.shape[1]), "lse")
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do"), (idx, "idx"), (lse, "lse")):
         _dev(t, n)
     B, N, H, D = q.shape
@@ -331,6 +394,10 @@ def bsa_forward_noalloc(q, k, v, block_size: int, topk_ratio: float, out: torch.
     """bsa_forward with its intermediates in the library's fixed device scratch
     (for callers that cannot allocate device memory; see include/bsa.h for the
     size limit and the sharing rules)."""
+    _check_qkv(q, k, v)
+    _shape(k, q.shape, "k")  # one key/value head per query head
+    if out is not None:
+        _check_out(out, q)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _dev(t, n)
     if not (q.dtype == k.dtype == v.dtype):

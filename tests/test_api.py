@@ -242,3 +242,41 @@ def test_grouped_training_workspace_is_per_key_value_head(bsa):
     assert f(B, N, H, Hkv, 128, bs) == a(B * Hkv * nb * ((nb + 31) // 32) * 4) + a(B * H * N * 4)
     assert bsa.lib.bsa_sparse_attn_bwd_workspace_bytes(B, N, H, 128, bs) == f(B, N, H, H, 128, bs)
     assert f(B, N, H, 3, 128, bs) == 0
+
+
+def test_binding_refuses_mismatched_shapes_before_the_device(bsa):
+    """The C ABI takes plain pointers, so the binding checks the tensors'
+    shapes first: a mismatch would otherwise read past a buffer on the GPU.
+    CPU tensors reach these checks before the device check."""
+    q = torch.zeros(1, 512, 4, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 512, 2, 64, dtype=torch.bfloat16)
+    bad = [
+        lambda: bsa.bsa_forward(q, k, torch.zeros(1, 512, 4, 64, dtype=torch.bfloat16), 64, 0.5),  # v != k
+        lambda: bsa.bsa_forward(q, torch.zeros(1, 512, 3, 64, dtype=torch.bfloat16),
+                                torch.zeros(1, 512, 3, 64, dtype=torch.bfloat16), 64, 0.5),  # 4 % 3
+        lambda: bsa.bsa_forward(q, torch.zeros(1, 256, 2, 64, dtype=torch.bfloat16),
+                                torch.zeros(1, 256, 2, 64, dtype=torch.bfloat16), 64, 0.5),  # N differs
+        lambda: bsa.bsa_forward(q, k, k, 64, 0.5, out=torch.zeros(1, 512, 2, 64, dtype=torch.bfloat16)),
+        lambda: bsa.bsa_sparse_attn_fwd(q, k, k, torch.zeros(1, 4, 8, 2, dtype=torch.int32), 64),  # idx per kv head
+        lambda: bsa.bsa_sparse_attn_fwd_train(q, k, k, torch.zeros(1, 2, 8, 2, dtype=torch.int32), 64,
+                                              lse=torch.zeros(1, 512, 4)),
+        lambda: bsa.bsa_sparse_attn_bwd(q, k, k, q, q[:, :256], torch.zeros(1, 2, 8, 2, dtype=torch.int32),
+                                        torch.zeros(1, 4, 512), 64),  # do
+        lambda: bsa.bsa_forward_noalloc(q, k, k, 64, 0.5),  # no grouped queries there
+        lambda: bsa.bsa_forward_host(q, k, k, 64, 0.5, out=torch.zeros(1, 512, 4, 64)),  # out dtype
+        lambda: bsa.bsa_block_scores_topk(torch.zeros(1, 4, 8, 64), torch.zeros(1, 2, 9, 64), 2),
+        lambda: bsa.bsa_block_pool(q, 64, out=torch.zeros(1, 4, 4, 64)),
+    ]
+    for i, f in enumerate(bad):
+        with pytest.raises((ValueError, TypeError)) as e:
+            f()
+        assert "CUDA tensor" not in str(e.value), (i, str(e.value))
+    # consistent shapes pass these checks and stop at the device check
+    idx = torch.zeros(1, 2, 8, 2, dtype=torch.int32)
+    for f in (lambda: bsa.bsa_forward(q, k, k, 64, 0.5),
+              lambda: bsa.bsa_sparse_attn_fwd(q, k, k, idx, 64),
+              lambda: bsa.bsa_sparse_attn_fwd_train(q, k, k, idx, 64, lse=torch.zeros(1, 4, 512)),
+              lambda: bsa.bsa_sparse_attn_bwd(q, k, k, q, q, idx, torch.zeros(1, 4, 512), 64),
+              lambda: bsa.bsa_block_scores_topk(torch.zeros(1, 4, 8, 64), torch.zeros(1, 2, 8, 64), 2)):
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            f()
