@@ -38,10 +38,11 @@ import workloads as W  # noqa: E402
 
 METRIC = "block-sparse attn fwd tokens/s & effective TFLOP/s (% roofline), 1 B200"
 
-# DRAM read + write bytes per launch of the attention kernel, from the ncu
-# capture recorded in profiles/sparse_attn_tc2_traffic.md (the kernel as it
-# stands); workloads not captured report null.
-NCU_TRAFFIC = {"c3": 810.46e6 + 249.09e6, "c4": 4.93e9 + 588.97e6}
+# DRAM read + write bytes per launch of the attention kernel from an ncu
+# capture of the kernel as it stands, per workload; null where there is none.
+# (The captures in profiles/sparse_attn_tc2_traffic.md predate the kernel's
+# programmatic-launch entry instructions, so they are not used here.)
+NCU_TRAFFIC = {}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
