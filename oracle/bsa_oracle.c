@@ -163,58 +163,21 @@ void oracle_topk(const double* S, long nrows_total, int nb, int k, int* idx) {
   for (long r = 0; r < nrows_total; ++r) oracle_topk_row(S + r * nb, nb, k, idx + r * k);
 }
 
+void oracle_sparse_attn_gqa(const void* q, const void* kmat, const void* v, int dtype, int B, int N,
+                            int H, int Hkv, int D, int bs, const int* idx, int k, const int* rows,
+                            int nrows, double scale, int flags, double* o);
+
 /* [SF] step 3 / [MSA] §2.1-§2.2: for every query row n of query block i,
  *   l_t = scale * sum_d q[b,n,h,d] * k[b,t,h,d]   for t in the selected blocks,
  *   o[n] = sum_t exp(l_t - max l) v[b,t,h,:] / sum_t exp(l_t - max l).
  * The selected blocks of (b, h, rows[b,h,r]) are idx[b, h, r, 0..k).
- * Output o is [B, H, nrows, bs, D] (float64). rows == NULL means all nb. */
+ * Output o is [B, H, nrows, bs, D] (float64). rows == NULL means all nb.
+ * The arithmetic is written out once, in oracle_sparse_attn_gqa below (with
+ * one key/value head per query head it is exactly this definition). */
 void oracle_sparse_attn(const void* q, const void* kmat, const void* v, int dtype, int B, int N,
                         int H, int D, int bs, const int* idx, int k, const int* rows, int nrows,
                         double scale, double* o) {
-  int nb = N / bs;
-  (void)nb;
-  long ntok = (long)k * bs;
-#pragma omp parallel
-  {
-    double* logit = (double*)malloc((size_t)ntok * sizeof(double));
-    double* qrow = (double*)malloc((size_t)D * sizeof(double));
-#pragma omp for collapse(4) schedule(dynamic, 4)
-    for (int b = 0; b < B; ++b)
-      for (int h = 0; h < H; ++h)
-        for (int r = 0; r < nrows; ++r)
-          for (int t_q = 0; t_q < bs; ++t_q) {
-            size_t bh = (size_t)b * H + h;
-            int i = rows ? rows[bh * nrows + r] : r;
-            const int* sel = idx + (bh * nrows + r) * k;
-            int n = i * bs + t_q;
-            for (int d = 0; d < D; ++d) qrow[d] = elem(q, dtype, at_bnhd(N, H, D, b, n, h, d));
-            /* logits over the tokens of the selected blocks */
-            double m = -INFINITY;
-            for (int s = 0; s < k; ++s)
-              for (int u = 0; u < bs; ++u) {
-                int t = sel[s] * bs + u;
-                double dot = 0.0;
-                for (int d = 0; d < D; ++d) dot += qrow[d] * elem(kmat, dtype, at_bnhd(N, H, D, b, t, h, d));
-                double l = scale * dot;
-                logit[(long)s * bs + u] = l;
-                if (l > m) m = l;
-              }
-            /* softmax weights and the weighted sum of v */
-            double* out = o + ((bh * nrows + r) * bs + t_q) * D;
-            for (int d = 0; d < D; ++d) out[d] = 0.0;
-            double z = 0.0;
-            for (int s = 0; s < k; ++s)
-              for (int u = 0; u < bs; ++u) {
-                int t = sel[s] * bs + u;
-                double w = exp(logit[(long)s * bs + u] - m);
-                z += w;
-                for (int d = 0; d < D; ++d) out[d] += w * elem(v, dtype, at_bnhd(N, H, D, b, t, h, d));
-              }
-            for (int d = 0; d < D; ++d) out[d] /= z;
-          }
-    free(logit);
-    free(qrow);
-  }
+  oracle_sparse_attn_gqa(q, kmat, v, dtype, B, N, H, H, D, bs, idx, k, rows, nrows, scale, 0, o);
 }
 
 /* Number of OpenMP threads the oracle runs with (reported by the CPU baseline). */
@@ -278,57 +241,11 @@ void oracle_topk_ex(const double* S, long nrows_total, int nb, int k, const int*
 
 /* oracle_sparse_attn with flags: entries of idx below 0 select nothing, and
  * with ORACLE_CAUSAL key token t is left out of the softmax of query token n
- * when t > n. */
+ * when t > n. (Written out in oracle_sparse_attn_gqa, with Hkv = H.) */
 void oracle_sparse_attn_ex(const void* q, const void* kmat, const void* v, int dtype, int B, int N,
                            int H, int D, int bs, const int* idx, int k, const int* rows, int nrows,
                            double scale, int flags, double* o) {
-  long ntok = (long)k * bs;
-#pragma omp parallel
-  {
-    double* logit = (double*)malloc((size_t)ntok * sizeof(double));
-    double* qrow = (double*)malloc((size_t)D * sizeof(double));
-#pragma omp for collapse(4) schedule(dynamic, 4)
-    for (int b = 0; b < B; ++b)
-      for (int h = 0; h < H; ++h)
-        for (int r = 0; r < nrows; ++r)
-          for (int t_q = 0; t_q < bs; ++t_q) {
-            size_t bh = (size_t)b * H + h;
-            int i = rows ? rows[bh * nrows + r] : r;
-            const int* sel = idx + (bh * nrows + r) * k;
-            int n = i * bs + t_q;
-            for (int d = 0; d < D; ++d) qrow[d] = elem(q, dtype, at_bnhd(N, H, D, b, n, h, d));
-            double m = -INFINITY;
-            for (int s = 0; s < k; ++s)
-              for (int u = 0; u < bs; ++u) {
-                double l = -INFINITY; /* masked or unselected */
-                if (sel[s] >= 0) {
-                  int t = sel[s] * bs + u;
-                  if (!(flags & ORACLE_CAUSAL) || t <= n) {
-                    double dot = 0.0;
-                    for (int d = 0; d < D; ++d) dot += qrow[d] * elem(kmat, dtype, at_bnhd(N, H, D, b, t, h, d));
-                    l = scale * dot;
-                  }
-                }
-                logit[(long)s * bs + u] = l;
-                if (l > m) m = l;
-              }
-            double* out = o + ((bh * nrows + r) * bs + t_q) * D;
-            for (int d = 0; d < D; ++d) out[d] = 0.0;
-            double z = 0.0;
-            for (int s = 0; s < k; ++s)
-              for (int u = 0; u < bs; ++u) {
-                double l = logit[(long)s * bs + u];
-                if (l == -INFINITY) continue;
-                int t = sel[s] * bs + u;
-                double w = exp(l - m);
-                z += w;
-                for (int d = 0; d < D; ++d) out[d] += w * elem(v, dtype, at_bnhd(N, H, D, b, t, h, d));
-              }
-            for (int d = 0; d < D; ++d) out[d] /= z;
-          }
-    free(logit);
-    free(qrow);
-  }
+  oracle_sparse_attn_gqa(q, kmat, v, dtype, B, N, H, H, D, bs, idx, k, rows, nrows, scale, flags, o);
 }
 
 /* ------------------------------------------------------------------------
@@ -340,60 +257,84 @@ void oracle_sparse_attn_ex(const void* q, const void* kmat, const void* v, int d
  * linearity is the mean of the G heads' block scores.
  * ------------------------------------------------------------------------ */
 
-/* oracle_sparse_attn_ex with Hkv key/value heads: q and o have H heads, k and
- * v have Hkv; idx and rows are per query head ([B, H, nrows, k], [B, H, nrows]). */
+/* The attention over the kept blocks, with Hkv key/value heads: q and o have
+ * H heads, k and v have Hkv; idx and rows are per query head ([B, H, nrows, k],
+ * [B, H, nrows]). For every query row n of query block i = rows[b,h,r]:
+ *   l_t = scale * sum_d q[b,n,h,d] * k[b,t,g,d]  (g = h / G) for the tokens t
+ *         of the kept blocks (an entry below 0 keeps nothing; with
+ *         ORACLE_CAUSAL, t > n is left out),
+ *   m = max_t l_t,  w_t = exp(l_t - m),  o[n] = sum_t w_t v[b,t,g,:] / sum_t w_t.
+ * Each key/value head's k and v rows are first converted (exactly) to one
+ * contiguous float64 array, so the sums below read plain doubles; every sum
+ * runs in the order written. Parallel over query rows only. */
 void oracle_sparse_attn_gqa(const void* q, const void* kmat, const void* v, int dtype, int B, int N,
                             int H, int Hkv, int D, int bs, const int* idx, int k, const int* rows,
                             int nrows, double scale, int flags, double* o) {
   long ntok = (long)k * bs;
   int G = H / Hkv;
+  double* kd = (double*)malloc((size_t)N * D * sizeof(double));
+  double* vd = (double*)malloc((size_t)N * D * sizeof(double));
+  for (int b = 0; b < B; ++b)
+    for (int g = 0; g < Hkv; ++g) {
+      /* k[b, :, g, :] and v[b, :, g, :] as float64 [N, D] */
+#pragma omp parallel for schedule(static)
+      for (int n = 0; n < N; ++n)
+        for (int d = 0; d < D; ++d) {
+          kd[(size_t)n * D + d] = elem(kmat, dtype, at_bnhd(N, Hkv, D, b, n, g, d));
+          vd[(size_t)n * D + d] = elem(v, dtype, at_bnhd(N, Hkv, D, b, n, g, d));
+        }
 #pragma omp parallel
-  {
-    double* logit = (double*)malloc((size_t)ntok * sizeof(double));
-    double* qrow = (double*)malloc((size_t)D * sizeof(double));
-#pragma omp for collapse(4) schedule(dynamic, 4)
-    for (int b = 0; b < B; ++b)
-      for (int h = 0; h < H; ++h)
-        for (int r = 0; r < nrows; ++r)
-          for (int t_q = 0; t_q < bs; ++t_q) {
-            size_t bh = (size_t)b * H + h;
-            int g = h / G;
-            int i = rows ? rows[bh * nrows + r] : r;
-            const int* sel = idx + (bh * nrows + r) * k;
-            int n = i * bs + t_q;
-            for (int d = 0; d < D; ++d) qrow[d] = elem(q, dtype, at_bnhd(N, H, D, b, n, h, d));
-            double m = -INFINITY;
-            for (int s = 0; s < k; ++s)
-              for (int u = 0; u < bs; ++u) {
-                double l = -INFINITY; /* masked or unselected */
-                if (sel[s] >= 0) {
-                  int t = sel[s] * bs + u;
-                  if (!(flags & ORACLE_CAUSAL) || t <= n) {
-                    double dot = 0.0;
-                    for (int d = 0; d < D; ++d) dot += qrow[d] * elem(kmat, dtype, at_bnhd(N, Hkv, D, b, t, g, d));
-                    l = scale * dot;
+      {
+        double* logit = (double*)malloc((size_t)ntok * sizeof(double));
+        double* qrow = (double*)malloc((size_t)D * sizeof(double));
+#pragma omp for collapse(3) schedule(dynamic, 4)
+        for (int hg = 0; hg < G; ++hg)
+          for (int r = 0; r < nrows; ++r)
+            for (int t_q = 0; t_q < bs; ++t_q) {
+              int h = g * G + hg;
+              size_t bh = (size_t)b * H + h;
+              int i = rows ? rows[bh * nrows + r] : r;
+              const int* sel = idx + (bh * nrows + r) * k;
+              int n = i * bs + t_q;
+              for (int d = 0; d < D; ++d) qrow[d] = elem(q, dtype, at_bnhd(N, H, D, b, n, h, d));
+              /* logits over the tokens of the selected blocks */
+              double m = -INFINITY;
+              for (int s = 0; s < k; ++s)
+                for (int u = 0; u < bs; ++u) {
+                  double l = -INFINITY; /* masked or unselected */
+                  if (sel[s] >= 0) {
+                    int t = sel[s] * bs + u;
+                    if (!(flags & ORACLE_CAUSAL) || t <= n) {
+                      const double* kt = kd + (size_t)t * D;
+                      double dot = 0.0;
+                      for (int d = 0; d < D; ++d) dot += qrow[d] * kt[d];
+                      l = scale * dot;
+                    }
                   }
+                  logit[(long)s * bs + u] = l;
+                  if (l > m) m = l;
                 }
-                logit[(long)s * bs + u] = l;
-                if (l > m) m = l;
-              }
-            double* out = o + ((bh * nrows + r) * bs + t_q) * D;
-            for (int d = 0; d < D; ++d) out[d] = 0.0;
-            double z = 0.0;
-            for (int s = 0; s < k; ++s)
-              for (int u = 0; u < bs; ++u) {
-                double l = logit[(long)s * bs + u];
-                if (l == -INFINITY) continue;
-                int t = sel[s] * bs + u;
-                double w = exp(l - m);
-                z += w;
-                for (int d = 0; d < D; ++d) out[d] += w * elem(v, dtype, at_bnhd(N, Hkv, D, b, t, g, d));
-              }
-            for (int d = 0; d < D; ++d) out[d] /= z;
-          }
-    free(logit);
-    free(qrow);
-  }
+              /* softmax weights and the weighted sum of v */
+              double* out = o + ((bh * nrows + r) * bs + t_q) * D;
+              for (int d = 0; d < D; ++d) out[d] = 0.0;
+              double z = 0.0;
+              for (int s = 0; s < k; ++s)
+                for (int u = 0; u < bs; ++u) {
+                  double l = logit[(long)s * bs + u];
+                  if (l == -INFINITY) continue;
+                  const double* vt = vd + (size_t)(sel[s] * bs + u) * D;
+                  double w = exp(l - m);
+                  z += w;
+                  for (int d = 0; d < D; ++d) out[d] += w * vt[d];
+                }
+              for (int d = 0; d < D; ++d) out[d] /= z;
+            }
+        free(logit);
+        free(qrow);
+      }
+    }
+  free(kd);
+  free(vd);
 }
 
 /* ------------------------------------------------------------------------

@@ -68,9 +68,9 @@ class Config:
 CONFIGS = {
     "c1": Config("c1", 1, 512, 2, 64, 64, 0.25, "f32", 1.0, 0, None,
                  "tiny fp32 non-causal MHA; also run at topk_ratio=1.0 (dense)"),
-    "c2": Config("c2", 32, 8192, 16, 64, 64, 0.3, "bf16", 1.0, 1, 2,
+    "c2": Config("c2", 32, 8192, 16, 64, 64, 0.3, "bf16", 1.0, 1, None,
                  "page-1 benchmark shape: seq 8192, hidden 1024 = 16 x 64, batch 32"),
-    "c3": Config("c3", 2, 32768, 16, 128, 128, 0.2, "bf16", 0.5, 2, 4,
+    "c3": Config("c3", 2, 32768, 16, 128, 128, 0.2, "bf16", 0.5, 2, None,
                  "closer block scores (offset sigma 0.5)"),
     "c4": Config("c4", 1, 131072, 16, 128, 128, 0.15, "bf16", 1.0, 3, 32,
                  "long context"),
