@@ -14,10 +14,16 @@ max) and by at most the weight itself below it, so per output element
 bfloat16 rounding of o. The first term is computed here exactly with the
 oracle run on |v| (same weights); the small-weight term and the rounding are
 covered by an absolute 2^-8 * max|v| and a relative 2^-8 |o|. Over a whole
-output the weights' rounding errors (uniform, at most 2^-4 of each weight)
-have an rms of 2^-4 / sqrt(3) = 0.036 of the weights, and o's error is a
-weighted combination of them: relative L2 <= 0.036. Index lists follow the
-near-tie rule (pooling reads the exact e4m3 values).
+output o's error is a weighted combination of the weights' rounding errors.
+A weight p = 2^x rounded to nearest in e4m3 (spacing 2^-3 of its binade) has
+an error uniform within half a spacing, so its relative error has rms
+2^-4 / (sqrt(3) m) for mantissa m in [1, 2). The weights are exponentials of
+smoothly spread logits, so their mantissas are log-uniform, E[1/m^2] =
+3 / (8 ln 2), and the relative rms is 2^-4 sqrt(1 / (8 ln 2)) = 0.0265 (the
+distribution-free bound, m -> 1, is 2^-4 / sqrt(3) = 0.036). Relative L2 of
+the output: <= 0.03, that expectation with a 13% margin (measured 0.022 to
+0.026 on these cases). Index lists follow the near-tie rule (pooling reads
+the exact e4m3 values).
 """
 import numpy as np
 import pytest
@@ -45,7 +51,7 @@ def check_fp8_output(o_gpu, o_ref, o_abs, vmax):
     rel = np.linalg.norm(o_gpu - o_ref) / np.linalg.norm(o_ref)
     print(f"fp8: max|d| {d.max():.3g}, max|d|/bound {(d / bound).max():.3g}, rel L2 {rel:.3g}")
     assert np.all(d <= bound), f"max|d|/bound = {(d / bound).max()}"
-    assert rel <= 2.0 ** -4 / np.sqrt(3.0), f"rel L2 = {rel}"
+    assert rel <= 0.03, f"rel L2 = {rel}"
 
 
 CASES = [  # (B, N, H, H_kv, block_size, ratio, causal)
