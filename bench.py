@@ -39,9 +39,8 @@ import workloads as W  # noqa: E402
 METRIC = "block-sparse attn fwd tokens/s & effective TFLOP/s (% roofline), 1 B200"
 
 # DRAM read + write bytes per launch of the attention kernel from an ncu
-# capture of the kernel as it stands, per workload; null where there is none.
-# (The captures in profiles/sparse_attn_tc2_traffic.md predate the kernel's
-# programmatic-launch entry instructions, so they are not used here.)
+# capture of the kernel as it stands, per workload; null where there is none
+# (a capture of an earlier version of the kernel does not count).
 NCU_TRAFFIC = {}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -172,6 +171,18 @@ def oracle_sample(q, k, v, cfg: W.Config, heads, blocks_per_head: int, seed: int
     return tokens, secs, oracle.num_threads()
 
 
+def workload_config(cfg: W.Config, args, world: int, training: bool = False) -> dict:
+    """The `config` object of the JSON line, the same for both arms."""
+    variant = (" causal" + (" force_diag" if args.force_diag else "")) if args.causal else ""
+    what = " training step (forward with lse + backward)" if training else ""
+    big = cfg.B * cfg.N * cfg.H * cfg.D * cfg.elem_bytes
+    names = "q, k, v, dO" if training else "q, k, v"
+    return {"workload": f"{cfg.name}{variant}{what}: {cfg.describe()}", "seed": cfg.seed,
+            "l2": (f"inputs larger than L2 ({names} {big / 1e6:.0f} MB each)" if big > 126e6 else
+                   f"inputs smaller than L2 ({names} {big / 1e6:.1f} MB each), not flushed"),
+            "parallelism": f"replica per GPU x{world}"}
+
+
 def run_reference(args, cfg, rank, world):
     if rank != 0:
         return
@@ -192,9 +203,7 @@ def run_reference(args, cfg, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": f"{cfg.name}{' causal' if args.causal else ''}"
-                                   f"{' force_diag' if args.force_diag else ''}: {cfg.describe()}",
-                       "seed": cfg.seed},
+            "config": workload_config(cfg, args, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -288,9 +297,7 @@ def run_backward(args, cfg, dev, rank, world, dist, bsa, flags, variant):
         "metric": METRIC, "value": job_tokens_per_s(B * N, world, args.steps, total_ms), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-        "config": {"workload": f"{cfg.name}{variant} training step (forward with lse + backward): {cfg.describe()}",
-                   "seed": cfg.seed, "l2": f"inputs larger than L2 (q, k, v, dO {nbytes / 1e6:.0f} MB each)",
-                   "parallelism": f"replica per GPU x{world}"},
+        "config": workload_config(cfg, args, world, training=True),
         "gpu_launches": 5 * args.steps,
         "stages_ms": {"fwd_train": fwd_ms, "bwd": bwd_ms},
         "e2e": {"value": job_tokens_per_s(B * N, world, args.e2e_steps, e2e_ms), "unit": "tokens/s",
@@ -516,9 +523,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-        "config": {"workload": f"{cfg.name}{variant}: {cfg.describe()}", "seed": cfg.seed,
-                   "l2": f"inputs larger than L2 (q, k, v {tensor_bytes / 1e6:.0f} MB each)",
-                   "parallelism": f"replica per GPU x{world}"},
+        "config": workload_config(cfg, args, world),
         "tflops_effective": flops / (step_ms / 1e3) / 1e12,
         "gpu_launches": 5 * args.steps,
         "stages_ms": {"pool_qk": pool_ms, "scores_topk": sel_ms, "sparse_attn": attn_ms,

@@ -763,8 +763,8 @@ bsa_status bsa_device_error(int* code_out, void* stream) {
 
 // ==================================================================== forward without allocation
 //
-// bsa_forward needs a workspace (pooled q, pooled k, index list) that the
-// caller allocates. Some callers cannot allocate device memory at all: a
+// bsa_forward needs a workspace (pooled q, pooled k, the index list and the
+// block-score matrix) that the caller allocates. Some callers cannot allocate device memory at all: a
 // plugin running inside a host application that owns the whole device-memory
 // budget, or a latency-critical loop where a cudaMalloc (and the implicit
 // device synchronisation it may bring) is not allowed. bsa_forward_noalloc
@@ -781,20 +781,53 @@ namespace {
 
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[64] = {};
+unsigned long long g_noalloc_ctx[64] = {};  // id of the context the address belongs to
 
-// Device address of g_noalloc_scratch on the current device; the first call
-// on each device performs the lookup (with that device current).
+// Unique id of the current context (cuCtxGetId: ids are never reused within
+// a process), 0 when it cannot be read.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_noalloc_scratch on the current device. The lookup
+// (with that device current) runs on the first call on each device and again
+// whenever the device's context has changed since (a cudaDeviceReset destroys
+// the context and the next one loads the module anew, possibly elsewhere);
+// when the context id cannot be read, it runs on every call.
 bsa_status noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(BSA_ERR_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= 64) return fail(BSA_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+  // 0 when no context is current yet: the lookup below then creates it
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  if (g_noalloc_ptr[dev] == nullptr || ctx == 0 || g_noalloc_ctx[dev] != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = current_context_id();  // the context the address belongs to
   }
   *out = g_noalloc_ptr[dev];
   return BSA_OK;
@@ -819,7 +852,7 @@ extern "C" bsa_status bsa_forward_noalloc(const void* q, const void* k, const vo
   if ((s = check_device()) != BSA_OK) return s;
   void* scratch = nullptr;
   if ((s = noalloc_scratch(&scratch)) != BSA_OK) return s;
-  // Nothing in the scratch has to start at zero: every byte the three
+  // Nothing in the scratch has to start at zero: every byte the forward's
   // kernels read was written earlier in the same call.
   return bsa_forward(q, k, v, o, B, N, H, D, block_size, topk_ratio, dt, scratch,
                      static_cast<size_t>(BSA_NOALLOC_SCRATCH_BYTES), stream);

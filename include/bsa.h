@@ -15,7 +15,7 @@
  *
  * Conventions for every entry point:
  *   - Tensors are dense and row-major. q, k, v, o are [B, N, H, D] (the head
- *     axis inside the token axis, as the page's listing takes them); pooled
+ *     axis inside the token axis, as the "SparseFormer 注意力实现" section takes them); pooled
  *     tensors are [B, H, nb, D] float32; index lists are [B, H, nb, k] int32,
  *     each row strictly ascending by key-block id.
  *   - All pointers are DEVICE pointers unless stated otherwise. The caller owns
@@ -68,8 +68,8 @@ typedef enum {
 } bsa_dtype;
 
 /* Number of kept key blocks: floor(topk_ratio * nb) evaluated in IEEE double,
- * which equals Python's int(topk_ratio * num_blocks) in the page's listing
- * (step 2). Returns -1 if nb < 1 or topk_ratio is negative or not finite.
+ * which equals the Python int() of that product that page "2026 新一代卷积与
+ * Transformer 网络架构" (section "SparseFormer 注意力实现", step 2) uses. Returns -1 if nb < 1 or topk_ratio is negative or not finite.
  * Pure host function. */
 int bsa_topk_count(int nb, double topk_ratio);
 
@@ -79,15 +79,18 @@ int bsa_topk_count(int nb, double topk_ratio);
  * are invalid. Pure host function. */
 size_t bsa_forward_workspace_bytes(int B, int N, int H, int D, int block_size, double topk_ratio);
 
-/* Step 1a (page listing, step 1: x.view(B, nb, bs, H, D).mean(2)):
+/* Step 1a (page "2026 新一代卷积与 Transformer 网络架构", section "SparseFormer
+ * 注意力实现", step 1: the mean of each block of block_size consecutive tokens,
+ * per batch entry and head):
  *   x_pooled[b, h, i, d] = (1/block_size) * sum_{t<block_size} x[b, i*block_size + t, h, d]
  * x: [B, N, H, D] of dtype dt (read only). x_pooled: [B, H, nb, D] float32
  * (written). Sums are accumulated in float32. */
 bsa_status bsa_block_pool(const void* x, float* x_pooled, int B, int N, int H, int D,
                           int block_size, bsa_dtype dt, void* stream);
 
-/* Steps 1b + 2 (page listing: einsum of the pooled tensors per (b, h), then
- * torch.topk over the key-block axis):
+/* Steps 1b + 2 (same page and section, steps 1 and 2: the dot product of every
+ * pooled query block with every pooled key block of the same (b, h), then the
+ * topk largest of each row):
  *   S[b, h, i, j] = sum_d q_pooled[b, h, i, d] * k_pooled[b, h, j, d]
  *   idx[b, h, i, :] = the topk key blocks j with the largest S[b, h, i, j],
  *                     ties to the lower j, written in ascending j.
@@ -100,8 +103,9 @@ bsa_status bsa_block_pool(const void* x, float* x_pooled, int B, int N, int H, i
 bsa_status bsa_block_scores_topk(const float* q_pooled, const float* k_pooled, float* scores,
                                  int32_t* idx, int B, int H, int nb, int D, int topk, void* stream);
 
-/* Step 3 (page listing: sparse_attn_cuda(q, k, v, topk_indices, block_size,
- * scale)): for every (b, h, query block i) and every row n of that block,
+/* Step 3 (same page and section, step 3: softmax attention of each query row
+ * over the tokens of its block's kept key blocks, with a given scale): for
+ * every (b, h, query block i) and every row n of that block,
  *   o[b, n, h, :] = sum_t softmax_t(scale * q[b,n,h,:] . k[b,t,h,:]) v[b,t,h,:]
  * over the tokens t of the key blocks idx[b, h, i, 0..topk).
  * q, k, v: [B, N, H, D] of dtype dt (read). idx: [B, H, nb, topk] int32 with
@@ -234,7 +238,7 @@ bsa_status bsa_forward_host(const void* q, const void* k, const void* v, void* o
                             void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---- Training: forward with the row log-sum-exp, and the backward -------
- * The page listing's step 2 keeps blocks with torch.topk, whose indices
+ * Step 2 of the "SparseFormer 注意力实现" section keeps blocks by a top-k, whose indices
  * carry no gradient, so the backward is the gradient of step 3 (the
  * attention over the kept blocks) with the index lists held fixed. Per query
  * token n and kept key token t (p = softmax weight, o = output):
@@ -301,12 +305,17 @@ bsa_status bsa_sparse_attn_bwd_gqa(const void* q, const void* k, const void* v, 
  * entry point; it only changes where the intermediates live.
  *
  * Arguments and results are those of bsa_forward minus the workspace. The
- * pooled q, pooled k and index list go to a fixed 256-byte aligned array of
- * BSA_NOALLOC_SCRATCH_BYTES in the library's device image: every GPU that
- * loads libbsa holds it until the process exits. Sizes whose workspace
- * (bsa_forward_workspace_bytes) exceeds it return BSA_ERR_WORKSPACE before
- * anything is launched. The call allocates nothing (no cudaMalloc/cudaFree).
- * The first call on each device looks up the array's device address
+ * whole bsa_forward workspace -- pooled q, pooled k, the index list and the
+ * [B, H, nb, nb] float32 block-score matrix, which is most of it (B*H*nb^2*4
+ * bytes: 64 MiB is reached at B*H*nb^2 = 2^24, e.g. 16 heads at nb = 1024) --
+ * goes to a fixed 256-byte aligned array of BSA_NOALLOC_SCRATCH_BYTES in the
+ * library's device image: every GPU that loads libbsa holds it until the
+ * process exits. Sizes whose workspace (bsa_forward_workspace_bytes) exceeds
+ * it return BSA_ERR_WORKSPACE before anything is launched. The call
+ * allocates nothing (no cudaMalloc/cudaFree).
+ * The first call on each device (and the first call after the device's
+ * context was destroyed, e.g. by cudaDeviceReset, which reloads the module
+ * and may move the array) looks up the array's device address
  * (cudaGetSymbolAddress, with that device current), so make that first call
  * before any stream capture. All calls on a device share the one array and
  * it keeps the last call's contents (nothing in it needs to start at zero):

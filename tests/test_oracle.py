@@ -286,27 +286,38 @@ def test_batch_head_permutation_and_block_relabel(oracle_mod, small_case):
     np.testing.assert_allclose(oracle_mod.o_to_bnhd(r2["o"]), o, rtol=1e-12, atol=1e-12)
 
 
-# ---------------------------------------------------------------- the page's listing, restated
+# ---------------------------------------------------------------- the definition, written out again
 
-def test_matches_restated_page_listing_in_torch(oracle_mod):
-    """The [SF] listing run in float64 torch on CPU, with the einsum applied to
-    head-major pooled tensors and the custom kernel replaced by dense attention
-    under the block mask; the random data has no exact score ties."""
+def test_matches_definition_written_out_in_numpy(oracle_mod):
+    """The three steps of page "2026 新一代卷积与 Transformer 网络架构" (section
+    "SparseFormer 注意力实现") written out independently of the C oracle: block
+    means as explicit per-block sums, the selection as a full sort of
+    (score descending, block id ascending), and each query row's softmax over
+    the tokens of its kept blocks. The random data has no exact score ties."""
     B, N, H, D, bs, ratio = 2, 96, 3, 16, 8, 0.3
-    q, k, v = (torch.from_numpy(_rand((B, N, H, D), s, bs=bs)) for s in (60, 61, 62))
+    q, k, v = (_rand((B, N, H, D), s, bs=bs).astype(np.float64) for s in (60, 61, 62))
     nb = N // bs
-    qb = q.view(B, nb, bs, H, D).mean(2).permute(0, 2, 1, 3)
-    kb = k.view(B, nb, bs, H, D).mean(2).permute(0, 2, 1, 3)
-    scores = torch.einsum("bhid,bhjd->bhij", qb, kb)
-    _, top = torch.topk(scores, k=int(ratio * nb), dim=-1)
-    mask = torch.zeros(B, H, nb, nb, dtype=torch.bool).scatter_(-1, top, True)
-    tok_mask = mask.repeat_interleave(bs, 2).repeat_interleave(bs, 3)
-    t = lambda x: x.permute(0, 2, 1, 3)
-    ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), attn_mask=tok_mask,
-                                                           scale=1.0 / math.sqrt(D))
-    r = oracle_mod.forward(q.numpy(), k.numpy(), v.numpy(), bs, ratio)
-    np.testing.assert_array_equal(r["idx"], np.sort(top.numpy(), -1))
-    np.testing.assert_allclose(oracle_mod.o_to_bnhd(r["o"]), t(ref).numpy(), rtol=1e-12, atol=1e-12)
+    kk = int(ratio * nb)
+    want_idx = np.empty((B, H, nb, kk), np.int32)
+    want_o = np.empty((B, N, H, D))
+    for b in range(B):
+        for h in range(H):
+            qbar = [sum(q[b, i * bs + t, h] for t in range(bs)) / bs for i in range(nb)]
+            kbar = [sum(k[b, j * bs + t, h] for t in range(bs)) / bs for j in range(nb)]
+            for i in range(nb):
+                score = [float(np.dot(qbar[i], kbar[j])) for j in range(nb)]
+                ranked = sorted(range(nb), key=lambda j: (-score[j], j))
+                kept = sorted(ranked[:kk])
+                want_idx[b, h, i] = kept
+                toks = [j * bs + t for j in kept for t in range(bs)]
+                for t_q in range(bs):
+                    n = i * bs + t_q
+                    logits = np.array([np.dot(q[b, n, h], k[b, t, h]) for t in toks]) / math.sqrt(D)
+                    w = np.exp(logits - logits.max())
+                    want_o[b, n, h] = sum(w[c] * v[b, t, h] for c, t in enumerate(toks)) / w.sum()
+    r = oracle_mod.forward(q, k, v, bs, ratio)
+    np.testing.assert_array_equal(r["idx"], want_idx)
+    np.testing.assert_allclose(oracle_mod.o_to_bnhd(r["o"]), want_o, rtol=1e-12, atol=1e-12)
 
 
 # ---------------------------------------------------------------- causal variant
