@@ -41,7 +41,7 @@ METRIC = "block-sparse attn fwd tokens/s & effective TFLOP/s (% roofline), 1 B20
 # DRAM read + write bytes per launch of the attention kernel from an ncu
 # capture of the kernel as it stands, per workload; null where there is none
 # (a capture of an earlier version of the kernel does not count).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {"c4": 5035535360 + 589144320}  # one launch, the current kernel
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
