@@ -256,6 +256,10 @@ bsa_status launch_topk(const float* S, int32_t* idx, int B, int H, int nb, int k
   if (nb <= 1024) {
     e = launch_pdl(bsa::block_topk_kernel, static_cast<unsigned>(grid), bsa::kSelThreads, 0, st, S, idx, rows, nb,
                    k, flags);
+  } else if (nb <= 4096) {
+    if (rows > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "top-k grid too large");
+    e = launch_pdl(bsa::block_topk_group_kernel, static_cast<unsigned>(rows), bsa::kSelGroupThreads, 0, st, S,
+                   idx, rows, nb, k, flags);
   } else {
     // long rows: each warp stages its row's keys in shared memory when they fit
     const size_t stage_bytes = static_cast<size_t>(bsa::kSelWarps) * bsa::staged_row_keys(nb) * sizeof(uint32_t);

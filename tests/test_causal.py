@@ -127,10 +127,10 @@ def test_causal_attention_with_oracle_indices(bsa, oracle_mod, ci):
         check_output(gpu_rows(o, rows, bs), o_ref, cfg.dtype)
 
 
-@pytest.mark.parametrize("nb", [40, 100, 1024, 1501])
+@pytest.mark.parametrize("nb", [40, 100, 1024, 1501, 4500])
 def test_causal_selection_on_integer_scores(bsa, oracle_mod, nb):
     """Integer-valued pooled inputs give exact scores with many ties: the
-    causal index lists must equal the oracle's bit for bit (register path,
+    causal index lists must equal the oracle's bit for bit (register paths,
     ragged rows and rows staged in shared memory)."""
     B, H, D = 1, 2, 64
     rng = np.random.default_rng(900 + nb)
