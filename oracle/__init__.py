@@ -63,6 +63,9 @@ def _load():
         lib.oracle_topk_count.argtypes = [i, d]
         lib.oracle_topk_count.restype = i
         lib.oracle_block_pool.argtypes = [P, i, i, i, i, i, i, P]
+        lib.oracle_block_pool_max.argtypes = [P, i, i, i, i, i, i, P]
+        lib.oracle_adaptive_block_size.argtypes = [ctypes.c_longlong]
+        lib.oracle_adaptive_block_size.restype = i
         lib.oracle_block_scores.argtypes = [P, P, i, i, i, i, P, i, P]
         lib.oracle_topk_row.argtypes = [P, i, i, P]
         lib.oracle_topk.argtypes = [P, ctypes.c_long, i, i, P]
@@ -112,16 +115,27 @@ def topk_count(nb: int, topk_ratio: float) -> int:
     return _load().oracle_topk_count(int(nb), float(topk_ratio))
 
 
-def block_pool(x: np.ndarray, block_size: int) -> np.ndarray:
-    """[B,N,H,D] -> block means [B,H,nb,D] in float64 ([SF] step 1)."""
+def block_pool(x: np.ndarray, block_size: int, pool: str = "mean") -> np.ndarray:
+    """[B,N,H,D] -> block means [B,H,nb,D] in float64 ([SF] step 1), or with
+    ``pool="max"`` the element-wise block maxima ([MSA] §2.2, "block-internal
+    extreme value")."""
     x, code = _as_input(x)
     B, N, H, D = x.shape
     if N % block_size:
         raise ValueError("N must be a multiple of block_size")
+    if pool not in ("mean", "max"):
+        raise ValueError("pool must be 'mean' or 'max'")
     nb = N // block_size
     out = np.empty((B, H, nb, D), np.float64)
-    _load().oracle_block_pool(_ptr(x), code, B, N, H, D, block_size, _ptr(out))
+    fn = _load().oracle_block_pool if pool == "mean" else _load().oracle_block_pool_max
+    fn(_ptr(x), code, B, N, H, D, block_size, _ptr(out))
     return out
+
+
+def adaptive_block_size(seq_len: int) -> int:
+    """Block size for an input length ([MSA] §4.2): 64 below 500,000 tokens,
+    128 below 1,000,000, else 256; -1 for a length below 1."""
+    return _load().oracle_adaptive_block_size(int(seq_len))
 
 
 def _rows(rows, B: int, H: int, nb: int):
@@ -214,19 +228,19 @@ def sparse_attn(q, k, v, idx, block_size: int, scale: float | None = None, rows=
 
 
 def forward(q, k, v, block_size: int, topk_ratio: float, rows=None, scale=None,
-            causal: bool = False, force_diag: bool = False) -> dict:
+            causal: bool = False, force_diag: bool = False, pool: str = "mean") -> dict:
     """The whole path of the [SF] listing on the oracle: pool, score, select, attend.
 
     ``rows`` (int [B,H,nrows]) restricts the scored / attended query blocks to
     a sample; pooling of k always covers every block since selection needs all
-    of them.  Returns a dict with qp, kp, scores, idx, o, k and timings."""
+    of them. ``pool`` is "mean" (the listing) or "max" (block maxima).  Returns a dict with qp, kp, scores, idx, o, k and timings."""
     t0 = time.perf_counter()
     qn, _ = _as_input(q)
     B, N, H, D = qn.shape
     nb = N // block_size
     kk = topk_count(nb, topk_ratio)
-    qp = block_pool(q, block_size)
-    kp = block_pool(k, block_size)
+    qp = block_pool(q, block_size, pool)
+    kp = block_pool(k, block_size, pool)
     S = block_scores(qp, kp, rows)
     idx = topk(S, kk, causal=causal, force_diag=force_diag, qblocks=rows)
     o = sparse_attn(q, k, v, idx, block_size, scale=scale, rows=rows, causal=causal)
@@ -309,7 +323,7 @@ def sparse_attn_gqa(q, k, v, idx, block_size: int, scale: float | None = None, r
 
 
 def forward_gqa(q, k, v, block_size: int, topk_ratio: float, rows=None, scale=None,
-                causal: bool = False, force_diag: bool = False) -> dict:
+                causal: bool = False, force_diag: bool = False, pool: str = "mean") -> dict:
     """The whole path with grouped queries. ``rows`` (int [B,Hkv,nrows]) picks
     query blocks per key/value head; every query head of the group is attended
     for those blocks. Returns qp (per head), qg (group means), kp, scores and
@@ -324,9 +338,9 @@ def forward_gqa(q, k, v, block_size: int, topk_ratio: float, rows=None, scale=No
     kk = topk_count(nb, topk_ratio)
     if rows is not None:
         _, _, rows = _rows(rows, B, Hkv, nb)
-    qp = block_pool(q, block_size)
+    qp = block_pool(q, block_size, pool)
     qg = group_pool(qp, Hkv)
-    kp = block_pool(k, block_size)
+    kp = block_pool(k, block_size, pool)
     S = block_scores(qg, kp, rows)
     idx = topk(S, kk, causal=causal, force_diag=force_diag, qblocks=rows)
     idx_q = np.repeat(idx, G, axis=1)

@@ -102,6 +102,37 @@ void oracle_block_pool(const void* x, int dtype, int B, int N, int H, int D, int
         }
 }
 
+/* Max-pooled variant ([MSA] §2.2, the comparison table: block-based methods
+ * such as MSA/MoBA score blocks by their "block-internal extreme value").
+ * Reading: the pooled vector of a block is its element-wise maximum over
+ * the block's block_size rows, for q and k alike, in place of the mean:
+ * xp[b, h, i, d] = max_{t < bs} x[b, i*bs + t, h, d]. Output [B, H, nb, D]. */
+void oracle_block_pool_max(const void* x, int dtype, int B, int N, int H, int D, int bs, double* xp) {
+  int nb = N / bs;
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int i = 0; i < nb; ++i)
+        for (int d = 0; d < D; ++d) {
+          double m = elem(x, dtype, at_bnhd(N, H, D, b, i * bs, h, d));
+          for (int t = 1; t < bs; ++t) {
+            double e = elem(x, dtype, at_bnhd(N, H, D, b, i * bs + t, h, d));
+            if (e > m) m = e;
+          }
+          xp[(((size_t)b * H + h) * nb + i) * D + d] = m;
+        }
+}
+
+/* [MSA] §4.2 (performance tuning, dynamic block selection): the block size
+ * chosen from the input length: 64 below 500,000 tokens, 128 below
+ * 1,000,000, else 256. Returns -1 for a length below 1. */
+int oracle_adaptive_block_size(long long seq_len) {
+  if (seq_len < 1) return -1;
+  if (seq_len < 500000) return 64;
+  if (seq_len < 1000000) return 128;
+  return 256;
+}
+
 /* [SF] step 1 (einsum of pooled q and pooled k, per (b, h)):
  * S[b, h, r, j] = sum_d qp[b, h, rows[b,h,r], d] * kp[b, h, j, d]
  * for the nrows query blocks listed per (b, h) in rows[B, H, nrows]

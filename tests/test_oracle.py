@@ -16,6 +16,8 @@ import numpy as np
 import pytest
 import torch
 
+import workloads as W
+
 HERE = os.path.dirname(os.path.abspath(__file__))
 
 
@@ -60,6 +62,60 @@ def test_hw1_hand_worked(oracle_mod):
     rt = oracle_mod.forward(q, kt, v, bs, g["topk_ratio"])
     np.testing.assert_array_equal(rt["kp"][0, 0, :, 0], g["tie_variant"]["k_pooled"])
     np.testing.assert_array_equal(rt["idx"][0, 0], g["tie_variant"]["idx"])
+
+
+def test_hw2_max_pool_hand_worked(oracle_mod):
+    g = json.load(open(os.path.join(HERE, "golden", "hw2_max_pool.json")))
+    shp = (g["B"], g["N"], g["H"], g["D"])
+    q, k, v = (np.array(g[n], np.float64).reshape(shp) for n in ("q", "k", "v"))
+    bs = g["block_size"]
+    r = oracle_mod.forward(q, k, v, bs, g["topk_ratio"], pool="max")
+    np.testing.assert_array_equal(r["qp"][0, 0, :, 0], g["q_pooled_max"])
+    np.testing.assert_array_equal(r["kp"][0, 0, :, 0], g["k_pooled_max"])
+    np.testing.assert_array_equal(r["scores"][0, 0], g["scores_max"])
+    np.testing.assert_array_equal(r["idx"][0, 0], g["idx_max"])
+    o = oracle_mod.o_to_bnhd(r["o"]).reshape(-1)
+    np.testing.assert_allclose(o, [_closed(e) for e in g["o_closed_form"]], rtol=1e-15, atol=0)
+    # the mean-pooled path keeps the other block in both rows
+    np.testing.assert_array_equal(oracle_mod.forward(q, k, v, bs, g["topk_ratio"])["idx"][0, 0], g["idx_mean"])
+
+
+# ---------------------------------------------------------------- max pooling, adaptive block size
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "e4m3"])
+def test_max_pool_matches_numpy_max(oracle_mod, dtype):
+    B, N, H, D, bs = 2, 96, 3, 16, 8
+    x = torch.from_numpy(_rand((B, N, H, D), 70)).to({"f32": torch.float32, "bf16": torch.bfloat16,
+                                                       "e4m3": torch.float8_e4m3fn}[dtype])
+    xa = W.to_oracle_array(x)
+    got = oracle_mod.block_pool(xa, bs, pool="max")
+    want = x.to(torch.float64).numpy().reshape(B, N // bs, bs, H, D).max(axis=2).transpose(0, 2, 1, 3)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_max_pool_brute_force_and_invariants(oracle_mod):
+    B, N, H, D, bs = 1, 24, 2, 5, 4
+    x = _rand((B, N, H, D), 71)
+    got = oracle_mod.block_pool(x, bs, pool="max")
+    for h in range(H):
+        for i in range(N // bs):
+            for d in range(D):
+                assert got[0, h, i, d] == max(x[0, i * bs + t, h, d] for t in range(bs))
+    # block_size 1 is the identity; rows permuted inside a block change nothing;
+    # a constant block pools to its row; the maximum is never below the mean
+    np.testing.assert_array_equal(oracle_mod.block_pool(x, 1, pool="max")[0].transpose(1, 0, 2), x[0])
+    perm = np.concatenate([i * bs + np.random.default_rng(i).permutation(bs) for i in range(N // bs)])
+    np.testing.assert_array_equal(oracle_mod.block_pool(x[:, perm], bs, pool="max"), got)
+    c = np.repeat(x[:, ::bs], bs, axis=1)
+    np.testing.assert_array_equal(oracle_mod.block_pool(c, bs, pool="max"), oracle_mod.block_pool(c, bs))
+    assert np.all(got >= oracle_mod.block_pool(x, bs) - 1e-15)
+
+
+@pytest.mark.parametrize("n,want", [(1, 64), (8192, 64), (499_999, 64), (500_000, 128), (999_999, 128),
+                                    (1_000_000, 256), (1 << 40, 256), (0, -1), (-5, -1)])
+def test_adaptive_block_size_thresholds(oracle_mod, n, want):
+    # page "从M2.7到M3" §4.2: 64 below 500,000 tokens, 128 below 1,000,000, else 256
+    assert oracle_mod.adaptive_block_size(n) == want
 
 
 # ---------------------------------------------------------------- k = int(ratio * nb)
