@@ -350,6 +350,46 @@ def forward_gqa(q, k, v, block_size: int, topk_ratio: float, rows=None, scale=No
             "o": o, "k": kk}
 
 
+# ---------------------------------------------------------------- global heads
+# Reading ("从M2.7到M3" §5.3: add global attention heads, e.g. one global head in
+# every four): query head h is global when h % period == 0 (the first head of
+# every run of `period` heads); a global head attends to every key block (with
+# the causal flag: every block j <= i, token-masked as usual), the other heads
+# to their selected blocks.
+
+def global_head_rows(idx_q: np.ndarray, nb: int, period: int, causal: bool = False, rows=None) -> np.ndarray:
+    """Per-query-head index rows with global heads: ``idx_q`` [B,H,nrows,k]
+    (the selection of each query head's rows) widened to nb entries; rows of
+    global heads list every key block (causal: blocks 0..i, then -1), the
+    others their k blocks followed by -1. ``rows`` [B,H,nrows] gives the query
+    block of each row (None: all nb blocks in order)."""
+    B, H, nrows, k = idx_q.shape
+    out = np.full((B, H, nrows, nb), -1, np.int32)
+    out[..., :k] = idx_q
+    qb = np.broadcast_to(np.arange(nrows), (B, H, nrows)) if rows is None else np.broadcast_to(rows, (B, H, nrows))
+    for h in range(0, H, period):
+        for b in range(B):
+            for r in range(nrows):
+                n = qb[b, h, r] + 1 if causal else nb
+                out[b, h, r, :] = -1
+                out[b, h, r, :n] = np.arange(n)
+    return out
+
+
+def forward_global(q, k, v, block_size: int, topk_ratio: float, period: int, causal: bool = False,
+                   force_diag: bool = False, pool: str = "mean", rows=None) -> dict:
+    """forward_gqa with global heads every ``period`` query heads. Returns the
+    forward_gqa dict with idx_q replaced by the widened per-query-head rows
+    and o recomputed over them."""
+    r = forward_gqa(q, k, v, block_size, topk_ratio, rows=rows, causal=causal, force_diag=force_diag, pool=pool)
+    qn, _ = _as_input(q)
+    nb = qn.shape[1] // block_size
+    idx_w = global_head_rows(r["idx_q"], nb, period, causal, r["rows_q"])
+    r["idx_q"] = idx_w
+    r["o"] = sparse_attn_gqa(q, k, v, idx_w, block_size, rows=r["rows_q"], causal=causal)
+    return r
+
+
 def o_to_bnhd(o: np.ndarray) -> np.ndarray:
     """Reorder an all-rows oracle output [B,H,nb,bs,D] to [B,N,H,D]."""
     B, H, nb, bs, D = o.shape

@@ -118,6 +118,39 @@ def test_adaptive_block_size_thresholds(oracle_mod, n, want):
     assert oracle_mod.adaptive_block_size(n) == want
 
 
+# ---------------------------------------------------------------- global heads
+# Reading ("从M2.7到M3" §5.3): query head h is global when h % period == 0 and
+# attends to every key block; the other heads keep their selection.
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("H,Hkv,period", [(4, 4, 4), (4, 2, 2), (3, 3, 1), (6, 3, 4)])
+def test_global_heads_are_dense_attention(oracle_mod, causal, H, Hkv, period):
+    B, N, D, bs, ratio = 2, 96, 8, 8, 0.25
+    q = _rand((B, N, H, D), 80, bs=bs)
+    k = _rand((B, N, Hkv, D), 81, bs=bs)
+    v = _rand((B, N, Hkv, D), 82, offsets=False)
+    r = oracle_mod.forward_global(q, k, v, bs, ratio, period, causal=causal)
+    o = oracle_mod.o_to_bnhd(r["o"])
+    plain = oracle_mod.o_to_bnhd(oracle_mod.forward_gqa(q, k, v, bs, ratio, causal=causal)["o"])
+    G = H // Hkv
+    t = lambda x: torch.from_numpy(x).permute(0, 2, 1, 3)
+    kr, vr = np.repeat(k, G, axis=2), np.repeat(v, G, axis=2)
+    dense = torch.nn.functional.scaled_dot_product_attention(t(q), t(kr), t(vr), is_causal=causal,
+                                                             scale=1.0 / math.sqrt(D)).permute(0, 2, 1, 3).numpy()
+    for h in range(H):
+        want = dense[:, :, h] if h % period == 0 else plain[:, :, h]
+        np.testing.assert_allclose(o[:, :, h], want, rtol=1e-12, atol=1e-12)
+
+
+def test_global_head_rows_layout(oracle_mod):
+    idx = np.array([[[[1], [0], [2]], [[2], [2], [0]]]], np.int32)  # B=1, H=2, nb=3, k=1
+    w = oracle_mod.global_head_rows(idx, 3, 2, causal=True)
+    np.testing.assert_array_equal(w[0, 0], [[0, -1, -1], [0, 1, -1], [0, 1, 2]])
+    np.testing.assert_array_equal(w[0, 1], [[2, -1, -1], [2, -1, -1], [0, -1, -1]])
+    w = oracle_mod.global_head_rows(idx, 3, 2)
+    np.testing.assert_array_equal(w[0, 0], [[0, 1, 2]] * 3)
+
+
 # ---------------------------------------------------------------- k = int(ratio * nb)
 
 @pytest.mark.parametrize("nb,ratio,want", [
