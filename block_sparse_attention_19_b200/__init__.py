@@ -8,7 +8,8 @@ raises.
 
 Functions carry the C names:
 
-* ``bsa_block_pool(x, block_size)``                -> pooled [B, H, nb, D] float32
+* ``bsa_block_pool(x, block_size, flags=0)``       -> pooled [B, H, nb, D] float32
+  (block means, or block maxima with BSA_FLAG_MAX_POOL)
 * ``bsa_block_scores_topk(q_pooled, k_pooled, topk, scores=False)`` -> idx (, S)
 * ``bsa_sparse_attn_fwd(q, k, v, idx, block_size, scale=None, flags=0)`` -> o
 * ``bsa_forward(q, k, v, block_size, topk_ratio, workspace=None, flags=0)`` -> o
@@ -18,14 +19,15 @@ Functions carry the C names:
   device allocation (a fixed scratch in the library)
 * ``bsa_sparse_attn_fwd_train(q, k, v, idx, block_size)`` -> (o, lse) and
   ``bsa_sparse_attn_bwd(q, k, v, o, do, idx, lse, block_size)`` -> (dq, dk, dv)
+* ``bsa_adaptive_block_size(seq_len)`` -> 64, 128 or 256
 * ``bsa_topk_count``, ``bsa_forward_workspace_bytes``,
   ``bsa_forward_host_workspace_bytes``, ``workspace_views``, ``bsa_device_error``
 
 q, o are [B, N, H, D]; k, v are [B, N, H_kv, D] with H a multiple of H_kv
 (grouped queries; H_kv = H otherwise), contiguous, on one CUDA device
 (except for bsa_forward_host). Inputs are float32, bfloat16 or
-float8_e4m3fn (e4m3 gives a bfloat16 o). ``flags`` takes BSA_FLAG_CAUSAL and
-BSA_FLAG_FORCE_DIAG.
+float8_e4m3fn (e4m3 gives a bfloat16 o). ``flags`` takes BSA_FLAG_CAUSAL,
+BSA_FLAG_FORCE_DIAG, BSA_FLAG_MAX_POOL and BSA_GLOBAL_HEAD_PERIOD(p).
 """
 from __future__ import annotations
 
@@ -50,10 +52,19 @@ EXPORTED = ("bsa_topk_count", "bsa_forward_workspace_bytes", "bsa_block_pool",
             "bsa_forward_gqa_workspace_bytes", "bsa_block_scores_topk_gqa", "bsa_sparse_attn_fwd_gqa",
             "bsa_forward_gqa", "bsa_sparse_attn_fwd_train", "bsa_sparse_attn_bwd_workspace_bytes",
             "bsa_sparse_attn_bwd", "bsa_forward_host_workspace_bytes", "bsa_forward_host",
-            "bsa_sparse_attn_fwd_train_gqa", "bsa_sparse_attn_bwd_gqa_workspace_bytes", "bsa_sparse_attn_bwd_gqa")
+            "bsa_sparse_attn_fwd_train_gqa", "bsa_sparse_attn_bwd_gqa_workspace_bytes", "bsa_sparse_attn_bwd_gqa",
+            "bsa_adaptive_block_size", "bsa_block_pool_ex")
 
 #: variant flags of the *_ex entry points (include/bsa.h)
-BSA_FLAG_CAUSAL, BSA_FLAG_FORCE_DIAG = 1, 2
+BSA_FLAG_CAUSAL, BSA_FLAG_FORCE_DIAG, BSA_FLAG_MAX_POOL = 1, 2, 4
+
+
+def BSA_GLOBAL_HEAD_PERIOD(p: int) -> int:
+    """Flag bits for global heads every p query heads (heads h with h % p == 0
+    attend to every key block); p in 1..255."""
+    if not 1 <= p <= 255:
+        raise ValueError("the global-head period must lie in 1..255")
+    return (p & 0xFF) << 8
 
 
 class BsaError(RuntimeError):
@@ -95,6 +106,8 @@ def _load() -> ctypes.CDLL:
         "bsa_sparse_attn_bwd_gqa_workspace_bytes": ([I, I, I, I, I, I], Z),
         "bsa_sparse_attn_bwd_gqa": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, U, P, Z, P], I),
         "bsa_forward_host": ([P, P, P, P, I, I, I, I, I, I, D, I, U, P, Z, P], I),
+        "bsa_adaptive_block_size": ([ctypes.c_longlong], I),
+        "bsa_block_pool_ex": ([P, P, I, I, I, I, I, I, U, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -184,7 +197,12 @@ def bsa_forward_workspace_bytes(B: int, N: int, H: int, D: int, block_size: int,
     return lib.bsa_forward_gqa_workspace_bytes(B, N, H, H_kv, D, block_size, float(topk_ratio))
 
 
-def bsa_block_pool(x: torch.Tensor, block_size: int, out: torch.Tensor | None = None) -> torch.Tensor:
+def bsa_adaptive_block_size(seq_len: int) -> int:
+    return lib.bsa_adaptive_block_size(int(seq_len))
+
+
+def bsa_block_pool(x: torch.Tensor, block_size: int, out: torch.Tensor | None = None,
+                   flags: int = 0) -> torch.Tensor:
     if x.dim() != 4:
         raise ValueError("x must be [B, N, H, D]")
     B, N, H, D = x.shape
@@ -193,7 +211,7 @@ def bsa_block_pool(x: torch.Tensor, block_size: int, out: torch.Tensor | None = 
     _dev(x, "x")
     if out is None:
         out = torch.empty((B, H, N // block_size, D), device=x.device, dtype=torch.float32)
-    _check(lib.bsa_block_pool(_p(x), _p(out), B, N, H, D, block_size, _dtype_code(x), _stream(x)))
+    _check(lib.bsa_block_pool_ex(_p(x), _p(out), B, N, H, D, block_size, _dtype_code(x), flags, _stream(x)))
     return out
 
 

@@ -34,13 +34,14 @@ struct SimtSmem {
   float p[4][kSimtKeys];      // per-warp probabilities of the current row
 };
 
-// grid.x = B * H * nb * (bs / kSimtRows)
+// grid.x = B * H * nb * (bs / kSimtRows). gperiod > 0: query heads h with
+// h % gperiod == 0 are global heads (every key block, 0..i when causal).
 template <int D>
 __global__ void __launch_bounds__(kSimtThreads)
     sparse_attn_simt_kernel(const float* __restrict__ q, const float* __restrict__ kmat,
                             const float* __restrict__ v, const int32_t* __restrict__ idx,
                             float* __restrict__ o, int N, int H, int Hkv, int bs, int k, float scale,
-                            unsigned flags) {
+                            unsigned flags, int gperiod) {
   pdl_launch_dependents();
   pdl_wait();
   extern __shared__ __align__(16) unsigned char simt_raw[];
@@ -83,8 +84,11 @@ __global__ void __launch_bounds__(kSimtThreads)
   const int32_t* sel = idx + ((b * Hkv + g) * static_cast<long>(nb) + i) * k;
   const int tiles_per_block = bs / kSimtKeys;
   const bool causal = (flags & kFlagCausal) != 0;
-  for (int s = 0; s < k; ++s) {
-    int blk = sel[s];
+  // a global head (h % gperiod == 0) attends to every block, 0..i when causal
+  const bool dense = gperiod > 0 && h % gperiod == 0;
+  const int nsel = dense ? (causal ? i + 1 : nb) : k;
+  for (int s = 0; s < nsel; ++s) {
+    int blk = dense ? s : sel[s];
     if (blk < 0) {
       if (s > 0) break;  // the row's valid entries end here (a row of only -1 reads block 0)
       blk = 0;

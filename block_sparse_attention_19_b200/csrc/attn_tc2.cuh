@@ -96,14 +96,24 @@ struct Tc2Barriers {
 };
 static_assert(sizeof(Tc2Barriers) <= 512, "barrier area");
 
+// Key block of entry t of an index row; a global head has no index row
+// (sel == nullptr) and walks every block in order.
+__device__ __forceinline__ int sel_block(const int32_t* sel, int t, int nb) {
+  return sel ? clamp_block(__ldg(sel + t), nb) : t;
+}
+
+// Valid entries of an index row; for a global head (sel == nullptr) every
+// block, or with the causal mask the blocks 0..i of query block i.
+template <bool kCausal>
+__device__ __forceinline__ int sel_valid(const int32_t* sel, int k, int i, int nb) {
+  return sel ? index_row_valid(sel, k) : (kCausal ? i + 1 : nb);
+}
+
 // Token row where 64-row half `hf` of stream `x`'s key tile t starts.
 __device__ __forceinline__ int tc2_key_row(const int32_t* sel_a, const int32_t* sel_b, int x,
                                            int t, int hf, int bs, int nb) {
-  if (bs == 128) {
-    const int32_t* sel = x == 0 ? sel_a : sel_b;
-    return clamp_block(__ldg(sel + t), nb) * 128 + hf * 64;
-  }
-  return clamp_block(__ldg(sel_a + t / 2), nb) * 256 + (t % 2) * 128 + hf * 64;  // bs == 256
+  if (bs == 128) return sel_block(x == 0 ? sel_a : sel_b, t, nb) * 128 + hf * 64;
+  return sel_block(sel_a, t / 2, nb) * 256 + (t % 2) * 128 + hf * 64;  // bs == 256
 }
 
 // Causal mask on 32 scores of a row: column c0 + e becomes -inf when it is
@@ -187,13 +197,17 @@ __device__ __forceinline__ void tc2_make_p32(const uint32_t (&sv)[32], float m, 
 // thread in use).
 // kCausal: key tokens after the query token are masked (kFlagCausal).
 // lse (optional, [B, H, N] float32): ln sum_t exp(scale q_n . k_t) per row.
+// gperiod > 0: query heads h with h % gperiod == 0 are global heads, which
+// read no index row and attend to every key block (blocks 0..i when causal);
+// query heads are then never paired in a CTA.
 template <int D, bool kCausal, bool kF8 = false, bool kStack = false>
 __global__ void __launch_bounds__(kTc2Threads, 1)
     sparse_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v,
                            const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ o, int N,
-                           int H, int Hkv, int bs, int k, float scale_log2, float* __restrict__ lse) {
+                           int H, int Hkv, int bs, int k, float scale_log2, float* __restrict__ lse,
+                           int gperiod) {
   using L = Tc2Layout<D, kF8>;
   // MMA steps: K = 32 bytes of the row per instruction (16 bf16 or 32 e4m3)
   constexpr int kStepsS = D * L::kElem / 32;
@@ -221,7 +235,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
   // In the first two the streams read the same key tiles (one selection),
   // so each K and V tile is loaded once for both.
   const int G = H / Hkv;
-  const bool head_pairs = !kStack && bs == 128 && (G % 2) == 0;
+  const bool head_pairs = !kStack && bs == 128 && (G % 2) == 0 && gperiod == 0;
   const bool shared_kv = !kStack && (bs == 256 || head_pairs);
   long u = blockIdx.x;
   int iA, b, qh[2];
@@ -252,15 +266,19 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
   const int row0[2] = {iA * bs, kStack ? (iA + 2) * 64
                                        : (bs == 256 ? iA * bs + 128 : (head_pairs ? iA * bs : (iA + 1) * bs))};
   const long bg = static_cast<long>(b) * Hkv + g;
-  const int32_t* sel_a = idx + (bg * nb + iA) * k;
-  const int32_t* sel_b = shared_kv ? sel_a : idx + (bg * nb + (iA + 1 < nb ? iA + 1 : iA)) * k;
+  // both streams belong to one query head whenever global heads exist
+  const bool dense = gperiod > 0 && qh[0] % gperiod == 0;
+  const int iB = iA + 1 < nb ? iA + 1 : iA;
+  const int32_t* sel_a = dense ? nullptr : idx + (bg * nb + iA) * k;
+  const int32_t* sel_b = shared_kv ? sel_a : (dense ? nullptr : idx + (bg * nb + iB) * k);
   // kStack: index rows of query blocks iA + q (an absent second block of a
   // stream takes its first block's row, whose rows are then not written)
   const int32_t* sel4[4];
+  int blk4[4];
   if (kStack)
     for (int q = 0; q < 4; ++q) {
-      const int blk = iA + q < nb ? iA + q : min(iA + (q & 2), nb - 1);
-      sel4[q] = idx + (bg * nb + blk) * k;
+      blk4[q] = iA + q < nb ? iA + q : min(iA + (q & 2), nb - 1);
+      sel4[q] = dense ? nullptr : idx + (bg * nb + blk4[q]) * k;
     }
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -289,12 +307,13 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     // so that a row of only -1 still reads block 0 instead of nothing)
     if (kStack) {
       // a stream walks as many tiles as the longer of its two rows
-      for (int q = 0; q < 4; ++q) bar.valid[q] = q / 2 < nstreams ? max(index_row_valid(sel4[q], k), 1) : 0;
+      for (int q = 0; q < 4; ++q)
+        bar.valid[q] = q / 2 < nstreams ? max(sel_valid<kCausal>(sel4[q], k, blk4[q], nb), 1) : 0;
       bar.tiles[0] = max(bar.valid[0], bar.valid[1]);
       bar.tiles[1] = max(bar.valid[2], bar.valid[3]);
     } else {
-      const int ta = max(index_row_valid(sel_a, k), 1);
-      const int tb = nstreams == 2 && !shared_kv ? max(index_row_valid(sel_b, k), 1) : 0;
+      const int ta = max(sel_valid<kCausal>(sel_a, k, iA, nb), 1);
+      const int tb = nstreams == 2 && !shared_kv ? max(sel_valid<kCausal>(sel_b, k, iB, nb), 1) : 0;
       const int tpb = bs == 256 ? 2 : 1;  // key tiles per block
       bar.tiles[0] = tpb * ta;
       bar.tiles[1] = shared_kv ? tpb * ta : tb;
@@ -356,7 +375,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         const int t = shared_kv ? n : (n < 2 * Tmin ? (n >> 1) : Tmin + (n - 2 * Tmin));
         int r[2];
         for (int hf = 0; hf < 2; ++hf)
-          r[hf] = kStack ? clamp_block(__ldg(sel4[2 * x + hf] + t), nb) * 64  // -1 entries load block 0, unused
+          r[hf] = kStack ? sel_block(sel4[2 * x + hf], t, nb) * 64  // -1 entries load block 0, unused
                          : tc2_key_row(sel_a, sel_b, x, t, hf, bs, nb);
         if (n >= S) ok = mbar_wait(&empty[s], (use - 1) & 1, abort_flag, is_k ? 111 : 112);
         if (!ok) break;
@@ -509,7 +528,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
           tmem_wait_ld();
           if (kCausal) {
             // keys c > lim of the block follow the thread's query token
-            const int lim = row0[x] + row - clamp_block(__ldg(sel4[2 * x + hf] + j), nb) * 64;
+            const int lim = row0[x] + row - sel_block(sel4[2 * x + hf], j, nb) * 64;
             if (lim < 63) {
               tc2_mask_after(s0, 0, lim);
               tc2_mask_after(s1, 32, lim);

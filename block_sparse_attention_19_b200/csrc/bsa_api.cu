@@ -67,8 +67,11 @@ bsa_status check_dims(int B, int N, int H, int D, int block_size) {
 static_assert(BSA_FLAG_CAUSAL == bsa::kFlagCausal && BSA_FLAG_FORCE_DIAG == bsa::kFlagForceDiag,
               "flag values of the header and the kernels");
 
+// The global-head period carried in bits 8-15 of the flags (0: none).
+int global_period(unsigned flags) { return static_cast<int>((flags >> 8) & 0xFFu); }
+
 bsa_status check_flags(unsigned flags) {
-  if (flags & ~(BSA_FLAG_CAUSAL | BSA_FLAG_FORCE_DIAG))
+  if (flags & ~(BSA_FLAG_CAUSAL | BSA_FLAG_FORCE_DIAG | BSA_FLAG_MAX_POOL | BSA_GLOBAL_HEAD_PERIOD(255)))
     return fail(BSA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
   if ((flags & BSA_FLAG_FORCE_DIAG) && !(flags & BSA_FLAG_CAUSAL))
     return fail(BSA_ERR_INVALID_ARG, "BSA_FLAG_FORCE_DIAG needs BSA_FLAG_CAUSAL");
@@ -164,7 +167,7 @@ cudaError_t launch_pdl(void (*kernel)(Params...), unsigned grid, unsigned block,
 }
 
 bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int ntasks, int B,
-                       int N, int H, int D, int bs, bsa_dtype dt, cudaStream_t st) {
+                       int N, int H, int D, int bs, bsa_dtype dt, unsigned flags, cudaStream_t st) {
   const int V = dt == BSA_F32 ? 4 : (dt == BSA_E4M3 ? 16 : 8);  // elements per 16 bytes
   const int C = H * D / V;
   const int cw = bsa::pool_column_group(C);
@@ -173,13 +176,19 @@ bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int
   bsa::PoolTask t0{x0, p0}, t1{x1 ? x1 : x0, p1 ? p1 : p0};
   const unsigned g = static_cast<unsigned>(grid);
   const unsigned threads = static_cast<unsigned>(bsa::kPoolRowGroups * cw);
+  const bool maxp = (flags & BSA_FLAG_MAX_POOL) != 0;
   cudaError_t e;
   if (dt == BSA_F32)
-    e = launch_pdl(bsa::block_pool_kernel<float>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw);
+    e = maxp ? launch_pdl(bsa::block_pool_kernel<float, true>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw)
+             : launch_pdl(bsa::block_pool_kernel<float>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw);
   else if (dt == BSA_E4M3)
-    e = launch_pdl(bsa::block_pool_kernel<__nv_fp8_e4m3>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw);
+    e = maxp ? launch_pdl(bsa::block_pool_kernel<__nv_fp8_e4m3, true>, g, threads, 0, st, t0, t1, B, N, H, D, bs,
+                          cw)
+             : launch_pdl(bsa::block_pool_kernel<__nv_fp8_e4m3>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw);
   else
-    e = launch_pdl(bsa::block_pool_kernel<__nv_bfloat16>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw);
+    e = maxp ? launch_pdl(bsa::block_pool_kernel<__nv_bfloat16, true>, g, threads, 0, st, t0, t1, B, N, H, D, bs,
+                          cw)
+             : launch_pdl(bsa::block_pool_kernel<__nv_bfloat16>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_pool_kernel launch");
 }
@@ -303,7 +312,7 @@ bsa_status launch_attn_simt(const float* q, const float* k, const float* v, cons
   const long grid = static_cast<long>(B) * H * (N / bs) * (bs / bsa::kSimtRows);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   cudaError_t e = launch_pdl(bsa::sparse_attn_simt_kernel<D>, static_cast<unsigned>(grid), bsa::kSimtThreads, smem,
-                             st, q, k, v, idx, o, N, H, Hkv, bs, kk, scale, flags);
+                             st, q, k, v, idx, o, N, H, Hkv, bs, kk, scale, flags, global_period(flags));
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_simt_kernel launch");
 }
@@ -311,7 +320,7 @@ bsa_status launch_attn_simt(const float* q, const float* k, const float* v, cons
 template <int D, bool kCausal, bool kF8, bool kStack>
 bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                               int B, int N, int H, int Hkv, int bs, int kk, float scale,
-                              float* lse, cudaStream_t st) {
+                              float* lse, int gperiod, cudaStream_t st) {
   using L = bsa::Tc2Layout<D, kF8>;
   CUtensorMap mq, mk, mv;
   bsa_status s;
@@ -340,7 +349,7 @@ bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const
   // the kernel's CTA layouts: halves of a 256-block; two query heads of a
   // group on one block (an even group size); two blocks of one head
   // block_size 64: two streams of two stacked query blocks each
-  const bool head_pairs = bs == 128 && ((H / Hkv) % 2) == 0;
+  const bool head_pairs = bs == 128 && ((H / Hkv) % 2) == 0 && gperiod == 0;
   const long grid = kStack       ? static_cast<long>(B) * H * ((nb + 3) / 4)
                     : head_pairs ? static_cast<long>(B) * (H / 2) * nb
                                  : static_cast<long>(B) * H * (bs == 256 ? nb : (nb + 1) / 2);
@@ -348,7 +357,7 @@ bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const
   const float scale_log2 = scale * 1.4426950408889634f;
   cudaError_t e = launch_pdl(bsa::sparse_attn_tc2_kernel<D, kCausal, kF8, kStack>, static_cast<unsigned>(grid),
                              bsa::kTc2Threads, L::kBytes, st, mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H,
-                             Hkv, bs, kk, scale_log2, lse);
+                             Hkv, bs, kk, scale_log2, lse, gperiod);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc2_kernel launch");
 }
@@ -357,9 +366,10 @@ template <int D, bool kF8 = false, bool kStack = false>
 bsa_status launch_attn_tc2(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                            int B, int N, int H, int Hkv, int bs, int kk, float scale, unsigned flags,
                            float* lse, cudaStream_t st) {
+  const int gp = global_period(flags);
   return (flags & BSA_FLAG_CAUSAL)
-             ? launch_attn_tc2_as<D, true, kF8, kStack>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, st)
-             : launch_attn_tc2_as<D, false, kF8, kStack>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, st);
+             ? launch_attn_tc2_as<D, true, kF8, kStack>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, gp, st)
+             : launch_attn_tc2_as<D, false, kF8, kStack>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, gp, st);
 }
 
 bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
@@ -529,18 +539,31 @@ const char* bsa_status_string(bsa_status s) {
 
 const char* bsa_last_error_detail(void) { return g_detail; }
 
-bsa_status bsa_block_pool(const void* x, float* x_pooled, int B, int N, int H, int D,
-                          int block_size, bsa_dtype dt, void* stream) {
+int bsa_adaptive_block_size(long long seq_len) {
+  if (seq_len < 1) return -1;
+  if (seq_len < 500000) return 64;
+  if (seq_len < 1000000) return 128;
+  return 256;
+}
+
+bsa_status bsa_block_pool_ex(const void* x, float* x_pooled, int B, int N, int H, int D, int block_size,
+                             bsa_dtype dt, unsigned flags, void* stream) {
   bsa_status s;
+  if ((s = check_flags(flags)) != BSA_OK) return s;
   if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
   if ((s = check_dtype(dt)) != BSA_OK) return s;
   if (!x || !x_pooled) return fail(BSA_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(x) || !aligned16(x_pooled)) return fail(BSA_ERR_MISALIGNED, "x or x_pooled");
   if ((s = check_device()) != BSA_OK) return s;
-  if ((s = launch_pool(x, x_pooled, nullptr, nullptr, 1, B, N, H, D, block_size, dt,
+  if ((s = launch_pool(x, x_pooled, nullptr, nullptr, 1, B, N, H, D, block_size, dt, flags,
                        static_cast<cudaStream_t>(stream))) != BSA_OK)
     return s;
   return ok();
+}
+
+bsa_status bsa_block_pool(const void* x, float* x_pooled, int B, int N, int H, int D,
+                          int block_size, bsa_dtype dt, void* stream) {
+  return bsa_block_pool_ex(x, x_pooled, B, N, H, D, block_size, dt, 0u, stream);
 }
 
 bsa_status bsa_block_scores_topk_gqa(const float* q_pooled, const float* k_pooled, float* scores,
@@ -635,10 +658,10 @@ bsa_status bsa_forward_gqa(const void* q, const void* k, const void* v, void* o,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   if (H == Hkv) {
-    if ((s = launch_pool(q, w.qp, k, w.kp, 2, B, N, H, D, block_size, dt, st)) != BSA_OK) return s;
+    if ((s = launch_pool(q, w.qp, k, w.kp, 2, B, N, H, D, block_size, dt, flags, st)) != BSA_OK) return s;
   } else {
-    if ((s = launch_pool(q, w.qp, nullptr, nullptr, 1, B, N, H, D, block_size, dt, st)) != BSA_OK) return s;
-    if ((s = launch_pool(k, w.kp, nullptr, nullptr, 1, B, N, Hkv, D, block_size, dt, st)) != BSA_OK) return s;
+    if ((s = launch_pool(q, w.qp, nullptr, nullptr, 1, B, N, H, D, block_size, dt, flags, st)) != BSA_OK) return s;
+    if ((s = launch_pool(k, w.kp, nullptr, nullptr, 1, B, N, Hkv, D, block_size, dt, flags, st)) != BSA_OK) return s;
   }
   if ((s = launch_select(w.qp, w.kp, w.scores, w.idx, B, H, Hkv, nb, D, kk, flags, st)) != BSA_OK) return s;
   if ((s = launch_attn(q, k, v, w.idx, o, B, N, H, Hkv, D, block_size, kk, scale, dt, flags, st)) != BSA_OK)
@@ -670,6 +693,7 @@ bsa_status check_train(int B, int N, int H, int Hkv, int D, int block_size, int 
   if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
   if ((s = check_heads(H, Hkv)) != BSA_OK) return s;
   if (dt != BSA_BF16) return fail(BSA_ERR_UNSUPPORTED, "training entry points take bf16");
+  if (global_period(flags) != 0) return fail(BSA_ERR_UNSUPPORTED, "training entry points have no global heads");
   if (block_size == 64) return fail(BSA_ERR_UNSUPPORTED, "training entry points need block_size 128 or 256");
   const int nb = N / block_size;
   if (kk < 1 || kk > nb) return fail(BSA_ERR_INVALID_ARG, "k=%d outside [1, nb=%d]", kk, nb);

@@ -1,9 +1,13 @@
 // pool.cuh -- step 1a: block mean-pooling of q and k.
 //
 // Page "2026 新一代卷积与 Transformer 网络架构" (qqiyuan.cn), section
-// "SparseFormer 注意力实现", step 1: q.view(B, nb, bs, H, D).mean(2), and the
-// same for k. Output layout here is head-major [B, H, nb, D] float32 so that
-// each (b, h) score matrix reads contiguous rows.
+// "SparseFormer 注意力实现", step 1: the mean over each block of block_size
+// tokens, per batch entry and head, of q and of k. Output layout here is
+// head-major [B, H, nb, D] float32 so that each (b, h) score matrix reads
+// contiguous rows. With kMax the pooled vector is the element-wise maximum
+// over the block's rows instead (page "从M2.7到M3：多模态模型稀疏注意力架构设计与实现全解析"
+// §2.2: block-based methods score blocks by their block-internal extreme
+// value); the maximum of stored values is exact.
 //
 // HBM-bound: every element of q and k is read exactly once with 16-byte
 // vector loads; the block's rows for all heads are contiguous in memory
@@ -29,27 +33,36 @@ struct PoolTask {
   float* xp;      // [B, H, nb, D]
 };
 
+// Accumulation of one element: a sum (mean pooling) or a maximum.
+template <bool kMax>
+__device__ __forceinline__ void pool_acc(float& a, float x) {
+  if constexpr (kMax) a = fmaxf(a, x);
+  else a += x;
+}
+
 template <typename T>
-struct Vec16;  // 16 bytes of T, converted to floats
+struct Vec16;  // 16 bytes of T, converted to floats and accumulated
 template <>
 struct Vec16<float> {
   static constexpr int kN = 4;
+  template <bool kMax>
   __device__ __forceinline__ static void add(float* acc, const uint4& u) {
-    acc[0] += __uint_as_float(u.x);
-    acc[1] += __uint_as_float(u.y);
-    acc[2] += __uint_as_float(u.z);
-    acc[3] += __uint_as_float(u.w);
+    pool_acc<kMax>(acc[0], __uint_as_float(u.x));
+    pool_acc<kMax>(acc[1], __uint_as_float(u.y));
+    pool_acc<kMax>(acc[2], __uint_as_float(u.z));
+    pool_acc<kMax>(acc[3], __uint_as_float(u.w));
   }
 };
 template <>
 struct Vec16<__nv_bfloat16> {
   static constexpr int kN = 8;
+  template <bool kMax>
   __device__ __forceinline__ static void add(float* acc, const uint4& u) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      acc[2 * t] += __uint_as_float(w[t] << 16);
-      acc[2 * t + 1] += __uint_as_float(w[t] & 0xFFFF0000u);
+      pool_acc<kMax>(acc[2 * t], __uint_as_float(w[t] << 16));
+      pool_acc<kMax>(acc[2 * t + 1], __uint_as_float(w[t] & 0xFFFF0000u));
     }
   }
 };
@@ -57,6 +70,7 @@ struct Vec16<__nv_bfloat16> {
 template <>
 struct Vec16<__nv_fp8_e4m3> {
   static constexpr int kN = 16;
+  template <bool kMax>
   __device__ __forceinline__ static void add(float* acc, const uint4& u) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -64,10 +78,10 @@ struct Vec16<__nv_fp8_e4m3> {
       __nv_fp8x4_e4m3 x;
       x.__x = w[t];
       const float4 f = static_cast<float4>(x);  // exact: byte 0 -> .x
-      acc[4 * t] += f.x;
-      acc[4 * t + 1] += f.y;
-      acc[4 * t + 2] += f.z;
-      acc[4 * t + 3] += f.w;
+      pool_acc<kMax>(acc[4 * t], f.x);
+      pool_acc<kMax>(acc[4 * t + 1], f.y);
+      pool_acc<kMax>(acc[4 * t + 2], f.z);
+      pool_acc<kMax>(acc[4 * t + 3], f.w);
     }
   }
 };
@@ -84,7 +98,7 @@ inline int pool_column_group(int C) {
 // CTA reduces bs rows of one group of cw 16-byte columns of one block; row r
 // goes to row group r % kPoolRowGroups, and the groups' partial sums are
 // added in group order.
-template <typename T>
+template <typename T, bool kMax = false>
 __global__ void __launch_bounds__(kPoolThreads)
     block_pool_kernel(PoolTask t0, PoolTask t1, int B, int N, int H, int D, int bs, int cw) {
   pdl_launch_dependents();
@@ -111,7 +125,7 @@ __global__ void __launch_bounds__(kPoolThreads)
 
   float acc[V];
 #pragma unroll
-  for (int e = 0; e < V; ++e) acc[e] = 0.f;
+  for (int e = 0; e < V; ++e) acc[e] = kMax ? -INFINITY : 0.f;
 
   if (rg < G) {
     const uint4* base = reinterpret_cast<const uint4*>(task.x) +
@@ -123,12 +137,12 @@ __global__ void __launch_bounds__(kPoolThreads)
       uint4 u1 = __ldg(base + static_cast<size_t>(r + G) * C);
       uint4 u2 = __ldg(base + static_cast<size_t>(r + 2 * G) * C);
       uint4 u3 = __ldg(base + static_cast<size_t>(r + 3 * G) * C);
-      Vec16<T>::add(acc, u0);
-      Vec16<T>::add(acc, u1);
-      Vec16<T>::add(acc, u2);
-      Vec16<T>::add(acc, u3);
+      Vec16<T>::template add<kMax>(acc, u0);
+      Vec16<T>::template add<kMax>(acc, u1);
+      Vec16<T>::template add<kMax>(acc, u2);
+      Vec16<T>::template add<kMax>(acc, u3);
     }
-    for (; r < bs; r += G) Vec16<T>::add(acc, __ldg(base + static_cast<size_t>(r) * C));
+    for (; r < bs; r += G) Vec16<T>::template add<kMax>(acc, __ldg(base + static_cast<size_t>(r) * C));
   }
 
   // combine the row groups
@@ -141,8 +155,8 @@ __global__ void __launch_bounds__(kPoolThreads)
   if (rg == 0) {
     for (int g = 1; g < G; ++g)
 #pragma unroll
-      for (int e = 0; e < V; ++e) acc[e] += part[(g * cw + col) * V + e];
-    const float inv = 1.0f / static_cast<float>(bs);  // bs is a power of two: exact
+      for (int e = 0; e < V; ++e) pool_acc<kMax>(acc[e], part[(g * cw + col) * V + e]);
+    const float inv = kMax ? 1.0f : 1.0f / static_cast<float>(bs);  // bs is a power of two: exact
     const int h = (c * V) / D;
     const int d0 = (c * V) % D;
     float* out = task.xp + ((static_cast<size_t>(b) * H + h) * nb + i) * D + d0;

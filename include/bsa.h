@@ -127,6 +127,11 @@ bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int
                        int D, int block_size, double topk_ratio, bsa_dtype dt, void* workspace,
                        size_t workspace_bytes, void* stream);
 
+/* Block size for an input length (page "从M2.7到M3：多模态模型稀疏注意力架构设计与
+ * 实现全解析" §4.2, dynamic block selection): 64 below 500,000 tokens, 128
+ * below 1,000,000, else 256. Returns -1 for seq_len < 1. Pure host function. */
+int bsa_adaptive_block_size(long long seq_len);
+
 /* ---- Variants (flags of the _ex entry points) -------------------------
  * The base entry points above are the _ex ones with flags = 0.
  *
@@ -140,9 +145,34 @@ bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int
  *     blocks, only the diagonal block i is masked token by token).
  * BSA_FLAG_FORCE_DIAG (with BSA_FLAG_CAUSAL): block i is always kept and the
  *   other n_i - 1 are the highest-scoring blocks j < i.
- * Other bits are reserved and rejected (BSA_ERR_INVALID_ARG). */
+ * Other bits (beyond those defined below) are reserved and rejected
+ * (BSA_ERR_INVALID_ARG). */
 #define BSA_FLAG_CAUSAL 1u
 #define BSA_FLAG_FORCE_DIAG 2u
+/* BSA_FLAG_MAX_POOL: blocks are pooled by their element-wise maximum over
+ *   the block's rows instead of the mean, for q and k alike (page "从M2.7到M3：
+ *   多模态模型稀疏注意力架构设计与实现全解析" §2.2, comparison table: block-based
+ *   methods such as MSA/MoBA score a block by its block-internal extreme
+ *   value). Read by the pooling step (bsa_block_pool_ex and the whole-path
+ *   entry points); the score, selection and attention steps are unchanged
+ *   and ignore it. Composes with the causal flags. */
+#define BSA_FLAG_MAX_POOL 4u
+/* BSA_GLOBAL_HEAD_PERIOD(p), p in 1..255 (bits 8-15 of the flags): global
+ *   attention heads (page "从M2.7到M3：多模态模型稀疏注意力架构设计与实现全解析" §5.3:
+ *   one global head in every four, against losses at block boundaries).
+ *   Reading: query head h is global when h % p == 0 and attends to every key
+ *   block (with BSA_FLAG_CAUSAL: every block j <= i, token-masked as usual),
+ *   reading no index row; the other heads attend over their selection.
+ *   Read by the attention step (and the whole-path entry points, which still
+ *   select blocks for every head); the training entry points refuse it
+ *   (BSA_ERR_UNSUPPORTED). p = 1 makes every head dense. */
+#define BSA_GLOBAL_HEAD_PERIOD(p) ((((unsigned)(p)) & 0xFFu) << 8)
+
+/* bsa_block_pool with variant flags: BSA_FLAG_MAX_POOL pools by the
+ * element-wise block maximum (x_pooled[b, h, i, d] = max_t x[b, i*block_size
+ * + t, h, d], exact); the causal flags do not change pooling. */
+bsa_status bsa_block_pool_ex(const void* x, float* x_pooled, int B, int N, int H, int D, int block_size,
+                             bsa_dtype dt, unsigned flags, void* stream);
 
 /* bsa_block_scores_topk with variant flags (see above). With
  * BSA_FLAG_CAUSAL, scores is still written in full (all nb x nb entries). */

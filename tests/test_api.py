@@ -42,6 +42,13 @@ def test_topk_count_is_python_int(bsa, nb, ratio):
     assert bsa.bsa_topk_count(nb, ratio) == int(ratio * nb)
 
 
+@pytest.mark.parametrize("n,want", [(1, 64), (499_999, 64), (500_000, 128), (999_999, 128),
+                                    (1_000_000, 256), (1 << 40, 256), (0, -1)])
+def test_adaptive_block_size(bsa, oracle_mod, n, want):
+    # the page's rule ("从M2.7到M3" §4.2), and the oracle's restatement of it
+    assert bsa.bsa_adaptive_block_size(n) == want == oracle_mod.adaptive_block_size(n)
+
+
 def test_topk_count_rejects_bad_input(bsa):
     assert bsa.bsa_topk_count(0, 0.5) == -1
     assert bsa.bsa_topk_count(8, -0.1) == -1
@@ -126,8 +133,10 @@ def test_ex_entry_points_reject_bad_flags(bsa):
     P = ctypes.c_void_p
     fake = P(0x10000)
     # unknown bit
-    st = bsa_lib.bsa_forward_ex(fake, fake, fake, P(0x20000), 1, 1024, 2, 64, 64, 0.25, 1, 4, fake,
+    st = bsa_lib.bsa_forward_ex(fake, fake, fake, P(0x20000), 1, 1024, 2, 64, 64, 0.25, 1, 8, fake,
                                 1 << 30, P(0))
+    assert st == 1 and b"flag" in bsa_lib.bsa_last_error_detail()
+    st = bsa_lib.bsa_block_pool_ex(fake, P(0x20000), 1, 1024, 2, 64, 64, 1, 8, P(0))
     assert st == 1 and b"flag" in bsa_lib.bsa_last_error_detail()
     # forcing the diagonal block only makes sense with the causal flag
     st = bsa_lib.bsa_sparse_attn_fwd_ex(fake, fake, fake, fake, P(0x20000), 1, 1024, 2, 64, 64, 4,
@@ -209,7 +218,7 @@ def _host_fwd(bsa, q=A, k=A, v=A, o=A + 0x100, B=1, N=512, H=2, Hkv=2, D=64, bs=
 
 @pytest.mark.parametrize("kw,status", [
     (dict(q=0), 1), (dict(o=0), 1), (dict(N=500), 1), (dict(Hkv=3), 1), (dict(ratio=0.01), 1),
-    (dict(flags=4), 1), (dict(flags=2), 1), (dict(D=96), 2), (dict(dt=7), 2), (dict(ws=0), 4),
+    (dict(flags=8), 1), (dict(flags=2), 1), (dict(D=96), 2), (dict(dt=7), 2), (dict(ws=0), 4),
     (dict(wsb=16), 4), (dict(ws=A + 0x210), 3),
 ])
 def test_host_entry_point_rejects_bad_arguments(bsa, kw, status):
