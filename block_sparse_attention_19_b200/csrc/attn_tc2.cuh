@@ -65,10 +65,19 @@ template <int D, bool F8 = false>
 struct Tc2Layout {
   static constexpr int kElem = F8 ? 1 : 2;                  // bytes per element
   static constexpr uint32_t kTileBytes = 128 * D * kElem;  // a 128-row Q, K or V tile
-  static constexpr int kKStages = F8 ? 6 : (D == 128 ? 3 : 6);
-  static constexpr int kVStages = F8 ? 6 : (D == 128 ? 2 : 6);
-  static constexpr int kChunks = D * kElem / 128;          // 128-byte column chunks of a row
-  static constexpr int kChunkElems = 128 / kElem;          // elements per chunk (TMA box width)
+  static constexpr int kKStages = F8 ? (D == 64 ? 12 : 6) : (D == 128 ? 3 : 6);
+  static constexpr int kVStages = F8 ? (D == 64 ? 12 : 6) : (D == 128 ? 2 : 6);
+  // A tile is stored as column chunks of kRowBytes per row in the swizzled
+  // layout the MMA reads: 128-byte rows (128-byte swizzle), or 64-byte rows
+  // (64-byte swizzle) when a whole row is 64 bytes (e4m3 with D = 64).
+  static constexpr uint32_t kRowBytes = D * kElem < 128 ? D * kElem : 128;
+  static constexpr int kChunks = D * kElem / kRowBytes;     // column chunks of a row
+  static constexpr int kChunkElems = kRowBytes / kElem;     // elements per chunk (TMA box width)
+  static constexpr uint32_t kChunkBytes = 128 * kRowBytes;  // one chunk of a 128-row tile
+  static constexpr uint32_t kHalfBytes = 64 * kRowBytes;    // 64 rows of a chunk (one TMA box)
+  static constexpr uint32_t kSBO = 8 * kRowBytes;           // 8-row swizzle atom
+  static constexpr uint32_t kLayout = kRowBytes == 128 ? 2u : 4u;  // descriptor layout field
+  static constexpr int kStepsPerRow = kRowBytes / 32;       // 32-byte MMA K steps per chunk row
   static constexpr uint32_t kQOff = 0;  // Q_A, Q_B
   static constexpr uint32_t kKOff = 2 * kTileBytes;
   static constexpr uint32_t kVOff = kKOff + kKStages * kTileBytes;
@@ -365,7 +374,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         for (int x = 0; x < nstreams; ++x)
           for (int hh = 0; hh < 2; ++hh)
             for (int c = 0; c < L::kChunks; ++c)
-              tma_load_4d(smem + L::kQOff + x * L::kTileBytes + c * (128 * 128) + hh * 64 * 128,
+              tma_load_4d(smem + L::kQOff + x * L::kTileBytes + c * L::kChunkBytes + hh * L::kHalfBytes,
                           &tm_q, &bar.q_full, c * L::kChunkElems, qh[x], row0[x] + hh * 64, b, stream);
       }
       for (int n = 0; n < nloads && ok; ++n) {
@@ -382,7 +391,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         mbar_arrive_expect_tx(&full[s], L::kTileBytes);
         for (int hf = 0; hf < 2; ++hf)
           for (int c = 0; c < L::kChunks; ++c)
-            tma_load_4d(smem + ring + s * L::kTileBytes + c * (128 * 128) + hf * 64 * 128, map,
+            tma_load_4d(smem + ring + s * L::kTileBytes + c * L::kChunkBytes + hf * L::kHalfBytes, map,
                         &full[s], c * L::kChunkElems, g, r[hf], b, keep);
         issued[s] = use + 1;
       }
@@ -401,13 +410,13 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     // commit per group is the one the softmax needs (ring entries are released
     // by the softmax warps, which see each S complete).
     if (lane == 0) {
-      constexpr uint32_t kSBO = 1024;  // 8 rows x 128 bytes
       const uint32_t idesc_s = kF8 ? idesc_e4m3_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 128, 0, 0);
       // P from TMEM, V MN-major
       const uint32_t idesc_pv = kF8 ? idesc_e4m3_f32(128, D, 0, 1) : idesc_bf16_f32(128, D, 0, 1);
-      const uint64_t dq0 = smem_desc_sw128(sbase + L::kQOff, 16, kSBO);
-      const uint64_t dk0 = smem_desc_sw128(sbase + L::kKOff, 16, kSBO);
-      const uint64_t dv0 = smem_desc_sw128(sbase + L::kVOff, 128 * 128, kSBO);
+      const uint64_t dq0 = smem_desc_swz(sbase + L::kQOff, 16, L::kSBO, L::kLayout);
+      const uint64_t dk0 = smem_desc_swz(sbase + L::kKOff, 16, L::kSBO, L::kLayout);
+      // V MN-major: the leading offset steps between column chunks of D
+      const uint64_t dv0 = smem_desc_swz(sbase + L::kVOff, L::kChunkBytes, L::kSBO, L::kLayout);
       constexpr uint64_t kTileStep = L::kTileBytes >> 4;
       // ring index of stream x's tile t (K and V rings are filled in the same order)
       bool ok = mbar_wait(&bar.q_full, 0, abort_flag, 211);
@@ -427,7 +436,8 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         const uint64_t dq = dq0 + x * kTileStep, dk = dk0 + (n % KS) * kTileStep;
 #pragma unroll
         for (int kk = 0; kk < kStepsS; ++kk) {
-          const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+          const uint64_t off =
+              ((kk / L::kStepsPerRow) * L::kChunkBytes + (kk % L::kStepsPerRow) * 32) >> 4;
           if (kF8)
             mma_f8_ss(tmem + L::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
           else
@@ -456,8 +466,8 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
           const uint32_t a_tmem = tmem + L::col_s(x);
 #pragma unroll
           for (int kk = 0; kk < kStepsPV; ++kk) {
-            // kKeysPerStep keys: 8 TMEM columns of P, kKeysPerStep 128-byte rows of V
-            const uint64_t bv = dv + ((kk * kKeysPerStep * 128) >> 4);
+            // kKeysPerStep keys: 8 TMEM columns of P, kKeysPerStep rows of V
+            const uint64_t bv = dv + ((kk * kKeysPerStep * L::kRowBytes) >> 4);
             if (kF8)
               mma_f8_ts(tmem + L::col_o(x), a_tmem + kk * 8, bv, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
             else
@@ -469,7 +479,8 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
             const uint64_t dq = dq0 + x * kTileStep, dk = dk0 + (nk % KS) * kTileStep;
 #pragma unroll
             for (int kk = 0; kk < kStepsS; ++kk) {
-              const uint64_t off = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+              const uint64_t off =
+              ((kk / L::kStepsPerRow) * L::kChunkBytes + (kk % L::kStepsPerRow) * 32) >> 4;
               if (kF8)
                 mma_f8_ss(tmem + L::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
               else

@@ -125,22 +125,25 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // [B, N, H, D] bf16 (or e4m3 with e4m3 = true) tensor as a 4-D TMA map
 // {D, H, N, B}; box = 128 bytes of a row (64 bf16 or 128 e4m3 columns) x 1
-// head x 64 rows x 1 batch, 128-byte swizzle (the UMMA K-/MN-major layout).
+// head x 64 rows x 1 batch, 128-byte swizzle (the UMMA K-/MN-major layout);
+// a row of only 64 bytes (e4m3, D = 64) is one 64-byte box with the 64-byte
+// swizzle.
 bsa_status make_bnhd_map(CUtensorMap* map, const void* base, int B, int N, int H, int D,
                          bool e4m3 = false) {
   auto encode = tensor_map_encoder();
   if (!encode) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const cuuint64_t es = e4m3 ? 1 : 2;
+  const cuuint32_t row_bytes = static_cast<cuuint64_t>(D) * es < 128 ? static_cast<cuuint32_t>(D * es) : 128u;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * es, static_cast<cuuint64_t>(H) * D * es,
                            static_cast<cuuint64_t>(N) * H * D * es};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / es), 1, 64, 1};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(row_bytes / es), 1, 64, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = encode(map, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                       const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                      row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return BSA_OK;
 }
@@ -383,7 +386,9 @@ bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_
                    : launch_attn_simt<128>(fq, fk, fv, idx, fo, B, N, H, Hkv, bs, kk, scale, flags, st);
   }
   if (dt == BSA_E4M3) {
-    if (D != 128) return fail(BSA_ERR_UNSUPPORTED, "e4m3 inputs need D = 128");
+    if (D == 64)
+      return bs == 64 ? launch_attn_tc2<64, true, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st)
+                      : launch_attn_tc2<64, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st);
     return bs == 64 ? launch_attn_tc2<128, true, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st)
                     : launch_attn_tc2<128, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st);
   }

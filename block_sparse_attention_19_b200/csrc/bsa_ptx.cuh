@@ -331,15 +331,22 @@ __device__ __forceinline__ void tmem_wait_st() {
 // Shared-memory matrix descriptor, SWIZZLE_128B, sm_100 format (version 1):
 // start address, leading-dimension byte offset and stride-dimension byte
 // offset are stored >> 4.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
-                                                    uint32_t sbo_bytes) {
+// Shared-memory matrix descriptor with a swizzled layout: `layout` is the
+// descriptor's layout field (2 = 128-byte swizzle, 4 = 64-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc_swz(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                                  uint32_t layout) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
   d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= 1ull << 46;  // descriptor version for sm_100
-  d |= 2ull << 61;  // layout: 128-byte swizzle
+  d |= static_cast<uint64_t>(layout & 7u) << 61;
   return d;
+}
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                    uint32_t sbo_bytes) {
+  return smem_desc_swz(saddr, lbo_bytes, sbo_bytes, 2u);  // 128-byte swizzle
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and f32 accumulate.

@@ -63,7 +63,7 @@ typedef enum {
    * v scale). Both products run as tcgen05 kind::f8f6f4 with float32
    * accumulation; the softmax weights P are rounded to e4m3 (round to
    * nearest, saturating) for the P.V product, the row sums use float32 P.
-   * Supported for D = 128 (else BSA_ERR_UNSUPPORTED). */
+   * D = 64 and 128. */
   BSA_E4M3 = 2
 } bsa_dtype;
 

@@ -54,30 +54,37 @@ def check_fp8_output(o_gpu, o_ref, o_abs, vmax):
     assert rel <= 0.03, f"rel L2 = {rel}"
 
 
-CASES = [  # (B, N, H, H_kv, block_size, ratio, causal)
-    (1, 2048, 2, 2, 128, 0.25, False),
-    (1, 2048, 4, 2, 128, 0.3, False),   # grouped queries, heads paired in a CTA
-    (1, 1920, 2, 2, 128, 0.4, True),    # causal, odd nb
-    (1, 4096, 2, 2, 256, 0.3, False),   # block_size 256
-    (1, 1024, 2, 2, 128, 1.0, False),   # k = nb
-    (1, 2048, 2, 2, 64, 0.25, False),   # block_size 64: two query blocks stacked per tile
-    (1, 1344, 4, 2, 64, 0.3, True),     # block_size 64, causal, nb 21 (a CTA with one block)
+CASES = [  # (B, N, H, H_kv, D, block_size, ratio, causal)
+    (1, 2048, 2, 2, 128, 128, 0.25, False),
+    (1, 2048, 4, 2, 128, 128, 0.3, False),   # grouped queries, heads paired in a CTA
+    (1, 1920, 2, 2, 128, 128, 0.4, True),    # causal, odd nb
+    (1, 4096, 2, 2, 128, 256, 0.3, False),   # block_size 256
+    (1, 1024, 2, 2, 128, 128, 1.0, False),   # k = nb
+    (1, 2048, 2, 2, 128, 64, 0.25, False),   # block_size 64: two query blocks stacked per tile
+    (1, 1344, 4, 2, 128, 64, 0.3, True),     # block_size 64, causal, nb 21 (a CTA with one block)
+    # D = 64: 64-byte rows in the 64-byte swizzled layout
+    (2, 8192, 4, 4, 64, 64, 0.3, False),     # the page's benchmark shape (seq 8192, D 64, block_size 64)
+    (1, 2048, 2, 2, 64, 128, 0.25, False),
+    (1, 2048, 4, 2, 64, 128, 0.3, False),    # grouped queries, heads paired in a CTA
+    (1, 4096, 2, 2, 64, 256, 0.3, True),     # block_size 256, causal
+    (1, 1344, 4, 2, 64, 64, 0.3, True),      # block_size 64, causal, nb 21
+    (1, 1024, 2, 2, 64, 128, 1.0, False),    # k = nb
 ]
 
 
 @pytest.mark.parametrize("ci", range(len(CASES)))
 def test_fp8_full_path(bsa, oracle_mod, ci):
-    B, N, H, Hkv, bs, ratio, causal = CASES[ci]
-    cfg = W.Config(f"fp8{ci}", B, N, H, 128, bs, ratio, "e4m3", 1.0, 950 + ci, None, H_kv=Hkv)
+    B, N, H, Hkv, D, bs, ratio, causal = CASES[ci]
+    cfg = W.Config(f"fp8{ci}", B, N, H, D, bs, ratio, "e4m3", 1.0, 950 + ci, None, H_kv=Hkv)
     q, k, v = W.make_inputs(cfg, device="cuda")
     assert q.dtype == torch.float8_e4m3fn
     flags = bsa.BSA_FLAG_CAUSAL if causal else 0
-    ws = torch.empty(bsa.bsa_forward_workspace_bytes(B, N, H, 128, bs, ratio, H_kv=Hkv), device="cuda",
+    ws = torch.empty(bsa.bsa_forward_workspace_bytes(B, N, H, D, bs, ratio, H_kv=Hkv), device="cuda",
                      dtype=torch.uint8)
     o = bsa.bsa_forward(q, k, v, bs, ratio, workspace=ws, flags=flags)
     torch.cuda.synchronize()
     assert bsa.bsa_device_error() == 0 and o.dtype == torch.bfloat16
-    _, _, idx_g = bsa.workspace_views(ws, B, N, H, 128, bs, ratio, H_kv=Hkv)
+    _, _, idx_g = bsa.workspace_views(ws, B, N, H, D, bs, ratio, H_kv=Hkv)
     qa, ka, va = _host(q), _host(k), _host(v)
     ref = oracle_mod.forward_gqa(qa, ka, va, bs, ratio, causal=causal)
     g = idx_g.cpu().numpy()
@@ -95,10 +102,21 @@ def test_fp8_full_path(bsa, oracle_mod, ci):
     check_fp8_output(gpu_rows(o, rows, bs), o_ref, o_abs, vabs.max())
 
 
-def test_fp8_refused_where_unsupported(bsa):
-    """FP8 inputs need D = 128."""
-    q = torch.zeros(1, 512, 2, 64, device="cuda", dtype=torch.float8_e4m3fn)
-    with pytest.raises(bsa.BsaError, match="UNSUPPORTED"):
-        bsa.bsa_forward(q, q, q, 128, 0.5)
-    with pytest.raises(bsa.BsaError, match="UNSUPPORTED"):
-        bsa.bsa_forward(q, q, q, 64, 0.5)
+def test_fp8_attention_alone_d64(bsa, oracle_mod):
+    """bsa_sparse_attn_fwd on e4m3 D = 64 inputs with random index rows
+    (non-contiguous blocks), block_size 64 and 128."""
+    for bs in (64, 128):
+        cfg = W.Config("fp8_d64", 1, 4096, 2, 64, bs, 0.25, "e4m3", 1.0, 990 + bs, None)
+        q, k, v = W.make_inputs(cfg, device="cuda")
+        rng = np.random.default_rng(bs)
+        idx = np.sort(np.stack([[rng.choice(cfg.nb, cfg.k, replace=False) for _ in range(cfg.nb)]
+                                for _ in range(cfg.H)])[None], -1).astype(np.int32)
+        o = bsa.bsa_sparse_attn_fwd(q, k, v, torch.from_numpy(idx).cuda(), bs)
+        torch.cuda.synchronize()
+        assert bsa.bsa_device_error() == 0
+        o_ref = oracle_mod.sparse_attn(_host(q), _host(k), _host(v), idx, bs)
+        q64, k64 = (x.to(torch.float64).cpu().numpy() for x in (q, k))
+        vabs = np.abs(v.to(torch.float64).cpu().numpy())
+        o_abs = oracle_mod.sparse_attn(q64, k64, vabs, idx, bs)
+        rows = np.broadcast_to(np.arange(cfg.nb, dtype=np.int32), (1, 2, cfg.nb)).copy()
+        check_fp8_output(gpu_rows(o, rows, bs), o_ref, o_abs, vabs.max())
