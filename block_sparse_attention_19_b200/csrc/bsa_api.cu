@@ -418,7 +418,7 @@ BwdWorkspace bwd_workspace_layout(void* base, int B, int N, int H, int Hkv, int 
   return w;
 }
 
-template <int D, bool kCausal>
+template <int D, bool kCausal, bool kStack>
 bsa_status launch_bwd_as(const void* q, const void* k, const void* v, const void* o, const void* dO,
                          const int32_t* idx, const float* lse, const BwdWorkspace& w, void* dq, void* dk,
                          void* dv, int B, int N, int H, int Hkv, int bs, int kk, float scale, cudaStream_t st) {
@@ -433,10 +433,10 @@ bsa_status launch_bwd_as(const void* q, const void* k, const void* v, const void
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(bsa::bwd_dq_kernel<D, kCausal>,
+    cudaError_t e = cudaFuncSetAttribute(bsa::bwd_dq_kernel<D, kCausal, kStack>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(bsa::bwd_dkdv_kernel<D, kCausal>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(bsa::bwd_dkdv_kernel<D, kCausal, kStack>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                L::kBytes);
     if (e != cudaSuccess) return cuda_fail(e, "backward smem attribute");
     attr_set[dev] = true;
@@ -453,13 +453,15 @@ bsa_status launch_bwd_as(const void* q, const void* k, const void* v, const void
   bsa::bwd_rowdot_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), w.dsum, rows, N, H, D);
   // 3. dQ per query tile, 4. dK and dV per key tile of each key/value head
-  const long qtiles = static_cast<long>(B) * H * nb * (bs / 128);
-  const long ktiles = static_cast<long>(B) * Hkv * nb * (bs / 128);
+  // (block_size 64: one tile per pair of blocks, stacked)
+  const long tiles_per_bh = kStack ? (nb + 1) / 2 : static_cast<long>(nb) * (bs / 128);
+  const long qtiles = static_cast<long>(B) * H * tiles_per_bh;
+  const long ktiles = static_cast<long>(B) * Hkv * tiles_per_bh;
   if (qtiles > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "backward grid too large");
   const float scale_log2 = scale * 1.4426950408889634f;
-  bsa::bwd_dq_kernel<D, kCausal><<<static_cast<unsigned>(qtiles), bsa::kBwdThreads, L::kBytes, st>>>(
+  bsa::bwd_dq_kernel<D, kCausal, kStack><<<static_cast<unsigned>(qtiles), bsa::kBwdThreads, L::kBytes, st>>>(
       mq, mk, mv, mdo, idx, lse, w.dsum, static_cast<__nv_bfloat16*>(dq), N, H, Hkv, bs, kk, scale, scale_log2);
-  bsa::bwd_dkdv_kernel<D, kCausal><<<static_cast<unsigned>(ktiles), bsa::kBwdThreads, L::kBytes, st>>>(
+  bsa::bwd_dkdv_kernel<D, kCausal, kStack><<<static_cast<unsigned>(ktiles), bsa::kBwdThreads, L::kBytes, st>>>(
       mq, mk, mv, mdo, w.mask, lse, w.dsum, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), N,
       H, Hkv, bs, scale, scale_log2);
   e = cudaGetLastError();
@@ -471,11 +473,16 @@ bsa_status launch_bwd(const void* q, const void* k, const void* v, const void* o
                       int B, int N, int H, int Hkv, int D, int bs, int kk, float scale, unsigned flags,
                       cudaStream_t st) {
   const bool causal = (flags & BSA_FLAG_CAUSAL) != 0;
+#define BSA_BWD_ARGS q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, Hkv, bs, kk, scale, st
+  if (bs == 64) {
+    if (D == 64)
+      return causal ? launch_bwd_as<64, true, true>(BSA_BWD_ARGS) : launch_bwd_as<64, false, true>(BSA_BWD_ARGS);
+    return causal ? launch_bwd_as<128, true, true>(BSA_BWD_ARGS) : launch_bwd_as<128, false, true>(BSA_BWD_ARGS);
+  }
   if (D == 64)
-    return causal ? launch_bwd_as<64, true>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, Hkv, bs, kk, scale, st)
-                  : launch_bwd_as<64, false>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, Hkv, bs, kk, scale, st);
-  return causal ? launch_bwd_as<128, true>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, Hkv, bs, kk, scale, st)
-                : launch_bwd_as<128, false>(q, k, v, o, dO, idx, lse, w, dq, dk, dv, B, N, H, Hkv, bs, kk, scale, st);
+    return causal ? launch_bwd_as<64, true, false>(BSA_BWD_ARGS) : launch_bwd_as<64, false, false>(BSA_BWD_ARGS);
+  return causal ? launch_bwd_as<128, true, false>(BSA_BWD_ARGS) : launch_bwd_as<128, false, false>(BSA_BWD_ARGS);
+#undef BSA_BWD_ARGS
 }
 
 struct Workspace {
@@ -691,7 +698,7 @@ bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int
 // ---- training: the forward with the row log-sum-exp, and the backward
 
 // The shapes the training entry points cover: bf16, D in {64, 128},
-// block_size 128 or 256, H a multiple of H_kv.
+// block_size 64, 128 or 256, H a multiple of H_kv.
 bsa_status check_train(int B, int N, int H, int Hkv, int D, int block_size, int kk, bsa_dtype dt, unsigned flags) {
   bsa_status s;
   if ((s = check_flags(flags)) != BSA_OK) return s;
@@ -699,7 +706,6 @@ bsa_status check_train(int B, int N, int H, int Hkv, int D, int block_size, int 
   if ((s = check_heads(H, Hkv)) != BSA_OK) return s;
   if (dt != BSA_BF16) return fail(BSA_ERR_UNSUPPORTED, "training entry points take bf16");
   if (global_period(flags) != 0) return fail(BSA_ERR_UNSUPPORTED, "training entry points have no global heads");
-  if (block_size == 64) return fail(BSA_ERR_UNSUPPORTED, "training entry points need block_size 128 or 256");
   const int nb = N / block_size;
   if (kk < 1 || kk > nb) return fail(BSA_ERR_INVALID_ARG, "k=%d outside [1, nb=%d]", kk, nb);
   return BSA_OK;

@@ -111,6 +111,7 @@ struct BwdBarriers {
   int abort;
   int tiles;   // key tiles (dq) or query tiles (dkdv) this CTA walks
   int blocks;  // dkdv: query blocks that kept this key block (per query head of the group)
+  int half[2];  // block_size 64: valid key blocks (dq) or keeping query blocks (dkdv) of each stacked block
 };
 static_assert(sizeof(BwdBarriers) <= 256, "barrier area");
 
@@ -135,6 +136,24 @@ __device__ __forceinline__ void bwd_load_tile(unsigned char* dst, const CUtensor
       tma_load_4d(dst + c * (128 * 128) + hf * 64 * 128, map, bar, c * 64, h, row + hf * 64, b, policy);
 }
 
+// The same tile from two 64-row pieces at token rows row0 (rows 0-63) and
+// row1 (rows 64-127): block_size 64 stacks two blocks in one tile.
+template <int D>
+__device__ __forceinline__ void bwd_load_tile2(unsigned char* dst, const CUtensorMap* map, uint64_t* bar,
+                                               int h, int row0, int row1, int b, uint64_t policy) {
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+    for (int c = 0; c < BwdLayout<D>::kChunks; ++c)
+      tma_load_4d(dst + c * (128 * 128) + hf * 64 * 128, map, bar, c * 64, h, hf == 0 ? row0 : row1, b, policy);
+}
+
+// Key block of entry t of an index row (-1 padding reads block 0).
+__device__ __forceinline__ int bwd_entry_block(const int32_t* sel, int t, int nb) {
+  const int blk = __ldg(sel + t);
+  return blk < 0 ? 0 : (blk >= nb ? nb - 1 : blk);
+}
+
 // 32 bf16 pairs of a row chunk to 16 packed words.
 __device__ __forceinline__ void bwd_pack16(const float (&v)[32], uint32_t (&w)[16]) {
 #pragma unroll
@@ -144,12 +163,18 @@ __device__ __forceinline__ void bwd_pack16(const float (&v)[32], uint32_t (&w)[1
 // ---------------------------------------------------------------- dQ
 // grid.x = B * H * nb * (bs / 128): one CTA per 128-row query tile, which
 // walks the key tiles of its query block's kept blocks.
+// kStack (block_size 64): grid.x = B * H * ceil(nb / 2); the 128-row tile
+// stacks query blocks 2u (rows 0-63) and 2u + 1 (rows 64-127, absent when
+// 2u + 1 = nb), and key tile t stacks the t-th kept block of each (keys
+// 0-63, 64-127), as in the forward. Rows see only their own block's 64 key
+// columns (and none once their list has ended), so dS is zero on the other
+// quadrants and dQ += dS K sums each row's own keys only.
 // TMEM: S [0, 128), dP [128, 256), dQ [256, 256 + D), dS (bf16) [384, 448).
 // dS has columns of its own, so the products of tile t+1 need only wait
 // until the compute warps have read tile t's S and dP into registers: dP(t+1)
 // runs while tile t's dS is being computed, S(t+1) right after its last S
 // load, and dQ += dS(t) K(t) after them.
-template <int D, bool kCausal>
+template <int D, bool kCausal, bool kStack = false>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -168,18 +193,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   constexpr uint32_t kColS = 0, kColP = 128, kColQ = 256, kColDS = 384;
   constexpr int XS = L::kXStages, YS = L::kYStages;
 
-  const int nb = N / bs, tpb = bs / 128;
+  const int nb = N / bs, tpb = kStack ? 1 : bs / 128;
   long u = blockIdx.x;
-  const int part = static_cast<int>(u % tpb);
-  u /= tpb;
-  const int i = static_cast<int>(u % nb);
-  u /= nb;
+  int part = 0, i;
+  if (kStack) {
+    const int per = (nb + 1) / 2;
+    i = 2 * static_cast<int>(u % per);  // blocks i and i + 1
+    u /= per;
+  } else {
+    part = static_cast<int>(u % tpb);
+    u /= tpb;
+    i = static_cast<int>(u % nb);
+    u /= nb;
+  }
   const int h = static_cast<int>(u % H);
   const int b = static_cast<int>(u / H);
   const long bh = static_cast<long>(b) * H + h;
   const int g = h / (H / Hkv);  // the key/value head (and selection) of query head h
-  const int qrow0 = i * bs + part * 128;
+  const int qrow0 = kStack ? i * 64 : i * bs + part * 128;
+  const bool second = kStack && i + 1 < nb;  // the stacked second block exists
   const int32_t* sel = idx + ((static_cast<long>(b) * Hkv + g) * nb + i) * k;
+  const int32_t* sel1 = second ? sel + k : sel;  // kStack: the index row of block i + 1
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
@@ -200,7 +234,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&bar.done, 1);
     mbar_init(&bar.drained, 1);
     bar.abort = 0;
-    bar.tiles = max(index_row_valid(sel, k), 1) * tpb;  // a row of only -1 reads block 0
+    if (kStack) {
+      bar.half[0] = max(index_row_valid(sel, k), 1);
+      bar.half[1] = second ? max(index_row_valid(sel1, k), 1) : 0;
+      bar.tiles = max(bar.half[0], bar.half[1]);
+    } else {
+      bar.tiles = max(index_row_valid(sel, k), 1) * tpb;  // a row of only -1 reads block 0
+    }
     fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -235,11 +275,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bool ok = true;
       for (int t = 0; t < T && ok; ++t) {
         const int s = t % S, use = t / S;
-        const int row = bwd_tile_row(sel, t, 0, bs, nb);
         if (t >= S) ok = mbar_wait(&empty[s], (use - 1) & 1, abort_flag, is_x ? 711 : 712);
         if (!ok) break;
         mbar_arrive_expect_tx(&full[s], L::kTile);
-        bwd_load_tile<D>(smem + ring + s * L::kTile, map, &full[s], g, row, b, keep);
+        if (kStack)  // entries past a list's end read block 0 (their columns are masked)
+          bwd_load_tile2<D>(smem + ring + s * L::kTile, map, &full[s], g, bwd_entry_block(sel, t, nb) * 64,
+                            bwd_entry_block(sel1, t, nb) * 64, b, keep);
+        else
+          bwd_load_tile<D>(smem + ring + s * L::kTile, map, &full[s], g, bwd_tile_row(sel, t, 0, bs, nb), b, keep);
         issued[s] = use + 1;
       }
       if (is_x) mbar_wait_teardown(&bar.a_full, 0);
@@ -319,15 +362,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const long n = qrow0 + row;
-    const float lse2 = __ldg(lse + bh * N + n) * 1.4426950408889634f;  // log2 units
-    const float dn = __ldg(dsum + bh * N + n);
+    // kStack: rows 64 hq.. belong to stacked block hq; an absent block's rows are skipped
+    const int hq = kStack ? row / 64 : 0;
+    const bool live = !kStack || hq == 0 || second;
+    const float lse2 = live ? __ldg(lse + bh * N + n) * 1.4426950408889634f : 0.f;  // log2 units
+    const float dn = live ? __ldg(dsum + bh * N + n) : 0.f;
+    const int vt = kStack ? (live ? bar.half[hq] : 0) : T;  // tiles holding keys of this row
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bar.prod_full, t & 1, abort_flag, 731));
       if (!ok) break;
       tc_fence_after();
-      // keys c of this tile with kbase + c > n are masked (causal)
-      const int lim = kCausal ? static_cast<int>(n - bwd_tile_row(sel, t, 0, bs, nb)) : (1 << 30);
+      // the row's key columns of this tile are [clo, lim]: keys c with
+      // kbase + c > n are masked (causal); kStack: only the row's own block's
+      // 64 columns, none past the end of its list
+      int clo = 0, lim = 1 << 30;
+      if (kStack) {
+        clo = 64 * hq;
+        lim = t < vt ? clo + 63 : -1;
+        if (kCausal && t < vt)
+          lim = min(lim, static_cast<int>(n - bwd_entry_block(hq == 0 ? sel : sel1, t, nb) * 64) + clo);
+      } else if (kCausal) {
+        lim = static_cast<int>(n - bwd_tile_row(sel, t, 0, bs, nb));
+      }
       // the whole dP row, then the tensor core may overwrite it
       uint32_t p0[32], p1[32], p2[32], p3[32];
       tmem_ld32(lane_base + kColP, p0);
@@ -352,7 +409,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         float ds[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float p = (c * 32 + e > lim) ? 0.f : fast_exp2(fmaf(__uint_as_float(sv[e]), scale_log2, -lse2));
+          const int col = c * 32 + e;
+          const float p =
+              (col > lim || col < clo) ? 0.f : fast_exp2(fmaf(__uint_as_float(sv[e]), scale_log2, -lse2));
           ds[e] = p * (__uint_as_float(pv[e]) - dn);
         }
         bwd_pack16(ds, w);
@@ -379,7 +438,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.done, 0, abort_flag, 732));
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* out = dq + ((static_cast<long>(b) * N + n) * H + h) * D;
+      __nv_bfloat16* out = dq + ((static_cast<long>(b) * N + (live ? n : 0)) * H + h) * D;
       uint32_t r[32];
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -392,7 +451,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           w4.y = pack_bf16x2(__uint_as_float(r[e + 2]) * scale, __uint_as_float(r[e + 3]) * scale);
           w4.z = pack_bf16x2(__uint_as_float(r[e + 4]) * scale, __uint_as_float(r[e + 5]) * scale);
           w4.w = pack_bf16x2(__uint_as_float(r[e + 6]) * scale, __uint_as_float(r[e + 7]) * scale);
-          *reinterpret_cast<uint4*>(out + c * 32 + e) = w4;
+          if (live) *reinterpret_cast<uint4*>(out + c * 32 + e) = w4;
         }
       }
     }
@@ -425,7 +484,13 @@ __device__ __forceinline__ int bwd_next_block(const uint32_t* row, int words, in
 // while tile t's P^T and dS^T are made; those go over dP^T, 32-query piece
 // c at columns 128 + 32c: P^T in its first 16 columns, dS^T in the last 16
 // (each piece is read before it is overwritten).
-template <int D, bool kCausal>
+// kStack (block_size 64): grid.x = B * Hkv * ceil(nb / 2); the 128-key tile
+// stacks key blocks 2u (keys 0-63) and 2u + 1 (keys 64-127, absent when
+// 2u + 1 = nb), and query tile t stacks the t-th query block that kept each
+// (queries 0-63, 64-127), so S^T is used on its diagonal quadrants only:
+// a key row sees only its own block's 64 query columns, none once its bit
+// row is exhausted, and P^T and dS^T are zero elsewhere.
+template <int D, bool kCausal, bool kStack = false>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -446,17 +511,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   constexpr uint32_t kColS = 0, kColP = 128, kColV = 256, kColK = 256 + D;
   constexpr int XS = L::kXStages, YS = L::kYStages;
 
-  const int nb = N / bs, tpb = bs / 128, words = (nb + 31) / 32;
+  const int nb = N / bs, tpb = kStack ? 1 : bs / 128, words = (nb + 31) / 32;
   long u = blockIdx.x;
-  const int part = static_cast<int>(u % tpb);
-  u /= tpb;
-  const int j = static_cast<int>(u % nb);
-  u /= nb;
+  int part = 0, j;
+  if (kStack) {
+    const int per = (nb + 1) / 2;
+    j = 2 * static_cast<int>(u % per);  // key blocks j and j + 1
+    u /= per;
+  } else {
+    part = static_cast<int>(u % tpb);
+    u /= tpb;
+    j = static_cast<int>(u % nb);
+    u /= nb;
+  }
   const int g = static_cast<int>(u % Hkv);
   const int b = static_cast<int>(u / Hkv);
   const int G = H / Hkv;
-  const int krow0 = j * bs + part * 128;  // first key token of this tile
+  const int krow0 = kStack ? j * 64 : j * bs + part * 128;  // first key token of this tile
+  const bool second = kStack && j + 1 < nb;                  // the stacked second key block exists
   const uint32_t* mrow = mask + ((static_cast<long>(b) * Hkv + g) * nb + j) * words;
+  const uint32_t* mrow1 = second ? mrow + words : mrow;      // kStack: the bit row of key block j + 1
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
@@ -479,6 +553,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bar.abort = 0;
     int blocks = 0;
     for (int w = 0; w < words; ++w) blocks += __popc(__ldg(mrow + w));
+    if (kStack) {
+      int blocks1 = 0;
+      if (second)
+        for (int w = 0; w < words; ++w) blocks1 += __popc(__ldg(mrow1 + w));
+      bar.half[0] = blocks;
+      bar.half[1] = blocks1;
+      blocks = max(blocks, blocks1);  // query tiles per query head
+    }
     bar.blocks = blocks;
     bar.tiles = G * blocks * tpb;
     fence_mbarrier_init();
@@ -492,6 +574,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
   const int U = bar.tiles, UB = bar.blocks * tpb;  // tiles in all, tiles per query head
+  const int H0 = kStack ? bar.half[0] : 0, H1 = kStack ? bar.half[1] : 0;
   const uint32_t sbase = smem_u32(smem);
   // Tile t is query tile t % UB of query head g * G + t / UB; the bit row is
   // walked again for each query head.
@@ -504,6 +587,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     if (tt % tpb == 0) qb = bwd_next_block(mrow, words, w, cur);
     return qb * bs + (tt % tpb) * 128;  // first query token of the tile
+  };
+  // kStack: both bit rows walked side by side; a row already exhausted keeps
+  // query block 0 (its columns are masked). Returns the tile's query blocks
+  // of the two halves (qb0 for keys 0-63, qb1 for keys 64-127).
+  auto walk2 = [&](int t, int (&w2)[2], uint32_t (&cur2)[2], int (&qb2)[2], int& hq) {
+    const int tt = t % UB;
+    if (tt == 0) {
+      w2[0] = w2[1] = 0;
+      cur2[0] = __ldg(mrow);
+      cur2[1] = __ldg(mrow1);
+      hq = g * G + t / UB;
+    }
+    qb2[0] = tt < H0 ? bwd_next_block(mrow, words, w2[0], cur2[0]) : 0;
+    qb2[1] = tt < H1 ? bwd_next_block(mrow1, words, w2[1], cur2[1]) : 0;
   };
 
   if (warp == 0) {
@@ -525,15 +622,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       int issued[XS] = {};
       bool ok = true;
-      int w = 0, qb = 0, hq = 0;
-      uint32_t cur = 0;
+      int w = 0, qb = 0, hq = 0, w2[2] = {0, 0}, qb2[2] = {0, 0};
+      uint32_t cur = 0, cur2[2] = {0u, 0u};
       for (int t = 0; t < U && ok; ++t) {
         const int s = t % S, use = t / S;
-        const int row = walk(t, w, cur, qb, hq);
+        int row = 0;
+        if (kStack) walk2(t, w2, cur2, qb2, hq);
+        else row = walk(t, w, cur, qb, hq);
         if (t >= S) ok = mbar_wait(&empty[s], (use - 1) & 1, abort_flag, is_x ? 741 : 742);
         if (!ok) break;
         mbar_arrive_expect_tx(&full[s], L::kTile);
-        bwd_load_tile<D>(smem + ring + s * L::kTile, map, &full[s], hq, row, b, keep);
+        if (kStack)
+          bwd_load_tile2<D>(smem + ring + s * L::kTile, map, &full[s], hq, qb2[0] * 64, qb2[1] * 64, b, keep);
+        else
+          bwd_load_tile<D>(smem + ring + s * L::kTile, map, &full[s], hq, row, b, keep);
         issued[s] = use + 1;
       }
       if (is_x) mbar_wait_teardown(&bar.a_full, 0);
@@ -625,12 +727,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int kr = quad * 32 + lane;  // key row of the tile
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const long key = krow0 + kr;
+    // kStack: key rows 64 hk.. belong to stacked key block hk; an absent
+    // block's rows are not written
+    const int hk = kStack ? kr / 64 : 0;
+    const bool live = !kStack || hk == 0 || second;
     bool ok = true;
-    int w = 0, qb = 0, hq = 0;
-    uint32_t cur = 0;
+    int w = 0, qb = 0, hq = 0, w2[2] = {0, 0}, qb2[2] = {0, 0};
+    uint32_t cur = 0, cur2[2] = {0u, 0u};
     float* stats = reinterpret_cast<float*>(smem + L::kStatOff);
     for (int t = 0; t < U; ++t) {
-      const int qrow0 = walk(t, w, cur, qb, hq);
+      // query token of the thread's column kr (stats), and of column 0 of the tile
+      int qrow0 = 0, qtok;
+      if (kStack) {
+        walk2(t, w2, cur2, qb2, hq);
+        qtok = qb2[kr / 64] * 64 + kr % 64;
+      } else {
+        qrow0 = walk(t, w, cur, qb, hq);
+        qtok = qrow0 + kr;
+      }
       const long bh = static_cast<long>(b) * H + hq;
       // the tile's per-query ln-sum (as log2) and D, one query per thread,
       // into slot t % 2. The slot's previous tile, t - 2, is done: this warp
@@ -638,8 +752,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // only after every compute warp has stored tile t - 2's operands.
       float* st_lse = stats + (t & 1) * 256;
       float* st_dn = st_lse + 128;
-      st_lse[kr] = __ldg(lse + bh * N + qrow0 + kr) * 1.4426950408889634f;
-      st_dn[kr] = __ldg(dsum + bh * N + qrow0 + kr);
+      st_lse[kr] = __ldg(lse + bh * N + qtok) * 1.4426950408889634f;
+      st_dn[kr] = __ldg(dsum + bh * N + qtok);
+      // kStack: the row's query columns [clo, chi] (its own block's, none once
+      // its bit row is exhausted) and the first query token of its block
+      const int tt = t % (UB > 0 ? UB : 1);
+      const int clo = kStack ? 64 * hk : 0;
+      const int chi = kStack ? ((live && tt < (hk == 0 ? H0 : H1)) ? clo + 63 : -1) : 127;
+      const int qbase = kStack ? qb2[hk] * 64 - clo : qrow0;  // query token of column c: qbase + c
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.stats_ready[t & 1]);
       ok = __all_sync(0xffffffffu, mbar_wait(&bar.prod_full, t & 1, abort_flag, 761));
@@ -675,7 +795,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int e = 0; e < 32; ++e) {
           const float lse2 = lq[e];
           const float dn = dq_[e];
-          const bool masked = kCausal && key > qrow0 + c * 32 + e;
+          const int col = c * 32 + e;
+          const bool masked = col < clo || col > chi || (kCausal && key > qbase + col);
           const float p = masked ? 0.f : fast_exp2(fmaf(__uint_as_float(sv[e]), scale_log2, -lse2));
           pt[e] = p;
           dst[e] = p * (__uint_as_float(pv[e]) - dn);
@@ -727,7 +848,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             w4.y = pack_bf16x2(__uint_as_float(r[e + 2]) * f, __uint_as_float(r[e + 3]) * f);
             w4.z = pack_bf16x2(__uint_as_float(r[e + 4]) * f, __uint_as_float(r[e + 5]) * f);
             w4.w = pack_bf16x2(__uint_as_float(r[e + 6]) * f, __uint_as_float(r[e + 7]) * f);
-            *reinterpret_cast<uint4*>(out + c * 32 + e) = w4;
+            if (live) *reinterpret_cast<uint4*>(out + c * 32 + e) = w4;
           }
         }
       }

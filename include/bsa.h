@@ -274,8 +274,9 @@ bsa_status bsa_forward_host(const void* q, const void* k, const void* v, void* o
  * token n and kept key token t (p = softmax weight, o = output):
  *   D_n = dO_n . o_n,  dS = p (dO_n . v_t - D_n),
  *   dq_n = scale sum_t dS k_t,  dk_t = scale sum_n dS q_n,  dv_t = sum_n p dO_n.
- * Covered shapes: dt = BSA_BF16, D = 64 or 128, block_size 128 or 256 (others:
- * BSA_ERR_UNSUPPORTED); H a multiple of H_kv in the _gqa forms, where query
+ * Covered shapes: dt = BSA_BF16, D = 64 or 128, block_size 64, 128 or 256
+ * (others: BSA_ERR_UNSUPPORTED; block_size 64 stacks two blocks per 128-row
+ * tile as the forward does); H a multiple of H_kv in the _gqa forms, where query
  * head h reads key/value head h / (H / H_kv) and that head's selection (idx
  * [B, H_kv, nb, topk], as bsa_sparse_attn_fwd_gqa reads it), and dk, dv sum
  * over the group's query heads. Flags: as for the _ex entry points

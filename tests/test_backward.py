@@ -46,6 +46,11 @@ CASES = [  # (B, N, H, D, block_size, ratio, causal)
     (2, 1024, 2, 128, 256, 0.5, False),
     (1, 2048, 2, 128, 256, 0.5, True),
     (1, 1536, 2, 128, 128, 1.0, True),  # dense causal
+    # block_size 64: two blocks stacked per 128-row tile (query and key side)
+    (1, 2048, 2, 64, 64, 0.25, False),
+    (2, 1024, 2, 128, 64, 0.3, True),
+    (1, 1344, 2, 64, 64, 0.3, True),    # nb 21: the last tile holds one block
+    (1, 1024, 2, 64, 64, 1.0, False),   # k = nb
 ]
 
 
@@ -100,16 +105,18 @@ def test_lse_is_the_log_softmax_denominator(bsa, oracle_mod):
 
 
 def test_backward_refuses_uncovered_shapes(bsa):
-    q = torch.zeros(1, 512, 2, 64, device="cuda", dtype=torch.bfloat16)
+    q = torch.zeros(1, 512, 2, 64, device="cuda", dtype=torch.float32)
     idx = torch.zeros(1, 2, 8, 2, device="cuda", dtype=torch.int32)
     with pytest.raises(bsa.BsaError, match="UNSUPPORTED"):
-        bsa.bsa_sparse_attn_fwd_train(q, q, q, idx, 64)  # block_size 64
+        bsa.bsa_sparse_attn_fwd_train(q, q, q, idx, 64)  # float32 inputs
 
 
 GQA_CASES = [  # (B, N, H, H_kv, D, block_size, ratio, causal)
     (1, 2048, 4, 2, 128, 128, 0.25, False),
     (1, 2048, 6, 2, 64, 128, 0.3, True),     # G = 3
     (2, 1024, 4, 1, 128, 256, 0.5, False),   # all query heads in one group, block_size 256
+    (1, 2048, 4, 2, 64, 64, 0.3, True),      # block_size 64, causal
+    (1, 1344, 6, 2, 128, 64, 0.25, False),   # block_size 64, G = 3, nb 21
 ]
 
 
