@@ -390,6 +390,107 @@ def forward_global(q, k, v, block_size: int, topk_ratio: float, period: int, cau
     return r
 
 
+# ---------------------------------------------------------------- overlapping key blocks
+# Reading ("从M2.7到M3" §5.3: against losses at block boundaries, overlapping
+# blocks with overlap_ratio = 0.25): key blocks become windows of block_size
+# tokens that overlap their neighbours by ov = int(overlap_ratio * block_size)
+# tokens, i.e. start every s = block_size - ov tokens; the last window is
+# moved back to end at token N, so nb_k = ceil((N - block_size) / s) + 1
+# windows cover the sequence. Query blocks stay disjoint. Each window is
+# scored by its mean key, k = int(topk_ratio * nb_k) windows are kept per
+# query block, and each query row attends to the union of the kept windows'
+# tokens (a token two kept windows share counts once).
+
+def window_starts(N: int, block_size: int, ov: int) -> np.ndarray:
+    """First token of every key window."""
+    if not 0 <= ov < block_size or N < block_size:
+        raise ValueError("need 0 <= ov < block_size <= N")
+    s = block_size - ov
+    nbk = -(-(N - block_size) // s) + 1
+    return np.minimum(np.arange(nbk) * s, N - block_size)
+
+
+def window_pool(x, block_size: int, ov: int) -> np.ndarray:
+    """Mean of every key window: [B,N,H,D] -> [B,H,nb_k,D] float64."""
+    xn, code = _as_input(x)
+    xd = _to_f64(xn, code)
+    B, N, H, D = xd.shape
+    w = window_starts(N, block_size, ov)
+    out = np.empty((B, H, len(w), D))
+    for j, t0 in enumerate(w):
+        out[:, :, j] = xd[:, t0:t0 + block_size].sum(axis=1) / block_size
+    return out
+
+
+def _to_f64(x: np.ndarray, code: int) -> np.ndarray:
+    """Exact float64 values of an oracle input array."""
+    if code == BF16:
+        return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    if code == E4M3:
+        lut = np.array([e4m3_to_double(c) for c in range(256)])
+        return lut[x]
+    return x.astype(np.float64)
+
+
+def attend_token_sets(q, k, v, tokens, block_size: int, scale: float | None = None) -> np.ndarray:
+    """Softmax attention of every query row of block i over an explicit token
+    set: tokens[b][g][i] is the sorted array of key tokens of (b, key/value
+    head g, query block i). q [B,N,H,D], k and v [B,N,Hkv,D]; query head h
+    reads key/value head h // (H / Hkv). Returns float64 [B,H,nb,bs,D]."""
+    qn, cq = _as_input(q)
+    kn, ck = _as_input(k)
+    vn, cv = _as_input(v)
+    qd, kd, vd = _to_f64(qn, cq), _to_f64(kn, ck), _to_f64(vn, cv)
+    B, N, H, D = qd.shape
+    Hkv = kd.shape[2]
+    G = H // Hkv
+    nb = N // block_size
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    out = np.empty((B, H, nb, block_size, D))
+    for b in range(B):
+        for h in range(H):
+            g = h // G
+            for i in range(nb):
+                t = np.asarray(tokens[b][g][i])
+                logits = qd[b, i * block_size:(i + 1) * block_size, h] @ kd[b, t, g].T * scale
+                w = np.exp(logits - logits.max(axis=1, keepdims=True))
+                out[b, h, i] = (w @ vd[b, t, g]) / w.sum(axis=1, keepdims=True)
+    return out
+
+
+def window_token_sets(idx: np.ndarray, N: int, block_size: int, ov: int):
+    """The union of the tokens of each row's kept windows: idx [B,Hkv,nb,k]
+    (window ids, entries below 0 select nothing) -> nested lists of sorted
+    token arrays [b][g][i]."""
+    w = window_starts(N, block_size, ov)
+    B, Hkv, nb, _ = idx.shape
+    return [[[np.unique(np.concatenate([np.arange(w[j], w[j] + block_size) for j in idx[b, g, i] if j >= 0]))
+              for i in range(nb)] for g in range(Hkv)] for b in range(B)]
+
+
+def forward_overlap(q, k, v, block_size: int, topk_ratio: float, overlap_ratio: float, pool: str = "mean") -> dict:
+    """The whole path with overlapping key windows (see above); grouped
+    queries as in forward_gqa. Returns qp, qg, kp (window means), scores
+    [B,Hkv,nb,nb_k], idx [B,Hkv,nb,k], o [B,H,nb,bs,D], ov and nb_k."""
+    if pool != "mean":
+        raise ValueError("overlapping windows are mean-pooled")
+    qn, _ = _as_input(q)
+    kn, _ = _as_input(k)
+    B, N, H, D = qn.shape
+    Hkv = kn.shape[2]
+    ov = int(overlap_ratio * block_size)
+    qp = block_pool(q, block_size)
+    qg = group_pool(qp, Hkv)
+    kp = window_pool(k, block_size, ov)
+    nbk = kp.shape[2]
+    kk = topk_count(nbk, topk_ratio)
+    S = np.matmul(qg, kp.transpose(0, 1, 3, 2))  # [B, Hkv, nb, nb_k]
+    idx = topk(S, kk)
+    o = attend_token_sets(q, k, v, window_token_sets(idx, N, block_size, ov), block_size)
+    return {"qp": qp, "qg": qg, "kp": kp, "scores": S, "idx": idx, "o": o, "ov": ov, "nbk": nbk, "k": kk}
+
+
 def o_to_bnhd(o: np.ndarray) -> np.ndarray:
     """Reorder an all-rows oracle output [B,H,nb,bs,D] to [B,N,H,D]."""
     B, H, nb, bs, D = o.shape

@@ -151,6 +151,65 @@ def test_global_head_rows_layout(oracle_mod):
     np.testing.assert_array_equal(w[0, 0], [[0, 1, 2]] * 3)
 
 
+# ---------------------------------------------------------------- overlapping key windows
+# Reading ("从M2.7到M3" §5.3, overlap_ratio = 0.25): key windows of block_size
+# tokens start every block_size - ov tokens (the last one moved back to end at
+# N); query blocks stay disjoint; each row attends to the union of its kept
+# windows' tokens.
+
+def test_hw3_overlap_hand_worked(oracle_mod):
+    g = json.load(open(os.path.join(HERE, "golden", "hw3_overlap.json")))
+    shp = (g["B"], g["N"], g["H"], g["D"])
+    q, k, v = (np.array(g[n], np.float64).reshape(shp) for n in ("q", "k", "v"))
+    r = oracle_mod.forward_overlap(q, k, v, g["block_size"], g["topk_ratio"], g["overlap_ratio"])
+    np.testing.assert_array_equal(oracle_mod.window_starts(g["N"], g["block_size"], r["ov"]), g["window_starts"])
+    np.testing.assert_array_equal(r["qp"][0, 0, :, 0], g["q_pooled"])
+    np.testing.assert_array_equal(r["kp"][0, 0, :, 0], g["k_window_means"])
+    np.testing.assert_array_equal(r["scores"][0, 0], g["scores"])
+    assert r["k"] == g["k_selected"]
+    np.testing.assert_array_equal(r["idx"][0, 0], g["idx"])
+    o = oracle_mod.o_to_bnhd(r["o"]).reshape(-1)
+    np.testing.assert_allclose(o, [_closed(e) for e in g["o_closed_form"]], rtol=1e-15, atol=0)
+
+
+@pytest.mark.parametrize("H,Hkv", [(3, 3), (4, 2)])
+def test_overlap_zero_is_the_plain_path(oracle_mod, H, Hkv):
+    B, N, D, bs, ratio = 2, 96, 8, 8, 0.3
+    q, k, v = _rand((B, N, H, D), 90, bs=bs), _rand((B, N, Hkv, D), 91, bs=bs), _rand((B, N, Hkv, D), 92)
+    r = oracle_mod.forward_overlap(q, k, v, bs, ratio, 0.0)
+    p = oracle_mod.forward_gqa(q, k, v, bs, ratio)
+    np.testing.assert_array_equal(r["idx"], p["idx"])
+    np.testing.assert_allclose(r["o"], p["o"], rtol=1e-12, atol=1e-12)
+
+
+def test_overlap_all_windows_is_dense_attention(oracle_mod):
+    B, N, H, D, bs = 1, 128, 2, 8, 16  # ov 4: windows start every 12 tokens, the last moved back to 112
+    q, k, v = (_rand((B, N, H, D), s, bs=8) for s in (93, 94, 95))
+    r = oracle_mod.forward_overlap(q, k, v, bs, 1.0, 0.25)
+    assert r["nbk"] == 11 and r["k"] == 11
+    o = oracle_mod.o_to_bnhd(r["o"])
+    t = lambda x: torch.from_numpy(x).permute(0, 2, 1, 3)
+    ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), scale=1.0 / math.sqrt(D))
+    np.testing.assert_allclose(o, ref.permute(0, 2, 1, 3).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_window_pool_is_a_sliding_mean(oracle_mod):
+    B, N, H, D, bs, ov = 2, 200, 3, 4, 16, 5
+    x = _rand((B, N, H, D), 96)
+    got = oracle_mod.window_pool(x, bs, ov)
+    starts = oracle_mod.window_starts(N, bs, ov)
+    assert starts[0] == 0 and starts[-1] == N - bs and np.all(np.diff(starts)[:-1] == bs - ov)
+    slide = np.lib.stride_tricks.sliding_window_view(x, bs, axis=1).mean(axis=-1)  # [B, N-bs+1, H, D]
+    np.testing.assert_allclose(got, slide[:, starts].transpose(0, 2, 1, 3), rtol=1e-13, atol=1e-13)
+
+
+def test_overlapping_kept_windows_count_shared_tokens_once(oracle_mod):
+    idx = np.array([[[[0, 1], [2, 4]]]], np.int32)  # two query blocks, windows of 8 starting every 6
+    sets = oracle_mod.window_token_sets(idx, 32, 8, 2)
+    np.testing.assert_array_equal(sets[0][0][0], np.arange(0, 14))
+    np.testing.assert_array_equal(sets[0][0][1], np.concatenate([np.arange(12, 20), np.arange(24, 32)]))
+
+
 # ---------------------------------------------------------------- k = int(ratio * nb)
 
 @pytest.mark.parametrize("nb,ratio,want", [
