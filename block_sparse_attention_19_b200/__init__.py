@@ -20,6 +20,8 @@ Functions carry the C names:
 * ``bsa_sparse_attn_fwd_train(q, k, v, idx, block_size)`` -> (o, lse) and
   ``bsa_sparse_attn_bwd(q, k, v, o, do, idx, lse, block_size)`` -> (dq, dk, dv)
 * ``bsa_adaptive_block_size(seq_len)`` -> 64, 128 or 256
+* ``bsa_forward_overlap(q, k, v, block_size, topk_ratio, overlap_ratio)`` -> o
+  with overlapping key windows (and ``bsa_sparse_attn_fwd_overlap``)
 * ``bsa_topk_count``, ``bsa_forward_workspace_bytes``,
   ``bsa_forward_host_workspace_bytes``, ``workspace_views``, ``bsa_device_error``
 
@@ -53,7 +55,8 @@ EXPORTED = ("bsa_topk_count", "bsa_forward_workspace_bytes", "bsa_block_pool",
             "bsa_forward_gqa", "bsa_sparse_attn_fwd_train", "bsa_sparse_attn_bwd_workspace_bytes",
             "bsa_sparse_attn_bwd", "bsa_forward_host_workspace_bytes", "bsa_forward_host",
             "bsa_sparse_attn_fwd_train_gqa", "bsa_sparse_attn_bwd_gqa_workspace_bytes", "bsa_sparse_attn_bwd_gqa",
-            "bsa_adaptive_block_size", "bsa_block_pool_ex")
+            "bsa_adaptive_block_size", "bsa_block_pool_ex", "bsa_overlap_window_count",
+            "bsa_forward_overlap_workspace_bytes", "bsa_sparse_attn_fwd_overlap", "bsa_forward_overlap")
 
 #: variant flags of the *_ex entry points (include/bsa.h)
 BSA_FLAG_CAUSAL, BSA_FLAG_FORCE_DIAG, BSA_FLAG_MAX_POOL = 1, 2, 4
@@ -108,6 +111,10 @@ def _load() -> ctypes.CDLL:
         "bsa_forward_host": ([P, P, P, P, I, I, I, I, I, I, D, I, U, P, Z, P], I),
         "bsa_adaptive_block_size": ([ctypes.c_longlong], I),
         "bsa_block_pool_ex": ([P, P, I, I, I, I, I, I, U, P], I),
+        "bsa_overlap_window_count": ([I, I, D], I),
+        "bsa_forward_overlap_workspace_bytes": ([I, I, I, I, I, I, D, D], Z),
+        "bsa_sparse_attn_fwd_overlap": ([P, P, P, P, P, I, I, I, I, I, I, I, D, F, I, U, P], I),
+        "bsa_forward_overlap": ([P, P, P, P, I, I, I, I, I, I, D, D, I, U, P, Z, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -195,6 +202,80 @@ def bsa_forward_workspace_bytes(B: int, N: int, H: int, D: int, block_size: int,
     if H_kv is None or H_kv == H:
         return lib.bsa_forward_workspace_bytes(B, N, H, D, block_size, float(topk_ratio))
     return lib.bsa_forward_gqa_workspace_bytes(B, N, H, H_kv, D, block_size, float(topk_ratio))
+
+
+def bsa_overlap_window_count(N: int, block_size: int, overlap_ratio: float) -> int:
+    return lib.bsa_overlap_window_count(int(N), int(block_size), float(overlap_ratio))
+
+
+def bsa_forward_overlap_workspace_bytes(B: int, N: int, H: int, D: int, block_size: int, topk_ratio: float,
+                                        overlap_ratio: float, H_kv: int | None = None) -> int:
+    return lib.bsa_forward_overlap_workspace_bytes(B, N, H, H if H_kv is None else H_kv, D, block_size,
+                                                   float(topk_ratio), float(overlap_ratio))
+
+
+def bsa_forward_overlap(q, k, v, block_size: int, topk_ratio: float, overlap_ratio: float,
+                        workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                        flags: int = 0) -> torch.Tensor:
+    """The whole path with overlapping key windows (see include/bsa.h)."""
+    _check_qkv(q, k, v)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    B, N, H, D = q.shape
+    Hk = k.shape[2]
+    need = bsa_forward_overlap_workspace_bytes(B, N, H, D, block_size, topk_ratio, overlap_ratio, H_kv=Hk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=q.device, dtype=torch.uint8)
+    _dev(workspace, "workspace")
+    o = out if out is not None else _out_like(q)
+    if out is not None:
+        _check_out(out, q)
+    _check(lib.bsa_forward_overlap(_p(q), _p(k), _p(v), _p(o), B, N, H, Hk, D, block_size, float(topk_ratio),
+                                   float(overlap_ratio), _dtype_code(q), flags, _p(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(q)))
+    return o
+
+
+def bsa_sparse_attn_fwd_overlap(q, k, v, idx, block_size: int, overlap_ratio: float, scale: float | None = None,
+                                out: torch.Tensor | None = None, flags: int = 0) -> torch.Tensor:
+    """The attention over overlapping key windows: idx [B, H_kv, nb, k] of window ids."""
+    _check_qkv(q, k, v)
+    _check_idx(idx, q.shape[0], k.shape[2], q.shape[1], block_size)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (idx, "idx")):
+        _dev(t, n)
+    if idx.dtype != torch.int32:
+        raise TypeError("idx must be int32")
+    B, N, H, D = q.shape
+    o = out if out is not None else _out_like(q)
+    if out is not None:
+        _check_out(out, q)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    _check(lib.bsa_sparse_attn_fwd_overlap(_p(q), _p(k), _p(v), _p(idx), _p(o), B, N, H, k.shape[2], D, block_size,
+                                           idx.shape[-1], float(overlap_ratio), float(scale), _dtype_code(q), flags,
+                                           _stream(q)))
+    return o
+
+
+def overlap_workspace_views(ws: torch.Tensor, B: int, N: int, H: int, D: int, block_size: int, topk_ratio: float,
+                            overlap_ratio: float, H_kv: int | None = None):
+    """The pooled q [B,H,nb,D], window means of k [B,H_kv,nb_k,D], index list
+    [B,H_kv,nb,k] and scores [B,H_kv,nb,nb_k] sections of a
+    bsa_forward_overlap workspace."""
+    Hk = H if H_kv is None else H_kv
+    nb = N // block_size
+    nbk = bsa_overlap_window_count(N, block_size, overlap_ratio)
+    kk = bsa_topk_count(nbk, topk_ratio)
+    a256 = lambda x: (x + 255) // 256 * 256
+    qpb, kpb, idxb = a256(B * H * nb * D * 4), a256(B * Hk * nbk * D * 4), a256(B * Hk * nb * kk * 4)
+    base = ws.view(torch.uint8)
+    qp = base[:B * H * nb * D * 4].view(torch.float32).view(B, H, nb, D)
+    kp = base[qpb:qpb + B * Hk * nbk * D * 4].view(torch.float32).view(B, Hk, nbk, D)
+    idx = base[qpb + kpb:qpb + kpb + B * Hk * nb * kk * 4].view(torch.int32).view(B, Hk, nb, kk)
+    off = qpb + kpb + idxb
+    S = base[off:off + B * Hk * nb * nbk * 4].view(torch.float32).view(B, Hk, nb, nbk)
+    return qp, kp, idx, S
 
 
 def bsa_adaptive_block_size(seq_len: int) -> int:

@@ -36,12 +36,14 @@ struct SimtSmem {
 
 // grid.x = B * H * nb * (bs / kSimtRows). gperiod > 0: query heads h with
 // h % gperiod == 0 are global heads (every key block, 0..i when causal).
+// ws < bs: index entries name key windows starting at min(e * ws, N - bs)
+// (nkb of them), and keys the previous kept window holds are masked.
 template <int D>
 __global__ void __launch_bounds__(kSimtThreads)
     sparse_attn_simt_kernel(const float* __restrict__ q, const float* __restrict__ kmat,
                             const float* __restrict__ v, const int32_t* __restrict__ idx,
                             float* __restrict__ o, int N, int H, int Hkv, int bs, int k, float scale,
-                            unsigned flags, int gperiod) {
+                            unsigned flags, int gperiod, int ws, int nkb) {
   pdl_launch_dependents();
   pdl_wait();
   extern __shared__ __align__(16) unsigned char simt_raw[];
@@ -87,15 +89,21 @@ __global__ void __launch_bounds__(kSimtThreads)
   // a global head (h % gperiod == 0) attends to every block, 0..i when causal
   const bool dense = gperiod > 0 && h % gperiod == 0;
   const int nsel = dense ? (causal ? i + 1 : nb) : k;
+  int prev_end = 0;  // overlapping windows: first token past the previous kept window
   for (int s = 0; s < nsel; ++s) {
     int blk = dense ? s : sel[s];
     if (blk < 0) {
       if (s > 0) break;  // the row's valid entries end here (a row of only -1 reads block 0)
       blk = 0;
     }
-    blk = blk >= nb ? nb - 1 : blk;
+    const int lim_blk = dense ? nb : nkb;
+    blk = blk >= lim_blk ? lim_blk - 1 : blk;
+    const int w0 = dense ? blk * bs : min(blk * ws, N - bs);  // first token of the window
+    // keys of this window before `dup_end` were in the previous kept window
+    const int dup_end = (!dense && s > 0 && ws < bs) ? prev_end : 0;
+    prev_end = w0 + bs;
     for (int tt = 0; tt < tiles_per_block; ++tt) {
-      const int t0 = blk * bs + tt * kSimtKeys;
+      const int t0 = w0 + tt * kSimtKeys;
       __syncthreads();  // previous tile fully consumed
       for (int e = tid; e < kSimtKeys * D; e += kSimtThreads) {
         const int r = e / D, d = e % D;
@@ -120,6 +128,8 @@ __global__ void __launch_bounds__(kSimtThreads)
           if (t0 + lane > n0 + r) s0 = -INFINITY;
           if (t0 + lane + 32 > n0 + r) s1 = -INFINITY;
         }
+        if (t0 + lane < dup_end) s0 = -INFINITY;
+        if (t0 + lane + 32 < dup_end) s1 = -INFINITY;
         float mx = fmaxf(s0, s1);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));

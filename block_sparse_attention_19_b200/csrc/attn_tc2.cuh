@@ -111,6 +111,24 @@ __device__ __forceinline__ int sel_block(const int32_t* sel, int t, int nb) {
   return sel ? clamp_block(__ldg(sel + t), nb) : t;
 }
 
+// Key windows: entry t of an index row names key window e, whose first token
+// is min(e * ws, N - bs) (ws = bs: the disjoint blocks; ws < bs: windows that
+// overlap by bs - ws tokens, the last one ending at token N). A global head
+// (sel == nullptr) walks the disjoint blocks. nkb: windows per head.
+struct KeyWin {
+  int bs, N, ws, nkb;
+};
+__device__ __forceinline__ int win_start(const int32_t* sel, int t, const KeyWin& kw) {
+  if (!sel) return t * kw.bs;
+  return min(clamp_block(__ldg(sel + t), kw.nkb) * kw.ws, kw.N - kw.bs);
+}
+// Leading tokens of entry t's window that entry t - 1's window already holds
+// (entries ascend, so only the previous window can reach into this one).
+__device__ __forceinline__ int win_dup(const int32_t* sel, int t, const KeyWin& kw) {
+  if (!sel || t == 0 || kw.ws >= kw.bs || __ldg(sel + t) < 0) return 0;
+  return max(0, win_start(sel, t - 1, kw) + kw.bs - win_start(sel, t, kw));
+}
+
 // Valid entries of an index row; for a global head (sel == nullptr) every
 // block, or with the causal mask the blocks 0..i of query block i.
 template <bool kCausal>
@@ -120,9 +138,17 @@ __device__ __forceinline__ int sel_valid(const int32_t* sel, int k, int i, int n
 
 // Token row where 64-row half `hf` of stream `x`'s key tile t starts.
 __device__ __forceinline__ int tc2_key_row(const int32_t* sel_a, const int32_t* sel_b, int x,
-                                           int t, int hf, int bs, int nb) {
-  if (bs == 128) return sel_block(x == 0 ? sel_a : sel_b, t, nb) * 128 + hf * 64;
-  return sel_block(sel_a, t / 2, nb) * 256 + (t % 2) * 128 + hf * 64;  // bs == 256
+                                           int t, int hf, const KeyWin& kw) {
+  if (kw.bs == 128) return win_start(x == 0 ? sel_a : sel_b, t, kw) + hf * 64;
+  return win_start(sel_a, t / 2, kw) + (t % 2) * 128 + hf * 64;  // bs == 256
+}
+
+// Columns c < lo of 32 scores of a row become -inf (keys another kept window
+// already contributed).
+__device__ __forceinline__ void tc2_mask_before(uint32_t (&r)[32], int c0, int lo) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e)
+    if (c0 + e < lo) r[e] = __float_as_uint(-INFINITY);
 }
 
 // Causal mask on 32 scores of a row: column c0 + e becomes -inf when it is
@@ -209,6 +235,9 @@ __device__ __forceinline__ void tc2_make_p32(const uint32_t (&sv)[32], float m, 
 // gperiod > 0: query heads h with h % gperiod == 0 are global heads, which
 // read no index row and attend to every key block (blocks 0..i when causal);
 // query heads are then never paired in a CTA.
+// ws < bs: the index rows name overlapping key windows (see KeyWin; nkb
+// windows per head); a key that the row's previous kept window already
+// holds is masked, so each token of the union counts once (not causal).
 template <int D, bool kCausal, bool kF8 = false, bool kStack = false>
 __global__ void __launch_bounds__(kTc2Threads, 1)
     sparse_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -216,7 +245,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
                            const __grid_constant__ CUtensorMap tm_v,
                            const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ o, int N,
                            int H, int Hkv, int bs, int k, float scale_log2, float* __restrict__ lse,
-                           int gperiod) {
+                           int gperiod, int ws, int nkb) {
   using L = Tc2Layout<D, kF8>;
   // MMA steps: K = 32 bytes of the row per instruction (16 bf16 or 32 e4m3)
   constexpr int kStepsS = D * L::kElem / 32;
@@ -236,6 +265,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
   volatile int* abort_flag = &bar.abort;
 
   const int nb = N / bs;
+  const KeyWin kw{kStack ? 64 : bs, N, ws, nkb};
   // What the two query tiles (streams) of a CTA are:
   //  - block_size 256: the two 128-row halves of one query block of one head;
   //  - block_size 128, an even number G of query heads per key/value head:
@@ -384,8 +414,8 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         const int t = shared_kv ? n : (n < 2 * Tmin ? (n >> 1) : Tmin + (n - 2 * Tmin));
         int r[2];
         for (int hf = 0; hf < 2; ++hf)
-          r[hf] = kStack ? sel_block(sel4[2 * x + hf], t, nb) * 64  // -1 entries load block 0, unused
-                         : tc2_key_row(sel_a, sel_b, x, t, hf, bs, nb);
+          r[hf] = kStack ? win_start(sel4[2 * x + hf], t, kw)  // -1 entries load block 0, unused
+                         : tc2_key_row(sel_a, sel_b, x, t, hf, kw);
         if (n >= S) ok = mbar_wait(&empty[s], (use - 1) & 1, abort_flag, is_k ? 111 : 112);
         if (!ok) break;
         mbar_arrive_expect_tx(&full[s], L::kTileBytes);
@@ -539,10 +569,18 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
           tmem_wait_ld();
           if (kCausal) {
             // keys c > lim of the block follow the thread's query token
-            const int lim = row0[x] + row - sel_block(sel4[2 * x + hf], j, nb) * 64;
+            const int lim = row0[x] + row - win_start(sel4[2 * x + hf], j, kw);
             if (lim < 63) {
               tc2_mask_after(s0, 0, lim);
               tc2_mask_after(s1, 32, lim);
+            }
+          }
+          if (ws < 64) {
+            // overlapping windows: keys the previous kept window holds
+            const int dup = win_dup(sel4[2 * x + hf], j, kw);
+            if (dup > 0) {
+              tc2_mask_before(s0, 0, dup);
+              tc2_mask_before(s1, 32, dup);
             }
           }
           const float mt = tc2_max64(s0, s1) * scale_log2;
@@ -579,7 +617,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         // first key token of this tile; with the causal flag a tile that
         // reaches past the tile's first query token masks key c for row r when
         // kbase + c > qbase + r (only the diagonal block does)
-        const int kbase = kCausal ? tc2_key_row(sel_a, sel_b, x, j, 0, bs, nb) : 0;
+        const int kbase = kCausal ? tc2_key_row(sel_a, sel_b, x, j, 0, kw) : 0;
         const bool mask_tile = kCausal && kbase + 127 > row0[x];
         // The whole S row in registers: four TMEM loads, one wait.
         uint32_t sa[32], sb[32], sc[32], sd[32];
@@ -595,6 +633,17 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
           tc2_mask_after(sb, 32, lim);
           tc2_mask_after(sc, 64, lim);
           tc2_mask_after(sd, 96, lim);
+        }
+        if (ws < bs) {
+          // overlapping windows: keys of this tile the previous kept window
+          // holds (block_size 256: the window's second tile starts at key 128)
+          const int lo = win_dup(x == 0 ? sel_a : sel_b, bs == 256 ? j / 2 : j, kw) - (bs == 256 ? (j % 2) * 128 : 0);
+          if (lo > 0) {
+            tc2_mask_before(sa, 0, lo);
+            tc2_mask_before(sb, 32, lo);
+            tc2_mask_before(sc, 64, lo);
+            tc2_mask_before(sd, 96, lo);
+          }
         }
 #define BSA_S(i) __uint_as_float((i) < 32 ? sa[(i) & 31] : (i) < 64 ? sb[(i) & 31] : (i) < 96 ? sc[(i) & 31] : sd[(i) & 31])
         float m4[4];

@@ -169,12 +169,19 @@ cudaError_t launch_pdl(void (*kernel)(Params...), unsigned grid, unsigned block,
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// stride < bs pools overlapping windows (stride rows apart, nwin of them);
+// 0 means the disjoint blocks.
 bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int ntasks, int B,
-                       int N, int H, int D, int bs, bsa_dtype dt, unsigned flags, cudaStream_t st) {
+                       int N, int H, int D, int bs, bsa_dtype dt, unsigned flags, cudaStream_t st,
+                       int stride = 0, int nwin = 0) {
   const int V = dt == BSA_F32 ? 4 : (dt == BSA_E4M3 ? 16 : 8);  // elements per 16 bytes
   const int C = H * D / V;
   const int cw = bsa::pool_column_group(C);
-  const long grid = static_cast<long>(ntasks) * B * (N / bs) * (C / cw);
+  if (stride <= 0) {
+    stride = bs;
+    nwin = N / bs;
+  }
+  const long grid = static_cast<long>(ntasks) * B * nwin * (C / cw);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "pool grid too large");
   bsa::PoolTask t0{x0, p0}, t1{x1 ? x1 : x0, p1 ? p1 : p0};
   const unsigned g = static_cast<unsigned>(grid);
@@ -182,16 +189,16 @@ bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int
   const bool maxp = (flags & BSA_FLAG_MAX_POOL) != 0;
   cudaError_t e;
   if (dt == BSA_F32)
-    e = maxp ? launch_pdl(bsa::block_pool_kernel<float, true>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw)
-             : launch_pdl(bsa::block_pool_kernel<float>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw);
+    e = maxp ? launch_pdl(bsa::block_pool_kernel<float, true>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw, stride, nwin)
+             : launch_pdl(bsa::block_pool_kernel<float>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw, stride, nwin);
   else if (dt == BSA_E4M3)
     e = maxp ? launch_pdl(bsa::block_pool_kernel<__nv_fp8_e4m3, true>, g, threads, 0, st, t0, t1, B, N, H, D, bs,
-                          cw)
-             : launch_pdl(bsa::block_pool_kernel<__nv_fp8_e4m3>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw);
+                          cw, stride, nwin)
+             : launch_pdl(bsa::block_pool_kernel<__nv_fp8_e4m3>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw, stride, nwin);
   else
     e = maxp ? launch_pdl(bsa::block_pool_kernel<__nv_bfloat16, true>, g, threads, 0, st, t0, t1, B, N, H, D, bs,
-                          cw)
-             : launch_pdl(bsa::block_pool_kernel<__nv_bfloat16>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw);
+                          cw, stride, nwin)
+             : launch_pdl(bsa::block_pool_kernel<__nv_bfloat16>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw, stride, nwin);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_pool_kernel launch");
 }
@@ -213,7 +220,8 @@ int sm_count() {
 // H query heads, Hkv key/value heads (score matrices); H > Hkv averages each
 // group's pooled queries.
 bsa_status launch_scores(const float* qp, const float* kp, float* S, int B, int H, int Hkv, int nb,
-                         int D, cudaStream_t st) {
+                         int D, cudaStream_t st, int nbk = 0) {
+  if (nbk <= 0) nbk = nb;  // key windows per head (nb but for overlapping windows)
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -228,19 +236,19 @@ bsa_status launch_scores(const float* qp, const float* kp, float* S, int B, int 
   // 128-wide score tiles up to nb = 256 (256-wide ones would leave most SMs
   // idle there), 256-wide beyond; the choice depends on nb alone, so that a
   // subset of the heads is scored exactly like the whole tensor
-  const int ntile = nb <= 256 ? 128 : 256;
+  const int ntile = nbk <= 256 ? 128 : 256;
   const long ntiles = static_cast<long>(B) * Hkv * ((nb + bsa::kScM - 1) / bsa::kScM) *
-                      ((nb + ntile - 1) / ntile);
-  const int tma_store = (nb % 4 == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0) ? 1 : 0;
+                      ((nbk + ntile - 1) / ntile);
+  const int tma_store = (nbk % 4 == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0) ? 1 : 0;
   CUtensorMap tm_s;
   std::memset(&tm_s, 0, sizeof(tm_s));
   if (tma_store) {
     auto encode = tensor_map_encoder();
     if (!encode) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(nb),
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(nbk), static_cast<cuuint64_t>(nb),
                           static_cast<cuuint64_t>(B) * Hkv};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(nb) * 4,
-                             static_cast<cuuint64_t>(nb) * nb * 4};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(nbk) * 4,
+                             static_cast<cuuint64_t>(nb) * nbk * 4};
     cuuint32_t box[3] = {32, 32, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = encode(&tm_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, S, dims, strides, box, estr,
@@ -253,15 +261,17 @@ bsa_status launch_scores(const float* qp, const float* kp, float* S, int B, int 
   const bool grouped = H != Hkv;
   auto kern = ntile == 128 ? (grouped ? bsa::block_scores_tc_kernel<128, true> : bsa::block_scores_tc_kernel<128, false>)
                             : (grouped ? bsa::block_scores_tc_kernel<256, true> : bsa::block_scores_tc_kernel<256, false>);
-  cudaError_t e = launch_pdl(kern, gr, bsa::kScThreads, bsa::kScSmem, st, qp, kp, S, tm_s, nb, D, ntiles, tma_store,
-                             H, Hkv);
+  cudaError_t e = launch_pdl(kern, gr, bsa::kScThreads, bsa::kScSmem, st, qp, kp, S, tm_s, nb, nbk, D, ntiles,
+                             tma_store, H, Hkv);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_scores_tc_kernel launch");
 }
 
+// rows = B * H * nbq rows of nb scores each (nbq = nb but for overlapping
+// key windows, which are not causal).
 bsa_status launch_topk(const float* S, int32_t* idx, int B, int H, int nb, int k, unsigned flags,
-                       cudaStream_t st) {
-  const long rows = static_cast<long>(B) * H * nb;
+                       cudaStream_t st, int nbq = 0) {
+  const long rows = static_cast<long>(B) * H * (nbq > 0 ? nbq : nb);
   const long grid = (rows + bsa::kSelWarps - 1) / bsa::kSelWarps;
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "top-k grid too large");
   cudaError_t e;
@@ -292,16 +302,17 @@ bsa_status launch_topk(const float* S, int32_t* idx, int B, int H, int nb, int k
 }
 
 bsa_status launch_select(const float* qp, const float* kp, float* S, int32_t* idx, int B, int H,
-                         int Hkv, int nb, int D, int k, unsigned flags, cudaStream_t st) {
+                         int Hkv, int nb, int D, int k, unsigned flags, cudaStream_t st, int nbk = 0) {
   bsa_status s;
-  if ((s = launch_scores(qp, kp, S, B, H, Hkv, nb, D, st)) != BSA_OK) return s;
-  return launch_topk(S, idx, B, Hkv, nb, k, flags, st);
+  if (nbk <= 0) nbk = nb;
+  if ((s = launch_scores(qp, kp, S, B, H, Hkv, nb, D, st, nbk)) != BSA_OK) return s;
+  return launch_topk(S, idx, B, Hkv, nbk, k, flags, st, nb);
 }
 
 template <int D>
 bsa_status launch_attn_simt(const float* q, const float* k, const float* v, const int32_t* idx,
                             float* o, int B, int N, int H, int Hkv, int bs, int kk, float scale,
-                            unsigned flags, cudaStream_t st) {
+                            unsigned flags, cudaStream_t st, int ws, int nkb) {
   const size_t smem = sizeof(bsa::SimtSmem<D>);
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -315,7 +326,7 @@ bsa_status launch_attn_simt(const float* q, const float* k, const float* v, cons
   const long grid = static_cast<long>(B) * H * (N / bs) * (bs / bsa::kSimtRows);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   cudaError_t e = launch_pdl(bsa::sparse_attn_simt_kernel<D>, static_cast<unsigned>(grid), bsa::kSimtThreads, smem,
-                             st, q, k, v, idx, o, N, H, Hkv, bs, kk, scale, flags, global_period(flags));
+                             st, q, k, v, idx, o, N, H, Hkv, bs, kk, scale, flags, global_period(flags), ws, nkb);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_simt_kernel launch");
 }
@@ -323,7 +334,7 @@ bsa_status launch_attn_simt(const float* q, const float* k, const float* v, cons
 template <int D, bool kCausal, bool kF8, bool kStack>
 bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                               int B, int N, int H, int Hkv, int bs, int kk, float scale,
-                              float* lse, int gperiod, cudaStream_t st) {
+                              float* lse, int gperiod, int ws, int nkb, cudaStream_t st) {
   using L = bsa::Tc2Layout<D, kF8>;
   CUtensorMap mq, mk, mv;
   bsa_status s;
@@ -360,7 +371,7 @@ bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const
   const float scale_log2 = scale * 1.4426950408889634f;
   cudaError_t e = launch_pdl(bsa::sparse_attn_tc2_kernel<D, kCausal, kF8, kStack>, static_cast<unsigned>(grid),
                              bsa::kTc2Threads, L::kBytes, st, mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H,
-                             Hkv, bs, kk, scale_log2, lse, gperiod);
+                             Hkv, bs, kk, scale_log2, lse, gperiod, ws, nkb);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_tc2_kernel launch");
 }
@@ -368,35 +379,43 @@ bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const
 template <int D, bool kF8 = false, bool kStack = false>
 bsa_status launch_attn_tc2(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                            int B, int N, int H, int Hkv, int bs, int kk, float scale, unsigned flags,
-                           float* lse, cudaStream_t st) {
+                           float* lse, cudaStream_t st, int ws, int nkb) {
   const int gp = global_period(flags);
   return (flags & BSA_FLAG_CAUSAL)
-             ? launch_attn_tc2_as<D, true, kF8, kStack>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, gp, st)
-             : launch_attn_tc2_as<D, false, kF8, kStack>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, gp, st);
+             ? launch_attn_tc2_as<D, true, kF8, kStack>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, gp, ws,
+                                                        nkb, st)
+             : launch_attn_tc2_as<D, false, kF8, kStack>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, gp, ws,
+                                                         nkb, st);
 }
 
+// ws < bs: index entries name overlapping key windows ws tokens apart (nkb
+// of them); 0 means the disjoint blocks.
 bsa_status launch_attn(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                        int B, int N, int H, int Hkv, int D, int bs, int kk, float scale, bsa_dtype dt,
-                       unsigned flags, cudaStream_t st, float* lse = nullptr) {
+                       unsigned flags, cudaStream_t st, float* lse = nullptr, int ws = 0, int nkb = 0) {
+  if (ws <= 0) {
+    ws = bs;
+    nkb = N / bs;
+  }
   if (dt == BSA_F32) {
     const float *fq = static_cast<const float*>(q), *fk = static_cast<const float*>(k),
                 *fv = static_cast<const float*>(v);
     float* fo = static_cast<float*>(o);
-    return D == 64 ? launch_attn_simt<64>(fq, fk, fv, idx, fo, B, N, H, Hkv, bs, kk, scale, flags, st)
-                   : launch_attn_simt<128>(fq, fk, fv, idx, fo, B, N, H, Hkv, bs, kk, scale, flags, st);
+    return D == 64 ? launch_attn_simt<64>(fq, fk, fv, idx, fo, B, N, H, Hkv, bs, kk, scale, flags, st, ws, nkb)
+                   : launch_attn_simt<128>(fq, fk, fv, idx, fo, B, N, H, Hkv, bs, kk, scale, flags, st, ws, nkb);
   }
   if (dt == BSA_E4M3) {
     if (D == 64)
-      return bs == 64 ? launch_attn_tc2<64, true, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st)
-                      : launch_attn_tc2<64, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st);
-    return bs == 64 ? launch_attn_tc2<128, true, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st)
-                    : launch_attn_tc2<128, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st);
+      return bs == 64 ? launch_attn_tc2<64, true, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st, ws, nkb)
+                      : launch_attn_tc2<64, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st, ws, nkb);
+    return bs == 64 ? launch_attn_tc2<128, true, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st, ws, nkb)
+                    : launch_attn_tc2<128, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st, ws, nkb);
   }
   if (bs == 64)
-    return D == 64 ? launch_attn_tc2<64, false, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st)
-                   : launch_attn_tc2<128, false, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st);
-  return D == 64 ? launch_attn_tc2<64>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st)
-                 : launch_attn_tc2<128>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st);
+    return D == 64 ? launch_attn_tc2<64, false, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st, ws, nkb)
+                   : launch_attn_tc2<128, false, true>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st, ws, nkb);
+  return D == 64 ? launch_attn_tc2<64>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st, ws, nkb)
+                 : launch_attn_tc2<128>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, flags, lse, st, ws, nkb);
 }
 
 // Backward: transpose of the selection (bit matrix), D_n, dQ, dK/dV.
@@ -693,6 +712,132 @@ bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int
                        size_t workspace_bytes, void* stream) {
   return bsa_forward_ex(q, k, v, o, B, N, H, D, block_size, topk_ratio, dt, 0u, workspace,
                         workspace_bytes, stream);
+}
+
+// ---- overlapping key windows
+
+namespace {
+
+// ov = int(overlap_ratio * block_size) tokens of overlap (Python int() of the
+// double product), windows ws = block_size - ov apart, nbk of them; false if
+// the ratio is outside [0, 1) or N < block_size.
+bool overlap_plan(int N, int bs, double overlap_ratio, int& ws, int& nbk) {
+  if (!std::isfinite(overlap_ratio) || overlap_ratio < 0.0 || overlap_ratio >= 1.0 || N < bs || bs < 1) return false;
+  const int ov = static_cast<int>(overlap_ratio * static_cast<double>(bs));
+  if (ov < 0 || ov >= bs) return false;
+  ws = bs - ov;
+  nbk = (N - bs + ws - 1) / ws + 1;
+  return true;
+}
+
+// q_pooled [B,H,nb,D] | k window means [B,Hkv,nbk,D] | idx [B,Hkv,nb,k] |
+// scores [B,Hkv,nb,nbk], each section 256-byte aligned
+Workspace overlap_workspace_layout(void* base, int B, int N, int H, int Hkv, int D, int bs, int nbk, int k) {
+  const size_t nb = static_cast<size_t>(N / bs);
+  const size_t qpb = align256(static_cast<size_t>(B) * H * nb * D * sizeof(float));
+  const size_t kpb = align256(static_cast<size_t>(B) * Hkv * nbk * D * sizeof(float));
+  const size_t idxb = align256(static_cast<size_t>(B) * Hkv * nb * k * sizeof(int32_t));
+  const size_t scb = align256(static_cast<size_t>(B) * Hkv * nb * nbk * sizeof(float));
+  unsigned char* p = static_cast<unsigned char*>(base);
+  Workspace w;
+  w.qp = reinterpret_cast<float*>(p);
+  w.kp = reinterpret_cast<float*>(p + qpb);
+  w.idx = reinterpret_cast<int32_t*>(p + qpb + kpb);
+  w.scores = reinterpret_cast<float*>(p + qpb + kpb + idxb);
+  w.bytes = qpb + kpb + idxb + scb;
+  return w;
+}
+
+bsa_status check_overlap_flags(unsigned flags) {
+  bsa_status s;
+  if ((s = check_flags(flags)) != BSA_OK) return s;
+  if (flags & (BSA_FLAG_CAUSAL | BSA_FLAG_FORCE_DIAG))
+    return fail(BSA_ERR_UNSUPPORTED, "overlapping key windows are not causal");
+  if (flags & BSA_FLAG_MAX_POOL) return fail(BSA_ERR_UNSUPPORTED, "overlapping key windows are mean-pooled");
+  return BSA_OK;
+}
+
+}  // namespace
+
+extern "C" int bsa_overlap_window_count(int N, int block_size, double overlap_ratio) {
+  int ws = 0, nbk = 0;
+  if (N < 1 || block_size < 1 || N % block_size != 0 || !overlap_plan(N, block_size, overlap_ratio, ws, nbk)) return -1;
+  return nbk;
+}
+
+extern "C" size_t bsa_forward_overlap_workspace_bytes(int B, int N, int H, int H_kv, int D, int block_size,
+                                                      double topk_ratio, double overlap_ratio) {
+  if (check_dims(B, N, H, D, block_size) != BSA_OK || check_heads(H, H_kv) != BSA_OK) return 0;
+  int ws = 0, nbk = 0;
+  if (!overlap_plan(N, block_size, overlap_ratio, ws, nbk) || nbk > 32768) return 0;
+  const int kk = bsa_topk_count(nbk, topk_ratio);
+  if (kk < 1 || kk > nbk) return 0;
+  return overlap_workspace_layout(nullptr, B, N, H, H_kv, D, block_size, nbk, kk).bytes;
+}
+
+extern "C" bsa_status bsa_sparse_attn_fwd_overlap(const void* q, const void* k, const void* v, const int32_t* idx,
+                                                  void* o, int B, int N, int H, int H_kv, int D, int block_size,
+                                                  int topk, double overlap_ratio, float scale, bsa_dtype dt,
+                                                  unsigned flags, void* stream) {
+  bsa_status s;
+  if ((s = check_overlap_flags(flags)) != BSA_OK) return s;
+  if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
+  if ((s = check_heads(H, H_kv)) != BSA_OK) return s;
+  if ((s = check_dtype(dt)) != BSA_OK) return s;
+  int ws = 0, nbk = 0;
+  if (!overlap_plan(N, block_size, overlap_ratio, ws, nbk))
+    return fail(BSA_ERR_INVALID_ARG, "overlap_ratio=%g outside [0, 1)", overlap_ratio);
+  if (topk < 1 || topk > nbk) return fail(BSA_ERR_INVALID_ARG, "k=%d outside [1, nb_k=%d]", topk, nbk);
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return fail(BSA_ERR_INVALID_ARG, "scale must be positive and finite");
+  if (!q || !k || !v || !idx || !o) return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(o))
+    return fail(BSA_ERR_MISALIGNED, "q, k, v, idx or o");
+  if (o == q || o == k || o == v) return fail(BSA_ERR_INVALID_ARG, "o aliases an input");
+  if ((s = check_device()) != BSA_OK) return s;
+  if ((s = launch_attn(q, k, v, idx, o, B, N, H, H_kv, D, block_size, topk, scale, dt, flags,
+                       static_cast<cudaStream_t>(stream), nullptr, ws, nbk)) != BSA_OK)
+    return s;
+  return ok();
+}
+
+extern "C" bsa_status bsa_forward_overlap(const void* q, const void* k, const void* v, void* o, int B, int N, int H,
+                                          int H_kv, int D, int block_size, double topk_ratio, double overlap_ratio,
+                                          bsa_dtype dt, unsigned flags, void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+  bsa_status s;
+  if ((s = check_overlap_flags(flags)) != BSA_OK) return s;
+  if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
+  if ((s = check_heads(H, H_kv)) != BSA_OK) return s;
+  if ((s = check_dtype(dt)) != BSA_OK) return s;
+  int ws = 0, nbk = 0;
+  if (!overlap_plan(N, block_size, overlap_ratio, ws, nbk))
+    return fail(BSA_ERR_INVALID_ARG, "overlap_ratio=%g outside [0, 1)", overlap_ratio);
+  if (nbk > 32768) return fail(BSA_ERR_UNSUPPORTED, "nb_k=%d > 32768", nbk);
+  if (!std::isfinite(topk_ratio) || topk_ratio < 0.0 || topk_ratio > 1.0)
+    return fail(BSA_ERR_INVALID_ARG, "topk_ratio=%g outside [0, 1]", topk_ratio);
+  const int kk = bsa_topk_count(nbk, topk_ratio);
+  if (kk < 1) return fail(BSA_ERR_INVALID_ARG, "k = int(%g * %d) = %d < 1", topk_ratio, nbk, kk);
+  if (!q || !k || !v || !o) return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(BSA_ERR_MISALIGNED, "q, k, v or o");
+  if (o == q || o == k || o == v) return fail(BSA_ERR_INVALID_ARG, "o aliases an input");
+  const Workspace w = overlap_workspace_layout(workspace, B, N, H, H_kv, D, block_size, nbk, kk);
+  if (!workspace || workspace_bytes < w.bytes)
+    return fail(BSA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", w.bytes, workspace ? workspace_bytes : 0);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(BSA_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  if ((s = check_device()) != BSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int nb = N / block_size;
+  const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  if ((s = launch_pool(q, w.qp, nullptr, nullptr, 1, B, N, H, D, block_size, dt, flags, st)) != BSA_OK) return s;
+  if ((s = launch_pool(k, w.kp, nullptr, nullptr, 1, B, N, H_kv, D, block_size, dt, flags, st, ws, nbk)) != BSA_OK)
+    return s;
+  if ((s = launch_select(w.qp, w.kp, w.scores, w.idx, B, H, H_kv, nb, D, kk, flags, st, nbk)) != BSA_OK) return s;
+  if ((s = launch_attn(q, k, v, w.idx, o, B, N, H, H_kv, D, block_size, kk, scale, dt, flags, st, nullptr, ws, nbk)) !=
+      BSA_OK)
+    return s;
+  return ok();
 }
 
 // ---- training: the forward with the row log-sum-exp, and the backward

@@ -95,8 +95,8 @@ struct ScTile {
   int i0, j0;
 };
 
-__device__ __forceinline__ ScTile sc_tile(long t, int nb, int ntile) {
-  const int mt = (nb + kScM - 1) / kScM, nt = (nb + ntile - 1) / ntile;
+__device__ __forceinline__ ScTile sc_tile(long t, int nbq, int nbk, int ntile) {
+  const int mt = (nbq + kScM - 1) / kScM, nt = (nbk + ntile - 1) / ntile;
   ScTile r;
   r.j0 = static_cast<int>(t % nt) * ntile;
   t /= nt;
@@ -105,16 +105,18 @@ __device__ __forceinline__ ScTile sc_tile(long t, int nb, int ntile) {
   return r;
 }
 
-// grid.x = min(tiles, SMs); S = qbar kbar^T as [B*H, nb, nb] float32.
-// tm_s describes S as {nb, nb, B*H} with 32 x 32 boxes (used when tma_store).
+// grid.x = min(tiles, SMs); S = qbar kbar^T as [B*H, nbq, nbk] float32 (nbq
+// query blocks, nbk key blocks or windows; nbq = nbk but for overlapping key
+// windows). tm_s describes S as {nbk, nbq, B*H} with 32 x 32 boxes (used when
+// tma_store).
 // kGroup: grouped queries (H = G * Hkv query heads): the A operand of score
 // matrix (b, g) is the mean of the pooled rows of query heads g*G .. g*G+G-1
 // (summed in float32, then scaled by 1/G).
 template <int NT, bool kGroup>
 __global__ void __launch_bounds__(kScThreads, 1)
     block_scores_tc_kernel(const float* __restrict__ qp, const float* __restrict__ kp,
-                           float* __restrict__ S, const __grid_constant__ CUtensorMap tm_s, int nb,
-                           int D, long ntiles, int tma_store, int H, int Hkv) {
+                           float* __restrict__ S, const __grid_constant__ CUtensorMap tm_s, int nbq,
+                           int nbk, int D, long ntiles, int tma_store, int H, int Hkv) {
   pdl_launch_dependents();
   pdl_wait();
   constexpr int ntile = NT;
@@ -161,17 +163,17 @@ __global__ void __launch_bounds__(kScThreads, 1)
     bool ok = true;
     long i = 0;
     for (long tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++i) {
-      const ScTile tl = sc_tile(tile, nb, ntile);
+      const ScTile tl = sc_tile(tile, nbq, nbk, ntile);
       // this thread's rows: i0 + rsub + 16 u of qbar, j0 + rsub + 16 u of kbar
       // tl.bh = b * Hkv + g: the query rows of (b, g) start at head g * G of batch b
       const int G = kGroup ? H / Hkv : 1;
       const long qhead = kGroup ? (tl.bh / Hkv) * H + (tl.bh % Hkv) * G : tl.bh;
       const float4* pa = reinterpret_cast<const float4*>(
-                             qp + (qhead * nb + tl.i0 + rsub) * static_cast<long>(D)) + q4;
-      const long hstep = static_cast<long>(nb) * D / 4;  // float4 per query head
+                             qp + (qhead * nbq + tl.i0 + rsub) * static_cast<long>(D)) + q4;
+      const long hstep = static_cast<long>(nbq) * D / 4;  // float4 per query head
       const float4* pb = reinterpret_cast<const float4*>(
-                             kp + (tl.bh * nb + tl.j0 + rsub) * static_cast<long>(D)) + q4;
-      const int ra = nb - tl.i0 - rsub, rb = nb - tl.j0 - rsub;  // rows left below this thread's first
+                             kp + (tl.bh * nbk + tl.j0 + rsub) * static_cast<long>(D)) + q4;
+      const int ra = nbq - tl.i0 - rsub, rb = nbk - tl.j0 - rsub;  // rows left below this thread's first
       const int step = 4 * D;                                   // float4 per 16 rows
       for (int c = 0; c < nch; ++c) {
         const long gi = i * nch + c;  // chunk number within this CTA; stage and group = gi % 2
@@ -276,16 +278,16 @@ __global__ void __launch_bounds__(kScThreads, 1)
     bool ok = true;
     long i = 0;
     for (long tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++i) {
-      const ScTile tl = sc_tile(tile, nb, ntile);
+      const ScTile tl = sc_tile(tile, nbq, nbk, ntile);
       const int buf = static_cast<int>(i & 1);
       ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], static_cast<uint32_t>((i >> 1) & 1), abort_flag, 604));
       if (!ok) break;
       tc_fence_after();
       const int row0 = tl.i0 + quarter * 32;
-      if (row0 < nb) {
+      if (row0 < nbq) {
         for (int cc = 0; cc < ntile / 32; ++cc) {
           const int col0 = tl.j0 + cc * 32;
-          if (col0 >= nb) break;
+          if (col0 >= nbk) break;
           uint32_t r[32];
           tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 256 + cc * 32), r);
           tmem_wait_ld();
@@ -306,11 +308,11 @@ __global__ void __launch_bounds__(kScThreads, 1)
             ++nstore;
           } else {
             const int row = row0 + lane;
-            if (row < nb) {
-              float* dst = S + (tl.bh * nb + row) * static_cast<long>(nb) + col0;
+            if (row < nbq) {
+              float* dst = S + (tl.bh * nbq + row) * static_cast<long>(nbk) + col0;
 #pragma unroll
               for (int e = 0; e < 32; ++e)
-                if (col0 + e < nb) dst[e] = __uint_as_float(r[e]);
+                if (col0 + e < nbk) dst[e] = __uint_as_float(r[e]);
             }
           }
         }

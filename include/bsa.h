@@ -238,6 +238,49 @@ bsa_status bsa_forward_gqa(const void* q, const void* k, const void* v, void* o,
                            int H, int H_kv, int D, int block_size, double topk_ratio, bsa_dtype dt,
                            unsigned flags, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Overlapping key windows ------------------------------------------
+ * Page "从M2.7到M3：多模态模型稀疏注意力架构设计与实现全解析" §5.3: overlapping blocks
+ * (overlap_ratio = 0.25) against losses at block boundaries. Readings: key
+ * blocks become windows of block_size tokens that overlap by
+ * ov = int(overlap_ratio * block_size) tokens, i.e. window e starts at token
+ * min(e * (block_size - ov), N - block_size) (the last window ends at token
+ * N); there are nb_k = ceil((N - block_size) / (block_size - ov)) + 1 of
+ * them. Query blocks stay the disjoint blocks of block_size tokens. Each
+ * window is scored by its mean key, k = int(topk_ratio * nb_k) windows are
+ * kept per query block (ties to the lower window, ascending), and each query
+ * row attends to the union of the kept windows' tokens (a token two kept
+ * windows share counts once). overlap_ratio in [0, 1); 0 is the plain
+ * method. Not causal (BSA_FLAG_CAUSAL and BSA_FLAG_MAX_POOL return
+ * BSA_ERR_UNSUPPORTED); global heads (BSA_GLOBAL_HEAD_PERIOD) attend to
+ * every token as usual. H a multiple of H_kv as in the _gqa entry points. */
+
+/* nb_k for these sizes, or -1 if N % block_size != 0 or overlap_ratio is
+ * outside [0, 1). Pure host function. */
+int bsa_overlap_window_count(int N, int block_size, double overlap_ratio);
+
+/* Workspace bytes of bsa_forward_overlap: pooled q [B, H, nb, D], window
+ * means of k [B, H_kv, nb_k, D], the index list [B, H_kv, nb, k] and the
+ * scores [B, H_kv, nb, nb_k] (float32), each section 256-byte aligned; 0 if
+ * the arguments are invalid. */
+size_t bsa_forward_overlap_workspace_bytes(int B, int N, int H, int H_kv, int D, int block_size,
+                                           double topk_ratio, double overlap_ratio);
+
+/* The attention step over overlapping key windows: idx [B, H_kv, nb, topk]
+ * holds window ids in [0, nb_k) (ascending; a negative entry ends its row),
+ * the rest as bsa_sparse_attn_fwd_gqa. */
+bsa_status bsa_sparse_attn_fwd_overlap(const void* q, const void* k, const void* v, const int32_t* idx,
+                                       void* o, int B, int N, int H, int H_kv, int D, int block_size,
+                                       int topk, double overlap_ratio, float scale, bsa_dtype dt,
+                                       unsigned flags, void* stream);
+
+/* The whole path with overlapping key windows: pooling of q (blocks) and of
+ * k (windows), scores [nb x nb_k] and selection per key/value head, the
+ * attention; five kernel launches on `stream`. */
+bsa_status bsa_forward_overlap(const void* q, const void* k, const void* v, void* o, int B, int N, int H,
+                               int H_kv, int D, int block_size, double topk_ratio, double overlap_ratio,
+                               bsa_dtype dt, unsigned flags, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
 /* ---- The whole path from host memory ----------------------------------
  * bsa_forward_gqa on HOST buffers: q [B, N, H, D], k and v [B, N, H_kv, D]
  * and o [B, N, H, D] live in host memory (page-locked memory lets the copies

@@ -235,7 +235,7 @@ def _bwd_gqa(bsa, H=4, Hkv=2, D=64, bs=128, kk=2, dt=1, flags=0, scale=0.125, ws
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(Hkv=3), 1), (dict(bs=64), 2), (dict(dt=0), 2), (dict(kk=0), 1), (dict(kk=9), 1),
+    (dict(Hkv=3), 1), (dict(flags=0x100), 2), (dict(dt=0), 2), (dict(kk=0), 1), (dict(kk=9), 1),
     (dict(scale=0.0), 1), (dict(flags=2), 1), (dict(dq=A), 1), (dict(ws=0), 4), (dict(wsb=8), 4),
 ])
 def test_grouped_backward_rejects_bad_arguments(bsa, kw, status):
@@ -289,3 +289,39 @@ def test_binding_refuses_mismatched_shapes_before_the_device(bsa):
               lambda: bsa.bsa_block_scores_topk(torch.zeros(1, 4, 8, 64), torch.zeros(1, 2, 8, 64), 2)):
         with pytest.raises(ValueError, match="CUDA tensor"):
             f()
+
+
+# ---------------------------------------------------------------- overlapping key windows
+
+@pytest.mark.parametrize("N,bs,ratio", [(4096, 128, 0.25), (8192, 64, 0.25), (131072, 128, 0.25), (2048, 256, 0.5),
+                                        (1024, 128, 0.0), (128, 128, 0.25)])
+def test_overlap_window_count_matches_the_oracle(bsa, oracle_mod, N, bs, ratio):
+    assert bsa.bsa_overlap_window_count(N, bs, ratio) == len(oracle_mod.window_starts(N, bs, int(ratio * bs)))
+
+
+def test_overlap_window_count_rejects_bad_input(bsa):
+    assert bsa.bsa_overlap_window_count(1000, 128, 0.25) == -1  # N % block_size
+    assert bsa.bsa_overlap_window_count(1024, 128, 1.0) == -1
+    assert bsa.bsa_overlap_window_count(1024, 128, -0.1) == -1
+
+
+def _ovl_fwd(bsa, flags=0, ratio=0.25, ovr=0.25, ws=A + 0x400, wsb=1 << 30, H=2, Hkv=2):
+    P = ctypes.c_void_p
+    return bsa.lib.bsa_forward_overlap(P(A), P(A + 0x100), P(A + 0x200), P(A + 0x300), 1, 1024, H, Hkv, 64, 128,
+                                       ratio, ovr, 1, flags, P(ws), wsb, P(0))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(flags=1), 2), (dict(flags=4), 2), (dict(flags=8), 1), (dict(ovr=1.0), 1), (dict(ovr=-0.5), 1),
+    (dict(ratio=0.01), 1), (dict(ws=0), 4), (dict(wsb=64), 4), (dict(ws=A + 0x410), 3), (dict(Hkv=3), 1),
+])
+def test_overlap_entry_point_rejects_bad_arguments(bsa, kw, status):
+    """bsa_forward_overlap validates on the host before touching a device."""
+    assert _ovl_fwd(bsa, **kw) == status
+
+
+def test_overlap_workspace_bytes(bsa):
+    # N 1024, block_size 128, overlap 32: 11 windows, k = int(0.25 * 11) = 2
+    got = bsa.bsa_forward_overlap_workspace_bytes(1, 1024, 2, 64, 128, 0.25, 0.25)
+    a = lambda x: (x + 255) // 256 * 256
+    assert got == a(2 * 8 * 64 * 4) + a(2 * 11 * 64 * 4) + a(2 * 8 * 2 * 4) + a(2 * 8 * 11 * 4)

@@ -170,3 +170,99 @@ def test_training_entry_points_refuse_global_heads(bsa):
     idx = torch.zeros((1, 2, cfg.nb, cfg.k), device="cuda", dtype=torch.int32)
     with pytest.raises(bsa.BsaError, match="UNSUPPORTED"):
         bsa.bsa_sparse_attn_fwd_train(q, k, v, idx, 128, flags=bsa.BSA_GLOBAL_HEAD_PERIOD(2))
+
+
+# ---------------------------------------------------------------- overlapping key windows
+# Reading ("从M2.7到M3" §5.3, overlap_ratio = 0.25): key windows of block_size
+# tokens overlap by ov = int(overlap_ratio * block_size) tokens (window e
+# starts at min(e (block_size - ov), N - block_size)); query blocks stay
+# disjoint; each row attends to the union of its kept windows' tokens. The
+# oracle attends over explicit token sets built from the GPU's window lists.
+
+OCASES = [  # (B, N, H, H_kv, D, block_size, ratio, overlap_ratio, dtype, flags)
+    (1, 4096, 2, 2, 128, 128, 0.25, 0.25, "bf16", 0),
+    (2, 2048, 3, 3, 64, 64, 0.3, 0.25, "bf16", 0),     # block_size 64 (stacked), 43 windows of 64
+    (1, 4096, 2, 2, 128, 256, 0.3, 0.25, "bf16", 0),
+    (1, 4096, 2, 2, 64, 256, 0.5, 0.6, "bf16", 0),     # overlap 153 > 128: a window's whole first tile repeats
+    (1, 2048, 4, 2, 128, 128, 0.3, 0.25, "bf16", 0),   # grouped queries, heads paired in a CTA
+    (1, 2048, 4, 4, 64, 128, 0.3, 0.25, "bf16", 0x200),  # global heads every 2
+    (2, 512, 2, 2, 64, 64, 0.4, 0.25, "f32", 0),
+    (1, 2048, 2, 2, 64, 128, 0.3, 0.25, "e4m3", 0),
+    (1, 8192, 2, 2, 64, 64, 0.3, 0.25, "bf16", 0),     # the page's block size: last window moved back
+]
+
+
+@pytest.mark.parametrize("ci", range(len(OCASES)))
+def test_overlap_full_path(bsa, oracle_mod, ci):
+    B, N, H, Hkv, D, bs, ratio, ovr, dt, flags = OCASES[ci]
+    cfg = W.Config(f"ovl{ci}", B, N, H, D, bs, ratio, dt, 1.0, 700 + ci, None, H_kv=Hkv)
+    q, k, v = W.make_inputs(cfg, device="cuda")
+    ws = torch.empty(bsa.bsa_forward_overlap_workspace_bytes(B, N, H, D, bs, ratio, ovr, H_kv=Hkv), device="cuda",
+                     dtype=torch.uint8)
+    o = bsa.bsa_forward_overlap(q, k, v, bs, ratio, ovr, workspace=ws, flags=flags)
+    torch.cuda.synchronize()
+    assert bsa.bsa_device_error() == 0
+    qa, ka, va = _host(q), _host(k), _host(v)
+    ref = oracle_mod.forward_overlap(qa, ka, va, bs, ratio, ovr)
+    nbk = bsa.bsa_overlap_window_count(N, bs, ovr)
+    assert nbk == ref["nbk"]
+    _, kp_g, idx_g, _ = bsa.overlap_workspace_views(ws, B, N, H, D, bs, ratio, ovr, H_kv=Hkv)
+    # window means: float32 sums of block_size values
+    absmean = oracle_mod.window_pool(np.abs(k.to(torch.float64).cpu().numpy()), bs, ref["ov"])
+    err = np.abs(kp_g.cpu().numpy().astype(np.float64) - ref["kp"])
+    assert np.all(err <= (bs - 1) * 2.0 ** -24 * absmean * 1.0001 + 1e-30)
+    g = idx_g.cpu().numpy()
+    assert g.shape[-1] == ref["k"]
+    accept_index_rows(g, ref["scores"], ref["k"], ref["idx"])
+    # the union of the GPU's kept windows (global heads: every token)
+    sets = oracle_mod.window_token_sets(g, N, bs, ref["ov"])
+    o_ref = oracle_mod.attend_token_sets(qa, ka, va, sets, bs)
+    if flags:
+        period = flags >> 8
+        dense = oracle_mod.attend_token_sets(qa, ka, va, [[[np.arange(N)] * cfg.nb] * Hkv] * B, bs)
+        for h in range(0, H, period):
+            o_ref[:, h] = dense[:, h]
+    rows = np.broadcast_to(np.arange(cfg.nb, dtype=np.int32), (B, H, cfg.nb)).copy()
+    got = gpu_rows(o, rows, bs)
+    if dt == "e4m3":
+        from test_fp8 import check_fp8_output
+        q64, k64 = (x.to(torch.float64).cpu().numpy() for x in (q, k))
+        vabs = np.abs(v.to(torch.float64).cpu().numpy())
+        check_fp8_output(got, o_ref, oracle_mod.attend_token_sets(q64, k64, vabs, sets, bs), vabs.max())
+    else:
+        check_output(got, o_ref, dt)
+
+
+def test_overlap_zero_is_the_plain_path(bsa):
+    cfg = W.Config("ovl0", 1, 4096, 2, 128, 128, 0.25, "bf16", 1.0, 730, None)
+    q, k, v = W.make_inputs(cfg, device="cuda")
+    a = bsa.bsa_forward(q, k, v, 128, 0.25)
+    b = bsa.bsa_forward_overlap(q, k, v, 128, 0.25, 0.0)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("bs,D", [(64, 64), (128, 128), (256, 64)])
+def test_overlap_attention_alone_with_adjacent_windows(bsa, oracle_mod, bs, D):
+    """bsa_sparse_attn_fwd_overlap on window lists made of runs of adjacent
+    windows, so most kept windows share tokens with the previous one."""
+    N, H, ovr = 4096, 2, 0.25
+    cfg = W.Config("ovl_attn", 1, N, H, D, bs, 0.25, "bf16", 1.0, 740 + bs, None)
+    q, k, v = W.make_inputs(cfg, device="cuda")
+    nbk = bsa.bsa_overlap_window_count(N, bs, ovr)
+    rng = np.random.default_rng(bs)
+    kk = 6
+    idx = np.empty((1, H, cfg.nb, kk), np.int32)
+    for h in range(H):
+        for i in range(cfg.nb):
+            s0, s1 = sorted(rng.choice(nbk - 3, 2, replace=False))
+            idx[0, h, i] = np.unique(np.concatenate([np.arange(s0, s0 + 3), np.arange(s1, s1 + 3)]))[:kk] \
+                if s1 >= s0 + 3 else np.arange(s0, s0 + kk) % nbk
+            idx[0, h, i] = np.sort(idx[0, h, i])
+    o = bsa.bsa_sparse_attn_fwd_overlap(q, k, v, torch.from_numpy(idx).cuda(), bs, ovr)
+    torch.cuda.synchronize()
+    assert bsa.bsa_device_error() == 0
+    sets = oracle_mod.window_token_sets(idx, N, bs, int(ovr * bs))
+    o_ref = oracle_mod.attend_token_sets(_host(q), _host(k), _host(v), sets, bs)
+    rows = np.broadcast_to(np.arange(cfg.nb, dtype=np.int32), (1, H, cfg.nb)).copy()
+    check_output(gpu_rows(o, rows, bs), o_ref, "bf16")
