@@ -115,10 +115,14 @@ __device__ __forceinline__ int sel_block(const int32_t* sel, int t, int nb) {
 // is min(e * ws, N - bs) (ws = bs: the disjoint blocks; ws < bs: windows that
 // overlap by bs - ws tokens, the last one ending at token N). A global head
 // (sel == nullptr) walks the disjoint blocks. nkb: windows per head.
+// kVar = false compiles the plain method only (an index row of disjoint
+// blocks for every head), so its kernels carry none of this.
 struct KeyWin {
   int bs, N, ws, nkb;
 };
+template <bool kVar>
 __device__ __forceinline__ int win_start(const int32_t* sel, int t, const KeyWin& kw) {
+  if constexpr (!kVar) return clamp_block(__ldg(sel + t), kw.nkb) * kw.bs;
   if (!sel) return t * kw.bs;
   return min(clamp_block(__ldg(sel + t), kw.nkb) * kw.ws, kw.N - kw.bs);
 }
@@ -126,21 +130,22 @@ __device__ __forceinline__ int win_start(const int32_t* sel, int t, const KeyWin
 // (entries ascend, so only the previous window can reach into this one).
 __device__ __forceinline__ int win_dup(const int32_t* sel, int t, const KeyWin& kw) {
   if (!sel || t == 0 || kw.ws >= kw.bs || __ldg(sel + t) < 0) return 0;
-  return max(0, win_start(sel, t - 1, kw) + kw.bs - win_start(sel, t, kw));
+  return max(0, win_start<true>(sel, t - 1, kw) + kw.bs - win_start<true>(sel, t, kw));
 }
 
 // Valid entries of an index row; for a global head (sel == nullptr) every
 // block, or with the causal mask the blocks 0..i of query block i.
 template <bool kCausal>
 __device__ __forceinline__ int sel_valid(const int32_t* sel, int k, int i, int nb) {
-  return sel ? index_row_valid(sel, k) : (kCausal ? i + 1 : nb);
+  return sel ? index_row_valid(sel, k) : (kCausal ? i + 1 : nb);  // sel == nullptr only with kVar
 }
 
 // Token row where 64-row half `hf` of stream `x`'s key tile t starts.
+template <bool kVar>
 __device__ __forceinline__ int tc2_key_row(const int32_t* sel_a, const int32_t* sel_b, int x,
                                            int t, int hf, const KeyWin& kw) {
-  if (kw.bs == 128) return win_start(x == 0 ? sel_a : sel_b, t, kw) + hf * 64;
-  return win_start(sel_a, t / 2, kw) + (t % 2) * 128 + hf * 64;  // bs == 256
+  if (kw.bs == 128) return win_start<kVar>(x == 0 ? sel_a : sel_b, t, kw) + hf * 64;
+  return win_start<kVar>(sel_a, t / 2, kw) + (t % 2) * 128 + hf * 64;  // bs == 256
 }
 
 // Columns c < lo of 32 scores of a row become -inf (keys another kept window
@@ -238,7 +243,9 @@ __device__ __forceinline__ void tc2_make_p32(const uint32_t (&sv)[32], float m, 
 // ws < bs: the index rows name overlapping key windows (see KeyWin; nkb
 // windows per head); a key that the row's previous kept window already
 // holds is masked, so each token of the union counts once (not causal).
-template <int D, bool kCausal, bool kF8 = false, bool kStack = false>
+// Both need kVar; the plain method's instances (kVar = false) ignore
+// gperiod, ws and nkb.
+template <int D, bool kCausal, bool kF8 = false, bool kStack = false, bool kVar = false>
 __global__ void __launch_bounds__(kTc2Threads, 1)
     sparse_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
@@ -265,7 +272,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
   volatile int* abort_flag = &bar.abort;
 
   const int nb = N / bs;
-  const KeyWin kw{kStack ? 64 : bs, N, ws, nkb};
+  const KeyWin kw{bs, N, kVar ? ws : bs, kVar ? nkb : nb};
   // What the two query tiles (streams) of a CTA are:
   //  - block_size 256: the two 128-row halves of one query block of one head;
   //  - block_size 128, an even number G of query heads per key/value head:
@@ -274,7 +281,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
   // In the first two the streams read the same key tiles (one selection),
   // so each K and V tile is loaded once for both.
   const int G = H / Hkv;
-  const bool head_pairs = !kStack && bs == 128 && (G % 2) == 0 && gperiod == 0;
+  const bool head_pairs = !kStack && bs == 128 && (G % 2) == 0 && (!kVar || gperiod == 0);
   const bool shared_kv = !kStack && (bs == 256 || head_pairs);
   long u = blockIdx.x;
   int iA, b, qh[2];
@@ -306,7 +313,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
                                        : (bs == 256 ? iA * bs + 128 : (head_pairs ? iA * bs : (iA + 1) * bs))};
   const long bg = static_cast<long>(b) * Hkv + g;
   // both streams belong to one query head whenever global heads exist
-  const bool dense = gperiod > 0 && qh[0] % gperiod == 0;
+  const bool dense = kVar && gperiod > 0 && qh[0] % gperiod == 0;
   const int iB = iA + 1 < nb ? iA + 1 : iA;
   const int32_t* sel_a = dense ? nullptr : idx + (bg * nb + iA) * k;
   const int32_t* sel_b = shared_kv ? sel_a : (dense ? nullptr : idx + (bg * nb + iB) * k);
@@ -414,8 +421,8 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         const int t = shared_kv ? n : (n < 2 * Tmin ? (n >> 1) : Tmin + (n - 2 * Tmin));
         int r[2];
         for (int hf = 0; hf < 2; ++hf)
-          r[hf] = kStack ? win_start(sel4[2 * x + hf], t, kw)  // -1 entries load block 0, unused
-                         : tc2_key_row(sel_a, sel_b, x, t, hf, kw);
+          r[hf] = kStack ? win_start<kVar>(sel4[2 * x + hf], t, kw)  // -1 entries load block 0, unused
+                         : tc2_key_row<kVar>(sel_a, sel_b, x, t, hf, kw);
         if (n >= S) ok = mbar_wait(&empty[s], (use - 1) & 1, abort_flag, is_k ? 111 : 112);
         if (!ok) break;
         mbar_arrive_expect_tx(&full[s], L::kTileBytes);
@@ -569,13 +576,13 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
           tmem_wait_ld();
           if (kCausal) {
             // keys c > lim of the block follow the thread's query token
-            const int lim = row0[x] + row - win_start(sel4[2 * x + hf], j, kw);
+            const int lim = row0[x] + row - win_start<kVar>(sel4[2 * x + hf], j, kw);
             if (lim < 63) {
               tc2_mask_after(s0, 0, lim);
               tc2_mask_after(s1, 32, lim);
             }
           }
-          if (ws < 64) {
+          if constexpr (kVar) {
             // overlapping windows: keys the previous kept window holds
             const int dup = win_dup(sel4[2 * x + hf], j, kw);
             if (dup > 0) {
@@ -617,7 +624,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         // first key token of this tile; with the causal flag a tile that
         // reaches past the tile's first query token masks key c for row r when
         // kbase + c > qbase + r (only the diagonal block does)
-        const int kbase = kCausal ? tc2_key_row(sel_a, sel_b, x, j, 0, kw) : 0;
+        const int kbase = kCausal ? tc2_key_row<kVar>(sel_a, sel_b, x, j, 0, kw) : 0;
         const bool mask_tile = kCausal && kbase + 127 > row0[x];
         // The whole S row in registers: four TMEM loads, one wait.
         uint32_t sa[32], sb[32], sc[32], sd[32];
@@ -634,7 +641,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
           tc2_mask_after(sc, 64, lim);
           tc2_mask_after(sd, 96, lim);
         }
-        if (ws < bs) {
+        if constexpr (kVar) {
           // overlapping windows: keys of this tile the previous kept window
           // holds (block_size 256: the window's second tile starts at key 128)
           const int lo = win_dup(x == 0 ? sel_a : sel_b, bs == 256 ? j / 2 : j, kw) - (bs == 256 ? (j % 2) * 128 : 0);

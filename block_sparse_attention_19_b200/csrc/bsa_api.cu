@@ -169,19 +169,29 @@ cudaError_t launch_pdl(void (*kernel)(Params...), unsigned grid, unsigned block,
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// stride < bs pools overlapping windows (stride rows apart, nwin of them);
-// 0 means the disjoint blocks.
+// One pooling launch for element type T: the block maxima with max pooling,
+// the key windows when `win` (mean only), else the block means.
+template <typename T>
+cudaError_t launch_pool_t(bool maxp, bool win, unsigned g, unsigned threads, cudaStream_t st, bsa::PoolTask t0,
+                          bsa::PoolTask t1, int B, int N, int H, int D, int bs, int cw, int stride, int nwin) {
+  if (win)
+    return launch_pdl(bsa::block_pool_kernel<T, false, true>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw, stride,
+                      nwin);
+  if (maxp)
+    return launch_pdl(bsa::block_pool_kernel<T, true>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw, stride, nwin);
+  return launch_pdl(bsa::block_pool_kernel<T>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw, stride, nwin);
+}
+
+// stride > 0 pools overlapping key windows (stride rows apart, nwin of
+// them); 0 means the disjoint blocks.
 bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int ntasks, int B,
                        int N, int H, int D, int bs, bsa_dtype dt, unsigned flags, cudaStream_t st,
                        int stride = 0, int nwin = 0) {
   const int V = dt == BSA_F32 ? 4 : (dt == BSA_E4M3 ? 16 : 8);  // elements per 16 bytes
   const int C = H * D / V;
   const int cw = bsa::pool_column_group(C);
-  if (stride <= 0) {
-    stride = bs;
-    nwin = N / bs;
-  }
-  const long grid = static_cast<long>(ntasks) * B * nwin * (C / cw);
+  const bool win = stride > 0;
+  const long grid = static_cast<long>(ntasks) * B * (win ? nwin : N / bs) * (C / cw);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "pool grid too large");
   bsa::PoolTask t0{x0, p0}, t1{x1 ? x1 : x0, p1 ? p1 : p0};
   const unsigned g = static_cast<unsigned>(grid);
@@ -189,16 +199,11 @@ bsa_status launch_pool(const void* x0, float* p0, const void* x1, float* p1, int
   const bool maxp = (flags & BSA_FLAG_MAX_POOL) != 0;
   cudaError_t e;
   if (dt == BSA_F32)
-    e = maxp ? launch_pdl(bsa::block_pool_kernel<float, true>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw, stride, nwin)
-             : launch_pdl(bsa::block_pool_kernel<float>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw, stride, nwin);
+    e = launch_pool_t<float>(maxp, win, g, threads, st, t0, t1, B, N, H, D, bs, cw, stride, nwin);
   else if (dt == BSA_E4M3)
-    e = maxp ? launch_pdl(bsa::block_pool_kernel<__nv_fp8_e4m3, true>, g, threads, 0, st, t0, t1, B, N, H, D, bs,
-                          cw, stride, nwin)
-             : launch_pdl(bsa::block_pool_kernel<__nv_fp8_e4m3>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw, stride, nwin);
+    e = launch_pool_t<__nv_fp8_e4m3>(maxp, win, g, threads, st, t0, t1, B, N, H, D, bs, cw, stride, nwin);
   else
-    e = maxp ? launch_pdl(bsa::block_pool_kernel<__nv_bfloat16, true>, g, threads, 0, st, t0, t1, B, N, H, D, bs,
-                          cw, stride, nwin)
-             : launch_pdl(bsa::block_pool_kernel<__nv_bfloat16>, g, threads, 0, st, t0, t1, B, N, H, D, bs, cw, stride, nwin);
+    e = launch_pool_t<__nv_bfloat16>(maxp, win, g, threads, st, t0, t1, B, N, H, D, bs, cw, stride, nwin);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "block_pool_kernel launch");
 }
@@ -331,7 +336,7 @@ bsa_status launch_attn_simt(const float* q, const float* k, const float* v, cons
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "sparse_attn_simt_kernel launch");
 }
 
-template <int D, bool kCausal, bool kF8, bool kStack>
+template <int D, bool kCausal, bool kF8, bool kStack, bool kVar>
 bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const int32_t* idx, void* o,
                               int B, int N, int H, int Hkv, int bs, int kk, float scale,
                               float* lse, int gperiod, int ws, int nkb, cudaStream_t st) {
@@ -345,14 +350,14 @@ bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_tc2_kernel<D, kCausal, kF8, kStack>,
+    cudaError_t e = cudaFuncSetAttribute(bsa::sparse_attn_tc2_kernel<D, kCausal, kF8, kStack, kVar>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return cuda_fail(e, "tc2 smem attribute");
     // The kernel moves registers between warp groups (setmaxnreg); an increase
     // that the launch allocation cannot cover would wait forever, so refuse
     // to launch unless the compiled register count covers the split.
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, bsa::sparse_attn_tc2_kernel<D, kCausal, kF8, kStack>);
+    e = cudaFuncGetAttributes(&fa, bsa::sparse_attn_tc2_kernel<D, kCausal, kF8, kStack, kVar>);
     if (e != cudaSuccess) return cuda_fail(e, "tc2 attributes");
     if (fa.numRegs < static_cast<int>(bsa::kTc2LaunchRegs))
       return fail(BSA_ERR_UNSUPPORTED, "attention kernel built with %d registers/thread, its register split needs %u",
@@ -369,7 +374,7 @@ bsa_status launch_attn_tc2_as(const void* q, const void* k, const void* v, const
                                  : static_cast<long>(B) * H * (bs == 256 ? nb : (nb + 1) / 2);
   if (grid > 0x7fffffffL) return fail(BSA_ERR_UNSUPPORTED, "attention grid too large");
   const float scale_log2 = scale * 1.4426950408889634f;
-  cudaError_t e = launch_pdl(bsa::sparse_attn_tc2_kernel<D, kCausal, kF8, kStack>, static_cast<unsigned>(grid),
+  cudaError_t e = launch_pdl(bsa::sparse_attn_tc2_kernel<D, kCausal, kF8, kStack, kVar>, static_cast<unsigned>(grid),
                              bsa::kTc2Threads, L::kBytes, st, mq, mk, mv, idx, static_cast<__nv_bfloat16*>(o), N, H,
                              Hkv, bs, kk, scale_log2, lse, gperiod, ws, nkb);
   if (e == cudaSuccess) e = cudaGetLastError();
@@ -381,11 +386,16 @@ bsa_status launch_attn_tc2(const void* q, const void* k, const void* v, const in
                            int B, int N, int H, int Hkv, int bs, int kk, float scale, unsigned flags,
                            float* lse, cudaStream_t st, int ws, int nkb) {
   const int gp = global_period(flags);
-  return (flags & BSA_FLAG_CAUSAL)
-             ? launch_attn_tc2_as<D, true, kF8, kStack>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, gp, ws,
-                                                        nkb, st)
-             : launch_attn_tc2_as<D, false, kF8, kStack>(q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, gp, ws,
-                                                         nkb, st);
+  // global heads and overlapping windows run their own instances, so the
+  // plain method's kernels carry none of their code
+  const bool var = gp > 0 || ws < bs;
+#define BSA_TC2_ARGS q, k, v, idx, o, B, N, H, Hkv, bs, kk, scale, lse, gp, ws, nkb, st
+  if (flags & BSA_FLAG_CAUSAL)
+    return var ? launch_attn_tc2_as<D, true, kF8, kStack, true>(BSA_TC2_ARGS)
+               : launch_attn_tc2_as<D, true, kF8, kStack, false>(BSA_TC2_ARGS);
+  return var ? launch_attn_tc2_as<D, false, kF8, kStack, true>(BSA_TC2_ARGS)
+             : launch_attn_tc2_as<D, false, kF8, kStack, false>(BSA_TC2_ARGS);
+#undef BSA_TC2_ARGS
 }
 
 // ws < bs: index entries name overlapping key windows ws tokens apart (nkb

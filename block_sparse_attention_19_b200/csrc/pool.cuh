@@ -97,16 +97,19 @@ inline int pool_column_group(int C) {
 // grid.x = ntasks * B * nb * (C / cw), blockDim.x = kPoolRowGroups * cw. Each
 // CTA reduces bs rows of one group of cw 16-byte columns of one block; row r
 // goes to row group r % kPoolRowGroups, and the groups' partial sums are
-// added in group order. Block i covers rows min(i * stride, N - bs) ..
-// + bs - 1 of nb blocks: stride = bs gives the disjoint blocks, stride < bs
-// overlapping key windows (the last one ending at row N).
-template <typename T, bool kMax = false>
+// added in group order. kWin: item i is the key window of rows
+// min(i * stride, N - bs) .. + bs - 1 (stride < bs: overlapping windows, the
+// last one ending at row N), one of nwin; otherwise block i of the N / bs
+// disjoint blocks (stride and nwin unused: measured 8% faster on c4 than the
+// general form, which keeps the plain method on its own instance).
+template <typename T, bool kMax = false, bool kWin = false>
 __global__ void __launch_bounds__(kPoolThreads)
     block_pool_kernel(PoolTask t0, PoolTask t1, int B, int N, int H, int D, int bs, int cw, int stride,
-                      int nb) {
+                      int nwin) {
   pdl_launch_dependents();
   pdl_wait();
   constexpr int V = Vec16<T>::kN;
+  const int nb = kWin ? nwin : N / bs;
   const int C = H * D / V;  // 16-byte columns per row
   const int ngroups = C / cw;
   const int G = blockDim.x / cw;  // kPoolRowGroups (read at run time: the compiled loop is faster)
@@ -130,9 +133,8 @@ __global__ void __launch_bounds__(kPoolThreads)
   for (int e = 0; e < V; ++e) acc[e] = kMax ? -INFINITY : 0.f;
 
   if (rg < G) {
-    const int row0 = min(i * stride, N - bs);
-    const uint4* base = reinterpret_cast<const uint4*>(task.x) +
-                        (static_cast<size_t>(b) * N + static_cast<size_t>(row0)) * C + c;
+    const size_t row0 = kWin ? static_cast<size_t>(min(i * stride, N - bs)) : static_cast<size_t>(i) * bs;
+    const uint4* base = reinterpret_cast<const uint4*>(task.x) + (static_cast<size_t>(b) * N + row0) * C + c;
     int r = rg;
     // 4 independent loads in flight per thread
     for (; r + 3 * G < bs; r += 4 * G) {
