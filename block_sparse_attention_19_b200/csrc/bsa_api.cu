@@ -542,6 +542,51 @@ Workspace workspace_layout(void* base, int B, int N, int H, int Hkv, int D, int 
 
 }  // namespace
 
+// ---- overlapping key windows: window plan, workspace layout, flag checks
+
+namespace {
+
+// ov = int(overlap_ratio * block_size) tokens of overlap (Python int() of the
+// double product), windows ws = block_size - ov apart, nbk of them; false if
+// the ratio is outside [0, 1) or N < block_size.
+bool overlap_plan(int N, int bs, double overlap_ratio, int& ws, int& nbk) {
+  if (!std::isfinite(overlap_ratio) || overlap_ratio < 0.0 || overlap_ratio >= 1.0 || N < bs || bs < 1) return false;
+  const int ov = static_cast<int>(overlap_ratio * static_cast<double>(bs));
+  if (ov < 0 || ov >= bs) return false;
+  ws = bs - ov;
+  nbk = (N - bs + ws - 1) / ws + 1;
+  return true;
+}
+
+// q_pooled [B,H,nb,D] | k window means [B,Hkv,nbk,D] | idx [B,Hkv,nb,k] |
+// scores [B,Hkv,nb,nbk], each section 256-byte aligned
+Workspace overlap_workspace_layout(void* base, int B, int N, int H, int Hkv, int D, int bs, int nbk, int k) {
+  const size_t nb = static_cast<size_t>(N / bs);
+  const size_t qpb = align256(static_cast<size_t>(B) * H * nb * D * sizeof(float));
+  const size_t kpb = align256(static_cast<size_t>(B) * Hkv * nbk * D * sizeof(float));
+  const size_t idxb = align256(static_cast<size_t>(B) * Hkv * nb * k * sizeof(int32_t));
+  const size_t scb = align256(static_cast<size_t>(B) * Hkv * nb * nbk * sizeof(float));
+  unsigned char* p = static_cast<unsigned char*>(base);
+  Workspace w;
+  w.qp = reinterpret_cast<float*>(p);
+  w.kp = reinterpret_cast<float*>(p + qpb);
+  w.idx = reinterpret_cast<int32_t*>(p + qpb + kpb);
+  w.scores = reinterpret_cast<float*>(p + qpb + kpb + idxb);
+  w.bytes = qpb + kpb + idxb + scb;
+  return w;
+}
+
+bsa_status check_overlap_flags(unsigned flags) {
+  bsa_status s;
+  if ((s = check_flags(flags)) != BSA_OK) return s;
+  if (flags & (BSA_FLAG_CAUSAL | BSA_FLAG_FORCE_DIAG))
+    return fail(BSA_ERR_UNSUPPORTED, "overlapping key windows are not causal");
+  if (flags & BSA_FLAG_MAX_POOL) return fail(BSA_ERR_UNSUPPORTED, "overlapping key windows are mean-pooled");
+  return BSA_OK;
+}
+
+}  // namespace
+
 // ==================================================================== C ABI
 
 extern "C" {
@@ -725,49 +770,6 @@ bsa_status bsa_forward(const void* q, const void* k, const void* v, void* o, int
 }
 
 // ---- overlapping key windows
-
-namespace {
-
-// ov = int(overlap_ratio * block_size) tokens of overlap (Python int() of the
-// double product), windows ws = block_size - ov apart, nbk of them; false if
-// the ratio is outside [0, 1) or N < block_size.
-bool overlap_plan(int N, int bs, double overlap_ratio, int& ws, int& nbk) {
-  if (!std::isfinite(overlap_ratio) || overlap_ratio < 0.0 || overlap_ratio >= 1.0 || N < bs || bs < 1) return false;
-  const int ov = static_cast<int>(overlap_ratio * static_cast<double>(bs));
-  if (ov < 0 || ov >= bs) return false;
-  ws = bs - ov;
-  nbk = (N - bs + ws - 1) / ws + 1;
-  return true;
-}
-
-// q_pooled [B,H,nb,D] | k window means [B,Hkv,nbk,D] | idx [B,Hkv,nb,k] |
-// scores [B,Hkv,nb,nbk], each section 256-byte aligned
-Workspace overlap_workspace_layout(void* base, int B, int N, int H, int Hkv, int D, int bs, int nbk, int k) {
-  const size_t nb = static_cast<size_t>(N / bs);
-  const size_t qpb = align256(static_cast<size_t>(B) * H * nb * D * sizeof(float));
-  const size_t kpb = align256(static_cast<size_t>(B) * Hkv * nbk * D * sizeof(float));
-  const size_t idxb = align256(static_cast<size_t>(B) * Hkv * nb * k * sizeof(int32_t));
-  const size_t scb = align256(static_cast<size_t>(B) * Hkv * nb * nbk * sizeof(float));
-  unsigned char* p = static_cast<unsigned char*>(base);
-  Workspace w;
-  w.qp = reinterpret_cast<float*>(p);
-  w.kp = reinterpret_cast<float*>(p + qpb);
-  w.idx = reinterpret_cast<int32_t*>(p + qpb + kpb);
-  w.scores = reinterpret_cast<float*>(p + qpb + kpb + idxb);
-  w.bytes = qpb + kpb + idxb + scb;
-  return w;
-}
-
-bsa_status check_overlap_flags(unsigned flags) {
-  bsa_status s;
-  if ((s = check_flags(flags)) != BSA_OK) return s;
-  if (flags & (BSA_FLAG_CAUSAL | BSA_FLAG_FORCE_DIAG))
-    return fail(BSA_ERR_UNSUPPORTED, "overlapping key windows are not causal");
-  if (flags & BSA_FLAG_MAX_POOL) return fail(BSA_ERR_UNSUPPORTED, "overlapping key windows are mean-pooled");
-  return BSA_OK;
-}
-
-}  // namespace
 
 extern "C" int bsa_overlap_window_count(int N, int block_size, double overlap_ratio) {
   int ws = 0, nbk = 0;

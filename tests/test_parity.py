@@ -195,12 +195,12 @@ def test_attention_with_oracle_indices(bsa, oracle_mod, case):
 
 
 @pytest.mark.parametrize("nb,D", [(8, 64), (100, 128), (300, 64), (1024, 128), (1501, 64), (4096, 128),
-                                  (4500, 64)])
+                                  (4500, 64), (8192, 64)])
 def test_scores_topk_stage(bsa, oracle_mod, nb, D):
     """bsa_block_scores_topk fed float32 pooled inputs: scores within the
     float32 FFMA bound, index lists by the near-tie rule (ragged tiles, rows
-    of up to 4096 keys in registers, longer rows staged in shared memory, odd
-    nb)."""
+    of up to 4096 keys in registers, rows of up to 6400 keys staged in shared
+    memory, longer rows searched from L2, odd nb)."""
     B, H = 1, 2
     rng = np.random.default_rng(nb)
     qp = (rng.standard_normal((B, H, nb, D)) * 0.3 + rng.standard_normal((B, H, nb, 1))).astype(np.float32)
@@ -220,7 +220,7 @@ def test_scores_topk_stage(bsa, oracle_mod, nb, D):
         accept_index_rows(idx.cpu().numpy(), S_ref, kk, idx_ref)
 
 
-@pytest.mark.parametrize("nb", [40, 100, 1024, 1501, 4500])
+@pytest.mark.parametrize("nb", [40, 100, 1024, 1501, 4500, 8192])
 def test_integer_scores_with_many_ties(bsa, oracle_mod, nb):
     """Small-integer pooled inputs make every score an exact integer (or a
     zero of either sign), so ties straddle the k-th score in most rows: the
