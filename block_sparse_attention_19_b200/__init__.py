@@ -56,7 +56,8 @@ EXPORTED = ("bsa_topk_count", "bsa_forward_workspace_bytes", "bsa_block_pool",
             "bsa_sparse_attn_bwd", "bsa_forward_host_workspace_bytes", "bsa_forward_host",
             "bsa_sparse_attn_fwd_train_gqa", "bsa_sparse_attn_bwd_gqa_workspace_bytes", "bsa_sparse_attn_bwd_gqa",
             "bsa_adaptive_block_size", "bsa_block_pool_ex", "bsa_overlap_window_count",
-            "bsa_forward_overlap_workspace_bytes", "bsa_sparse_attn_fwd_overlap", "bsa_forward_overlap")
+            "bsa_forward_overlap_workspace_bytes", "bsa_sparse_attn_fwd_overlap", "bsa_forward_overlap",
+            "bsa_block_pool_qk")
 
 #: variant flags of the *_ex entry points (include/bsa.h)
 BSA_FLAG_CAUSAL, BSA_FLAG_FORCE_DIAG, BSA_FLAG_MAX_POOL = 1, 2, 4
@@ -111,6 +112,7 @@ def _load() -> ctypes.CDLL:
         "bsa_forward_host": ([P, P, P, P, I, I, I, I, I, I, D, I, U, P, Z, P], I),
         "bsa_adaptive_block_size": ([ctypes.c_longlong], I),
         "bsa_block_pool_ex": ([P, P, I, I, I, I, I, I, U, P], I),
+        "bsa_block_pool_qk": ([P, P, P, P, I, I, I, I, I, I, I, U, P], I),
         "bsa_overlap_window_count": ([I, I, D], I),
         "bsa_forward_overlap_workspace_bytes": ([I, I, I, I, I, I, D, D], Z),
         "bsa_sparse_attn_fwd_overlap": ([P, P, P, P, P, I, I, I, I, I, I, I, D, F, I, U, P], I),
@@ -294,6 +296,28 @@ def bsa_block_pool(x: torch.Tensor, block_size: int, out: torch.Tensor | None = 
         out = torch.empty((B, H, N // block_size, D), device=x.device, dtype=torch.float32)
     _check(lib.bsa_block_pool_ex(_p(x), _p(out), B, N, H, D, block_size, _dtype_code(x), flags, _stream(x)))
     return out
+
+
+def bsa_block_pool_qk(q: torch.Tensor, k: torch.Tensor, block_size: int, q_out: torch.Tensor | None = None,
+                      k_out: torch.Tensor | None = None, flags: int = 0):
+    """Pooled q [B, H, nb, D] and pooled k [B, H_kv, nb, D] (one launch when H = H_kv)."""
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be [B, N, heads, D]")
+    _check_qkv(q, k, k)
+    if q.dtype != k.dtype:
+        raise TypeError("q and k must share one dtype")
+    B, N, H, D = q.shape
+    Hk = k.shape[2]
+    nb = N // max(block_size, 1)
+    qo = q_out if q_out is not None else torch.empty((B, H, nb, D), device=q.device, dtype=torch.float32)
+    ko = k_out if k_out is not None else torch.empty((B, Hk, nb, D), device=q.device, dtype=torch.float32)
+    _shape(qo, (B, H, nb, D), "q_out")
+    _shape(ko, (B, Hk, nb, D), "k_out")
+    for t, n in ((q, "q"), (k, "k"), (qo, "q_out"), (ko, "k_out")):
+        _dev(t, n)
+    _check(lib.bsa_block_pool_qk(_p(q), _p(k), _p(qo), _p(ko), B, N, H, Hk, D, block_size, _dtype_code(q), flags,
+                                 _stream(q)))
+    return qo, ko
 
 
 def bsa_block_scores_topk(q_pooled: torch.Tensor, k_pooled: torch.Tensor, topk: int,

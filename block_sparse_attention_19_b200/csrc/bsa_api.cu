@@ -652,6 +652,26 @@ bsa_status bsa_block_pool(const void* x, float* x_pooled, int B, int N, int H, i
   return bsa_block_pool_ex(x, x_pooled, B, N, H, D, block_size, dt, 0u, stream);
 }
 
+bsa_status bsa_block_pool_qk(const void* q, const void* k, float* q_pooled, float* k_pooled, int B, int N, int H,
+                             int H_kv, int D, int block_size, bsa_dtype dt, unsigned flags, void* stream) {
+  bsa_status s;
+  if ((s = check_flags(flags)) != BSA_OK) return s;
+  if ((s = check_dims(B, N, H, D, block_size)) != BSA_OK) return s;
+  if ((s = check_heads(H, H_kv)) != BSA_OK) return s;
+  if ((s = check_dtype(dt)) != BSA_OK) return s;
+  if (!q || !k || !q_pooled || !k_pooled) return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_pooled) || !aligned16(k_pooled))
+    return fail(BSA_ERR_MISALIGNED, "q, k, q_pooled or k_pooled");
+  if ((s = check_device()) != BSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (H == H_kv)  // one launch for both tensors, as bsa_forward pools them
+    return (s = launch_pool(q, q_pooled, k, k_pooled, 2, B, N, H, D, block_size, dt, flags, st)) != BSA_OK ? s : ok();
+  if ((s = launch_pool(q, q_pooled, nullptr, nullptr, 1, B, N, H, D, block_size, dt, flags, st)) != BSA_OK) return s;
+  if ((s = launch_pool(k, k_pooled, nullptr, nullptr, 1, B, N, H_kv, D, block_size, dt, flags, st)) != BSA_OK)
+    return s;
+  return ok();
+}
+
 bsa_status bsa_block_scores_topk_gqa(const float* q_pooled, const float* k_pooled, float* scores,
                                      int32_t* idx, int B, int H, int Hkv, int nb, int D, int k,
                                      unsigned flags, void* stream) {

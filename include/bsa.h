@@ -88,6 +88,13 @@ size_t bsa_forward_workspace_bytes(int B, int N, int H, int D, int block_size, d
 bsa_status bsa_block_pool(const void* x, float* x_pooled, int B, int N, int H, int D,
                           int block_size, bsa_dtype dt, void* stream);
 
+/* Step 1a for q and k together: q_pooled [B, H, nb, D] and k_pooled
+ * [B, H_kv, nb, D] as bsa_block_pool_ex writes them (H a multiple of H_kv;
+ * flags as for bsa_block_pool_ex). One kernel launch when H = H_kv (the
+ * pooling bsa_forward runs), two otherwise. */
+bsa_status bsa_block_pool_qk(const void* q, const void* k, float* q_pooled, float* k_pooled, int B, int N, int H,
+                             int H_kv, int D, int block_size, bsa_dtype dt, unsigned flags, void* stream);
+
 /* Steps 1b + 2 (same page and section, steps 1 and 2: the dot product of every
  * pooled query block with every pooled key block of the same (b, h), then the
  * topk largest of each row):

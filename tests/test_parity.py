@@ -313,6 +313,17 @@ def test_pool_stage_alone(bsa, oracle_mod):
         check_pool(p, q, oracle_mod.block_pool(_host(q), cfg.block_size), cfg.block_size)
 
 
+@pytest.mark.parametrize("H,Hkv", [(3, 3), (4, 2)])
+def test_pool_qk_matches_separate_pooling(bsa, H, Hkv):
+    """bsa_block_pool_qk (one launch for q and k when H = H_kv) gives the same
+    bits as pooling each tensor alone."""
+    cfg = W.Config("poolqk", 2, 2048, H, 128, 128, 0.5, "bf16", 1.0, 15, None, H_kv=Hkv)
+    q, k, _ = W.make_inputs(cfg, device="cuda")
+    qp, kp = bsa.bsa_block_pool_qk(q, k, 128)
+    torch.cuda.synchronize()
+    assert torch.equal(qp, bsa.bsa_block_pool(q, 128)) and torch.equal(kp, bsa.bsa_block_pool(k, 128))
+
+
 def test_repeat_calls_are_deterministic(bsa):
     cfg = _small_cfg((1, 2048, 2, 128, 128, 0.3, "bf16"), seed=21)
     q, k, v = W.make_inputs(cfg, device="cuda")
