@@ -87,7 +87,8 @@ def _fwd(bsa, q=A, k=A, v=A, o=A + 0x100, B=1, N=512, H=2, D=64, bs=64, ratio=0.
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(q=0), 1), (dict(o=0), 1), (dict(N=500), 1), (dict(B=0), 1), (dict(ratio=0.1), 1),
+    (dict(q=0), 1), (dict(o=0), 1), (dict(N=500), 1), (dict(B=0), 1), (dict(N=0), 1), (dict(H=0), 1),
+    (dict(B=-1), 1), (dict(ratio=0.1), 1),
     (dict(ratio=1.5), 1), (dict(ratio=float("nan")), 1), (dict(D=96), 2), (dict(bs=32, N=512), 2),
     (dict(dt=7), 2), (dict(q=M), 3), (dict(v=M), 3), (dict(ws=0), 4), (dict(wsb=16), 4),
     (dict(ws=A + 0x210), 3), (dict(o=A), 1),

@@ -154,3 +154,32 @@ def test_backward_gqa_matches_oracle(bsa, oracle_mod, ci):
     check_grad(dq, rq, "dq")
     check_grad(dk, rk, "dk")
     check_grad(dv, rv, "dv")
+
+
+def test_backward_dq_at_c3_size_on_sampled_query_blocks(bsa, oracle_mod):
+    """The c3 workload (B=2 N=32768 H=16 D=128 block_size=128 k=51): dq of a
+    sample of query blocks (two per (b, h)) against the oracle, which sums a
+    query block's own contributions in full when it is in the sample."""
+    cfg = W.CONFIGS["c3"]
+    B, N, H, D, bs, ratio = cfg.B, cfg.N, cfg.H, cfg.D, cfg.block_size, cfg.topk_ratio
+    q, k, v = W.make_inputs(cfg, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(1700)
+    do = torch.randn(q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    ws = torch.empty(bsa.bsa_forward_workspace_bytes(B, N, H, D, bs, ratio), device="cuda", dtype=torch.uint8)
+    bsa.bsa_forward(q, k, v, bs, ratio, workspace=ws)
+    idx = bsa.workspace_views(ws, B, N, H, D, bs, ratio)[2].clone()
+    o, lse = bsa.bsa_sparse_attn_fwd_train(q, k, v, idx, bs)
+    dq, _, _ = bsa.bsa_sparse_attn_bwd(q, k, v, o, do, idx, lse, bs)
+    torch.cuda.synchronize()
+    assert bsa.bsa_device_error() == 0
+    rows = W.sample_query_blocks(cfg, count=2)
+    rq, _, _ = oracle_mod.sparse_attn_bwd(_host(q), _host(k), _host(v), _host(do), idx.cpu().numpy(), bs, rows=rows)
+    # the sampled rows of dq, [B, H, nrows * bs, D]
+    tok = (rows[..., None] * bs + np.arange(bs)).reshape(B, H, -1)
+    got = dq.to(torch.float64).cpu().numpy()
+    g_rows = np.stack([np.stack([got[b, tok[b, h], h] for h in range(H)]) for b in range(B)])
+    r_rows = np.stack([np.stack([rq[b, tok[b, h], h] for h in range(H)]) for b in range(B)])
+    d = np.abs(g_rows - r_rows)
+    rel = np.linalg.norm(g_rows - r_rows) / np.linalg.norm(r_rows)
+    print(f"c3 dq (sampled): max|d| {d.max():.3g} (max|ref| {np.abs(r_rows).max():.3g}), rel L2 {rel:.3g}")
+    assert rel <= 1e-2 and d.max() <= 2e-2 * np.abs(r_rows).max()
