@@ -234,7 +234,10 @@ __device__ __forceinline__ void tc2_make_p32(const uint32_t (&sv)[32], float m, 
 // rows 64-127 keys 64-127; the other quadrants are computed and discarded,
 // and P is zero there, so one M = 128 product serves both blocks (the same
 // tensor time as two M = 64 products, with every TMEM lane and softmax
-// thread in use).
+// thread in use). With e4m3 inputs P.V is issued per block instead, with the
+// output-lane mask: each block's P (its 64 keys, 16 columns) times its half
+// of the V tile into its own lanes of O, so no zero half is stored and a
+// block whose list has ended issues no P.V.
 // kCausal: key tokens after the query token are masked (kFlagCausal).
 // lse (optional, [B, H, N] float32): ln sum_t exp(scale q_n . k_t) per row.
 // gperiod > 0: query heads h with h % gperiod == 0 are global heads, which
@@ -354,7 +357,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     if (kStack) {
       // a stream walks as many tiles as the longer of its two rows
       for (int q = 0; q < 4; ++q)
-        bar.valid[q] = q / 2 < nstreams ? max(sel_valid<kCausal>(sel4[q], k, blk4[q], nb), 1) : 0;
+        bar.valid[q] = iA + q < nb ? max(sel_valid<kCausal>(sel4[q], k, blk4[q], nb), 1) : 0;
       bar.tiles[0] = max(bar.valid[0], bar.valid[1]);
       bar.tiles[1] = max(bar.valid[2], bar.valid[3]);
     } else {
@@ -457,6 +460,10 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
       constexpr uint64_t kTileStep = L::kTileBytes >> 4;
       // ring index of stream x's tile t (K and V rings are filled in the same order)
       bool ok = mbar_wait(&bar.q_full, 0, abort_flag, 211);
+      // kStack with e4m3: valid index entries of the four query blocks (0: absent)
+      int vq[4] = {0, 0, 0, 0};
+      if constexpr (kStack && kF8)
+        for (int q = 0; q < 4; ++q) vq[q] = bar.valid[q];
       // The rings are consumed in load order: kn and vn are the next K and
       // V loads (a load serves both streams, stream B last, when they share
       // their key tiles).
@@ -501,14 +508,32 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
           tc_fence_after();
           const uint64_t dv = dv0 + (nv % VS) * kTileStep;
           const uint32_t a_tmem = tmem + L::col_s(x);
+          if constexpr (kStack && kF8) {
+            // e4m3: block hf of the stream multiplies its own P (the first
+            // columns of S) by its half of the V tile, into its own lanes of
+            // O, and issues nothing once its list has ended. (With bf16 one
+            // P.V over the whole tile, with the other block's half of P zero,
+            // measured faster.)
 #pragma unroll
-          for (int kk = 0; kk < kStepsPV; ++kk) {
-            // kKeysPerStep keys: 8 TMEM columns of P, kKeysPerStep rows of V
-            const uint64_t bv = dv + ((kk * kKeysPerStep * L::kRowBytes) >> 4);
-            if (kF8)
-              mma_f8_ts(tmem + L::col_o(x), a_tmem + kk * 8, bv, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-            else
-              mma_bf16_ts(tmem + L::col_o(x), a_tmem + kk * 8, bv, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+            for (int hf = 0; hf < 2; ++hf) {
+              if (j >= vq[2 * x + hf]) continue;
+#pragma unroll
+              for (int kk = 0; kk < kStepsPV / 2; ++kk) {
+                const uint64_t bv = dv + ((((kStepsPV / 2) * hf + kk) * kKeysPerStep * L::kRowBytes) >> 4);
+                mma_f8_ts_half(tmem + L::col_o(x), a_tmem + kk * 8, bv, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u,
+                               hf == 0);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kStepsPV; ++kk) {
+              // kKeysPerStep keys: 8 TMEM columns of P, kKeysPerStep rows of V
+              const uint64_t bv = dv + ((kk * kKeysPerStep * L::kRowBytes) >> 4);
+              if (kF8)
+                mma_f8_ts(tmem + L::col_o(x), a_tmem + kk * 8, bv, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+              else
+                mma_bf16_ts(tmem + L::col_o(x), a_tmem + kk * 8, bv, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           // the V ring is shallow, so its entry is freed as soon as the product is done
           if (last_user) mma_commit(&bar.v_empty[nv % VS]);
@@ -563,12 +588,16 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
         // keys are columns 64 hf.. of the tile
         const int hf = quad / 2;
         if (j >= vt) {
-          // this block's list has ended: its P is zero on the whole tile
-          uint32_t z[32];
+          // this block's list has ended (or the block is absent): with bf16
+          // the tile's P.V reads its lanes, so its P is zero; with e4m3 its
+          // half of P.V is not issued
+          if constexpr (!kF8) {
+            uint32_t z[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) z[e] = 0;
-          tmem_st32(scol, z);
-          if constexpr (!kF8) tmem_st32(scol + 32, z);
+            for (int e = 0; e < 32; ++e) z[e] = 0;
+            tmem_st32(scol, z);
+            tmem_st32(scol + 32, z);
+          }
         } else {
           uint32_t s0[32], s1[32];
           tmem_ld32(scol + 64 * hf, s0);
@@ -600,17 +629,19 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
           }
           m_run = m_new;
           uint64_t ps[4] = {0, 0, 0, 0};
-          uint32_t pk0[kF8 ? 8 : 16], pk1[kF8 ? 8 : 16], z[kF8 ? 16 : 32];
+          uint32_t pk0[kF8 ? 8 : 16], pk1[kF8 ? 8 : 16];
           tc2_make_p32<kF8>(s0, m_new, scale_log2, pk0, ps);
           tc2_make_p32<kF8>(s1, m_new, scale_log2, pk1, ps);
-#pragma unroll
-          for (int e = 0; e < (kF8 ? 16 : 32); ++e) z[e] = 0;
-          // P of the block's keys; zeros where the tile holds the other block's
           if constexpr (kF8) {
-            tmem_st8(scol + 16 * hf, pk0);
-            tmem_st8(scol + 16 * hf + 8, pk1);
-            tmem_st16(scol + 16 * (1 - hf), z);
+            // the block's 64 keys over the first columns of S, which its
+            // half of P.V reads in its own lanes
+            tmem_st8(scol, pk0);
+            tmem_st8(scol + 8, pk1);
           } else {
+            // P of the block's keys; zeros where the tile holds the other block's
+            uint32_t z[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) z[e] = 0;
             tmem_st16(scol + 32 * hf, pk0);
             tmem_st16(scol + 32 * hf + 16, pk1);
             tmem_st32(scol + 32 * (1 - hf), z);

@@ -230,6 +230,21 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// An e4m3 product with A from TMEM that writes only the accumulator lanes
+// 0-63 (lo) or 64-127 (!lo) of D, through the output-lane mask of
+// tcgen05.mma (one bit per lane, lane 0 in the lowest bit of the first word;
+// a set bit leaves the lane unchanged).
+__device__ __forceinline__ void mma_f8_ts_half(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate, bool lo) {
+  const uint32_t off_lo = lo ? 0u : 0xffffffffu, off_hi = lo ? 0xffffffffu : 0u;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, {%5, %5, %6, %6}, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(off_lo), "r"(off_hi)
+      : "memory");
+}
+
 // D (+)= A . B^T with FP8 E4M3 A and B (K = 32 per instruction), both from
 // shared memory; and with A from TMEM (four e4m3 per 32-bit column, the
 // lowest byte holding the lowest k).
