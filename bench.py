@@ -563,9 +563,11 @@ def main():
         }
         if bs == 64:
             # two query blocks share one 128 x 128 score tile, of which the
-            # block-diagonal half is used: the tensor core runs twice the
-            # algorithmic FLOPs, so frac cannot exceed 0.5
-            line["roofline"]["tensor_flops_per_launch"] = 2 * flops
+            # block-diagonal half is used: the score product runs twice its
+            # algorithmic FLOPs. P.V does too with bf16 (one product over the
+            # whole tile, the other block's half of P zero); with e4m3 it is
+            # issued per block. So frac cannot exceed 0.5 (bf16) or 2/3 (e4m3).
+            line["roofline"]["tensor_flops_per_launch"] = (1.5 if cfg.dtype == "e4m3" else 2.0) * flops
     line["selection_stage"] = {
         "bytes": sel_bytes, "ms": stage_ms,
         "GB/s": sel_bytes / (stage_ms / 1e3) / 1e9,
