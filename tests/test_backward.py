@@ -7,10 +7,14 @@ kept blocks with the lists held fixed; the oracle computes them in float64
 from the same bf16 inputs and lists.
 
 Tolerance, from the arithmetic: the GPU path rounds three things to bf16
-(relative 2^-9 each): the softmax weights P (operand of dV), the score
-gradients dS (operand of dQ and dK) and the gradients it writes; sums are
-float32. Per gradient tensor: relative L2 <= 1e-2 (about 3 * 2^-9 = 6e-3
-with margin) and max|d| <= 2e-2 * max|reference|.
+(unit roundoff u = 2^-8, 8 significant bits): the softmax weights P (operand
+of dV), the score gradients dS (operand of dQ and dK) and the gradients it
+writes; sums are float32. Each gradient element passes through two of these
+roundings, each with a relative rms error of about u / sqrt(3) * 0.73 = 1.6e-3
+for log-uniformly spread mantissas, so about 2.3e-3 together. Per gradient
+tensor: relative L2 <= 5e-3 (the forward's bf16 bar; measured at most 3.4e-3
+over these cases) and max|d| <= 2e-2 * max|reference| (measured at most
+7e-3).
 """
 import numpy as np
 import pytest
@@ -36,7 +40,7 @@ def check_grad(got: torch.Tensor, ref: np.ndarray, name: str):
     d = np.abs(g - ref)
     rel = np.linalg.norm(g - ref) / np.linalg.norm(ref)
     print(f"{name}: max|d| {d.max():.3g} (max|ref| {np.abs(ref).max():.3g}), rel L2 {rel:.3g}")
-    assert rel <= 1e-2, f"{name}: rel L2 {rel}"
+    assert rel <= 5e-3, f"{name}: rel L2 {rel}"
     assert d.max() <= 2e-2 * np.abs(ref).max(), f"{name}: max|d| {d.max()}"
 
 
@@ -182,4 +186,4 @@ def test_backward_dq_at_c3_size_on_sampled_query_blocks(bsa, oracle_mod):
     d = np.abs(g_rows - r_rows)
     rel = np.linalg.norm(g_rows - r_rows) / np.linalg.norm(r_rows)
     print(f"c3 dq (sampled): max|d| {d.max():.3g} (max|ref| {np.abs(r_rows).max():.3g}), rel L2 {rel:.3g}")
-    assert rel <= 1e-2 and d.max() <= 2e-2 * np.abs(r_rows).max()
+    assert rel <= 5e-3 and d.max() <= 2e-2 * np.abs(r_rows).max()
