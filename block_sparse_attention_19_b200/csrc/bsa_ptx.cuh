@@ -459,7 +459,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // 2^x for a pair of floats on the FMA/ALU pipes, for x <= 8: round-to-nearest
 // split x = n + f with f in [-1/2, 1/2] (adding and subtracting 1.5 * 2^23),
 // a degree-3 polynomial for 2^f fitted here by Remez exchange on the relative
-// error (max 7.5e-5 in float32, far below the 2^-9 of the bf16 P it feeds),
+// error (max 7.5e-5 in float32, far below the up to 2^-8 rounding of the bf16 P it feeds),
 // and n added to the exponent field. The low 9 bits of the rounding constant
 // are zero, so bits(x + 1.5 * 2^23) << 23 equals n << 23 and one integer
 // multiply-add adds it. Inputs below -125 are clamped (2^-125 is negligible

@@ -189,7 +189,7 @@ def test_polynomial_exp2_of_the_softmax():
     the header defines it, evaluated step by step in float32: the range
     split, the degree-3 polynomial and the exponent added through
     bits(x + 1.5 * 2^23) << 23. Its relative error stays below 1e-4 on the
-    range the softmax uses (far below the bf16 rounding of P, 2^-9), and the
+    range the softmax uses (far below the bf16 rounding of P, up to 2^-8), and the
     clamp gives 2^-125-sized values below it."""
     import numpy as np
 
