@@ -26,8 +26,11 @@
 //     release K ring entries (they see each S complete); the issuing thread
 //     commits only the S the softmax waits for and the V entry it just read.
 //     S_X lives in TMEM columns of stream X; P_X (bf16, or e4m3) is written
-//     over the first 64 (32) of them and read from TMEM as the A operand of
-//     PV_X; O_X accumulates in TMEM. Because tcgen05.mma ops of one thread run
+//     over the first 64 (32) of them (block_size 64 with e4m3: 16, each block
+//     in its own lanes) and read from TMEM as the A operand of PV_X; O_X
+//     accumulates in TMEM. With the causal mask and one query block per
+//     stream (bf16), the first half of PV_X(j) starts once the first half of
+//     P_X(j) is stored. Because tcgen05.mma ops of one thread run
 //     in order, S_X(j+1) cannot overwrite P_X(j) before PV_X(j) has read it,
 //     and the completion of S_X(j+1) implies that PV_X(j) is done (so O_X is
 //     stable).
